@@ -1,0 +1,446 @@
+"""Float64 CPU oracle for the per-matrix Muon / Muon+ / SOAP / FOAM optimizer step.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path (the C-ABI library, its
+Python binding, the kernels) may import or call this module.  It exists so that
+the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
+can check the CUDA path against a plain, slow, obviously correct statement of
+what the method computes.
+
+Everything here is NumPy in float64, one matrix at a time, in the order the
+source pages give.  Library primitives used as single steps: ``@`` (matmul),
+``numpy.linalg.qr`` (Householder QR), and, only in the self-check helpers at the
+bottom, ``numpy.linalg.svd`` / ``numpy.linalg.eigh``.
+
+Sources (cited by page title and section):
+  [SMB-review]  "SOAP, Muon and Beyond" (Korean review): §1-1 Problem definition
+                (AdamW and Shampoo factor equations), §2-1 Main contribution
+                (polar factor, Shampoo=Muon identity, RMS matching), §3-2 Module
+                breakdown (Muon recipe, SOAP rotation, real-time eigenbasis update).
+  [SMB-summary] "SOAP, Muon, and Beyond" (English summary): eq. (1) SOAP update,
+                "Update-RMS Matching", "SOAP Instability Diagnosis".
+  [FOAM-review] "Factored One-sided Adam-Moment for Practical and Scalable SOAP"
+                (Korean review): §1 Key Terms & Definitions, §3 Method & Key Results.
+  [MuonPlus]    "Muon+: Towards Better Muon via One Additional Normalization Step":
+                technical summary §2 Methodology.
+
+Readings taken where the pages are silent (each also listed in the design doc):
+  * Newton-Schulz form: the quintic X <- aX + (bA + cA^2)X with A = X X^T, run on
+    the wide orientation (transposed when m > n); default (a,b,c) =
+    (3.4445, -4.7750, 2.0315) each iteration.  The pages name Newton-Schulz only.
+  * Pre-normalisation X0 = M / (||M||_F + 1e-7) (recipe epsilon, [SMB-review] §3-2).
+  * Muon+ Norm^(d): l2 normalisation of each row / column, denominator norm+1e-7,
+    Col-Row = column first then row; applied before the lr*sqrt(m/n) scale.
+  * Decoupled weight decay W <- W(1 - lr*wd) (recipe value only on the pages).
+  * SOAP/FOAM Adam: bias-corrected, eps outside the square root; V is not
+    re-projected when the basis changes (only permuted with it).
+  * Eigenbasis refresh: one power step P = L Q then Q = qr(P) with a positive
+    diagonal in the triangular factor; optional sort of the basis by the
+    Rayleigh quotients diag(Q^T L Q), descending, stable, before the power step.
+  * FOAM tau uses the bias-corrected trace tr(R / (1 - beta2^t)); adaptive check:
+    on steps with (t-1) % pf == 0, rho = ||offdiag(Q^T R Q)||_F / ||Q^T R Q||_F,
+    refresh iff rho > tol.
+
+Parity pins for every function are in tests/test_oracle_*.py.  No function here
+is "parity unpinned".
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+# Default quintic Newton-Schulz coefficients (a, b, c), one triple per iteration.
+NS_DEFAULT_COEF = (3.4445, -4.7750, 2.0315)
+NS_EPS = 1e-7          # Frobenius pre-normalisation epsilon ([SMB-review] §3-2 recipe)
+NORM_EPS = 1e-7        # Muon+ row/column normalisation epsilon (reading)
+
+NORM_NONE, NORM_ROW, NORM_COL, NORM_COL_ROW, NORM_ROW_COL = 0, 1, 2, 3, 4
+REFRESH_EVERY_K, REFRESH_ADAPTIVE, REFRESH_NEVER = 0, 1, 2
+
+
+def _f64(a) -> np.ndarray:
+    return np.asarray(a, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------
+# Muon  ([MuonPlus] §2 Methodology; [SMB-review] §2-1 (2), §3-2 (2))
+# --------------------------------------------------------------------------
+
+def newton_schulz(M, coefs=None, steps: int = 5, eps: float = NS_EPS, dtype=np.float64):
+    """Approximate the polar factor U V^T of M (M = U S V^T) by Newton-Schulz.
+
+    [SMB-review] §2-1 (2): Muon approximates Polar(M) = U V^T by a Newton-Schulz
+    iteration.  Steps: X0 = M / (||M||_F + eps); if M has more rows than
+    columns, iterate on X0^T; each iteration with coefficients (a, b, c):
+        A = X X^T ;  B = b A + c A A ;  X = a X + B X.
+    The result is returned in M's orientation.
+    """
+    X = np.asarray(M, dtype=dtype)
+    if coefs is None:
+        coefs = [NS_DEFAULT_COEF] * steps
+    transposed = X.shape[0] > X.shape[1]
+    X = X / (np.sqrt(np.sum(X * X)) + dtype(eps))
+    if transposed:
+        X = X.T
+    for (a, b, c) in coefs:
+        A = X @ X.T
+        B = dtype(b) * A + dtype(c) * (A @ A)
+        X = dtype(a) * X + B @ X
+    return X.T if transposed else X
+
+
+def muon_plus_norm(O, mode: int, eps: float = NORM_EPS):
+    """Muon+ normalisation Norm^(d) applied to the orthogonalised update.
+
+    [MuonPlus] §2 Methodology: O_t = Norm^(d)(Ortho(M_t)) with d = row, column,
+    Col-Row or Row-Col.  Reading: each row (column) is divided by its l2 norm
+    plus eps; the combined modes apply the first-named direction first.
+    """
+    O = _f64(O)
+
+    def rows(X):
+        return X / (np.sqrt(np.sum(X * X, axis=1, keepdims=True)) + eps)
+
+    def cols(X):
+        return X / (np.sqrt(np.sum(X * X, axis=0, keepdims=True)) + eps)
+
+    if mode == NORM_NONE:
+        return O.copy()
+    if mode == NORM_ROW:
+        return rows(O)
+    if mode == NORM_COL:
+        return cols(O)
+    if mode == NORM_COL_ROW:
+        return rows(cols(O))
+    if mode == NORM_ROW_COL:
+        return cols(rows(O))
+    raise ValueError(f"unknown norm mode {mode}")
+
+
+def muon_step(W, G, M, *, mu: float, lr: float, wd: float = 0.0, ns_coefs=None,
+              ns_steps: int = 5, norm: int = NORM_NONE):
+    """One Muon (or Muon+) step on one m x n matrix.
+
+    [MuonPlus] §2 Methodology: M <- mu M + (1-mu) G; O = Ortho(M) (Newton-Schulz);
+    optionally O <- Norm^(d)(O); W <- W - lr sqrt(m/n) O.  Decoupled weight decay
+    W(1 - lr wd) is the reading of the recipe's weight decay ([SMB-review] §3-2).
+    Returns (W_new, M_new, O) with O the final (normalised) direction.
+    """
+    W, G, M = _f64(W), _f64(G), _f64(M)
+    m, n = W.shape
+    M_new = mu * M + (1.0 - mu) * G                       # M1
+    O = newton_schulz(M_new, ns_coefs, ns_steps)          # M2 + M3
+    O = muon_plus_norm(O, norm)                           # M4
+    W_new = W * (1.0 - lr * wd) - lr * np.sqrt(m / n) * O  # M5
+    return W_new, M_new, O
+
+
+# --------------------------------------------------------------------------
+# Shared SOAP / FOAM pieces
+# --------------------------------------------------------------------------
+
+def qr_positive(P):
+    """Q factor of P = Q R with diag(R) > 0 (unique for full-rank P).
+
+    The per-step QR orthogonalisation of the eigenbasis ([SMB-review] §3-2 (4),
+    [SMB-summary] "SOAP Instability Diagnosis").  numpy's Householder QR is
+    sign-fixed so that every diagonal entry of R is positive.
+    """
+    Q, R = np.linalg.qr(_f64(P))
+    s = np.sign(np.diag(R))
+    s[s == 0] = 1.0
+    return Q * s[None, :]
+
+
+def rayleigh_keys(F, Q):
+    """key_i = Q[:, i]^T F Q[:, i], i.e. diag(Q^T F Q)."""
+    F, Q = _f64(F), _f64(Q)
+    return np.einsum("ki,ki->i", Q, F @ Q)
+
+
+def sort_perm(keys):
+    """Stable descending argsort (ties keep the lower index first)."""
+    keys = _f64(keys)
+    return np.argsort(-keys, kind="stable").astype(np.int32)
+
+
+def refresh_basis(F, Q, sort: bool):
+    """One eigenbasis refresh of the factor F from the current basis Q.
+
+    [SMB-review] §3-2 (4): refresh the basis from the updated factor, then QR.
+    Reading: optional stable descending sort of Q's columns by diag(Q^T F Q),
+    then one power step P = F Q and Q <- qr(P) (positive diagonal).
+    Returns (Q_new, perm) where perm[i] is the old column placed at i.
+    """
+    F, Q = _f64(F), _f64(Q)
+    k = Q.shape[1]
+    perm = sort_perm(rayleigh_keys(F, Q)) if sort else np.arange(k, dtype=np.int32)
+    Qp = Q[:, perm]
+    P = F @ Qp
+    return qr_positive(P), perm
+
+
+def offdiag_ratio(D):
+    """rho = ||D - diag(D)||_F / ||D||_F."""
+    D = _f64(D)
+    off = D - np.diag(np.diag(D))
+    den = np.sqrt(np.sum(D * D))
+    return float(np.sqrt(np.sum(off * off)) / den) if den > 0 else 0.0
+
+
+def refresh_decision(kind: int, t: int, k: int = 1, pf: int = 10, tol: float = 0.1,
+                     F=None, Q=None):
+    """Whether a basis refresh happens at step t (1-based), and the check ratio.
+
+    EVERY_K: (t-1) % k == 0 ([SMB-summary] "SOAP Instability Diagnosis": every
+    step, or every 10 steps for the stale baseline).  ADAPTIVE ([FOAM-review] §3,
+    the Purifying-Shampoo tolerance criterion with pf=10, tol=0.1; the criterion
+    itself is not printed -- reading): on steps with (t-1) % pf == 0, compute
+    D = Q^T F Q and refresh iff ||offdiag D||_F / ||D||_F > tol.
+    Returns (refresh, rho) with rho = -1.0 when no check ran.
+    """
+    if kind == REFRESH_NEVER:
+        return False, -1.0
+    if kind == REFRESH_EVERY_K:
+        return ((t - 1) % k) == 0, -1.0
+    if kind == REFRESH_ADAPTIVE:
+        if (t - 1) % pf != 0:
+            return False, -1.0
+        D = _f64(Q).T @ _f64(F) @ _f64(Q)
+        rho = offdiag_ratio(D)
+        return rho > tol, rho
+    raise ValueError(f"unknown refresh kind {kind}")
+
+
+# --------------------------------------------------------------------------
+# SOAP  ([SMB-review] §1-1, §3-2 (3)(4); [SMB-summary] eq. (1))
+# --------------------------------------------------------------------------
+
+@dataclass
+class SoapState:
+    M: np.ndarray
+    V: np.ndarray
+    L: np.ndarray
+    R: np.ndarray
+    QL: np.ndarray
+    QR: np.ndarray
+
+    @staticmethod
+    def init(m: int, n: int, eps_init: float = 1e-6) -> "SoapState":
+        """L = R = eps_init * I, Q = I, M = V = 0 (initial state reading)."""
+        return SoapState(np.zeros((m, n)), np.zeros((m, n)), eps_init * np.eye(m),
+                         eps_init * np.eye(n), np.eye(m), np.eye(n))
+
+    def copy(self) -> "SoapState":
+        return SoapState(*(np.array(x, dtype=np.float64, copy=True) for x in
+                           (self.M, self.V, self.L, self.R, self.QL, self.QR)))
+
+
+@dataclass
+class SoapResult:
+    W: np.ndarray
+    state: SoapState
+    U: np.ndarray
+    perm_L: np.ndarray
+    perm_R: np.ndarray
+    refreshed_L: bool
+    refreshed_R: bool
+    rho_L: float = -1.0
+    rho_R: float = -1.0
+
+
+def soap_step(W, G, state: SoapState, *, t: int, beta1: float, beta2: float,
+              eps: float, lr: float, wd: float = 0.0, refresh_kind: int = REFRESH_EVERY_K,
+              k: int = 1, pf: int = 10, tol: float = 0.1, sort: bool = True) -> SoapResult:
+    """One two-sided SOAP step with the real-time eigenbasis refresh.
+
+    Order ([SMB-review] §3-2 (4)): the current gradient enters the factors first,
+    then the basis is refreshed from them (power step + QR), then the momentum is
+    preconditioned in the refreshed basis:
+      S1  L <- b2 L + (1-b2) G G^T ;  R <- b2 R + (1-b2) G^T G   ([SMB-review] §1-1)
+      S2  refresh decision
+      S3  sort keys diag(Q^T F Q), permutation, power step P = F Q
+      S4  Q <- qr(P)
+      S5  M <- b1 M + (1-b1) G
+      S6  Gh = QL^T G QR ;  Mh = QL^T M QR                         (eq. (1))
+      S7  V <- b2 V + (1-b2) Gh^2 ;  N = (Mh/(1-b1^t)) / (sqrt(V/(1-b2^t)) + eps)
+      S8  U = QL N QR^T ;  W <- W(1 - lr wd) - lr U                   (eq. (1))
+    """
+    W, G = _f64(W), _f64(G)
+    s = state.copy()
+    m, n = W.shape
+    # S1
+    s.L = beta2 * s.L + (1.0 - beta2) * (G @ G.T)
+    s.R = beta2 * s.R + (1.0 - beta2) * (G.T @ G)
+    # S2
+    refL, rhoL = refresh_decision(refresh_kind, t, k, pf, tol, s.L, s.QL)
+    refR, rhoR = refresh_decision(refresh_kind, t, k, pf, tol, s.R, s.QR)
+    permL = np.arange(m, dtype=np.int32)
+    permR = np.arange(n, dtype=np.int32)
+    # S3 + S4 (V follows the permutation of its basis; no re-projection)
+    if refL:
+        s.QL, permL = refresh_basis(s.L, s.QL, sort)
+        s.V = s.V[permL, :]
+    if refR:
+        s.QR, permR = refresh_basis(s.R, s.QR, sort)
+        s.V = s.V[:, permR]
+    # S5
+    s.M = beta1 * s.M + (1.0 - beta1) * G
+    # S6
+    Gh = s.QL.T @ G @ s.QR
+    Mh = s.QL.T @ s.M @ s.QR
+    # S7
+    s.V = beta2 * s.V + (1.0 - beta2) * Gh * Gh
+    mhat = Mh / (1.0 - beta1 ** t)
+    vhat = s.V / (1.0 - beta2 ** t)
+    N = mhat / (np.sqrt(vhat) + eps)
+    # S8
+    U = s.QL @ N @ s.QR.T
+    W_new = W * (1.0 - lr * wd) - lr * U
+    return SoapResult(W_new, s, U, permL, permR, refL, refR, rhoL, rhoR)
+
+
+# --------------------------------------------------------------------------
+# FOAM  ([FOAM-review] §1 Key Terms, §3 Method)
+# --------------------------------------------------------------------------
+
+@dataclass
+class FoamState:
+    M: np.ndarray
+    r: np.ndarray
+    c: np.ndarray
+    R: np.ndarray
+    QR: np.ndarray
+
+    @staticmethod
+    def init(m: int, n: int, eps_init: float = 1e-6) -> "FoamState":
+        """R = eps_init * I, Q_R = I, M = r = c = 0 (initial state reading)."""
+        return FoamState(np.zeros((m, n)), np.zeros(m), np.zeros(n), eps_init * np.eye(n), np.eye(n))
+
+    def copy(self) -> "FoamState":
+        return FoamState(*(np.array(x, dtype=np.float64, copy=True) for x in
+                           (self.M, self.r, self.c, self.R, self.QR)))
+
+
+@dataclass
+class FoamResult:
+    W: np.ndarray
+    state: FoamState
+    U: np.ndarray
+    perm_R: np.ndarray
+    refreshed: bool
+    rho: float
+    tau: float
+
+
+def foam_tau(R, r, c, t: int, beta2: float, raw_trace: bool = False) -> float:
+    """Trace normalisation tau = tr(R^) / (||r^||_1 ||c^||_1).
+
+    [FOAM-review] §1 (Factored Adam-Moment).  Reading: every statistic carries the
+    Adam bias correction 1/(1-b2^t); raw_trace=True uses the literal tr(R).
+    """
+    bc = 1.0 - beta2 ** t
+    tr = float(np.trace(_f64(R)))
+    if not raw_trace:
+        tr = tr / bc
+    rn = float(np.sum(np.abs(_f64(r)))) / bc
+    cn = float(np.sum(np.abs(_f64(c)))) / bc
+    return tr / (rn * cn)
+
+
+def foam_step(W, G, state: FoamState, *, t: int, beta1: float, beta2: float, eps: float,
+              lr: float, wd: float = 0.0, refresh_kind: int = REFRESH_ADAPTIVE, k: int = 1,
+              pf: int = 10, tol: float = 0.1, sort: bool = True,
+              raw_trace: bool = False) -> FoamResult:
+    """One FOAM step (input-only preconditioning, factored Adam moment).
+
+    [FOAM-review] §1, §3:
+      F1  R <- b2 R + (1-b2) G^T G             (input-side factor only; L dropped)
+      F2  refresh decision (adaptive criterion, pf, tol)
+      F3  refresh Q_R as in SOAP; the permutation also permutes c
+      F4  M <- b1 M + (1-b1) G ;  Gr = G Q_R ;  Mr = M Q_R     (G_rot = G Q_R)
+      F5  r <- b2 r + (1-b2) rowmean(Gr^2) ; c <- b2 c + (1-b2) colmean(Gr^2);
+          v^_ij = tau r^_i c^_j ;  N = (Mr/(1-b1^t)) / (sqrt(v^) + eps)
+      F6  U = N Q_R^T ;  W <- W(1 - lr wd) - lr U
+    """
+    W, G = _f64(W), _f64(G)
+    s = state.copy()
+    m, n = W.shape
+    # F1
+    s.R = beta2 * s.R + (1.0 - beta2) * (G.T @ G)
+    # F2
+    ref, rho = refresh_decision(refresh_kind, t, k, pf, tol, s.R, s.QR)
+    perm = np.arange(n, dtype=np.int32)
+    # F3
+    if ref:
+        s.QR, perm = refresh_basis(s.R, s.QR, sort)
+        s.c = s.c[perm]
+    # F4
+    s.M = beta1 * s.M + (1.0 - beta1) * G
+    Gr = G @ s.QR
+    Mr = s.M @ s.QR
+    # F5
+    G2 = Gr * Gr
+    s.r = beta2 * s.r + (1.0 - beta2) * np.mean(G2, axis=1)
+    s.c = beta2 * s.c + (1.0 - beta2) * np.mean(G2, axis=0)
+    tau = foam_tau(s.R, s.r, s.c, t, beta2, raw_trace)
+    bc2 = 1.0 - beta2 ** t
+    vhat = tau * np.outer(s.r / bc2, s.c / bc2)
+    N = (Mr / (1.0 - beta1 ** t)) / (np.sqrt(vhat) + eps)
+    # F6
+    U = N @ s.QR.T
+    W_new = W * (1.0 - lr * wd) - lr * U
+    return FoamResult(W_new, s, U, perm, ref, rho, tau)
+
+
+# --------------------------------------------------------------------------
+# State accounting ([FOAM-review] §1 Key Terms, §3 Method)
+# --------------------------------------------------------------------------
+
+def soap_state_elems(m: int, n: int) -> int:
+    """SOAP state: M, V (m x n each), L, Q_L (m x m), R, Q_R (n x n) = 2mn+2m^2+2n^2."""
+    return 2 * m * n + 2 * m * m + 2 * n * n
+
+
+def foam_state_elems(m: int, n: int) -> int:
+    """FOAM state: M (m x n), R, Q_R (n x n), r (m), c (n) = mn+2n^2+m+n."""
+    return m * n + 2 * n * n + m + n
+
+
+# --------------------------------------------------------------------------
+# Self-check helpers (used only by the oracle's own pins)
+# --------------------------------------------------------------------------
+
+def polar_svd(M):
+    """Exact polar factor U V^T of M from the SVD ([SMB-review] §2-1 (2))."""
+    U, _, Vt = np.linalg.svd(_f64(M), full_matrices=False)
+    return U @ Vt
+
+
+def ns_closed_form(M, coefs, eps: float = NS_EPS):
+    """Newton-Schulz in closed form: U diag(phi_k o ... o phi_1(s_i/(||M||_F+eps))) V^T.
+
+    Each iteration maps every singular value of the normalised matrix through the
+    odd polynomial phi(x) = a x + b x^3 + c x^5 and leaves the singular vectors alone.
+    """
+    M = _f64(M)
+    U, S, Vt = np.linalg.svd(M, full_matrices=False)
+    x = S / (np.sqrt(np.sum(M * M)) + eps)
+    for (a, b, c) in coefs:
+        x = a * x + b * x ** 3 + c * x ** 5
+    return (U * x[None, :]) @ Vt
+
+
+def _inv_quarter_root_psd(S, rtol: float = 1e-12):
+    """S^{-1/4} on the range of a symmetric PSD matrix (pseudo-inverse root)."""
+    w, V = np.linalg.eigh(_f64(S))
+    keep = w > rtol * max(w.max(), 0.0)
+    wr = np.zeros_like(w)
+    wr[keep] = w[keep] ** -0.25
+    return (V * wr[None, :]) @ V.T
+
+
+def shampoo_update(G, L, R):
+    """Shampoo preconditioned update L^{-1/4} G R^{-1/4} ([SMB-review] §1-1)."""
+    return _inv_quarter_root_psd(L) @ _f64(G) @ _inv_quarter_root_psd(R)
