@@ -1,0 +1,417 @@
+"""Benchmark of the optimizer-step hot path on synthetic layer sets.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl mine|reference]
+
+One "step" applies the library's optimizer step(s) to one full synthetic layer
+set resident in HBM (per rank: N ranks each own one layer set, no collective on
+the data path = weak scaling).  Rank 0 prints one JSON line.
+
+Timing: W untimed warm-up steps; K timed steps between a barrier and
+cudaDeviceSynchronize on both sides, CUDA events on the launching stream, max
+over ranks.  Inputs exceed the 126 MB L2 many times over.  Every library launch
+inside the timed region is bracketed by events (mao_profile_start), which gives
+each kernel's live duration for the roofline entry and the launch count.
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+WORKLOADS = {
+    # name: (description, optimizers run per step, default gradient dtype bf16?)
+    "dense8b_moe": ("8B-dense block (7 matrices) + 256-expert MoE bank (768 matrices), bf16 G ~ N(0,0.01^2)*s_e",
+                    True),
+    "gpt2_124m": ("GPT-2-124M-shaped set, 48 matrices, bf16 G ~ N(0,0.02^2), Muon+ Col-Row", True),
+    "gpt2_760m": ("GPT-2-760M-shaped set, 96 matrices, fp32 G ~ N(0,0.01^2)", False),
+    "muon_single": ("one 256x512 fp32 weight", False),
+}
+MUON_NORM = {"gpt2_124m": "col_row"}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
+    ap.add_argument("--workload", default="dense8b_moe", choices=sorted(WORKLOADS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    return ap.parse_args()
+
+
+def specs_for(workload, seed):
+    from matrix_aware_optimizers_02_b200 import synth
+    if workload == "dense8b_moe":
+        return synth.specs_dense8b_moe(256, seed)
+    return synth.WORKLOADS[workload]()
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- peaks / traffic
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    cs = os.path.join(ROOT, "matrix_aware_optimizers_02_b200", "csrc")
+    for fn in sorted(os.listdir(cs)):
+        if fn.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(cs, fn), "rb") as f:
+                h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_name, workload):
+    """DRAM bytes per launch from a committed ncu capture, if its sources match."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    e = d.get("kernels", {}).get(f"{workload}/{kernel_name}")
+    return None if e is None else e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- CPU (oracle) leg
+def cpu_oracle_sample(workload, budget_s, seed):
+    """Time the float64 oracle on a bounded sample of the workload's matrices and
+    scale to one full layer set.  Returns (ms per layer set, cores, sample text)."""
+    from matrix_aware_optimizers_02_b200 import synth
+    from oracle import mao_oracle as O
+    specs = specs_for(workload, seed)
+    norm = {"col_row": O.NORM_COL_ROW}.get(MUON_NORM.get(workload, "none"), O.NORM_NONE)
+    # distinct shapes with multiplicities, cheapest first
+    shapes = {}
+    for s in specs:
+        shapes[(s.m, s.n)] = shapes.get((s.m, s.n), 0) + 1
+
+    def ns_flops(m, n):
+        a, b = min(m, n), max(m, n)
+        return 5 * (4 * a * a * b + 2 * a ** 3)
+
+    order = sorted(shapes, key=lambda k: ns_flops(*k))
+    rng = np.random.default_rng(seed)
+    timed = {}
+    spent = 0.0
+    for (m, n) in order:
+        if spent > budget_s * 0.6 and timed:
+            break
+        W = rng.standard_normal((m, n)) * 0.02
+        G = rng.standard_normal((m, n)) * 0.01
+        M = np.zeros((m, n))
+        t0 = time.perf_counter()
+        O.muon_step(W, G, M, mu=0.95, lr=0.02, norm=norm)
+        dt = time.perf_counter() - t0
+        timed[(m, n)] = dt
+        spent += dt
+    # shapes not timed: scale by Newton-Schulz FLOPs at the best timed rate (largest shape)
+    rate = max(ns_flops(*k) / v for k, v in timed.items())
+    total = 0.0
+    for k, cnt in shapes.items():
+        total += cnt * (timed[k] if k in timed else ns_flops(*k) / rate)
+    cores = len(os.sched_getaffinity(0))
+    sample = ("oracle muon_step (float64 NumPy) timed once on shapes " +
+              ", ".join(f"{m}x{n}" for (m, n) in timed) +
+              "; each shape's time x its multiplicity" +
+              ("" if len(timed) == len(shapes) else "; untimed shapes scaled by Newton-Schulz FLOPs") +
+              f"; {spent:.1f} s of CPU work")
+    return total * 1e3, cores, sample
+
+
+# ----------------------------------------------------------------------------- main (mine)
+def run_mine(args, rank, world, dist):
+    import torch
+
+    from matrix_aware_optimizers_02_b200 import _lib as L
+    from matrix_aware_optimizers_02_b200 import api, synth
+
+    lib = L.load()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    desc, g_bf16 = WORKLOADS[args.workload]
+    specs = specs_for(args.workload, args.seed)
+    mats = synth.torch_muon_inputs(specs, args.seed + 7919 * rank, dev, g_bf16=g_bf16)
+    norm = MUON_NORM.get(args.workload, "none")
+    step = api.MuonBatch(mats, mu=0.95, lr=0.02, norm=norm, with_stats=True)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = step.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    # launch profiler sized for the timed steps
+    cap = 4096
+    Ev = ctypes.c_void_p * (2 * cap)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * cap)]
+    for e in evs:  # torch creates the CUDA event object on its first record
+        e.record(stream)
+    torch.cuda.synchronize()
+    ev_arr = Ev(*[ctypes.c_void_p(e.cuda_event) for e in evs])
+    info = (L.LaunchInfo * cap)()
+
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    L.check(lib.mao_profile_start(ev_arr, info, cap))
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step()
+    t_end.record(stream)
+    n_launch = lib.mao_profile_stop()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop() if clocks else None
+    ms = t_start.elapsed_time(t_end) / args.steps
+    status = step.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after timed steps")
+
+    # per-kernel live durations
+    per = {}
+    for i in range(min(n_launch, cap)):
+        k = info[i].kernel
+        d = evs[2 * i].elapsed_time(evs[2 * i + 1])
+        e = per.setdefault(k, {"ms": 0.0, "n": 0, "flops": 0.0, "bytes": 0.0})
+        e["ms"] += d
+        e["n"] += 1
+        e["flops"] += info[i].flops
+        e["bytes"] += info[i].bytes
+
+    # end-to-end: gradients from pinned host memory, step, stats back to host
+    host_g = [g.cpu().pin_memory() for (_, g, _) in mats]
+    h2d = sum(g.numel() * g.element_size() for g in host_g)
+    stats_host = torch.empty_like(step.stats, device="cpu").pin_memory()
+    d2h = stats_host.numel() * stats_host.element_size()
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        for (_, g, _), hg in zip(mats, host_g):
+            g.copy_(hg, non_blocking=True)
+        step()
+        stats_host.copy_(step.stats, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+
+    t = torch.tensor([ms, e2e_ms], device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max, e2e_max = t.tolist()
+    if rank != 0:
+        return None
+
+    peaks, peak_src = measured_peaks()
+    names = L.KERNEL_NAMES
+    dom = max(per, key=lambda k: per[k]["ms"]) if per else None
+    roof = None
+    if dom is not None:
+        e = per[dom]
+        avg_ms = e["ms"] / e["n"]
+        if e["flops"] > 0:
+            achieved = (e["flops"] / e["n"]) / (avg_ms * 1e-3) / 1e12
+            peak = peaks["bf16_tflops_sustained"]
+            roof = {"bound": "tensor", "kernel": names.get(dom, str(dom)), "achieved": round(achieved, 1),
+                    "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)"}
+        else:
+            achieved = (e["bytes"] / e["n"]) / (avg_ms * 1e-3) / 1e9
+            peak = peaks["hbm_gbs"]
+            roof = {"bound": "hbm", "kernel": names.get(dom, str(dom)), "achieved": round(achieved, 1),
+                    "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                    "peak_source": f"{peak_src} HBM copy"}
+        roof["traffic"] = ncu_traffic(names.get(dom, str(dom)), args.workload)
+        roof["launches"] = e["n"]
+        roof["avg_launch_ms"] = round(avg_ms, 4)
+    kernels = {names.get(k, str(k)): {"launches": v["n"], "ms_total": round(v["ms"], 3),
+                                      "share": round(v["ms"] / max(sum(x["ms"] for x in per.values()), 1e-9), 4),
+                                      **({"tflops": round(v["flops"] / (v["ms"] * 1e-3) / 1e12, 1)}
+                                         if v["flops"] > 0 else
+                                         {"gbs": round(v["bytes"] / (v["ms"] * 1e-3) / 1e9, 1)})}
+               for k, v in sorted(per.items())}
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu_ms, cores, sample = cpu_oracle_sample(args.workload, args.cpu_budget_s, args.seed)
+        cpu = {"value": round(cpu_ms, 1), "unit": "ms", "cores": cores, "kind": "oracle", "sample": sample}
+
+    n_elems = sum(s.m * s.n for s in specs)
+    line = {
+        "metric": "Muon/SOAP/FOAM step ms per layer set; % of tensor-core peak and HBM GB/s",
+        "value": round(ms_max / world, 4),
+        "unit": "ms",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max, 4),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 operands / fp32 accumulate (Newton-Schulz), fp32 states",
+        "data": "synthetic (seeded Gaussian gradients, random weights)",
+        "config": {"workload": args.workload, "description": desc, "optimizers": ["muon"],
+                   "muon": {"mu": 0.95, "lr": 0.02, "ns_steps": 5, "norm": norm},
+                   "matrices_per_rank": len(specs), "elements_per_rank": n_elems,
+                   "l2_policy": "inputs larger than L2 (no flush)", "parallelism": f"independent layer sets x{world}"},
+        "roofline": roof,
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_max / world, 4), "unit": "ms", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(n_launch),
+        "clocks": clk,
+    }
+    return line
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm, on the host cores, rank 0 only."""
+    if rank != 0:
+        return None
+    per_step = []
+    info = None
+    for i in range(args.warmup + args.steps):
+        ms, cores, sample = cpu_oracle_sample(args.workload, args.cpu_budget_s / max(args.steps, 1), args.seed + i)
+        if i >= args.warmup:
+            per_step.append(ms)
+            info = (cores, sample)
+    v = statistics.median(per_step)
+    desc, _ = WORKLOADS[args.workload]
+    return {
+        "impl": "reference",
+        "metric": "Muon/SOAP/FOAM step ms per layer set; % of tensor-core peak and HBM GB/s",
+        "value": round(v, 1), "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(v, 1), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded Gaussian)",
+        "config": {"workload": args.workload, "description": desc, "optimizers": ["muon"]},
+        "cpu_baseline": {"value": round(v, 1), "unit": "ms", "cores": info[0], "kind": "oracle", "sample": info[1]},
+        "e2e": {"value": round(v, 1), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as D
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        D.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = D
+    try:
+        line = run_mine(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

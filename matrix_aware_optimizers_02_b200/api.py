@@ -1,0 +1,147 @@
+"""Thin Python binding over libmao: builds the C descriptors from torch tensors
+and calls the library on the current CUDA stream.  Argument marshalling only;
+every arithmetic step runs in the library's kernels.
+
+    from matrix_aware_optimizers_02_b200 import api
+    step = api.MuonBatch([(W, G, M), ...], mu=0.95, lr=0.02, norm="col_row")
+    step()            # one optimizer step on torch.cuda.current_stream()
+"""
+
+from __future__ import annotations
+
+import ctypes
+from typing import Iterable, Optional, Sequence, Tuple
+
+import torch
+
+from . import _lib as L
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _g_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return L.MAO_F32
+    if t.dtype == torch.bfloat16:
+        return L.MAO_BF16
+    raise TypeError(f"gradient dtype {t.dtype} not supported (float32 or bfloat16)")
+
+
+def _check_mat(name: str, t: torch.Tensor, shape, dtype=torch.float32):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    # 256-byte alignment: the caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+class MuonBatch:
+    """One Muon / Muon+ step over a fixed list of (W, G, M) matrices.
+
+    W, M: float32 (m, n) contiguous CUDA tensors updated in place; G: float32 or
+    bfloat16 (m, n).  The descriptors and the workspace are built once; calling
+    the object enqueues one step on the given (or current) stream.
+    """
+
+    def __init__(self, mats: Sequence[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]], *, mu: float, lr: float,
+                 wd: float = 0.0, eps: float = 1e-7, ns_steps: int = 5,
+                 ns_coef: Optional[Sequence[Sequence[float]]] = None, norm: str = "none",
+                 workspace: Optional[torch.Tensor] = None, with_stats: bool = False):
+        self.lib = L.load()
+        self.mats = list(mats)
+        n = len(self.mats)
+        arr = (L.MuonMat * max(n, 1))()
+        dev = None
+        for i, (W, G, M) in enumerate(self.mats):
+            m_, n_ = W.shape
+            _check_mat("W", W, (m_, n_))
+            _check_mat("G", G, (m_, n_), None)
+            _check_mat("M", M, (m_, n_))
+            arr[i] = L.MuonMat(m_, n_, W.data_ptr(), G.data_ptr(), _g_dtype(G), M.data_ptr())
+            dev = W.device
+        self.arr = arr
+        self.count = n
+        self._coef = None
+        coef_ptr = None
+        if ns_coef is not None:
+            flat = [float(x) for triple in ns_coef for x in triple]
+            if len(flat) != 3 * ns_steps:
+                raise ValueError("ns_coef must hold ns_steps (a, b, c) triples")
+            self._coef = (ctypes.c_float * len(flat))(*flat)
+            coef_ptr = ctypes.cast(self._coef, ctypes.POINTER(ctypes.c_float))
+        if norm not in L.NORM_MODES:
+            raise ValueError(f"norm must be one of {sorted(L.NORM_MODES)}")
+        self.params = L.MuonParams(mu, lr, wd, eps, ns_steps, coef_ptr, L.NORM_MODES[norm])
+        nbytes = ctypes.c_size_t(0)
+        L.check(self.lib.mao_muon_workspace_size(arr, n, ctypes.byref(self.params), ctypes.byref(nbytes)),
+                "mao_muon_workspace_size")
+        self.ws_bytes = nbytes.value
+        if workspace is None:
+            workspace = _alloc_workspace(self.ws_bytes, dev if dev is not None else "cuda")
+        elif workspace.numel() * workspace.element_size() < self.ws_bytes:
+            raise ValueError("workspace too small")
+        self.workspace = workspace
+        self.stats = None
+        if with_stats:
+            self.stats = torch.zeros((max(n, 1), 4), dtype=torch.float32, device=workspace.device)
+
+    def __call__(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+        st = self.lib.mao_muon_step(self.arr, self.count, ctypes.byref(self.params), self.workspace.data_ptr(),
+                                    self.ws_bytes, self.stats.data_ptr() if self.stats is not None else None,
+                                    _stream_handle(stream))
+        L.check(st, "mao_muon_step")
+
+    def device_status(self, stream: Optional[torch.cuda.Stream] = None) -> int:
+        """Status word recorded on the device by the last step (synchronises the stream)."""
+        where = ctypes.c_int32(0)
+        return self.lib.mao_workspace_status(self.workspace.data_ptr(), _stream_handle(stream), ctypes.byref(where))
+
+    def stats_dict(self):
+        """Per-matrix diagnostics of the last step (update_rms, nonfinite)."""
+        if self.stats is None:
+            return None
+        s = self.stats[: self.count].cpu()
+        nonfinite = s[:, 3].contiguous().view(torch.int32)
+        return {"update_rms": s[:, 0].tolist(), "nonfinite": nonfinite.tolist()}
+
+
+def muon_step(mats, **kw) -> None:
+    """Functional form: build a MuonBatch and run one step."""
+    MuonBatch(mats, **kw)()
+
+
+def gemm(A: torch.Tensor, B: torch.Tensor, *, kind: str = "bf16", a_mn_major: bool = False,
+         b_mn_major: bool = False, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Verification entry: D[b] = A[b] @ B[b]^T through the tensor-core GEMM core.
+
+    A is (batch, M, K) (or (batch, K, M) when a_mn_major); B is (batch, N, K)
+    (or (batch, K, N) when b_mn_major).  kind "bf16" (bf16 operands) or
+    "tf32x3" (fp32 operands, split hi/lo).  Returns fp32 (batch, M, N).
+    """
+    lib = L.load()
+    k = {"bf16": 0, "tf32x3": 1}[kind]
+    batch = A.shape[0]
+    M = A.shape[2] if a_mn_major else A.shape[1]
+    K = A.shape[1] if a_mn_major else A.shape[2]
+    N = B.shape[2] if b_mn_major else B.shape[1]
+    D = torch.empty((batch, M, N), dtype=torch.float32, device=A.device)
+    nbytes = ctypes.c_size_t(0)
+    L.check(lib.mao_test_gemm_workspace_size(k, batch, M, N, K, ctypes.byref(nbytes)), "gemm workspace")
+    ws = _alloc_workspace(nbytes.value, A.device)
+    L.check(lib.mao_test_gemm(k, int(a_mn_major), int(b_mn_major), A.data_ptr(), B.data_ptr(), D.data_ptr(), batch,
+                              M, N, K, ws.data_ptr(), nbytes.value, _stream_handle(stream)), "mao_test_gemm")
+    where = ctypes.c_int32(0)
+    st = lib.mao_workspace_status(ws.data_ptr(), _stream_handle(stream), ctypes.byref(where))
+    L.check(st, f"gemm device status (site {where.value})")
+    return D

@@ -1,0 +1,390 @@
+// mao_muon_step: one Muon / Muon+ step over a batch of matrices.
+//
+// Launch sequence on the caller's stream (no host synchronisation):
+//   1. muon_prep_kernel      momentum EMA, sum-of-squares partials, bf16 X / X^T
+//   2. muon_scale_kernel     per-matrix 1/(||M||_F + eps)
+//   3. ns_steps x 3 grouped tcgen05 GEMMs over every shape class at once:
+//        A = s^2 X X^T                     (EPI_GRAM, s = the scale on iteration 0)
+//        B = b A + c A A                   (EPI_POLY; A is symmetric, so A A = A A^T)
+//        X' = s (a X + B X), and X'^T      (EPI_AXPY_T)
+//      Iteration 0 works on the unnormalised bf16(M) and applies the per-matrix
+//      scale s in the epilogues, which equals normalising first:
+//        s^2 X X^T = (sX)(sX)^T and s (a X + B X) = a (sX) + B (sX).
+//   4. Muon+ row/column scales (optional)
+//   5. muon_update_kernel    W <- W (1 - lr wd) - lr sqrt(m/n) Norm(O)
+//   6. muon_stats_kernel     (optional)
+#include <algorithm>
+#include <cmath>
+#include <map>
+
+#include "host_common.h"
+#include "muon_kernels.cuh"
+
+namespace mao {
+
+namespace {
+
+constexpr float kDefaultCoef[3] = {3.4445f, -4.7750f, 2.0315f};
+constexpr int kMaxNsSteps = 16;
+
+struct MuonClass {
+  int s = 0, l = 0;           // X is s x l
+  std::vector<int> mats;      // global matrix indices, in batch order
+  int ld_l = 0, ld_s = 0;     // padded leading dimensions (multiples of 8)
+  size_t off_X[2] = {}, off_XT[2] = {}, off_A = 0, off_B = 0;
+  int scale_begin = 0;        // first slot in the scale array
+};
+
+struct MuonPlan {
+  std::vector<MuonClass> cls;
+  std::vector<int> mat_class, mat_slot;  // class of matrix p, its index in the class
+  size_t off_table = 0, off_scale = 0, off_partial = 0, off_rowscale = 0, off_colscale = 0, off_colpart = 0,
+         off_rowbegin = 0, off_updpart = 0, off_updbad = 0;
+  int prep_blocks = 0, colsq_blocks = 0, upd_blocks = 0, total_rows = 0;
+  size_t total = 0;
+  bool use_rows = false, use_cols = false;
+  std::vector<MuonMatDev> table;  // filled without device pointers by plan()
+};
+
+bool norm_uses_rows(int mode) { return mode == MAO_NORM_ROW || mode == MAO_NORM_COL_ROW || mode == MAO_NORM_ROW_COL; }
+bool norm_uses_cols(int mode) { return mode == MAO_NORM_COL || mode == MAO_NORM_COL_ROW || mode == MAO_NORM_ROW_COL; }
+
+mao_status validate(const mao_muon_mat* mats, int32_t count, const mao_muon_params* p, bool check_ptrs) {
+  if (p == nullptr || count < 0 || (count > 0 && mats == nullptr)) return MAO_ERR_INVALID_ARG;
+  if (p->ns_steps < 0 || p->ns_steps > kMaxNsSteps) return MAO_ERR_INVALID_ARG;
+  if (p->norm < MAO_NORM_NONE || p->norm > MAO_NORM_ROW_COL) return MAO_ERR_INVALID_ARG;
+  if (!std::isfinite(p->mu) || !std::isfinite(p->lr) || !std::isfinite(p->wd) || !std::isfinite(p->eps) ||
+      p->eps < 0.0f)
+    return MAO_ERR_INVALID_ARG;
+  if (p->ns_coef != nullptr)
+    for (int i = 0; i < 3 * p->ns_steps; ++i)
+      if (!std::isfinite(p->ns_coef[i])) return MAO_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    const mao_muon_mat& a = mats[i];
+    if (a.m < 1 || a.n < 1) return MAO_ERR_SHAPE;
+    if ((long long)a.m * a.n > (1ll << 31) - 1) return MAO_ERR_SHAPE;
+    if (a.g_dtype != MAO_F32 && a.g_dtype != MAO_BF16) return MAO_ERR_DTYPE;
+    if (a.n % 4 != 0) return MAO_ERR_SHAPE;
+    if (a.g_dtype == MAO_BF16 && a.n % 8 != 0) return MAO_ERR_SHAPE;
+    if (check_ptrs) {
+      if (a.W == nullptr || a.G == nullptr || a.M == nullptr) return MAO_ERR_INVALID_ARG;
+      if (!aligned16(a.W) || !aligned16(a.G) || !aligned16(a.M)) return MAO_ERR_ALIGN;
+    }
+  }
+  return MAO_OK;
+}
+
+void plan(const mao_muon_mat* mats, int count, const mao_muon_params* p, MuonPlan& P) {
+  P = MuonPlan();
+  P.use_rows = norm_uses_rows(p->norm);
+  P.use_cols = norm_uses_cols(p->norm);
+  std::map<std::pair<int, int>, int> idx;
+  P.mat_class.resize(count);
+  P.mat_slot.resize(count);
+  for (int i = 0; i < count; ++i) {
+    const int s = std::min(mats[i].m, mats[i].n), l = std::max(mats[i].m, mats[i].n);
+    auto key = std::make_pair(s, l);
+    auto it = idx.find(key);
+    if (it == idx.end()) {
+      it = idx.emplace(key, (int)P.cls.size()).first;
+      MuonClass c;
+      c.s = s;
+      c.l = l;
+      c.ld_l = round_up_int(l, 8);
+      c.ld_s = round_up_int(s, 8);
+      P.cls.push_back(c);
+    }
+    P.mat_class[i] = it->second;
+    P.mat_slot[i] = (int)P.cls[it->second].mats.size();
+    P.cls[it->second].mats.push_back(i);
+  }
+  Carver cv;
+  cv.take(kStatusBytes);
+  P.off_table = cv.take(sizeof(MuonMatDev) * (size_t)std::max(count, 1));
+  P.off_scale = cv.take(sizeof(float) * (size_t)std::max(count, 1));
+  int sb = 0;
+  for (auto& c : P.cls) {
+    c.scale_begin = sb;
+    sb += (int)c.mats.size();
+  }
+  // per-matrix block bookkeeping
+  P.table.assign(count, MuonMatDev());
+  int prep = 0, colsq = 0, upd = 0, rows = 0;
+  size_t rs_elems = 0, cs_elems = 0, cp_elems = 0;
+  for (int i = 0; i < count; ++i) {
+    MuonMatDev& D = P.table[i];
+    D.m = mats[i].m;
+    D.n = mats[i].n;
+    D.g_bf16 = mats[i].g_dtype == MAO_BF16;
+    D.ldw = round_up_int(D.n, 8);
+    D.ldt = round_up_int(D.m, 8);
+    const int tr = (D.m + kPrepTile - 1) / kPrepTile, tc = (D.n + kPrepTile - 1) / kPrepTile;
+    D.prep_tiles_c = tc;
+    D.prep_begin = prep;
+    D.prep_count = tr * tc;
+    prep += tr * tc;
+    D.col_chunks = (D.m + kColChunkRows - 1) / kColChunkRows;
+    D.colsq_begin = colsq;
+    if (P.use_cols) colsq += D.col_chunks * ((D.n + 255) / 256);
+    const long long el = (long long)D.m * D.n;
+    D.upd_begin = upd;
+    D.upd_count = (int)((el + kUpdElems - 1) / kUpdElems);
+    upd += D.upd_count;
+    D.out_scale = p->lr * std::sqrt((float)D.m / (float)D.n);
+    rs_elems += D.m;
+    cs_elems += D.n;
+    cp_elems += (size_t)D.col_chunks * D.n;
+    rows += D.m;
+  }
+  P.prep_blocks = prep;
+  P.colsq_blocks = colsq;
+  P.upd_blocks = upd;
+  P.total_rows = rows;
+  P.off_partial = cv.take(sizeof(float) * (size_t)std::max(prep, 1));
+  if (P.use_rows) P.off_rowscale = cv.take(sizeof(float) * rs_elems);
+  if (P.use_cols) {
+    P.off_colscale = cv.take(sizeof(float) * cs_elems);
+    P.off_colpart = cv.take(sizeof(float) * cp_elems);
+  }
+  if (P.use_rows) P.off_rowbegin = cv.take(sizeof(int) * (size_t)std::max(count, 1));
+  P.off_updpart = cv.take(sizeof(float) * (size_t)std::max(upd, 1));
+  P.off_updbad = cv.take(sizeof(int) * (size_t)std::max(upd, 1));
+  for (auto& c : P.cls) {
+    const size_t cnt = c.mats.size();
+    for (int k = 0; k < 2; ++k) {
+      c.off_X[k] = cv.take(2 * cnt * (size_t)c.s * c.ld_l);
+      c.off_XT[k] = cv.take(2 * cnt * (size_t)c.l * c.ld_s);
+    }
+    c.off_A = cv.take(2 * cnt * (size_t)c.s * c.ld_s);
+    c.off_B = cv.take(2 * cnt * (size_t)c.s * c.ld_s);
+  }
+  P.total = cv.total();
+}
+
+}  // namespace
+
+}  // namespace mao
+
+using namespace mao;
+
+extern "C" mao_status mao_muon_workspace_size(const mao_muon_mat* mats, int32_t count, const mao_muon_params* p,
+                                              size_t* bytes) {
+  if (bytes == nullptr) return MAO_ERR_INVALID_ARG;
+  MAO_TRY(validate(mats, count, p, false));
+  MuonPlan P;
+  plan(mats, count, p, P);
+  *bytes = P.total;
+  return MAO_OK;
+}
+
+extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, const mao_muon_params* p,
+                                   void* workspace, size_t ws_bytes, mao_stats* stats, mao_stream_t stream_) {
+  MAO_TRY(validate(mats, count, p, true));
+  if (count == 0) return MAO_OK;
+  MuonPlan P;
+  plan(mats, count, p, P);
+  if (workspace == nullptr || ws_bytes < P.total) return MAO_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MAO_ERR_ALIGN;
+  if (stats != nullptr && !aligned16(stats)) return MAO_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  MAO_TRY(device_info(&dev));
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DevStatus* status = reinterpret_cast<DevStatus*>(ws);
+  float* scale = reinterpret_cast<float*>(ws + P.off_scale);
+  float* partial = reinterpret_cast<float*>(ws + P.off_partial);
+  float* rowscale = P.use_rows ? reinterpret_cast<float*>(ws + P.off_rowscale) : nullptr;
+  float* colscale = P.use_cols ? reinterpret_cast<float*>(ws + P.off_colscale) : nullptr;
+  float* colpart = P.use_cols ? reinterpret_cast<float*>(ws + P.off_colpart) : nullptr;
+  int* rowbegin = P.use_rows ? reinterpret_cast<int*>(ws + P.off_rowbegin) : nullptr;
+  float* updpart = reinterpret_cast<float*>(ws + P.off_updpart);
+  int* updbad = reinterpret_cast<int*>(ws + P.off_updbad);
+  const int fin = p->ns_steps % 2;
+
+  // device table
+  std::vector<int> rb(count);
+  size_t rs_off = 0, cs_off = 0, cp_off = 0;
+  int rows = 0;
+  for (int i = 0; i < count; ++i) {
+    MuonMatDev& D = P.table[i];
+    const MuonClass& C = P.cls[P.mat_class[i]];
+    const int b = P.mat_slot[i];
+    D.W = mats[i].W;
+    D.G = mats[i].G;
+    D.M = mats[i].M;
+    __nv_bfloat16* X0 = reinterpret_cast<__nv_bfloat16*>(ws + C.off_X[0]) + (size_t)b * C.s * C.ld_l;
+    __nv_bfloat16* XT0 = reinterpret_cast<__nv_bfloat16*>(ws + C.off_XT[0]) + (size_t)b * C.l * C.ld_s;
+    __nv_bfloat16* Xf = reinterpret_cast<__nv_bfloat16*>(ws + C.off_X[fin]) + (size_t)b * C.s * C.ld_l;
+    __nv_bfloat16* XTf = reinterpret_cast<__nv_bfloat16*>(ws + C.off_XT[fin]) + (size_t)b * C.l * C.ld_s;
+    const bool wide = D.m <= D.n;
+    D.Xw = wide ? X0 : XT0;
+    D.Xt = wide ? XT0 : X0;
+    D.O = wide ? Xf : XTf;
+    D.rowscale = rowscale ? rowscale + rs_off : nullptr;
+    D.colscale = colscale ? colscale + cs_off : nullptr;
+    D.colpart = colpart ? colpart + cp_off : nullptr;
+    D.oscale = (p->ns_steps == 0) ? scale + C.scale_begin + b : nullptr;
+    D.scale_slot = C.scale_begin + b;
+    rs_off += D.m;
+    cs_off += D.n;
+    cp_off += (size_t)D.col_chunks * D.n;
+    rb[i] = rows;
+    rows += D.m;
+  }
+  MAO_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream));
+  MAO_CUDA_TRY(cudaMemcpyAsync(ws + P.off_table, P.table.data(), sizeof(MuonMatDev) * count,
+                               cudaMemcpyHostToDevice, stream));
+  if (rowbegin)
+    MAO_CUDA_TRY(cudaMemcpyAsync(rowbegin, rb.data(), sizeof(int) * count, cudaMemcpyHostToDevice, stream));
+  const MuonMatDev* T = reinterpret_cast<const MuonMatDev*>(ws + P.off_table);
+
+  // algorithmic bytes of the elementwise passes
+  double elems = 0.0, g_bytes = 0.0;
+  for (int i = 0; i < count; ++i) {
+    const double e = (double)mats[i].m * mats[i].n;
+    elems += e;
+    g_bytes += e * (mats[i].g_dtype == MAO_BF16 ? 2.0 : 4.0);
+  }
+
+  // 1-2: momentum, partial norms, bf16 operands, per-matrix scale
+  {
+    LaunchScope ls(stream, MAO_K_MUON_PREP, 0.0, g_bytes + elems * (4.0 + 4.0 + 2.0 + 2.0));
+    muon_prep_kernel<<<P.prep_blocks, 256, 0, stream>>>(T, count, p->mu, partial);
+  }
+  MAO_CUDA_TRY(cudaGetLastError());
+  {
+    LaunchScope ls(stream, MAO_K_MUON_SCALE, 0.0, 4.0 * P.prep_blocks);
+    muon_scale_kernel<<<(count + 7) / 8, 256, 0, stream>>>(T, count, partial, p->eps, scale);
+  }
+  MAO_CUDA_TRY(cudaGetLastError());
+
+  // 3: Newton-Schulz over every class, at most kMaxClasses per launch
+  if (p->ns_steps > 0) {
+    const int ncls = (int)P.cls.size();
+    // descriptors per class: X[k] (K-major, rows s), XT[k] (rows l), A, B
+    struct ClassMaps {
+      CUtensorMap XA[2], XB[2], XTB[2], AA, AB, BA;
+    };
+    std::vector<ClassMaps> maps(ncls);
+    for (int c = 0; c < ncls; ++c) {
+      const MuonClass& C = P.cls[c];
+      const uint64_t cnt = C.mats.size();
+      for (int k = 0; k < 2; ++k) {
+        OperandView xv{ws + C.off_X[k], (uint64_t)C.l, (uint64_t)C.s, cnt, (uint64_t)C.ld_l,
+                       (uint64_t)C.s * C.ld_l};
+        MAO_TRY(encode_operand(&maps[c].XA[k], OP_BF16, 0, 128, xv));
+        MAO_TRY(encode_operand(&maps[c].XB[k], OP_BF16, 0, 256, xv));
+        OperandView tv{ws + C.off_XT[k], (uint64_t)C.s, (uint64_t)C.l, cnt, (uint64_t)C.ld_s,
+                       (uint64_t)C.l * C.ld_s};
+        MAO_TRY(encode_operand(&maps[c].XTB[k], OP_BF16, 0, 256, tv));
+      }
+      OperandView av{ws + C.off_A, (uint64_t)C.s, (uint64_t)C.s, cnt, (uint64_t)C.ld_s, (uint64_t)C.s * C.ld_s};
+      MAO_TRY(encode_operand(&maps[c].AA, OP_BF16, 0, 128, av));
+      MAO_TRY(encode_operand(&maps[c].AB, OP_BF16, 0, 256, av));
+      OperandView bv{ws + C.off_B, (uint64_t)C.s, (uint64_t)C.s, cnt, (uint64_t)C.ld_s, (uint64_t)C.s * C.ld_s};
+      MAO_TRY(encode_operand(&maps[c].BA, OP_BF16, 0, 128, bv));
+    }
+    for (int it = 0; it < p->ns_steps; ++it) {
+      const float* cf = p->ns_coef ? p->ns_coef + 3 * it : kDefaultCoef;
+      const int cur = it % 2, nxt = (it + 1) % 2;
+      for (int g0 = 0; g0 < ncls; g0 += kMaxClasses) {
+        const int g1 = std::min(ncls, g0 + kMaxClasses);
+        GemmParams g1p, g2p, g3p;
+        std::memset(&g1p, 0, sizeof(g1p));
+        std::memset(&g2p, 0, sizeof(g2p));
+        std::memset(&g3p, 0, sizeof(g3p));
+        g1p.nclasses = g2p.nclasses = g3p.nclasses = g1 - g0;
+        g1p.status = g2p.status = g3p.status = status;
+        g2p.beta = cf[1];
+        g2p.gamma = cf[2];
+        g3p.alpha = cf[0];
+        for (int c = g0; c < g1; ++c) {
+          const MuonClass& C = P.cls[c];
+          const int k = c - g0;
+          const int cnt = (int)C.mats.size();
+          const long long xs = (long long)C.s * C.ld_l, ts = (long long)C.l * C.ld_s,
+                          as = (long long)C.s * C.ld_s;
+          const float* sc = (it == 0) ? scale + C.scale_begin : nullptr;
+          // A = s^2 X X^T
+          g1p.mapA[k] = maps[c].XA[cur];
+          g1p.mapB[k] = maps[c].XB[cur];
+          g1p.cls[k] = GemmClass{C.s, C.s, C.l, cnt, 0, 0, 0, ws + C.off_A, as, C.ld_s, nullptr, 0, 0,
+                                 nullptr, 0, 0, sc};
+          // B = b A + c A A^T
+          g2p.mapA[k] = maps[c].AA;
+          g2p.mapB[k] = maps[c].AB;
+          g2p.cls[k] = GemmClass{C.s, C.s, C.s, cnt, 0, 0, 0, ws + C.off_B, as, C.ld_s, nullptr, 0, 0,
+                                 ws + C.off_A, as, C.ld_s, nullptr};
+          // X' = s (a X + B X), X'^T
+          g3p.mapA[k] = maps[c].BA;
+          g3p.mapB[k] = maps[c].XTB[cur];
+          g3p.cls[k] = GemmClass{C.s, C.l, C.s, cnt, 0, 0, 0, ws + C.off_X[nxt], xs, C.ld_l, ws + C.off_XT[nxt],
+                                 ts, C.ld_s, ws + C.off_X[cur], xs, C.ld_l, sc};
+        }
+        finalize_classes(g1p);
+        finalize_classes(g2p);
+        finalize_classes(g3p);
+        MAO_TRY(launch_gemm(OP_BF16, 0, 0, EPI_GRAM, g1p, nullptr, stream, MAO_K_NS_GRAM));
+        MAO_TRY(launch_gemm(OP_BF16, 0, 0, EPI_POLY, g2p, nullptr, stream, MAO_K_NS_POLY));
+        MAO_TRY(launch_gemm(OP_BF16, 0, 0, EPI_AXPY_T, g3p, nullptr, stream, MAO_K_NS_AXPY));
+      }
+    }
+  }
+
+  // 4: Muon+ scales
+  const int mode = p->norm;
+  auto colpass = [&](int use_rows_flag) -> mao_status {
+    {
+      LaunchScope ls(stream, MAO_K_MUON_COLSQ, 0.0, 2.0 * elems);
+      muon_colsq_kernel<<<P.colsq_blocks, 256, 0, stream>>>(T, count, use_rows_flag);
+    }
+    MAO_CUDA_TRY(cudaGetLastError());
+    int maxn = 0;
+    for (int i = 0; i < count; ++i) maxn = std::max(maxn, mats[i].n);
+    dim3 g((maxn + 255) / 256, count);
+    {
+      LaunchScope ls(stream, MAO_K_MUON_COLSCALE, 0.0, 0.0);
+      muon_colscale_kernel<<<g, 256, 0, stream>>>(T, count);
+    }
+    MAO_CUDA_TRY(cudaGetLastError());
+    return MAO_OK;
+  };
+  auto rowpass = [&](int use_cols_flag) -> mao_status {
+    {
+      LaunchScope ls(stream, MAO_K_MUON_ROWSCALE, 0.0, 2.0 * elems);
+      muon_rowscale_kernel<<<(P.total_rows + 7) / 8, 256, 0, stream>>>(T, count, rowbegin, P.total_rows,
+                                                                         use_cols_flag);
+    }
+    MAO_CUDA_TRY(cudaGetLastError());
+    return MAO_OK;
+  };
+  if (mode == MAO_NORM_COL) {
+    MAO_TRY(colpass(0));
+  } else if (mode == MAO_NORM_ROW) {
+    MAO_TRY(rowpass(0));
+  } else if (mode == MAO_NORM_COL_ROW) {
+    MAO_TRY(colpass(0));
+    MAO_TRY(rowpass(1));
+  } else if (mode == MAO_NORM_ROW_COL) {
+    MAO_TRY(rowpass(0));
+    MAO_TRY(colpass(1));
+  }
+
+  // 5-6: update and stats
+  const float decay = 1.0f - p->lr * p->wd;
+  {
+    LaunchScope ls(stream, MAO_K_MUON_UPDATE, 0.0, elems * (2.0 + 4.0 + 4.0));
+    muon_update_kernel<<<P.upd_blocks, 256, 0, stream>>>(T, count, decay, P.use_rows ? 1 : 0, P.use_cols ? 1 : 0,
+                                                        stats ? updpart : nullptr, stats ? updbad : nullptr);
+  }
+  MAO_CUDA_TRY(cudaGetLastError());
+  if (stats) {
+    {
+      LaunchScope ls(stream, MAO_K_MUON_STATS, 0.0, 8.0 * P.upd_blocks);
+      muon_stats_kernel<<<(count + 7) / 8, 256, 0, stream>>>(T, count, updpart, updbad, stats);
+    }
+    MAO_CUDA_TRY(cudaGetLastError());
+  }
+  (void)dev;
+  return MAO_OK;
+}

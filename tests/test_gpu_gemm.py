@@ -1,0 +1,63 @@
+"""The grouped tcgen05 GEMM core against a plain fp32 PyTorch product of the
+same operands (bf16 and 3xTF32 kinds, all four operand-major combinations,
+shapes spanning several tiles with ragged tails)."""
+
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def api():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from matrix_aware_optimizers_02_b200 import api as A
+    return A
+
+
+def _operands(batch, M, N, K, a_mn, b_mn, dtype, gen):
+    A = torch.randn((batch, M, K), generator=gen, device="cuda").to(dtype)
+    B = torch.randn((batch, N, K), generator=gen, device="cuda").to(dtype)
+    Ain = A.transpose(1, 2).contiguous() if a_mn else A
+    Bin = B.transpose(1, 2).contiguous() if b_mn else B
+    return A, B, Ain, Bin
+
+
+SHAPES = [(1, 128, 256, 64), (3, 200, 328, 136), (2, 384, 520, 1000), (1, 8, 8, 8)]
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_bf16_gemm_matches_fp32_product(api, shape, a_mn, b_mn):
+    batch, M, N, K = shape
+    gen = torch.Generator(device="cuda").manual_seed(1234)
+    A, B, Ain, Bin = _operands(batch, M, N, K, a_mn, b_mn, torch.bfloat16, gen)
+    D = api.gemm(Ain, Bin, kind="bf16", a_mn_major=bool(a_mn), b_mn_major=bool(b_mn))
+    ref = torch.bmm(A.double(), B.double().transpose(1, 2))
+    # exact bf16 products, fp32 accumulation: error ~ sqrt(K) * 2^-24 * |a||b|
+    err = (D.double() - ref).abs().max().item()
+    assert err <= 1e-5 * K ** 0.5 * 4, err
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_tf32x3_gemm_is_fp32_faithful(api, shape, a_mn, b_mn):
+    batch, M, N, K = shape
+    gen = torch.Generator(device="cuda").manual_seed(99)
+    A, B, Ain, Bin = _operands(batch, M, N, K, a_mn, b_mn, torch.float32, gen)
+    D = api.gemm(Ain, Bin, kind="tf32x3", a_mn_major=bool(a_mn), b_mn_major=bool(b_mn))
+    ref = torch.bmm(A.double(), B.double().transpose(1, 2))
+    scale = torch.bmm(A.double().abs(), B.double().abs().transpose(1, 2))
+    rel = ((D.double() - ref).abs() / scale).max().item()
+    # a plain tf32 product would sit near 1e-3 here; three passes reach ~1e-6
+    assert rel < 2e-5, rel
+
+
+def test_gemm_repeatable_bitwise(api):
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    A = torch.randn((4, 256, 512), generator=gen, device="cuda").to(torch.bfloat16)
+    B = torch.randn((4, 512, 512), generator=gen, device="cuda").to(torch.bfloat16)
+    d1 = api.gemm(A, B)
+    d2 = api.gemm(A, B)
+    assert torch.equal(d1, d2)

@@ -1,0 +1,133 @@
+"""Muon / Muon+ through the C ABI against the float64 oracle on the same seeded
+inputs.  Tolerance: 2e-2 relative Frobenius error on the orthogonalised
+direction O and on the weight update dW (Newton-Schulz runs with bf16 operands,
+whose unit roundoff is 2^-8); the momentum is fp32 arithmetic and must agree to
+fp32 rounding."""
+
+import numpy as np
+import pytest
+import torch
+
+from matrix_aware_optimizers_02_b200 import synth
+from oracle import mao_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+NS_TOL = 2e-2
+
+
+@pytest.fixture(scope="module")
+def api():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from matrix_aware_optimizers_02_b200 import api as A
+    return A
+
+
+def _rel(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def _run(api, inputs, g_bf16, **kw):
+    """Run one GPU step; return per matrix (W_new, M_new) as float64 numpy."""
+    dev = []
+    for (W, G, M) in inputs:
+        Wt = torch.from_numpy(W).cuda()
+        Gt = torch.from_numpy(G).cuda()
+        if g_bf16:
+            Gt = Gt.to(torch.bfloat16)
+        Mt = torch.from_numpy(M).cuda()
+        dev.append((Wt, Gt, Mt))
+    step = api.MuonBatch(dev, **kw)
+    step()
+    assert step.device_status() == 0
+    torch.cuda.synchronize()
+    return [(w.double().cpu().numpy(), m.double().cpu().numpy()) for (w, _, m) in dev], step
+
+
+def _check(inputs, outs, *, mu, lr, wd=0.0, norm=O.NORM_NONE, ns_steps=5, coefs=None):
+    worst = 0.0
+    for (W, G, M), (Wg, Mg) in zip(inputs, outs):
+        m, n = W.shape
+        Wo, Mo, Oo = O.muon_step(W, G, M, mu=mu, lr=lr, wd=wd, norm=norm, ns_steps=ns_steps, ns_coefs=coefs)
+        # momentum: fp32 fused multiply-add vs float64
+        assert np.allclose(Mg, Mo, rtol=1e-5, atol=1e-7 * max(np.abs(Mo).max(), 1e-30))
+        dW_gpu = Wg - W
+        dW_ref = Wo - W
+        e = _rel(dW_gpu, dW_ref)
+        if wd == 0.0:
+            # O = -dW / (lr sqrt(m/n))
+            e = max(e, _rel(-dW_gpu / (lr * np.sqrt(m / n)), Oo))
+        worst = max(worst, e)
+        assert e < NS_TOL, (m, n, e)
+    return worst
+
+
+def test_muon_single_256x512(api):
+    """The single-weight case: W, G, M ~ N(0, 0.02^2), seed 0, mu 0.95, lr 0.02, 5 NS steps."""
+    W, G, M = synth.muon_single_inputs(0)
+    inputs = [(W.astype(np.float64), G.astype(np.float64), M.astype(np.float64))]
+    outs, _ = _run(api, [(W, G, M)], False, mu=0.95, lr=0.02)
+    _check(inputs, outs, mu=0.95, lr=0.02)
+
+
+RAGGED = [synth.MatSpec(200, 328, 0.02), synth.MatSpec(328, 200, 0.02), synth.MatSpec(64, 64, 0.02),
+          synth.MatSpec(8, 1000, 0.02), synth.MatSpec(1000, 8, 0.02), synth.MatSpec(264, 264, 0.02),
+          synth.MatSpec(520, 136, 0.02)]
+
+
+@pytest.mark.parametrize("g_bf16", [False, True])
+def test_muon_ragged_batch(api, g_bf16):
+    """Mixed shapes (several tiles, ragged tails, both orientations) in one call."""
+    inputs = synth.muon_inputs(RAGGED, seed=3, g_bf16=g_bf16, m_std=0.02)
+    outs, _ = _run(api, inputs, g_bf16, mu=0.9, lr=0.05, wd=0.1)
+    _check([tuple(a.astype(np.float64) for a in x) for x in inputs], outs, mu=0.9, lr=0.05, wd=0.1)
+
+
+@pytest.mark.parametrize("norm", ["row", "col", "col_row", "row_col"])
+def test_muon_plus_modes(api, norm):
+    specs = [synth.MatSpec(192, 320, 0.02), synth.MatSpec(320, 192, 0.02), synth.MatSpec(128, 128, 0.02)]
+    inputs = synth.muon_inputs(specs, seed=4, g_bf16=True)
+    outs, _ = _run(api, inputs, True, mu=0.95, lr=0.02, norm=norm)
+    mode = {"row": O.NORM_ROW, "col": O.NORM_COL, "col_row": O.NORM_COL_ROW, "row_col": O.NORM_ROW_COL}[norm]
+    _check([tuple(a.astype(np.float64) for a in x) for x in inputs], outs, mu=0.95, lr=0.02, norm=mode)
+
+
+def test_custom_coefficients_and_step_counts(api):
+    specs = [synth.MatSpec(96, 160, 0.02)]
+    inputs = synth.muon_inputs(specs, seed=5, m_std=0.02)
+    f64 = [tuple(a.astype(np.float64) for a in x) for x in inputs]
+    coefs = [(3.0, -3.2, 1.2), (2.0, -1.5, 0.5), (1.875, -1.25, 0.375)]
+    outs, _ = _run(api, inputs, False, mu=0.95, lr=0.02, ns_steps=3, ns_coef=coefs)
+    _check(f64, outs, mu=0.95, lr=0.02, ns_steps=3, coefs=coefs)
+    for k in (0, 1, 2):
+        outs, _ = _run(api, inputs, False, mu=0.95, lr=0.02, ns_steps=k)
+        _check(f64, outs, mu=0.95, lr=0.02, ns_steps=k)
+
+
+def test_gpt2_124m_batch_sampled(api):
+    """The GPT-2-124M-shaped Muon+ set (48 matrices, bf16 G ~ N(0, 0.02^2), Col-Row) in one
+    call; one matrix of each shape compared with the oracle."""
+    specs = synth.specs_gpt2_124m()
+    inputs = synth.muon_inputs(specs, seed=0, g_bf16=True)
+    outs, _ = _run(api, inputs, True, mu=0.95, lr=0.02, norm="col_row")
+    pick = [0, 1, 2, 3, 45]
+    _check([tuple(a.astype(np.float64) for a in inputs[i]) for i in pick], [outs[i] for i in pick], mu=0.95,
+           lr=0.02, norm=O.NORM_COL_ROW)
+
+
+def test_deterministic_and_stats(api):
+    specs = [synth.MatSpec(256, 768, 0.02), synth.MatSpec(768, 256, 0.02)]
+    inputs = synth.muon_inputs(specs, seed=6, g_bf16=True, m_std=0.01)
+    o1, s1 = _run(api, inputs, True, mu=0.95, lr=0.02, with_stats=True)
+    o2, _ = _run(api, inputs, True, mu=0.95, lr=0.02, with_stats=True)
+    for (a, b), (c, d) in zip(o1, o2):
+        assert np.array_equal(a, c) and np.array_equal(b, d)
+    st = s1.stats_dict()
+    for i, (W, G, M) in enumerate(inputs):
+        dw = o1[i][0] - W.astype(np.float64)
+        rms = np.linalg.norm(dw) / np.sqrt(dw.size)
+        assert abs(st["update_rms"][i] - rms) <= 1e-3 * rms
+        assert st["nonfinite"][i] == 0
