@@ -167,13 +167,16 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 //   K-major: rows of 128 B along K, 8-row atoms of 1024 B; SBO = 1024 B, LBO unused (16 B).
 //   MN-major: 128 B along MN per K row, 8 K-rows per 1024-B atom; SBO = 1024 B between
 //   8-row K groups, LBO = byte distance between consecutive 128-B MN chunks.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+//   32-bit MN-major operands use the 128-byte swizzle with 32-byte atoms
+//   instead (layout type 1): 4 K-rows of 128 B per 512-B atom, SBO = 512 B.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                                    uint32_t layout_type = 2) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
   d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= 1ull << 46;  // descriptor version for sm_100
-  d |= 2ull << 61;  // SWIZZLE_128B
+  d |= 1ull << 46;                                      // descriptor version for sm_100
+  d |= static_cast<uint64_t>(layout_type & 7u) << 61;  // 2 = SWIZZLE_128B, 1 = SWIZZLE_128B_BASE32B
   return d;
 }
 

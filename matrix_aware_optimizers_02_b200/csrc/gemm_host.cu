@@ -49,7 +49,7 @@ mao_status device_info(DeviceInfo** out) {
 
 mao_status encode_3d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* base, uint64_t inner,
                      uint64_t rows, uint64_t batch, uint64_t ld_elems, uint64_t batch_stride_elems,
-                     uint32_t box_inner, uint32_t box_rows) {
+                     uint32_t box_inner, uint32_t box_rows, bool atom32) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   MAO_TRY(get_encode(&enc));
   cuuint64_t dims[3] = {inner, rows, batch};
@@ -57,7 +57,8 @@ mao_status encode_3d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const 
   cuuint32_t box[3] = {box_inner, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   atom32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MAO_OK : MAO_ERR_CUDA;
 }
@@ -67,9 +68,11 @@ mao_status encode_operand(CUtensorMap* map, int kind, int mn_major, int R, const
   const CUtensorMapDataType dt =
       (kind == OP_BF16) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const uint32_t row_elems = 128 / esize;  // elements in one 128-byte swizzle row
-  if (!mn_major) return encode_3d(map, dt, esize, v.base, v.inner, v.rows, v.batch, v.ld, v.bstride, row_elems, R);
-  (void)R;
-  return encode_3d(map, dt, esize, v.base, v.inner, v.rows, v.batch, v.ld, v.bstride, row_elems, row_elems);
+  if (!mn_major)
+    return encode_3d(map, dt, esize, v.base, v.inner, v.rows, v.batch, v.ld, v.bstride, row_elems, R, false);
+  // MN-major 32-bit operands need the 32-byte-atom variant of the 128-byte swizzle
+  return encode_3d(map, dt, esize, v.base, v.inner, v.rows, v.batch, v.ld, v.bstride, row_elems, row_elems,
+                   esize == 4);
 }
 
 void finalize_classes(GemmParams& p) {

@@ -106,6 +106,8 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int k) {
     // BK*128 bytes; a k-step covers UMMA_K K-rows = (32/ESIZE) rows of 128 B.
     constexpr int BK = 128 / ESIZE;
     constexpr int ROWS_PER_STEP = UMMA_K_BYTES / ESIZE;
+    if constexpr (ESIZE == 4)  // tf32: 128-byte swizzle of 32-byte atoms, 4-row (512 B) groups
+      return smem_desc_sw128(base + k * ROWS_PER_STEP * 128, BK * 128, 512, 1);
     return smem_desc_sw128(base + k * ROWS_PER_STEP * 128, BK * 128, 1024);
   }
 }

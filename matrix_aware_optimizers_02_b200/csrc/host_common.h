@@ -54,7 +54,7 @@ struct DeviceInfo {
 mao_status device_info(DeviceInfo** out);
 mao_status encode_3d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* base, uint64_t inner,
                      uint64_t rows, uint64_t batch, uint64_t ld_elems, uint64_t batch_stride_elems,
-                     uint32_t box_inner, uint32_t box_rows);
+                     uint32_t box_inner, uint32_t box_rows, bool atom32 = false);
 
 // Operand descriptor for one class of a grouped GEMM: tensor [batch][rows][ld]
 // (rows x inner valid), plus the box shape the kernel expects for its major.
