@@ -150,6 +150,33 @@ MAO_API mao_status mao_muon_workspace_size(const mao_muon_mat* mats, int32_t cou
 MAO_API mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, const mao_muon_params* p, void* workspace,
                          size_t ws_bytes, mao_stats* stats, mao_stream_t stream);
 
+/* Size of the static device scratch behind mao_muon_step_noalloc. */
+#define MAO_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * mao_muon_step_noalloc — an addition of this library with no counterpart in
+ * the source pages.  Some callers cannot allocate device memory for the step's
+ * scratch workspace: a host program that runs under a device-memory budget fixed
+ * at start-up, or a caller inside a framework whose own caching allocator owns
+ * the device memory, has no allocator at hand for a raw scratch buffer.  This
+ * entry point runs the same step as mao_muon_step but takes its scratch from one
+ * static device array of MAO_NOALLOC_SCRATCH_BYTES (64 MiB) built into the
+ * library, which every GPU that loads the library holds until the process exits.
+ *   - The caller still passes the matrices (W, G, M) and optional stats.
+ *   - A batch whose mao_muon_workspace_size() exceeds MAO_NOALLOC_SCRATCH_BYTES is
+ *     rejected with MAO_ERR_WORKSPACE before anything is enqueued.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *     first call before any stream capture on that device.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - Every call shares the one array, and the array keeps the last call's
+ *     contents; each call clears what must start at zero (the status word).
+ *     Calls whose work overlaps on the GPU (different streams, or different
+ *     threads without ordering) race on the array: serialise them.
+ */
+MAO_API mao_status mao_muon_step_noalloc(const mao_muon_mat* mats, int32_t count, const mao_muon_params* p,
+                                         mao_stats* stats, mao_stream_t stream);
+
 /* ------------------------------------------------------------------ SOAP */
 
 typedef struct {

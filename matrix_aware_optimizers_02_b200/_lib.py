@@ -84,6 +84,7 @@ SIGNATURES = {
     "mao_muon_workspace_size": (c_int32, [POINTER(MuonMat), c_int32, POINTER(MuonParams), POINTER(c_size_t)]),
     "mao_muon_step": (c_int32, [POINTER(MuonMat), c_int32, POINTER(MuonParams), c_void_p, c_size_t, c_void_p,
                                 c_void_p]),
+    "mao_muon_step_noalloc": (c_int32, [POINTER(MuonMat), c_int32, POINTER(MuonParams), c_void_p, c_void_p]),
     "mao_soap_workspace_size": (c_int32, [POINTER(SoapMat), c_int32, POINTER(SoapParams), POINTER(c_size_t)]),
     "mao_soap_step": (c_int32, [POINTER(SoapMat), c_int32, POINTER(SoapParams), c_void_p, c_size_t, c_void_p,
                                 c_void_p]),
