@@ -138,8 +138,8 @@ mao_status launch_gemm(int kind, int a_mn, int b_mn, int epi, const GemmParams& 
                        cudaStream_t stream, int k) {
   if (kind == OP_BF16) {
     if (!a_mn && !b_mn) return launch_epi<OP_BF16, 0, 0>(epi, p, lo, stream, k);
+    if (!a_mn && b_mn) return launch_epi<OP_BF16, 0, 1>(epi, p, lo, stream, k);
     if (epi != EPI_STORE_F32) return MAO_ERR_UNSUPPORTED;
-    if (!a_mn && b_mn) return launch_one<OP_BF16, 0, 1, EPI_STORE_F32>(p, lo, stream, k);
     if (a_mn && !b_mn) return launch_one<OP_BF16, 1, 0, EPI_STORE_F32>(p, lo, stream, k);
     return launch_one<OP_BF16, 1, 1, EPI_STORE_F32>(p, lo, stream, k);
   }
@@ -155,12 +155,6 @@ mao_status launch_gemm(int kind, int a_mn, int b_mn, int epi, const GemmParams& 
 
 // ------------------------------------------------------------------ tf32 split
 namespace {
-
-__device__ __forceinline__ float tf32_rna(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return __uint_as_float(r);
-}
 
 // x = hi + lo with hi = tf32(x) and lo = tf32(x - hi): both exactly representable
 // in tf32, so the tensor core sees them without further rounding.

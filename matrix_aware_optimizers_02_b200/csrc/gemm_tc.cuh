@@ -36,7 +36,7 @@ enum EpiKind : int {
   EPI_STORE_F32 = 0,  // out0 (f32) = alpha * acc
   EPI_GRAM = 1,       // out0 (bf16) = acc * s_b^2                    (A = X X^T)
   EPI_POLY = 2,       // out0 (bf16) = beta * aux + gamma * acc       (B = b A + c A A)
-  EPI_AXPY_T = 3,     // v = s_b * (alpha * aux + acc); out0 (bf16) = v, out1 = v^T  (X = a X + B X)
+  EPI_AXPY_T = 3,     // v = s_b * (alpha * aux + acc); out0 (bf16) = v, out1 = v^T if given  (X = a X + B X)
 };
 
 struct GemmClass {
@@ -209,12 +209,14 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, const GemmCl
       for (int j = 0; j < 32 && col0 + j < C.N; ++j) out[j] = __float2bfloat16_rn(v[j]);
     }
     if constexpr (EPI == EPI_AXPY_T) {
-      // transposed copy: for each column j, the 32 lanes (consecutive rows) write
-      // 32 consecutive elements of row (col0 + j) of out1.
-      __nv_bfloat16* t = reinterpret_cast<__nv_bfloat16*>(C.out1) + (long long)b * C.out1_bs + row;
+      if (C.out1 != nullptr) {
+        // optional transposed copy: for each column j, the 32 lanes (consecutive
+        // rows) write 32 consecutive elements of row (col0 + j) of out1.
+        __nv_bfloat16* t = reinterpret_cast<__nv_bfloat16*>(C.out1) + (long long)b * C.out1_bs + row;
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (col0 + j < C.N) t[(long long)(col0 + j) * C.out1_ld] = __float2bfloat16_rn(v[j]);
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j < C.N) t[(long long)(col0 + j) * C.out1_ld] = __float2bfloat16_rn(v[j]);
+      }
     }
   }
 }

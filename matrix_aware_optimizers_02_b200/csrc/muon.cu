@@ -1,16 +1,16 @@
 // mao_muon_step: one Muon / Muon+ step over a batch of matrices.
 //
 // Launch sequence on the caller's stream (no host synchronisation):
-//   1. muon_prep_kernel      momentum EMA, sum-of-squares partials, bf16 X / X^T
+//   1. muon_prep_kernel      momentum EMA, sum-of-squares partials, bf16 X (s x l)
 //   2. muon_scale_kernel     per-matrix 1/(||M||_F + eps)
 //   3. ns_steps x 3 grouped tcgen05 GEMMs over every shape class at once:
-//        A = s^2 X X^T                     (EPI_GRAM, s = the scale on iteration 0)
-//        B = b A + c A A                   (EPI_POLY; A is symmetric, so A A = A A^T)
-//        X' = s (a X + B X), and X'^T      (EPI_AXPY_T)
+//        A = s^2 X X^T            (EPI_GRAM; both operands X, K-major)
+//        B = b A + c A A          (EPI_POLY; A is symmetric, so A A = A A^T, K-major)
+//        X' = s (a X + B X)       (EPI_AXPY_T; B K-major, X read MN-major)
 //      Iteration 0 works on the unnormalised bf16(M) and applies the per-matrix
 //      scale s in the epilogues, which equals normalising first:
 //        s^2 X X^T = (sX)(sX)^T and s (a X + B X) = a (sX) + B (sX).
-//   4. Muon+ row/column scales (optional)
+//   4. Muon+ row/column scales (optional), 64 x 64 tile passes
 //   5. muon_update_kernel    W <- W (1 - lr wd) - lr sqrt(m/n) Norm(O)
 //   6. muon_stats_kernel     (optional)
 #include <algorithm>
@@ -31,16 +31,16 @@ struct MuonClass {
   int s = 0, l = 0;           // X is s x l
   std::vector<int> mats;      // global matrix indices, in batch order
   int ld_l = 0, ld_s = 0;     // padded leading dimensions (multiples of 8)
-  size_t off_X[2] = {}, off_XT[2] = {}, off_A = 0, off_B = 0;
+  size_t off_X[2] = {}, off_A = 0, off_B = 0;
   int scale_begin = 0;        // first slot in the scale array
 };
 
 struct MuonPlan {
   std::vector<MuonClass> cls;
   std::vector<int> mat_class, mat_slot;  // class of matrix p, its index in the class
-  size_t off_table = 0, off_scale = 0, off_partial = 0, off_rowscale = 0, off_colscale = 0, off_colpart = 0,
-         off_rowbegin = 0, off_updpart = 0, off_updbad = 0;
-  int prep_blocks = 0, colsq_blocks = 0, upd_blocks = 0, total_rows = 0;
+  size_t off_table = 0, off_scale = 0, off_partial = 0, off_rowscale = 0, off_colscale = 0, off_rowpart = 0,
+         off_colpart = 0, off_updpart = 0, off_updbad = 0;
+  int tiles = 0;
   size_t total = 0;
   bool use_rows = false, use_cols = false;
   std::vector<MuonMatDev> table;  // filled without device pointers by plan()
@@ -107,54 +107,41 @@ void plan(const mao_muon_mat* mats, int count, const mao_muon_params* p, MuonPla
     c.scale_begin = sb;
     sb += (int)c.mats.size();
   }
-  // per-matrix block bookkeeping
   P.table.assign(count, MuonMatDev());
-  int prep = 0, colsq = 0, upd = 0, rows = 0;
-  size_t rs_elems = 0, cs_elems = 0, cp_elems = 0;
+  int tiles = 0;
+  size_t rs_elems = 0, cs_elems = 0, rp_elems = 0, cp_elems = 0;
   for (int i = 0; i < count; ++i) {
     MuonMatDev& D = P.table[i];
     D.m = mats[i].m;
     D.n = mats[i].n;
     D.g_bf16 = mats[i].g_dtype == MAO_BF16;
-    D.ldw = round_up_int(D.n, 8);
-    D.ldt = round_up_int(D.m, 8);
-    const int tr = (D.m + kPrepTile - 1) / kPrepTile, tc = (D.n + kPrepTile - 1) / kPrepTile;
-    D.prep_tiles_c = tc;
-    D.prep_begin = prep;
-    D.prep_count = tr * tc;
-    prep += tr * tc;
-    D.col_chunks = (D.m + kColChunkRows - 1) / kColChunkRows;
-    D.colsq_begin = colsq;
-    if (P.use_cols) colsq += D.col_chunks * ((D.n + 255) / 256);
-    const long long el = (long long)D.m * D.n;
-    D.upd_begin = upd;
-    D.upd_count = (int)((el + kUpdElems - 1) / kUpdElems);
-    upd += D.upd_count;
+    D.trans = D.m > D.n ? 1 : 0;
+    D.ldx = round_up_int(std::max(D.m, D.n), 8);
+    D.tiles_r = (D.m + kTile - 1) / kTile;
+    D.tiles_c = (D.n + kTile - 1) / kTile;
+    D.tile_begin = tiles;
+    tiles += D.tiles_r * D.tiles_c;
     D.out_scale = p->lr * std::sqrt((float)D.m / (float)D.n);
     rs_elems += D.m;
     cs_elems += D.n;
-    cp_elems += (size_t)D.col_chunks * D.n;
-    rows += D.m;
+    rp_elems += (size_t)D.tiles_c * D.m;
+    cp_elems += (size_t)D.tiles_r * D.n;
   }
-  P.prep_blocks = prep;
-  P.colsq_blocks = colsq;
-  P.upd_blocks = upd;
-  P.total_rows = rows;
-  P.off_partial = cv.take(sizeof(float) * (size_t)std::max(prep, 1));
-  if (P.use_rows) P.off_rowscale = cv.take(sizeof(float) * rs_elems);
+  P.tiles = tiles;
+  P.off_partial = cv.take(sizeof(float) * (size_t)std::max(tiles, 1));
+  if (P.use_rows) {
+    P.off_rowscale = cv.take(sizeof(float) * rs_elems);
+    P.off_rowpart = cv.take(sizeof(float) * rp_elems);
+  }
   if (P.use_cols) {
     P.off_colscale = cv.take(sizeof(float) * cs_elems);
     P.off_colpart = cv.take(sizeof(float) * cp_elems);
   }
-  if (P.use_rows) P.off_rowbegin = cv.take(sizeof(int) * (size_t)std::max(count, 1));
-  P.off_updpart = cv.take(sizeof(float) * (size_t)std::max(upd, 1));
-  P.off_updbad = cv.take(sizeof(int) * (size_t)std::max(upd, 1));
+  P.off_updpart = cv.take(sizeof(float) * (size_t)std::max(tiles, 1));
+  P.off_updbad = cv.take(sizeof(int) * (size_t)std::max(tiles, 1));
   for (auto& c : P.cls) {
     const size_t cnt = c.mats.size();
-    for (int k = 0; k < 2; ++k) {
-      c.off_X[k] = cv.take(2 * cnt * (size_t)c.s * c.ld_l);
-      c.off_XT[k] = cv.take(2 * cnt * (size_t)c.l * c.ld_s);
-    }
+    for (int k = 0; k < 2; ++k) c.off_X[k] = cv.take(2 * cnt * (size_t)c.s * c.ld_l);
     c.off_A = cv.take(2 * cnt * (size_t)c.s * c.ld_s);
     c.off_B = cv.take(2 * cnt * (size_t)c.s * c.ld_s);
   }
@@ -194,17 +181,15 @@ extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, con
   float* scale = reinterpret_cast<float*>(ws + P.off_scale);
   float* partial = reinterpret_cast<float*>(ws + P.off_partial);
   float* rowscale = P.use_rows ? reinterpret_cast<float*>(ws + P.off_rowscale) : nullptr;
+  float* rowpart = P.use_rows ? reinterpret_cast<float*>(ws + P.off_rowpart) : nullptr;
   float* colscale = P.use_cols ? reinterpret_cast<float*>(ws + P.off_colscale) : nullptr;
   float* colpart = P.use_cols ? reinterpret_cast<float*>(ws + P.off_colpart) : nullptr;
-  int* rowbegin = P.use_rows ? reinterpret_cast<int*>(ws + P.off_rowbegin) : nullptr;
   float* updpart = reinterpret_cast<float*>(ws + P.off_updpart);
   int* updbad = reinterpret_cast<int*>(ws + P.off_updbad);
   const int fin = p->ns_steps % 2;
 
   // device table
-  std::vector<int> rb(count);
-  size_t rs_off = 0, cs_off = 0, cp_off = 0;
-  int rows = 0;
+  size_t rs_off = 0, cs_off = 0, rp_off = 0, cp_off = 0;
   for (int i = 0; i < count; ++i) {
     MuonMatDev& D = P.table[i];
     const MuonClass& C = P.cls[P.mat_class[i]];
@@ -212,48 +197,42 @@ extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, con
     D.W = mats[i].W;
     D.G = mats[i].G;
     D.M = mats[i].M;
-    __nv_bfloat16* X0 = reinterpret_cast<__nv_bfloat16*>(ws + C.off_X[0]) + (size_t)b * C.s * C.ld_l;
-    __nv_bfloat16* XT0 = reinterpret_cast<__nv_bfloat16*>(ws + C.off_XT[0]) + (size_t)b * C.l * C.ld_s;
-    __nv_bfloat16* Xf = reinterpret_cast<__nv_bfloat16*>(ws + C.off_X[fin]) + (size_t)b * C.s * C.ld_l;
-    __nv_bfloat16* XTf = reinterpret_cast<__nv_bfloat16*>(ws + C.off_XT[fin]) + (size_t)b * C.l * C.ld_s;
-    const bool wide = D.m <= D.n;
-    D.Xw = wide ? X0 : XT0;
-    D.Xt = wide ? XT0 : X0;
-    D.O = wide ? Xf : XTf;
+    D.X0 = reinterpret_cast<__nv_bfloat16*>(ws + C.off_X[0]) + (size_t)b * C.s * C.ld_l;
+    D.O = reinterpret_cast<__nv_bfloat16*>(ws + C.off_X[fin]) + (size_t)b * C.s * C.ld_l;
     D.rowscale = rowscale ? rowscale + rs_off : nullptr;
+    D.rowpart = rowpart ? rowpart + rp_off : nullptr;
     D.colscale = colscale ? colscale + cs_off : nullptr;
     D.colpart = colpart ? colpart + cp_off : nullptr;
     D.oscale = (p->ns_steps == 0) ? scale + C.scale_begin + b : nullptr;
     D.scale_slot = C.scale_begin + b;
     rs_off += D.m;
     cs_off += D.n;
-    cp_off += (size_t)D.col_chunks * D.n;
-    rb[i] = rows;
-    rows += D.m;
+    rp_off += (size_t)D.tiles_c * D.m;
+    cp_off += (size_t)D.tiles_r * D.n;
   }
   MAO_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream));
   MAO_CUDA_TRY(cudaMemcpyAsync(ws + P.off_table, P.table.data(), sizeof(MuonMatDev) * count,
                                cudaMemcpyHostToDevice, stream));
-  if (rowbegin)
-    MAO_CUDA_TRY(cudaMemcpyAsync(rowbegin, rb.data(), sizeof(int) * count, cudaMemcpyHostToDevice, stream));
   const MuonMatDev* T = reinterpret_cast<const MuonMatDev*>(ws + P.off_table);
 
   // algorithmic bytes of the elementwise passes
   double elems = 0.0, g_bytes = 0.0;
+  int maxdim = 0;
   for (int i = 0; i < count; ++i) {
     const double e = (double)mats[i].m * mats[i].n;
     elems += e;
     g_bytes += e * (mats[i].g_dtype == MAO_BF16 ? 2.0 : 4.0);
+    maxdim = std::max(maxdim, std::max(mats[i].m, mats[i].n));
   }
 
-  // 1-2: momentum, partial norms, bf16 operands, per-matrix scale
+  // 1-2: momentum, partial norms, bf16 operand, per-matrix scale
   {
-    LaunchScope ls(stream, MAO_K_MUON_PREP, 0.0, g_bytes + elems * (4.0 + 4.0 + 2.0 + 2.0));
-    muon_prep_kernel<<<P.prep_blocks, 256, 0, stream>>>(T, count, p->mu, partial);
+    LaunchScope ls(stream, MAO_K_MUON_PREP, 0.0, g_bytes + elems * (4.0 + 4.0 + 2.0));
+    muon_prep_kernel<<<P.tiles, 256, 0, stream>>>(T, count, p->mu, partial);
   }
   MAO_CUDA_TRY(cudaGetLastError());
   {
-    LaunchScope ls(stream, MAO_K_MUON_SCALE, 0.0, 4.0 * P.prep_blocks);
+    LaunchScope ls(stream, MAO_K_MUON_SCALE, 0.0, 4.0 * P.tiles);
     muon_scale_kernel<<<(count + 7) / 8, 256, 0, stream>>>(T, count, partial, p->eps, scale);
   }
   MAO_CUDA_TRY(cudaGetLastError());
@@ -261,9 +240,8 @@ extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, con
   // 3: Newton-Schulz over every class, at most kMaxClasses per launch
   if (p->ns_steps > 0) {
     const int ncls = (int)P.cls.size();
-    // descriptors per class: X[k] (K-major, rows s), XT[k] (rows l), A, B
     struct ClassMaps {
-      CUtensorMap XA[2], XB[2], XTB[2], AA, AB, BA;
+      CUtensorMap XA[2], XB[2], XMN[2], AA, AB, BA;
     };
     std::vector<ClassMaps> maps(ncls);
     for (int c = 0; c < ncls; ++c) {
@@ -274,9 +252,7 @@ extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, con
                        (uint64_t)C.s * C.ld_l};
         MAO_TRY(encode_operand(&maps[c].XA[k], OP_BF16, 0, 128, xv));
         MAO_TRY(encode_operand(&maps[c].XB[k], OP_BF16, 0, 256, xv));
-        OperandView tv{ws + C.off_XT[k], (uint64_t)C.s, (uint64_t)C.l, cnt, (uint64_t)C.ld_s,
-                       (uint64_t)C.l * C.ld_s};
-        MAO_TRY(encode_operand(&maps[c].XTB[k], OP_BF16, 0, 256, tv));
+        MAO_TRY(encode_operand(&maps[c].XMN[k], OP_BF16, 1, 256, xv));  // X as K x N (K = s rows)
       }
       OperandView av{ws + C.off_A, (uint64_t)C.s, (uint64_t)C.s, cnt, (uint64_t)C.ld_s, (uint64_t)C.s * C.ld_s};
       MAO_TRY(encode_operand(&maps[c].AA, OP_BF16, 0, 128, av));
@@ -302,8 +278,7 @@ extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, con
           const MuonClass& C = P.cls[c];
           const int k = c - g0;
           const int cnt = (int)C.mats.size();
-          const long long xs = (long long)C.s * C.ld_l, ts = (long long)C.l * C.ld_s,
-                          as = (long long)C.s * C.ld_s;
+          const long long xs = (long long)C.s * C.ld_l, as = (long long)C.s * C.ld_s;
           const float* sc = (it == 0) ? scale + C.scale_begin : nullptr;
           // A = s^2 X X^T
           g1p.mapA[k] = maps[c].XA[cur];
@@ -315,72 +290,63 @@ extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, con
           g2p.mapB[k] = maps[c].AB;
           g2p.cls[k] = GemmClass{C.s, C.s, C.s, cnt, 0, 0, 0, ws + C.off_B, as, C.ld_s, nullptr, 0, 0,
                                  ws + C.off_A, as, C.ld_s, nullptr};
-          // X' = s (a X + B X), X'^T
+          // X' = s (a X + B X)
           g3p.mapA[k] = maps[c].BA;
-          g3p.mapB[k] = maps[c].XTB[cur];
-          g3p.cls[k] = GemmClass{C.s, C.l, C.s, cnt, 0, 0, 0, ws + C.off_X[nxt], xs, C.ld_l, ws + C.off_XT[nxt],
-                                 ts, C.ld_s, ws + C.off_X[cur], xs, C.ld_l, sc};
+          g3p.mapB[k] = maps[c].XMN[cur];
+          g3p.cls[k] = GemmClass{C.s, C.l, C.s, cnt, 0, 0, 0, ws + C.off_X[nxt], xs, C.ld_l, nullptr, 0, 0,
+                                 ws + C.off_X[cur], xs, C.ld_l, sc};
         }
         finalize_classes(g1p);
         finalize_classes(g2p);
         finalize_classes(g3p);
         MAO_TRY(launch_gemm(OP_BF16, 0, 0, EPI_GRAM, g1p, nullptr, stream, MAO_K_NS_GRAM));
         MAO_TRY(launch_gemm(OP_BF16, 0, 0, EPI_POLY, g2p, nullptr, stream, MAO_K_NS_POLY));
-        MAO_TRY(launch_gemm(OP_BF16, 0, 0, EPI_AXPY_T, g3p, nullptr, stream, MAO_K_NS_AXPY));
+        MAO_TRY(launch_gemm(OP_BF16, 0, 1, EPI_AXPY_T, g3p, nullptr, stream, MAO_K_NS_AXPY));
       }
     }
   }
 
-  // 4: Muon+ scales
-  const int mode = p->norm;
-  auto colpass = [&](int use_rows_flag) -> mao_status {
+  // 4: Muon+ scales (each direction: tile partials, then a fixed-order final sum)
+  auto norm_pass = [&](int rows_dir, int use_other) -> mao_status {
     {
-      LaunchScope ls(stream, MAO_K_MUON_COLSQ, 0.0, 2.0 * elems);
-      muon_colsq_kernel<<<P.colsq_blocks, 256, 0, stream>>>(T, count, use_rows_flag);
+      LaunchScope ls(stream, rows_dir ? MAO_K_MUON_ROWSCALE : MAO_K_MUON_COLSQ, 0.0, 2.0 * elems);
+      muon_norm_tile_kernel<<<P.tiles, 256, 0, stream>>>(T, count, rows_dir ? 0 : 1, rows_dir ? 1 : 0,
+                                                         (!rows_dir && use_other) ? 1 : 0,
+                                                         (rows_dir && use_other) ? 1 : 0);
     }
     MAO_CUDA_TRY(cudaGetLastError());
-    int maxn = 0;
-    for (int i = 0; i < count; ++i) maxn = std::max(maxn, mats[i].n);
-    dim3 g((maxn + 255) / 256, count);
+    dim3 g((maxdim + 255) / 256, count);
     {
       LaunchScope ls(stream, MAO_K_MUON_COLSCALE, 0.0, 0.0);
-      muon_colscale_kernel<<<g, 256, 0, stream>>>(T, count);
+      muon_norm_final_kernel<<<g, 256, 0, stream>>>(T, count, rows_dir ? 0 : 1);
     }
     MAO_CUDA_TRY(cudaGetLastError());
     return MAO_OK;
   };
-  auto rowpass = [&](int use_cols_flag) -> mao_status {
-    {
-      LaunchScope ls(stream, MAO_K_MUON_ROWSCALE, 0.0, 2.0 * elems);
-      muon_rowscale_kernel<<<(P.total_rows + 7) / 8, 256, 0, stream>>>(T, count, rowbegin, P.total_rows,
-                                                                         use_cols_flag);
-    }
-    MAO_CUDA_TRY(cudaGetLastError());
-    return MAO_OK;
-  };
+  const int mode = p->norm;
   if (mode == MAO_NORM_COL) {
-    MAO_TRY(colpass(0));
+    MAO_TRY(norm_pass(0, 0));
   } else if (mode == MAO_NORM_ROW) {
-    MAO_TRY(rowpass(0));
+    MAO_TRY(norm_pass(1, 0));
   } else if (mode == MAO_NORM_COL_ROW) {
-    MAO_TRY(colpass(0));
-    MAO_TRY(rowpass(1));
+    MAO_TRY(norm_pass(0, 0));
+    MAO_TRY(norm_pass(1, 1));
   } else if (mode == MAO_NORM_ROW_COL) {
-    MAO_TRY(rowpass(0));
-    MAO_TRY(colpass(1));
+    MAO_TRY(norm_pass(1, 0));
+    MAO_TRY(norm_pass(0, 1));
   }
 
   // 5-6: update and stats
   const float decay = 1.0f - p->lr * p->wd;
   {
     LaunchScope ls(stream, MAO_K_MUON_UPDATE, 0.0, elems * (2.0 + 4.0 + 4.0));
-    muon_update_kernel<<<P.upd_blocks, 256, 0, stream>>>(T, count, decay, P.use_rows ? 1 : 0, P.use_cols ? 1 : 0,
-                                                        stats ? updpart : nullptr, stats ? updbad : nullptr);
+    muon_update_kernel<<<P.tiles, 256, 0, stream>>>(T, count, decay, P.use_rows ? 1 : 0, P.use_cols ? 1 : 0,
+                                                   stats ? updpart : nullptr, stats ? updbad : nullptr);
   }
   MAO_CUDA_TRY(cudaGetLastError());
   if (stats) {
     {
-      LaunchScope ls(stream, MAO_K_MUON_STATS, 0.0, 8.0 * P.upd_blocks);
+      LaunchScope ls(stream, MAO_K_MUON_STATS, 0.0, 8.0 * P.tiles);
       muon_stats_kernel<<<(count + 7) / 8, 256, 0, stream>>>(T, count, updpart, updbad, stats);
     }
     MAO_CUDA_TRY(cudaGetLastError());
