@@ -63,6 +63,14 @@ def _f64(a) -> np.ndarray:
     return np.asarray(a, dtype=np.float64)
 
 
+# Working precision of the SOAP / FOAM functions below.  float64 is the oracle;
+# float32 runs the same steps in single precision and serves only to measure the
+# inherent fp32 rounding floor of a case (the tests' tolerance for quantities the
+# method amplifies).
+def _w(a, dtype):
+    return np.asarray(a, dtype=dtype)
+
+
 # --------------------------------------------------------------------------
 # Muon  ([MuonPlus] §2 Methodology; [SMB-review] §2-1 (2), §3-2 (2))
 # --------------------------------------------------------------------------
@@ -140,14 +148,14 @@ def muon_step(W, G, M, *, mu: float, lr: float, wd: float = 0.0, ns_coefs=None,
 # Shared SOAP / FOAM pieces
 # --------------------------------------------------------------------------
 
-def qr_positive(P):
+def qr_positive(P, dtype=np.float64):
     """Q factor of P = Q R with diag(R) > 0 (unique for full-rank P).
 
     The per-step QR orthogonalisation of the eigenbasis ([SMB-review] §3-2 (4),
     [SMB-summary] "SOAP Instability Diagnosis").  numpy's Householder QR is
     sign-fixed so that every diagonal entry of R is positive.
     """
-    Q, R = np.linalg.qr(_f64(P))
+    Q, R = np.linalg.qr(_w(P, dtype))
     s = np.sign(np.diag(R))
     s[s == 0] = 1.0
     return Q * s[None, :]
@@ -165,7 +173,7 @@ def sort_perm(keys):
     return np.argsort(-keys, kind="stable").astype(np.int32)
 
 
-def refresh_basis(F, Q, sort: bool):
+def refresh_basis(F, Q, sort: bool, dtype=np.float64):
     """One eigenbasis refresh of the factor F from the current basis Q.
 
     [SMB-review] §3-2 (4): refresh the basis from the updated factor, then QR.
@@ -173,12 +181,12 @@ def refresh_basis(F, Q, sort: bool):
     then one power step P = F Q and Q <- qr(P) (positive diagonal).
     Returns (Q_new, perm) where perm[i] is the old column placed at i.
     """
-    F, Q = _f64(F), _f64(Q)
+    F, Q = _w(F, dtype), _w(Q, dtype)
     k = Q.shape[1]
     perm = sort_perm(rayleigh_keys(F, Q)) if sort else np.arange(k, dtype=np.int32)
     Qp = Q[:, perm]
     P = F @ Qp
-    return qr_positive(P), perm
+    return qr_positive(P, dtype), perm
 
 
 def offdiag_ratio(D):
@@ -190,7 +198,7 @@ def offdiag_ratio(D):
 
 
 def refresh_decision(kind: int, t: int, k: int = 1, pf: int = 10, tol: float = 0.1,
-                     F=None, Q=None):
+                     F=None, Q=None, dtype=np.float64):
     """Whether a basis refresh happens at step t (1-based), and the check ratio.
 
     EVERY_K: (t-1) % k == 0 ([SMB-summary] "SOAP Instability Diagnosis": every
@@ -207,7 +215,7 @@ def refresh_decision(kind: int, t: int, k: int = 1, pf: int = 10, tol: float = 0
     if kind == REFRESH_ADAPTIVE:
         if (t - 1) % pf != 0:
             return False, -1.0
-        D = _f64(Q).T @ _f64(F) @ _f64(Q)
+        D = _w(Q, dtype).T @ _w(F, dtype) @ _w(Q, dtype)
         rho = offdiag_ratio(D)
         return rho > tol, rho
     raise ValueError(f"unknown refresh kind {kind}")
@@ -232,8 +240,8 @@ class SoapState:
         return SoapState(np.zeros((m, n)), np.zeros((m, n)), eps_init * np.eye(m),
                          eps_init * np.eye(n), np.eye(m), np.eye(n))
 
-    def copy(self) -> "SoapState":
-        return SoapState(*(np.array(x, dtype=np.float64, copy=True) for x in
+    def copy(self, dtype=np.float64) -> "SoapState":
+        return SoapState(*(np.array(x, dtype=dtype, copy=True) for x in
                            (self.M, self.V, self.L, self.R, self.QL, self.QR)))
 
 
@@ -252,7 +260,8 @@ class SoapResult:
 
 def soap_step(W, G, state: SoapState, *, t: int, beta1: float, beta2: float,
               eps: float, lr: float, wd: float = 0.0, refresh_kind: int = REFRESH_EVERY_K,
-              k: int = 1, pf: int = 10, tol: float = 0.1, sort: bool = True) -> SoapResult:
+              k: int = 1, pf: int = 10, tol: float = 0.1, sort: bool = True,
+              dtype=np.float64) -> SoapResult:
     """One two-sided SOAP step with the real-time eigenbasis refresh.
 
     Order ([SMB-review] §3-2 (4)): the current gradient enters the factors first,
@@ -267,23 +276,23 @@ def soap_step(W, G, state: SoapState, *, t: int, beta1: float, beta2: float,
       S7  V <- b2 V + (1-b2) Gh^2 ;  N = (Mh/(1-b1^t)) / (sqrt(V/(1-b2^t)) + eps)
       S8  U = QL N QR^T ;  W <- W(1 - lr wd) - lr U                   (eq. (1))
     """
-    W, G = _f64(W), _f64(G)
-    s = state.copy()
+    W, G = _w(W, dtype), _w(G, dtype)
+    s = state.copy(dtype)
     m, n = W.shape
     # S1
     s.L = beta2 * s.L + (1.0 - beta2) * (G @ G.T)
     s.R = beta2 * s.R + (1.0 - beta2) * (G.T @ G)
     # S2
-    refL, rhoL = refresh_decision(refresh_kind, t, k, pf, tol, s.L, s.QL)
-    refR, rhoR = refresh_decision(refresh_kind, t, k, pf, tol, s.R, s.QR)
+    refL, rhoL = refresh_decision(refresh_kind, t, k, pf, tol, s.L, s.QL, dtype)
+    refR, rhoR = refresh_decision(refresh_kind, t, k, pf, tol, s.R, s.QR, dtype)
     permL = np.arange(m, dtype=np.int32)
     permR = np.arange(n, dtype=np.int32)
     # S3 + S4 (V follows the permutation of its basis; no re-projection)
     if refL:
-        s.QL, permL = refresh_basis(s.L, s.QL, sort)
+        s.QL, permL = refresh_basis(s.L, s.QL, sort, dtype)
         s.V = s.V[permL, :]
     if refR:
-        s.QR, permR = refresh_basis(s.R, s.QR, sort)
+        s.QR, permR = refresh_basis(s.R, s.QR, sort, dtype)
         s.V = s.V[:, permR]
     # S5
     s.M = beta1 * s.M + (1.0 - beta1) * G
@@ -318,8 +327,8 @@ class FoamState:
         """R = eps_init * I, Q_R = I, M = r = c = 0 (initial state reading)."""
         return FoamState(np.zeros((m, n)), np.zeros(m), np.zeros(n), eps_init * np.eye(n), np.eye(n))
 
-    def copy(self) -> "FoamState":
-        return FoamState(*(np.array(x, dtype=np.float64, copy=True) for x in
+    def copy(self, dtype=np.float64) -> "FoamState":
+        return FoamState(*(np.array(x, dtype=dtype, copy=True) for x in
                            (self.M, self.r, self.c, self.R, self.QR)))
 
 
@@ -352,7 +361,7 @@ def foam_tau(R, r, c, t: int, beta2: float, raw_trace: bool = False) -> float:
 def foam_step(W, G, state: FoamState, *, t: int, beta1: float, beta2: float, eps: float,
               lr: float, wd: float = 0.0, refresh_kind: int = REFRESH_ADAPTIVE, k: int = 1,
               pf: int = 10, tol: float = 0.1, sort: bool = True,
-              raw_trace: bool = False) -> FoamResult:
+              raw_trace: bool = False, dtype=np.float64) -> FoamResult:
     """One FOAM step (input-only preconditioning, factored Adam moment).
 
     [FOAM-review] §1, §3:
@@ -364,17 +373,17 @@ def foam_step(W, G, state: FoamState, *, t: int, beta1: float, beta2: float, eps
           v^_ij = tau r^_i c^_j ;  N = (Mr/(1-b1^t)) / (sqrt(v^) + eps)
       F6  U = N Q_R^T ;  W <- W(1 - lr wd) - lr U
     """
-    W, G = _f64(W), _f64(G)
-    s = state.copy()
+    W, G = _w(W, dtype), _w(G, dtype)
+    s = state.copy(dtype)
     m, n = W.shape
     # F1
     s.R = beta2 * s.R + (1.0 - beta2) * (G.T @ G)
     # F2
-    ref, rho = refresh_decision(refresh_kind, t, k, pf, tol, s.R, s.QR)
+    ref, rho = refresh_decision(refresh_kind, t, k, pf, tol, s.R, s.QR, dtype)
     perm = np.arange(n, dtype=np.int32)
     # F3
     if ref:
-        s.QR, perm = refresh_basis(s.R, s.QR, sort)
+        s.QR, perm = refresh_basis(s.R, s.QR, sort, dtype)
         s.c = s.c[perm]
     # F4
     s.M = beta1 * s.M + (1.0 - beta1) * G
