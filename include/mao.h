@@ -105,7 +105,7 @@ typedef struct {
 
 /* Optional per-matrix diagnostics, written on the device (array of `count`). */
 typedef struct {
-  float update_rms;    /* ||W_new - W_old||_F / sqrt(m n) */
+  float update_rms;    /* ||W_new - W_old||_F / sqrt(m n) (Muon); -1 where not computed (SOAP, FOAM) */
   float offdiag_ratio; /* FOAM/SOAP adaptive check ratio of this step, -1 if none ran */
   int32_t refreshed;   /* bit 0: right basis refreshed, bit 1: left basis refreshed */
   int32_t nonfinite;   /* number of non-finite entries in W_new */
@@ -210,7 +210,9 @@ typedef struct {
  *   Gh = Q_L^T G Q_R ; Mh = Q_L^T M Q_R
  *   V <- b2 V + (1-b2) Gh^2 ; N = (Mh / (1-b1^t)) / (sqrt(V / (1-b2^t)) + eps)
  *   U = Q_L N Q_R^T ; W <- W (1 - lr wd) - lr U
- * Contractions use fp32-faithful tensor-core arithmetic (3xTF32).
+ * Contractions use fp32-faithful tensor-core arithmetic: every fp32 operand is
+ * held as three bf16 planes and the six significant cross products accumulate
+ * in fp32.
  */
 MAO_API mao_status mao_soap_workspace_size(const mao_soap_mat* mats, int32_t count, const mao_soap_params* p,
                                    size_t* bytes);
@@ -287,8 +289,16 @@ typedef enum {
   MAO_K_MUON_ROWSCALE = 8,
   MAO_K_MUON_UPDATE = 9,   /* weight update (HBM) */
   MAO_K_MUON_STATS = 10,
-  MAO_K_TF32_SPLIT = 11,
-  MAO_K_GEMM_TEST = 12
+  MAO_K_SPLIT3 = 11,         /* fp32 -> three bf16 planes (GEMM verification entry) */
+  MAO_K_GEMM_TEST = 12,
+  MAO_K_PC_ELEMENTWISE = 13, /* SOAP/FOAM momentum, splits, Adam, r/c/tau, N (HBM) */
+  MAO_K_PC_FACTOR = 14,      /* L / R EMA products (tensor cores, fp32-faithful SPLIT3) */
+  MAO_K_PC_CHECK = 15,       /* adaptive check D = Q^T F Q and its ratio */
+  MAO_K_PC_POWER = 16,       /* power step P = F Q */
+  MAO_K_PC_SORT = 17,        /* sort keys, argsort, gathers */
+  MAO_K_PC_QR = 18,          /* QR panels: projections, Gram, Cholesky, apply */
+  MAO_K_PC_ROTATE = 19,      /* rotations into the eigenbasis and back (before the update) */
+  MAO_K_PC_UPDATE = 20       /* last rotation fused with the weight update */
 } mao_kernel_id;
 
 /* What one recorded launch was: its kernel and its algorithmic work (useful

@@ -14,21 +14,22 @@
 extern "C" {
 #endif
 
-typedef enum { MAO_GEMM_BF16 = 0, MAO_GEMM_TF32X3 = 1 } mao_gemm_kind;
+typedef enum { MAO_GEMM_BF16 = 0, MAO_GEMM_SPLIT3 = 1 } mao_gemm_kind;
 
 /*
  * D[b] = A[b] * B[b]^T for b < batch, with fp32 accumulation and fp32 D.
  *   kind MAO_GEMM_BF16:   A, B bf16; one bf16 tensor-core product.
- *   kind MAO_GEMM_TF32X3: A, B fp32; each split into hi + lo tf32 parts and
- *                         D = Ahi Bhi + Ahi Blo + Alo Bhi (fp32-faithful).
+ *   kind MAO_GEMM_SPLIT3: A, B fp32; each split into three bf16 planes
+ *                         x = x0 + x1 + x2 and the six significant cross
+ *                         products accumulated in fp32 (fp32-faithful).
  * Layouts (row-major, contiguous batches):
  *   a_mn_major = 0: A is [batch][M][K]; 1: A is [batch][K][M]
  *   b_mn_major = 0: B is [batch][N][K]; 1: B is [batch][K][N]
  *   D is [batch][M][N].
- * The innermost extent of A and B must be a multiple of 8 (bf16) or 4 (fp32)
- * elements, N a multiple of 4.  workspace: >= mao_test_gemm_workspace_size()
- * bytes, 256-byte aligned (holds the device status word and, for TF32X3, the
- * split operands).
+ * The innermost extent of A and B must be a multiple of 8 elements, N a
+ * multiple of 4.  workspace: >= mao_test_gemm_workspace_size() bytes, 256-byte
+ * aligned (holds the device status word and, for SPLIT3, the split operands and
+ * the problem descriptors).
  */
 MAO_API mao_status mao_test_gemm_workspace_size(int32_t kind, int32_t batch, int32_t M, int32_t N, int32_t K,
                                         size_t* bytes);

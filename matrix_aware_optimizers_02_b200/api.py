@@ -127,10 +127,10 @@ def gemm(A: torch.Tensor, B: torch.Tensor, *, kind: str = "bf16", a_mn_major: bo
 
     A is (batch, M, K) (or (batch, K, M) when a_mn_major); B is (batch, N, K)
     (or (batch, K, N) when b_mn_major).  kind "bf16" (bf16 operands) or
-    "tf32x3" (fp32 operands, split hi/lo).  Returns fp32 (batch, M, N).
+    "split3" (fp32 operands held as three bf16 planes, fp32-faithful).  Returns fp32 (batch, M, N).
     """
     lib = L.load()
-    k = {"bf16": 0, "tf32x3": 1}[kind]
+    k = {"bf16": 0, "split3": 1}[kind]
     batch = A.shape[0]
     M = A.shape[2] if a_mn_major else A.shape[1]
     K = A.shape[1] if a_mn_major else A.shape[2]
@@ -145,3 +145,118 @@ def gemm(A: torch.Tensor, B: torch.Tensor, *, kind: str = "bf16", a_mn_major: bo
     st = lib.mao_workspace_status(ws.data_ptr(), _stream_handle(stream), ctypes.byref(where))
     L.check(st, f"gemm device status (site {where.value})")
     return D
+
+
+def _refresh(kind: str, k: int, pf: int, tol: float, sort: bool) -> "L.Refresh":
+    kinds = {"every_k": L.REFRESH_EVERY_K, "adaptive": L.REFRESH_ADAPTIVE, "never": L.REFRESH_NEVER}
+    if kind not in kinds:
+        raise ValueError(f"refresh must be one of {sorted(kinds)}")
+    return L.Refresh(kinds[kind], int(k), int(pf), float(tol), int(bool(sort)))
+
+
+class _PrecondBatch:
+    """Shared plumbing of SoapBatch / FoamBatch."""
+
+    def _finish(self, size_fn, n, device, workspace, with_stats):
+        nbytes = ctypes.c_size_t(0)
+        L.check(size_fn(self.arr, n, ctypes.byref(self.params), ctypes.byref(nbytes)), size_fn.__name__)
+        self.ws_bytes = nbytes.value
+        if workspace is None:
+            workspace = _alloc_workspace(self.ws_bytes, device)
+        elif workspace.numel() * workspace.element_size() < self.ws_bytes:
+            raise ValueError("workspace too small")
+        self.workspace = workspace
+        self.stats = torch.zeros((max(n, 1), 4), dtype=torch.float32, device=device) if with_stats else None
+
+    def device_status(self, stream: Optional[torch.cuda.Stream] = None) -> int:
+        where = ctypes.c_int32(0)
+        return self.lib.mao_workspace_status(self.workspace.data_ptr(), _stream_handle(stream), ctypes.byref(where))
+
+    def stats_dict(self):
+        if self.stats is None:
+            return None
+        s = self.stats[: self.count].cpu()
+        return {"offdiag_ratio": s[:, 1].tolist(), "refreshed": s[:, 2].contiguous().view(torch.int32).tolist()}
+
+
+class SoapBatch(_PrecondBatch):
+    """One two-sided SOAP step over a fixed list of matrices.
+
+    Each entry is a dict with CUDA tensors W (m, n) fp32, G (m, n) fp32/bf16 and
+    the state M, V (m, n), L, QL (m, m), R, QR (n, n) fp32; optional int32
+    perm_L (m) / perm_R (n) receive the basis permutations of the step.
+    Call with the 1-based step number t.
+    """
+
+    def __init__(self, mats, *, beta1: float, beta2: float, eps: float, lr: float, wd: float = 0.0,
+                 refresh: str = "every_k", k: int = 1, pf: int = 10, tol: float = 0.1, sort: bool = True,
+                 workspace: Optional[torch.Tensor] = None, with_stats: bool = False, t: int = 1):
+        self.lib = L.load()
+        self.mats = list(mats)
+        n = len(self.mats)
+        self.arr = (L.SoapMat * max(n, 1))()
+        dev = None
+        for i, d in enumerate(self.mats):
+            W = d["W"]
+            m_, n_ = W.shape
+            for name, shape in (("W", (m_, n_)), ("M", (m_, n_)), ("V", (m_, n_)), ("L", (m_, m_)),
+                                ("QL", (m_, m_)), ("R", (n_, n_)), ("QR", (n_, n_))):
+                _check_mat(name, d[name], shape)
+            _check_mat("G", d["G"], (m_, n_), None)
+            pl, pr = d.get("perm_L"), d.get("perm_R")
+            self.arr[i] = L.SoapMat(m_, n_, W.data_ptr(), d["G"].data_ptr(), _g_dtype(d["G"]), d["M"].data_ptr(),
+                                    d["V"].data_ptr(), d["L"].data_ptr(), d["R"].data_ptr(), d["QL"].data_ptr(),
+                                    d["QR"].data_ptr(), pl.data_ptr() if pl is not None else None,
+                                    pr.data_ptr() if pr is not None else None)
+            dev = W.device
+        self.count = n
+        self.params = L.SoapParams(beta1, beta2, eps, lr, wd, int(t), _refresh(refresh, k, pf, tol, sort))
+        self._finish(self.lib.mao_soap_workspace_size, n, dev if dev is not None else "cuda", workspace, with_stats)
+
+    def __call__(self, t: int, stream: Optional[torch.cuda.Stream] = None) -> None:
+        self.params.t = int(t)
+        st = self.lib.mao_soap_step(self.arr, self.count, ctypes.byref(self.params), self.workspace.data_ptr(),
+                                    self.ws_bytes, self.stats.data_ptr() if self.stats is not None else None,
+                                    _stream_handle(stream))
+        L.check(st, "mao_soap_step")
+
+
+class FoamBatch(_PrecondBatch):
+    """One FOAM step over a fixed list of matrices.
+
+    Each entry is a dict with W (m, n), G (m, n), M (m, n), r (m), c (n), R and
+    QR (n, n); optional int32 perm_R (n).  Call with the 1-based step number t.
+    """
+
+    def __init__(self, mats, *, beta1: float, beta2: float, eps: float, lr: float, wd: float = 0.0,
+                 refresh: str = "adaptive", k: int = 1, pf: int = 10, tol: float = 0.1, sort: bool = True,
+                 tau_raw_trace: bool = False, workspace: Optional[torch.Tensor] = None, with_stats: bool = False,
+                 t: int = 1):
+        self.lib = L.load()
+        self.mats = list(mats)
+        n = len(self.mats)
+        self.arr = (L.FoamMat * max(n, 1))()
+        dev = None
+        for i, d in enumerate(self.mats):
+            W = d["W"]
+            m_, n_ = W.shape
+            for name, shape in (("W", (m_, n_)), ("M", (m_, n_)), ("r", (m_,)), ("c", (n_,)), ("R", (n_, n_)),
+                                ("QR", (n_, n_))):
+                _check_mat(name, d[name], shape)
+            _check_mat("G", d["G"], (m_, n_), None)
+            pr = d.get("perm_R")
+            self.arr[i] = L.FoamMat(m_, n_, W.data_ptr(), d["G"].data_ptr(), _g_dtype(d["G"]), d["M"].data_ptr(),
+                                    d["r"].data_ptr(), d["c"].data_ptr(), d["R"].data_ptr(), d["QR"].data_ptr(),
+                                    pr.data_ptr() if pr is not None else None)
+            dev = W.device
+        self.count = n
+        self.params = L.FoamParams(beta1, beta2, eps, lr, wd, int(t), _refresh(refresh, k, pf, tol, sort),
+                                   int(bool(tau_raw_trace)))
+        self._finish(self.lib.mao_foam_workspace_size, n, dev if dev is not None else "cuda", workspace, with_stats)
+
+    def __call__(self, t: int, stream: Optional[torch.cuda.Stream] = None) -> None:
+        self.params.t = int(t)
+        st = self.lib.mao_foam_step(self.arr, self.count, ctypes.byref(self.params), self.workspace.data_ptr(),
+                                    self.ws_bytes, self.stats.data_ptr() if self.stats is not None else None,
+                                    _stream_handle(stream))
+        L.check(st, "mao_foam_step")

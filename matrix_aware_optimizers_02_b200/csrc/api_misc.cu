@@ -55,29 +55,37 @@ extern "C" mao_status mao_workspace_status(const void* workspace, mao_stream_t s
 
 // ------------------------------------------------------------------ GEMM check
 namespace {
-mao_status gemm_ws(int32_t kind, int32_t batch, int32_t M, int32_t N, int32_t K, Carver& cv, size_t* a_hi,
-                   size_t* a_lo, size_t* b_hi, size_t* b_lo) {
+
+struct TestLayout {
+  size_t planes[2] = {0, 0};  // SPLIT3: planes of A and B
+  size_t arena = 0, arena_bytes = 0;
+  size_t total = 0;
+};
+
+mao_status gemm_layout(int32_t kind, int32_t batch, int32_t M, int32_t N, int32_t K, TestLayout& T) {
   if (batch < 1 || M < 1 || N < 1 || K < 1) return MAO_ERR_SHAPE;
-  if (kind != MAO_GEMM_BF16 && kind != MAO_GEMM_TF32X3) return MAO_ERR_INVALID_ARG;
+  if (kind != MAO_GEMM_BF16 && kind != MAO_GEMM_SPLIT3) return MAO_ERR_INVALID_ARG;
+  Carver cv;
   cv.take(kStatusBytes);
-  if (kind == MAO_GEMM_TF32X3) {
-    const size_t an = (size_t)batch * M * K, bn = (size_t)batch * N * K;
-    *a_hi = cv.take(4 * an);
-    *a_lo = cv.take(4 * an);
-    *b_hi = cv.take(4 * bn);
-    *b_lo = cv.take(4 * bn);
+  if (kind == MAO_GEMM_SPLIT3) {
+    T.planes[0] = cv.take(3 * 2 * (size_t)batch * M * K);
+    T.planes[1] = cv.take(3 * 2 * (size_t)batch * N * K);
+    // per batch element: one problem and six descriptors
+    T.arena_bytes = align_up(sizeof(GemmProblem) * batch, 64) + sizeof(CUtensorMap) * 6 * batch + 256;
+    T.arena = cv.take(T.arena_bytes);
   }
+  T.total = cv.total();
   return MAO_OK;
 }
+
 }  // namespace
 
 extern "C" mao_status mao_test_gemm_workspace_size(int32_t kind, int32_t batch, int32_t M, int32_t N, int32_t K,
                                                    size_t* bytes) {
   if (bytes == nullptr) return MAO_ERR_INVALID_ARG;
-  Carver cv;
-  size_t a, b, c, d;
-  MAO_TRY(gemm_ws(kind, batch, M, N, K, cv, &a, &b, &c, &d));
-  *bytes = cv.total();
+  TestLayout T;
+  MAO_TRY(gemm_layout(kind, batch, M, N, K, T));
+  *bytes = T.total;
   return MAO_OK;
 }
 
@@ -86,66 +94,72 @@ extern "C" mao_status mao_test_gemm(int32_t kind, int32_t a_mn_major, int32_t b_
                                     void* workspace, size_t ws_bytes, mao_stream_t stream_) {
   if (A == nullptr || B == nullptr || D == nullptr || workspace == nullptr) return MAO_ERR_INVALID_ARG;
   if ((a_mn_major != 0 && a_mn_major != 1) || (b_mn_major != 0 && b_mn_major != 1)) return MAO_ERR_INVALID_ARG;
-  Carver cv;
-  size_t oah = 0, oal = 0, obh = 0, obl = 0;
-  MAO_TRY(gemm_ws(kind, batch, M, N, K, cv, &oah, &oal, &obh, &obl));
-  if (ws_bytes < cv.total()) return MAO_ERR_WORKSPACE;
+  TestLayout T;
+  MAO_TRY(gemm_layout(kind, batch, M, N, K, T));
+  if (ws_bytes < T.total) return MAO_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MAO_ERR_ALIGN;
   if (!aligned16(A) || !aligned16(B) || !aligned16(D)) return MAO_ERR_ALIGN;
-  const int vec = (kind == MAO_GEMM_BF16) ? 8 : 4;
   const int a_inner = a_mn_major ? M : K, b_inner = b_mn_major ? N : K;
-  if (a_inner % vec || b_inner % vec || N % 4) return MAO_ERR_SHAPE;
+  if (a_inner % 8 || b_inner % 8 || N % 4) return MAO_ERR_SHAPE;
   DeviceInfo* dev = nullptr;
   MAO_TRY(device_info(&dev));
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DevStatus* status = reinterpret_cast<DevStatus*>(ws);
   MAO_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(DevStatus), stream));
+  const int a_rows = a_mn_major ? K : M, b_rows = b_mn_major ? K : N;
 
-  const int okind = (kind == MAO_GEMM_BF16) ? OP_BF16 : OP_TF32X3;
-  const void* a_src = A;
-  const void* b_src = B;
+  if (kind == MAO_GEMM_BF16) {
+    auto view = [&](const void* base, int rows, int inner) {
+      OperandView v;
+      v.base = base;
+      v.batch = (uint64_t)batch;
+      v.inner = (uint64_t)inner;
+      v.rows = (uint64_t)rows;
+      v.ld = v.inner;
+      v.bstride = (uint64_t)rows * inner;
+      return v;
+    };
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.nclasses = 1;
+    p.alpha = 1.0f;
+    p.status = status;
+    MAO_TRY(encode_operand(&p.mapA[0], OP_BF16, a_mn_major, 128, view(A, a_rows, a_inner)));
+    MAO_TRY(encode_operand(&p.mapB[0], OP_BF16, b_mn_major, 256, view(B, b_rows, b_inner)));
+    p.cls[0] = GemmClass{M, N, K, batch, 0, 0, 0, D, (long long)M * N, N, nullptr, 0, 0, nullptr, 0, 0, nullptr};
+    finalize_classes(p);
+    return launch_gemm(OP_BF16, a_mn_major, b_mn_major, EPI_STORE_F32, p, stream, MAO_K_GEMM_TEST);
+  }
+
+  // SPLIT3: three bf16 planes of each operand, then one table-mode problem per batch element
   const size_t an = (size_t)batch * M * K, bn = (size_t)batch * N * K;
-  GemmLoMaps lo;
-  std::memset(&lo, 0, sizeof(lo));
-  if (okind == OP_TF32X3) {
-    MAO_TRY(launch_tf32_split(static_cast<const float*>(A), reinterpret_cast<float*>(ws + oah),
-                              reinterpret_cast<float*>(ws + oal), an, stream));
-    MAO_TRY(launch_tf32_split(static_cast<const float*>(B), reinterpret_cast<float*>(ws + obh),
-                              reinterpret_cast<float*>(ws + obl), bn, stream));
-    a_src = ws + oah;
-    b_src = ws + obh;
+  __nv_bfloat16* ap = reinterpret_cast<__nv_bfloat16*>(ws + T.planes[0]);
+  __nv_bfloat16* bp = reinterpret_cast<__nv_bfloat16*>(ws + T.planes[1]);
+  MAO_TRY(launch_split3(static_cast<const float*>(A), ap, ap + an, ap + 2 * an, an, stream));
+  MAO_TRY(launch_split3(static_cast<const float*>(B), bp, bp + bn, bp + 2 * bn, bn, stream));
+  Arena arena;
+  arena.dev = ws + T.arena;
+  MapSet maps;
+  TableLaunch L;
+  L.a_mn = a_mn_major;
+  L.b_mn = b_mn_major;
+  L.kernel_id = MAO_K_GEMM_TEST;
+  for (int b = 0; b < batch; ++b) {
+    const size_t ao = (size_t)b * M * K, bo = (size_t)b * N * K;
+    const Split3 As{{ap + ao, ap + an + ao, ap + 2 * an + ao}, a_rows, a_inner, a_inner};
+    const Split3 Bs{{bp + bo, bp + bn + bo, bp + 2 * bn + bo}, b_rows, b_inner, b_inner};
+    MAO_TRY(table_add(L, maps, As, Bs, M, N, K, 0, 0, D + (size_t)b * M * N, nullptr, N, nullptr, 0, 1.f, 0.f,
+                      nullptr));
   }
-  auto view = [&](const void* base, int mn, int mn_major) {
-    OperandView v;
-    v.base = base;
-    v.batch = (uint64_t)batch;
-    if (mn_major) {
-      v.inner = (uint64_t)mn;
-      v.rows = (uint64_t)K;
-    } else {
-      v.inner = (uint64_t)K;
-      v.rows = (uint64_t)mn;
-    }
-    v.ld = v.inner;
-    v.bstride = (uint64_t)mn * K;
-    return v;
-  };
-  GemmParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.nclasses = 1;
-  p.alpha = 1.0f;
-  p.status = reinterpret_cast<DevStatus*>(ws);
-  MAO_TRY(encode_operand(&p.mapA[0], okind, a_mn_major, 128, view(a_src, M, a_mn_major)));
-  MAO_TRY(encode_operand(&p.mapB[0], okind, b_mn_major, 256, view(b_src, N, b_mn_major)));
-  if (okind == OP_TF32X3) {
-    MAO_TRY(encode_operand(&lo.mapAlo[0], okind, a_mn_major, 128, view(ws + oal, M, a_mn_major)));
-    MAO_TRY(encode_operand(&lo.mapBlo[0], okind, b_mn_major, 256, view(ws + obl, N, b_mn_major)));
-  }
-  p.cls[0] = GemmClass{M, N, K, batch, 0, 0, 0, D, (long long)M * N, N, nullptr, 0, 0, nullptr, 0, 0, nullptr};
-  finalize_classes(p);
+  MAO_TRY(maps.encode_all());
+  const size_t maps_off = arena.take(sizeof(CUtensorMap) * maps.maps.size(), 64);
+  std::memcpy(arena.host.data() + maps_off, maps.maps.data(), sizeof(CUtensorMap) * maps.maps.size());
+  const StagedLaunch S = table_stage(arena, L, maps_off);
+  if (arena.host.size() > T.arena_bytes) return MAO_ERR_WORKSPACE;
+  MAO_CUDA_TRY(cudaMemcpyAsync(arena.dev, arena.host.data(), arena.host.size(), cudaMemcpyHostToDevice, stream));
   (void)dev;
-  return launch_gemm(okind, a_mn_major, b_mn_major, EPI_STORE_F32, p, okind == OP_TF32X3 ? &lo : nullptr, stream,
-                     MAO_K_GEMM_TEST);
+  return table_launch(arena, S, status, stream);
 }
 
 namespace mao {

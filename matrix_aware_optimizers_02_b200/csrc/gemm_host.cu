@@ -1,6 +1,6 @@
 // Host side of the grouped tcgen05 GEMM: device facts, TMA descriptor
-// encoding, tile bookkeeping and the launch dispatcher; plus the fp32 -> hi/lo
-// tf32 split used by the fp32-faithful (3xTF32) products.
+// encoding, tile bookkeeping and the launch dispatchers; plus the fp32 ->
+// three bf16 planes split used by the fp32-faithful (SPLIT3) products.
 #include <cudaTypedefs.h>
 
 #include "host_common.h"
@@ -64,15 +64,10 @@ mao_status encode_3d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const 
 }
 
 mao_status encode_operand(CUtensorMap* map, int kind, int mn_major, int R, const OperandView& v) {
-  const int esize = (kind == OP_BF16) ? 2 : 4;
-  const CUtensorMapDataType dt =
-      (kind == OP_BF16) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  const uint32_t row_elems = 128 / esize;  // elements in one 128-byte swizzle row
-  if (!mn_major)
-    return encode_3d(map, dt, esize, v.base, v.inner, v.rows, v.batch, v.ld, v.bstride, row_elems, R, false);
-  // MN-major 32-bit operands need the 32-byte-atom variant of the 128-byte swizzle
-  return encode_3d(map, dt, esize, v.base, v.inner, v.rows, v.batch, v.ld, v.bstride, row_elems, row_elems,
-                   esize == 4);
+  (void)kind;  // every operand plane is bf16
+  const uint32_t row_elems = 64;  // bf16 elements in one 128-byte swizzle row
+  return encode_3d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v.base, v.inner, v.rows, v.batch, v.ld, v.bstride,
+                   row_elems, mn_major ? row_elems : (uint32_t)R, false);
 }
 
 void finalize_classes(GemmParams& p) {
@@ -91,7 +86,7 @@ void finalize_classes(GemmParams& p) {
 namespace {
 
 template <int KIND, int A_MN, int B_MN, int EPI>
-mao_status launch_one(const GemmParams& p, const GemmLoMaps* lo, cudaStream_t stream, int kernel_id) {
+mao_status launch_one(const GemmParams& p, cudaStream_t stream, int kernel_id) {
   using Cfg = GemmCfg<KIND, A_MN, B_MN>;
   DeviceInfo* d = nullptr;
   MAO_TRY(device_info(&d));
@@ -105,7 +100,6 @@ mao_status launch_one(const GemmParams& p, const GemmLoMaps* lo, cudaStream_t st
     }
   }
   if (p.total_tiles <= 0) return MAO_OK;
-  static const GemmLoMaps kEmptyLo = {};
   const int grid = p.total_tiles < d->sm_count ? p.total_tiles : d->sm_count;
   double flops = 0.0, bytes = 0.0;
   const double es = Cfg::ESIZE, ob = (EPI == EPI_STORE_F32) ? 4.0 : 2.0;
@@ -117,80 +111,191 @@ mao_status launch_one(const GemmParams& p, const GemmLoMaps* lo, cudaStream_t st
                         ((EPI == EPI_POLY || EPI == EPI_AXPY_T) ? 2.0 * C.M * C.N : 0.0));
   }
   LaunchScope ls(stream, kernel_id, flops, bytes);
-  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(p, lo ? *lo : kEmptyLo);
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? MAO_OK : MAO_ERR_CUDA;
 }
 
 template <int KIND, int A_MN, int B_MN>
-mao_status launch_epi(int epi, const GemmParams& p, const GemmLoMaps* lo, cudaStream_t s, int k) {
+mao_status launch_epi(int epi, const GemmParams& p, cudaStream_t s, int k) {
   switch (epi) {
-    case EPI_STORE_F32: return launch_one<KIND, A_MN, B_MN, EPI_STORE_F32>(p, lo, s, k);
-    case EPI_GRAM: return launch_one<KIND, A_MN, B_MN, EPI_GRAM>(p, lo, s, k);
-    case EPI_POLY: return launch_one<KIND, A_MN, B_MN, EPI_POLY>(p, lo, s, k);
-    case EPI_AXPY_T: return launch_one<KIND, A_MN, B_MN, EPI_AXPY_T>(p, lo, s, k);
+    case EPI_STORE_F32: return launch_one<KIND, A_MN, B_MN, EPI_STORE_F32>(p, s, k);
+    case EPI_GRAM: return launch_one<KIND, A_MN, B_MN, EPI_GRAM>(p, s, k);
+    case EPI_POLY: return launch_one<KIND, A_MN, B_MN, EPI_POLY>(p, s, k);
+    case EPI_AXPY_T: return launch_one<KIND, A_MN, B_MN, EPI_AXPY_T>(p, s, k);
     default: return MAO_ERR_INVALID_ARG;
   }
 }
 
 }  // namespace
 
-mao_status launch_gemm(int kind, int a_mn, int b_mn, int epi, const GemmParams& p, const GemmLoMaps* lo,
-                       cudaStream_t stream, int k) {
-  if (kind == OP_BF16) {
-    if (!a_mn && !b_mn) return launch_epi<OP_BF16, 0, 0>(epi, p, lo, stream, k);
-    if (!a_mn && b_mn) return launch_epi<OP_BF16, 0, 1>(epi, p, lo, stream, k);
-    if (epi != EPI_STORE_F32) return MAO_ERR_UNSUPPORTED;
-    if (a_mn && !b_mn) return launch_one<OP_BF16, 1, 0, EPI_STORE_F32>(p, lo, stream, k);
-    return launch_one<OP_BF16, 1, 1, EPI_STORE_F32>(p, lo, stream, k);
-  }
-  if (kind == OP_TF32X3) {
-    if (epi != EPI_STORE_F32 || lo == nullptr) return MAO_ERR_UNSUPPORTED;
-    if (!a_mn && !b_mn) return launch_one<OP_TF32X3, 0, 0, EPI_STORE_F32>(p, lo, stream, k);
-    if (!a_mn && b_mn) return launch_one<OP_TF32X3, 0, 1, EPI_STORE_F32>(p, lo, stream, k);
-    if (a_mn && !b_mn) return launch_one<OP_TF32X3, 1, 0, EPI_STORE_F32>(p, lo, stream, k);
-    return launch_one<OP_TF32X3, 1, 1, EPI_STORE_F32>(p, lo, stream, k);
-  }
-  return MAO_ERR_INVALID_ARG;
+mao_status launch_gemm(int kind, int a_mn, int b_mn, int epi, const GemmParams& p, cudaStream_t stream, int k) {
+  if (kind != OP_BF16) return MAO_ERR_UNSUPPORTED;
+  if (!a_mn && !b_mn) return launch_epi<OP_BF16, 0, 0>(epi, p, stream, k);
+  if (!a_mn && b_mn) return launch_epi<OP_BF16, 0, 1>(epi, p, stream, k);
+  if (epi != EPI_STORE_F32) return MAO_ERR_UNSUPPORTED;
+  if (a_mn && !b_mn) return launch_one<OP_BF16, 1, 0, EPI_STORE_F32>(p, stream, k);
+  return launch_one<OP_BF16, 1, 1, EPI_STORE_F32>(p, stream, k);
 }
 
-// ------------------------------------------------------------------ tf32 split
+// ------------------------------------------------------------------ three-plane split
 namespace {
 
-// x = hi + lo with hi = tf32(x) and lo = tf32(x - hi): both exactly representable
-// in tf32, so the tensor core sees them without further rounding.
-__global__ void tf32_split_kernel(const float* __restrict__ src, float* __restrict__ hi, float* __restrict__ lo,
-                                  size_t n) {
-  size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
-  const size_t stride = (size_t)gridDim.x * blockDim.x * 4;
+// x = p0 + p1 + p2 with each plane the bf16 rounding of what the previous planes
+// left over; the three planes keep 24 significant bits of x.
+__global__ void split3_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ p0,
+                              __nv_bfloat16* __restrict__ p1, __nv_bfloat16* __restrict__ p2, size_t n) {
+  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (; i < n; i += stride) {
-    if (i + 4 <= n) {
-      float4 x = *reinterpret_cast<const float4*>(src + i);
-      float4 h = make_float4(tf32_rna(x.x), tf32_rna(x.y), tf32_rna(x.z), tf32_rna(x.w));
-      float4 l = make_float4(tf32_rna(x.x - h.x), tf32_rna(x.y - h.y), tf32_rna(x.z - h.z), tf32_rna(x.w - h.w));
-      *reinterpret_cast<float4*>(hi + i) = h;
-      *reinterpret_cast<float4*>(lo + i) = l;
-    } else {
-      for (size_t j = i; j < n; ++j) {
-        float h = tf32_rna(src[j]);
-        hi[j] = h;
-        lo[j] = tf32_rna(src[j] - h);
-      }
-    }
+    float r = src[i];
+    const __nv_bfloat16 a = __float2bfloat16_rn(r);
+    r -= __bfloat162float(a);
+    const __nv_bfloat16 b = __float2bfloat16_rn(r);
+    r -= __bfloat162float(b);
+    p0[i] = a;
+    p1[i] = b;
+    p2[i] = __float2bfloat16_rn(r);
   }
 }
 
 }  // namespace
 
-mao_status launch_tf32_split(const float* src, float* hi, float* lo, size_t n, cudaStream_t stream) {
+mao_status launch_split3(const float* src, __nv_bfloat16* p0, __nv_bfloat16* p1, __nv_bfloat16* p2, size_t n,
+                         cudaStream_t stream) {
   if (n == 0) return MAO_OK;
   DeviceInfo* d = nullptr;
   MAO_TRY(device_info(&d));
-  size_t blocks = (n / 4 + 255) / 256 + 1;
+  size_t blocks = (n + 255) / 256;
   const size_t cap = (size_t)d->sm_count * 8;
   if (blocks > cap) blocks = cap;
-  LaunchScope ls(stream, MAO_K_TF32_SPLIT, 0.0, 12.0 * (double)n);
-  tf32_split_kernel<<<(unsigned)blocks, 256, 0, stream>>>(src, hi, lo, n);
+  LaunchScope ls(stream, MAO_K_SPLIT3, 0.0, 10.0 * (double)n);
+  split3_kernel<<<(unsigned)blocks, 256, 0, stream>>>(src, p0, p1, p2, n);
   return cudaGetLastError() == cudaSuccess ? MAO_OK : MAO_ERR_CUDA;
+}
+
+}  // namespace mao
+
+// ------------------------------------------------------------------ table mode
+namespace mao {
+
+int MapSet::get(const void* p, int inner, int rows, int ld, int box_rows, int mn) {
+  MapKey k{p, inner, rows, ld, box_rows, mn};
+  auto it = index.find(k);
+  if (it != index.end()) return it->second;
+  keys.push_back(k);
+  const int i = (int)keys.size() - 1;
+  index.emplace(k, i);
+  return i;
+}
+
+mao_status MapSet::encode_all() {
+  maps.resize(keys.size());
+  for (size_t i = 0; i < keys.size(); ++i) {
+    const MapKey& k = keys[i];
+    MAO_TRY(encode_3d(&maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k.p, (uint64_t)k.inner, (uint64_t)k.rows, 1,
+                      (uint64_t)k.ld, (uint64_t)k.ld * k.rows, 64, (uint32_t)k.box_rows, false));
+  }
+  return MAO_OK;
+}
+
+mao_status table_add(TableLaunch& L, MapSet& maps, const Split3& A, const Split3& B, int M, int N, int K,
+                     int m_off, int n_off, float* out, const Split3* outp, int ld_out, const float* aux,
+                     int ld_aux, float alpha, float beta, const int* flag) {
+  if (M <= 0 || N <= 0 || K <= 0) return MAO_OK;
+  if ((L.a_mn && (m_off & 7)) || (L.b_mn && (n_off & 7))) return MAO_ERR_INVALID_ARG;
+  if ((A.ld & 7) || (B.ld & 7)) return MAO_ERR_SHAPE;
+  // operand views: inner extent = the stored matrix's columns, rows = its rows
+  const int abox = L.a_mn ? 64 : 128, bbox = L.b_mn ? 64 : 128;
+  int idx[6];
+  for (int q = 0; q < 3; ++q) {
+    idx[q] = maps.get(A.p[q], A.cols, A.rows, A.ld, abox, L.a_mn);
+    idx[3 + q] = maps.get(B.p[q], B.cols, B.rows, B.ld, bbox, L.b_mn);
+  }
+  GemmProblem P;
+  std::memset(&P, 0, sizeof(P));
+  P.out = out;
+  if (outp) {
+    if (outp->ld & 7) return MAO_ERR_SHAPE;
+    for (int q = 0; q < 3; ++q) P.out_p[q] = const_cast<__nv_bfloat16*>(outp->p[q]);
+    P.ld_outp = outp->ld;
+  }
+  P.aux = aux;
+  P.flag = flag;
+  P.M = M;
+  P.N = N;
+  P.K = K;
+  P.m_off = m_off;
+  P.n_off = n_off;
+  P.ld_out = ld_out;
+  P.ld_aux = ld_aux;
+  P.tiles_n = (N + 127) / 128;
+  P.alpha = alpha;
+  P.beta = beta;
+  L.probs.push_back(P);
+  L.map_idx.insert(L.map_idx.end(), idx, idx + 6);
+  return MAO_OK;
+}
+
+StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off) {
+  StagedLaunch S;
+  S.nprob = (int)L.probs.size();
+  S.a_mn = L.a_mn;
+  S.b_mn = L.b_mn;
+  S.kernel_id = L.kernel_id;
+  if (S.nprob == 0) return S;
+  S.probs_off = A.take(sizeof(GemmProblem) * S.nprob, 64);
+  GemmProblem* hp = A.hptr<GemmProblem>(S.probs_off);
+  const CUtensorMap* mbase = A.dptr<const CUtensorMap>(maps_off);
+  int t = 0;
+  for (int i = 0; i < S.nprob; ++i) {
+    GemmProblem P = L.probs[i];
+    for (int q = 0; q < 3; ++q) {
+      P.mapA[q] = mbase ? mbase + L.map_idx[6 * i + q] : nullptr;
+      P.mapB[q] = mbase ? mbase + L.map_idx[6 * i + 3 + q] : nullptr;
+    }
+    P.tile_begin = t;
+    t += ((P.M + 127) / 128) * P.tiles_n;
+    S.flops += 2.0 * P.M * (double)P.N * P.K;
+    hp[i] = P;
+  }
+  S.total_tiles = t;
+  return S;
+}
+
+namespace {
+template <int A_MN, int B_MN>
+mao_status launch_table_one(const GemmTableParams& p, cudaStream_t stream, int kernel_id, double flops) {
+  using Cfg = GemmCfg<OP_SPLIT3, A_MN, B_MN>;
+  DeviceInfo* d = nullptr;
+  MAO_TRY(device_info(&d));
+  auto kern = gemm_tc_table_kernel<OP_SPLIT3, A_MN, B_MN>;
+  const int slot = 40 + A_MN * 2 + B_MN;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!d->gemm_attr_set[slot]) {
+      MAO_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
+      d->gemm_attr_set[slot] = true;
+    }
+  }
+  if (p.total_tiles <= 0) return MAO_OK;
+  const int grid = p.total_tiles < d->sm_count ? p.total_tiles : d->sm_count;
+  LaunchScope ls(stream, kernel_id, flops, 0.0);
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? MAO_OK : MAO_ERR_CUDA;
+}
+}  // namespace
+
+mao_status table_launch(const Arena& A, const StagedLaunch& S, DevStatus* status, cudaStream_t stream) {
+  if (S.nprob == 0) return MAO_OK;
+  GemmTableParams p;
+  p.probs = A.dptr<const GemmProblem>(S.probs_off);
+  p.nprob = S.nprob;
+  p.total_tiles = S.total_tiles;
+  p.status = status;
+  if (!S.a_mn && !S.b_mn) return launch_table_one<0, 0>(p, stream, S.kernel_id, S.flops);
+  if (!S.a_mn && S.b_mn) return launch_table_one<0, 1>(p, stream, S.kernel_id, S.flops);
+  if (S.a_mn && !S.b_mn) return launch_table_one<1, 0>(p, stream, S.kernel_id, S.flops);
+  return launch_table_one<1, 1>(p, stream, S.kernel_id, S.flops);
 }
 
 }  // namespace mao

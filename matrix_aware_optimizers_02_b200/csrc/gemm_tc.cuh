@@ -1,25 +1,40 @@
 // Grouped, persistent tcgen05 GEMM for sm_100a.
 //
-// D[b] = A[b] * B[b]^T over many problems at once.  Problems are grouped into
-// "classes" of identical (M, N, K); a class's operands are 3-D tensors
-// [count][rows][cols] reached through one TMA descriptor each, so a batch of
-// hundreds of same-shape matrices costs two descriptors.  One CTA per SM walks
-// the linear tile space (class, matrix, tile_m, tile_n) with a static stride.
+// D = A * B^T over many problems at once, one CTA per SM walking a linear tile
+// space with a static stride.  Two ways of describing the problems:
+//
+//   class mode  (GemmParams)  problems are grouped into "classes" of identical
+//               (M, N, K); a class's operands are 3-D tensors [count][rows][cols]
+//               reached through one TMA descriptor each (kernel parameters), so a
+//               batch of hundreds of same-shape matrices costs two descriptors.
+//               bf16 epilogues for Newton-Schulz (EPI_GRAM / EPI_POLY / EPI_AXPY_T)
+//               and an fp32 store (EPI_STORE_F32).
+//   table mode  (GemmTableParams) one entry per problem in a device array, each
+//               with its own descriptors in global memory (operands are separate
+//               buffers), SPLIT3 operands and an fp32 epilogue
+//                   out = alpha * acc + beta * aux          (aux optional, may alias out)
+//               that can also emit the three bf16 planes of `out` for a following
+//               fp32-faithful product.  A problem can be gated by a device flag
+//               (skipped when the flag is 0) for data-dependent work.
 //
 // Warp roles (192 threads):
 //   warp 0      TMA producer (one elected lane): fills a STAGES-deep ring of
 //               A/B tiles in shared memory, 128-byte swizzled.
 //   warp 1      TMEM owner + MMA issuer (one elected lane): tcgen05.mma into one
-//               of two TMEM accumulators (BN fp32 columns each), commits free
-//               the smem slots and hand finished accumulators to the epilogue.
+//               of two TMEM accumulators (BN fp32 columns each); commits free the
+//               smem slots and hand finished accumulators to the epilogue.
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
 //               lanes 32*(w%4)..+31 = tile rows), fused arithmetic, stores.
 // The two accumulators let the epilogue of tile i overlap the MMAs of tile i+1.
 //
 // Operand kinds:
-//   BF16   kind::f16, bf16 operands, fp32 accumulate, BK = 64 (128 B rows).
-//   TF32X3 kind::tf32 with each fp32 operand pre-split into hi + lo tf32
-//          planes; D = Ahi*Bhi + Ahi*Blo + Alo*Bhi (fp32-faithful), BK = 32.
+//   BF16    kind::f16, bf16 operands, fp32 accumulate, BK = 64 (128 B rows).
+//   SPLIT3  fp32-faithful product on the bf16 tensor cores: each fp32 operand is
+//           held as three bf16 planes x = x0 + x1 + x2 (24 significant bits), and
+//           the six products whose size reaches the fp32 unit roundoff,
+//           x1y1 + x0y2 + x2y0 + x0y1 + x1y0 + x0y0 (smallest first), accumulate
+//           in one fp32 TMEM accumulator.  Same MMA count per K as a three-pass
+//           tf32 scheme, but with fp32-level accuracy.
 // Operand majors: K-major (rows of the operand run along K) or MN-major
 // (rows run along M/N, i.e. the row-major matrix is K x MN).
 #pragma once
@@ -30,13 +45,14 @@ namespace mao {
 
 constexpr int kMaxClasses = 8;
 
-enum OperandKind : int { OP_BF16 = 0, OP_TF32X3 = 1 };
+enum OperandKind : int { OP_BF16 = 0, OP_SPLIT3 = 1 };
 
 enum EpiKind : int {
   EPI_STORE_F32 = 0,  // out0 (f32) = alpha * acc
   EPI_GRAM = 1,       // out0 (bf16) = acc * s_b^2                    (A = X X^T)
   EPI_POLY = 2,       // out0 (bf16) = beta * aux + gamma * acc       (B = b A + c A A)
   EPI_AXPY_T = 3,     // v = s_b * (alpha * aux + acc); out0 (bf16) = v, out1 = v^T if given  (X = a X + B X)
+  EPI_TABLE = 4,      // table mode fp32 epilogue (see GemmProblem)
 };
 
 struct GemmClass {
@@ -58,7 +74,6 @@ struct GemmClass {
 };
 
 struct GemmParams {
-  // Per class: A and B descriptors; for TF32X3 also the lo planes.
   CUtensorMap mapA[kMaxClasses];
   CUtensorMap mapB[kMaxClasses];
   GemmClass cls[kMaxClasses];
@@ -68,28 +83,43 @@ struct GemmParams {
   DevStatus* status;
 };
 
-// TF32X3 needs the lo planes too; they live in a second parameter block so the
-// bf16 kernels keep a small parameter footprint.
-struct GemmLoMaps {
-  CUtensorMap mapAlo[kMaxClasses];
-  CUtensorMap mapBlo[kMaxClasses];
+// Table mode: one entry per problem (device memory, 64-byte aligned maps).
+struct GemmProblem {
+  const CUtensorMap* mapA[3];  // the three bf16 planes of A and of B
+  const CUtensorMap* mapB[3];
+  float* out;                  // M x N fp32 (ld_out), or nullptr
+  __nv_bfloat16* out_p[3];     // three-plane split of the result (ld_outp), or nullptr
+  const float* aux;            // M x N fp32 (ld_aux), or nullptr; may equal out
+  const int* flag;             // nullptr, or skip this problem when *flag == 0
+  int M, N, K;
+  int m_off, n_off;            // operand coordinates of output row/column 0 (sub-block views)
+  int ld_out, ld_aux, ld_outp;
+  int tiles_n, tile_begin;
+  float alpha, beta;
+};
+
+struct GemmTableParams {
+  const GemmProblem* probs;
+  int nprob;
+  int total_tiles;
+  DevStatus* status;
 };
 
 template <int KIND, int A_MN, int B_MN>
 struct GemmCfg {
   static constexpr int BM = 128;
-  static constexpr int BN = 256;
-  static constexpr int ESIZE = (KIND == OP_BF16) ? 2 : 4;
-  static constexpr int BK = 128 / ESIZE;              // elements per 128-byte row
-  static constexpr int UMMA_K = (KIND == OP_BF16) ? 16 : 8;  // 32 bytes of K per MMA
-  static constexpr int PLANES = (KIND == OP_BF16) ? 1 : 2;
+  static constexpr int BN = (KIND == OP_BF16) ? 256 : 128;
+  static constexpr int ESIZE = 2;                      // bf16 planes
+  static constexpr int BK = 64;                        // elements per 128-byte row
+  static constexpr int UMMA_K = 16;                    // 32 bytes of K per MMA
+  static constexpr int PLANES = (KIND == OP_BF16) ? 1 : 3;
   static constexpr int A_TILE = BM * 128;              // bytes per plane
   static constexpr int B_TILE = BN * 128;
   static constexpr int STAGE_BYTES = PLANES * (A_TILE + B_TILE);
   static constexpr int STAGES = (KIND == OP_BF16) ? 4 : 2;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
   static constexpr int TMEM_COLS = 2 * BN;  // two accumulators
-  static constexpr uint32_t IDESC = make_idesc(KIND == OP_BF16 ? 1u : 2u, A_MN, B_MN, BM, BN);
+  static constexpr uint32_t IDESC = make_idesc(1u, A_MN, B_MN, BM, BN);
   static constexpr int THREADS = 192;
 };
 
@@ -106,8 +136,6 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int k) {
     // BK*128 bytes; a k-step covers UMMA_K K-rows = (32/ESIZE) rows of 128 B.
     constexpr int BK = 128 / ESIZE;
     constexpr int ROWS_PER_STEP = UMMA_K_BYTES / ESIZE;
-    if constexpr (ESIZE == 4)  // tf32: 128-byte swizzle of 32-byte atoms, 4-row (512 B) groups
-      return smem_desc_sw128(base + k * ROWS_PER_STEP * 128, BK * 128, 512, 1);
     return smem_desc_sw128(base + k * ROWS_PER_STEP * 128, BK * 128, 1024);
   }
 }
@@ -124,13 +152,6 @@ __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* ma
 #pragma unroll
     for (int c = 0; c < R / CHUNK; ++c) tma_load_3d(dst + c * BK * 128, map, bar, mn0 + c * CHUNK, k0, b);
   }
-}
-
-__device__ __forceinline__ int find_class(const GemmParams& p, int tile) {
-  int c = 0;
-#pragma unroll 1
-  while (c + 1 < p.nclasses && tile >= p.cls[c + 1].tile_begin) ++c;
-  return c;
 }
 
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v) {
@@ -161,69 +182,212 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float* v)
   }
 }
 
-// Epilogue for 32 consecutive columns [col0, col0+32) of one tile row.
-template <int EPI>
-__device__ __forceinline__ void epilogue_chunk(const GemmParams& p, const GemmClass& C, int b, int row,
-                                               int col0, float* v) {
-  if (row >= C.M) return;
-  const bool full = (col0 + 32 <= C.N);
-  if constexpr (EPI == EPI_STORE_F32) {
-    float* out = reinterpret_cast<float*>(C.out0) + (long long)b * C.out0_bs + (long long)row * C.out0_ld + col0;
-    if (full) {
-#pragma unroll
-      for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4*>(out + j) =
-            make_float4(p.alpha * v[j], p.alpha * v[j + 1], p.alpha * v[j + 2], p.alpha * v[j + 3]);
-    } else {
-      for (int j = 0; j < 32 && col0 + j < C.N; ++j) out[j] = p.alpha * v[j];
+// What one tile needs from its problem description.
+struct TileInfo {
+  const CUtensorMap* mapA[3];
+  const CUtensorMap* mapB[3];
+  int idx;     // class (class mode) or problem (table mode)
+  int b;       // batch index inside the class (class mode), 0 in table mode
+  int m0, n0;
+  int K;
+  bool valid;  // false: the tile's problem is gated off
+  int am, bn;  // operand coordinate offsets along M (A) and N (B)
+};
+
+// ------------------------------------------------------------------ class mode
+struct ClassSource {
+  const GemmParams& p;
+  __device__ explicit ClassSource(const GemmParams& p_) : p(p_) {}
+  __device__ int total_tiles() const { return p.total_tiles; }
+  __device__ DevStatus* status() const { return p.status; }
+  __device__ void prefetch() const {
+    for (int c = 0; c < p.nclasses; ++c) {
+      tma_prefetch_desc(&p.mapA[c]);
+      tma_prefetch_desc(&p.mapB[c]);
     }
-  } else {
-    const float s = C.scale ? C.scale[b] : 1.0f;
-    if constexpr (EPI == EPI_GRAM) {
-      const float s2 = s * s;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] *= s2;
-    } else {
-      float a[32];
-      const __nv_bfloat16* aux = reinterpret_cast<const __nv_bfloat16*>(C.aux) + (long long)b * C.aux_bs +
-                                 (long long)row * C.aux_ld + col0;
+  }
+  __device__ TileInfo decode(int tile, int BM, int BN) const {
+    int c = 0;
+#pragma unroll 1
+    while (c + 1 < p.nclasses && tile >= p.cls[c + 1].tile_begin) ++c;
+    const GemmClass& C = p.cls[c];
+    const int local = tile - C.tile_begin;
+    const int b = local / C.tiles_per_mat;
+    const int r = local - b * C.tiles_per_mat;
+    TileInfo t;
+    t.mapA[0] = &p.mapA[c];
+    t.mapB[0] = &p.mapB[c];
+    t.mapA[1] = t.mapA[2] = t.mapB[1] = t.mapB[2] = nullptr;
+    t.idx = c;
+    t.b = b;
+    t.m0 = (r / C.tiles_n) * BM;
+    t.n0 = (r % C.tiles_n) * BN;
+    t.K = C.K;
+    t.valid = true;
+    t.am = 0;
+    t.bn = 0;
+    return t;
+  }
+  __device__ int cols(const TileInfo& t) const { return p.cls[t.idx].N; }
+
+  // Epilogue for 32 consecutive columns [col0, col0+32) of one tile row.
+  template <int EPI>
+  __device__ __forceinline__ void epilogue(const TileInfo& t, int row, int col0, float* v) const {
+    const GemmClass& C = p.cls[t.idx];
+    const int b = t.b;
+    if (row >= C.M) return;
+    const bool full = (col0 + 32 <= C.N);
+    if constexpr (EPI == EPI_STORE_F32) {
+      float* out =
+          reinterpret_cast<float*>(C.out0) + (long long)b * C.out0_bs + (long long)row * C.out0_ld + col0;
       if (full) {
-        load_bf16x32(aux, a);
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(out + j) =
+              make_float4(p.alpha * v[j], p.alpha * v[j + 1], p.alpha * v[j + 2], p.alpha * v[j + 3]);
       } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) a[j] = (col0 + j < C.N) ? __bfloat162float(aux[j]) : 0.0f;
+        for (int j = 0; j < 32 && col0 + j < C.N; ++j) out[j] = p.alpha * v[j];
       }
-      if constexpr (EPI == EPI_POLY) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = p.beta * a[j] + p.gamma * v[j];
-      } else {  // EPI_AXPY_T
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = s * (p.alpha * a[j] + v[j]);
-      }
-    }
-    __nv_bfloat16* out =
-        reinterpret_cast<__nv_bfloat16*>(C.out0) + (long long)b * C.out0_bs + (long long)row * C.out0_ld + col0;
-    if (full) {
-      store_bf16x32(out, v);
     } else {
-      for (int j = 0; j < 32 && col0 + j < C.N; ++j) out[j] = __float2bfloat16_rn(v[j]);
-    }
-    if constexpr (EPI == EPI_AXPY_T) {
-      if (C.out1 != nullptr) {
-        // optional transposed copy: for each column j, the 32 lanes (consecutive
-        // rows) write 32 consecutive elements of row (col0 + j) of out1.
-        __nv_bfloat16* t = reinterpret_cast<__nv_bfloat16*>(C.out1) + (long long)b * C.out1_bs + row;
+      const float s = C.scale ? C.scale[b] : 1.0f;
+      if constexpr (EPI == EPI_GRAM) {
+        const float s2 = s * s;
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (col0 + j < C.N) t[(long long)(col0 + j) * C.out1_ld] = __float2bfloat16_rn(v[j]);
+        for (int j = 0; j < 32; ++j) v[j] *= s2;
+      } else {
+        float a[32];
+        const __nv_bfloat16* aux = reinterpret_cast<const __nv_bfloat16*>(C.aux) + (long long)b * C.aux_bs +
+                                   (long long)row * C.aux_ld + col0;
+        if (full) {
+          load_bf16x32(aux, a);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) a[j] = (col0 + j < C.N) ? __bfloat162float(aux[j]) : 0.0f;
+        }
+        if constexpr (EPI == EPI_POLY) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = p.beta * a[j] + p.gamma * v[j];
+        } else {  // EPI_AXPY_T
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = s * (p.alpha * a[j] + v[j]);
+        }
+      }
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(C.out0) + (long long)b * C.out0_bs +
+                           (long long)row * C.out0_ld + col0;
+      if (full) {
+        store_bf16x32(out, v);
+      } else {
+        for (int j = 0; j < 32 && col0 + j < C.N; ++j) out[j] = __float2bfloat16_rn(v[j]);
+      }
+      if constexpr (EPI == EPI_AXPY_T) {
+        if (C.out1 != nullptr) {
+          // optional transposed copy: for each column j, the 32 lanes (consecutive
+          // rows) write 32 consecutive elements of row (col0 + j) of out1.
+          __nv_bfloat16* tp = reinterpret_cast<__nv_bfloat16*>(C.out1) + (long long)b * C.out1_bs + row;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (col0 + j < C.N) tp[(long long)(col0 + j) * C.out1_ld] = __float2bfloat16_rn(v[j]);
+        }
       }
     }
   }
-}
+};
 
-template <int KIND, int A_MN, int B_MN, int EPI>
-__global__ void __launch_bounds__(192, 1)
-    gemm_tc_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ GemmLoMaps lo) {
+// ------------------------------------------------------------------ table mode
+struct TableSource {
+  const GemmTableParams& p;
+  __device__ explicit TableSource(const GemmTableParams& p_) : p(p_) {}
+  __device__ int total_tiles() const { return p.total_tiles; }
+  __device__ DevStatus* status() const { return p.status; }
+  __device__ void prefetch() const {}
+  __device__ TileInfo decode(int tile, int BM, int BN) const {
+    int lo = 0, hi = p.nprob - 1;
+#pragma unroll 1
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.probs[mid].tile_begin <= tile) lo = mid; else hi = mid - 1;
+    }
+    const GemmProblem& P = p.probs[lo];
+    const int r = tile - P.tile_begin;
+    TileInfo t;
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      t.mapA[q] = P.mapA[q];
+      t.mapB[q] = P.mapB[q];
+    }
+    t.idx = lo;
+    t.b = 0;
+    t.m0 = (r / P.tiles_n) * BM;
+    t.n0 = (r % P.tiles_n) * BN;
+    t.K = P.K;
+    t.valid = (P.flag == nullptr) || (*P.flag != 0);
+    t.am = P.m_off;
+    t.bn = P.n_off;
+    return t;
+  }
+  __device__ int cols(const TileInfo& t) const { return p.probs[t.idx].N; }
+
+  template <int EPI>
+  __device__ __forceinline__ void epilogue(const TileInfo& t, int row, int col0, float* v) const {
+    const GemmProblem& P = p.probs[t.idx];
+    if (row >= P.M) return;
+    const bool full = (col0 + 32 <= P.N);
+    if (P.aux != nullptr) {
+      const float* a = P.aux + (long long)row * P.ld_aux + col0;
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float4 q = *reinterpret_cast<const float4*>(a + j);
+          v[j] = P.alpha * v[j] + P.beta * q.x;
+          v[j + 1] = P.alpha * v[j + 1] + P.beta * q.y;
+          v[j + 2] = P.alpha * v[j + 2] + P.beta * q.z;
+          v[j + 3] = P.alpha * v[j + 3] + P.beta * q.w;
+        }
+      } else {
+        for (int j = 0; j < 32; ++j) v[j] = (col0 + j < P.N) ? P.alpha * v[j] + P.beta * a[j] : 0.0f;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= P.alpha;
+    }
+    const long long off = (long long)row * P.ld_out + col0;
+    if (P.out != nullptr) {
+      float* o = P.out + off;
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(o + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      } else {
+        for (int j = 0; j < 32 && col0 + j < P.N; ++j) o[j] = v[j];
+      }
+    }
+    if (P.out_p[0] != nullptr) {
+      const long long offp = (long long)row * P.ld_outp + col0;
+      float r[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) r[j] = v[j];
+#pragma unroll
+      for (int q = 0; q < 3; ++q) {
+        float pq[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          pq[j] = __bfloat162float(__float2bfloat16_rn(r[j]));
+          r[j] -= pq[j];
+        }
+        __nv_bfloat16* o = P.out_p[q] + offp;
+        if (full) {
+          store_bf16x32(o, pq);
+        } else {
+          for (int j = 0; j < 32 && col0 + j < P.N; ++j) o[j] = __float2bfloat16_rn(pq[j]);
+        }
+      }
+    }
+  }
+};
+
+// ------------------------------------------------------------------ kernel body
+template <int KIND, int A_MN, int B_MN, int EPI, class Src>
+__device__ __forceinline__ void gemm_body(const Src& src) {
   using Cfg = GemmCfg<KIND, A_MN, B_MN>;
   constexpr int BM = Cfg::BM, BN = Cfg::BN, BK = Cfg::BK, STAGES = Cfg::STAGES;
 
@@ -242,6 +406,7 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  DevStatus* status = src.status();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -263,48 +428,46 @@ __global__ void __launch_bounds__(192, 1)
     tmem_alloc(&tmem_base_sh, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) {
-    for (int c = 0; c < p.nclasses; ++c) {
-      tma_prefetch_desc(&p.mapA[c]);
-      tma_prefetch_desc(&p.mapB[c]);
-    }
-  }
+  if (warp == 0 && lane == 0) src.prefetch();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
   volatile int* abort_flag = &abort_sh;
+  const int total = src.total_tiles();
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
       int it = 0;
-      for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
-        const int c = find_class(p, tile);
-        const GemmClass& C = p.cls[c];
-        const int local = tile - C.tile_begin;
-        const int b = local / C.tiles_per_mat;
-        const int r = local - b * C.tiles_per_mat;
-        const int m0 = (r / C.tiles_n) * BM;
-        const int n0 = (r % C.tiles_n) * BN;
-        const int nk = (C.K + BK - 1) / BK;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        const TileInfo t = src.decode(tile, BM, BN);
+        if (!t.valid) continue;
+        if constexpr (EPI == EPI_TABLE) {
+#pragma unroll
+          for (int q = 0; q < Cfg::PLANES; ++q) {
+            tensormap_acquire(t.mapA[q]);
+            tensormap_acquire(t.mapB[q]);
+          }
+        }
+        const int nk = (t.K + BK - 1) / BK;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(&empty_bar[s], ph ^ 1, p.status, 1, abort_flag)) {
+          if (!mbar_wait(&empty_bar[s], ph ^ 1, status, 1, abort_flag)) {
             ok = false;
             break;
           }
           uint8_t* st = smem + s * Cfg::STAGE_BYTES;
           mbar_arrive_expect_tx(&full_bar[s], Cfg::STAGE_BYTES);
-          load_operand<A_MN, BM, Cfg::ESIZE>(st, &p.mapA[c], &full_bar[s], kb * BK, m0, b);
-          load_operand<B_MN, BN, Cfg::ESIZE>(st + Cfg::A_TILE, &p.mapB[c], &full_bar[s], kb * BK, n0, b);
-          if constexpr (KIND == OP_TF32X3) {
-            load_operand<A_MN, BM, Cfg::ESIZE>(st + Cfg::A_TILE + Cfg::B_TILE, &lo.mapAlo[c], &full_bar[s],
-                                               kb * BK, m0, b);
-            load_operand<B_MN, BN, Cfg::ESIZE>(st + 2 * Cfg::A_TILE + Cfg::B_TILE, &lo.mapBlo[c],
-                                               &full_bar[s], kb * BK, n0, b);
+          const int am = t.am + t.m0, bn = t.bn + t.n0;
+          // stage layout: A planes, then B planes
+#pragma unroll
+          for (int q = 0; q < Cfg::PLANES; ++q) {
+            load_operand<A_MN, BM, Cfg::ESIZE>(st + q * Cfg::A_TILE, t.mapA[q], &full_bar[s], kb * BK, am, t.b);
+            load_operand<B_MN, BN, Cfg::ESIZE>(st + Cfg::PLANES * Cfg::A_TILE + q * Cfg::B_TILE, t.mapB[q],
+                                               &full_bar[s], kb * BK, bn, t.b);
           }
         }
         if (!ok) break;
@@ -314,43 +477,43 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      int it = 0, tl = 0;
-      for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++tl) {
-        const int c = find_class(p, tile);
-        const GemmClass& C = p.cls[c];
-        const int nk = (C.K + BK - 1) / BK;
-        const int acc = tl & 1;
-        const uint32_t aph = (tl >> 1) & 1;
-        if (!mbar_wait(&tempty_bar[acc], aph ^ 1, p.status, 2, abort_flag)) break;
+      int it = 0, used = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        const TileInfo t = src.decode(tile, BM, BN);
+        if (!t.valid) continue;
+        const int nk = (t.K + BK - 1) / BK;
+        const int acc = used & 1;
+        const uint32_t aph = (used >> 1) & 1;
+        ++used;
+        if (!mbar_wait(&tempty_bar[acc], aph ^ 1, status, 2, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(&full_bar[s], ph, p.status, 3, abort_flag)) {
+          if (!mbar_wait(&full_bar[s], ph, status, 3, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + s * Cfg::STAGE_BYTES);
-          const uint32_t b_base = a_base + Cfg::A_TILE;
+          const uint32_t b_base = a_base + Cfg::PLANES * Cfg::A_TILE;
 #pragma unroll
           for (int k = 0; k < BK / Cfg::UMMA_K; ++k) {
-            const uint64_t ad = operand_desc<A_MN, BM, Cfg::ESIZE>(a_base, k);
-            const uint64_t bd = operand_desc<B_MN, BN, Cfg::ESIZE>(b_base, k);
             const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
             if constexpr (KIND == OP_BF16) {
-              umma_f16(d_tmem, ad, bd, Cfg::IDESC, accum);
+              umma_f16(d_tmem, operand_desc<A_MN, BM, Cfg::ESIZE>(a_base, k),
+                       operand_desc<B_MN, BN, Cfg::ESIZE>(b_base, k), Cfg::IDESC, accum);
             } else {
-              const uint32_t alo_base = b_base + Cfg::B_TILE;
-              const uint32_t blo_base = alo_base + Cfg::A_TILE;
-              const uint64_t adl = operand_desc<A_MN, BM, Cfg::ESIZE>(alo_base, k);
-              const uint64_t bdl = operand_desc<B_MN, BN, Cfg::ESIZE>(blo_base, k);
-              // small cross terms first, the dominant hi*hi product last
-              umma_tf32(d_tmem, adl, bd, Cfg::IDESC, accum);
-              umma_tf32(d_tmem, ad, bdl, Cfg::IDESC, 1u);
-              umma_tf32(d_tmem, ad, bd, Cfg::IDESC, 1u);
+              // (A plane, B plane) products, smallest magnitude first
+              constexpr int pa[6] = {1, 0, 2, 0, 1, 0};
+              constexpr int pb[6] = {1, 2, 0, 1, 0, 0};
+#pragma unroll
+              for (int q = 0; q < 6; ++q)
+                umma_f16(d_tmem, operand_desc<A_MN, BM, Cfg::ESIZE>(a_base + pa[q] * Cfg::A_TILE, k),
+                         operand_desc<B_MN, BN, Cfg::ESIZE>(b_base + pb[q] * Cfg::B_TILE, k), Cfg::IDESC,
+                         q == 0 ? accum : 1u);
             }
           }
           umma_commit(&empty_bar[s]);
@@ -361,27 +524,24 @@ __global__ void __launch_bounds__(192, 1)
       // every MMA this thread issued has finished before TMEM is released
       mma_it_sh = it;
       umma_commit(&drain_bar);
-      mbar_wait(&drain_bar, 0, p.status, 5, abort_flag, false);
+      mbar_wait(&drain_bar, 0, status, 5, abort_flag, false);
     }
   } else {
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;
     const int row_in_tile = q * 32 + lane;
-    int tl = 0;
-    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++tl) {
-      const int acc = tl & 1;
-      const uint32_t aph = (tl >> 1) & 1;
-      const bool ok = mbar_wait(&tfull_bar[acc], aph, p.status, 4, abort_flag);
+    int used = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const TileInfo t = src.decode(tile, BM, BN);
+      if (!t.valid) continue;
+      const int acc = used & 1;
+      const uint32_t aph = (used >> 1) & 1;
+      ++used;
+      const bool ok = mbar_wait(&tfull_bar[acc], aph, status, 4, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const int c = find_class(p, tile);
-      const GemmClass& C = p.cls[c];
-      const int local = tile - C.tile_begin;
-      const int b = local / C.tiles_per_mat;
-      const int r = local - b * C.tiles_per_mat;
-      const int m0 = (r / C.tiles_n) * BM;
-      const int n0 = (r % C.tiles_n) * BN;
-      const int row = m0 + row_in_tile;
+      const int row = t.m0 + row_in_tile;
+      const int ncols = src.cols(t);
 #pragma unroll 1
       for (int ch = 0; ch < BN / 32; ++ch) {
         uint32_t rr[32];
@@ -390,7 +550,7 @@ __global__ void __launch_bounds__(192, 1)
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(rr[j]);
-        if (n0 + ch * 32 < C.N) epilogue_chunk<EPI>(p, C, b, row, n0 + ch * 32, v);
+        if (t.n0 + ch * 32 < ncols) src.template epilogue<EPI>(t, row, t.n0 + ch * 32, v);
       }
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
@@ -401,7 +561,7 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0 && lane == 0) {
     // after an early exit, let TMA loads still in flight land before the CTA ends
     for (int j = mma_it_sh; j < prod_it_sh; ++j)
-      mbar_wait(&full_bar[j % STAGES], (j / STAGES) & 1, p.status, 6, abort_flag, false);
+      mbar_wait(&full_bar[j % STAGES], (j / STAGES) & 1, status, 6, abort_flag, false);
   }
   tc_fence_before();
   __syncthreads();
@@ -410,6 +570,18 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }
+}
+
+template <int KIND, int A_MN, int B_MN, int EPI>
+__global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ GemmParams p) {
+  ClassSource src(p);
+  gemm_body<KIND, A_MN, B_MN, EPI>(src);
+}
+
+template <int KIND, int A_MN, int B_MN>
+__global__ void __launch_bounds__(192, 1) gemm_tc_table_kernel(const __grid_constant__ GemmTableParams p) {
+  TableSource src(p);
+  gemm_body<KIND, A_MN, B_MN, EPI_TABLE>(src);
 }
 
 }  // namespace mao

@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 #include <vector>
 
 #include "gemm_tc.cuh"
@@ -68,15 +69,17 @@ struct OperandView {
 // boxes {128 B of MN, BK K-rows}.
 mao_status encode_operand(CUtensorMap* map, int kind, int mn_major, int R, const OperandView& v);
 
-// Launch one grouped GEMM of the given instantiation.  `lo` may be null for bf16.
+// Launch one class-mode (bf16) grouped GEMM of the given instantiation;
 // kernel_id tags the launch for the profiler.
-mao_status launch_gemm(int kind, int a_mn, int b_mn, int epi, const GemmParams& p, const GemmLoMaps* lo,
-                       cudaStream_t stream, int kernel_id);
+mao_status launch_gemm(int kind, int a_mn, int b_mn, int epi, const GemmParams& p, cudaStream_t stream,
+                       int kernel_id);
 
 // Fill tile bookkeeping of the classes in p (M, N, K, count must be set).
 void finalize_classes(GemmParams& p);
 
-mao_status launch_tf32_split(const float* src, float* hi, float* lo, size_t n, cudaStream_t stream);
+// fp32 -> three bf16 planes (x = p0 + p1 + p2).
+mao_status launch_split3(const float* src, __nv_bfloat16* p0, __nv_bfloat16* p1, __nv_bfloat16* p2, size_t n,
+                         cudaStream_t stream);
 
 }  // namespace mao
 
@@ -115,5 +118,90 @@ struct LaunchScope {
     if (slot >= 0) cudaEventRecord(static_cast<cudaEvent_t>(profiler().events[2 * slot + 1]), s);
   }
 };
+
+}  // namespace mao
+
+namespace mao {
+
+// ---------------------------------------------------------------- staging arena
+// Host image of a device region: everything a step needs in device memory that
+// the host prepares (problem tables, tensor maps, per-matrix descriptors) is
+// laid out here and copied with one cudaMemcpyAsync.
+struct Arena {
+  uint8_t* dev = nullptr;   // device base (inside the workspace), or nullptr while sizing
+  size_t cap = 0;
+  std::vector<uint8_t> host;
+  size_t take(size_t bytes, size_t align = 64) {
+    size_t at = align_up(host.size(), align);
+    host.resize(at + bytes);
+    return at;
+  }
+  template <class T>
+  T* hptr(size_t off) { return reinterpret_cast<T*>(host.data() + off); }
+  template <class T>
+  T* dptr(size_t off) const { return dev ? reinterpret_cast<T*>(dev + off) : nullptr; }
+};
+
+// An fp32 row-major matrix held as three bf16 planes x = p0 + p1 + p2 (operand
+// of an fp32-faithful SPLIT3 product); ld in elements, a multiple of 8.
+struct Split3 {
+  const __nv_bfloat16* p[3];
+  int rows, cols, ld;
+};
+
+// Collects the problems of one table-mode SPLIT3 launch (fixed operand majors):
+//   out (M x N) = alpha * op(A) op(B) + beta * aux
+// with op(A) = A (a_mn = 0, A stored M x K) or A^T (a_mn = 1, A stored K x M), and
+// op(B) = B^T (b_mn = 0, B stored N x K) or B (b_mn = 1, B stored K x N).
+struct TableLaunch {
+  int a_mn = 0, b_mn = 0;
+  int kernel_id = 0;
+  std::vector<GemmProblem> probs;
+  std::vector<int> map_idx;  // 6 per problem: A planes 0..2, B planes 0..2 (indices into the step's map list)
+};
+
+struct MapKey {
+  const void* p;
+  int inner, rows, ld, box_rows, mn;
+  bool operator==(const MapKey& o) const {
+    return p == o.p && inner == o.inner && rows == o.rows && ld == o.ld && box_rows == o.box_rows && mn == o.mn;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    size_t h = std::hash<const void*>()(k.p);
+    h ^= (size_t)k.inner * 0x9E3779B97F4A7C15ull + (size_t)k.rows * 0xC2B2AE3D27D4EB4Full +
+         (size_t)k.ld * 0x165667B19E3779F9ull + (size_t)k.box_rows * 31 + (size_t)k.mn;
+    return h;
+  }
+};
+
+// The tensor maps one step needs, de-duplicated.
+struct MapSet {
+  std::vector<MapKey> keys;
+  std::vector<CUtensorMap> maps;
+  std::unordered_map<MapKey, int, MapKeyHash> index;
+  int get(const void* p, int inner, int rows, int ld, int box_rows, int mn);  // index (encodes lazily)
+  mao_status encode_all();
+};
+
+// Add a problem; A/B describe the stored matrices (see TableLaunch).  m_off / n_off
+// shift the operand coordinates (sub-block products); they must be multiples of 8
+// when the operand is MN-major (TMA inner coordinate alignment).  `outp`, when
+// given, receives the three-plane split of the result.
+mao_status table_add(TableLaunch& L, MapSet& maps, const Split3& A, const Split3& B, int M, int N, int K,
+                     int m_off, int n_off, float* out, const Split3* outp, int ld_out, const float* aux,
+                     int ld_aux, float alpha, float beta, const int* flag);
+
+// Stage a launch's problem table into the arena (maps live at maps_off) and launch it.
+struct StagedLaunch {
+  size_t probs_off = 0;
+  int nprob = 0;
+  int total_tiles = 0;
+  int a_mn = 0, b_mn = 0, kernel_id = 0;
+  double flops = 0.0;
+};
+StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off);
+mao_status table_launch(const Arena& A, const StagedLaunch& S, DevStatus* status, cudaStream_t stream);
 
 }  // namespace mao

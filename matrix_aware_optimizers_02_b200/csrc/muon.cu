@@ -299,9 +299,9 @@ extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, con
         finalize_classes(g1p);
         finalize_classes(g2p);
         finalize_classes(g3p);
-        MAO_TRY(launch_gemm(OP_BF16, 0, 0, EPI_GRAM, g1p, nullptr, stream, MAO_K_NS_GRAM));
-        MAO_TRY(launch_gemm(OP_BF16, 0, 0, EPI_POLY, g2p, nullptr, stream, MAO_K_NS_POLY));
-        MAO_TRY(launch_gemm(OP_BF16, 0, 1, EPI_AXPY_T, g3p, nullptr, stream, MAO_K_NS_AXPY));
+        MAO_TRY(launch_gemm(OP_BF16, 0, 0, EPI_GRAM, g1p, stream, MAO_K_NS_GRAM));
+        MAO_TRY(launch_gemm(OP_BF16, 0, 0, EPI_POLY, g2p, stream, MAO_K_NS_POLY));
+        MAO_TRY(launch_gemm(OP_BF16, 0, 1, EPI_AXPY_T, g3p, stream, MAO_K_NS_AXPY));
       }
     }
   }

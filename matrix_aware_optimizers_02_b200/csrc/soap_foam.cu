@@ -1,11 +1,32 @@
-// mao_soap_step / mao_foam_step: argument validation and workspace planning.
+// mao_soap_step / mao_foam_step: one SOAP or FOAM step over a batch of matrices.
+//
+// Matrices are processed in groups whose scratch fits a fixed budget; each group
+// runs the whole step with every phase batched over the group's matrices:
+//
+//   momentum      M <- b1 M + (1-b1) G; three-plane bf16 splits of G and M
+//   factor EMAs   L <- b2 L + (1-b2) G G^T (SOAP), R <- b2 R + (1-b2) G^T G
+//                 (fp32-faithful SPLIT3 tensor-core GEMMs with the EMA in the epilogue)
+//   refresh       per side, when the policy says so: [adaptive check D = Q^T F Q,
+//                 rho, flag] -> P = F Q -> keys diag(Q^T F Q) in fp64 -> stable
+//                 descending argsort -> gathered P -> QR (block Gram-Schmidt with
+//                 re-orthogonalisation; panels of 64 columns orthonormalised by
+//                 two fp64 Cholesky-QR passes) -> Q.  Every refresh kernel reads a
+//                 per-matrix device flag, so adaptive refreshes need no host sync.
+//   SOAP          Gh, Mh = Q_L^T {G, M} Q_R ; Adam in the eigenbasis (V follows the
+//                 permutations) ; U = Q_L N Q_R^T fused with W <- W(1 - lr wd) - lr U
+//   FOAM          Gr, Mr = {G, M} Q_R ; r, c EMAs of row/column means of Gr^2 ; tau ;
+//                 N = (Mr/bc1)/(sqrt(tau r c^T)+eps) ; U = N Q_R^T fused with the W update
+#include <algorithm>
 #include <cmath>
 
 #include "host_common.h"
+#include "precond_kernels.cuh"
 
 using namespace mao;
 
 namespace {
+
+constexpr size_t kGroupBudget = (size_t)24 << 30;  // scratch bytes per group of matrices
 
 mao_status check_refresh(const mao_refresh& r) {
   if (r.kind < MAO_REFRESH_EVERY_K || r.kind > MAO_REFRESH_NEVER) return MAO_ERR_INVALID_ARG;
@@ -22,13 +43,954 @@ mao_status check_hyper(float b1, float b2, float eps, float lr, float wd, int64_
   return MAO_OK;
 }
 
-mao_status check_mat(int m, int n, const void* G, int g_dtype) {
+mao_status check_mat(int m, int n, int g_dtype) {
   if (m < 1 || n < 1) return MAO_ERR_SHAPE;
-  if ((long long)m * n > (1ll << 31) - 1) return MAO_ERR_SHAPE;
+  if ((long long)m * n > (1ll << 31) - 1 || (long long)m * m > (1ll << 31) - 1 || (long long)n * n > (1ll << 31) - 1)
+    return MAO_ERR_SHAPE;
   if (g_dtype != MAO_F32 && g_dtype != MAO_BF16) return MAO_ERR_DTYPE;
   if (m % 4 || n % 4) return MAO_ERR_SHAPE;
   if (g_dtype == MAO_BF16 && n % 8) return MAO_ERR_SHAPE;
-  (void)G;
+  return MAO_OK;
+}
+
+// Unified per-matrix view.
+struct PcMat {
+  int m, n;
+  float* W;
+  const void* G;
+  int g_bf16;
+  float* M;
+  float* V;             // SOAP
+  float *L, *R, *QL, *QR;
+  int *perm_L, *perm_R;
+  float *r, *c;         // FOAM
+};
+
+// Refresh decision known on the host: 0 = no refresh, 1 = refresh, 2 = adaptive check on device.
+int host_refresh_mode(const mao_refresh& rf, int64_t t) {
+  if (rf.kind == MAO_REFRESH_NEVER) return 0;
+  if (rf.kind == MAO_REFRESH_EVERY_K) return ((t - 1) % rf.k) == 0 ? 1 : 0;
+  return ((t - 1) % rf.pf) == 0 ? 2 : 0;
+}
+
+inline int ldp_of(int cols) { return round_up_int(cols, 8); }
+
+// Bytes of a three-plane bf16 set of a rows x cols matrix.
+inline size_t planes_bytes(int rows, int cols) { return 3 * 2 * (size_t)rows * ldp_of(cols); }
+
+// Scratch of one side (k x k factor F with basis Q) of one matrix.
+struct SideBuf {
+  size_t Fp, Qp, P, Ps, Psp;
+  size_t W, Wp, Cp;
+  size_t gram, rinv, keys, perm, flag, rho, bad;
+  size_t Tp, D;  // adaptive check
+};
+
+struct MatBuf {
+  size_t Gp, Mp, T1G, T1M, Vtmp, Gh, Mh;  // SOAP (N reuses T1G, T2 reuses Mp)
+  size_t Gr, Mr;                          // FOAM (N reuses Gp)
+  size_t rowpart, colpart, ctmp, tau;
+  SideBuf L, R;
+};
+
+void side_layout(int k, bool check, Carver& cv, SideBuf& s) {
+  const size_t kk = (size_t)k * k;
+  const int chunks = (k + kGramRows - 1) / kGramRows;
+  s.Fp = cv.take(planes_bytes(k, k));
+  s.Qp = cv.take(planes_bytes(k, k));
+  s.P = cv.take(4 * kk);
+  s.Ps = cv.take(4 * kk);
+  s.Psp = cv.take(planes_bytes(k, k));
+  s.W = cv.take(4 * (size_t)k * kPanel);
+  s.Wp = cv.take(planes_bytes(k, kPanel));
+  s.Cp = cv.take(planes_bytes(k, kPanel));
+  s.gram = cv.take(8 * (size_t)chunks * kPanel * kPanel);
+  s.rinv = cv.take(8 * (size_t)kPanel * kPanel);
+  s.keys = cv.take(8 * (size_t)k);
+  s.perm = cv.take(4 * (size_t)k);
+  s.flag = cv.take(64);  // flag, rho and the failure counter share one 64-byte block
+  s.rho = s.flag + 16;
+  s.bad = s.flag + 32;
+  if (check) {
+    s.Tp = cv.take(planes_bytes(k, k));
+    s.D = cv.take(4 * kk);
+  }
+}
+
+struct Ctx {
+  bool foam;
+  const PcMat* mats;
+  int count;
+  float b1, b2, eps, lr, wd;
+  int64_t t;
+  mao_refresh rf;
+  int raw_trace;
+  int mode;  // host refresh mode
+};
+
+struct GroupPlan {
+  int g0 = 0, g1 = 0;   // matrices [g0, g1)
+  size_t scratch = 0;   // bytes of per-matrix scratch
+  std::vector<MatBuf> mb;
+};
+
+void plan_group_scratch(const Ctx& X, GroupPlan& G, size_t base) {
+  Carver cv;
+  cv.off = base;
+  G.mb.assign(G.g1 - G.g0, MatBuf());
+  const bool check = X.mode == 2;
+  for (int i = G.g0; i < G.g1; ++i) {
+    const PcMat& a = X.mats[i];
+    MatBuf& b = G.mb[i - G.g0];
+    const size_t mn = (size_t)a.m * a.n;
+    b.Gp = cv.take(planes_bytes(a.m, a.n));
+    b.Mp = cv.take(planes_bytes(a.m, a.n));
+    if (!X.foam) {
+      b.T1G = cv.take(planes_bytes(a.m, a.n));
+      b.T1M = cv.take(planes_bytes(a.m, a.n));
+      b.Vtmp = cv.take(4 * mn);
+      b.Gh = cv.take(4 * mn);
+      b.Mh = cv.take(4 * mn);
+      side_layout(a.m, check, cv, b.L);
+    } else {
+      b.Gr = cv.take(4 * mn);
+      b.Mr = cv.take(4 * mn);
+      const int tr = (a.m + 63) / 64, tc = (a.n + 63) / 64;
+      b.rowpart = cv.take(4 * (size_t)tc * a.m);
+      b.colpart = cv.take(4 * (size_t)tr * a.n);
+      b.ctmp = cv.take(4 * (size_t)a.n);
+      b.tau = cv.take(16);
+    }
+    side_layout(a.n, check, cv, b.R);
+  }
+  G.scratch = cv.off - base;
+}
+
+size_t mat_scratch_estimate(const Ctx& X, int i) {
+  GroupPlan g;
+  g.g0 = i;
+  g.g1 = i + 1;
+  plan_group_scratch(X, g, 0);
+  return g.scratch;
+}
+
+void make_groups(const Ctx& X, std::vector<GroupPlan>& groups) {
+  groups.clear();
+  int i = 0;
+  while (i < X.count) {
+    GroupPlan g;
+    g.g0 = i;
+    size_t acc = 0;
+    int j = i;
+    while (j < X.count) {
+      const size_t s = mat_scratch_estimate(X, j);
+      if (j > i && acc + s > kGroupBudget) break;
+      acc += s;
+      ++j;
+    }
+    g.g1 = j;
+    groups.push_back(g);
+    i = j;
+  }
+}
+
+// ------------------------------------------------------------------ the builder
+// Records every launch of one group into `ops`, with all device data staged in
+// the arena; in sizing mode (ws == nullptr) only the sizes matter.
+struct Op {
+  enum Kind { GEMM, EW, SPLIT, ADAM, KEYS, ARGSORT, GATHER, VPERM, GRAM, CHOL, APPLY, RC, TAU, FOAMN, CHECK } kind;
+  size_t jobs = 0;
+  int njobs = 0;
+  int blocks = 0;
+  double bytes = 0.0;
+};
+
+struct Builder {
+  const Ctx& X;
+  uint8_t* ws;      // workspace base or nullptr
+  Arena arena;
+  MapSet maps;
+  std::vector<TableLaunch> gemms;  // staged after all maps are known
+  std::vector<Op> ops;
+  std::vector<int> gemm_of_op;     // op index -> gemm index (or -1)
+  size_t zero_flag_off = 0;        // an int 0 in the arena
+
+  Builder(const Ctx& x, uint8_t* w) : X(x), ws(w) {}
+
+  // In sizing mode, pointers are fake but non-null and 16-byte aligned (never dereferenced).
+  template <class T>
+  T* wp(size_t off) const { return ws ? reinterpret_cast<T*>(ws + off) : reinterpret_cast<T*>(off + 16); }
+
+  // Plane set at workspace offset `off` of a rows x cols matrix.
+  Split3 planes(size_t off, int rows, int cols) const {
+    const int ldp = ldp_of(cols);
+    __nv_bfloat16* b = wp<__nv_bfloat16>(off);
+    const size_t st = (size_t)rows * ldp;
+    return Split3{{b, b + st, b + 2 * st}, rows, cols, ldp};
+  }
+  long long pstride(int rows, int cols) const { return (long long)rows * ldp_of(cols); }
+
+  TableLaunch& new_gemm(int a_mn, int b_mn, int kernel_id) {
+    gemms.emplace_back();
+    gemms.back().a_mn = a_mn;
+    gemms.back().b_mn = b_mn;
+    gemms.back().kernel_id = kernel_id;
+    Op o;
+    o.kind = Op::GEMM;
+    ops.push_back(o);
+    gemm_of_op.push_back((int)gemms.size() - 1);
+    return gemms.back();
+  }
+
+  template <class J>
+  J* new_jobs(Op::Kind kind, int n, size_t& off) {
+    off = arena.take(sizeof(J) * std::max(n, 1), 64);
+    Op o;
+    o.kind = kind;
+    o.jobs = off;
+    o.njobs = n;
+    ops.push_back(o);
+    gemm_of_op.push_back(-1);
+    J* p = arena.hptr<J>(off);
+    std::memset(static_cast<void*>(p), 0, sizeof(J) * std::max(n, 1));
+    return p;
+  }
+};
+
+int ew_blocks(int rows, int cols) {
+  const long long e = (long long)rows * cols;
+  return (int)((e + kElemsPerBlock - 1) / kElemsPerBlock);
+}
+
+// Adds the jobs of one side's refresh for every matrix of the group.
+mao_status build_refresh_side(Builder& B, GroupPlan& G, bool left) {
+  const Ctx& X = B.X;
+  const bool check = X.mode == 2;
+  const int nm = G.g1 - G.g0;
+  auto side = [&](int i) -> SideBuf& { return left ? G.mb[i].L : G.mb[i].R; };
+  auto kof = [&](int i) { return left ? X.mats[G.g0 + i].m : X.mats[G.g0 + i].n; };
+  auto Fp = [&](int i) { return left ? X.mats[G.g0 + i].L : X.mats[G.g0 + i].R; };
+  auto Qp = [&](int i) { return left ? X.mats[G.g0 + i].QL : X.mats[G.g0 + i].QR; };
+  auto flagp = [&](int i) -> const int* { return check ? B.wp<int>(side(i).flag) : nullptr; };
+
+  // three-plane splits of F and Q
+  {
+    size_t off;
+    EwJob* J = B.new_jobs<EwJob>(Op::SPLIT, 2 * nm, off);
+    int blk = 0;
+    for (int i = 0; i < nm; ++i) {
+      const int k = kof(i);
+      for (int w = 0; w < 2; ++w) {
+        EwJob& j = J[2 * i + w];
+        j.a = w == 0 ? Fp(i) : Qp(i);
+        j.pa = B.wp<__nv_bfloat16>(w == 0 ? side(i).Fp : side(i).Qp);
+        j.pstride = B.pstride(k, k);
+        j.rows = k;
+        j.cols = k;
+        j.lda = k;
+        j.ldp = ldp_of(k);
+        j.blk_begin = blk;
+        blk += ew_blocks(k, k);
+      }
+    }
+    B.ops.back().blocks = blk;
+  }
+  if (check) {
+    // D = Q^T F Q: T = Q^T F (A = Q stored K x M), D = T Q (B = Q stored K x N)
+    TableLaunch& g1 = B.new_gemm(1, 1, MAO_K_PC_CHECK);
+    for (int i = 0; i < nm; ++i) {
+      const int k = kof(i);
+      const Split3 Tp = B.planes(side(i).Tp, k, k);
+      MAO_TRY(table_add(g1, B.maps, B.planes(side(i).Qp, k, k), B.planes(side(i).Fp, k, k), k, k, k, 0, 0, nullptr,
+                        &Tp, k, nullptr, 0, 1.f, 0.f, nullptr));
+    }
+    TableLaunch& g2 = B.new_gemm(0, 1, MAO_K_PC_CHECK);
+    for (int i = 0; i < nm; ++i) {
+      const int k = kof(i);
+      MAO_TRY(table_add(g2, B.maps, B.planes(side(i).Tp, k, k), B.planes(side(i).Qp, k, k), k, k, k, 0, 0,
+                        B.wp<float>(side(i).D), nullptr, k, nullptr, 0, 1.f, 0.f, nullptr));
+    }
+    size_t off;
+    CheckJob* J = B.new_jobs<CheckJob>(Op::CHECK, nm, off);
+    for (int i = 0; i < nm; ++i) {
+      J[i].D = B.wp<float>(side(i).D);
+      J[i].flag = B.wp<int>(side(i).flag);
+      J[i].rho = B.wp<float>(side(i).rho);
+      J[i].k = kof(i);
+    }
+    B.ops.back().blocks = nm;
+  }
+  // power step P = F Q (A = F K-major, B = Q stored K x N)
+  {
+    TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_POWER);
+    for (int i = 0; i < nm; ++i) {
+      const int k = kof(i);
+      MAO_TRY(table_add(g, B.maps, B.planes(side(i).Fp, k, k), B.planes(side(i).Qp, k, k), k, k, k, 0, 0,
+                        B.wp<float>(side(i).P), nullptr, k, nullptr, 0, 1.f, 0.f, flagp(i)));
+    }
+  }
+  // keys and argsort
+  {
+    size_t off;
+    SortJob* J = B.new_jobs<SortJob>(Op::KEYS, nm, off);
+    int blk = 0;
+    for (int i = 0; i < nm; ++i) {
+      const int k = kof(i);
+      SortJob& j = J[i];
+      j.Q = Qp(i);
+      j.P = B.wp<float>(side(i).P);
+      j.key = B.wp<double>(side(i).keys);
+      j.perm = B.wp<int>(side(i).perm);
+      j.perm_out = left ? X.mats[G.g0 + i].perm_L : X.mats[G.g0 + i].perm_R;
+      j.flag = flagp(i);
+      j.k = k;
+      j.col_blk_begin = blk;
+      blk += (k + 255) / 256;
+    }
+    B.ops.back().blocks = blk;
+    Op o = B.ops.back();  // the argsort reuses the job array
+    o.kind = Op::ARGSORT;
+    B.ops.push_back(o);
+    B.gemm_of_op.push_back(-1);
+  }
+  // gathered P and its planes
+  {
+    size_t off;
+    GatherJob* J = B.new_jobs<GatherJob>(Op::GATHER, nm, off);
+    int blk = 0;
+    for (int i = 0; i < nm; ++i) {
+      const int k = kof(i);
+      GatherJob& j = J[i];
+      j.src = B.wp<float>(side(i).P);
+      j.dst = B.wp<float>(side(i).Ps);
+      j.dstp = B.wp<__nv_bfloat16>(side(i).Psp);
+      j.pstride = B.pstride(k, k);
+      j.perm = B.wp<int>(side(i).perm);
+      j.flag = flagp(i);
+      j.rows = k;
+      j.cols = k;
+      j.ld = k;
+      j.ldp = ldp_of(k);
+      j.blk_begin = blk;
+      blk += ew_blocks(k, k);
+    }
+    B.ops.back().blocks = blk;
+  }
+  // QR by blocks of 64 columns
+  int maxk = 0;
+  for (int i = 0; i < nm; ++i) maxk = std::max(maxk, kof(i));
+  const int npanels = (maxk + kPanel - 1) / kPanel;
+  for (int pj = 0; pj < npanels; ++pj) {
+    const int c0 = pj * kPanel;
+    std::vector<int> act;
+    for (int i = 0; i < nm; ++i)
+      if (kof(i) > c0) act.push_back(i);
+    auto wdt = [&](int i) { return std::min(kPanel, kof(i) - c0); };
+    // one Cholesky-QR pass on the panel of every active matrix;
+    // target: 0 = in place, 1 = also W's plane set, 2 = the final Q columns and planes
+    auto cholqr = [&](bool first_panel, int target) {
+      std::vector<PanelJob> jl(act.size());
+      int gblk = 0, ablk = 0;
+      for (size_t a = 0; a < act.size(); ++a) {
+        const int i = act[a];
+        const int k = kof(i);
+        PanelJob& j = jl[a];
+        std::memset(&j, 0, sizeof(j));
+        if (first_panel) {
+          j.W = B.wp<float>(side(i).Ps) + c0;
+          j.ld = k;
+        } else {
+          j.W = B.wp<float>(side(i).W);
+          j.ld = kPanel;
+        }
+        if (target == 1) {
+          j.Wp = B.wp<__nv_bfloat16>(side(i).Wp);
+          j.wps = B.pstride(k, kPanel);
+        }
+        if (target == 2) {
+          j.Q = Qp(i) + c0;
+          j.ldq = k;
+          j.Qp = B.wp<__nv_bfloat16>(side(i).Qp) + c0;
+          j.qps = B.pstride(k, k);
+          j.ldqp = ldp_of(k);
+        }
+        j.gram = B.wp<double>(side(i).gram);
+        j.rinv = B.wp<double>(side(i).rinv);
+        j.bad = B.wp<int>(side(i).bad);
+        j.flag = flagp(i);
+        j.rows = k;
+        j.w = wdt(i);
+        j.chunks = (k + kGramRows - 1) / kGramRows;
+        j.blk_begin = gblk;
+        gblk += j.chunks;
+      }
+      size_t off;
+      PanelJob* Jg = B.new_jobs<PanelJob>(Op::GRAM, (int)act.size(), off);
+      for (size_t a = 0; a < act.size(); ++a) Jg[a] = jl[a];
+      B.ops.back().blocks = gblk;
+      PanelJob* Jc = B.new_jobs<PanelJob>(Op::CHOL, (int)act.size(), off);
+      for (size_t a = 0; a < act.size(); ++a) Jc[a] = jl[a];
+      B.ops.back().blocks = (int)act.size();
+      PanelJob* Ja = B.new_jobs<PanelJob>(Op::APPLY, (int)act.size(), off);
+      for (size_t a = 0; a < act.size(); ++a) {
+        jl[a].blk_begin = ablk;
+        ablk += (jl[a].rows + kApplyRows - 1) / kApplyRows;
+        Ja[a] = jl[a];
+      }
+      B.ops.back().blocks = ablk;
+    };
+    // project out the finished columns: C = Q[:, :c0]^T Y ; W = Y - Q[:, :c0] C
+    auto project = [&](bool from_ps) -> mao_status {
+      TableLaunch& gc = B.new_gemm(1, 1, MAO_K_PC_QR);
+      for (int i : act) {
+        const int k = kof(i);
+        const Split3 Y = from_ps ? B.planes(side(i).Psp, k, k) : B.planes(side(i).Wp, k, kPanel);
+        const Split3 C = B.planes(side(i).Cp, k, kPanel);
+        MAO_TRY(table_add(gc, B.maps, B.planes(side(i).Qp, k, k), Y, c0, wdt(i), k, 0, from_ps ? c0 : 0, nullptr,
+                          &C, kPanel, nullptr, 0, 1.f, 0.f, flagp(i)));
+      }
+      TableLaunch& gw = B.new_gemm(0, 1, MAO_K_PC_QR);
+      for (int i : act) {
+        const int k = kof(i);
+        const float* aux = from_ps ? B.wp<float>(side(i).Ps) + c0 : B.wp<float>(side(i).W);
+        MAO_TRY(table_add(gw, B.maps, B.planes(side(i).Qp, k, k), B.planes(side(i).Cp, k, kPanel), k, wdt(i), c0, 0,
+                          0, B.wp<float>(side(i).W), nullptr, kPanel, aux, from_ps ? k : kPanel, -1.f, 1.f,
+                          flagp(i)));
+      }
+      return MAO_OK;
+    };
+    if (pj == 0) {
+      cholqr(true, 0);
+      cholqr(true, 2);
+    } else {
+      MAO_TRY(project(true));
+      cholqr(false, 0);
+      cholqr(false, 1);
+      MAO_TRY(project(false));
+      cholqr(false, 2);
+    }
+  }
+  return MAO_OK;
+}
+
+mao_status build_group(Builder& B, GroupPlan& G) {
+  const Ctx& X = B.X;
+  const int nm = G.g1 - G.g0;
+  const bool foam = X.foam;
+  auto A = [&](int i) -> const PcMat& { return X.mats[G.g0 + i]; };
+  B.zero_flag_off = B.arena.take(16, 16);
+  std::memset(B.arena.hptr<int>(B.zero_flag_off), 0, 16);
+
+  // momentum + planes of G and M
+  {
+    size_t off;
+    EwJob* J = B.new_jobs<EwJob>(Op::EW, nm, off);
+    int blk = 0;
+    double bytes = 0;
+    for (int i = 0; i < nm; ++i) {
+      const PcMat& a = A(i);
+      EwJob& j = J[i];
+      j.a = a.G;
+      j.a_bf16 = a.g_bf16;
+      j.f0 = a.M;
+      j.pa = B.wp<__nv_bfloat16>(G.mb[i].Gp);
+      j.pb = B.wp<__nv_bfloat16>(G.mb[i].Mp);
+      j.pstride = B.pstride(a.m, a.n);
+      j.rows = a.m;
+      j.cols = a.n;
+      j.lda = a.n;
+      j.ldf = a.n;
+      j.ldp = ldp_of(a.n);
+      j.blk_begin = blk;
+      blk += ew_blocks(a.m, a.n);
+      bytes += (double)a.m * a.n * ((a.g_bf16 ? 2 : 4) + 8 + 12);
+    }
+    B.ops.back().blocks = blk;
+    B.ops.back().bytes = bytes;
+  }
+  // factor EMAs
+  if (!foam) {
+    TableLaunch& g = B.new_gemm(0, 0, MAO_K_PC_FACTOR);
+    for (int i = 0; i < nm; ++i) {
+      const PcMat& a = A(i);
+      const Split3 Gs = B.planes(G.mb[i].Gp, a.m, a.n);
+      MAO_TRY(table_add(g, B.maps, Gs, Gs, a.m, a.m, a.n, 0, 0, a.L, nullptr, a.m, a.L, a.m, 1.f - X.b2, X.b2,
+                        nullptr));
+    }
+  }
+  {
+    TableLaunch& g = B.new_gemm(1, 1, MAO_K_PC_FACTOR);
+    for (int i = 0; i < nm; ++i) {
+      const PcMat& a = A(i);
+      const Split3 Gs = B.planes(G.mb[i].Gp, a.m, a.n);
+      MAO_TRY(table_add(g, B.maps, Gs, Gs, a.n, a.n, a.m, 0, 0, a.R, nullptr, a.n, a.R, a.n, 1.f - X.b2, X.b2,
+                        nullptr));
+    }
+  }
+  // refresh, or plain planes of the bases
+  if (X.mode != 0) {
+    if (!foam) MAO_TRY(build_refresh_side(B, G, true));
+    MAO_TRY(build_refresh_side(B, G, false));
+  } else {
+    size_t off;
+    const int per = foam ? 1 : 2;
+    EwJob* J = B.new_jobs<EwJob>(Op::SPLIT, per * nm, off);
+    int blk = 0;
+    for (int i = 0; i < nm; ++i) {
+      const PcMat& a = A(i);
+      for (int s = 0; s < per; ++s) {
+        const bool right = foam || s == 1;
+        const int k = right ? a.n : a.m;
+        EwJob& j = J[per * i + s];
+        j.a = right ? a.QR : a.QL;
+        j.pa = B.wp<__nv_bfloat16>(right ? G.mb[i].R.Qp : G.mb[i].L.Qp);
+        j.pstride = B.pstride(k, k);
+        j.rows = k;
+        j.cols = k;
+        j.lda = k;
+        j.ldp = ldp_of(k);
+        j.blk_begin = blk;
+        blk += ew_blocks(k, k);
+      }
+    }
+    B.ops.back().blocks = blk;
+    // identity permutations for the callers that asked for them
+    bool any = false;
+    for (int i = 0; i < nm; ++i) any = any || A(i).perm_R || (!foam && A(i).perm_L);
+    if (any) {
+      size_t off2;
+      SortJob* S = B.new_jobs<SortJob>(Op::ARGSORT, per * nm, off2);
+      int blk2 = 0;
+      int* zero = B.arena.dev ? B.arena.dptr<int>(B.zero_flag_off) : reinterpret_cast<int*>(16);
+      for (int i = 0; i < nm; ++i)
+        for (int s = 0; s < per; ++s) {
+          const bool right = foam || s == 1;
+          SortJob& j = S[per * i + s];
+          j.perm_out = right ? A(i).perm_R : A(i).perm_L;
+          j.flag = zero;
+          j.k = right ? A(i).n : A(i).m;
+          j.col_blk_begin = blk2;
+          blk2 += (j.k + 255) / 256;
+        }
+      B.ops.back().blocks = blk2;
+    }
+  }
+
+  if (!foam) {
+    // V follows the refresh permutations
+    if (X.mode != 0) {
+      size_t off;
+      VPermJob* J = B.new_jobs<VPermJob>(Op::VPERM, nm, off);
+      int blk = 0;
+      for (int i = 0; i < nm; ++i) {
+        const PcMat& a = A(i);
+        VPermJob& j = J[i];
+        j.V = a.V;
+        j.dst = B.wp<float>(G.mb[i].Vtmp);
+        j.pl = B.wp<int>(G.mb[i].L.perm);
+        j.pr = B.wp<int>(G.mb[i].R.perm);
+        j.fl = X.mode == 2 ? B.wp<int>(G.mb[i].L.flag) : nullptr;
+        j.fr = X.mode == 2 ? B.wp<int>(G.mb[i].R.flag) : nullptr;
+        j.m = a.m;
+        j.n = a.n;
+        j.blk_begin = blk;
+        blk += ew_blocks(a.m, a.n);
+      }
+      B.ops.back().blocks = blk;
+    }
+    // T1 = Q_L^T {G, M}  (A = Q_L stored K x M, B = G / M stored K x N)
+    {
+      TableLaunch& g = B.new_gemm(1, 1, MAO_K_PC_ROTATE);
+      for (int i = 0; i < nm; ++i) {
+        const PcMat& a = A(i);
+        const Split3 Ql = B.planes(G.mb[i].L.Qp, a.m, a.m);
+        const Split3 T1G = B.planes(G.mb[i].T1G, a.m, a.n), T1M = B.planes(G.mb[i].T1M, a.m, a.n);
+        MAO_TRY(table_add(g, B.maps, Ql, B.planes(G.mb[i].Gp, a.m, a.n), a.m, a.n, a.m, 0, 0, nullptr, &T1G, a.n,
+                          nullptr, 0, 1.f, 0.f, nullptr));
+        MAO_TRY(table_add(g, B.maps, Ql, B.planes(G.mb[i].Mp, a.m, a.n), a.m, a.n, a.m, 0, 0, nullptr, &T1M, a.n,
+                          nullptr, 0, 1.f, 0.f, nullptr));
+      }
+    }
+    // Gh, Mh = T1 Q_R (fp32)
+    {
+      TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_ROTATE);
+      for (int i = 0; i < nm; ++i) {
+        const PcMat& a = A(i);
+        const Split3 Qr = B.planes(G.mb[i].R.Qp, a.n, a.n);
+        MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].T1G, a.m, a.n), Qr, a.m, a.n, a.n, 0, 0,
+                          B.wp<float>(G.mb[i].Gh), nullptr, a.n, nullptr, 0, 1.f, 0.f, nullptr));
+        MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].T1M, a.m, a.n), Qr, a.m, a.n, a.n, 0, 0,
+                          B.wp<float>(G.mb[i].Mh), nullptr, a.n, nullptr, 0, 1.f, 0.f, nullptr));
+      }
+    }
+    // Adam: V and the planes of N (into T1G's planes)
+    {
+      size_t off;
+      EwJob* J = B.new_jobs<EwJob>(Op::ADAM, nm, off);
+      int blk = 0;
+      double bytes = 0;
+      for (int i = 0; i < nm; ++i) {
+        const PcMat& a = A(i);
+        EwJob& j = J[i];
+        j.a = B.wp<float>(G.mb[i].Gh);
+        j.b = B.wp<float>(G.mb[i].Mh);
+        j.f0 = a.V;
+        j.f1 = X.mode != 0 ? B.wp<float>(G.mb[i].Vtmp) : nullptr;
+        j.pa = B.wp<__nv_bfloat16>(G.mb[i].T1G);
+        j.pstride = B.pstride(a.m, a.n);
+        j.rows = a.m;
+        j.cols = a.n;
+        j.lda = a.n;
+        j.ldb = a.n;
+        j.ldf = a.n;
+        j.ldp = ldp_of(a.n);
+        j.blk_begin = blk;
+        blk += ew_blocks(a.m, a.n);
+        bytes += (double)a.m * a.n * (4 + 4 + 8 + 6);
+      }
+      B.ops.back().blocks = blk;
+      B.ops.back().bytes = bytes;
+    }
+    // T2 = Q_L N -> the (free) M planes
+    {
+      TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_ROTATE);
+      for (int i = 0; i < nm; ++i) {
+        const PcMat& a = A(i);
+        const Split3 T2 = B.planes(G.mb[i].Mp, a.m, a.n);
+        MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].L.Qp, a.m, a.m), B.planes(G.mb[i].T1G, a.m, a.n), a.m, a.n,
+                          a.m, 0, 0, nullptr, &T2, a.n, nullptr, 0, 1.f, 0.f, nullptr));
+      }
+    }
+    // U = T2 Q_R^T ; W <- W (1 - lr wd) - lr U
+    {
+      TableLaunch& g = B.new_gemm(0, 0, MAO_K_PC_UPDATE);
+      for (int i = 0; i < nm; ++i) {
+        const PcMat& a = A(i);
+        MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].Mp, a.m, a.n), B.planes(G.mb[i].R.Qp, a.n, a.n), a.m, a.n,
+                          a.n, 0, 0, a.W, nullptr, a.n, a.W, a.n, -X.lr, 1.f - X.lr * X.wd, nullptr));
+      }
+    }
+  } else {
+    // Gr, Mr = {G, M} Q_R  (A K-major, B = Q_R stored K x N)
+    {
+      TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_ROTATE);
+      for (int i = 0; i < nm; ++i) {
+        const PcMat& a = A(i);
+        const Split3 Qr = B.planes(G.mb[i].R.Qp, a.n, a.n);
+        MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].Gp, a.m, a.n), Qr, a.m, a.n, a.n, 0, 0,
+                          B.wp<float>(G.mb[i].Gr), nullptr, a.n, nullptr, 0, 1.f, 0.f, nullptr));
+        MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].Mp, a.m, a.n), Qr, a.m, a.n, a.n, 0, 0,
+                          B.wp<float>(G.mb[i].Mr), nullptr, a.n, nullptr, 0, 1.f, 0.f, nullptr));
+      }
+    }
+    // row/col partials of Gr^2, r/c EMAs and tau, N
+    {
+      size_t off;
+      RcJob* J = B.new_jobs<RcJob>(Op::RC, nm, off);
+      int blk = 0;
+      for (int i = 0; i < nm; ++i) {
+        const PcMat& a = A(i);
+        RcJob& j = J[i];
+        j.Gr = B.wp<float>(G.mb[i].Gr);
+        j.rowpart = B.wp<float>(G.mb[i].rowpart);
+        j.colpart = B.wp<float>(G.mb[i].colpart);
+        j.m = a.m;
+        j.n = a.n;
+        j.tiles_c = (a.n + 63) / 64;
+        j.tiles_r = (a.m + 63) / 64;
+        j.blk_begin = blk;
+        blk += j.tiles_c * j.tiles_r;
+      }
+      B.ops.back().blocks = blk;
+    }
+    {
+      size_t off;
+      TauJob* J = B.new_jobs<TauJob>(Op::TAU, nm, off);
+      for (int i = 0; i < nm; ++i) {
+        const PcMat& a = A(i);
+        TauJob& j = J[i];
+        j.r = a.r;
+        j.c = a.c;
+        j.rowpart = B.wp<float>(G.mb[i].rowpart);
+        j.colpart = B.wp<float>(G.mb[i].colpart);
+        j.R = a.R;
+        j.perm = X.mode != 0 ? B.wp<int>(G.mb[i].R.perm) : nullptr;
+        j.flag = X.mode == 2 ? B.wp<int>(G.mb[i].R.flag) : nullptr;
+        j.c_tmp = B.wp<float>(G.mb[i].ctmp);
+        j.tau = B.wp<float>(G.mb[i].tau);
+        j.m = a.m;
+        j.n = a.n;
+        j.tiles_c = (a.n + 63) / 64;
+        j.tiles_r = (a.m + 63) / 64;
+      }
+      B.ops.back().blocks = nm;
+    }
+    {
+      size_t off;
+      EwJob* J = B.new_jobs<EwJob>(Op::FOAMN, nm, off);
+      int blk = 0;
+      for (int i = 0; i < nm; ++i) {
+        const PcMat& a = A(i);
+        EwJob& j = J[i];
+        j.a = B.wp<float>(G.mb[i].Mr);
+        j.b = B.wp<float>(G.mb[i].tau);
+        j.vr = a.r;
+        j.vc = a.c;
+        j.pa = B.wp<__nv_bfloat16>(G.mb[i].Gp);
+        j.pstride = B.pstride(a.m, a.n);
+        j.rows = a.m;
+        j.cols = a.n;
+        j.lda = a.n;
+        j.ldp = ldp_of(a.n);
+        j.blk_begin = blk;
+        blk += ew_blocks(a.m, a.n);
+      }
+      B.ops.back().blocks = blk;
+    }
+    // U = N Q_R^T ; W update
+    {
+      TableLaunch& g = B.new_gemm(0, 0, MAO_K_PC_UPDATE);
+      for (int i = 0; i < nm; ++i) {
+        const PcMat& a = A(i);
+        MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].Gp, a.m, a.n), B.planes(G.mb[i].R.Qp, a.n, a.n), a.m, a.n,
+                          a.n, 0, 0, a.W, nullptr, a.n, a.W, a.n, -X.lr, 1.f - X.lr * X.wd, nullptr));
+      }
+    }
+  }
+  return MAO_OK;
+}
+
+struct BuiltGroup {
+  size_t maps_off = 0;
+  std::vector<StagedLaunch> staged;
+};
+
+mao_status finish_build(Builder& B, BuiltGroup& out) {
+  // maps after all problems are known
+  out.maps_off = B.arena.take(sizeof(CUtensorMap) * std::max<size_t>(B.maps.keys.size(), 1), 64);
+  if (B.ws) {
+    MAO_TRY(B.maps.encode_all());
+    std::memcpy(B.arena.host.data() + out.maps_off, B.maps.maps.data(), sizeof(CUtensorMap) * B.maps.maps.size());
+  }
+  out.staged.clear();
+  for (const TableLaunch& L : B.gemms) out.staged.push_back(table_stage(B.arena, L, out.maps_off));
+  return MAO_OK;
+}
+
+mao_status run_ops(Builder& B, const BuiltGroup& bg, DevStatus* status, cudaStream_t s) {
+  const Ctx& X = B.X;
+  const float bc1 = (float)(1.0 - std::pow((double)X.b1, (double)X.t));
+  const float bc2 = (float)(1.0 - std::pow((double)X.b2, (double)X.t));
+  for (size_t o = 0; o < B.ops.size(); ++o) {
+    const Op& op = B.ops[o];
+    if (op.kind == Op::GEMM) {
+      MAO_TRY(table_launch(B.arena, bg.staged[B.gemm_of_op[o]], status, s));
+      continue;
+    }
+    if (op.blocks <= 0) continue;
+    const int n = op.njobs;
+    switch (op.kind) {
+      case Op::EW: {
+        LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, op.bytes);
+        pc_momentum_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<EwJob>(op.jobs), n, X.b1);
+        break;
+      }
+      case Op::SPLIT: {
+        LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, 0.0);
+        pc_split_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<EwJob>(op.jobs), n);
+        break;
+      }
+      case Op::ADAM: {
+        LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, op.bytes);
+        soap_adam_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<EwJob>(op.jobs), n, X.b2, 1.f / bc1, 1.f / bc2, X.eps);
+        break;
+      }
+      case Op::KEYS: {
+        LaunchScope ls(s, MAO_K_PC_SORT, 0.0, 0.0);
+        if (X.rf.sort)
+          pc_keys_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<SortJob>(op.jobs), n);
+        else
+          pc_identity_keys_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<SortJob>(op.jobs), n);
+        break;
+      }
+      case Op::ARGSORT: {
+        LaunchScope ls(s, MAO_K_PC_SORT, 0.0, 0.0);
+        pc_argsort_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<SortJob>(op.jobs), n);
+        break;
+      }
+      case Op::GATHER: {
+        LaunchScope ls(s, MAO_K_PC_SORT, 0.0, 0.0);
+        pc_gather_cols_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<GatherJob>(op.jobs), n);
+        break;
+      }
+      case Op::VPERM: {
+        LaunchScope ls(s, MAO_K_PC_SORT, 0.0, 0.0);
+        soap_vperm_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<VPermJob>(op.jobs), n);
+        break;
+      }
+      case Op::GRAM: {
+        LaunchScope ls(s, MAO_K_PC_QR, 0.0, 0.0);
+        qr_gram_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<PanelJob>(op.jobs), n);
+        break;
+      }
+      case Op::CHOL: {
+        LaunchScope ls(s, MAO_K_PC_QR, 0.0, 0.0);
+        qr_chol_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<PanelJob>(op.jobs), n);
+        break;
+      }
+      case Op::APPLY: {
+        LaunchScope ls(s, MAO_K_PC_QR, 0.0, 0.0);
+        qr_apply_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<PanelJob>(op.jobs), n);
+        break;
+      }
+      case Op::RC: {
+        LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, 0.0);
+        foam_rc_partial_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<RcJob>(op.jobs), n);
+        break;
+      }
+      case Op::TAU: {
+        LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, 0.0);
+        foam_tau_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<TauJob>(op.jobs), X.b2, 1.f / bc2, X.raw_trace);
+        break;
+      }
+      case Op::FOAMN: {
+        LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, 0.0);
+        foam_n_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<EwJob>(op.jobs), n, 1.f / bc1, 1.f / bc2, X.eps);
+        break;
+      }
+      case Op::CHECK: {
+        LaunchScope ls(s, MAO_K_PC_CHECK, 0.0, 0.0);
+        pc_check_kernel<<<n, 256, 0, s>>>(B.arena.dptr<CheckJob>(op.jobs), X.rf.tol);
+        break;
+      }
+      default:
+        return MAO_ERR_INVALID_ARG;
+    }
+    MAO_CUDA_TRY(cudaGetLastError());
+  }
+  return MAO_OK;
+}
+
+// Workspace = status | scratch (max over groups) | arena (max over groups)
+struct Layout {
+  size_t scratch_off = 0, scratch = 0, arena_off = 0, arena = 0, total = 0;
+};
+
+mao_status layout_for(const Ctx& X, std::vector<GroupPlan>& groups, Layout& L) {
+  make_groups(X, groups);
+  L.scratch_off = align_up(kStatusBytes, 256);
+  for (GroupPlan& g : groups) {
+    plan_group_scratch(X, g, L.scratch_off);
+    L.scratch = std::max(L.scratch, g.scratch);
+  }
+  L.arena_off = align_up(L.scratch_off + L.scratch, 256);
+  for (GroupPlan& g : groups) {
+    Builder B(X, nullptr);
+    MAO_TRY(build_group(B, g));
+    BuiltGroup bg;
+    MAO_TRY(finish_build(B, bg));
+    L.arena = std::max(L.arena, B.arena.host.size());
+  }
+  L.total = align_up(L.arena_off + L.arena + 64, 256);
+  return MAO_OK;
+}
+
+mao_status run_step(const Ctx& X, void* workspace, size_t ws_bytes, mao_stats* stats, cudaStream_t s) {
+  std::vector<GroupPlan> groups;
+  Layout L;
+  MAO_TRY(layout_for(X, groups, L));
+  if (workspace == nullptr || ws_bytes < L.total) return MAO_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MAO_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  MAO_TRY(device_info(&dev));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DevStatus* status = reinterpret_cast<DevStatus*>(ws);
+  MAO_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(DevStatus), s));
+  for (GroupPlan& g : groups) {
+    Builder B(X, ws);
+    B.arena.dev = ws + L.arena_off;
+    MAO_TRY(build_group(B, g));
+    BuiltGroup bg;
+    MAO_TRY(finish_build(B, bg));
+    if (B.arena.host.size() > L.arena) return MAO_ERR_WORKSPACE;
+    // refresh flags (adaptive) and failure counters start at zero
+    for (int i = 0; i < g.g1 - g.g0; ++i) {
+      for (int side = 0; side < 2; ++side) {
+        if (X.foam && side == 0) continue;
+        const SideBuf& sb = side == 0 ? g.mb[i].L : g.mb[i].R;
+        MAO_CUDA_TRY(cudaMemsetAsync(ws + sb.flag, 0, 48, s));  // flag, rho, bad
+      }
+    }
+    MAO_CUDA_TRY(cudaMemcpyAsync(B.arena.dev, B.arena.host.data(), B.arena.host.size(), cudaMemcpyHostToDevice, s));
+    MAO_TRY(run_ops(B, bg, status, s));
+    if (stats) {
+      for (int i = 0; i < g.g1 - g.g0; ++i) {
+        mao_stats* st = stats + g.g0 + i;
+        const SideBuf& R = g.mb[i].R;
+        const SideBuf* Lb = X.foam ? nullptr : &g.mb[i].L;
+        if (X.mode == 2) {
+          pc_stats_kernel<<<1, 32, 0, s>>>(st, reinterpret_cast<const int*>(ws + R.flag),
+                                          Lb ? reinterpret_cast<const int*>(ws + Lb->flag) : nullptr,
+                                          reinterpret_cast<const float*>(ws + R.rho), -1);
+        } else {
+          pc_stats_kernel<<<1, 32, 0, s>>>(st, nullptr, nullptr, nullptr, X.mode == 1 ? (X.foam ? 1 : 3) : 0);
+        }
+        MAO_CUDA_TRY(cudaGetLastError());
+      }
+    }
+  }
+  return MAO_OK;
+}
+
+// ------------------------------------------------------------------ ABI helpers
+mao_status soap_ctx(const mao_soap_mat* mats, int32_t count, const mao_soap_params* p, std::vector<PcMat>& v,
+                    Ctx& X, bool ptrs) {
+  if (p == nullptr || count < 0 || (count > 0 && mats == nullptr)) return MAO_ERR_INVALID_ARG;
+  MAO_TRY(check_refresh(p->refresh));
+  MAO_TRY(check_hyper(p->beta1, p->beta2, p->eps, p->lr, p->wd, p->t));
+  v.resize(count);
+  for (int i = 0; i < count; ++i) {
+    const mao_soap_mat& a = mats[i];
+    MAO_TRY(check_mat(a.m, a.n, a.g_dtype));
+    if (ptrs) {
+      const void* req[] = {a.W, a.G, a.M, a.V, a.L, a.R, a.QL, a.QR};
+      for (const void* q : req) {
+        if (q == nullptr) return MAO_ERR_INVALID_ARG;
+        if (!aligned16(q)) return MAO_ERR_ALIGN;
+      }
+      if ((a.perm_L && !aligned16(a.perm_L)) || (a.perm_R && !aligned16(a.perm_R))) return MAO_ERR_ALIGN;
+    }
+    v[i] = PcMat{a.m, a.n, a.W, a.G, a.g_dtype == MAO_BF16, a.M, a.V, a.L, a.R, a.QL, a.QR, a.perm_L, a.perm_R,
+                 nullptr, nullptr};
+  }
+  X = Ctx{false, v.data(), count, p->beta1, p->beta2, p->eps, p->lr, p->wd, p->t, p->refresh, 0,
+          host_refresh_mode(p->refresh, p->t)};
+  return MAO_OK;
+}
+
+mao_status foam_ctx(const mao_foam_mat* mats, int32_t count, const mao_foam_params* p, std::vector<PcMat>& v,
+                    Ctx& X, bool ptrs) {
+  if (p == nullptr || count < 0 || (count > 0 && mats == nullptr)) return MAO_ERR_INVALID_ARG;
+  MAO_TRY(check_refresh(p->refresh));
+  MAO_TRY(check_hyper(p->beta1, p->beta2, p->eps, p->lr, p->wd, p->t));
+  if (p->tau_raw_trace != 0 && p->tau_raw_trace != 1) return MAO_ERR_INVALID_ARG;
+  v.resize(count);
+  for (int i = 0; i < count; ++i) {
+    const mao_foam_mat& a = mats[i];
+    MAO_TRY(check_mat(a.m, a.n, a.g_dtype));
+    if (ptrs) {
+      const void* req[] = {a.W, a.G, a.M, a.r, a.c, a.R, a.QR};
+      for (const void* q : req) {
+        if (q == nullptr) return MAO_ERR_INVALID_ARG;
+        if (!aligned16(q)) return MAO_ERR_ALIGN;
+      }
+      if (a.perm_R && !aligned16(a.perm_R)) return MAO_ERR_ALIGN;
+    }
+    v[i] = PcMat{a.m, a.n, a.W, a.G, a.g_dtype == MAO_BF16, a.M, nullptr, nullptr, a.R, nullptr, a.QR, nullptr,
+                 a.perm_R, a.r, a.c};
+  }
+  X = Ctx{true, v.data(), count, p->beta1, p->beta2, p->eps, p->lr, p->wd, p->t, p->refresh, p->tau_raw_trace,
+          host_refresh_mode(p->refresh, p->t)};
   return MAO_OK;
 }
 
@@ -36,43 +998,46 @@ mao_status check_mat(int m, int n, const void* G, int g_dtype) {
 
 extern "C" mao_status mao_soap_workspace_size(const mao_soap_mat* mats, int32_t count, const mao_soap_params* p,
                                               size_t* bytes) {
-  if (bytes == nullptr || p == nullptr || count < 0 || (count > 0 && mats == nullptr)) return MAO_ERR_INVALID_ARG;
-  MAO_TRY(check_refresh(p->refresh));
-  MAO_TRY(check_hyper(p->beta1, p->beta2, p->eps, p->lr, p->wd, p->t));
-  for (int i = 0; i < count; ++i) MAO_TRY(check_mat(mats[i].m, mats[i].n, mats[i].G, mats[i].g_dtype));
-  *bytes = kStatusBytes;
+  if (bytes == nullptr) return MAO_ERR_INVALID_ARG;
+  std::vector<PcMat> v;
+  Ctx X;
+  MAO_TRY(soap_ctx(mats, count, p, v, X, false));
+  std::vector<GroupPlan> groups;
+  Layout L;
+  MAO_TRY(layout_for(X, groups, L));
+  *bytes = L.total;
   return MAO_OK;
 }
 
 extern "C" mao_status mao_soap_step(const mao_soap_mat* mats, int32_t count, const mao_soap_params* p,
                                    void* workspace, size_t ws_bytes, mao_stats* stats, mao_stream_t stream) {
-  size_t need = 0;
-  MAO_TRY(mao_soap_workspace_size(mats, count, p, &need));
-  (void)workspace;
-  (void)ws_bytes;
-  (void)stats;
-  (void)stream;
-  return MAO_ERR_UNSUPPORTED;
+  std::vector<PcMat> v;
+  Ctx X;
+  MAO_TRY(soap_ctx(mats, count, p, v, X, true));
+  if (count == 0) return MAO_OK;
+  if (stats != nullptr && !aligned16(stats)) return MAO_ERR_ALIGN;
+  return run_step(X, workspace, ws_bytes, stats, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" mao_status mao_foam_workspace_size(const mao_foam_mat* mats, int32_t count, const mao_foam_params* p,
                                               size_t* bytes) {
-  if (bytes == nullptr || p == nullptr || count < 0 || (count > 0 && mats == nullptr)) return MAO_ERR_INVALID_ARG;
-  MAO_TRY(check_refresh(p->refresh));
-  MAO_TRY(check_hyper(p->beta1, p->beta2, p->eps, p->lr, p->wd, p->t));
-  if (p->tau_raw_trace != 0 && p->tau_raw_trace != 1) return MAO_ERR_INVALID_ARG;
-  for (int i = 0; i < count; ++i) MAO_TRY(check_mat(mats[i].m, mats[i].n, mats[i].G, mats[i].g_dtype));
-  *bytes = kStatusBytes;
+  if (bytes == nullptr) return MAO_ERR_INVALID_ARG;
+  std::vector<PcMat> v;
+  Ctx X;
+  MAO_TRY(foam_ctx(mats, count, p, v, X, false));
+  std::vector<GroupPlan> groups;
+  Layout L;
+  MAO_TRY(layout_for(X, groups, L));
+  *bytes = L.total;
   return MAO_OK;
 }
 
 extern "C" mao_status mao_foam_step(const mao_foam_mat* mats, int32_t count, const mao_foam_params* p,
                                    void* workspace, size_t ws_bytes, mao_stats* stats, mao_stream_t stream) {
-  size_t need = 0;
-  MAO_TRY(mao_foam_workspace_size(mats, count, p, &need));
-  (void)workspace;
-  (void)ws_bytes;
-  (void)stats;
-  (void)stream;
-  return MAO_ERR_UNSUPPORTED;
+  std::vector<PcMat> v;
+  Ctx X;
+  MAO_TRY(foam_ctx(mats, count, p, v, X, true));
+  if (count == 0) return MAO_OK;
+  if (stats != nullptr && !aligned16(stats)) return MAO_ERR_ALIGN;
+  return run_step(X, workspace, ws_bytes, stats, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -173,17 +173,22 @@ def sort_perm(keys):
     return np.argsort(-keys, kind="stable").astype(np.int32)
 
 
-def refresh_basis(F, Q, sort: bool, dtype=np.float64):
+def refresh_basis(F, Q, sort: bool, dtype=np.float64, perm=None):
     """One eigenbasis refresh of the factor F from the current basis Q.
 
     [SMB-review] §3-2 (4): refresh the basis from the updated factor, then QR.
     Reading: optional stable descending sort of Q's columns by diag(Q^T F Q),
     then one power step P = F Q and Q <- qr(P) (positive diagonal).
     Returns (Q_new, perm) where perm[i] is the old column placed at i.
+    `perm`, when given, replaces the sort (replay of an ordering decided
+    elsewhere, e.g. at near-equal keys; tests only).
     """
     F, Q = _w(F, dtype), _w(Q, dtype)
     k = Q.shape[1]
-    perm = sort_perm(rayleigh_keys(F, Q)) if sort else np.arange(k, dtype=np.int32)
+    if perm is not None:
+        perm = np.asarray(perm, dtype=np.int32)
+    else:
+        perm = sort_perm(rayleigh_keys(F, Q)) if sort else np.arange(k, dtype=np.int32)
     Qp = Q[:, perm]
     P = F @ Qp
     return qr_positive(P, dtype), perm
@@ -261,7 +266,7 @@ class SoapResult:
 def soap_step(W, G, state: SoapState, *, t: int, beta1: float, beta2: float,
               eps: float, lr: float, wd: float = 0.0, refresh_kind: int = REFRESH_EVERY_K,
               k: int = 1, pf: int = 10, tol: float = 0.1, sort: bool = True,
-              dtype=np.float64) -> SoapResult:
+              dtype=np.float64, force_perm_L=None, force_perm_R=None) -> SoapResult:
     """One two-sided SOAP step with the real-time eigenbasis refresh.
 
     Order ([SMB-review] §3-2 (4)): the current gradient enters the factors first,
@@ -289,10 +294,10 @@ def soap_step(W, G, state: SoapState, *, t: int, beta1: float, beta2: float,
     permR = np.arange(n, dtype=np.int32)
     # S3 + S4 (V follows the permutation of its basis; no re-projection)
     if refL:
-        s.QL, permL = refresh_basis(s.L, s.QL, sort, dtype)
+        s.QL, permL = refresh_basis(s.L, s.QL, sort, dtype, force_perm_L)
         s.V = s.V[permL, :]
     if refR:
-        s.QR, permR = refresh_basis(s.R, s.QR, sort, dtype)
+        s.QR, permR = refresh_basis(s.R, s.QR, sort, dtype, force_perm_R)
         s.V = s.V[:, permR]
     # S5
     s.M = beta1 * s.M + (1.0 - beta1) * G
@@ -361,7 +366,7 @@ def foam_tau(R, r, c, t: int, beta2: float, raw_trace: bool = False) -> float:
 def foam_step(W, G, state: FoamState, *, t: int, beta1: float, beta2: float, eps: float,
               lr: float, wd: float = 0.0, refresh_kind: int = REFRESH_ADAPTIVE, k: int = 1,
               pf: int = 10, tol: float = 0.1, sort: bool = True,
-              raw_trace: bool = False, dtype=np.float64) -> FoamResult:
+              raw_trace: bool = False, dtype=np.float64, force_perm=None) -> FoamResult:
     """One FOAM step (input-only preconditioning, factored Adam moment).
 
     [FOAM-review] §1, §3:
@@ -383,7 +388,7 @@ def foam_step(W, G, state: FoamState, *, t: int, beta1: float, beta2: float, eps
     perm = np.arange(n, dtype=np.int32)
     # F3
     if ref:
-        s.QR, perm = refresh_basis(s.R, s.QR, sort, dtype)
+        s.QR, perm = refresh_basis(s.R, s.QR, sort, dtype, force_perm)
         s.c = s.c[perm]
     # F4
     s.M = beta1 * s.M + (1.0 - beta1) * G

@@ -198,3 +198,19 @@ def test_every_k_schedule_and_v_permutation():
     assert np.array_equal(res.perm_L, perm)
     # G = 0: V' = b2 * V[perm_L][:, perm_R]
     assert np.allclose(res.state.V, 0.9 * st.V[perm][:, res.perm_R], atol=1e-15)
+
+
+def test_forced_permutation_replays_the_sort():
+    """Handing the sort's own permutation back reproduces the step exactly; another
+    permutation changes the basis (so a replayed decision is really used)."""
+    rng = np.random.default_rng(21)
+    m, n = 5, 4
+    st = O.SoapState.init(m, n)
+    G = rng.standard_normal((m, n))
+    a = O.soap_step(np.zeros((m, n)), G, st, t=1, beta1=0.9, beta2=0.9, eps=1e-8, lr=1.0)
+    b = O.soap_step(np.zeros((m, n)), G, st, t=1, beta1=0.9, beta2=0.9, eps=1e-8, lr=1.0,
+                    force_perm_L=a.perm_L, force_perm_R=a.perm_R)
+    assert np.array_equal(a.W, b.W) and np.array_equal(a.state.QL, b.state.QL)
+    c = O.soap_step(np.zeros((m, n)), G, st, t=1, beta1=0.9, beta2=0.9, eps=1e-8, lr=1.0,
+                    force_perm_L=a.perm_L[::-1].copy(), force_perm_R=a.perm_R)
+    assert not np.allclose(c.state.QL, a.state.QL)
