@@ -30,11 +30,15 @@
 // Operand kinds:
 //   BF16    kind::f16, bf16 operands, fp32 accumulate, BK = 64 (128 B rows).
 //   SPLIT3  fp32-faithful product on the bf16 tensor cores: each fp32 operand is
-//           held as three bf16 planes x = x0 + x1 + x2 (24 significant bits), and
-//           the six products whose size reaches the fp32 unit roundoff,
-//           x1y1 + x0y2 + x2y0 + x0y1 + x1y0 + x0y0 (smallest first), accumulate
-//           in one fp32 TMEM accumulator.  Same MMA count per K as a three-pass
-//           tf32 scheme, but with fp32-level accuracy.
+//           held as three bf16 planes x = x0 + x1 + x2 (24 significant bits).  The
+//           main product x0 y0 accumulates in one fp32 TMEM accumulator and the
+//           five cross products whose size reaches the fp32 unit roundoff
+//           (x1y1, x0y2, x2y0, x0y1, x1y0) in a second one, so the large running
+//           sum is rounded once per k-step only.  The tensor core's accumulation
+//           truncates, so its error grows with every add: TMEM accumulates 256 of
+//           K at a time and the epilogue warps fold those partial sums (main +
+//           correction) into fp32 registers with round-to-nearest.  Same MMA count
+//           per K as a three-pass tf32 scheme, with fp32-level accuracy.
 // Operand majors: K-major (rows of the operand run along K) or MN-major
 // (rows run along M/N, i.e. the row-major matrix is K x MN).
 #pragma once
@@ -118,7 +122,9 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = PLANES * (A_TILE + B_TILE);
   static constexpr int STAGES = (KIND == OP_BF16) ? 4 : 2;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
-  static constexpr int TMEM_COLS = 2 * BN;  // two accumulators
+  static constexpr int ACC_COLS = (KIND == OP_BF16) ? BN : 2 * BN;  // main (+ correction) accumulator
+  static constexpr int KCH = 4;  // SPLIT3: k-blocks (4 x 64 = 256 of K) per TMEM accumulation item
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;                   // double-buffered
   static constexpr uint32_t IDESC = make_idesc(1u, A_MN, B_MN, BM, BN);
   static constexpr int THREADS = 192;
 };
@@ -477,49 +483,62 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
+      // One accumulation item per (tile, K-chunk): SPLIT3 accumulates KCH k-blocks
+      // per item (the epilogue folds the items in fp32 registers), bf16 the whole K.
       int it = 0, used = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileInfo t = src.decode(tile, BM, BN);
         if (!t.valid) continue;
         const int nk = (t.K + BK - 1) / BK;
-        const int acc = used & 1;
-        const uint32_t aph = (used >> 1) & 1;
-        ++used;
-        if (!mbar_wait(&tempty_bar[acc], aph ^ 1, status, 2, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
-        bool ok = true;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(&full_bar[s], ph, status, 3, abort_flag)) {
+        const int nch = (KIND == OP_SPLIT3) ? (nk + Cfg::KCH - 1) / Cfg::KCH : 1;
+        for (int c = 0; c < nch && ok; ++c) {
+          const int acc = used & 1;
+          const uint32_t aph = (used >> 1) & 1;
+          ++used;
+          if (!mbar_wait(&tempty_bar[acc], aph ^ 1, status, 2, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + s * Cfg::STAGE_BYTES);
-          const uint32_t b_base = a_base + Cfg::PLANES * Cfg::A_TILE;
-#pragma unroll
-          for (int k = 0; k < BK / Cfg::UMMA_K; ++k) {
-            const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
-            if constexpr (KIND == OP_BF16) {
-              umma_f16(d_tmem, operand_desc<A_MN, BM, Cfg::ESIZE>(a_base, k),
-                       operand_desc<B_MN, BN, Cfg::ESIZE>(b_base, k), Cfg::IDESC, accum);
-            } else {
-              // (A plane, B plane) products, smallest magnitude first
-              constexpr int pa[6] = {1, 0, 2, 0, 1, 0};
-              constexpr int pb[6] = {1, 2, 0, 1, 0, 0};
-#pragma unroll
-              for (int q = 0; q < 6; ++q)
-                umma_f16(d_tmem, operand_desc<A_MN, BM, Cfg::ESIZE>(a_base + pa[q] * Cfg::A_TILE, k),
-                         operand_desc<B_MN, BN, Cfg::ESIZE>(b_base + pb[q] * Cfg::B_TILE, k), Cfg::IDESC,
-                         q == 0 ? accum : 1u);
+          const uint32_t d_tmem = tmem_base + acc * Cfg::ACC_COLS;
+          const int kb0 = (KIND == OP_SPLIT3) ? c * Cfg::KCH : 0;
+          const int kb1 = (KIND == OP_SPLIT3) ? min(nk, kb0 + Cfg::KCH) : nk;
+          for (int kb = kb0; kb < kb1; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            if (!mbar_wait(&full_bar[s], ph, status, 3, abort_flag)) {
+              ok = false;
+              break;
             }
+            tc_fence_after();
+            const uint32_t a_base = smem_u32(smem + s * Cfg::STAGE_BYTES);
+            const uint32_t b_base = a_base + Cfg::PLANES * Cfg::A_TILE;
+#pragma unroll
+            for (int k = 0; k < BK / Cfg::UMMA_K; ++k) {
+              const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
+              if constexpr (KIND == OP_BF16) {
+                umma_f16(d_tmem, operand_desc<A_MN, BM, Cfg::ESIZE>(a_base, k),
+                         operand_desc<B_MN, BN, Cfg::ESIZE>(b_base, k), Cfg::IDESC, accum);
+              } else {
+                // cross products (smallest first) into the correction accumulator,
+                // the main product into its own
+                constexpr int pa[5] = {1, 0, 2, 0, 1};
+                constexpr int pb[5] = {1, 2, 0, 1, 0};
+#pragma unroll
+                for (int q = 0; q < 5; ++q)
+                  umma_f16(d_tmem + BN, operand_desc<A_MN, BM, Cfg::ESIZE>(a_base + pa[q] * Cfg::A_TILE, k),
+                           operand_desc<B_MN, BN, Cfg::ESIZE>(b_base + pb[q] * Cfg::B_TILE, k), Cfg::IDESC,
+                           q == 0 ? accum : 1u);
+                umma_f16(d_tmem, operand_desc<A_MN, BM, Cfg::ESIZE>(a_base, k),
+                         operand_desc<B_MN, BN, Cfg::ESIZE>(b_base, k), Cfg::IDESC, accum);
+              }
+            }
+            umma_commit(&empty_bar[s]);
           }
-          umma_commit(&empty_bar[s]);
+          if (!ok) break;
+          umma_commit(&tfull_bar[acc]);
         }
-        if (!ok) break;
-        umma_commit(&tfull_bar[acc]);
       }
       // every MMA this thread issued has finished before TMEM is released
       mma_it_sh = it;
@@ -531,29 +550,70 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
     const int q = warp & 3;
     const int row_in_tile = q * 32 + lane;
     int used = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       const TileInfo t = src.decode(tile, BM, BN);
       if (!t.valid) continue;
-      const int acc = used & 1;
-      const uint32_t aph = (used >> 1) & 1;
-      ++used;
-      const bool ok = mbar_wait(&tfull_bar[acc], aph, status, 4, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
       const int row = t.m0 + row_in_tile;
       const int ncols = src.cols(t);
+      if constexpr (KIND == OP_BF16) {
+        const int acc = used & 1;
+        const uint32_t aph = (used >> 1) & 1;
+        ++used;
+        const bool w = mbar_wait(&tfull_bar[acc], aph, status, 4, abort_flag);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS;
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        uint32_t rr[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + ch * 32, rr);
-        tmem_wait_ld();
-        float v[32];
+        for (int ch = 0; ch < BN / 32; ++ch) {
+          uint32_t rr[32];
+          tmem_ld_32x32b_x32(tacc + ch * 32, rr);
+          tmem_wait_ld();
+          float v[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(rr[j]);
-        if (t.n0 + ch * 32 < ncols) src.template epilogue<EPI>(t, row, t.n0 + ch * 32, v);
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(rr[j]);
+          if (t.n0 + ch * 32 < ncols) src.template epilogue<EPI>(t, row, t.n0 + ch * 32, v);
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty_bar[acc]);
+      } else {
+        // fold the K-chunk accumulators (main + correction) into fp32 registers
+        const int nk = (t.K + BK - 1) / BK;
+        const int nch = (nk + Cfg::KCH - 1) / Cfg::KCH;
+        float run[BN];
+#pragma unroll
+        for (int j = 0; j < BN; ++j) run[j] = 0.0f;
+        for (int c = 0; c < nch; ++c) {
+          const int acc = used & 1;
+          const uint32_t aph = (used >> 1) & 1;
+          ++used;
+          const bool w = mbar_wait(&tfull_bar[acc], aph, status, 4, abort_flag);
+          if (!__all_sync(0xffffffffu, w)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS;
+#pragma unroll
+          for (int ch = 0; ch < BN / 32; ++ch) {
+            uint32_t rm[32], rc[32];
+            tmem_ld_32x32b_x32(tacc + ch * 32, rm);
+            tmem_ld_32x32b_x32(tacc + BN + ch * 32, rc);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) run[ch * 32 + j] += __uint_as_float(rm[j]) + __uint_as_float(rc[j]);
+          }
+          tc_fence_before();
+          mbar_arrive(&tempty_bar[acc]);
+        }
+        if (!ok) break;
+#pragma unroll
+        for (int ch = 0; ch < BN / 32; ++ch)
+          if (t.n0 + ch * 32 < ncols) src.template epilogue<EPI>(t, row, t.n0 + ch * 32, &run[ch * 32]);
       }
-      tc_fence_before();
-      mbar_arrive(&tempty_bar[acc]);
     }
   }
 
