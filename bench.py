@@ -2,9 +2,11 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl mine|reference]
 
-One "step" applies the library's optimizer step(s) to one full synthetic layer
-set resident in HBM (per rank: N ranks each own one layer set, no collective on
-the data path = weak scaling).  Rank 0 prints one JSON line.
+One "step" applies the whole hot path to one full synthetic layer set resident
+in HBM: a Muon step, a SOAP step (eigenbasis refresh every step) and a FOAM step
+(adaptive refresh check every 10 steps), all on the same weights and gradients
+(per rank: N ranks each own one layer set, no collective on the data path =
+weak scaling).  Rank 0 prints one JSON line.
 
 Timing: W untimed warm-up steps; K timed steps between a barrier and
 cudaDeviceSynchronize on both sides, CUDA events on the launching stream, max
@@ -46,11 +48,12 @@ MUON_NORM = {"gpt2_124m": "col_row"}
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
     ap.add_argument("--workload", default="dense8b_moe", choices=sorted(WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--optimizers", default="muon,soap,foam", help="comma list of muon, soap, foam")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
     return ap.parse_args()
@@ -154,49 +157,133 @@ def ncu_traffic(kernel_name, workload):
 
 
 # ----------------------------------------------------------------------------- CPU (oracle) leg
-def cpu_oracle_sample(workload, budget_s, seed):
+def _ns_flops(m, n):
+    a, b = min(m, n), max(m, n)
+    return 5 * (4 * a * a * b + 2 * a ** 3)
+
+
+def _soap_flops(m, n):
+    # factors, power step, QR (Householder with explicit Q), two rotations in, one back
+    return 2 * m * m * n + 2 * m * n * n + 2 * (m ** 3 + n ** 3) + 8 / 3 * (m ** 3 + n ** 3) + 6 * (m * m * n + m * n * n)
+
+
+def _foam_flops(m, n, check):
+    f = 8 * m * n * n
+    if check:
+        f += 4 * n ** 3 + 2 * n ** 3 + 8 / 3 * n ** 3
+    return f
+
+
+def cpu_oracle_sample(workload, budget_s, seed, optimizers, t_foam=1):
     """Time the float64 oracle on a bounded sample of the workload's matrices and
     scale to one full layer set.  Returns (ms per layer set, cores, sample text)."""
-    from matrix_aware_optimizers_02_b200 import synth
     from oracle import mao_oracle as O
     specs = specs_for(workload, seed)
     norm = {"col_row": O.NORM_COL_ROW}.get(MUON_NORM.get(workload, "none"), O.NORM_NONE)
-    # distinct shapes with multiplicities, cheapest first
     shapes = {}
     for s in specs:
         shapes[(s.m, s.n)] = shapes.get((s.m, s.n), 0) + 1
-
-    def ns_flops(m, n):
-        a, b = min(m, n), max(m, n)
-        return 5 * (4 * a * a * b + 2 * a ** 3)
-
-    order = sorted(shapes, key=lambda k: ns_flops(*k))
+    models = {"muon": _ns_flops, "soap": _soap_flops, "foam": lambda m, n: _foam_flops(m, n, True)}
     rng = np.random.default_rng(seed)
-    timed = {}
-    spent = 0.0
-    for (m, n) in order:
-        if spent > budget_s * 0.6 and timed:
-            break
-        W = rng.standard_normal((m, n)) * 0.02
-        G = rng.standard_normal((m, n)) * 0.01
-        M = np.zeros((m, n))
-        t0 = time.perf_counter()
-        O.muon_step(W, G, M, mu=0.95, lr=0.02, norm=norm)
-        dt = time.perf_counter() - t0
-        timed[(m, n)] = dt
-        spent += dt
-    # shapes not timed: scale by Newton-Schulz FLOPs at the best timed rate (largest shape)
-    rate = max(ns_flops(*k) / v for k, v in timed.items())
-    total = 0.0
-    for k, cnt in shapes.items():
-        total += cnt * (timed[k] if k in timed else ns_flops(*k) / rate)
+    total_ms = 0.0
+    parts = []
+    per_opt_budget = budget_s / max(len(optimizers), 1)
+    for opt in optimizers:
+        flops = models[opt]
+        order = sorted(shapes, key=lambda k: flops(*k))
+        timed, spent = {}, 0.0
+        for (m, n) in order:
+            if spent > per_opt_budget * 0.5 and timed:
+                break
+            if timed and flops(m, n) / max(flops(*k) / v for k, v in timed.items()) > per_opt_budget:
+                break  # one more shape would blow the budget: extrapolate instead
+            W = rng.standard_normal((m, n)) * 0.02
+            G = rng.standard_normal((m, n)) * 0.01
+            t0 = time.perf_counter()
+            if opt == "muon":
+                O.muon_step(W, G, np.zeros((m, n)), mu=0.95, lr=0.02, norm=norm)
+            elif opt == "soap":
+                O.soap_step(W, G, O.SoapState.init(m, n), t=1, beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3)
+            else:
+                O.foam_step(W, G, O.FoamState.init(m, n), t=1, beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3)
+            dt = time.perf_counter() - t0
+            timed[(m, n)] = dt
+            spent += dt
+        rate = max(flops(*k) / v for k, v in timed.items())
+        opt_s = sum(cnt * (timed[k] if k in timed else flops(*k) / rate) for k, cnt in shapes.items())
+        total_ms += opt_s * 1e3
+        parts.append(f"{opt}: timed {', '.join(f'{m}x{n}' for (m, n) in timed)} ({spent:.1f} s)" +
+                     ("" if len(timed) == len(shapes) else ", other shapes scaled by the step's FLOP model"))
     cores = len(os.sched_getaffinity(0))
-    sample = ("oracle muon_step (float64 NumPy) timed once on shapes " +
-              ", ".join(f"{m}x{n}" for (m, n) in timed) +
-              "; each shape's time x its multiplicity" +
-              ("" if len(timed) == len(shapes) else "; untimed shapes scaled by Newton-Schulz FLOPs") +
-              f"; {spent:.1f} s of CPU work")
-    return total * 1e3, cores, sample
+    sample = ("float64 NumPy oracle, each distinct shape's step time x its multiplicity (SOAP and FOAM steps "
+              "with a basis refresh); " + "; ".join(parts))
+    return total_ms, cores, sample
+
+
+# ----------------------------------------------------------------------------- the layer set on the GPU
+class LayerSet:
+    """W, G and the optimizer states of one synthetic layer set, plus one batch
+    object per optimizer (sharing W, G and one workspace)."""
+
+    def __init__(self, specs, seed, dev, g_bf16, optimizers, norm):
+        import torch
+
+        from matrix_aware_optimizers_02_b200 import api, synth
+        self.torch = torch
+        base = synth.torch_muon_inputs(specs, seed, dev, g_bf16=g_bf16)
+        self.W = [w for (w, _, _) in base]
+        self.G = [g for (_, g, _) in base]
+        del base
+        self.batches = {}
+        z = torch.zeros
+        if "muon" in optimizers:
+            mats = [(w, g, z(w.shape, device=dev)) for w, g in zip(self.W, self.G)]
+            self.batches["muon"] = api.MuonBatch(mats, mu=0.95, lr=0.02, norm=norm, with_stats=True,
+                                                 allocate=False)
+        if "soap" in optimizers:
+            mats = []
+            for w, g in zip(self.W, self.G):
+                m, n = w.shape
+                mats.append({"W": w, "G": g, "M": z((m, n), device=dev), "V": z((m, n), device=dev),
+                             "L": torch.eye(m, device=dev) * 1e-6, "R": torch.eye(n, device=dev) * 1e-6,
+                             "QL": torch.eye(m, device=dev), "QR": torch.eye(n, device=dev)})
+            self.batches["soap"] = api.SoapBatch(mats, beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3,
+                                                 refresh="every_k", k=1, with_stats=True, allocate=False)
+        if "foam" in optimizers:
+            mats = []
+            for w, g in zip(self.W, self.G):
+                m, n = w.shape
+                mats.append({"W": w, "G": g, "M": z((m, n), device=dev), "r": z(m, device=dev),
+                             "c": z(n, device=dev), "R": torch.eye(n, device=dev) * 1e-6,
+                             "QR": torch.eye(n, device=dev)})
+            self.batches["foam"] = api.FoamBatch(mats, beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3,
+                                                 refresh="adaptive", pf=10, tol=0.1, with_stats=True,
+                                                 allocate=False)
+        self.order = [o for o in ("muon", "soap", "foam") if o in self.batches]
+        # the steps run in order on one stream, so one workspace serves all of them
+        ws_bytes = max(b.ws_bytes for b in self.batches.values())
+        self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        for b in self.batches.values():
+            b.attach_workspace(self.workspace)
+
+    def step(self, t, stream, events=None):
+        for i, name in enumerate(self.order):
+            b = self.batches[name]
+            if events is not None:
+                events[name][0].record(stream)
+            if name == "muon":
+                b()
+            else:
+                b(t)
+            if events is not None:
+                events[name][1].record(stream)
+
+    def status(self):
+        for name, b in self.batches.items():
+            st = b.device_status()
+            if st != 0:
+                return name, st
+        return None
 
 
 # ----------------------------------------------------------------------------- main (mine)
@@ -204,35 +291,42 @@ def run_mine(args, rank, world, dist):
     import torch
 
     from matrix_aware_optimizers_02_b200 import _lib as L
-    from matrix_aware_optimizers_02_b200 import api, synth
 
     lib = L.load()
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
     desc, g_bf16 = WORKLOADS[args.workload]
     specs = specs_for(args.workload, args.seed)
-    mats = synth.torch_muon_inputs(specs, args.seed + 7919 * rank, dev, g_bf16=g_bf16)
+    optimizers = [o.strip() for o in args.optimizers.split(",") if o.strip()]
     norm = MUON_NORM.get(args.workload, "none")
-    step = api.MuonBatch(mats, mu=0.95, lr=0.02, norm=norm, with_stats=True)
+    LS = LayerSet(specs, args.seed + 7919 * rank, dev, g_bf16, optimizers, norm)
     stream = torch.cuda.current_stream()
 
     def barrier():
         if dist is not None:
             dist.barrier()
 
+    t = 0
     for _ in range(args.warmup):
-        step()
+        t += 1
+        LS.step(t, stream)
     torch.cuda.synchronize()
-    status = step.device_status()
-    if status != 0:
-        raise RuntimeError(f"device status {status} after warm-up")
+    bad = LS.status()
+    if bad:
+        raise RuntimeError(f"device status {bad} after warm-up")
 
-    # launch profiler sized for the timed steps
-    cap = 4096
+    # launch profiler: one probe step counts the launches, then events for the timed steps
+    lib.mao_profile_start(None, None, 0)
+    t += 1
+    LS.step(t, stream)
+    per_step_launches = lib.mao_profile_stop()
+    torch.cuda.synchronize()
+    cap = min(per_step_launches * args.steps + 16, 60000)
     Ev = ctypes.c_void_p * (2 * cap)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * cap)]
     for e in evs:  # torch creates the CUDA event object on its first record
         e.record(stream)
+    opt_ev = {o: [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)] for o in LS.order}
     torch.cuda.synchronize()
     ev_arr = Ev(*[ctypes.c_void_p(e.cuda_event) for e in evs])
     info = (L.LaunchInfo * cap)()
@@ -247,33 +341,37 @@ def run_mine(args, rank, world, dist):
     t_end = torch.cuda.Event(enable_timing=True)
     L.check(lib.mao_profile_start(ev_arr, info, cap))
     t_start.record(stream)
-    for _ in range(args.steps):
-        step()
+    for k in range(args.steps):
+        t += 1
+        LS.step(t, stream, {o: (opt_ev[o][2 * k], opt_ev[o][2 * k + 1]) for o in LS.order})
     t_end.record(stream)
     n_launch = lib.mao_profile_stop()
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop() if clocks else None
     ms = t_start.elapsed_time(t_end) / args.steps
-    status = step.device_status()
-    if status != 0:
-        raise RuntimeError(f"device status {status} after timed steps")
+    opt_ms = {o: round(sum(opt_ev[o][2 * k].elapsed_time(opt_ev[o][2 * k + 1]) for k in range(args.steps))
+                       / args.steps, 3) for o in LS.order}
+    bad = LS.status()
+    if bad:
+        raise RuntimeError(f"device status {bad} after timed steps")
 
     # per-kernel live durations
     per = {}
     for i in range(min(n_launch, cap)):
-        k = info[i].kernel
+        kk = info[i].kernel
         d = evs[2 * i].elapsed_time(evs[2 * i + 1])
-        e = per.setdefault(k, {"ms": 0.0, "n": 0, "flops": 0.0, "bytes": 0.0})
+        e = per.setdefault(kk, {"ms": 0.0, "n": 0, "flops": 0.0, "bytes": 0.0})
         e["ms"] += d
         e["n"] += 1
         e["flops"] += info[i].flops
         e["bytes"] += info[i].bytes
 
-    # end-to-end: gradients from pinned host memory, step, stats back to host
-    host_g = [g.cpu().pin_memory() for (_, g, _) in mats]
+    # end-to-end: gradients from pinned host memory, the step, stats back to host
+    host_g = [g.cpu().pin_memory() for g in LS.G]
     h2d = sum(g.numel() * g.element_size() for g in host_g)
-    stats_host = torch.empty_like(step.stats, device="cpu").pin_memory()
+    res = LS.batches[LS.order[0]].stats
+    stats_host = torch.empty_like(res, device="cpu").pin_memory()
     d2h = stats_host.numel() * stats_host.element_size()
     barrier()
     torch.cuda.synchronize()
@@ -281,19 +379,20 @@ def run_mine(args, rank, world, dist):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        for (_, g, _), hg in zip(mats, host_g):
+        t += 1
+        for g, hg in zip(LS.G, host_g):
             g.copy_(hg, non_blocking=True)
-        step()
-        stats_host.copy_(step.stats, non_blocking=True)
+        LS.step(t, stream)
+        stats_host.copy_(res, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1) / args.steps
 
-    t = torch.tensor([ms, e2e_ms], device=dev)
+    tt = torch.tensor([ms, e2e_ms], device=dev)
     if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max, e2e_max = t.tolist()
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    ms_max, e2e_max = tt.tolist()
     if rank != 0:
         return None
 
@@ -319,16 +418,19 @@ def run_mine(args, rank, world, dist):
         roof["traffic"] = ncu_traffic(names.get(dom, str(dom)), args.workload)
         roof["launches"] = e["n"]
         roof["avg_launch_ms"] = round(avg_ms, 4)
-    kernels = {names.get(k, str(k)): {"launches": v["n"], "ms_total": round(v["ms"], 3),
-                                      "share": round(v["ms"] / max(sum(x["ms"] for x in per.values()), 1e-9), 4),
-                                      **({"tflops": round(v["flops"] / (v["ms"] * 1e-3) / 1e12, 1)}
-                                         if v["flops"] > 0 else
-                                         {"gbs": round(v["bytes"] / (v["ms"] * 1e-3) / 1e9, 1)})}
-               for k, v in sorted(per.items())}
+    tot = max(sum(x["ms"] for x in per.values()), 1e-9)
+    kernels = {}
+    for k, v in sorted(per.items()):
+        rec = {"launches": v["n"], "ms_total": round(v["ms"], 3), "share": round(v["ms"] / tot, 4)}
+        if v["flops"] > 0:
+            rec["tflops"] = round(v["flops"] / (v["ms"] * 1e-3) / 1e12, 1)
+        elif v["bytes"] > 0:
+            rec["gbs"] = round(v["bytes"] / (v["ms"] * 1e-3) / 1e9, 1)
+        kernels[names.get(k, str(k))] = rec
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        cpu_ms, cores, sample = cpu_oracle_sample(args.workload, args.cpu_budget_s, args.seed)
+        cpu_ms, cores, sample = cpu_oracle_sample(args.workload, args.cpu_budget_s, args.seed, LS.order)
         cpu = {"value": round(cpu_ms, 1), "unit": "ms", "cores": cores, "kind": "oracle", "sample": sample}
 
     n_elems = sum(s.m * s.n for s in specs)
@@ -343,10 +445,15 @@ def run_mine(args, rank, world, dist):
         "higher_is_better": False,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16 operands / fp32 accumulate (Newton-Schulz), fp32 states",
+        "dtype": "bf16 operands / fp32 accumulate (Newton-Schulz); fp32-faithful split-bf16 products and fp32 "
+                 "states (SOAP, FOAM)",
         "data": "synthetic (seeded Gaussian gradients, random weights)",
-        "config": {"workload": args.workload, "description": desc, "optimizers": ["muon"],
+        "config": {"workload": args.workload, "description": desc, "optimizers": LS.order,
+                   "optimizer_ms": opt_ms,
                    "muon": {"mu": 0.95, "lr": 0.02, "ns_steps": 5, "norm": norm},
+                   "soap": {"beta1": 0.95, "beta2": 0.95, "eps": 1e-8, "refresh": "every step, sorted"},
+                   "foam": {"beta1": 0.95, "beta2": 0.95, "eps": 1e-8, "refresh": "adaptive pf=10 tol=0.1"},
+                   "timed_steps_t": [args.warmup + 2, args.warmup + 1 + args.steps],
                    "matrices_per_rank": len(specs), "elements_per_rank": n_elems,
                    "l2_policy": "inputs larger than L2 (no flush)", "parallelism": f"independent layer sets x{world}"},
         "roofline": roof,
@@ -364,10 +471,12 @@ def run_reference(args, rank, world):
     """The oracle as the reference arm, on the host cores, rank 0 only."""
     if rank != 0:
         return None
+    optimizers = [o.strip() for o in args.optimizers.split(",") if o.strip()]
     per_step = []
     info = None
     for i in range(args.warmup + args.steps):
-        ms, cores, sample = cpu_oracle_sample(args.workload, args.cpu_budget_s / max(args.steps, 1), args.seed + i)
+        ms, cores, sample = cpu_oracle_sample(args.workload, args.cpu_budget_s / max(args.steps, 1), args.seed + i,
+                                              optimizers)
         if i >= args.warmup:
             per_step.append(ms)
             info = (cores, sample)
@@ -379,7 +488,7 @@ def run_reference(args, rank, world):
         "value": round(v, 1), "unit": "ms", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(v, 1), "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded Gaussian)",
-        "config": {"workload": args.workload, "description": desc, "optimizers": ["muon"]},
+        "config": {"workload": args.workload, "description": desc, "optimizers": optimizers},
         "cpu_baseline": {"value": round(v, 1), "unit": "ms", "cores": info[0], "kind": "oracle", "sample": info[1]},
         "e2e": {"value": round(v, 1), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

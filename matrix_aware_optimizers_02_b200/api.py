@@ -57,7 +57,7 @@ class MuonBatch:
     def __init__(self, mats: Sequence[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]], *, mu: float, lr: float,
                  wd: float = 0.0, eps: float = 1e-7, ns_steps: int = 5,
                  ns_coef: Optional[Sequence[Sequence[float]]] = None, norm: str = "none",
-                 workspace: Optional[torch.Tensor] = None, with_stats: bool = False):
+                 workspace: Optional[torch.Tensor] = None, with_stats: bool = False, allocate: bool = True):
         self.lib = L.load()
         self.mats = list(mats)
         n = len(self.mats)
@@ -87,14 +87,20 @@ class MuonBatch:
         L.check(self.lib.mao_muon_workspace_size(arr, n, ctypes.byref(self.params), ctypes.byref(nbytes)),
                 "mao_muon_workspace_size")
         self.ws_bytes = nbytes.value
-        if workspace is None:
-            workspace = _alloc_workspace(self.ws_bytes, dev if dev is not None else "cuda")
-        elif workspace.numel() * workspace.element_size() < self.ws_bytes:
-            raise ValueError("workspace too small")
-        self.workspace = workspace
+        dev = dev if dev is not None else torch.device("cuda")
+        self.workspace = None
+        if workspace is not None or allocate:
+            self.attach_workspace(workspace if workspace is not None else _alloc_workspace(self.ws_bytes, dev))
         self.stats = None
         if with_stats:
-            self.stats = torch.zeros((max(n, 1), 4), dtype=torch.float32, device=workspace.device)
+            self.stats = torch.zeros((max(n, 1), 4), dtype=torch.float32, device=dev)
+
+    def attach_workspace(self, workspace: torch.Tensor) -> None:
+        """Use `workspace` (uint8 CUDA tensor of at least ws_bytes) from now on; several
+        batches run on one stream may share one workspace."""
+        if workspace.numel() * workspace.element_size() < self.ws_bytes:
+            raise ValueError("workspace too small")
+        self.workspace = workspace
 
     def __call__(self, stream: Optional[torch.cuda.Stream] = None) -> None:
         st = self.lib.mao_muon_step(self.arr, self.count, ctypes.byref(self.params), self.workspace.data_ptr(),
@@ -157,16 +163,21 @@ def _refresh(kind: str, k: int, pf: int, tol: float, sort: bool) -> "L.Refresh":
 class _PrecondBatch:
     """Shared plumbing of SoapBatch / FoamBatch."""
 
-    def _finish(self, size_fn, n, device, workspace, with_stats):
+    def _finish(self, size_fn, n, device, workspace, with_stats, allocate=True):
         nbytes = ctypes.c_size_t(0)
         L.check(size_fn(self.arr, n, ctypes.byref(self.params), ctypes.byref(nbytes)), size_fn.__name__)
         self.ws_bytes = nbytes.value
-        if workspace is None:
-            workspace = _alloc_workspace(self.ws_bytes, device)
-        elif workspace.numel() * workspace.element_size() < self.ws_bytes:
+        self.workspace = None
+        if workspace is not None or allocate:
+            self.attach_workspace(workspace if workspace is not None else _alloc_workspace(self.ws_bytes, device))
+        self.stats = torch.zeros((max(n, 1), 4), dtype=torch.float32, device=device) if with_stats else None
+
+    def attach_workspace(self, workspace: torch.Tensor) -> None:
+        """Use `workspace` (uint8 CUDA tensor of at least ws_bytes); several batches run on
+        one stream may share one workspace."""
+        if workspace.numel() * workspace.element_size() < self.ws_bytes:
             raise ValueError("workspace too small")
         self.workspace = workspace
-        self.stats = torch.zeros((max(n, 1), 4), dtype=torch.float32, device=device) if with_stats else None
 
     def device_status(self, stream: Optional[torch.cuda.Stream] = None) -> int:
         where = ctypes.c_int32(0)
@@ -190,7 +201,8 @@ class SoapBatch(_PrecondBatch):
 
     def __init__(self, mats, *, beta1: float, beta2: float, eps: float, lr: float, wd: float = 0.0,
                  refresh: str = "every_k", k: int = 1, pf: int = 10, tol: float = 0.1, sort: bool = True,
-                 workspace: Optional[torch.Tensor] = None, with_stats: bool = False, t: int = 1):
+                 workspace: Optional[torch.Tensor] = None, with_stats: bool = False, t: int = 1,
+                 allocate: bool = True):
         self.lib = L.load()
         self.mats = list(mats)
         n = len(self.mats)
@@ -211,7 +223,8 @@ class SoapBatch(_PrecondBatch):
             dev = W.device
         self.count = n
         self.params = L.SoapParams(beta1, beta2, eps, lr, wd, int(t), _refresh(refresh, k, pf, tol, sort))
-        self._finish(self.lib.mao_soap_workspace_size, n, dev if dev is not None else "cuda", workspace, with_stats)
+        self._finish(self.lib.mao_soap_workspace_size, n, dev if dev is not None else "cuda", workspace, with_stats,
+                     allocate)
 
     def __call__(self, t: int, stream: Optional[torch.cuda.Stream] = None) -> None:
         self.params.t = int(t)
@@ -231,7 +244,7 @@ class FoamBatch(_PrecondBatch):
     def __init__(self, mats, *, beta1: float, beta2: float, eps: float, lr: float, wd: float = 0.0,
                  refresh: str = "adaptive", k: int = 1, pf: int = 10, tol: float = 0.1, sort: bool = True,
                  tau_raw_trace: bool = False, workspace: Optional[torch.Tensor] = None, with_stats: bool = False,
-                 t: int = 1):
+                 t: int = 1, allocate: bool = True):
         self.lib = L.load()
         self.mats = list(mats)
         n = len(self.mats)
@@ -252,7 +265,8 @@ class FoamBatch(_PrecondBatch):
         self.count = n
         self.params = L.FoamParams(beta1, beta2, eps, lr, wd, int(t), _refresh(refresh, k, pf, tol, sort),
                                    int(bool(tau_raw_trace)))
-        self._finish(self.lib.mao_foam_workspace_size, n, dev if dev is not None else "cuda", workspace, with_stats)
+        self._finish(self.lib.mao_foam_workspace_size, n, dev if dev is not None else "cuda", workspace, with_stats,
+                     allocate)
 
     def __call__(self, t: int, stream: Optional[torch.cuda.Stream] = None) -> None:
         self.params.t = int(t)

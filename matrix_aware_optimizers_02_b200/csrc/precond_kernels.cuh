@@ -606,15 +606,25 @@ __global__ void __launch_bounds__(256) pc_check_kernel(const CheckJob* __restric
 // Per-matrix diagnostics of a SOAP / FOAM step: refresh bits and the check ratio.
 // fixed_bits >= 0: the refresh was decided on the host (bits given); otherwise
 // read the device flags (bit 0 right side, bit 1 left side).
-__global__ void pc_stats_kernel(mao_stats* st, const int* flag_r, const int* flag_l, const float* rho,
-                                int fixed_bits) {
-  if (threadIdx.x != 0) return;
-  int bits = fixed_bits;
-  if (bits < 0) bits = ((flag_r && *flag_r) ? 1 : 0) | ((flag_l && *flag_l) ? 2 : 0);
-  st->update_rms = -1.0f;
-  st->offdiag_ratio = rho ? *rho : -1.0f;
-  st->refreshed = bits;
-  st->nonfinite = 0;
+struct StatsJob {
+  const int* flag_r;
+  const int* flag_l;
+  const float* rho;
+  int fixed_bits;
+  int index;  // position in the caller's stats array
+};
+
+__global__ void pc_stats_kernel(const StatsJob* __restrict__ J, int n, mao_stats* __restrict__ stats) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const StatsJob& j = J[i];
+  int bits = j.fixed_bits;
+  if (bits < 0) bits = ((j.flag_r && *j.flag_r) ? 1 : 0) | ((j.flag_l && *j.flag_l) ? 2 : 0);
+  mao_stats& st = stats[j.index];
+  st.update_rms = -1.0f;
+  st.offdiag_ratio = j.rho ? *j.rho : -1.0f;
+  st.refreshed = bits;
+  st.nonfinite = 0;
 }
 
 }  // namespace mao

@@ -18,6 +18,9 @@
 //                 N = (Mr/bc1)/(sqrt(tau r c^T)+eps) ; U = N Q_R^T fused with the W update
 #include <algorithm>
 #include <cmath>
+#include <list>
+#include <memory>
+#include <string>
 
 #include "host_common.h"
 #include "precond_kernels.cuh"
@@ -93,7 +96,7 @@ struct MatBuf {
   SideBuf L, R;
 };
 
-void side_layout(int k, bool check, Carver& cv, SideBuf& s) {
+void side_layout(int k, bool check, Carver& cv, SideBuf& s, size_t flag_block) {
   const size_t kk = (size_t)k * k;
   const int chunks = (k + kGramRows - 1) / kGramRows;
   s.Fp = cv.take(planes_bytes(k, k));
@@ -108,7 +111,7 @@ void side_layout(int k, bool check, Carver& cv, SideBuf& s) {
   s.rinv = cv.take(8 * (size_t)kPanel * kPanel);
   s.keys = cv.take(8 * (size_t)k);
   s.perm = cv.take(4 * (size_t)k);
-  s.flag = cv.take(64);  // flag, rho and the failure counter share one 64-byte block
+  s.flag = flag_block;  // flag, rho and the failure counter share one 64-byte block
   s.rho = s.flag + 16;
   s.bad = s.flag + 32;
   if (check) {
@@ -131,6 +134,7 @@ struct Ctx {
 struct GroupPlan {
   int g0 = 0, g1 = 0;   // matrices [g0, g1)
   size_t scratch = 0;   // bytes of per-matrix scratch
+  size_t flags = 0, flags_bytes = 0;  // all 64-byte flag blocks of the group, contiguous
   std::vector<MatBuf> mb;
 };
 
@@ -139,6 +143,8 @@ void plan_group_scratch(const Ctx& X, GroupPlan& G, size_t base) {
   cv.off = base;
   G.mb.assign(G.g1 - G.g0, MatBuf());
   const bool check = X.mode == 2;
+  G.flags_bytes = (size_t)64 * 2 * (G.g1 - G.g0);
+  G.flags = cv.take(G.flags_bytes);
   for (int i = G.g0; i < G.g1; ++i) {
     const PcMat& a = X.mats[i];
     MatBuf& b = G.mb[i - G.g0];
@@ -151,7 +157,7 @@ void plan_group_scratch(const Ctx& X, GroupPlan& G, size_t base) {
       b.Vtmp = cv.take(4 * mn);
       b.Gh = cv.take(4 * mn);
       b.Mh = cv.take(4 * mn);
-      side_layout(a.m, check, cv, b.L);
+      side_layout(a.m, check, cv, b.L, G.flags + (size_t)128 * (i - G.g0));
     } else {
       b.Gr = cv.take(4 * mn);
       b.Mr = cv.take(4 * mn);
@@ -161,7 +167,7 @@ void plan_group_scratch(const Ctx& X, GroupPlan& G, size_t base) {
       b.ctmp = cv.take(4 * (size_t)a.n);
       b.tau = cv.take(16);
     }
-    side_layout(a.n, check, cv, b.R);
+    side_layout(a.n, check, cv, b.R, G.flags + (size_t)128 * (i - G.g0) + 64);
   }
   G.scratch = cv.off - base;
 }
@@ -760,9 +766,15 @@ mao_status build_group(Builder& B, GroupPlan& G) {
   return MAO_OK;
 }
 
+// Everything one group needs at launch time, independent of the caller's
+// descriptor array: the staged host image of the arena and the launch list.
 struct BuiltGroup {
   size_t maps_off = 0;
   std::vector<StagedLaunch> staged;
+  std::vector<Op> ops;
+  std::vector<int> gemm_of_op;
+  std::vector<uint8_t> arena;
+  size_t stats_jobs = 0;  // StatsJob array in the arena
 };
 
 mao_status finish_build(Builder& B, BuiltGroup& out) {
@@ -777,14 +789,35 @@ mao_status finish_build(Builder& B, BuiltGroup& out) {
   return MAO_OK;
 }
 
-mao_status run_ops(Builder& B, const BuiltGroup& bg, DevStatus* status, cudaStream_t s) {
-  const Ctx& X = B.X;
+// Per-matrix diagnostics records of a group (one launch).
+void add_stats_jobs(Builder& B, GroupPlan& G, BuiltGroup& bg) {
+  const int nm = G.g1 - G.g0;
+  bg.stats_jobs = B.arena.take(sizeof(StatsJob) * std::max(nm, 1), 64);
+  StatsJob* S = B.arena.hptr<StatsJob>(bg.stats_jobs);
+  std::memset(static_cast<void*>(S), 0, sizeof(StatsJob) * std::max(nm, 1));
+  for (int i = 0; i < nm; ++i) {
+    StatsJob& j = S[i];
+    j.index = G.g0 + i;
+    if (B.X.mode == 2) {
+      j.flag_r = B.wp<int>(G.mb[i].R.flag);
+      j.flag_l = B.X.foam ? nullptr : B.wp<int>(G.mb[i].L.flag);
+      j.rho = B.wp<float>(G.mb[i].R.rho);
+      j.fixed_bits = -1;
+    } else {
+      j.fixed_bits = B.X.mode == 1 ? (B.X.foam ? 1 : 3) : 0;
+    }
+  }
+}
+
+mao_status run_ops(const Ctx& X, uint8_t* arena_dev, const BuiltGroup& bg, DevStatus* status, cudaStream_t s) {
+  Arena A;  // device view of the staged arena
+  A.dev = arena_dev;
   const float bc1 = (float)(1.0 - std::pow((double)X.b1, (double)X.t));
   const float bc2 = (float)(1.0 - std::pow((double)X.b2, (double)X.t));
-  for (size_t o = 0; o < B.ops.size(); ++o) {
-    const Op& op = B.ops[o];
+  for (size_t o = 0; o < bg.ops.size(); ++o) {
+    const Op& op = bg.ops[o];
     if (op.kind == Op::GEMM) {
-      MAO_TRY(table_launch(B.arena, bg.staged[B.gemm_of_op[o]], status, s));
+      MAO_TRY(table_launch(A, bg.staged[bg.gemm_of_op[o]], status, s));
       continue;
     }
     if (op.blocks <= 0) continue;
@@ -792,75 +825,75 @@ mao_status run_ops(Builder& B, const BuiltGroup& bg, DevStatus* status, cudaStre
     switch (op.kind) {
       case Op::EW: {
         LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, op.bytes);
-        pc_momentum_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<EwJob>(op.jobs), n, X.b1);
+        pc_momentum_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<EwJob>(op.jobs), n, X.b1);
         break;
       }
       case Op::SPLIT: {
         LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, 0.0);
-        pc_split_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<EwJob>(op.jobs), n);
+        pc_split_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<EwJob>(op.jobs), n);
         break;
       }
       case Op::ADAM: {
         LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, op.bytes);
-        soap_adam_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<EwJob>(op.jobs), n, X.b2, 1.f / bc1, 1.f / bc2, X.eps);
+        soap_adam_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<EwJob>(op.jobs), n, X.b2, 1.f / bc1, 1.f / bc2, X.eps);
         break;
       }
       case Op::KEYS: {
         LaunchScope ls(s, MAO_K_PC_SORT, 0.0, 0.0);
         if (X.rf.sort)
-          pc_keys_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<SortJob>(op.jobs), n);
+          pc_keys_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<SortJob>(op.jobs), n);
         else
-          pc_identity_keys_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<SortJob>(op.jobs), n);
+          pc_identity_keys_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<SortJob>(op.jobs), n);
         break;
       }
       case Op::ARGSORT: {
         LaunchScope ls(s, MAO_K_PC_SORT, 0.0, 0.0);
-        pc_argsort_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<SortJob>(op.jobs), n);
+        pc_argsort_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<SortJob>(op.jobs), n);
         break;
       }
       case Op::GATHER: {
         LaunchScope ls(s, MAO_K_PC_SORT, 0.0, 0.0);
-        pc_gather_cols_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<GatherJob>(op.jobs), n);
+        pc_gather_cols_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<GatherJob>(op.jobs), n);
         break;
       }
       case Op::VPERM: {
         LaunchScope ls(s, MAO_K_PC_SORT, 0.0, 0.0);
-        soap_vperm_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<VPermJob>(op.jobs), n);
+        soap_vperm_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<VPermJob>(op.jobs), n);
         break;
       }
       case Op::GRAM: {
         LaunchScope ls(s, MAO_K_PC_QR, 0.0, 0.0);
-        qr_gram_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<PanelJob>(op.jobs), n);
+        qr_gram_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<PanelJob>(op.jobs), n);
         break;
       }
       case Op::CHOL: {
         LaunchScope ls(s, MAO_K_PC_QR, 0.0, 0.0);
-        qr_chol_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<PanelJob>(op.jobs), n);
+        qr_chol_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<PanelJob>(op.jobs), n);
         break;
       }
       case Op::APPLY: {
         LaunchScope ls(s, MAO_K_PC_QR, 0.0, 0.0);
-        qr_apply_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<PanelJob>(op.jobs), n);
+        qr_apply_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<PanelJob>(op.jobs), n);
         break;
       }
       case Op::RC: {
         LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, 0.0);
-        foam_rc_partial_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<RcJob>(op.jobs), n);
+        foam_rc_partial_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<RcJob>(op.jobs), n);
         break;
       }
       case Op::TAU: {
         LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, 0.0);
-        foam_tau_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<TauJob>(op.jobs), X.b2, 1.f / bc2, X.raw_trace);
+        foam_tau_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<TauJob>(op.jobs), X.b2, 1.f / bc2, X.raw_trace);
         break;
       }
       case Op::FOAMN: {
         LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, 0.0);
-        foam_n_kernel<<<op.blocks, 256, 0, s>>>(B.arena.dptr<EwJob>(op.jobs), n, 1.f / bc1, 1.f / bc2, X.eps);
+        foam_n_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<EwJob>(op.jobs), n, 1.f / bc1, 1.f / bc2, X.eps);
         break;
       }
       case Op::CHECK: {
         LaunchScope ls(s, MAO_K_PC_CHECK, 0.0, 0.0);
-        pc_check_kernel<<<n, 256, 0, s>>>(B.arena.dptr<CheckJob>(op.jobs), X.rf.tol);
+        pc_check_kernel<<<n, 256, 0, s>>>(A.dptr<CheckJob>(op.jobs), X.rf.tol);
         break;
       }
       default:
@@ -876,69 +909,138 @@ struct Layout {
   size_t scratch_off = 0, scratch = 0, arena_off = 0, arena = 0, total = 0;
 };
 
-mao_status layout_for(const Ctx& X, std::vector<GroupPlan>& groups, Layout& L) {
-  make_groups(X, groups);
+// A whole step's launch plan for one (descriptor array, parameters, workspace).
+struct StepPlan {
+  Layout L;
+  std::vector<GroupPlan> groups;
+  std::vector<BuiltGroup> built;
+};
+
+// ws == nullptr: sizing only (layout), nothing encoded.
+mao_status make_plan(const Ctx& X, uint8_t* ws, StepPlan& P) {
+  make_groups(X, P.groups);
+  Layout& L = P.L;
   L.scratch_off = align_up(kStatusBytes, 256);
-  for (GroupPlan& g : groups) {
+  for (GroupPlan& g : P.groups) {
     plan_group_scratch(X, g, L.scratch_off);
     L.scratch = std::max(L.scratch, g.scratch);
   }
   L.arena_off = align_up(L.scratch_off + L.scratch, 256);
-  for (GroupPlan& g : groups) {
-    Builder B(X, nullptr);
+  P.built.assign(P.groups.size(), BuiltGroup());
+  for (size_t gi = 0; gi < P.groups.size(); ++gi) {
+    GroupPlan& g = P.groups[gi];
+    Builder B(X, ws);
+    if (ws) B.arena.dev = ws + L.arena_off;
     MAO_TRY(build_group(B, g));
-    BuiltGroup bg;
+    BuiltGroup& bg = P.built[gi];
+    add_stats_jobs(B, g, bg);
     MAO_TRY(finish_build(B, bg));
     L.arena = std::max(L.arena, B.arena.host.size());
+    if (ws) {
+      bg.ops = std::move(B.ops);
+      bg.gemm_of_op = std::move(B.gemm_of_op);
+      bg.arena = std::move(B.arena.host);
+    }
   }
   L.total = align_up(L.arena_off + L.arena + 64, 256);
   return MAO_OK;
 }
 
-mao_status run_step(const Ctx& X, void* workspace, size_t ws_bytes, mao_stats* stats, cudaStream_t s) {
-  std::vector<GroupPlan> groups;
-  Layout L;
-  MAO_TRY(layout_for(X, groups, L));
-  if (workspace == nullptr || ws_bytes < L.total) return MAO_ERR_WORKSPACE;
+// Recently used plans, keyed by the exact bytes of everything they depend on
+// (descriptor array, hyper-parameters, refresh mode, workspace).  A training loop
+// that calls the step with the same buffers every iteration builds its plan
+// (tables, tensor maps) once per refresh mode.
+struct PlanCache {
+  std::mutex mu;
+  std::list<std::pair<std::string, std::shared_ptr<StepPlan>>> lru;
+  static constexpr size_t kMax = 8;
+};
+PlanCache& plan_cache() {
+  static PlanCache c;
+  return c;
+}
+
+std::string plan_key(const Ctx& X, const void* mats, size_t mats_bytes, const void* ws, size_t ws_bytes) {
+  struct Head {
+    int foam, count, mode, raw_trace;
+    float b1, b2, eps, lr, wd;
+    mao_refresh rf;
+    const void* ws;
+    size_t ws_bytes;
+  } h;
+  std::memset(&h, 0, sizeof(h));
+  h.foam = X.foam;
+  h.count = X.count;
+  h.mode = X.mode;
+  h.raw_trace = X.raw_trace;
+  h.b1 = X.b1;
+  h.b2 = X.b2;
+  h.eps = X.eps;
+  h.lr = X.lr;
+  h.wd = X.wd;
+  h.rf = X.rf;
+  h.ws = ws;
+  h.ws_bytes = ws_bytes;
+  std::string k(reinterpret_cast<const char*>(&h), sizeof(h));
+  k.append(reinterpret_cast<const char*>(mats), mats_bytes);
+  return k;
+}
+
+mao_status run_step(const Ctx& X, const void* mats, size_t mats_bytes, void* workspace, size_t ws_bytes,
+                    mao_stats* stats, cudaStream_t s) {
+  if (workspace == nullptr) return MAO_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MAO_ERR_ALIGN;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const std::string key = plan_key(X, mats, mats_bytes, workspace, ws_bytes);
+  std::shared_ptr<StepPlan> P;
+  {
+    PlanCache& C = plan_cache();
+    std::lock_guard<std::mutex> lk(C.mu);
+    for (auto it = C.lru.begin(); it != C.lru.end(); ++it)
+      if (it->first == key) {
+        P = it->second;
+        C.lru.splice(C.lru.begin(), C.lru, it);
+        break;
+      }
+  }
+  if (!P) {
+    StepPlan sizing;
+    MAO_TRY(make_plan(X, nullptr, sizing));
+    if (ws_bytes < sizing.L.total) return MAO_ERR_WORKSPACE;
+    P = std::make_shared<StepPlan>();
+    MAO_TRY(make_plan(X, ws, *P));
+    if (P->L.total != sizing.L.total) return MAO_ERR_WORKSPACE;
+    PlanCache& C = plan_cache();
+    std::lock_guard<std::mutex> lk(C.mu);
+    C.lru.emplace_front(key, P);
+    if (C.lru.size() > PlanCache::kMax) C.lru.pop_back();
+  }
   DeviceInfo* dev = nullptr;
   MAO_TRY(device_info(&dev));
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
   DevStatus* status = reinterpret_cast<DevStatus*>(ws);
   MAO_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(DevStatus), s));
-  for (GroupPlan& g : groups) {
-    Builder B(X, ws);
-    B.arena.dev = ws + L.arena_off;
-    MAO_TRY(build_group(B, g));
-    BuiltGroup bg;
-    MAO_TRY(finish_build(B, bg));
-    if (B.arena.host.size() > L.arena) return MAO_ERR_WORKSPACE;
-    // refresh flags (adaptive) and failure counters start at zero
-    for (int i = 0; i < g.g1 - g.g0; ++i) {
-      for (int side = 0; side < 2; ++side) {
-        if (X.foam && side == 0) continue;
-        const SideBuf& sb = side == 0 ? g.mb[i].L : g.mb[i].R;
-        MAO_CUDA_TRY(cudaMemsetAsync(ws + sb.flag, 0, 48, s));  // flag, rho, bad
-      }
-    }
-    MAO_CUDA_TRY(cudaMemcpyAsync(B.arena.dev, B.arena.host.data(), B.arena.host.size(), cudaMemcpyHostToDevice, s));
-    MAO_TRY(run_ops(B, bg, status, s));
+  uint8_t* arena_dev = ws + P->L.arena_off;
+  for (size_t gi = 0; gi < P->groups.size(); ++gi) {
+    const GroupPlan& g = P->groups[gi];
+    const BuiltGroup& bg = P->built[gi];
+    // refresh flags, check ratios and failure counters start at zero
+    MAO_CUDA_TRY(cudaMemsetAsync(ws + g.flags, 0, g.flags_bytes, s));
+    MAO_CUDA_TRY(cudaMemcpyAsync(arena_dev, bg.arena.data(), bg.arena.size(), cudaMemcpyHostToDevice, s));
+    MAO_TRY(run_ops(X, arena_dev, bg, status, s));
     if (stats) {
-      for (int i = 0; i < g.g1 - g.g0; ++i) {
-        mao_stats* st = stats + g.g0 + i;
-        const SideBuf& R = g.mb[i].R;
-        const SideBuf* Lb = X.foam ? nullptr : &g.mb[i].L;
-        if (X.mode == 2) {
-          pc_stats_kernel<<<1, 32, 0, s>>>(st, reinterpret_cast<const int*>(ws + R.flag),
-                                          Lb ? reinterpret_cast<const int*>(ws + Lb->flag) : nullptr,
-                                          reinterpret_cast<const float*>(ws + R.rho), -1);
-        } else {
-          pc_stats_kernel<<<1, 32, 0, s>>>(st, nullptr, nullptr, nullptr, X.mode == 1 ? (X.foam ? 1 : 3) : 0);
-        }
-        MAO_CUDA_TRY(cudaGetLastError());
-      }
+      const int nm = g.g1 - g.g0;
+      pc_stats_kernel<<<(nm + 127) / 128, 128, 0, s>>>(reinterpret_cast<const StatsJob*>(arena_dev + bg.stats_jobs),
+                                                         nm, stats);
+      MAO_CUDA_TRY(cudaGetLastError());
     }
   }
+  return MAO_OK;
+}
+
+mao_status workspace_size(const Ctx& X, size_t* bytes) {
+  StepPlan sizing;
+  MAO_TRY(make_plan(X, nullptr, sizing));
+  *bytes = sizing.L.total;
   return MAO_OK;
 }
 
@@ -1002,11 +1104,7 @@ extern "C" mao_status mao_soap_workspace_size(const mao_soap_mat* mats, int32_t 
   std::vector<PcMat> v;
   Ctx X;
   MAO_TRY(soap_ctx(mats, count, p, v, X, false));
-  std::vector<GroupPlan> groups;
-  Layout L;
-  MAO_TRY(layout_for(X, groups, L));
-  *bytes = L.total;
-  return MAO_OK;
+  return workspace_size(X, bytes);
 }
 
 extern "C" mao_status mao_soap_step(const mao_soap_mat* mats, int32_t count, const mao_soap_params* p,
@@ -1016,7 +1114,8 @@ extern "C" mao_status mao_soap_step(const mao_soap_mat* mats, int32_t count, con
   MAO_TRY(soap_ctx(mats, count, p, v, X, true));
   if (count == 0) return MAO_OK;
   if (stats != nullptr && !aligned16(stats)) return MAO_ERR_ALIGN;
-  return run_step(X, workspace, ws_bytes, stats, reinterpret_cast<cudaStream_t>(stream));
+  return run_step(X, mats, sizeof(mao_soap_mat) * (size_t)count, workspace, ws_bytes, stats,
+                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" mao_status mao_foam_workspace_size(const mao_foam_mat* mats, int32_t count, const mao_foam_params* p,
@@ -1025,11 +1124,7 @@ extern "C" mao_status mao_foam_workspace_size(const mao_foam_mat* mats, int32_t 
   std::vector<PcMat> v;
   Ctx X;
   MAO_TRY(foam_ctx(mats, count, p, v, X, false));
-  std::vector<GroupPlan> groups;
-  Layout L;
-  MAO_TRY(layout_for(X, groups, L));
-  *bytes = L.total;
-  return MAO_OK;
+  return workspace_size(X, bytes);
 }
 
 extern "C" mao_status mao_foam_step(const mao_foam_mat* mats, int32_t count, const mao_foam_params* p,
@@ -1039,5 +1134,6 @@ extern "C" mao_status mao_foam_step(const mao_foam_mat* mats, int32_t count, con
   MAO_TRY(foam_ctx(mats, count, p, v, X, true));
   if (count == 0) return MAO_OK;
   if (stats != nullptr && !aligned16(stats)) return MAO_ERR_ALIGN;
-  return run_step(X, workspace, ws_bytes, stats, reinterpret_cast<cudaStream_t>(stream));
+  return run_step(X, mats, sizeof(mao_foam_mat) * (size_t)count, workspace, ws_bytes, stats,
+                  reinterpret_cast<cudaStream_t>(stream));
 }
