@@ -38,6 +38,8 @@ WORKLOADS = {
     # name: (description, optimizers run per step, default gradient dtype bf16?)
     "dense8b_moe": ("8B-dense block (7 matrices) + 256-expert MoE bank (768 matrices), bf16 G ~ N(0,0.01^2)*s_e",
                     True),
+    "dense8b_block": ("8B-dense block alone (7 matrices), bf16 G ~ N(0,0.01^2)", True),
+    "moe_bank": ("256-expert MoE bank alone (768 matrices), bf16 G ~ N(0,0.01^2)*s_e", True),
     "gpt2_124m": ("GPT-2-124M-shaped set, 48 matrices, bf16 G ~ N(0,0.02^2), Muon+ Col-Row", True),
     "gpt2_760m": ("GPT-2-760M-shaped set, 96 matrices, fp32 G ~ N(0,0.01^2)", False),
     "muon_single": ("one 256x512 fp32 weight", False),

@@ -212,7 +212,9 @@ typedef struct {
  *   U = Q_L N Q_R^T ; W <- W (1 - lr wd) - lr U
  * Contractions use fp32-faithful tensor-core arithmetic: every fp32 operand is
  * held as three bf16 planes and the six significant cross products accumulate
- * in fp32.
+ * in fp32 (a bf16 G is exact in one plane: G G^T is one product, Q_L^T G three).
+ * The workspace size depends on the descriptors and on the refresh policy but
+ * not on t: one workspace serves every step of the descriptor set.
  */
 MAO_API mao_status mao_soap_workspace_size(const mao_soap_mat* mats, int32_t count, const mao_soap_params* p,
                                    size_t* bytes);
@@ -251,6 +253,7 @@ typedef struct {
  *   r <- b2 r + (1-b2) rowmean(Gr^2) ; c <- b2 c + (1-b2) colmean(Gr^2)
  *   tau = tr(R^) / (|r^|_1 |c^|_1) ; v_ij = tau r^_i c^_j (never materialised)
  *   N = (Mr / (1-b1^t)) / (sqrt(v) + eps) ; U = N Q_R^T ; W <- W (1 - lr wd) - lr U
+ * Arithmetic and workspace as for mao_soap_step.
  */
 MAO_API mao_status mao_foam_workspace_size(const mao_foam_mat* mats, int32_t count, const mao_foam_params* p,
                                    size_t* bytes);
@@ -296,9 +299,11 @@ typedef enum {
   MAO_K_PC_CHECK = 15,       /* adaptive check D = Q^T F Q and its ratio */
   MAO_K_PC_POWER = 16,       /* power step P = F Q */
   MAO_K_PC_SORT = 17,        /* sort keys, argsort, gathers */
-  MAO_K_PC_QR = 18,          /* QR panels: projections, Gram, Cholesky, apply */
+  MAO_K_PC_QR = 18,          /* QR tensor-core products: panel projections, W R^{-1} */
   MAO_K_PC_ROTATE = 19,      /* rotations into the eigenbasis and back (before the update) */
-  MAO_K_PC_UPDATE = 20       /* last rotation fused with the weight update */
+  MAO_K_PC_UPDATE = 20,      /* last rotation fused with the weight update */
+  MAO_K_PC_PANEL = 21,       /* QR panel Gram products (tensor cores, K slices) */
+  MAO_K_PC_CHOL = 22         /* QR panel Cholesky and R^{-1} (fp64, one block per matrix) */
 } mao_kernel_id;
 
 /* What one recorded launch was: its kernel and its algorithmic work (useful

@@ -14,14 +14,31 @@
 extern "C" {
 #endif
 
-typedef enum { MAO_GEMM_BF16 = 0, MAO_GEMM_SPLIT3 = 1 } mao_gemm_kind;
+typedef enum {
+  MAO_GEMM_BF16 = 0,
+  MAO_GEMM_SPLIT3 = 1,
+  MAO_GEMM_BF16_FOLD = 2,
+  MAO_GEMM_SPLIT3_BF16 = 3,
+  MAO_GEMM_BF16_SPLIT3 = 4,
+  MAO_GEMM_SPLIT2 = 5
+} mao_gemm_kind;
 
 /*
  * D[b] = A[b] * B[b]^T for b < batch, with fp32 accumulation and fp32 D.
- *   kind MAO_GEMM_BF16:   A, B bf16; one bf16 tensor-core product.
+ *   kind MAO_GEMM_BF16:   A, B bf16; one bf16 tensor-core product, accumulated
+ *                         over the whole K in the tensor memory (the Newton-Schulz
+ *                         kernels' core).
  *   kind MAO_GEMM_SPLIT3: A, B fp32; each split into three bf16 planes
  *                         x = x0 + x1 + x2 and the six significant cross
  *                         products accumulated in fp32 (fp32-faithful).
+ *   kind MAO_GEMM_BF16_FOLD:   A, B bf16; the exact bf16 product with partial
+ *                         sums over 256 of K folded in fp32 registers (the
+ *                         SOAP/FOAM factor products of a bf16 gradient).
+ *   kind MAO_GEMM_SPLIT3_BF16: A fp32 (three planes), B bf16 (one plane): three
+ *                         products, fp32-faithful.
+ *   kind MAO_GEMM_BF16_SPLIT3: A bf16, B fp32: the mirror of the previous kind.
+ *   kind MAO_GEMM_SPLIT2: A, B fp32 held as two bf16 planes each, products
+ *                         x0 y0 + x0 y1 + x1 y0 (about 16 significant bits).
  * Layouts (row-major, contiguous batches):
  *   a_mn_major = 0: A is [batch][M][K]; 1: A is [batch][K][M]
  *   b_mn_major = 0: B is [batch][N][K]; 1: B is [batch][K][N]

@@ -132,11 +132,17 @@ def gemm(A: torch.Tensor, B: torch.Tensor, *, kind: str = "bf16", a_mn_major: bo
     """Verification entry: D[b] = A[b] @ B[b]^T through the tensor-core GEMM core.
 
     A is (batch, M, K) (or (batch, K, M) when a_mn_major); B is (batch, N, K)
-    (or (batch, K, N) when b_mn_major).  kind "bf16" (bf16 operands) or
-    "split3" (fp32 operands held as three bf16 planes, fp32-faithful).  Returns fp32 (batch, M, N).
+    (or (batch, K, N) when b_mn_major).  Kinds:
+      "bf16"        bf16 operands, accumulated over all of K in the tensor memory;
+      "split3"      fp32 operands held as three bf16 planes, fp32-faithful;
+      "bf16_fold"   bf16 operands, partial sums over 256 of K folded in fp32;
+      "split3_bf16" fp32 A (three planes) times bf16 B;
+      "bf16_split3" bf16 A times fp32 B (three planes);
+      "split2"      fp32 operands held as two bf16 planes each, three products.
+    Returns fp32 (batch, M, N).
     """
     lib = L.load()
-    k = {"bf16": 0, "split3": 1}[kind]
+    k = {"bf16": 0, "split3": 1, "bf16_fold": 2, "split3_bf16": 3, "bf16_split3": 4, "split2": 5}[kind]
     batch = A.shape[0]
     M = A.shape[2] if a_mn_major else A.shape[1]
     K = A.shape[1] if a_mn_major else A.shape[2]

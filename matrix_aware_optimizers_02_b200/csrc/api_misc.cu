@@ -62,12 +62,24 @@ struct TestLayout {
   size_t total = 0;
 };
 
+// planes of A and B for a table-mode kind (0 for the class-mode bf16 kind)
+void kind_planes(int32_t kind, int* pa, int* pb) {
+  switch (kind) {
+    case MAO_GEMM_SPLIT3: *pa = 3; *pb = 3; return;
+    case MAO_GEMM_BF16_FOLD: *pa = 1; *pb = 1; return;
+    case MAO_GEMM_SPLIT3_BF16: *pa = 3; *pb = 1; return;
+    case MAO_GEMM_BF16_SPLIT3: *pa = 1; *pb = 3; return;
+    case MAO_GEMM_SPLIT2: *pa = 2; *pb = 2; return;
+    default: *pa = 0; *pb = 0; return;
+  }
+}
+
 mao_status gemm_layout(int32_t kind, int32_t batch, int32_t M, int32_t N, int32_t K, TestLayout& T) {
   if (batch < 1 || M < 1 || N < 1 || K < 1) return MAO_ERR_SHAPE;
-  if (kind != MAO_GEMM_BF16 && kind != MAO_GEMM_SPLIT3) return MAO_ERR_INVALID_ARG;
+  if (kind < MAO_GEMM_BF16 || kind > MAO_GEMM_SPLIT2) return MAO_ERR_INVALID_ARG;
   Carver cv;
   cv.take(kStatusBytes);
-  if (kind == MAO_GEMM_SPLIT3) {
+  if (kind != MAO_GEMM_BF16) {
     T.planes[0] = cv.take(3 * 2 * (size_t)batch * M * K);
     T.planes[1] = cv.take(3 * 2 * (size_t)batch * N * K);
     // per batch element: one problem and six descriptors
@@ -132,23 +144,32 @@ extern "C" mao_status mao_test_gemm(int32_t kind, int32_t a_mn_major, int32_t b_
     return launch_gemm(OP_BF16, a_mn_major, b_mn_major, EPI_STORE_F32, p, stream, MAO_K_GEMM_TEST);
   }
 
-  // SPLIT3: three bf16 planes of each operand, then one table-mode problem per batch element
+  // table mode: the fp32 operands split into bf16 planes (a bf16 operand is its
+  // own single plane), then one problem per batch element
+  int pa = 0, pb = 0;
+  kind_planes(kind, &pa, &pb);
   const size_t an = (size_t)batch * M * K, bn = (size_t)batch * N * K;
   __nv_bfloat16* ap = reinterpret_cast<__nv_bfloat16*>(ws + T.planes[0]);
   __nv_bfloat16* bp = reinterpret_cast<__nv_bfloat16*>(ws + T.planes[1]);
-  MAO_TRY(launch_split3(static_cast<const float*>(A), ap, ap + an, ap + 2 * an, an, stream));
-  MAO_TRY(launch_split3(static_cast<const float*>(B), bp, bp + bn, bp + 2 * bn, bn, stream));
+  if (pa > 1) MAO_TRY(launch_split3(static_cast<const float*>(A), ap, ap + an, ap + 2 * an, an, stream));
+  if (pb > 1) MAO_TRY(launch_split3(static_cast<const float*>(B), bp, bp + bn, bp + 2 * bn, bn, stream));
+  const __nv_bfloat16* a0 = pa > 1 ? ap : static_cast<const __nv_bfloat16*>(A);
+  const __nv_bfloat16* b0 = pb > 1 ? bp : static_cast<const __nv_bfloat16*>(B);
   Arena arena;
   arena.dev = ws + T.arena;
   MapSet maps;
   TableLaunch L;
   L.a_mn = a_mn_major;
   L.b_mn = b_mn_major;
+  L.pa = pa;
+  L.pb = pb;
   L.kernel_id = MAO_K_GEMM_TEST;
   for (int b = 0; b < batch; ++b) {
     const size_t ao = (size_t)b * M * K, bo = (size_t)b * N * K;
-    const Split3 As{{ap + ao, ap + an + ao, ap + 2 * an + ao}, a_rows, a_inner, a_inner};
-    const Split3 Bs{{bp + bo, bp + bn + bo, bp + 2 * bn + bo}, b_rows, b_inner, b_inner};
+    Split3 As{{a0 + ao, nullptr, nullptr}, a_rows, a_inner, a_inner};
+    Split3 Bs{{b0 + bo, nullptr, nullptr}, b_rows, b_inner, b_inner};
+    for (int q = 1; q < pa; ++q) As.p[q] = ap + q * an + ao;
+    for (int q = 1; q < pb; ++q) Bs.p[q] = bp + q * bn + bo;
     MAO_TRY(table_add(L, maps, As, Bs, M, N, K, 0, 0, D + (size_t)b * M * N, nullptr, N, nullptr, 0, 1.f, 0.f,
                       nullptr));
   }

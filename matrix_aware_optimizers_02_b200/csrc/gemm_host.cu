@@ -106,7 +106,7 @@ mao_status launch_one(const GemmParams& p, cudaStream_t stream, int kernel_id) {
   for (int c = 0; c < p.nclasses; ++c) {
     const GemmClass& C = p.cls[c];
     flops += 2.0 * C.count * (double)C.M * C.N * C.K;
-    bytes += C.count * (es * ((double)C.M * C.K + (double)C.N * C.K) * Cfg::PLANES + ob * (double)C.M * C.N *
+    bytes += C.count * (es * ((double)C.M * C.K + (double)C.N * C.K) + ob * (double)C.M * C.N *
                                                                                          (EPI == EPI_AXPY_T ? 2 : 1) +
                         ((EPI == EPI_POLY || EPI == EPI_AXPY_T) ? 2.0 * C.M * C.N : 0.0));
   }
@@ -200,16 +200,21 @@ mao_status MapSet::encode_all() {
 
 mao_status table_add(TableLaunch& L, MapSet& maps, const Split3& A, const Split3& B, int M, int N, int K,
                      int m_off, int n_off, float* out, const Split3* outp, int ld_out, const float* aux,
-                     int ld_aux, float alpha, float beta, const int* flag) {
+                     int ld_aux, float alpha, float beta, const int* flag, int k_off) {
   if (M <= 0 || N <= 0 || K <= 0) return MAO_OK;
   if ((L.a_mn && (m_off & 7)) || (L.b_mn && (n_off & 7))) return MAO_ERR_INVALID_ARG;
+  if (k_off < 0 || ((!L.a_mn || !L.b_mn) && (k_off & 7))) return MAO_ERR_INVALID_ARG;
   if ((A.ld & 7) || (B.ld & 7)) return MAO_ERR_SHAPE;
+  for (int q = 0; q < L.pa; ++q)
+    if (A.p[q] == nullptr) return MAO_ERR_INVALID_ARG;
+  for (int q = 0; q < L.pb; ++q)
+    if (B.p[q] == nullptr) return MAO_ERR_INVALID_ARG;
   // operand views: inner extent = the stored matrix's columns, rows = its rows
   const int abox = L.a_mn ? 64 : 128, bbox = L.b_mn ? 64 : 128;
   int idx[6];
   for (int q = 0; q < 3; ++q) {
-    idx[q] = maps.get(A.p[q], A.cols, A.rows, A.ld, abox, L.a_mn);
-    idx[3 + q] = maps.get(B.p[q], B.cols, B.rows, B.ld, bbox, L.b_mn);
+    idx[q] = q < L.pa ? maps.get(A.p[q], A.cols, A.rows, A.ld, abox, L.a_mn) : -1;
+    idx[3 + q] = q < L.pb ? maps.get(B.p[q], B.cols, B.rows, B.ld, bbox, L.b_mn) : -1;
   }
   GemmProblem P;
   std::memset(&P, 0, sizeof(P));
@@ -226,6 +231,7 @@ mao_status table_add(TableLaunch& L, MapSet& maps, const Split3& A, const Split3
   P.K = K;
   P.m_off = m_off;
   P.n_off = n_off;
+  P.k_off = k_off;
   P.ld_out = ld_out;
   P.ld_aux = ld_aux;
   P.tiles_n = (N + 127) / 128;
@@ -241,6 +247,8 @@ StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off) {
   S.nprob = (int)L.probs.size();
   S.a_mn = L.a_mn;
   S.b_mn = L.b_mn;
+  S.pa = L.pa;
+  S.pb = L.pb;
   S.kernel_id = L.kernel_id;
   if (S.nprob == 0) return S;
   S.probs_off = A.take(sizeof(GemmProblem) * S.nprob, 64);
@@ -250,8 +258,9 @@ StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off) {
   for (int i = 0; i < S.nprob; ++i) {
     GemmProblem P = L.probs[i];
     for (int q = 0; q < 3; ++q) {
-      P.mapA[q] = mbase ? mbase + L.map_idx[6 * i + q] : nullptr;
-      P.mapB[q] = mbase ? mbase + L.map_idx[6 * i + 3 + q] : nullptr;
+      const int ia = L.map_idx[6 * i + q], ib = L.map_idx[6 * i + 3 + q];
+      P.mapA[q] = (mbase && ia >= 0) ? mbase + ia : nullptr;
+      P.mapB[q] = (mbase && ib >= 0) ? mbase + ib : nullptr;
     }
     P.tile_begin = t;
     t += ((P.M + 127) / 128) * P.tiles_n;
@@ -262,29 +271,6 @@ StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off) {
   return S;
 }
 
-namespace {
-template <int A_MN, int B_MN>
-mao_status launch_table_one(const GemmTableParams& p, cudaStream_t stream, int kernel_id, double flops) {
-  using Cfg = GemmCfg<OP_SPLIT3, A_MN, B_MN>;
-  DeviceInfo* d = nullptr;
-  MAO_TRY(device_info(&d));
-  auto kern = gemm_tc_table_kernel<OP_SPLIT3, A_MN, B_MN>;
-  const int slot = 40 + A_MN * 2 + B_MN;
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!d->gemm_attr_set[slot]) {
-      MAO_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
-      d->gemm_attr_set[slot] = true;
-    }
-  }
-  if (p.total_tiles <= 0) return MAO_OK;
-  const int grid = p.total_tiles < d->sm_count ? p.total_tiles : d->sm_count;
-  LaunchScope ls(stream, kernel_id, flops, 0.0);
-  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? MAO_OK : MAO_ERR_CUDA;
-}
-}  // namespace
-
 mao_status table_launch(const Arena& A, const StagedLaunch& S, DevStatus* status, cudaStream_t stream) {
   if (S.nprob == 0) return MAO_OK;
   GemmTableParams p;
@@ -292,10 +278,15 @@ mao_status table_launch(const Arena& A, const StagedLaunch& S, DevStatus* status
   p.nprob = S.nprob;
   p.total_tiles = S.total_tiles;
   p.status = status;
-  if (!S.a_mn && !S.b_mn) return launch_table_one<0, 0>(p, stream, S.kernel_id, S.flops);
-  if (!S.a_mn && S.b_mn) return launch_table_one<0, 1>(p, stream, S.kernel_id, S.flops);
-  if (S.a_mn && !S.b_mn) return launch_table_one<1, 0>(p, stream, S.kernel_id, S.flops);
-  return launch_table_one<1, 1>(p, stream, S.kernel_id, S.flops);
+  const int key = S.pa * 10 + S.pb;
+  switch (key) {
+    case 33: return launch_table_planes<3, 3>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops);
+    case 31: return launch_table_planes<3, 1>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops);
+    case 13: return launch_table_planes<1, 3>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops);
+    case 11: return launch_table_planes<1, 1>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops);
+    case 22: return launch_table_planes<2, 2>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops);
+    default: return MAO_ERR_INVALID_ARG;
+  }
 }
 
 }  // namespace mao

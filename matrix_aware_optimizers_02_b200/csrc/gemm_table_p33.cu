@@ -1,0 +1,6 @@
+// Table-mode GEMM kernels with 3 plane(s) of A and 3 plane(s) of B.
+#include "gemm_table.cuh"
+
+namespace mao {
+template mao_status launch_table_planes<3, 3>(const GemmTableParams&, int, int, cudaStream_t, int, double);
+}  // namespace mao

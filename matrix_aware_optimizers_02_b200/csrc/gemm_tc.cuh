@@ -97,6 +97,7 @@ struct GemmProblem {
   const int* flag;             // nullptr, or skip this problem when *flag == 0
   int M, N, K;
   int m_off, n_off;            // operand coordinates of output row/column 0 (sub-block views)
+  int k_off;                   // operand coordinate of K index 0 (a K slice; multiple of 8 for K-major operands)
   int ld_out, ld_aux, ld_outp;
   int tiles_n, tile_begin;
   float alpha, beta;
@@ -109,22 +110,28 @@ struct GemmTableParams {
   DevStatus* status;
 };
 
-template <int KIND, int A_MN, int B_MN>
+// PA / PB: bf16 planes held per operand (SPLIT3 kinds only; 1 = a plain bf16
+// operand, exact in one plane).  The products taken are the pairs (i, j), i < PA,
+// j < PB, with i + j <= max(PA, PB) - 1: all six terms at or above the fp32 unit
+// roundoff for (3, 3), x_i y_0 for (3, 1), the single exact product for (1, 1).
+template <int KIND, int A_MN, int B_MN, int PA = (KIND == OP_BF16 ? 1 : 3), int PB = PA>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BN = (KIND == OP_BF16) ? 256 : 128;
   static constexpr int ESIZE = 2;                      // bf16 planes
   static constexpr int BK = 64;                        // elements per 128-byte row
   static constexpr int UMMA_K = 16;                    // 32 bytes of K per MMA
-  static constexpr int PLANES = (KIND == OP_BF16) ? 1 : 3;
   static constexpr int A_TILE = BM * 128;              // bytes per plane
   static constexpr int B_TILE = BN * 128;
-  static constexpr int STAGE_BYTES = PLANES * (A_TILE + B_TILE);
-  static constexpr int STAGES = (KIND == OP_BF16) ? 4 : 2;
+  static constexpr int STAGE_BYTES = PA * A_TILE + PB * B_TILE;
+  static constexpr int STAGES_FIT = (200 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = (KIND == OP_BF16) ? 4 : (STAGES_FIT > 6 ? 6 : STAGES_FIT);
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
-  static constexpr int ACC_COLS = (KIND == OP_BF16) ? BN : 2 * BN;  // main (+ correction) accumulator
+  static constexpr int PMAX = (PA > PB ? PA : PB) - 1;  // largest i + j taken
+  static constexpr bool CORR = (PA > 1 || PB > 1);       // any cross product
+  static constexpr int ACC_COLS = CORR ? 2 * BN : BN;    // main (+ correction) accumulator
   static constexpr int KCH = 4;  // SPLIT3: k-blocks (4 x 64 = 256 of K) per TMEM accumulation item
-  static constexpr int TMEM_COLS = 2 * ACC_COLS;                   // double-buffered
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;         // double-buffered
   static constexpr uint32_t IDESC = make_idesc(1u, A_MN, B_MN, BM, BN);
   static constexpr int THREADS = 192;
 };
@@ -198,6 +205,7 @@ struct TileInfo {
   int K;
   bool valid;  // false: the tile's problem is gated off
   int am, bn;  // operand coordinate offsets along M (A) and N (B)
+  int ko;      // operand coordinate offset along K
 };
 
 // ------------------------------------------------------------------ class mode
@@ -232,6 +240,7 @@ struct ClassSource {
     t.valid = true;
     t.am = 0;
     t.bn = 0;
+    t.ko = 0;
     return t;
   }
   __device__ int cols(const TileInfo& t) const { return p.cls[t.idx].N; }
@@ -329,6 +338,7 @@ struct TableSource {
     t.valid = (P.flag == nullptr) || (*P.flag != 0);
     t.am = P.m_off;
     t.bn = P.n_off;
+    t.ko = P.k_off;
     return t;
   }
   __device__ int cols(const TileInfo& t) const { return p.probs[t.idx].N; }
@@ -392,9 +402,9 @@ struct TableSource {
 };
 
 // ------------------------------------------------------------------ kernel body
-template <int KIND, int A_MN, int B_MN, int EPI, class Src>
+template <int KIND, int A_MN, int B_MN, int EPI, class Src, int PA = (KIND == OP_BF16 ? 1 : 3), int PB = PA>
 __device__ __forceinline__ void gemm_body(const Src& src) {
-  using Cfg = GemmCfg<KIND, A_MN, B_MN>;
+  using Cfg = GemmCfg<KIND, A_MN, B_MN, PA, PB>;
   constexpr int BM = Cfg::BM, BN = Cfg::BN, BK = Cfg::BK, STAGES = Cfg::STAGES;
 
   extern __shared__ uint8_t smem_raw[];
@@ -451,10 +461,9 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
         if (!t.valid) continue;
         if constexpr (EPI == EPI_TABLE) {
 #pragma unroll
-          for (int q = 0; q < Cfg::PLANES; ++q) {
-            tensormap_acquire(t.mapA[q]);
-            tensormap_acquire(t.mapB[q]);
-          }
+          for (int q = 0; q < PA; ++q) tensormap_acquire(t.mapA[q]);
+#pragma unroll
+          for (int q = 0; q < PB; ++q) tensormap_acquire(t.mapB[q]);
         }
         const int nk = (t.K + BK - 1) / BK;
         bool ok = true;
@@ -467,14 +476,15 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
           }
           uint8_t* st = smem + s * Cfg::STAGE_BYTES;
           mbar_arrive_expect_tx(&full_bar[s], Cfg::STAGE_BYTES);
-          const int am = t.am + t.m0, bn = t.bn + t.n0;
+          const int am = t.am + t.m0, bn = t.bn + t.n0, kc = t.ko + kb * BK;
           // stage layout: A planes, then B planes
 #pragma unroll
-          for (int q = 0; q < Cfg::PLANES; ++q) {
-            load_operand<A_MN, BM, Cfg::ESIZE>(st + q * Cfg::A_TILE, t.mapA[q], &full_bar[s], kb * BK, am, t.b);
-            load_operand<B_MN, BN, Cfg::ESIZE>(st + Cfg::PLANES * Cfg::A_TILE + q * Cfg::B_TILE, t.mapB[q],
-                                               &full_bar[s], kb * BK, bn, t.b);
-          }
+          for (int q = 0; q < PA; ++q)
+            load_operand<A_MN, BM, Cfg::ESIZE>(st + q * Cfg::A_TILE, t.mapA[q], &full_bar[s], kc, am, t.b);
+#pragma unroll
+          for (int q = 0; q < PB; ++q)
+            load_operand<B_MN, BN, Cfg::ESIZE>(st + PA * Cfg::A_TILE + q * Cfg::B_TILE, t.mapB[q], &full_bar[s], kc,
+                                               bn, t.b);
         }
         if (!ok) break;
       }
@@ -513,7 +523,7 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
             }
             tc_fence_after();
             const uint32_t a_base = smem_u32(smem + s * Cfg::STAGE_BYTES);
-            const uint32_t b_base = a_base + Cfg::PLANES * Cfg::A_TILE;
+            const uint32_t b_base = a_base + PA * Cfg::A_TILE;
 #pragma unroll
             for (int k = 0; k < BK / Cfg::UMMA_K; ++k) {
               const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
@@ -525,11 +535,16 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
                 // the main product into its own
                 constexpr int pa[5] = {1, 0, 2, 0, 1};
                 constexpr int pb[5] = {1, 2, 0, 1, 0};
+                bool first = true;
 #pragma unroll
-                for (int q = 0; q < 5; ++q)
-                  umma_f16(d_tmem + BN, operand_desc<A_MN, BM, Cfg::ESIZE>(a_base + pa[q] * Cfg::A_TILE, k),
-                           operand_desc<B_MN, BN, Cfg::ESIZE>(b_base + pb[q] * Cfg::B_TILE, k), Cfg::IDESC,
-                           q == 0 ? accum : 1u);
+                for (int q = 0; q < 5; ++q) {
+                  if (pa[q] < PA && pb[q] < PB && pa[q] + pb[q] <= Cfg::PMAX) {
+                    umma_f16(d_tmem + BN, operand_desc<A_MN, BM, Cfg::ESIZE>(a_base + pa[q] * Cfg::A_TILE, k),
+                             operand_desc<B_MN, BN, Cfg::ESIZE>(b_base + pb[q] * Cfg::B_TILE, k), Cfg::IDESC,
+                             first ? accum : 1u);
+                    first = false;
+                  }
+                }
                 umma_f16(d_tmem, operand_desc<A_MN, BM, Cfg::ESIZE>(a_base, k),
                          operand_desc<B_MN, BN, Cfg::ESIZE>(b_base, k), Cfg::IDESC, accum);
               }
@@ -599,12 +614,19 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
           const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS;
 #pragma unroll
           for (int ch = 0; ch < BN / 32; ++ch) {
-            uint32_t rm[32], rc[32];
+            uint32_t rm[32];
             tmem_ld_32x32b_x32(tacc + ch * 32, rm);
-            tmem_ld_32x32b_x32(tacc + BN + ch * 32, rc);
-            tmem_wait_ld();
+            if constexpr (Cfg::CORR) {
+              uint32_t rc[32];
+              tmem_ld_32x32b_x32(tacc + BN + ch * 32, rc);
+              tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) run[ch * 32 + j] += __uint_as_float(rm[j]) + __uint_as_float(rc[j]);
+              for (int j = 0; j < 32; ++j) run[ch * 32 + j] += __uint_as_float(rm[j]) + __uint_as_float(rc[j]);
+            } else {
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) run[ch * 32 + j] += __uint_as_float(rm[j]);
+            }
           }
           tc_fence_before();
           mbar_arrive(&tempty_bar[acc]);
@@ -638,10 +660,10 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   gemm_body<KIND, A_MN, B_MN, EPI>(src);
 }
 
-template <int KIND, int A_MN, int B_MN>
+template <int A_MN, int B_MN, int PA, int PB>
 __global__ void __launch_bounds__(192, 1) gemm_tc_table_kernel(const __grid_constant__ GemmTableParams p) {
   TableSource src(p);
-  gemm_body<KIND, A_MN, B_MN, EPI_TABLE>(src);
+  gemm_body<OP_SPLIT3, A_MN, B_MN, EPI_TABLE, TableSource, PA, PB>(src);
 }
 
 }  // namespace mao

@@ -143,7 +143,8 @@ struct Arena {
 };
 
 // An fp32 row-major matrix held as three bf16 planes x = p0 + p1 + p2 (operand
-// of an fp32-faithful SPLIT3 product); ld in elements, a multiple of 8.
+// of an fp32-faithful SPLIT3 product); ld in elements, a multiple of 8.  A bf16
+// matrix is its own single plane (p[1] = p[2] = nullptr).
 struct Split3 {
   const __nv_bfloat16* p[3];
   int rows, cols, ld;
@@ -153,8 +154,13 @@ struct Split3 {
 //   out (M x N) = alpha * op(A) op(B) + beta * aux
 // with op(A) = A (a_mn = 0, A stored M x K) or A^T (a_mn = 1, A stored K x M), and
 // op(B) = B^T (b_mn = 0, B stored N x K) or B (b_mn = 1, B stored K x N).
+//
+// pa / pb: planes used per operand (1: a bf16 operand, exact in one plane; 3: an
+// fp32 operand; 2: a 16-bit-significand approximation).  Every problem of a
+// launch uses the same counts.
 struct TableLaunch {
   int a_mn = 0, b_mn = 0;
+  int pa = 3, pb = 3;
   int kernel_id = 0;
   std::vector<GemmProblem> probs;
   std::vector<int> map_idx;  // 6 per problem: A planes 0..2, B planes 0..2 (indices into the step's map list)
@@ -187,11 +193,13 @@ struct MapSet {
 
 // Add a problem; A/B describe the stored matrices (see TableLaunch).  m_off / n_off
 // shift the operand coordinates (sub-block products); they must be multiples of 8
-// when the operand is MN-major (TMA inner coordinate alignment).  `outp`, when
+// when the operand is MN-major (TMA inner coordinate alignment).  k_off starts the
+// product at K index k_off of both operands (a K slice); a multiple of 8 when
+// either operand is K-major.  `outp`, when
 // given, receives the three-plane split of the result.
 mao_status table_add(TableLaunch& L, MapSet& maps, const Split3& A, const Split3& B, int M, int N, int K,
                      int m_off, int n_off, float* out, const Split3* outp, int ld_out, const float* aux,
-                     int ld_aux, float alpha, float beta, const int* flag);
+                     int ld_aux, float alpha, float beta, const int* flag, int k_off = 0);
 
 // Stage a launch's problem table into the arena (maps live at maps_off) and launch it.
 struct StagedLaunch {
@@ -199,9 +207,15 @@ struct StagedLaunch {
   int nprob = 0;
   int total_tiles = 0;
   int a_mn = 0, b_mn = 0, kernel_id = 0;
+  int pa = 3, pb = 3;
   double flops = 0.0;
 };
 StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off);
 mao_status table_launch(const Arena& A, const StagedLaunch& S, DevStatus* status, cudaStream_t stream);
+
+// One table-mode launch for a plane pair (instantiated in gemm_table_p*.cu).
+template <int PA, int PB>
+mao_status launch_table_planes(const GemmTableParams& p, int a_mn, int b_mn, cudaStream_t stream, int kernel_id,
+                               double flops);
 
 }  // namespace mao

@@ -91,8 +91,8 @@ __device__ __forceinline__ float4 load4(const void* base, long long off, int is_
     }                                                                                      \
   }
 
-// M <- b1 M + (1-b1) G.  a = G (lda), f0 = M (in place, ldf); planes of G -> pa,
-// planes of the new M -> pb (ldp).
+// M <- b1 M + (1-b1) G.  a = G (lda), f0 = M (in place, ldf); planes of G -> pa
+// (unless nullptr), planes of the new M -> pb (ldp).
 __global__ void __launch_bounds__(256) pc_momentum_kernel(const EwJob* __restrict__ J, int n, float b1) {
   const EwJob& j = J[find_job(J, n, blockIdx.x)];
   const int local = blockIdx.x - j.blk_begin;
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(256) pc_momentum_kernel(const EwJob* __restric
                                   b1 * m.z + (1.f - b1) * g.z, b1 * m.w + (1.f - b1) * g.w);
     *reinterpret_cast<float4*>(mp) = mn;
     const long long o = (long long)r * j.ldp + c;
-    store_split3x4(g, j.pa, o, j.pstride);
+    if (j.pa) store_split3x4(g, j.pa, o, j.pstride);
     store_split3x4(mn, j.pb, o, j.pstride);
   })
 }
@@ -282,159 +282,199 @@ __global__ void __launch_bounds__(256) soap_vperm_kernel(const VPermJob* __restr
 }
 
 // ------------------------------------------------------------------ QR panel pieces
-// A panel W (rows x w, w <= 64, leading dimension ld) of one matrix.
-constexpr int kPanel = 64;
-constexpr int kGramRows = 512;  // rows per Gram partial block
+// Cholesky-QR of one panel W (rows x w, w <= kPanel) per matrix:
+//   Gram G = W^T W as fp32-faithful tensor-core products over K slices (fp32
+//   partials, summed here in fp64 in slice order)
+//   -> column scaling Gs = D^-1/2 G D^-1/2 (D = diag G), optional diagonal shift
+//   -> blocked Cholesky Gs = Rs^T Rs and blocked inverse Rs^-1 (fp64, one block per matrix)
+//   -> R^{-1} = D^-1/2 Rs^{-1}, written as three bf16 planes for the product W R^{-1}.
+// The shift (first Cholesky-QR of a panel only) keeps the factorisation defined
+// for nearly dependent columns; the following unshifted pass restores
+// orthogonality, and the triangular structure makes the final Q the positive-
+// diagonal QR factor either way.
+constexpr int kPanel = 128;
+constexpr int kPanelSq = kPanel * kPanel;
+constexpr int kLdA = kPanel + 1;
+constexpr int kCholSmem = (kPanel * kLdA + (kPanel - 32) * 32 + 2 * kPanel) * 8;
+constexpr int kMaxParts = 16;  // K slices of a panel Gram
+constexpr double kCholShift = 1e-5;  // relative to the unit diagonal of Gs
 
 struct PanelJob {
-  float* W;          // panel base (column 0 of the panel), fp32
-  __nv_bfloat16* Wp; // optional plane set written by the apply pass (ld kPanel, stride wps)
-  long long wps;
-  float* Q;          // optional final destination (column 0 of the panel in Q), or nullptr
-  __nv_bfloat16* Qp; // planes of Q (column 0 of the panel; ld ldqp, stride qps)
-  long long qps;
-  int ldqp;
-  double* gram;      // chunks x 64 x 64 partial Grams
-  double* rinv;      // 64 x 64 inverse of the Cholesky factor
-  int* bad;          // counts non-positive pivots
+  const float* part;     // nparts x kPanel x kPanel fp32 partial Grams (ld kPanel)
+  __nv_bfloat16* rinv;   // three planes (kPanel x kPanel each) of R^{-1}: upper triangle, zero elsewhere
+  int* bad;              // counts non-positive pivots
   const int* flag;
-  int rows, w, ld, ldq;
-  int chunks;        // ceil(rows / kGramRows)
-  int blk_begin;     // gram: chunk blocks; apply: row blocks of 64
+  int w, nparts, shift;
 };
 
-__device__ __forceinline__ int find_panel(const PanelJob* J, int n, int blk) {
-  int lo = 0, hi = n - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (J[mid].blk_begin <= blk) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
-// Partial Gram over kGramRows rows: thread (ty, tx) owns G[4ty..4ty+3][4tx..4tx+3].
-__global__ void __launch_bounds__(256) qr_gram_kernel(const PanelJob* __restrict__ J, int n) {
-  __shared__ float sw[32][kPanel + 1];
-  const PanelJob& j = J[find_panel(J, n, blockIdx.x)];
-  if (j.flag && *j.flag == 0) return;
-  const int chunk = blockIdx.x - j.blk_begin;
-  const int r0 = chunk * kGramRows, r1 = min(j.rows, r0 + kGramRows);
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  double acc[4][4] = {};
-  for (int rb = r0; rb < r1; rb += 32) {
-    __syncthreads();
-    for (int t = threadIdx.x; t < 32 * kPanel; t += 256) {
-      const int rr = t / kPanel, cc = t % kPanel;
-      const int r = rb + rr;
-      sw[rr][cc] = (r < r1 && cc < j.w) ? j.W[(long long)r * j.ld + cc] : 0.f;
-    }
-    __syncthreads();
-    const int nr = min(32, r1 - rb);
-    for (int rr = 0; rr < nr; ++rr) {
-      double a[4], b[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        a[e] = (double)sw[rr][4 * ty + e];
-        b[e] = (double)sw[rr][4 * tx + e];
-      }
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[p][q] += a[p] * b[q];
-    }
-  }
-  double* g = j.gram + (long long)chunk * kPanel * kPanel;
-#pragma unroll
-  for (int p = 0; p < 4; ++p)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) g[(4 * ty + p) * kPanel + 4 * tx + q] = acc[p][q];
-}
-
-// One block per matrix: G = sum of the partial Grams (fixed order), Cholesky
-// G = R^T R (R upper, positive diagonal), then R^{-1} (upper triangular).
-// R lives in the strict upper triangle of G with its diagonal in Rd; R^{-1} is
-// built transposed in the lower triangle (diagonal included).
-__global__ void __launch_bounds__(256) qr_chol_kernel(const PanelJob* __restrict__ J, int n) {
-  __shared__ double G[kPanel][kPanel + 1];
-  __shared__ double Rd[kPanel];
+__global__ void __launch_bounds__(256) qr_chol_kernel(const PanelJob* __restrict__ J) {
+  extern __shared__ double chol_smem[];
+  double* A = chol_smem;                 // [kPanel][kLdA]: Gs, then Rs (upper), then Rs^{-1} (upper)
+  double* T = A + kPanel * kLdA;         // [kPanel - 32][32] block-column workspace of the inverse
+  double* ds = T + (kPanel - 32) * 32;   // D^-1/2
+  double* rdi = ds + kPanel;             // 1 / Rs[k][k]
   const PanelJob& j = J[blockIdx.x];
   if (j.flag && *j.flag == 0) return;
   const int w = j.w;
-  for (int t = threadIdx.x; t < kPanel * kPanel; t += 256) {
-    const int a = t / kPanel, b = t % kPanel;
-    double s = 0.0;
-    for (int c = 0; c < j.chunks; ++c) s += j.gram[(long long)c * kPanel * kPanel + t];
-    G[a][b] = (a < w && b < w) ? s : (a == b ? 1.0 : 0.0);
+  const int nb = (w + 31) / 32, wp = nb * 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr unsigned FULL = 0xffffffffu;
+
+  // G: partials summed in slice order (all of a group's loads in flight at once);
+  // identity padding up to wp
+  for (int q = tid; q < kPanelSq / 4; q += 256) {
+    const int a = q >> 5, b0 = (q & 31) * 4;
+    if (a >= wp || b0 >= wp) continue;
+    double g[4] = {0.0, 0.0, 0.0, 0.0};
+    if (a < w) {
+      float4 v[kMaxParts];
+#pragma unroll
+      for (int p = 0; p < kMaxParts; ++p)
+        if (p < j.nparts) v[p] = *reinterpret_cast<const float4*>(j.part + (long long)p * kPanelSq + 4 * q);
+#pragma unroll
+      for (int p = 0; p < kMaxParts; ++p)
+        if (p < j.nparts) {
+          g[0] += (double)v[p].x;
+          g[1] += (double)v[p].y;
+          g[2] += (double)v[p].z;
+          g[3] += (double)v[p].w;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int b = b0 + e;
+      A[a * kLdA + b] = (a < w && b < w) ? g[e] : (a == b ? 1.0 : 0.0);
+    }
   }
   __syncthreads();
-  // right-looking Cholesky on the upper triangle: row k of R
-  for (int k = 0; k < kPanel; ++k) {
-    if (threadIdx.x == 0) {
-      double d = G[k][k];
-      if (!(d > 0.0)) {
-        atomicAdd(j.bad, 1);
-        d = 1e-300;
+  if (tid < wp) {
+    const double d = A[tid * kLdA + tid];
+    ds[tid] = (d > 0.0) ? rsqrt(d) : 1.0;
+  }
+  __syncthreads();
+  for (int t = tid; t < wp * wp; t += 256) {
+    const int a = t / wp, b = t % wp;
+    double g = A[a * kLdA + b] * ds[a] * ds[b];
+    if (a == b && j.shift) g += kCholShift;
+    A[a * kLdA + b] = g;
+  }
+  __syncthreads();
+
+  // ---- blocked Cholesky, upper: Gs = Rs^T Rs
+  for (int bk = 0; bk < nb; ++bk) {
+    const int o = bk * 32;
+    if (warp == 0) {
+      // lane c holds column o + c of the diagonal block (rows <= c)
+      double v[32];
+      int nbad = 0;
+#pragma unroll
+      for (int r = 0; r < 32; ++r) v[r] = (r <= lane) ? A[(o + r) * kLdA + o + lane] : 0.0;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        double d = __shfl_sync(FULL, v[k], k);
+        nbad += (d > 0.0) ? 0 : 1;
+        d = (d > 0.0) ? d : 1e-300;
+        const double ri = rsqrt(d);  // 1 / Rs[k][k]
+        const double rk = (lane == k) ? d * ri : (lane > k ? v[k] * ri : 0.0);  // Rs[k][c]
+        if (lane == k) rdi[o + k] = ri;
+        v[k] = rk;
+#pragma unroll
+        for (int i = 1; i < 32; ++i) {
+          if (i > k) {  // constant trip count keeps v[] in registers
+            const double rki = __shfl_sync(FULL, rk, i);
+            if (i <= lane) v[i] -= rki * rk;
+          }
+        }
       }
-      G[k][k] = sqrt(d);
-      Rd[k] = G[k][k];
+#pragma unroll
+      for (int r = 0; r < 32; ++r)
+        if (r <= lane) A[(o + r) * kLdA + o + lane] = v[r];
+      if (lane == 0 && nbad) atomicAdd(j.bad, nbad);
     }
     __syncthreads();
-    const double rkk = G[k][k];
-    for (int c = k + 1 + threadIdx.x; c < kPanel; c += 256) G[k][c] /= rkk;
+    const int nt = wp - o - 32;  // trailing columns
+    if (nt == 0) break;
+    // block row: Rs_bc = Rs_bb^{-T} G_bc, one column per thread (right-looking in registers)
+    if (tid < nt) {
+      const int c = o + 32 + tid;
+      double x[32];
+#pragma unroll
+      for (int r = 0; r < 32; ++r) x[r] = A[(o + r) * kLdA + c];
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        x[r] *= rdi[o + r];
+#pragma unroll
+        for (int i = r + 1; i < 32; ++i) x[i] -= A[(o + r) * kLdA + o + i] * x[r];
+      }
+#pragma unroll
+      for (int r = 0; r < 32; ++r) A[(o + r) * kLdA + c] = x[r];
+    }
     __syncthreads();
-    // trailing update G[a][b] -= R[k][a] R[k][b] for k < a <= b
-    for (int t = threadIdx.x; t < kPanel * kPanel; t += 256) {
-      const int a = t / kPanel, b = t % kPanel;
-      if (a > k && b >= a) G[a][b] -= G[k][a] * G[k][b];
+    // trailing update of the upper triangle: G_cd -= Rs_bc^T Rs_bd, c <= d
+    for (int t = tid; t < nt * nt; t += 256) {
+      const int c = o + 32 + t / nt, d = o + 32 + t % nt;
+      if (d < c) continue;
+      double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        s0 += A[(o + i) * kLdA + c] * A[(o + i) * kLdA + d];
+        s1 += A[(o + i + 1) * kLdA + c] * A[(o + i + 1) * kLdA + d];
+        s2 += A[(o + i + 2) * kLdA + c] * A[(o + i + 2) * kLdA + d];
+        s3 += A[(o + i + 3) * kLdA + c] * A[(o + i + 3) * kLdA + d];
+      }
+      A[c * kLdA + d] -= (s0 + s1) + (s2 + s3);
     }
     __syncthreads();
   }
-  // R^{-1}: thread c solves R x = e_c by back substitution; x_r is kept at G[c][r]
-  if (threadIdx.x < kPanel) {
-    const int c = threadIdx.x;
-    for (int r = c; r >= 0; --r) {
-      double s = (r == c) ? 1.0 : 0.0;
-      for (int k = r + 1; k <= c; ++k) s -= G[r][k] * G[c][k];
-      G[c][r] = s / Rd[r];
+
+  // ---- blocked inverse in place, by block columns: X_jj = Rs_jj^{-1};
+  //      X_ij = -(sum_{k=i..j-1} X_ik Rs_kj) X_jj for block rows i < j
+  for (int bj = 0; bj < nb; ++bj) {
+    const int oj = bj * 32;
+    // T[r][c] = sum_{k = r .. oj-1} X[r][k] Rs[k][oj + c]  (X upper: k >= r)
+    for (int t = tid; t < oj * 32; t += 256) {
+      const int r = t >> 5, c = t & 31;
+      double s0 = 0.0, s1 = 0.0;
+      int k = r;
+      for (; k + 1 < oj; k += 2) {
+        s0 += A[r * kLdA + k] * A[k * kLdA + oj + c];
+        s1 += A[r * kLdA + k + 1] * A[(k + 1) * kLdA + oj + c];
+      }
+      if (k < oj) s0 += A[r * kLdA + k] * A[k * kLdA + oj + c];
+      T[r * 32 + c] = s0 + s1;
     }
+    if (warp == 0) {
+      // column c = lane of Rs_jj^{-1}, from the last row up (right-looking in registers)
+      double acc[32], x[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) acc[i] = 0.0;
+#pragma unroll
+      for (int k = 31; k >= 0; --k) {
+        const double ri = rdi[oj + k];
+        x[k] = (k == lane) ? ri : (k < lane ? -acc[k] * ri : 0.0);
+#pragma unroll
+        for (int i = 0; i < k; ++i) acc[i] += A[(oj + i) * kLdA + oj + k] * x[k];
+      }
+      __syncwarp();
+#pragma unroll
+      for (int r = 0; r < 32; ++r)
+        if (r <= lane) A[(oj + r) * kLdA + oj + lane] = x[r];
+    }
+    __syncthreads();
+    // X_i,j = -T_i X_jj
+    for (int t = tid; t < oj * 32; t += 256) {
+      const int r = t >> 5, c = t & 31;
+      double s = 0.0;
+      for (int m = 0; m <= c; ++m) s += T[r * 32 + m] * A[(oj + m) * kLdA + oj + c];
+      A[r * kLdA + oj + c] = -s;
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  for (int t = threadIdx.x; t < kPanel * kPanel; t += 256) {
+  // R^{-1} = D^-1/2 Rs^{-1}: three bf16 planes over the full kPanel x kPanel square
+  for (int t = tid; t < kPanelSq; t += 256) {
     const int r = t / kPanel, c = t % kPanel;
-    j.rinv[t] = (r <= c) ? G[c][r] : 0.0;
-  }
-}
-
-// W <- W R^{-1} for kApplyRows rows per block (fp64 accumulation); optionally
-// also writes the result and its three-plane split to Q and to W's plane set.
-constexpr int kApplyRows = 32;
-
-__global__ void __launch_bounds__(256) qr_apply_kernel(const PanelJob* __restrict__ J, int n) {
-  __shared__ double Ri[kPanel][kPanel + 1];
-  __shared__ float sw[kApplyRows][kPanel + 1];
-  const PanelJob& j = J[find_panel(J, n, blockIdx.x)];
-  if (j.flag && *j.flag == 0) return;
-  const int r0 = (blockIdx.x - j.blk_begin) * kApplyRows;
-  for (int t = threadIdx.x; t < kPanel * kPanel; t += 256) Ri[t / kPanel][t % kPanel] = j.rinv[t];
-  for (int t = threadIdx.x; t < kApplyRows * kPanel; t += 256) {
-    const int rr = t / kPanel, cc = t % kPanel;
-    const int r = r0 + rr;
-    sw[rr][cc] = (r < j.rows && cc < j.w) ? j.W[(long long)r * j.ld + cc] : 0.f;
-  }
-  __syncthreads();
-  for (int t = threadIdx.x; t < kApplyRows * kPanel; t += 256) {
-    const int rr = t / kPanel, c = t % kPanel;
-    const int r = r0 + rr;
-    if (r >= j.rows || c >= j.w) continue;
-    double s = 0.0;
-    for (int a = 0; a <= c; ++a) s += (double)sw[rr][a] * Ri[a][c];
-    const float x = (float)s;
-    j.W[(long long)r * j.ld + c] = x;
-    if (j.Wp) store_split3(x, j.Wp, (long long)r * kPanel + c, j.wps);
-    if (j.Q) {
-      j.Q[(long long)r * j.ldq + c] = x;
-      store_split3(x, j.Qp, (long long)r * j.ldqp + c, j.qps);
-    }
+    const float x = (r <= c && c < w) ? (float)(ds[r] * A[r * kLdA + c]) : 0.0f;
+    store_split3(x, j.rinv, t, kPanelSq);
   }
 }
 

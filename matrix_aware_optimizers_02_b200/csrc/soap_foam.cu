@@ -78,14 +78,23 @@ int host_refresh_mode(const mao_refresh& rf, int64_t t) {
 
 inline int ldp_of(int cols) { return round_up_int(cols, 8); }
 
+// K slice of the panel Gram products of a launch with `nact` panels: enough
+// slices to give about two tiles per SM, at most kMaxParts, at least 256 rows each,
+// a multiple of 64 (whole K blocks, so slices never overlap).
+inline int gram_slice(int k, int nact) {
+  const int want = std::max(1, std::min(kMaxParts, (2 * 148 + nact - 1) / std::max(nact, 1)));
+  const int sl = round_up_int(std::max(256, (k + want - 1) / want), 64);
+  return std::max(sl, round_up_int((k + kMaxParts - 1) / kMaxParts, 64));
+}
+
 // Bytes of a three-plane bf16 set of a rows x cols matrix.
 inline size_t planes_bytes(int rows, int cols) { return 3 * 2 * (size_t)rows * ldp_of(cols); }
 
 // Scratch of one side (k x k factor F with basis Q) of one matrix.
 struct SideBuf {
   size_t Fp, Qp, P, Ps, Psp;
-  size_t W, Wp, Cp;
-  size_t gram, rinv, keys, perm, flag, rho, bad;
+  size_t W, Wp, Wb, Wbp, Cp;  // panel ping-pong buffers (k x kPanel) and the coefficients
+  size_t part, rinv, keys, perm, flag, rho, bad;
   size_t Tp, D;  // adaptive check
 };
 
@@ -98,7 +107,7 @@ struct MatBuf {
 
 void side_layout(int k, bool check, Carver& cv, SideBuf& s, size_t flag_block) {
   const size_t kk = (size_t)k * k;
-  const int chunks = (k + kGramRows - 1) / kGramRows;
+  const int parts = (k + gram_slice(k, 1) - 1) / gram_slice(k, 1);  // the most slices any launch uses
   s.Fp = cv.take(planes_bytes(k, k));
   s.Qp = cv.take(planes_bytes(k, k));
   s.P = cv.take(4 * kk);
@@ -106,9 +115,11 @@ void side_layout(int k, bool check, Carver& cv, SideBuf& s, size_t flag_block) {
   s.Psp = cv.take(planes_bytes(k, k));
   s.W = cv.take(4 * (size_t)k * kPanel);
   s.Wp = cv.take(planes_bytes(k, kPanel));
+  s.Wb = cv.take(4 * (size_t)k * kPanel);
+  s.Wbp = cv.take(planes_bytes(k, kPanel));
   s.Cp = cv.take(planes_bytes(k, kPanel));
-  s.gram = cv.take(8 * (size_t)chunks * kPanel * kPanel);
-  s.rinv = cv.take(8 * (size_t)kPanel * kPanel);
+  s.part = cv.take(4 * (size_t)parts * kPanelSq);
+  s.rinv = cv.take(2 * 3 * (size_t)kPanelSq);
   s.keys = cv.take(8 * (size_t)k);
   s.perm = cv.take(4 * (size_t)k);
   s.flag = flag_block;  // flag, rho and the failure counter share one 64-byte block
@@ -204,7 +215,7 @@ void make_groups(const Ctx& X, std::vector<GroupPlan>& groups) {
 // Records every launch of one group into `ops`, with all device data staged in
 // the arena; in sizing mode (ws == nullptr) only the sizes matter.
 struct Op {
-  enum Kind { GEMM, EW, SPLIT, ADAM, KEYS, ARGSORT, GATHER, VPERM, GRAM, CHOL, APPLY, RC, TAU, FOAMN, CHECK } kind;
+  enum Kind { GEMM, EW, SPLIT, ADAM, KEYS, ARGSORT, GATHER, VPERM, CHOL, RC, TAU, FOAMN, CHECK } kind;
   size_t jobs = 0;
   int njobs = 0;
   int blocks = 0;
@@ -382,98 +393,119 @@ mao_status build_refresh_side(Builder& B, GroupPlan& G, bool left) {
     }
     B.ops.back().blocks = blk;
   }
-  // QR by blocks of 64 columns
+  // QR by panels of kPanel columns: block Gram-Schmidt with two projection passes,
+  // Cholesky-QR inside each panel (twice after the first pass, once after the second)
   int maxk = 0;
   for (int i = 0; i < nm; ++i) maxk = std::max(maxk, kof(i));
   const int npanels = (maxk + kPanel - 1) / kPanel;
+  enum { PS = 0, WA = 1, WB = 2, QF = 3 };
   for (int pj = 0; pj < npanels; ++pj) {
     const int c0 = pj * kPanel;
     std::vector<int> act;
     for (int i = 0; i < nm; ++i)
       if (kof(i) > c0) act.push_back(i);
     auto wdt = [&](int i) { return std::min(kPanel, kof(i) - c0); };
-    // one Cholesky-QR pass on the panel of every active matrix;
-    // target: 0 = in place, 1 = also W's plane set, 2 = the final Q columns and planes
-    auto cholqr = [&](bool first_panel, int target) {
-      std::vector<PanelJob> jl(act.size());
-      int gblk = 0, ablk = 0;
+    // a panel's fp32 storage and plane view (columns c0 .. c0 + w of Ps / Q, or a scratch buffer)
+    auto fp = [&](int i, int where, int* ld) -> float* {
+      const int k = kof(i);
+      switch (where) {
+        case PS: *ld = k; return B.wp<float>(side(i).Ps) + c0;
+        case WA: *ld = kPanel; return B.wp<float>(side(i).W);
+        case WB: *ld = kPanel; return B.wp<float>(side(i).Wb);
+        default: *ld = k; return Qp(i) + c0;
+      }
+    };
+    auto pv = [&](int i, int where) -> Split3 {
+      const int k = kof(i), w = wdt(i);
+      Split3 v;
+      switch (where) {
+        case PS: v = B.planes(side(i).Psp, k, k); break;
+        case WA: v = B.planes(side(i).Wp, k, kPanel); break;
+        case WB: v = B.planes(side(i).Wbp, k, kPanel); break;
+        default: v = B.planes(side(i).Qp, k, k); break;
+      }
+      if (where == PS || where == QF)
+        for (int q = 0; q < 3; ++q) v.p[q] += c0;
+      v.cols = w;
+      return v;
+    };
+    // one Cholesky-QR of every active panel: dst = src R^{-1}; `shift` regularises
+    // the factorisation of a panel that may be nearly rank deficient
+    auto cholqr = [&](int src, int dst, bool shift) -> mao_status {
+      // Gram partials over K slices (fp32-faithful), one 128 x 128 tile each
+      TableLaunch& gg = B.new_gemm(1, 1, MAO_K_PC_PANEL);
+      const int nact = (int)act.size();
+      for (int i : act) {
+        const int k = kof(i), w = wdt(i);
+        const int sl = gram_slice(k, nact);
+        float* part = B.wp<float>(side(i).part);
+        const Split3 Wv = pv(i, src);
+        for (int s0 = 0, p = 0; s0 < k; s0 += sl, ++p)
+          MAO_TRY(table_add(gg, B.maps, Wv, Wv, w, w, std::min(sl, k - s0), 0, 0, part + (size_t)p * kPanelSq,
+                            nullptr, kPanel, nullptr, 0, 1.f, 0.f, flagp(i), s0));
+      }
+      size_t off;
+      PanelJob* J = B.new_jobs<PanelJob>(Op::CHOL, (int)act.size(), off);
       for (size_t a = 0; a < act.size(); ++a) {
         const int i = act[a];
         const int k = kof(i);
-        PanelJob& j = jl[a];
-        std::memset(&j, 0, sizeof(j));
-        if (first_panel) {
-          j.W = B.wp<float>(side(i).Ps) + c0;
-          j.ld = k;
-        } else {
-          j.W = B.wp<float>(side(i).W);
-          j.ld = kPanel;
-        }
-        if (target == 1) {
-          j.Wp = B.wp<__nv_bfloat16>(side(i).Wp);
-          j.wps = B.pstride(k, kPanel);
-        }
-        if (target == 2) {
-          j.Q = Qp(i) + c0;
-          j.ldq = k;
-          j.Qp = B.wp<__nv_bfloat16>(side(i).Qp) + c0;
-          j.qps = B.pstride(k, k);
-          j.ldqp = ldp_of(k);
-        }
-        j.gram = B.wp<double>(side(i).gram);
-        j.rinv = B.wp<double>(side(i).rinv);
+        PanelJob& j = J[a];
+        j.part = B.wp<float>(side(i).part);
+        j.rinv = B.wp<__nv_bfloat16>(side(i).rinv);
         j.bad = B.wp<int>(side(i).bad);
         j.flag = flagp(i);
-        j.rows = k;
         j.w = wdt(i);
-        j.chunks = (k + kGramRows - 1) / kGramRows;
-        j.blk_begin = gblk;
-        gblk += j.chunks;
+        j.nparts = (k + gram_slice(k, nact) - 1) / gram_slice(k, nact);
+        j.shift = shift ? 1 : 0;
       }
-      size_t off;
-      PanelJob* Jg = B.new_jobs<PanelJob>(Op::GRAM, (int)act.size(), off);
-      for (size_t a = 0; a < act.size(); ++a) Jg[a] = jl[a];
-      B.ops.back().blocks = gblk;
-      PanelJob* Jc = B.new_jobs<PanelJob>(Op::CHOL, (int)act.size(), off);
-      for (size_t a = 0; a < act.size(); ++a) Jc[a] = jl[a];
       B.ops.back().blocks = (int)act.size();
-      PanelJob* Ja = B.new_jobs<PanelJob>(Op::APPLY, (int)act.size(), off);
-      for (size_t a = 0; a < act.size(); ++a) {
-        jl[a].blk_begin = ablk;
-        ablk += (jl[a].rows + kApplyRows - 1) / kApplyRows;
-        Ja[a] = jl[a];
-      }
-      B.ops.back().blocks = ablk;
-    };
-    // project out the finished columns: C = Q[:, :c0]^T Y ; W = Y - Q[:, :c0] C
-    auto project = [&](bool from_ps) -> mao_status {
-      TableLaunch& gc = B.new_gemm(1, 1, MAO_K_PC_QR);
+      TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_QR);
       for (int i : act) {
-        const int k = kof(i);
-        const Split3 Y = from_ps ? B.planes(side(i).Psp, k, k) : B.planes(side(i).Wp, k, kPanel);
-        const Split3 C = B.planes(side(i).Cp, k, kPanel);
-        MAO_TRY(table_add(gc, B.maps, B.planes(side(i).Qp, k, k), Y, c0, wdt(i), k, 0, from_ps ? c0 : 0, nullptr,
-                          &C, kPanel, nullptr, 0, 1.f, 0.f, flagp(i)));
-      }
-      TableLaunch& gw = B.new_gemm(0, 1, MAO_K_PC_QR);
-      for (int i : act) {
-        const int k = kof(i);
-        const float* aux = from_ps ? B.wp<float>(side(i).Ps) + c0 : B.wp<float>(side(i).W);
-        MAO_TRY(table_add(gw, B.maps, B.planes(side(i).Qp, k, k), B.planes(side(i).Cp, k, kPanel), k, wdt(i), c0, 0,
-                          0, B.wp<float>(side(i).W), nullptr, kPanel, aux, from_ps ? k : kPanel, -1.f, 1.f,
+        const int k = kof(i), w = wdt(i);
+        __nv_bfloat16* r = B.wp<__nv_bfloat16>(side(i).rinv);
+        const Split3 Ri{{r, r + kPanelSq, r + 2 * kPanelSq}, w, w, kPanel};
+        const Split3 out_p = pv(i, dst);
+        int ld = 0;
+        float* out = fp(i, dst, &ld);
+        MAO_TRY(table_add(g, B.maps, pv(i, src), Ri, k, w, w, 0, 0, out, &out_p, ld, nullptr, 0, 1.f, 0.f,
                           flagp(i)));
       }
       return MAO_OK;
     };
+    // remove the finished columns: C = Q[:, :c0]^T Y ; W = Y - Q[:, :c0] C (fp32 and planes)
+    auto project = [&](int from) -> mao_status {
+      TableLaunch& gc = B.new_gemm(1, 1, MAO_K_PC_QR);
+      for (int i : act) {
+        const int k = kof(i), w = wdt(i);
+        Split3 C = B.planes(side(i).Cp, k, kPanel);
+        C.cols = w;
+        MAO_TRY(table_add(gc, B.maps, B.planes(side(i).Qp, k, k), pv(i, from), c0, w, k, 0, 0, nullptr, &C,
+                          kPanel, nullptr, 0, 1.f, 0.f, flagp(i)));
+      }
+      TableLaunch& gw = B.new_gemm(0, 1, MAO_K_PC_QR);
+      for (int i : act) {
+        const int k = kof(i), w = wdt(i);
+        Split3 C = B.planes(side(i).Cp, k, kPanel);
+        C.rows = c0;
+        C.cols = w;
+        const Split3 Wp = pv(i, WA);
+        int lda = 0, ldw = 0;
+        const float* aux = fp(i, from, &lda);
+        float* W = fp(i, WA, &ldw);
+        MAO_TRY(table_add(gw, B.maps, B.planes(side(i).Qp, k, k), C, k, w, c0, 0, 0, W, &Wp, ldw, aux, lda, -1.f,
+                          1.f, flagp(i)));
+      }
+      return MAO_OK;
+    };
     if (pj == 0) {
-      cholqr(true, 0);
-      cholqr(true, 2);
+      MAO_TRY(cholqr(PS, WB, true));
+      MAO_TRY(cholqr(WB, QF, false));
     } else {
-      MAO_TRY(project(true));
-      cholqr(false, 0);
-      cholqr(false, 1);
-      MAO_TRY(project(false));
-      cholqr(false, 2);
+      MAO_TRY(project(PS));
+      MAO_TRY(cholqr(WA, WB, true));
+      MAO_TRY(cholqr(WB, WA, false));
+      MAO_TRY(project(WA));
+      MAO_TRY(cholqr(WA, QF, false));
     }
   }
   return MAO_OK;
@@ -487,7 +519,21 @@ mao_status build_group(Builder& B, GroupPlan& G) {
   B.zero_flag_off = B.arena.take(16, 16);
   std::memset(B.arena.hptr<int>(B.zero_flag_off), 0, 16);
 
-  // momentum + planes of G and M
+  // A group whose gradients are all bf16 reads each G directly as a one-plane
+  // operand (exact); otherwise the momentum pass writes three planes of G.
+  bool g_one = true;
+  for (int i = 0; i < nm; ++i) g_one = g_one && A(i).g_bf16;
+  const int gpl = g_one ? 1 : 3;
+  auto Gop = [&](int i) -> Split3 {
+    const PcMat& a = A(i);
+    if (!g_one) return B.planes(G.mb[i].Gp, a.m, a.n);
+    // sizing mode: a distinct stand-in address per matrix, never dereferenced
+    const __nv_bfloat16* g = B.ws ? static_cast<const __nv_bfloat16*>(a.G)
+                                  : reinterpret_cast<const __nv_bfloat16*>((1ull << 60) + 256ull * (G.g0 + i));
+    return Split3{{g, nullptr, nullptr}, a.m, a.n, a.n};
+  };
+
+  // momentum + planes of M (and of G unless it is read directly)
   {
     size_t off;
     EwJob* J = B.new_jobs<EwJob>(Op::EW, nm, off);
@@ -499,7 +545,7 @@ mao_status build_group(Builder& B, GroupPlan& G) {
       j.a = a.G;
       j.a_bf16 = a.g_bf16;
       j.f0 = a.M;
-      j.pa = B.wp<__nv_bfloat16>(G.mb[i].Gp);
+      j.pa = g_one ? nullptr : B.wp<__nv_bfloat16>(G.mb[i].Gp);
       j.pb = B.wp<__nv_bfloat16>(G.mb[i].Mp);
       j.pstride = B.pstride(a.m, a.n);
       j.rows = a.m;
@@ -509,7 +555,7 @@ mao_status build_group(Builder& B, GroupPlan& G) {
       j.ldp = ldp_of(a.n);
       j.blk_begin = blk;
       blk += ew_blocks(a.m, a.n);
-      bytes += (double)a.m * a.n * ((a.g_bf16 ? 2 : 4) + 8 + 12);
+      bytes += (double)a.m * a.n * ((a.g_bf16 ? 2 : 4) + 8 + 6 + (g_one ? 0 : 6));
     }
     B.ops.back().blocks = blk;
     B.ops.back().bytes = bytes;
@@ -517,20 +563,20 @@ mao_status build_group(Builder& B, GroupPlan& G) {
   // factor EMAs
   if (!foam) {
     TableLaunch& g = B.new_gemm(0, 0, MAO_K_PC_FACTOR);
+    g.pa = g.pb = gpl;
     for (int i = 0; i < nm; ++i) {
       const PcMat& a = A(i);
-      const Split3 Gs = B.planes(G.mb[i].Gp, a.m, a.n);
-      MAO_TRY(table_add(g, B.maps, Gs, Gs, a.m, a.m, a.n, 0, 0, a.L, nullptr, a.m, a.L, a.m, 1.f - X.b2, X.b2,
-                        nullptr));
+      MAO_TRY(table_add(g, B.maps, Gop(i), Gop(i), a.m, a.m, a.n, 0, 0, a.L, nullptr, a.m, a.L, a.m, 1.f - X.b2,
+                        X.b2, nullptr));
     }
   }
   {
     TableLaunch& g = B.new_gemm(1, 1, MAO_K_PC_FACTOR);
+    g.pa = g.pb = gpl;
     for (int i = 0; i < nm; ++i) {
       const PcMat& a = A(i);
-      const Split3 Gs = B.planes(G.mb[i].Gp, a.m, a.n);
-      MAO_TRY(table_add(g, B.maps, Gs, Gs, a.n, a.n, a.m, 0, 0, a.R, nullptr, a.n, a.R, a.n, 1.f - X.b2, X.b2,
-                        nullptr));
+      MAO_TRY(table_add(g, B.maps, Gop(i), Gop(i), a.n, a.n, a.m, 0, 0, a.R, nullptr, a.n, a.R, a.n, 1.f - X.b2,
+                        X.b2, nullptr));
     }
   }
   // refresh, or plain planes of the bases
@@ -607,14 +653,19 @@ mao_status build_group(Builder& B, GroupPlan& G) {
     // T1 = Q_L^T {G, M}  (A = Q_L stored K x M, B = G / M stored K x N)
     {
       TableLaunch& g = B.new_gemm(1, 1, MAO_K_PC_ROTATE);
+      g.pb = gpl;
       for (int i = 0; i < nm; ++i) {
         const PcMat& a = A(i);
-        const Split3 Ql = B.planes(G.mb[i].L.Qp, a.m, a.m);
-        const Split3 T1G = B.planes(G.mb[i].T1G, a.m, a.n), T1M = B.planes(G.mb[i].T1M, a.m, a.n);
-        MAO_TRY(table_add(g, B.maps, Ql, B.planes(G.mb[i].Gp, a.m, a.n), a.m, a.n, a.m, 0, 0, nullptr, &T1G, a.n,
-                          nullptr, 0, 1.f, 0.f, nullptr));
-        MAO_TRY(table_add(g, B.maps, Ql, B.planes(G.mb[i].Mp, a.m, a.n), a.m, a.n, a.m, 0, 0, nullptr, &T1M, a.n,
-                          nullptr, 0, 1.f, 0.f, nullptr));
+        const Split3 T1G = B.planes(G.mb[i].T1G, a.m, a.n);
+        MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].L.Qp, a.m, a.m), Gop(i), a.m, a.n, a.m, 0, 0, nullptr, &T1G,
+                          a.n, nullptr, 0, 1.f, 0.f, nullptr));
+      }
+      TableLaunch& g2 = B.new_gemm(1, 1, MAO_K_PC_ROTATE);
+      for (int i = 0; i < nm; ++i) {
+        const PcMat& a = A(i);
+        const Split3 T1M = B.planes(G.mb[i].T1M, a.m, a.n);
+        MAO_TRY(table_add(g2, B.maps, B.planes(G.mb[i].L.Qp, a.m, a.m), B.planes(G.mb[i].Mp, a.m, a.n), a.m, a.n,
+                          a.m, 0, 0, nullptr, &T1M, a.n, nullptr, 0, 1.f, 0.f, nullptr));
       }
     }
     // Gh, Mh = T1 Q_R (fp32)
@@ -680,13 +731,17 @@ mao_status build_group(Builder& B, GroupPlan& G) {
     // Gr, Mr = {G, M} Q_R  (A K-major, B = Q_R stored K x N)
     {
       TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_ROTATE);
+      g.pa = gpl;
       for (int i = 0; i < nm; ++i) {
         const PcMat& a = A(i);
-        const Split3 Qr = B.planes(G.mb[i].R.Qp, a.n, a.n);
-        MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].Gp, a.m, a.n), Qr, a.m, a.n, a.n, 0, 0,
+        MAO_TRY(table_add(g, B.maps, Gop(i), B.planes(G.mb[i].R.Qp, a.n, a.n), a.m, a.n, a.n, 0, 0,
                           B.wp<float>(G.mb[i].Gr), nullptr, a.n, nullptr, 0, 1.f, 0.f, nullptr));
-        MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].Mp, a.m, a.n), Qr, a.m, a.n, a.n, 0, 0,
-                          B.wp<float>(G.mb[i].Mr), nullptr, a.n, nullptr, 0, 1.f, 0.f, nullptr));
+      }
+      TableLaunch& g2 = B.new_gemm(0, 1, MAO_K_PC_ROTATE);
+      for (int i = 0; i < nm; ++i) {
+        const PcMat& a = A(i);
+        MAO_TRY(table_add(g2, B.maps, B.planes(G.mb[i].Mp, a.m, a.n), B.planes(G.mb[i].R.Qp, a.n, a.n), a.m, a.n,
+                          a.n, 0, 0, B.wp<float>(G.mb[i].Mr), nullptr, a.n, nullptr, 0, 1.f, 0.f, nullptr));
       }
     }
     // row/col partials of Gr^2, r/c EMAs and tau, N
@@ -809,6 +864,21 @@ void add_stats_jobs(Builder& B, GroupPlan& G, BuiltGroup& bg) {
   }
 }
 
+// The Cholesky kernel's shared memory exceeds the default 48 KB: opt in once per device.
+mao_status chol_attr() {
+  static std::mutex mu;
+  static bool set[64] = {};
+  int dev = 0;
+  MAO_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return MAO_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!set[dev]) {
+    MAO_CUDA_TRY(cudaFuncSetAttribute(qr_chol_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCholSmem));
+    set[dev] = true;
+  }
+  return MAO_OK;
+}
+
 mao_status run_ops(const Ctx& X, uint8_t* arena_dev, const BuiltGroup& bg, DevStatus* status, cudaStream_t s) {
   Arena A;  // device view of the staged arena
   A.dev = arena_dev;
@@ -861,19 +931,10 @@ mao_status run_ops(const Ctx& X, uint8_t* arena_dev, const BuiltGroup& bg, DevSt
         soap_vperm_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<VPermJob>(op.jobs), n);
         break;
       }
-      case Op::GRAM: {
-        LaunchScope ls(s, MAO_K_PC_QR, 0.0, 0.0);
-        qr_gram_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<PanelJob>(op.jobs), n);
-        break;
-      }
       case Op::CHOL: {
-        LaunchScope ls(s, MAO_K_PC_QR, 0.0, 0.0);
-        qr_chol_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<PanelJob>(op.jobs), n);
-        break;
-      }
-      case Op::APPLY: {
-        LaunchScope ls(s, MAO_K_PC_QR, 0.0, 0.0);
-        qr_apply_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<PanelJob>(op.jobs), n);
+        MAO_TRY(chol_attr());
+        LaunchScope ls(s, MAO_K_PC_CHOL, 0.0, 0.0);
+        qr_chol_kernel<<<op.blocks, 256, kCholSmem, s>>>(A.dptr<PanelJob>(op.jobs));
         break;
       }
       case Op::RC: {
@@ -1009,7 +1070,7 @@ mao_status run_step(const Ctx& X, const void* mats, size_t mats_bytes, void* wor
     if (ws_bytes < sizing.L.total) return MAO_ERR_WORKSPACE;
     P = std::make_shared<StepPlan>();
     MAO_TRY(make_plan(X, ws, *P));
-    if (P->L.total != sizing.L.total) return MAO_ERR_WORKSPACE;
+    if (P->L.total > sizing.L.total) return MAO_ERR_WORKSPACE;
     PlanCache& C = plan_cache();
     std::lock_guard<std::mutex> lk(C.mu);
     C.lru.emplace_front(key, P);
@@ -1037,10 +1098,23 @@ mao_status run_step(const Ctx& X, const void* mats, size_t mats_bytes, void* wor
   return MAO_OK;
 }
 
+// Bytes that serve every step of this descriptor set, whatever t: the maximum
+// over the refresh modes the policy can take (plain steps, and refresh or check
+// steps).
 mao_status workspace_size(const Ctx& X, size_t* bytes) {
-  StepPlan sizing;
-  MAO_TRY(make_plan(X, nullptr, sizing));
-  *bytes = sizing.L.total;
+  int modes[2] = {0, 0};
+  int nmodes = 1;
+  if (X.rf.kind == MAO_REFRESH_EVERY_K) modes[nmodes++] = 1;
+  if (X.rf.kind == MAO_REFRESH_ADAPTIVE) modes[nmodes++] = 2;
+  size_t best = 0;
+  for (int i = 0; i < nmodes; ++i) {
+    Ctx Y = X;
+    Y.mode = modes[i];
+    StepPlan sizing;
+    MAO_TRY(make_plan(Y, nullptr, sizing));
+    best = std::max(best, sizing.L.total);
+  }
+  *bytes = best;
   return MAO_OK;
 }
 

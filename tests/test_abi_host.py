@@ -123,8 +123,31 @@ def test_soap_foam_validation(lib):
 def test_gemm_entry_validation(lib):
     b = ctypes.c_size_t(0)
     assert lib.mao_test_gemm_workspace_size(0, 1, 0, 8, 8, ctypes.byref(b)) == L.MAO_ERR_SHAPE
-    assert lib.mao_test_gemm_workspace_size(5, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_ERR_INVALID_ARG
+    assert lib.mao_test_gemm_workspace_size(6, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_ERR_INVALID_ARG
+    for kind in range(6):
+        assert lib.mao_test_gemm_workspace_size(kind, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_OK
     assert lib.mao_test_gemm_workspace_size(1, 2, 64, 64, 32, ctypes.byref(b)) == L.MAO_OK
     assert b.value >= 2 * 3 * 2 * (2 * 64 * 32)  # three bf16 planes of A and of B
     assert lib.mao_test_gemm(0, 0, 0, A16, A16, A16, 1, 8, 8, 12, A16, 1 << 20, None) == L.MAO_ERR_SHAPE
     assert lib.mao_test_gemm(0, 2, 0, A16, A16, A16, 1, 8, 8, 16, A16, 1 << 20, None) == L.MAO_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kind,k,pf", [(L.REFRESH_EVERY_K, 3, 10), (L.REFRESH_ADAPTIVE, 1, 4), (L.REFRESH_NEVER, 1, 10)])
+def test_precond_workspace_size_is_independent_of_t(lib, kind, k, pf):
+    """One workspace serves every step: plain, refresh and check steps alike."""
+    rf = L.Refresh(kind, k, pf, 0.1, 1)
+    mats = [L.SoapMat(m, n, A16, A16, 1, A16, A16, A16, A16, A16, A16, None, None)
+            for (m, n) in [(256, 512), (1024, 136), (8, 8)]]
+    arr = (L.SoapMat * 3)(*mats)
+    fm = [L.FoamMat(m, n, A16, A16, 1, A16, A16, A16, A16, A16, None) for (m, n) in [(256, 512), (1024, 136)]]
+    farr = (L.FoamMat * 2)(*fm)
+    sizes, fsizes = set(), set()
+    for t in range(1, 9):
+        b = ctypes.c_size_t(0)
+        sp = L.SoapParams(0.95, 0.95, 1e-8, 3e-3, 0.0, t, rf)
+        assert lib.mao_soap_workspace_size(arr, 3, ctypes.byref(sp), ctypes.byref(b)) == L.MAO_OK
+        sizes.add(b.value)
+        fp = L.FoamParams(0.95, 0.95, 1e-8, 3e-3, 0.0, t, rf, 0)
+        assert lib.mao_foam_workspace_size(farr, 2, ctypes.byref(fp), ctypes.byref(b)) == L.MAO_OK
+        fsizes.add(b.value)
+    assert len(sizes) == 1 and len(fsizes) == 1

@@ -62,3 +62,41 @@ def test_gemm_repeatable_bitwise(api):
     d1 = api.gemm(A, B)
     d2 = api.gemm(A, B)
     assert torch.equal(d1, d2)
+
+
+MIXED = [("bf16_fold", torch.bfloat16, torch.bfloat16), ("split3_bf16", torch.float32, torch.bfloat16),
+         ("bf16_split3", torch.bfloat16, torch.float32)]
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (1, 1), (0, 1)])
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("kind,adt,bdt", MIXED)
+def test_plane_pairs_are_fp32_faithful(api, kind, adt, bdt, shape, a_mn, b_mn):
+    """A bf16 operand is exact in one plane: a bf16 x bf16 product folded in fp32,
+    and fp32 x bf16 in three products, reach the fp32 accumulation level."""
+    batch, M, N, K = shape
+    gen = torch.Generator(device="cuda").manual_seed(7)
+    A = torch.randn((batch, M, K), generator=gen, device="cuda").to(adt)
+    B = torch.randn((batch, N, K), generator=gen, device="cuda").to(bdt)
+    Ain = A.transpose(1, 2).contiguous() if a_mn else A
+    Bin = B.transpose(1, 2).contiguous() if b_mn else B
+    D = api.gemm(Ain, Bin, kind=kind, a_mn_major=bool(a_mn), b_mn_major=bool(b_mn))
+    ref = torch.bmm(A.double(), B.double().transpose(1, 2))
+    scale = torch.bmm(A.double().abs(), B.double().abs().transpose(1, 2))
+    rel = ((D.double() - ref).abs() / scale).max().item()
+    assert rel < 4 * 2.0 ** -24 * K ** 0.5, rel
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_split2_has_sixteen_bit_products(api, shape):
+    """Two planes per operand and three products: about 16 significant bits per
+    product, far better than one bf16 product, far from fp32."""
+    batch, M, N, K = shape
+    gen = torch.Generator(device="cuda").manual_seed(8)
+    A = torch.randn((batch, M, K), generator=gen, device="cuda")
+    B = torch.randn((batch, N, K), generator=gen, device="cuda")
+    D = api.gemm(A, B, kind="split2")
+    ref = torch.bmm(A.double(), B.double().transpose(1, 2))
+    scale = torch.bmm(A.double().abs(), B.double().abs().transpose(1, 2))
+    rel = ((D.double() - ref).abs() / scale).max().item()
+    assert rel < 2.0 ** -15, rel
