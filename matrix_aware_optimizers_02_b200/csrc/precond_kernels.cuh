@@ -294,23 +294,31 @@ __global__ void __launch_bounds__(256) soap_vperm_kernel(const VPermJob* __restr
 // diagonal QR factor either way.
 constexpr int kPanel = 128;
 constexpr int kPanelSq = kPanel * kPanel;
-constexpr int kLdA = kPanel + 1;
-constexpr int kCholSmem = (kPanel * kLdA + (kPanel - 32) * 32 + 2 * kPanel) * 8;
-constexpr int kMaxParts = 16;  // K slices of a panel Gram
+constexpr int kPackedUpper = kPanel * (kPanel + 1) / 2;  // packed upper triangle, row-major
+constexpr int kMaxParts = 16;                             // K slices of a panel Gram
+constexpr int kCholSmem = (kPackedUpper + (kPanel - 32) * 32 + 2 * kPanel) * 8;
 constexpr double kCholShift = 1e-5;  // relative to the unit diagonal of Gs
+constexpr double kFastTol = 1e-4;    // ||Gs - I||_F below which Rs^{-1} = I - U (first order)
 
 struct PanelJob {
   const float* part;     // nparts x kPanel x kPanel fp32 partial Grams (ld kPanel)
   __nv_bfloat16* rinv;   // three planes (kPanel x kPanel each) of R^{-1}: upper triangle, zero elsewhere
   int* bad;              // counts non-positive pivots
+  int* again;            // first pass: set to 1 when a second Cholesky-QR pass is needed, else 0
   const int* flag;
-  int w, nparts, shift;
+  int w, nparts;
+  int first;             // first pass of a panel: full factorisation is shifted, sets *again
 };
 
-__global__ void __launch_bounds__(256) qr_chol_kernel(const PanelJob* __restrict__ J) {
+// (r, c), r <= c, of the packed upper triangle
+__device__ __forceinline__ int pk(int r, int c) { return ((r * (2 * kPanel + 1 - r)) >> 1) + (c - r); }
+
+// Two blocks fit on an SM (shared memory and registers), so one block's serial
+// phases overlap the other's.
+__global__ void __launch_bounds__(256, 2) qr_chol_kernel(const PanelJob* __restrict__ J) {
   extern __shared__ double chol_smem[];
-  double* A = chol_smem;                 // [kPanel][kLdA]: Gs, then Rs (upper), then Rs^{-1} (upper)
-  double* T = A + kPanel * kLdA;         // [kPanel - 32][32] block-column workspace of the inverse
+  double* A = chol_smem;                 // packed upper: Gs, then Rs, then Rs^{-1}
+  double* T = A + kPackedUpper;          // [kPanel - 32][32] block-column workspace of the inverse
   double* ds = T + (kPanel - 32) * 32;   // D^-1/2
   double* rdi = ds + kPanel;             // 1 / Rs[k][k]
   const PanelJob& j = J[blockIdx.x];
@@ -320,45 +328,87 @@ __global__ void __launch_bounds__(256) qr_chol_kernel(const PanelJob* __restrict
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr unsigned FULL = 0xffffffffu;
 
-  // G: partials summed in slice order (all of a group's loads in flight at once);
-  // identity padding up to wp
+  // diagonal of G first (for the column scaling), then the scaled upper triangle;
+  // partial Grams are summed in slice order with all slices' loads in flight
+  if (tid < wp) {
+    double d = 1.0;
+    if (tid < w) {
+      d = 0.0;
+      for (int p = 0; p < j.nparts; ++p) d += (double)j.part[(long long)p * kPanelSq + tid * (kPanel + 1)];
+    }
+    ds[tid] = (d > 0.0) ? rsqrt(d) : 1.0;
+  }
+  __syncthreads();
   for (int q = tid; q < kPanelSq / 4; q += 256) {
     const int a = q >> 5, b0 = (q & 31) * 4;
-    if (a >= wp || b0 >= wp) continue;
+    if (a >= wp || b0 >= wp || b0 + 3 < a) continue;
     double g[4] = {0.0, 0.0, 0.0, 0.0};
     if (a < w) {
-      float4 v[kMaxParts];
 #pragma unroll
-      for (int p = 0; p < kMaxParts; ++p)
-        if (p < j.nparts) v[p] = *reinterpret_cast<const float4*>(j.part + (long long)p * kPanelSq + 4 * q);
+      for (int p0 = 0; p0 < kMaxParts; p0 += 8) {
+        float4 v[8];
 #pragma unroll
-      for (int p = 0; p < kMaxParts; ++p)
-        if (p < j.nparts) {
-          g[0] += (double)v[p].x;
-          g[1] += (double)v[p].y;
-          g[2] += (double)v[p].z;
-          g[3] += (double)v[p].w;
-        }
+        for (int p = 0; p < 8; ++p)
+          if (p0 + p < j.nparts) v[p] = *reinterpret_cast<const float4*>(j.part + (long long)(p0 + p) * kPanelSq + 4 * q);
+#pragma unroll
+        for (int p = 0; p < 8; ++p)
+          if (p0 + p < j.nparts) {
+            g[0] += (double)v[p].x;
+            g[1] += (double)v[p].y;
+            g[2] += (double)v[p].z;
+            g[3] += (double)v[p].w;
+          }
+      }
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int b = b0 + e;
-      A[a * kLdA + b] = (a < w && b < w) ? g[e] : (a == b ? 1.0 : 0.0);
+      if (b < a) continue;
+      A[pk(a, b)] = (a < w && b < w) ? g[e] * ds[a] * ds[b] : (a == b ? 1.0 : 0.0);
     }
   }
   __syncthreads();
-  if (tid < wp) {
-    const double d = A[tid * kLdA + tid];
-    ds[tid] = (d > 0.0) ? rsqrt(d) : 1.0;
+
+  // Nearly orthonormal panel (the common case after a first Cholesky-QR): with
+  // Gs = I + E and ||E||_F <= kFastTol, Rs = I + U + O(E^2) where U is the strict
+  // upper triangle of E plus half its diagonal, so Rs^{-1} = I - U to O(E^2) <= 1e-8,
+  // below the fp32 unit roundoff: no factorisation needed, and no second pass.
+  {
+    double e2 = 0.0;
+    for (int t = tid; t < wp * wp; t += 256) {
+      const int a = t / wp, b = t % wp;
+      if (b < a) continue;
+      const double e = A[pk(a, b)] - (a == b ? 1.0 : 0.0);
+      e2 += (a == b ? 1.0 : 2.0) * e * e;
+    }
+    e2 = warp_sum_d(e2);
+    if (lane == 0) T[warp] = e2;
+    __syncthreads();
+    double tot = 0.0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) tot += T[i];
+    __syncthreads();
+    if (tot <= kFastTol * kFastTol) {
+      for (int t = tid; t < kPanelSq; t += 256) {
+        const int r = t / kPanel, c = t % kPanel;
+        float x = 0.0f;
+        if (r <= c && c < w) {
+          const double e = A[pk(r, c)] - (r == c ? 1.0 : 0.0);
+          x = (float)(ds[r] * ((r == c ? 1.0 : 0.0) - (r == c ? 0.5 * e : e)));
+        }
+        store_split3(x, j.rinv, t, kPanelSq);
+      }
+      if (j.first && tid == 0) *j.again = 0;
+      return;
+    }
   }
-  __syncthreads();
-  for (int t = tid; t < wp * wp; t += 256) {
-    const int a = t / wp, b = t % wp;
-    double g = A[a * kLdA + b] * ds[a] * ds[b];
-    if (a == b && j.shift) g += kCholShift;
-    A[a * kLdA + b] = g;
+  // full factorisation; on a first pass shifted (robust for nearly dependent
+  // columns) and followed by a second pass
+  if (j.first) {
+    if (tid < wp) A[pk(tid, tid)] += kCholShift;
+    if (tid == 0) *j.again = 1;
+    __syncthreads();
   }
-  __syncthreads();
 
   // ---- blocked Cholesky, upper: Gs = Rs^T Rs
   for (int bk = 0; bk < nb; ++bk) {
@@ -368,7 +418,7 @@ __global__ void __launch_bounds__(256) qr_chol_kernel(const PanelJob* __restrict
       double v[32];
       int nbad = 0;
 #pragma unroll
-      for (int r = 0; r < 32; ++r) v[r] = (r <= lane) ? A[(o + r) * kLdA + o + lane] : 0.0;
+      for (int r = 0; r < 32; ++r) v[r] = (r <= lane) ? A[pk(o + r, o + lane)] : 0.0;
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
         double d = __shfl_sync(FULL, v[k], k);
@@ -388,7 +438,7 @@ __global__ void __launch_bounds__(256) qr_chol_kernel(const PanelJob* __restrict
       }
 #pragma unroll
       for (int r = 0; r < 32; ++r)
-        if (r <= lane) A[(o + r) * kLdA + o + lane] = v[r];
+        if (r <= lane) A[pk(o + r, o + lane)] = v[r];
       if (lane == 0 && nbad) atomicAdd(j.bad, nbad);
     }
     __syncthreads();
@@ -399,15 +449,16 @@ __global__ void __launch_bounds__(256) qr_chol_kernel(const PanelJob* __restrict
       const int c = o + 32 + tid;
       double x[32];
 #pragma unroll
-      for (int r = 0; r < 32; ++r) x[r] = A[(o + r) * kLdA + c];
+      for (int r = 0; r < 32; ++r) x[r] = A[pk(o + r, c)];
 #pragma unroll
       for (int r = 0; r < 32; ++r) {
         x[r] *= rdi[o + r];
+        const int base = pk(o + r, o);
 #pragma unroll
-        for (int i = r + 1; i < 32; ++i) x[i] -= A[(o + r) * kLdA + o + i] * x[r];
+        for (int i = r + 1; i < 32; ++i) x[i] -= A[base + i] * x[r];
       }
 #pragma unroll
-      for (int r = 0; r < 32; ++r) A[(o + r) * kLdA + c] = x[r];
+      for (int r = 0; r < 32; ++r) A[pk(o + r, c)] = x[r];
     }
     __syncthreads();
     // trailing update of the upper triangle: G_cd -= Rs_bc^T Rs_bd, c <= d
@@ -417,63 +468,67 @@ __global__ void __launch_bounds__(256) qr_chol_kernel(const PanelJob* __restrict
       double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
 #pragma unroll
       for (int i = 0; i < 32; i += 4) {
-        s0 += A[(o + i) * kLdA + c] * A[(o + i) * kLdA + d];
-        s1 += A[(o + i + 1) * kLdA + c] * A[(o + i + 1) * kLdA + d];
-        s2 += A[(o + i + 2) * kLdA + c] * A[(o + i + 2) * kLdA + d];
-        s3 += A[(o + i + 3) * kLdA + c] * A[(o + i + 3) * kLdA + d];
+        const int r0 = pk(o + i, 0), r1 = pk(o + i + 1, 0), r2 = pk(o + i + 2, 0), r3 = pk(o + i + 3, 0);
+        s0 += A[r0 + c] * A[r0 + d];
+        s1 += A[r1 + c] * A[r1 + d];
+        s2 += A[r2 + c] * A[r2 + d];
+        s3 += A[r3 + c] * A[r3 + d];
       }
-      A[c * kLdA + d] -= (s0 + s1) + (s2 + s3);
+      A[pk(c, d)] -= (s0 + s1) + (s2 + s3);
     }
     __syncthreads();
   }
 
-  // ---- blocked inverse in place, by block columns: X_jj = Rs_jj^{-1};
-  //      X_ij = -(sum_{k=i..j-1} X_ik Rs_kj) X_jj for block rows i < j
-  for (int bj = 0; bj < nb; ++bj) {
+  // ---- inverse in place.  Diagonal blocks first, one warp each: column c = lane of
+  // Rs_bb^{-1}, from the last row up, written over Rs_bb as it goes (row k of the
+  // block is not read again once step k is done).
+  if (warp < nb) {
+    const int o = warp * 32;
+    double acc[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] = 0.0;
+#pragma unroll
+    for (int k = 31; k >= 0; --k) {
+      const double ri = rdi[o + k];
+      const double xk = (k == lane) ? ri : (k < lane ? -acc[k] * ri : 0.0);
+#pragma unroll
+      for (int i = 0; i < 31; ++i)
+        if (i < k) acc[i] += A[pk(o + i, o + k)] * xk;
+      __syncwarp();
+      if (k <= lane) A[pk(o + k, o + lane)] = xk;
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  // off-diagonal blocks by block columns: X_ij = -(sum_{k=i..j-1} X_ik Rs_kj) X_jj, i < j
+  for (int bj = 1; bj < nb; ++bj) {
     const int oj = bj * 32;
-    // T[r][c] = sum_{k = r .. oj-1} X[r][k] Rs[k][oj + c]  (X upper: k >= r)
+    // T[r][c] = sum_{k = r .. oj-1} X[r][k] Rs[k][oj + c]
     for (int t = tid; t < oj * 32; t += 256) {
       const int r = t >> 5, c = t & 31;
       double s0 = 0.0, s1 = 0.0;
       int k = r;
+      const int rb = pk(r, 0);
       for (; k + 1 < oj; k += 2) {
-        s0 += A[r * kLdA + k] * A[k * kLdA + oj + c];
-        s1 += A[r * kLdA + k + 1] * A[(k + 1) * kLdA + oj + c];
+        s0 += A[rb + k] * A[pk(k, oj + c)];
+        s1 += A[rb + k + 1] * A[pk(k + 1, oj + c)];
       }
-      if (k < oj) s0 += A[r * kLdA + k] * A[k * kLdA + oj + c];
+      if (k < oj) s0 += A[rb + k] * A[pk(k, oj + c)];
       T[r * 32 + c] = s0 + s1;
     }
-    if (warp == 0) {
-      // column c = lane of Rs_jj^{-1}, from the last row up (right-looking in registers)
-      double acc[32], x[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] = 0.0;
-#pragma unroll
-      for (int k = 31; k >= 0; --k) {
-        const double ri = rdi[oj + k];
-        x[k] = (k == lane) ? ri : (k < lane ? -acc[k] * ri : 0.0);
-#pragma unroll
-        for (int i = 0; i < k; ++i) acc[i] += A[(oj + i) * kLdA + oj + k] * x[k];
-      }
-      __syncwarp();
-#pragma unroll
-      for (int r = 0; r < 32; ++r)
-        if (r <= lane) A[(oj + r) * kLdA + oj + lane] = x[r];
-    }
     __syncthreads();
-    // X_i,j = -T_i X_jj
     for (int t = tid; t < oj * 32; t += 256) {
       const int r = t >> 5, c = t & 31;
       double s = 0.0;
-      for (int m = 0; m <= c; ++m) s += T[r * 32 + m] * A[(oj + m) * kLdA + oj + c];
-      A[r * kLdA + oj + c] = -s;
+      for (int m = 0; m <= c; ++m) s += T[r * 32 + m] * A[pk(oj + m, oj + c)];
+      A[pk(r, oj + c)] = -s;
     }
     __syncthreads();
   }
   // R^{-1} = D^-1/2 Rs^{-1}: three bf16 planes over the full kPanel x kPanel square
   for (int t = tid; t < kPanelSq; t += 256) {
     const int r = t / kPanel, c = t % kPanel;
-    const float x = (r <= c && c < w) ? (float)(ds[r] * A[r * kLdA + c]) : 0.0f;
+    const float x = (r <= c && c < w) ? (float)(ds[r] * A[pk(r, c)]) : 0.0f;
     store_split3(x, j.rinv, t, kPanelSq);
   }
 }

@@ -93,8 +93,8 @@ inline size_t planes_bytes(int rows, int cols) { return 3 * 2 * (size_t)rows * l
 // Scratch of one side (k x k factor F with basis Q) of one matrix.
 struct SideBuf {
   size_t Fp, Qp, P, Ps, Psp;
-  size_t W, Wp, Wb, Wbp, Cp;  // panel ping-pong buffers (k x kPanel) and the coefficients
-  size_t part, rinv, keys, perm, flag, rho, bad;
+  size_t W, Wp, Cp;  // panel buffer (k x kPanel, fp32 and planes) and the coefficients
+  size_t part, rinv, keys, perm, flag, rho, bad, again;
   size_t Tp, D;  // adaptive check
 };
 
@@ -115,16 +115,15 @@ void side_layout(int k, bool check, Carver& cv, SideBuf& s, size_t flag_block) {
   s.Psp = cv.take(planes_bytes(k, k));
   s.W = cv.take(4 * (size_t)k * kPanel);
   s.Wp = cv.take(planes_bytes(k, kPanel));
-  s.Wb = cv.take(4 * (size_t)k * kPanel);
-  s.Wbp = cv.take(planes_bytes(k, kPanel));
   s.Cp = cv.take(planes_bytes(k, kPanel));
   s.part = cv.take(4 * (size_t)parts * kPanelSq);
   s.rinv = cv.take(2 * 3 * (size_t)kPanelSq);
   s.keys = cv.take(8 * (size_t)k);
   s.perm = cv.take(4 * (size_t)k);
-  s.flag = flag_block;  // flag, rho and the failure counter share one 64-byte block
+  s.flag = flag_block;  // flag, rho, the failure counter and the second-pass flag share one 64-byte block
   s.rho = s.flag + 16;
   s.bad = s.flag + 32;
+  s.again = s.flag + 48;
   if (check) {
     s.Tp = cv.take(planes_bytes(k, k));
     s.D = cv.take(4 * kk);
@@ -279,23 +278,38 @@ int ew_blocks(int rows, int cols) {
   return (int)((e + kElemsPerBlock - 1) / kElemsPerBlock);
 }
 
-// Adds the jobs of one side's refresh for every matrix of the group.
-mao_status build_refresh_side(Builder& B, GroupPlan& G, bool left) {
+// Adds the jobs of the basis refresh of every factor of the group: both sides of
+// every SOAP matrix and the input side of every FOAM matrix, swept together so
+// that each launch covers all of them (and the QR advances every factor by one
+// panel per step).
+mao_status build_refresh(Builder& B, GroupPlan& G) {
   const Ctx& X = B.X;
   const bool check = X.mode == 2;
   const int nm = G.g1 - G.g0;
-  auto side = [&](int i) -> SideBuf& { return left ? G.mb[i].L : G.mb[i].R; };
-  auto kof = [&](int i) { return left ? X.mats[G.g0 + i].m : X.mats[G.g0 + i].n; };
-  auto Fp = [&](int i) { return left ? X.mats[G.g0 + i].L : X.mats[G.g0 + i].R; };
-  auto Qp = [&](int i) { return left ? X.mats[G.g0 + i].QL : X.mats[G.g0 + i].QR; };
-  auto flagp = [&](int i) -> const int* { return check ? B.wp<int>(side(i).flag) : nullptr; };
+  struct Unit {
+    int i;
+    bool left;
+  };
+  std::vector<Unit> units;
+  for (int i = 0; i < nm; ++i) {
+    if (!X.foam) units.push_back({i, true});
+    units.push_back({i, false});
+  }
+  const int nu = (int)units.size();
+  auto side = [&](int u) -> SideBuf& { return units[u].left ? G.mb[units[u].i].L : G.mb[units[u].i].R; };
+  auto mat = [&](int u) -> const PcMat& { return X.mats[G.g0 + units[u].i]; };
+  auto kof = [&](int u) { return units[u].left ? mat(u).m : mat(u).n; };
+  auto Fp = [&](int u) { return units[u].left ? mat(u).L : mat(u).R; };
+  auto Qp = [&](int u) { return units[u].left ? mat(u).QL : mat(u).QR; };
+  auto permo = [&](int u) { return units[u].left ? mat(u).perm_L : mat(u).perm_R; };
+  auto flagp = [&](int u) -> const int* { return check ? B.wp<int>(side(u).flag) : nullptr; };
 
   // three-plane splits of F and Q
   {
     size_t off;
-    EwJob* J = B.new_jobs<EwJob>(Op::SPLIT, 2 * nm, off);
+    EwJob* J = B.new_jobs<EwJob>(Op::SPLIT, 2 * nu, off);
     int blk = 0;
-    for (int i = 0; i < nm; ++i) {
+    for (int i = 0; i < nu; ++i) {
       const int k = kof(i);
       for (int w = 0; w < 2; ++w) {
         EwJob& j = J[2 * i + w];
@@ -315,32 +329,32 @@ mao_status build_refresh_side(Builder& B, GroupPlan& G, bool left) {
   if (check) {
     // D = Q^T F Q: T = Q^T F (A = Q stored K x M), D = T Q (B = Q stored K x N)
     TableLaunch& g1 = B.new_gemm(1, 1, MAO_K_PC_CHECK);
-    for (int i = 0; i < nm; ++i) {
+    for (int i = 0; i < nu; ++i) {
       const int k = kof(i);
       const Split3 Tp = B.planes(side(i).Tp, k, k);
       MAO_TRY(table_add(g1, B.maps, B.planes(side(i).Qp, k, k), B.planes(side(i).Fp, k, k), k, k, k, 0, 0, nullptr,
                         &Tp, k, nullptr, 0, 1.f, 0.f, nullptr));
     }
     TableLaunch& g2 = B.new_gemm(0, 1, MAO_K_PC_CHECK);
-    for (int i = 0; i < nm; ++i) {
+    for (int i = 0; i < nu; ++i) {
       const int k = kof(i);
       MAO_TRY(table_add(g2, B.maps, B.planes(side(i).Tp, k, k), B.planes(side(i).Qp, k, k), k, k, k, 0, 0,
                         B.wp<float>(side(i).D), nullptr, k, nullptr, 0, 1.f, 0.f, nullptr));
     }
     size_t off;
-    CheckJob* J = B.new_jobs<CheckJob>(Op::CHECK, nm, off);
-    for (int i = 0; i < nm; ++i) {
+    CheckJob* J = B.new_jobs<CheckJob>(Op::CHECK, nu, off);
+    for (int i = 0; i < nu; ++i) {
       J[i].D = B.wp<float>(side(i).D);
       J[i].flag = B.wp<int>(side(i).flag);
       J[i].rho = B.wp<float>(side(i).rho);
       J[i].k = kof(i);
     }
-    B.ops.back().blocks = nm;
+    B.ops.back().blocks = nu;
   }
   // power step P = F Q (A = F K-major, B = Q stored K x N)
   {
     TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_POWER);
-    for (int i = 0; i < nm; ++i) {
+    for (int i = 0; i < nu; ++i) {
       const int k = kof(i);
       MAO_TRY(table_add(g, B.maps, B.planes(side(i).Fp, k, k), B.planes(side(i).Qp, k, k), k, k, k, 0, 0,
                         B.wp<float>(side(i).P), nullptr, k, nullptr, 0, 1.f, 0.f, flagp(i)));
@@ -349,16 +363,16 @@ mao_status build_refresh_side(Builder& B, GroupPlan& G, bool left) {
   // keys and argsort
   {
     size_t off;
-    SortJob* J = B.new_jobs<SortJob>(Op::KEYS, nm, off);
+    SortJob* J = B.new_jobs<SortJob>(Op::KEYS, nu, off);
     int blk = 0;
-    for (int i = 0; i < nm; ++i) {
+    for (int i = 0; i < nu; ++i) {
       const int k = kof(i);
       SortJob& j = J[i];
       j.Q = Qp(i);
       j.P = B.wp<float>(side(i).P);
       j.key = B.wp<double>(side(i).keys);
       j.perm = B.wp<int>(side(i).perm);
-      j.perm_out = left ? X.mats[G.g0 + i].perm_L : X.mats[G.g0 + i].perm_R;
+      j.perm_out = permo(i);
       j.flag = flagp(i);
       j.k = k;
       j.col_blk_begin = blk;
@@ -373,9 +387,9 @@ mao_status build_refresh_side(Builder& B, GroupPlan& G, bool left) {
   // gathered P and its planes
   {
     size_t off;
-    GatherJob* J = B.new_jobs<GatherJob>(Op::GATHER, nm, off);
+    GatherJob* J = B.new_jobs<GatherJob>(Op::GATHER, nu, off);
     int blk = 0;
-    for (int i = 0; i < nm; ++i) {
+    for (int i = 0; i < nu; ++i) {
       const int k = kof(i);
       GatherJob& j = J[i];
       j.src = B.wp<float>(side(i).P);
@@ -396,13 +410,13 @@ mao_status build_refresh_side(Builder& B, GroupPlan& G, bool left) {
   // QR by panels of kPanel columns: block Gram-Schmidt with two projection passes,
   // Cholesky-QR inside each panel (twice after the first pass, once after the second)
   int maxk = 0;
-  for (int i = 0; i < nm; ++i) maxk = std::max(maxk, kof(i));
+  for (int i = 0; i < nu; ++i) maxk = std::max(maxk, kof(i));
   const int npanels = (maxk + kPanel - 1) / kPanel;
-  enum { PS = 0, WA = 1, WB = 2, QF = 3 };
+  enum { PS = 0, WA = 1, QF = 2 };
   for (int pj = 0; pj < npanels; ++pj) {
     const int c0 = pj * kPanel;
     std::vector<int> act;
-    for (int i = 0; i < nm; ++i)
+    for (int i = 0; i < nu; ++i)
       if (kof(i) > c0) act.push_back(i);
     auto wdt = [&](int i) { return std::min(kPanel, kof(i) - c0); };
     // a panel's fp32 storage and plane view (columns c0 .. c0 + w of Ps / Q, or a scratch buffer)
@@ -411,7 +425,6 @@ mao_status build_refresh_side(Builder& B, GroupPlan& G, bool left) {
       switch (where) {
         case PS: *ld = k; return B.wp<float>(side(i).Ps) + c0;
         case WA: *ld = kPanel; return B.wp<float>(side(i).W);
-        case WB: *ld = kPanel; return B.wp<float>(side(i).Wb);
         default: *ld = k; return Qp(i) + c0;
       }
     };
@@ -421,7 +434,6 @@ mao_status build_refresh_side(Builder& B, GroupPlan& G, bool left) {
       switch (where) {
         case PS: v = B.planes(side(i).Psp, k, k); break;
         case WA: v = B.planes(side(i).Wp, k, kPanel); break;
-        case WB: v = B.planes(side(i).Wbp, k, kPanel); break;
         default: v = B.planes(side(i).Qp, k, k); break;
       }
       if (where == PS || where == QF)
@@ -429,9 +441,11 @@ mao_status build_refresh_side(Builder& B, GroupPlan& G, bool left) {
       v.cols = w;
       return v;
     };
-    // one Cholesky-QR of every active panel: dst = src R^{-1}; `shift` regularises
-    // the factorisation of a panel that may be nearly rank deficient
-    auto cholqr = [&](int src, int dst, bool shift) -> mao_status {
+    // one Cholesky-QR of every active panel: dst = src R^{-1} (dst may be src).
+    // pass 0: first pass (decides whether pass 1 runs); 1: the gated second pass;
+    // 2: an ungated pass on a nearly orthonormal panel
+    auto cholqr = [&](int src, int dst, int pass) -> mao_status {
+      auto gate = [&](int u) -> const int* { return pass == 1 ? B.wp<int>(side(u).again) : flagp(u); };
       // Gram partials over K slices (fp32-faithful), one 128 x 128 tile each
       TableLaunch& gg = B.new_gemm(1, 1, MAO_K_PC_PANEL);
       const int nact = (int)act.size();
@@ -442,7 +456,7 @@ mao_status build_refresh_side(Builder& B, GroupPlan& G, bool left) {
         const Split3 Wv = pv(i, src);
         for (int s0 = 0, p = 0; s0 < k; s0 += sl, ++p)
           MAO_TRY(table_add(gg, B.maps, Wv, Wv, w, w, std::min(sl, k - s0), 0, 0, part + (size_t)p * kPanelSq,
-                            nullptr, kPanel, nullptr, 0, 1.f, 0.f, flagp(i), s0));
+                            nullptr, kPanel, nullptr, 0, 1.f, 0.f, gate(i), s0));
       }
       size_t off;
       PanelJob* J = B.new_jobs<PanelJob>(Op::CHOL, (int)act.size(), off);
@@ -453,10 +467,11 @@ mao_status build_refresh_side(Builder& B, GroupPlan& G, bool left) {
         j.part = B.wp<float>(side(i).part);
         j.rinv = B.wp<__nv_bfloat16>(side(i).rinv);
         j.bad = B.wp<int>(side(i).bad);
-        j.flag = flagp(i);
+        j.again = B.wp<int>(side(i).again);
+        j.flag = gate(i);
         j.w = wdt(i);
         j.nparts = (k + gram_slice(k, nact) - 1) / gram_slice(k, nact);
-        j.shift = shift ? 1 : 0;
+        j.first = pass == 0 ? 1 : 0;
       }
       B.ops.back().blocks = (int)act.size();
       TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_QR);
@@ -468,7 +483,7 @@ mao_status build_refresh_side(Builder& B, GroupPlan& G, bool left) {
         int ld = 0;
         float* out = fp(i, dst, &ld);
         MAO_TRY(table_add(g, B.maps, pv(i, src), Ri, k, w, w, 0, 0, out, &out_p, ld, nullptr, 0, 1.f, 0.f,
-                          flagp(i)));
+                          gate(i)));
       }
       return MAO_OK;
     };
@@ -497,15 +512,17 @@ mao_status build_refresh_side(Builder& B, GroupPlan& G, bool left) {
       }
       return MAO_OK;
     };
+    // The products W R^{-1} run in place (each output row block reads only its own
+    // rows of W, all of K in one tile).
     if (pj == 0) {
-      MAO_TRY(cholqr(PS, WB, true));
-      MAO_TRY(cholqr(WB, QF, false));
+      MAO_TRY(cholqr(PS, WA, 0));
+      MAO_TRY(cholqr(WA, QF, 2));
     } else {
       MAO_TRY(project(PS));
-      MAO_TRY(cholqr(WA, WB, true));
-      MAO_TRY(cholqr(WB, WA, false));
+      MAO_TRY(cholqr(WA, WA, 0));
+      MAO_TRY(cholqr(WA, WA, 1));
       MAO_TRY(project(WA));
-      MAO_TRY(cholqr(WA, QF, false));
+      MAO_TRY(cholqr(WA, QF, 2));
     }
   }
   return MAO_OK;
@@ -581,8 +598,7 @@ mao_status build_group(Builder& B, GroupPlan& G) {
   }
   // refresh, or plain planes of the bases
   if (X.mode != 0) {
-    if (!foam) MAO_TRY(build_refresh_side(B, G, true));
-    MAO_TRY(build_refresh_side(B, G, false));
+    MAO_TRY(build_refresh(B, G));
   } else {
     size_t off;
     const int per = foam ? 1 : 2;
