@@ -302,8 +302,8 @@ typedef enum {
   MAO_K_PC_QR = 18,          /* QR tensor-core products: panel projections, W R^{-1} */
   MAO_K_PC_ROTATE = 19,      /* rotations into the eigenbasis and back (before the update) */
   MAO_K_PC_UPDATE = 20,      /* last rotation fused with the weight update */
-  MAO_K_PC_PANEL = 21,       /* QR panel Gram products (tensor cores, K slices) */
-  MAO_K_PC_CHOL = 22         /* QR panel Cholesky and R^{-1} (fp64, one block per matrix) */
+  MAO_K_PC_PANEL = 21,       /* QR panel Gram products (tensor cores, K slices) and their reduction */
+  MAO_K_PC_CHOL = 22         /* QR panel Cholesky and R^{-1} (fp64, one block per panel) */
 } mao_kernel_id;
 
 /* What one recorded launch was: its kernel and its algorithmic work (useful

@@ -284,43 +284,133 @@ __global__ void __launch_bounds__(256) soap_vperm_kernel(const VPermJob* __restr
 // ------------------------------------------------------------------ QR panel pieces
 // Cholesky-QR of one panel W (rows x w, w <= kPanel) per matrix:
 //   Gram G = W^T W as fp32-faithful tensor-core products over K slices (fp32
-//   partials, summed here in fp64 in slice order)
-//   -> column scaling Gs = D^-1/2 G D^-1/2 (D = diag G), optional diagonal shift
-//   -> blocked Cholesky Gs = Rs^T Rs and blocked inverse Rs^-1 (fp64, one block per matrix)
-//   -> R^{-1} = D^-1/2 Rs^{-1}, written as three bf16 planes for the product W R^{-1}.
-// The shift (first Cholesky-QR of a panel only) keeps the factorisation defined
-// for nearly dependent columns; the following unshifted pass restores
-// orthogonality, and the triangular structure makes the final Q the positive-
-// diagonal QR factor either way.
+//   partials)
+//   -> reduction (many blocks per panel): the slices summed in fp64 in slice order,
+//      column scaling Gs = D^-1/2 G D^-1/2 (D = diag G), the packed upper triangle of
+//      Gs, ||Gs - I||_F partials, and the first-order inverse factor (below)
+//   -> Cholesky Gs = Rs^T Rs and blocked inverse Rs^-1 in fp64, one block per
+//      panel, only when Gs is not already close to the identity
+//   -> R^{-1} = D^-1/2 Rs^{-1}, three bf16 planes, for the product W R^{-1}.
+// Nearly orthonormal panel (the usual case after a first Cholesky-QR): with
+// Gs = I + E and ||E||_F <= kFastTol, Rs = I + U + O(E^2) where U is the strict
+// upper triangle of E plus half its diagonal, so Rs^{-1} = I - U to O(E^2) <= 1e-8,
+// below the fp32 unit roundoff.
+// A first pass of a panel that needs the full factorisation shifts Gs by
+// kCholShift (by kCholShiftRetry after a breakdown) so it stays defined for nearly
+// dependent columns, and asks for a second pass, which restores orthogonality; the
+// triangular structure makes the final Q the positive-diagonal QR factor either way.
 constexpr int kPanel = 128;
 constexpr int kPanelSq = kPanel * kPanel;
 constexpr int kPackedUpper = kPanel * (kPanel + 1) / 2;  // packed upper triangle, row-major
 constexpr int kMaxParts = 16;                             // K slices of a panel Gram
+constexpr int kRedRows = 8;                               // Gram rows per reduction block
+constexpr int kRedBlocks = kPanel / kRedRows;
+constexpr int kGsDoubles = kPackedUpper + kPanel + kRedBlocks;  // Gs | D^-1/2 | ||E||^2 partials
 constexpr int kCholSmem = (kPackedUpper + (kPanel - 32) * 32 + 2 * kPanel) * 8;
-constexpr double kCholShift = 1e-5;  // relative to the unit diagonal of Gs
-constexpr double kFastTol = 1e-4;    // ||Gs - I||_F below which Rs^{-1} = I - U (first order)
+constexpr double kCholShift = 1e-6;       // relative to the unit diagonal of Gs
+constexpr double kCholShiftRetry = 1e-4;  // after a non-positive pivot
+constexpr double kFastTol = 1e-4;
 
 struct PanelJob {
   const float* part;     // nparts x kPanel x kPanel fp32 partial Grams (ld kPanel)
+  double* gs;            // kGsDoubles
   __nv_bfloat16* rinv;   // three planes (kPanel x kPanel each) of R^{-1}: upper triangle, zero elsewhere
-  int* bad;              // counts non-positive pivots
+  int* bad;              // counts panels whose shifted factorisation still broke down
   int* again;            // first pass: set to 1 when a second Cholesky-QR pass is needed, else 0
+  const float* pnorm2;   // first pass after a projection: squared norms of the panel's columns
+                         // before the projection (else nullptr)
+  int* reorth;           // ... and the flag set to 1 when a second projection is needed, else 0
   const int* flag;
   int w, nparts;
-  int first;             // first pass of a panel: full factorisation is shifted, sets *again
+  int first;
 };
+
+// Selective reorthogonalisation (the classical criterion of Daniel, Gragg, Kaufman
+// and Stewart, per column): a second projection pass is needed when the first pass
+// removed more than half of some column's squared norm.
+constexpr double kReorthRatio = 0.5;
 
 // (r, c), r <= c, of the packed upper triangle
 __device__ __forceinline__ int pk(int r, int c) { return ((r * (2 * kPanel + 1 - r)) >> 1) + (c - r); }
 
-// Two blocks fit on an SM (shared memory and registers), so one block's serial
-// phases overlap the other's.
-__global__ void __launch_bounds__(256, 2) qr_chol_kernel(const PanelJob* __restrict__ J) {
+// kRedBlocks blocks per panel, block rb owns Gram rows [rb*kRedRows, +kRedRows).
+__global__ void __launch_bounds__(256) qr_gram_reduce_kernel(const PanelJob* __restrict__ J) {
+  __shared__ double dsh[kPanel];
+  __shared__ double red[8];
+  const PanelJob& j = J[blockIdx.x / kRedBlocks];
+  const int rb = blockIdx.x % kRedBlocks;
+  if (j.flag && *j.flag == 0) return;
+  const int w = j.w, tid = threadIdx.x;
+  int cancel = 0;
+  if (tid < kPanel) {
+    double d = 1.0;
+    if (tid < w) {
+      float v[kMaxParts];
+#pragma unroll
+      for (int p = 0; p < kMaxParts; ++p)
+        v[p] = p < j.nparts ? j.part[(long long)p * kPanelSq + tid * (kPanel + 1)] : 0.0f;
+      d = 0.0;
+#pragma unroll
+      for (int p = 0; p < kMaxParts; ++p) d += (double)v[p];
+      if (j.pnorm2 && rb == 0) cancel = d < kReorthRatio * (double)j.pnorm2[tid];
+    }
+    const double s = (d > 0.0) ? rsqrt(d) : 1.0;
+    dsh[tid] = s;
+    if (rb == 0) j.gs[kPackedUpper + tid] = s;
+  }
+  cancel = __syncthreads_or(cancel);
+  if (j.pnorm2 && rb == 0 && tid == 0) *j.reorth = cancel ? 1 : 0;
+  // one 4-column group of one row per thread
+  const int a = rb * kRedRows + (tid >> 5), b0 = (tid & 31) * 4;
+  double g[4] = {0.0, 0.0, 0.0, 0.0};
+  if (a < w && b0 < w) {
+    float4 v[kMaxParts];
+#pragma unroll
+    for (int p = 0; p < kMaxParts; ++p)
+      if (p < j.nparts) v[p] = *reinterpret_cast<const float4*>(j.part + (long long)p * kPanelSq + a * kPanel + b0);
+#pragma unroll
+    for (int p = 0; p < kMaxParts; ++p)
+      if (p < j.nparts) {
+        g[0] += (double)v[p].x;
+        g[1] += (double)v[p].y;
+        g[2] += (double)v[p].z;
+        g[3] += (double)v[p].w;
+      }
+  }
+  double e2 = 0.0;
+  float rv[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int b = b0 + e;
+    const double id = (a == b) ? 1.0 : 0.0;
+    const double x = (a < w && b < w) ? g[e] * dsh[a] * dsh[b] : id;
+    rv[e] = 0.0f;
+    if (b >= a) {
+      j.gs[pk(a, b)] = x;
+      const double ee = x - id;
+      e2 += (a == b ? 1.0 : 2.0) * ee * ee;
+      if (b < w) rv[e] = (float)(dsh[a] * (id - (a == b ? 0.5 * ee : ee)));
+    }
+  }
+  store_split3x4(make_float4(rv[0], rv[1], rv[2], rv[3]), j.rinv, (long long)a * kPanel + b0, kPanelSq);
+  e2 = warp_sum_d(e2);
+  if ((tid & 31) == 0) red[tid >> 5] = e2;
+  __syncthreads();
+  if (tid == 0) {
+    double t = 0.0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) t += red[i];
+    j.gs[kPackedUpper + kPanel + rb] = t;
+  }
+}
+
+__global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restrict__ J) {
   extern __shared__ double chol_smem[];
   double* A = chol_smem;                 // packed upper: Gs, then Rs, then Rs^{-1}
   double* T = A + kPackedUpper;          // [kPanel - 32][32] block-column workspace of the inverse
   double* ds = T + (kPanel - 32) * 32;   // D^-1/2
   double* rdi = ds + kPanel;             // 1 / Rs[k][k]
+  __shared__ int nbad_sh;
   const PanelJob& j = J[blockIdx.x];
   if (j.flag && *j.flag == 0) return;
   const int w = j.w;
@@ -328,88 +418,26 @@ __global__ void __launch_bounds__(256, 2) qr_chol_kernel(const PanelJob* __restr
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr unsigned FULL = 0xffffffffu;
 
-  // diagonal of G first (for the column scaling), then the scaled upper triangle;
-  // partial Grams are summed in slice order with all slices' loads in flight
-  if (tid < wp) {
-    double d = 1.0;
-    if (tid < w) {
-      d = 0.0;
-      for (int p = 0; p < j.nparts; ++p) d += (double)j.part[(long long)p * kPanelSq + tid * (kPanel + 1)];
-    }
-    ds[tid] = (d > 0.0) ? rsqrt(d) : 1.0;
+  double tot = 0.0;
+#pragma unroll
+  for (int i = 0; i < kRedBlocks; ++i) tot += j.gs[kPackedUpper + kPanel + i];
+  if (tot <= kFastTol * kFastTol) {  // the first-order inverse is already in place
+    if (j.first && tid == 0) *j.again = 0;
+    return;
   }
-  __syncthreads();
-  for (int q = tid; q < kPanelSq / 4; q += 256) {
-    const int a = q >> 5, b0 = (q & 31) * 4;
-    if (a >= wp || b0 >= wp || b0 + 3 < a) continue;
-    double g[4] = {0.0, 0.0, 0.0, 0.0};
-    if (a < w) {
-#pragma unroll
-      for (int p0 = 0; p0 < kMaxParts; p0 += 8) {
-        float4 v[8];
-#pragma unroll
-        for (int p = 0; p < 8; ++p)
-          if (p0 + p < j.nparts) v[p] = *reinterpret_cast<const float4*>(j.part + (long long)(p0 + p) * kPanelSq + 4 * q);
-#pragma unroll
-        for (int p = 0; p < 8; ++p)
-          if (p0 + p < j.nparts) {
-            g[0] += (double)v[p].x;
-            g[1] += (double)v[p].y;
-            g[2] += (double)v[p].z;
-            g[3] += (double)v[p].w;
-          }
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int b = b0 + e;
-      if (b < a) continue;
-      A[pk(a, b)] = (a < w && b < w) ? g[e] * ds[a] * ds[b] : (a == b ? 1.0 : 0.0);
-    }
-  }
-  __syncthreads();
+  if (tid < kPanel) ds[tid] = j.gs[kPackedUpper + tid];
 
-  // Nearly orthonormal panel (the common case after a first Cholesky-QR): with
-  // Gs = I + E and ||E||_F <= kFastTol, Rs = I + U + O(E^2) where U is the strict
-  // upper triangle of E plus half its diagonal, so Rs^{-1} = I - U to O(E^2) <= 1e-8,
-  // below the fp32 unit roundoff: no factorisation needed, and no second pass.
-  {
-    double e2 = 0.0;
-    for (int t = tid; t < wp * wp; t += 256) {
-      const int a = t / wp, b = t % wp;
-      if (b < a) continue;
-      const double e = A[pk(a, b)] - (a == b ? 1.0 : 0.0);
-      e2 += (a == b ? 1.0 : 2.0) * e * e;
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    {
+      const double2* src = reinterpret_cast<const double2*>(j.gs);
+      double2* dst = reinterpret_cast<double2*>(A);
+      for (int q = tid; q < kPackedUpper / 2; q += 256) dst[q] = src[q];
     }
-    e2 = warp_sum_d(e2);
-    if (lane == 0) T[warp] = e2;
+    if (tid == 0) nbad_sh = 0;
     __syncthreads();
-    double tot = 0.0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) tot += T[i];
+    const double shift = attempt ? kCholShiftRetry : (j.first ? kCholShift : 0.0);
+    if (tid < wp && shift > 0.0) A[pk(tid, tid)] += shift;
     __syncthreads();
-    if (tot <= kFastTol * kFastTol) {
-      for (int t = tid; t < kPanelSq; t += 256) {
-        const int r = t / kPanel, c = t % kPanel;
-        float x = 0.0f;
-        if (r <= c && c < w) {
-          const double e = A[pk(r, c)] - (r == c ? 1.0 : 0.0);
-          x = (float)(ds[r] * ((r == c ? 1.0 : 0.0) - (r == c ? 0.5 * e : e)));
-        }
-        store_split3(x, j.rinv, t, kPanelSq);
-      }
-      if (j.first && tid == 0) *j.again = 0;
-      return;
-    }
-  }
-  // full factorisation; on a first pass shifted (robust for nearly dependent
-  // columns) and followed by a second pass
-  if (j.first) {
-    if (tid < wp) A[pk(tid, tid)] += kCholShift;
-    if (tid == 0) *j.again = 1;
-    __syncthreads();
-  }
-
   // ---- blocked Cholesky, upper: Gs = Rs^T Rs
   for (int bk = 0; bk < nb; ++bk) {
     const int o = bk * 32;
@@ -439,7 +467,7 @@ __global__ void __launch_bounds__(256, 2) qr_chol_kernel(const PanelJob* __restr
 #pragma unroll
       for (int r = 0; r < 32; ++r)
         if (r <= lane) A[pk(o + r, o + lane)] = v[r];
-      if (lane == 0 && nbad) atomicAdd(j.bad, nbad);
+      if (lane == 0 && nbad) nbad_sh += nbad;
     }
     __syncthreads();
     const int nt = wp - o - 32;  // trailing columns
@@ -477,6 +505,14 @@ __global__ void __launch_bounds__(256, 2) qr_chol_kernel(const PanelJob* __restr
       A[pk(c, d)] -= (s0 + s1) + (s2 + s3);
     }
     __syncthreads();
+  }
+    __syncthreads();
+    if (nbad_sh == 0 || attempt == 1) break;  // retry once with the larger shift
+    __syncthreads();
+  }
+  if (tid == 0) {
+    if (nbad_sh) atomicAdd(j.bad, 1);
+    if (j.first) *j.again = 1;
   }
 
   // ---- inverse in place.  Diagonal blocks first, one warp each: column c = lane of
@@ -531,6 +567,102 @@ __global__ void __launch_bounds__(256, 2) qr_chol_kernel(const PanelJob* __restr
     const float x = (r <= c && c < w) ? (float)(ds[r] * A[pk(r, c)]) : 0.0f;
     store_split3(x, j.rinv, t, kPanelSq);
   }
+}
+
+// Sum of the K-slice partials of a panel's projection coefficients C (rows x
+// kPanel fp32 each, in slice order), written as three bf16 planes (ld kPanel).
+// 1024 elements per block.
+struct CoefJob {
+  const float* part;      // nparts partials, part_stride elements apart
+  __nv_bfloat16* cp;      // planes (plane stride pstride)
+  long long part_stride, pstride;
+  const int* flag;
+  int rows, nparts;
+  int blk_begin;
+};
+
+__global__ void __launch_bounds__(256) pc_coef_reduce_kernel(const CoefJob* __restrict__ J, int n) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (J[mid].blk_begin <= (int)blockIdx.x) lo = mid; else hi = mid - 1;
+  }
+  const CoefJob& j = J[lo];
+  if (j.flag && *j.flag == 0) return;
+  const long long e = ((long long)(blockIdx.x - j.blk_begin) * 256 + threadIdx.x) * 4;
+  if (e >= (long long)j.rows * kPanel) return;
+  float4 v[8];
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int p0 = 0; p0 < j.nparts; p0 += 8) {
+#pragma unroll
+    for (int p = 0; p < 8; ++p)
+      if (p0 + p < j.nparts) v[p] = *reinterpret_cast<const float4*>(j.part + (long long)(p0 + p) * j.part_stride + e);
+#pragma unroll
+    for (int p = 0; p < 8; ++p)
+      if (p0 + p < j.nparts) {
+        acc.x += v[p].x;
+        acc.y += v[p].y;
+        acc.z += v[p].z;
+        acc.w += v[p].w;
+      }
+  }
+  store_split3x4(acc, j.cp, e, j.pstride);
+}
+
+// Squared column norms of a k x k matrix (ld k): partial sums over 256-row blocks,
+// then their totals in row-block order (deterministic).
+struct ColsqJob {
+  const float* src;
+  float* part;       // rblocks x k
+  float* out;        // k
+  const int* flag;
+  int k, rblocks, cblocks;
+  int blk_begin;     // partial pass: rblocks * cblocks blocks of this job
+  int fin_begin;     // final pass: cblocks blocks of this job
+};
+
+template <bool FINAL>
+__device__ __forceinline__ int find_colsq(const ColsqJob* J, int n, int blk) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((FINAL ? J[mid].fin_begin : J[mid].blk_begin) <= blk) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(256) pc_colsq_partial_kernel(const ColsqJob* __restrict__ J, int n) {
+  const ColsqJob& j = J[find_colsq<false>(J, n, blockIdx.x)];
+  if (j.flag && *j.flag == 0) return;
+  const int local = blockIdx.x - j.blk_begin;
+  const int rb = local / j.cblocks, c = (local % j.cblocks) * 256 + threadIdx.x;
+  if (c >= j.k) return;
+  const int r0 = rb * 256, r1 = min(j.k, r0 + 256);
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+  int r = r0;
+  for (; r + 3 < r1; r += 4) {
+    const float a = j.src[(long long)r * j.k + c], b = j.src[(long long)(r + 1) * j.k + c];
+    const float e = j.src[(long long)(r + 2) * j.k + c], f = j.src[(long long)(r + 3) * j.k + c];
+    s0 += a * a;
+    s1 += b * b;
+    s2 += e * e;
+    s3 += f * f;
+  }
+  for (; r < r1; ++r) {
+    const float a = j.src[(long long)r * j.k + c];
+    s0 += a * a;
+  }
+  j.part[(long long)rb * j.k + c] = (s0 + s1) + (s2 + s3);
+}
+
+__global__ void __launch_bounds__(256) pc_colsq_final_kernel(const ColsqJob* __restrict__ J, int n) {
+  const ColsqJob& j = J[find_colsq<true>(J, n, blockIdx.x)];
+  if (j.flag && *j.flag == 0) return;
+  const int c = (blockIdx.x - j.fin_begin) * 256 + threadIdx.x;
+  if (c >= j.k) return;
+  float s = 0.f;
+  for (int rb = 0; rb < j.rblocks; ++rb) s += j.part[(long long)rb * j.k + c];
+  j.out[c] = s;
 }
 
 // ------------------------------------------------------------------ FOAM pieces

@@ -29,7 +29,9 @@ using namespace mao;
 
 namespace {
 
-constexpr size_t kGroupBudget = (size_t)24 << 30;  // scratch bytes per group of matrices
+constexpr size_t kGroupBudget = (size_t)48 << 30;  // scratch bytes per group of matrices
+constexpr int kCoefSplitMinK = 4096;  // factors at least this large may split their projection products over K
+constexpr int kMaxCoefParts = 8;
 
 mao_status check_refresh(const mao_refresh& r) {
   if (r.kind < MAO_REFRESH_EVERY_K || r.kind > MAO_REFRESH_NEVER) return MAO_ERR_INVALID_ARG;
@@ -94,7 +96,9 @@ inline size_t planes_bytes(int rows, int cols) { return 3 * 2 * (size_t)rows * l
 struct SideBuf {
   size_t Fp, Qp, P, Ps, Psp;
   size_t W, Wp, Cp;  // panel buffer (k x kPanel, fp32 and planes) and the coefficients
-  size_t part, rinv, keys, perm, flag, rho, bad, again;
+  size_t Cpart;      // K-slice partials of the coefficients (large factors only)
+  size_t cpart, pnorm2, reorth;  // column norms of the gathered P (partials, totals); reorthogonalise flag
+  size_t part, gs, rinv, keys, perm, flag, rho, bad, again;
   size_t Tp, D;  // adaptive check
 };
 
@@ -116,7 +120,9 @@ void side_layout(int k, bool check, Carver& cv, SideBuf& s, size_t flag_block) {
   s.W = cv.take(4 * (size_t)k * kPanel);
   s.Wp = cv.take(planes_bytes(k, kPanel));
   s.Cp = cv.take(planes_bytes(k, kPanel));
+  s.Cpart = k >= kCoefSplitMinK ? cv.take(4 * (size_t)kMaxCoefParts * k * kPanel) : 0;
   s.part = cv.take(4 * (size_t)parts * kPanelSq);
+  s.gs = cv.take(8 * (size_t)kGsDoubles);
   s.rinv = cv.take(2 * 3 * (size_t)kPanelSq);
   s.keys = cv.take(8 * (size_t)k);
   s.perm = cv.take(4 * (size_t)k);
@@ -124,6 +130,9 @@ void side_layout(int k, bool check, Carver& cv, SideBuf& s, size_t flag_block) {
   s.rho = s.flag + 16;
   s.bad = s.flag + 32;
   s.again = s.flag + 48;
+  s.reorth = s.flag + 56;
+  s.cpart = cv.take(4 * (size_t)((k + 255) / 256) * k);
+  s.pnorm2 = cv.take(4 * (size_t)k);
   if (check) {
     s.Tp = cv.take(planes_bytes(k, k));
     s.D = cv.take(4 * kk);
@@ -155,11 +164,13 @@ void plan_group_scratch(const Ctx& X, GroupPlan& G, size_t base) {
   const bool check = X.mode == 2;
   G.flags_bytes = (size_t)64 * 2 * (G.g1 - G.g0);
   G.flags = cv.take(G.flags_bytes);
+  bool g_one = true;  // every gradient of the group bf16: G is read directly (SOAP needs no plane copy)
+  for (int i = G.g0; i < G.g1; ++i) g_one = g_one && X.mats[i].g_bf16;
   for (int i = G.g0; i < G.g1; ++i) {
     const PcMat& a = X.mats[i];
     MatBuf& b = G.mb[i - G.g0];
     const size_t mn = (size_t)a.m * a.n;
-    b.Gp = cv.take(planes_bytes(a.m, a.n));
+    b.Gp = (X.foam || !g_one) ? cv.take(planes_bytes(a.m, a.n)) : 0;
     b.Mp = cv.take(planes_bytes(a.m, a.n));
     if (!X.foam) {
       b.T1G = cv.take(planes_bytes(a.m, a.n));
@@ -214,7 +225,8 @@ void make_groups(const Ctx& X, std::vector<GroupPlan>& groups) {
 // Records every launch of one group into `ops`, with all device data staged in
 // the arena; in sizing mode (ws == nullptr) only the sizes matter.
 struct Op {
-  enum Kind { GEMM, EW, SPLIT, ADAM, KEYS, ARGSORT, GATHER, VPERM, CHOL, RC, TAU, FOAMN, CHECK } kind;
+  enum Kind { GEMM, EW, SPLIT, ADAM, KEYS, ARGSORT, GATHER, COLSQ, COLSQFIN, VPERM, REDUCE, CHOL, COEFRED, RC, TAU,
+              FOAMN, CHECK } kind;
   size_t jobs = 0;
   int njobs = 0;
   int blocks = 0;
@@ -407,6 +419,33 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
     }
     B.ops.back().blocks = blk;
   }
+  // squared column norms of the gathered P (the reorthogonalisation criterion)
+  {
+    size_t off;
+    ColsqJob* J = B.new_jobs<ColsqJob>(Op::COLSQ, nu, off);
+    int blk = 0, fin = 0;
+    for (int i = 0; i < nu; ++i) {
+      const int k = kof(i);
+      ColsqJob& j = J[i];
+      j.src = B.wp<float>(side(i).Ps);
+      j.part = B.wp<float>(side(i).cpart);
+      j.out = B.wp<float>(side(i).pnorm2);
+      j.flag = flagp(i);
+      j.k = k;
+      j.rblocks = (k + 255) / 256;
+      j.cblocks = (k + 255) / 256;
+      j.blk_begin = blk;
+      blk += j.rblocks * j.cblocks;
+      j.fin_begin = fin;
+      fin += j.cblocks;
+    }
+    B.ops.back().blocks = blk;
+    Op o = B.ops.back();
+    o.kind = Op::COLSQFIN;
+    o.blocks = fin;
+    B.ops.push_back(o);
+    B.gemm_of_op.push_back(-1);
+  }
   // QR by panels of kPanel columns: block Gram-Schmidt with two projection passes,
   // Cholesky-QR inside each panel (twice after the first pass, once after the second)
   int maxk = 0;
@@ -459,12 +498,13 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
                             nullptr, kPanel, nullptr, 0, 1.f, 0.f, gate(i), s0));
       }
       size_t off;
-      PanelJob* J = B.new_jobs<PanelJob>(Op::CHOL, (int)act.size(), off);
+      PanelJob* J = B.new_jobs<PanelJob>(Op::REDUCE, (int)act.size(), off);
       for (size_t a = 0; a < act.size(); ++a) {
         const int i = act[a];
         const int k = kof(i);
         PanelJob& j = J[a];
         j.part = B.wp<float>(side(i).part);
+        j.gs = B.wp<double>(side(i).gs);
         j.rinv = B.wp<__nv_bfloat16>(side(i).rinv);
         j.bad = B.wp<int>(side(i).bad);
         j.again = B.wp<int>(side(i).again);
@@ -472,8 +512,17 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
         j.w = wdt(i);
         j.nparts = (k + gram_slice(k, nact) - 1) / gram_slice(k, nact);
         j.first = pass == 0 ? 1 : 0;
+        if (pass == 0 && c0 > 0) {
+          j.pnorm2 = B.wp<float>(side(i).pnorm2) + c0;
+          j.reorth = B.wp<int>(side(i).reorth);
+        }
       }
-      B.ops.back().blocks = (int)act.size();
+      B.ops.back().blocks = (int)act.size() * kRedBlocks;
+      Op ch = B.ops.back();  // the factorisation reuses the job array
+      ch.kind = Op::CHOL;
+      ch.blocks = (int)act.size();
+      B.ops.push_back(ch);
+      B.gemm_of_op.push_back(-1);
       TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_QR);
       for (int i : act) {
         const int k = kof(i), w = wdt(i);
@@ -488,14 +537,52 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
       return MAO_OK;
     };
     // remove the finished columns: C = Q[:, :c0]^T Y ; W = Y - Q[:, :c0] C (fp32 and planes)
+    // When the coefficient product has too few tiles to fill the GPU, the large
+    // factors split it over K into fp32 partials, summed (in slice order) into C's planes.
     auto project = [&](int from) -> mao_status {
+      // the second projection runs only where the first one cancelled (flag set on the device)
+      auto pflag = [&](int u) -> const int* { return from == WA ? B.wp<int>(side(u).reorth) : flagp(u); };
+      int tiles = 0;
+      for (int i : act) tiles += (c0 + 127) / 128;
+      const int want = std::min(kMaxCoefParts, std::max(1, (2 * 148 + tiles - 1) / std::max(tiles, 1)));
       TableLaunch& gc = B.new_gemm(1, 1, MAO_K_PC_QR);
+      std::vector<CoefJob> red;
+      int rblk = 0;
       for (int i : act) {
         const int k = kof(i), w = wdt(i);
         Split3 C = B.planes(side(i).Cp, k, kPanel);
         C.cols = w;
-        MAO_TRY(table_add(gc, B.maps, B.planes(side(i).Qp, k, k), pv(i, from), c0, w, k, 0, 0, nullptr, &C,
-                          kPanel, nullptr, 0, 1.f, 0.f, flagp(i)));
+        const int S = k >= kCoefSplitMinK ? want : 1;
+        if (S == 1) {
+          MAO_TRY(table_add(gc, B.maps, B.planes(side(i).Qp, k, k), pv(i, from), c0, w, k, 0, 0, nullptr, &C,
+                            kPanel, nullptr, 0, 1.f, 0.f, pflag(i)));
+          continue;
+        }
+        const int sl = round_up_int((k + S - 1) / S, 64);
+        float* part = B.wp<float>(side(i).Cpart);
+        const long long pst = (long long)k * kPanel;
+        int p = 0;
+        for (int s0 = 0; s0 < k; s0 += sl, ++p)
+          MAO_TRY(table_add(gc, B.maps, B.planes(side(i).Qp, k, k), pv(i, from), c0, w, std::min(sl, k - s0), 0, 0,
+                            part + p * pst, nullptr, kPanel, nullptr, 0, 1.f, 0.f, pflag(i), s0));
+        CoefJob cj;
+        std::memset(&cj, 0, sizeof(cj));
+        cj.part = part;
+        cj.cp = B.wp<__nv_bfloat16>(side(i).Cp);
+        cj.part_stride = pst;
+        cj.pstride = B.pstride(k, kPanel);
+        cj.flag = pflag(i);
+        cj.rows = c0;
+        cj.nparts = p;
+        cj.blk_begin = rblk;
+        rblk += (c0 * kPanel + 1023) / 1024;
+        red.push_back(cj);
+      }
+      if (!red.empty()) {
+        size_t off;
+        CoefJob* J = B.new_jobs<CoefJob>(Op::COEFRED, (int)red.size(), off);
+        for (size_t a = 0; a < red.size(); ++a) J[a] = red[a];
+        B.ops.back().blocks = rblk;
       }
       TableLaunch& gw = B.new_gemm(0, 1, MAO_K_PC_QR);
       for (int i : act) {
@@ -508,7 +595,7 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
         const float* aux = fp(i, from, &lda);
         float* W = fp(i, WA, &ldw);
         MAO_TRY(table_add(gw, B.maps, B.planes(side(i).Qp, k, k), C, k, w, c0, 0, 0, W, &Wp, ldw, aux, lda, -1.f,
-                          1.f, flagp(i)));
+                          1.f, pflag(i)));
       }
       return MAO_OK;
     };
@@ -945,6 +1032,26 @@ mao_status run_ops(const Ctx& X, uint8_t* arena_dev, const BuiltGroup& bg, DevSt
       case Op::VPERM: {
         LaunchScope ls(s, MAO_K_PC_SORT, 0.0, 0.0);
         soap_vperm_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<VPermJob>(op.jobs), n);
+        break;
+      }
+      case Op::REDUCE: {
+        LaunchScope ls(s, MAO_K_PC_PANEL, 0.0, 0.0);
+        qr_gram_reduce_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<PanelJob>(op.jobs));
+        break;
+      }
+      case Op::COEFRED: {
+        LaunchScope ls(s, MAO_K_PC_QR, 0.0, 0.0);
+        pc_coef_reduce_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<CoefJob>(op.jobs), n);
+        break;
+      }
+      case Op::COLSQ: {
+        LaunchScope ls(s, MAO_K_PC_SORT, 0.0, 0.0);
+        pc_colsq_partial_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<ColsqJob>(op.jobs), n);
+        break;
+      }
+      case Op::COLSQFIN: {
+        LaunchScope ls(s, MAO_K_PC_SORT, 0.0, 0.0);
+        pc_colsq_final_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<ColsqJob>(op.jobs), n);
         break;
       }
       case Op::CHOL: {
