@@ -242,6 +242,20 @@ mao_status table_add(TableLaunch& L, MapSet& maps, const Split3& A, const Split3
   return MAO_OK;
 }
 
+mao_status table_set_alt(TableLaunch& L, const int* sel, float* out2, const Split3* out2p, int ld_out2) {
+  if (L.probs.empty() || sel == nullptr) return MAO_ERR_INVALID_ARG;
+  GemmProblem& P = L.probs.back();
+  P.sel = sel;
+  P.out2 = out2;
+  P.ld_out2 = ld_out2;
+  if (out2p) {
+    if (out2p->ld & 7) return MAO_ERR_SHAPE;
+    for (int q = 0; q < 3; ++q) P.out2_p[q] = const_cast<__nv_bfloat16*>(out2p->p[q]);
+    P.ld_out2p = out2p->ld;
+  }
+  return MAO_OK;
+}
+
 StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off) {
   StagedLaunch S;
   S.nprob = (int)L.probs.size();
@@ -264,7 +278,9 @@ StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off) {
     }
     P.tile_begin = t;
     t += ((P.M + 127) / 128) * P.tiles_n;
-    S.flops += 2.0 * P.M * (double)P.N * P.K;
+    // work recorded for the profiler: only problems that always run (a problem gated
+    // by a device flag may be skipped, so it counts nothing: a lower bound)
+    if (P.flag == nullptr) S.flops += 2.0 * P.M * (double)P.N * P.K;
     hp[i] = P;
   }
   S.total_tiles = t;

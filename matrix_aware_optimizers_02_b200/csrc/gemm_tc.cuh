@@ -101,6 +101,12 @@ struct GemmProblem {
   int ld_out, ld_aux, ld_outp;
   int tiles_n, tile_begin;
   float alpha, beta;
+  // Alternate destination chosen on the device: when sel != nullptr and *sel == 0
+  // the result goes to out2 / out2_p (leading dimensions ld_out2 / ld_out2p) instead.
+  const int* sel;
+  float* out2;
+  __nv_bfloat16* out2_p[3];
+  int ld_out2, ld_out2p;
 };
 
 struct GemmTableParams {
@@ -366,9 +372,12 @@ struct TableSource {
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] *= P.alpha;
     }
-    const long long off = (long long)row * P.ld_out + col0;
-    if (P.out != nullptr) {
-      float* o = P.out + off;
+    const bool alt = (P.sel != nullptr) && (*P.sel == 0);
+    float* const out = alt ? P.out2 : P.out;
+    const int ld_out = alt ? P.ld_out2 : P.ld_out;
+    const long long off = (long long)row * ld_out + col0;
+    if (out != nullptr) {
+      float* o = out + off;
       if (full) {
 #pragma unroll
         for (int j = 0; j < 32; j += 4)
@@ -377,8 +386,9 @@ struct TableSource {
         for (int j = 0; j < 32 && col0 + j < P.N; ++j) o[j] = v[j];
       }
     }
-    if (P.out_p[0] != nullptr) {
-      const long long offp = (long long)row * P.ld_outp + col0;
+    __nv_bfloat16* const* out_p = alt ? P.out2_p : P.out_p;
+    if (out_p[0] != nullptr) {
+      const long long offp = (long long)row * (alt ? P.ld_out2p : P.ld_outp) + col0;
       float r[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) r[j] = v[j];
@@ -390,7 +400,7 @@ struct TableSource {
           pq[j] = __bfloat162float(__float2bfloat16_rn(r[j]));
           r[j] -= pq[j];
         }
-        __nv_bfloat16* o = P.out_p[q] + offp;
+        __nv_bfloat16* o = out_p[q] + offp;
         if (full) {
           store_bf16x32(o, pq);
         } else {

@@ -201,6 +201,10 @@ mao_status table_add(TableLaunch& L, MapSet& maps, const Split3& A, const Split3
                      int m_off, int n_off, float* out, const Split3* outp, int ld_out, const float* aux,
                      int ld_aux, float alpha, float beta, const int* flag, int k_off = 0);
 
+// Give the last problem added to L an alternate destination, used when *sel == 0
+// on the device (sel is read by every tile's epilogue).
+mao_status table_set_alt(TableLaunch& L, const int* sel, float* out2, const Split3* out2p, int ld_out2);
+
 // Stage a launch's problem table into the arena (maps live at maps_off) and launch it.
 struct StagedLaunch {
   size_t probs_off = 0;

@@ -153,35 +153,56 @@ struct SortJob {
   int* perm_out;      // caller's copy, or nullptr
   const int* flag;
   int k;
-  int col_blk_begin;  // blocks of 256 columns (keys) / 256 ranks (argsort)
+  int col_blk_begin;  // blocks of 256 ranks (argsort, identity keys)
+  int key_blk_begin;  // blocks of 32 columns (keys)
 };
 
+template <bool KEYS>
 __device__ __forceinline__ int find_sort(const SortJob* J, int n, int blk) {
   int lo = 0, hi = n - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (J[mid].col_blk_begin <= blk) lo = mid; else hi = mid - 1;
+    if ((KEYS ? J[mid].key_blk_begin : J[mid].col_blk_begin) <= blk) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
 
+// key_i = sum_r Q[r][i] P[r][i] in fp64: one block per 32 columns, warp w sums the
+// rows w, w + 8, ... (each warp reads 128 contiguous bytes per row of Q and P), then
+// the eight warp sums are added in warp order.
 __global__ void __launch_bounds__(256) pc_keys_kernel(const SortJob* __restrict__ J, int n) {
-  const SortJob& j = J[find_sort(J, n, blockIdx.x)];
+  __shared__ double part[8][32];
+  const SortJob& j = J[find_sort<true>(J, n, blockIdx.x)];
   if (j.flag && *j.flag == 0) return;
-  const int i = (blockIdx.x - j.col_blk_begin) * 256 + threadIdx.x;
-  if (i >= j.k) return;
-  double s = 0.0;
-  for (int r = 0; r < j.k; ++r) s += (double)j.Q[(long long)r * j.k + i] * (double)j.P[(long long)r * j.k + i];
-  if (!(s == s)) s = -INFINITY;  // a NaN key sorts last, so the permutation stays a bijection
-  j.key[i] = s;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int i = (blockIdx.x - j.key_blk_begin) * 32 + lane;
+  double s0 = 0.0, s1 = 0.0;
+  if (i < j.k) {
+    int r = warp;
+    for (; r + 8 < j.k; r += 16) {
+      s0 += (double)j.Q[(long long)r * j.k + i] * (double)j.P[(long long)r * j.k + i];
+      s1 += (double)j.Q[(long long)(r + 8) * j.k + i] * (double)j.P[(long long)(r + 8) * j.k + i];
+    }
+    if (r < j.k) s0 += (double)j.Q[(long long)r * j.k + i] * (double)j.P[(long long)r * j.k + i];
+  }
+  part[warp][lane] = s0 + s1;
+  __syncthreads();
+  if (warp == 0 && i < j.k) {
+    double s = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += part[w][lane];
+    if (!(s == s)) s = -INFINITY;  // a NaN key sorts last, so the permutation stays a bijection
+    j.key[i] = s;
+  }
 }
 
-// Sorting disabled: strictly decreasing keys, so the argsort yields the identity.
+// Sorting disabled: strictly decreasing keys, so the argsort yields the identity
+// (same block mapping as the key kernel: 32 columns per block).
 __global__ void __launch_bounds__(256) pc_identity_keys_kernel(const SortJob* __restrict__ J, int n) {
-  const SortJob& j = J[find_sort(J, n, blockIdx.x)];
+  const SortJob& j = J[find_sort<true>(J, n, blockIdx.x)];
   if (j.flag && *j.flag == 0) return;
-  const int i = (blockIdx.x - j.col_blk_begin) * 256 + threadIdx.x;
-  if (i < j.k) j.key[i] = -(double)i;
+  const int i = (blockIdx.x - j.key_blk_begin) * 32 + threadIdx.x;
+  if (threadIdx.x < 32 && i < j.k) j.key[i] = -(double)i;
 }
 
 // Stable descending argsort by rank counting: rank_i = #{key_j > key_i} + #{j < i: key_j == key_i};
@@ -189,7 +210,7 @@ __global__ void __launch_bounds__(256) pc_identity_keys_kernel(const SortJob* __
 // A refresh that does not run (flag 0) reports the identity permutation.
 __global__ void __launch_bounds__(256) pc_argsort_kernel(const SortJob* __restrict__ J, int n) {
   __shared__ double sk[2048];
-  const SortJob& j = J[find_sort(J, n, blockIdx.x)];
+  const SortJob& j = J[find_sort<false>(J, n, blockIdx.x)];
   const int i = (blockIdx.x - j.col_blk_begin) * 256 + threadIdx.x;
   if (j.flag && *j.flag == 0) {
     if (j.perm_out && i < j.k) j.perm_out[i] = i;
@@ -307,8 +328,9 @@ constexpr int kRedRows = 8;                               // Gram rows per reduc
 constexpr int kRedBlocks = kPanel / kRedRows;
 constexpr int kGsDoubles = kPackedUpper + kPanel + kRedBlocks;  // Gs | D^-1/2 | ||E||^2 partials
 constexpr int kCholSmem = (kPackedUpper + (kPanel - 32) * 32 + 2 * kPanel) * 8;
-constexpr double kCholShift = 1e-6;       // relative to the unit diagonal of Gs
-constexpr double kCholShiftRetry = 1e-4;  // after a non-positive pivot
+constexpr double kCholShift = 1e-4;  // relative to the unit diagonal of Gs, after a non-positive pivot
+constexpr double kAgainMeanInv = 16.0;  // mean of 1/eig(Gs) (= ||Rs^-1||_F^2 / w) above which a first
+                                        // pass is followed by a second one
 constexpr double kFastTol = 1e-4;
 
 struct PanelJob {
@@ -320,6 +342,8 @@ struct PanelJob {
   const float* pnorm2;   // first pass after a projection: squared norms of the panel's columns
                          // before the projection (else nullptr)
   int* reorth;           // ... and the flag set to 1 when a second projection is needed, else 0
+  int* fin;              // first pass: set to 1 when the panel needs a final Cholesky-QR pass
+                         // (a second pass or a second projection ran), else 0
   const int* flag;
   int w, nparts;
   int first;
@@ -422,11 +446,15 @@ __global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restr
 #pragma unroll
   for (int i = 0; i < kRedBlocks; ++i) tot += j.gs[kPackedUpper + kPanel + i];
   if (tot <= kFastTol * kFastTol) {  // the first-order inverse is already in place
-    if (j.first && tid == 0) *j.again = 0;
+    if (j.first && tid == 0) {
+      *j.again = 0;
+      *j.fin = j.reorth ? *j.reorth : 0;
+    }
     return;
   }
   if (tid < kPanel) ds[tid] = j.gs[kPackedUpper + tid];
 
+  int shifted = 0;
   for (int attempt = 0; attempt < 2; ++attempt) {
     {
       const double2* src = reinterpret_cast<const double2*>(j.gs);
@@ -435,8 +463,7 @@ __global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restr
     }
     if (tid == 0) nbad_sh = 0;
     __syncthreads();
-    const double shift = attempt ? kCholShiftRetry : (j.first ? kCholShift : 0.0);
-    if (tid < wp && shift > 0.0) A[pk(tid, tid)] += shift;
+    if (attempt && tid < wp) A[pk(tid, tid)] += kCholShift;
     __syncthreads();
   // ---- blocked Cholesky, upper: Gs = Rs^T Rs
   for (int bk = 0; bk < nb; ++bk) {
@@ -507,13 +534,11 @@ __global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restr
     __syncthreads();
   }
     __syncthreads();
-    if (nbad_sh == 0 || attempt == 1) break;  // retry once with the larger shift
+    shifted = attempt;
+    if (nbad_sh == 0 || attempt == 1) break;  // retry once, shifted
     __syncthreads();
   }
-  if (tid == 0) {
-    if (nbad_sh) atomicAdd(j.bad, 1);
-    if (j.first) *j.again = 1;
-  }
+  if (tid == 0 && nbad_sh) atomicAdd(j.bad, 1);
 
   // ---- inverse in place.  Diagonal blocks first, one warp each: column c = lane of
   // Rs_bb^{-1}, from the last row up, written over Rs_bb as it goes (row k of the
@@ -562,10 +587,31 @@ __global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restr
     __syncthreads();
   }
   // R^{-1} = D^-1/2 Rs^{-1}: three bf16 planes over the full kPanel x kPanel square
+  double x2 = 0.0;
   for (int t = tid; t < kPanelSq; t += 256) {
     const int r = t / kPanel, c = t % kPanel;
-    const float x = (r <= c && c < w) ? (float)(ds[r] * A[pk(r, c)]) : 0.0f;
+    float x = 0.0f;
+    if (r <= c && c < w) {
+      const double xs = A[pk(r, c)];
+      x2 += xs * xs;
+      x = (float)(ds[r] * xs);
+    }
     store_split3(x, j.rinv, t, kPanelSq);
+  }
+  if (j.first) {
+    // the first pass is final unless it had to be shifted or Gs is poorly conditioned
+    // (CholQR loses orthogonality in proportion to cond(Gs))
+    x2 = warp_sum_d(x2);
+    if (lane == 0) T[warp] = x2;
+    __syncthreads();
+    if (tid == 0) {
+      double tot2 = 0.0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) tot2 += T[i];
+      const int again = (shifted || tot2 > kAgainMeanInv * w) ? 1 : 0;
+      *j.again = again;
+      *j.fin = again | (j.reorth ? *j.reorth : 0);
+    }
   }
 }
 

@@ -97,7 +97,7 @@ struct SideBuf {
   size_t Fp, Qp, P, Ps, Psp;
   size_t W, Wp, Cp;  // panel buffer (k x kPanel, fp32 and planes) and the coefficients
   size_t Cpart;      // K-slice partials of the coefficients (large factors only)
-  size_t cpart, pnorm2, reorth;  // column norms of the gathered P (partials, totals); reorthogonalise flag
+  size_t cpart, pnorm2, reorth, fin;  // column norms of the gathered P (partials, totals); panel decisions
   size_t part, gs, rinv, keys, perm, flag, rho, bad, again;
   size_t Tp, D;  // adaptive check
 };
@@ -131,6 +131,7 @@ void side_layout(int k, bool check, Carver& cv, SideBuf& s, size_t flag_block) {
   s.bad = s.flag + 32;
   s.again = s.flag + 48;
   s.reorth = s.flag + 56;
+  s.fin = s.flag + 60;
   s.cpart = cv.take(4 * (size_t)((k + 255) / 256) * k);
   s.pnorm2 = cv.take(4 * (size_t)k);
   if (check) {
@@ -376,7 +377,7 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
   {
     size_t off;
     SortJob* J = B.new_jobs<SortJob>(Op::KEYS, nu, off);
-    int blk = 0;
+    int blk = 0, kblk = 0;
     for (int i = 0; i < nu; ++i) {
       const int k = kof(i);
       SortJob& j = J[i];
@@ -389,10 +390,13 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
       j.k = k;
       j.col_blk_begin = blk;
       blk += (k + 255) / 256;
+      j.key_blk_begin = kblk;
+      kblk += (k + 31) / 32;
     }
-    B.ops.back().blocks = blk;
+    B.ops.back().blocks = kblk;
     Op o = B.ops.back();  // the argsort reuses the job array
     o.kind = Op::ARGSORT;
+    o.blocks = blk;
     B.ops.push_back(o);
     B.gemm_of_op.push_back(-1);
   }
@@ -481,10 +485,14 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
       return v;
     };
     // one Cholesky-QR of every active panel: dst = src R^{-1} (dst may be src).
-    // pass 0: first pass (decides whether pass 1 runs); 1: the gated second pass;
-    // 2: an ungated pass on a nearly orthonormal panel
+    // pass 0: the first pass; it decides on the device whether the second pass
+    //         (flag again), the second projection (reorth) and the final pass (fin)
+    //         run, and writes straight into Q's columns when none does;
+    // pass 1: the second pass (gated by again); pass 2: the final pass (gated by fin)
     auto cholqr = [&](int src, int dst, int pass) -> mao_status {
-      auto gate = [&](int u) -> const int* { return pass == 1 ? B.wp<int>(side(u).again) : flagp(u); };
+      auto gate = [&](int u) -> const int* {
+        return pass == 1 ? B.wp<int>(side(u).again) : pass == 2 ? B.wp<int>(side(u).fin) : flagp(u);
+      };
       // Gram partials over K slices (fp32-faithful), one 128 x 128 tile each
       TableLaunch& gg = B.new_gemm(1, 1, MAO_K_PC_PANEL);
       const int nact = (int)act.size();
@@ -512,6 +520,7 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
         j.w = wdt(i);
         j.nparts = (k + gram_slice(k, nact) - 1) / gram_slice(k, nact);
         j.first = pass == 0 ? 1 : 0;
+        if (pass == 0) j.fin = B.wp<int>(side(i).fin);
         if (pass == 0 && c0 > 0) {
           j.pnorm2 = B.wp<float>(side(i).pnorm2) + c0;
           j.reorth = B.wp<int>(side(i).reorth);
@@ -533,6 +542,12 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
         float* out = fp(i, dst, &ld);
         MAO_TRY(table_add(g, B.maps, pv(i, src), Ri, k, w, w, 0, 0, out, &out_p, ld, nullptr, 0, 1.f, 0.f,
                           gate(i)));
+        if (pass == 0) {  // final already: Q's columns
+          const Split3 q_p = pv(i, QF);
+          int ldq = 0;
+          float* q = fp(i, QF, &ldq);
+          MAO_TRY(table_set_alt(g, B.wp<int>(side(i).fin), q, &q_p, ldq));
+        }
       }
       return MAO_OK;
     };
@@ -603,6 +618,7 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
     // rows of W, all of K in one tile).
     if (pj == 0) {
       MAO_TRY(cholqr(PS, WA, 0));
+      MAO_TRY(cholqr(WA, WA, 1));
       MAO_TRY(cholqr(WA, QF, 2));
     } else {
       MAO_TRY(project(PS));
