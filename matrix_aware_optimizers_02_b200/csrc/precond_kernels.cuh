@@ -327,7 +327,7 @@ constexpr int kMaxParts = 16;                             // K slices of a panel
 constexpr int kRedRows = 8;                               // Gram rows per reduction block
 constexpr int kRedBlocks = kPanel / kRedRows;
 constexpr int kGsDoubles = kPackedUpper + kPanel + kRedBlocks;  // Gs | D^-1/2 | ||E||^2 partials
-constexpr int kCholSmem = (kPackedUpper + (kPanel - 32) * 32 + 2 * kPanel) * 8;
+constexpr int kCholSmem = (kPanel * (kPanel + 1) + (kPanel - 32) * 32 + 2 * kPanel) * 8;
 constexpr double kCholShift = 1e-4;  // relative to the unit diagonal of Gs, after a non-positive pivot
 constexpr double kAgainMeanInv = 16.0;  // mean of 1/eig(Gs) (= ||Rs^-1||_F^2 / w) above which a first
                                         // pass is followed by a second one
@@ -428,13 +428,20 @@ __global__ void __launch_bounds__(256) qr_gram_reduce_kernel(const PanelJob* __r
   }
 }
 
+// Cholesky of Gs and the inverse of its factor, fp64 in shared memory (row-major,
+// leading dimension kLdA; only the upper triangle is meaningful).  Work is laid
+// out so that a warp's shared-memory accesses are a row segment across lanes or a
+// broadcast, and inner products keep several independent accumulators.
+constexpr int kLdA = kPanel + 1;
+
 __global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restrict__ J) {
   extern __shared__ double chol_smem[];
-  double* A = chol_smem;                 // packed upper: Gs, then Rs, then Rs^{-1}
-  double* T = A + kPackedUpper;          // [kPanel - 32][32] block-column workspace of the inverse
-  double* ds = T + (kPanel - 32) * 32;   // D^-1/2
-  double* rdi = ds + kPanel;             // 1 / Rs[k][k]
+  double* A = chol_smem;                  // [kPanel][kLdA]: Gs, then Rs, then Rs^{-1}
+  double* T = A + kPanel * kLdA;          // [kPanel - 32][32] block-column workspace of the inverse
+  double* ds = T + (kPanel - 32) * 32;    // D^-1/2
+  double* rdi = ds + kPanel;              // 1 / Rs[k][k]
   __shared__ int nbad_sh;
+  __shared__ double red_sh[8];
   const PanelJob& j = J[blockIdx.x];
   if (j.flag && *j.flag == 0) return;
   const int w = j.w;
@@ -456,83 +463,98 @@ __global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restr
 
   int shifted = 0;
   for (int attempt = 0; attempt < 2; ++attempt) {
-    {
-      const double2* src = reinterpret_cast<const double2*>(j.gs);
-      double2* dst = reinterpret_cast<double2*>(A);
-      for (int q = tid; q < kPackedUpper / 2; q += 256) dst[q] = src[q];
+    // unpack the upper triangle, row r by warp r % 8
+    for (int r = warp; r < wp; r += 8) {
+      const double* src = j.gs + pk(r, r) - r;  // so that src[c] = Gs[r][c] for c >= r
+      for (int c = r + lane; c < wp; c += 32) A[r * kLdA + c] = src[c];
     }
     if (tid == 0) nbad_sh = 0;
     __syncthreads();
-    if (attempt && tid < wp) A[pk(tid, tid)] += kCholShift;
+    if (attempt && tid < wp) A[tid * kLdA + tid] += kCholShift;
     __syncthreads();
-  // ---- blocked Cholesky, upper: Gs = Rs^T Rs
-  for (int bk = 0; bk < nb; ++bk) {
-    const int o = bk * 32;
-    if (warp == 0) {
-      // lane c holds column o + c of the diagonal block (rows <= c)
-      double v[32];
-      int nbad = 0;
+    // ---- blocked Cholesky, upper: Gs = Rs^T Rs
+    for (int bk = 0; bk < nb; ++bk) {
+      const int o = bk * 32;
+      if (warp == 0) {
+        // lane c holds column o + c of the diagonal block (rows <= c)
+        double v[32];
+        int nbad = 0;
 #pragma unroll
-      for (int r = 0; r < 32; ++r) v[r] = (r <= lane) ? A[pk(o + r, o + lane)] : 0.0;
+        for (int r = 0; r < 32; ++r) v[r] = (r <= lane) ? A[(o + r) * kLdA + o + lane] : 0.0;
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        double d = __shfl_sync(FULL, v[k], k);
-        nbad += (d > 0.0) ? 0 : 1;
-        d = (d > 0.0) ? d : 1e-300;
-        const double ri = rsqrt(d);  // 1 / Rs[k][k]
-        const double rk = (lane == k) ? d * ri : (lane > k ? v[k] * ri : 0.0);  // Rs[k][c]
-        if (lane == k) rdi[o + k] = ri;
-        v[k] = rk;
+        for (int k = 0; k < 32; ++k) {
+          double d = __shfl_sync(FULL, v[k], k);
+          nbad += (d > 0.0) ? 0 : 1;
+          d = (d > 0.0) ? d : 1e-300;
+          const double ri = rsqrt(d);  // 1 / Rs[k][k]
+          const double rk = (lane == k) ? d * ri : (lane > k ? v[k] * ri : 0.0);  // Rs[k][c]
+          if (lane == k) rdi[o + k] = ri;
+          v[k] = rk;
 #pragma unroll
-        for (int i = 1; i < 32; ++i) {
-          if (i > k) {  // constant trip count keeps v[] in registers
-            const double rki = __shfl_sync(FULL, rk, i);
-            if (i <= lane) v[i] -= rki * rk;
+          for (int i = 1; i < 32; ++i) {
+            if (i > k) {  // constant trip count keeps v[] in registers
+              const double rki = __shfl_sync(FULL, rk, i);
+              if (i <= lane) v[i] -= rki * rk;
+            }
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < 32; ++r)
+          if (r <= lane) A[(o + r) * kLdA + o + lane] = v[r];
+        if (lane == 0 && nbad) nbad_sh += nbad;
+      }
+      __syncthreads();
+      const int nt = wp - o - 32;  // trailing columns
+      if (nt == 0) break;
+      // block row: Rs_bc = Rs_bb^{-T} G_bc, one column per thread (right-looking in registers)
+      if (tid < nt) {
+        const int c = o + 32 + tid;
+        double x[32];
+#pragma unroll
+        for (int r = 0; r < 32; ++r) x[r] = A[(o + r) * kLdA + c];
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+          x[r] *= rdi[o + r];
+          const double* rrow = A + (o + r) * kLdA + o;
+#pragma unroll
+          for (int i = r + 1; i < 32; ++i) x[i] -= rrow[i] * x[r];
+        }
+#pragma unroll
+        for (int r = 0; r < 32; ++r) A[(o + r) * kLdA + c] = x[r];
+      }
+      __syncthreads();
+      // trailing update G_cd -= sum_i Rs[o+i][c] Rs[o+i][d] over the whole trailing
+      // square (the lower half is never read): a warp owns two rows c, lanes own
+      // columns d, d + 32, d + 64
+      {
+        const int t0 = o + 32;
+        for (int cp = warp * 2; cp < nt; cp += 16) {
+          const int c0 = t0 + cp, c1 = c0 + 1;
+          double acc[2][3] = {};
+#pragma unroll 4
+          for (int i = 0; i < 32; ++i) {
+            const double* row = A + (o + i) * kLdA;
+            const double a0 = row[c0], a1 = row[c1];
+#pragma unroll
+            for (int q = 0; q < 3; ++q) {
+              const int d = t0 + lane + 32 * q;
+              const double b = (d < wp) ? row[d] : 0.0;
+              acc[0][q] = fma(a0, b, acc[0][q]);
+              acc[1][q] = fma(a1, b, acc[1][q]);
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < 3; ++q) {
+            const int d = t0 + lane + 32 * q;
+            if (d < wp) {
+              A[c0 * kLdA + d] -= acc[0][q];
+              A[c1 * kLdA + d] -= acc[1][q];
+            }
           }
         }
       }
-#pragma unroll
-      for (int r = 0; r < 32; ++r)
-        if (r <= lane) A[pk(o + r, o + lane)] = v[r];
-      if (lane == 0 && nbad) nbad_sh += nbad;
+      __syncthreads();
     }
-    __syncthreads();
-    const int nt = wp - o - 32;  // trailing columns
-    if (nt == 0) break;
-    // block row: Rs_bc = Rs_bb^{-T} G_bc, one column per thread (right-looking in registers)
-    if (tid < nt) {
-      const int c = o + 32 + tid;
-      double x[32];
-#pragma unroll
-      for (int r = 0; r < 32; ++r) x[r] = A[pk(o + r, c)];
-#pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        x[r] *= rdi[o + r];
-        const int base = pk(o + r, o);
-#pragma unroll
-        for (int i = r + 1; i < 32; ++i) x[i] -= A[base + i] * x[r];
-      }
-#pragma unroll
-      for (int r = 0; r < 32; ++r) A[pk(o + r, c)] = x[r];
-    }
-    __syncthreads();
-    // trailing update of the upper triangle: G_cd -= Rs_bc^T Rs_bd, c <= d
-    for (int t = tid; t < nt * nt; t += 256) {
-      const int c = o + 32 + t / nt, d = o + 32 + t % nt;
-      if (d < c) continue;
-      double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-#pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        const int r0 = pk(o + i, 0), r1 = pk(o + i + 1, 0), r2 = pk(o + i + 2, 0), r3 = pk(o + i + 3, 0);
-        s0 += A[r0 + c] * A[r0 + d];
-        s1 += A[r1 + c] * A[r1 + d];
-        s2 += A[r2 + c] * A[r2 + d];
-        s3 += A[r3 + c] * A[r3 + d];
-      }
-      A[pk(c, d)] -= (s0 + s1) + (s2 + s3);
-    }
-    __syncthreads();
-  }
     __syncthreads();
     shifted = attempt;
     if (nbad_sh == 0 || attempt == 1) break;  // retry once, shifted
@@ -554,60 +576,69 @@ __global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restr
       const double xk = (k == lane) ? ri : (k < lane ? -acc[k] * ri : 0.0);
 #pragma unroll
       for (int i = 0; i < 31; ++i)
-        if (i < k) acc[i] += A[pk(o + i, o + k)] * xk;
+        if (i < k) acc[i] += A[(o + i) * kLdA + o + k] * xk;
       __syncwarp();
-      if (k <= lane) A[pk(o + k, o + lane)] = xk;
+      if (k <= lane) A[(o + k) * kLdA + o + lane] = xk;
       __syncwarp();
     }
   }
   __syncthreads();
-  // off-diagonal blocks by block columns: X_ij = -(sum_{k=i..j-1} X_ik Rs_kj) X_jj, i < j
+  // off-diagonal blocks by block columns: X_ij = -(sum_{k=i..j-1} X_ik Rs_kj) X_jj, i < j.
+  // A warp owns four rows r of T, lanes the 32 columns.
   for (int bj = 1; bj < nb; ++bj) {
     const int oj = bj * 32;
-    // T[r][c] = sum_{k = r .. oj-1} X[r][k] Rs[k][oj + c]
-    for (int t = tid; t < oj * 32; t += 256) {
-      const int r = t >> 5, c = t & 31;
-      double s0 = 0.0, s1 = 0.0;
-      int k = r;
-      const int rb = pk(r, 0);
-      for (; k + 1 < oj; k += 2) {
-        s0 += A[rb + k] * A[pk(k, oj + c)];
-        s1 += A[rb + k + 1] * A[pk(k + 1, oj + c)];
+    for (int r0 = warp * 4; r0 < oj; r0 += 32) {
+      double acc[4] = {0.0, 0.0, 0.0, 0.0};
+      for (int k = r0; k < oj; ++k) {
+        const double rkc = A[k * kLdA + oj + lane];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (r0 + q <= k) acc[q] = fma(A[(r0 + q) * kLdA + k], rkc, acc[q]);
       }
-      if (k < oj) s0 += A[rb + k] * A[pk(k, oj + c)];
-      T[r * 32 + c] = s0 + s1;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) T[(r0 + q) * 32 + lane] = acc[q];
     }
     __syncthreads();
-    for (int t = tid; t < oj * 32; t += 256) {
-      const int r = t >> 5, c = t & 31;
-      double s = 0.0;
-      for (int m = 0; m <= c; ++m) s += T[r * 32 + m] * A[pk(oj + m, oj + c)];
-      A[pk(r, oj + c)] = -s;
+    for (int r0 = warp * 4; r0 < oj; r0 += 32) {
+      double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 8
+      for (int m = 0; m < 32; ++m) {
+        const double xm = (m <= lane) ? A[(oj + m) * kLdA + oj + lane] : 0.0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[q] = fma(T[(r0 + q) * 32 + m], xm, acc[q]);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) A[(r0 + q) * kLdA + oj + lane] = -acc[q];
     }
     __syncthreads();
   }
   // R^{-1} = D^-1/2 Rs^{-1}: three bf16 planes over the full kPanel x kPanel square
   double x2 = 0.0;
-  for (int t = tid; t < kPanelSq; t += 256) {
-    const int r = t / kPanel, c = t % kPanel;
-    float x = 0.0f;
-    if (r <= c && c < w) {
-      const double xs = A[pk(r, c)];
-      x2 += xs * xs;
-      x = (float)(ds[r] * xs);
+  for (int q = tid; q < kPanelSq / 4; q += 256) {
+    const int r = q >> 5, c0 = (q & 31) * 4;
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = c0 + e;
+      v[e] = 0.0f;
+      if (r <= c && c < w) {
+        const double xs = A[r * kLdA + c];
+        x2 += xs * xs;
+        v[e] = (float)(ds[r] * xs);
+      }
     }
-    store_split3(x, j.rinv, t, kPanelSq);
+    store_split3x4(make_float4(v[0], v[1], v[2], v[3]), j.rinv, 4LL * q, kPanelSq);
   }
   if (j.first) {
     // the first pass is final unless it had to be shifted or Gs is poorly conditioned
-    // (CholQR loses orthogonality in proportion to cond(Gs))
+    // (Cholesky-QR loses orthogonality in proportion to cond(Gs))
     x2 = warp_sum_d(x2);
-    if (lane == 0) T[warp] = x2;
+    if (lane == 0) red_sh[warp] = x2;
     __syncthreads();
     if (tid == 0) {
       double tot2 = 0.0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) tot2 += T[i];
+      for (int i = 0; i < 8; ++i) tot2 += red_sh[i];
       const int again = (shifted || tot2 > kAgainMeanInv * w) ? 1 : 0;
       *j.again = again;
       *j.fin = again | (j.reorth ? *j.reorth : 0);
