@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define MAO_VERSION 1
+#define MAO_VERSION 2
 
 #if defined(__GNUC__)
 #define MAO_API __attribute__((visibility("default")))
@@ -299,11 +299,13 @@ typedef enum {
   MAO_K_PC_CHECK = 15,       /* adaptive check D = Q^T F Q and its ratio */
   MAO_K_PC_POWER = 16,       /* power step P = F Q */
   MAO_K_PC_SORT = 17,        /* sort keys, argsort, gathers */
-  MAO_K_PC_QR = 18,          /* QR tensor-core products: panel projections, W R^{-1} */
+  MAO_K_PC_QR = 18,          /* QR panel projections C = Q^T P, W = P - Q C (tensor cores) */
   MAO_K_PC_ROTATE = 19,      /* rotations into the eigenbasis and back (before the update) */
   MAO_K_PC_UPDATE = 20,      /* last rotation fused with the weight update */
   MAO_K_PC_PANEL = 21,       /* QR panel Gram products (tensor cores, K slices) and their reduction */
-  MAO_K_PC_CHOL = 22         /* QR panel Cholesky and R^{-1} (fp64, one block per panel) */
+  MAO_K_PC_CHOL = 22,        /* QR panel Cholesky and R^{-1} (fp64, one block per panel) */
+  MAO_K_PC_QR_APPLY = 23,    /* QR panel products W R^{-1} (tensor cores) */
+  MAO_K_PC_QR_REDUCE = 24    /* sum of the K-slice partials of the projection coefficients */
 } mao_kernel_id;
 
 /* What one recorded launch was: its kernel and its algorithmic work (useful
@@ -311,8 +313,12 @@ typedef enum {
 typedef struct {
   int32_t kernel; /* mao_kernel_id */
   int32_t pad;
-  double flops;
-  double bytes;
+  double flops;     /* algorithmic floating-point operations of the launch (2 per multiply-add);
+                       launches whose work is decided on the device count none */
+  double bytes;     /* algorithmic bytes moved (memory-bound kernels), else 0 */
+  double tc_flops;  /* tensor-core operations issued for `flops`: an fp32-faithful product of
+                       three-plane operands issues six bf16 products per multiply-add, a
+                       three-plane by one-plane product three, a bf16 product one */
 } mao_launch_info;
 
 /*

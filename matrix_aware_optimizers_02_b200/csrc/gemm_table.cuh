@@ -28,7 +28,9 @@ mao_status launch_table_majors(const GemmTableParams& p, cudaStream_t stream, in
   }
   if (p.total_tiles <= 0) return MAO_OK;
   const int grid = p.total_tiles < d->sm_count ? p.total_tiles : d->sm_count;
-  LaunchScope ls(stream, kernel_id, flops, 0.0);
+  // tensor-core products per multiply-add: pairs (i, j), i < PA, j < PB, i + j <= max(PA, PB) - 1
+  constexpr int kProducts = (PA == 3 && PB == 3) ? 6 : (PA == 1 && PB == 1) ? 1 : 3;
+  LaunchScope ls(stream, kernel_id, flops, 0.0, flops * kProducts);
   kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? MAO_OK : MAO_ERR_CUDA;
 }

@@ -101,7 +101,7 @@ Profiler& profiler();
 struct LaunchScope {
   cudaStream_t s;
   int slot = -1;
-  LaunchScope(cudaStream_t stream, int kernel, double flops, double bytes) : s(stream) {
+  LaunchScope(cudaStream_t stream, int kernel, double flops, double bytes, double tc_flops = -1.0) : s(stream) {
     Profiler& P = profiler();
     if (!P.active) return;
     const int i = P.count++;
@@ -111,6 +111,7 @@ struct LaunchScope {
       P.info[i].pad = 0;
       P.info[i].flops = flops;
       P.info[i].bytes = bytes;
+      P.info[i].tc_flops = tc_flops >= 0.0 ? tc_flops : flops;
       cudaEventRecord(static_cast<cudaEvent_t>(P.events[2 * i]), s);
     }
   }

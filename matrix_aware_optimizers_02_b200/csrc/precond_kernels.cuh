@@ -149,6 +149,10 @@ struct SortJob {
   const float* Q;
   const float* P;
   double* key;
+  float* pn;          // squared column norms of P (original order)
+  float* pn_sorted;   // ... in the sorted order (argsort), or nullptr
+  double* dg;         // diag(Q^T F Q) = the dot products (adaptive check), or nullptr
+  const int* kflag;   // gate of the key pass (nullptr: always runs)
   int* perm;          // workspace permutation (always written when the refresh runs)
   int* perm_out;      // caller's copy, or nullptr
   const int* flag;
@@ -167,42 +171,54 @@ __device__ __forceinline__ int find_sort(const SortJob* J, int n, int blk) {
   return lo;
 }
 
-// key_i = sum_r Q[r][i] P[r][i] in fp64: one block per 32 columns, warp w sums the
-// rows w, w + 8, ... (each warp reads 128 contiguous bytes per row of Q and P), then
-// the eight warp sums are added in warp order.
-__global__ void __launch_bounds__(256) pc_keys_kernel(const SortJob* __restrict__ J, int n) {
+// key_i = sum_r Q[r][i] P[r][i] in fp64 (or -i when sorting is off, which makes
+// the argsort the identity), and the squared column norms of P in the same pass:
+// one block per 32 columns, warp w sums the rows w, w + 8, ... (each warp reads 128
+// contiguous bytes per row of Q and P), then the eight warp sums are added in warp order.
+__global__ void __launch_bounds__(256) pc_keys_kernel(const SortJob* __restrict__ J, int n, int sort) {
   __shared__ double part[8][32];
+  __shared__ float partn[8][32];
   const SortJob& j = J[find_sort<true>(J, n, blockIdx.x)];
-  if (j.flag && *j.flag == 0) return;
+  if (j.kflag && *j.kflag == 0) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int i = (blockIdx.x - j.key_blk_begin) * 32 + lane;
+  const bool dots = sort || j.dg;
   double s0 = 0.0, s1 = 0.0;
+  float n0 = 0.f, n1 = 0.f;
   if (i < j.k) {
     int r = warp;
     for (; r + 8 < j.k; r += 16) {
-      s0 += (double)j.Q[(long long)r * j.k + i] * (double)j.P[(long long)r * j.k + i];
-      s1 += (double)j.Q[(long long)(r + 8) * j.k + i] * (double)j.P[(long long)(r + 8) * j.k + i];
+      const float p0 = j.P[(long long)r * j.k + i], p1 = j.P[(long long)(r + 8) * j.k + i];
+      n0 += p0 * p0;
+      n1 += p1 * p1;
+      if (dots) {
+        s0 += (double)j.Q[(long long)r * j.k + i] * (double)p0;
+        s1 += (double)j.Q[(long long)(r + 8) * j.k + i] * (double)p1;
+      }
     }
-    if (r < j.k) s0 += (double)j.Q[(long long)r * j.k + i] * (double)j.P[(long long)r * j.k + i];
+    if (r < j.k) {
+      const float p0 = j.P[(long long)r * j.k + i];
+      n0 += p0 * p0;
+      if (dots) s0 += (double)j.Q[(long long)r * j.k + i] * (double)p0;
+    }
   }
   part[warp][lane] = s0 + s1;
+  partn[warp][lane] = n0 + n1;
   __syncthreads();
   if (warp == 0 && i < j.k) {
     double s = 0.0;
+    float nn = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) s += part[w][lane];
+    for (int w = 0; w < 8; ++w) {
+      s += part[w][lane];
+      nn += partn[w][lane];
+    }
+    if (j.dg) j.dg[i] = s;
+    if (!sort) s = -(double)i;
     if (!(s == s)) s = -INFINITY;  // a NaN key sorts last, so the permutation stays a bijection
     j.key[i] = s;
+    j.pn[i] = nn;
   }
-}
-
-// Sorting disabled: strictly decreasing keys, so the argsort yields the identity
-// (same block mapping as the key kernel: 32 columns per block).
-__global__ void __launch_bounds__(256) pc_identity_keys_kernel(const SortJob* __restrict__ J, int n) {
-  const SortJob& j = J[find_sort<true>(J, n, blockIdx.x)];
-  if (j.flag && *j.flag == 0) return;
-  const int i = (blockIdx.x - j.key_blk_begin) * 32 + threadIdx.x;
-  if (threadIdx.x < 32 && i < j.k) j.key[i] = -(double)i;
 }
 
 // Stable descending argsort by rank counting: rank_i = #{key_j > key_i} + #{j < i: key_j == key_i};
@@ -233,6 +249,7 @@ __global__ void __launch_bounds__(256) pc_argsort_kernel(const SortJob* __restri
   if (i < j.k) {
     j.perm[rank] = i;
     if (j.perm_out) j.perm_out[rank] = i;
+    if (j.pn_sorted) j.pn_sorted[rank] = j.pn[i];
   }
 }
 
@@ -686,62 +703,6 @@ __global__ void __launch_bounds__(256) pc_coef_reduce_kernel(const CoefJob* __re
   store_split3x4(acc, j.cp, e, j.pstride);
 }
 
-// Squared column norms of a k x k matrix (ld k): partial sums over 256-row blocks,
-// then their totals in row-block order (deterministic).
-struct ColsqJob {
-  const float* src;
-  float* part;       // rblocks x k
-  float* out;        // k
-  const int* flag;
-  int k, rblocks, cblocks;
-  int blk_begin;     // partial pass: rblocks * cblocks blocks of this job
-  int fin_begin;     // final pass: cblocks blocks of this job
-};
-
-template <bool FINAL>
-__device__ __forceinline__ int find_colsq(const ColsqJob* J, int n, int blk) {
-  int lo = 0, hi = n - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if ((FINAL ? J[mid].fin_begin : J[mid].blk_begin) <= blk) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
-__global__ void __launch_bounds__(256) pc_colsq_partial_kernel(const ColsqJob* __restrict__ J, int n) {
-  const ColsqJob& j = J[find_colsq<false>(J, n, blockIdx.x)];
-  if (j.flag && *j.flag == 0) return;
-  const int local = blockIdx.x - j.blk_begin;
-  const int rb = local / j.cblocks, c = (local % j.cblocks) * 256 + threadIdx.x;
-  if (c >= j.k) return;
-  const int r0 = rb * 256, r1 = min(j.k, r0 + 256);
-  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-  int r = r0;
-  for (; r + 3 < r1; r += 4) {
-    const float a = j.src[(long long)r * j.k + c], b = j.src[(long long)(r + 1) * j.k + c];
-    const float e = j.src[(long long)(r + 2) * j.k + c], f = j.src[(long long)(r + 3) * j.k + c];
-    s0 += a * a;
-    s1 += b * b;
-    s2 += e * e;
-    s3 += f * f;
-  }
-  for (; r < r1; ++r) {
-    const float a = j.src[(long long)r * j.k + c];
-    s0 += a * a;
-  }
-  j.part[(long long)rb * j.k + c] = (s0 + s1) + (s2 + s3);
-}
-
-__global__ void __launch_bounds__(256) pc_colsq_final_kernel(const ColsqJob* __restrict__ J, int n) {
-  const ColsqJob& j = J[find_colsq<true>(J, n, blockIdx.x)];
-  if (j.flag && *j.flag == 0) return;
-  const int c = (blockIdx.x - j.fin_begin) * 256 + threadIdx.x;
-  if (c >= j.k) return;
-  float s = 0.f;
-  for (int rb = 0; rb < j.rblocks; ++rb) s += j.part[(long long)rb * j.k + c];
-  j.out[c] = s;
-}
-
 // ------------------------------------------------------------------ FOAM pieces
 // Row/column partial sums of Gr^2 over 64 x 64 tiles (Gr m x n fp32, ld n).
 struct RcJob {
@@ -872,8 +833,14 @@ __global__ void __launch_bounds__(256) foam_n_kernel(const EwJob* __restrict__ J
 }
 
 // Adaptive check: rho = ||offdiag D||_F / ||D||_F, flag = rho > tol (one block per matrix).
+// Adaptive refresh check.  With D = Q^T F Q and an orthogonal Q, ||D||_F = ||F||_F =
+// ||F Q||_F and diag(D)_i = q_i^T F q_i, so
+//   rho^2 = ||D - diag(D)||_F^2 / ||D||_F^2 = 1 - sum_i diag(D)_i^2 / ||P||_F^2,  P = F Q,
+// from the power product the refresh needs anyway (same value as forming D, up to
+// rounding).  One block per factor; sums in a fixed order.
 struct CheckJob {
-  const float* D;
+  const double* dg;   // diag(D) (k)
+  const float* pn;    // squared column norms of P (k)
   int* flag;
   float* rho;
   int k;
@@ -882,16 +849,14 @@ struct CheckJob {
 __global__ void __launch_bounds__(256) pc_check_kernel(const CheckJob* __restrict__ J, float tol) {
   __shared__ double red[2][256];
   const CheckJob& j = J[blockIdx.x];
-  double off = 0.0, tot = 0.0;
-  const long long total = (long long)j.k * j.k;
-  for (long long e = threadIdx.x; e < total; e += 256) {
-    const double x = j.D[e];
-    const int r = (int)(e / j.k), c = (int)(e - (long long)r * j.k);
-    tot += x * x;
-    if (r != c) off += x * x;
+  double d2 = 0.0, p2 = 0.0;
+  for (int i = threadIdx.x; i < j.k; i += 256) {
+    const double d = j.dg[i];
+    d2 += d * d;
+    p2 += (double)j.pn[i];
   }
-  red[0][threadIdx.x] = off;
-  red[1][threadIdx.x] = tot;
+  red[0][threadIdx.x] = d2;
+  red[1][threadIdx.x] = p2;
   __syncthreads();
   for (int o = 128; o > 0; o >>= 1) {
     if (threadIdx.x < o) {
@@ -901,7 +866,8 @@ __global__ void __launch_bounds__(256) pc_check_kernel(const CheckJob* __restric
     __syncthreads();
   }
   if (threadIdx.x == 0) {
-    const double rho = red[1][0] > 0.0 ? sqrt(red[0][0]) / sqrt(red[1][0]) : 0.0;
+    const double r2 = red[1][0] > 0.0 ? 1.0 - red[0][0] / red[1][0] : 0.0;
+    const double rho = r2 > 0.0 ? sqrt(r2) : 0.0;  // NaN input: no refresh
     *j.rho = (float)rho;
     *j.flag = (rho > (double)tol) ? 1 : 0;
   }

@@ -97,9 +97,9 @@ struct SideBuf {
   size_t Fp, Qp, P, Ps, Psp;
   size_t W, Wp, Cp;  // panel buffer (k x kPanel, fp32 and planes) and the coefficients
   size_t Cpart;      // K-slice partials of the coefficients (large factors only)
-  size_t cpart, pnorm2, reorth, fin;  // column norms of the gathered P (partials, totals); panel decisions
+  size_t pn, pnorm2, reorth, fin;  // squared column norms of P (original, sorted order); panel decisions
   size_t part, gs, rinv, keys, perm, flag, rho, bad, again;
-  size_t Tp, D;  // adaptive check
+  size_t dg;     // adaptive check: diag(Q^T F Q)
 };
 
 struct MatBuf {
@@ -132,12 +132,9 @@ void side_layout(int k, bool check, Carver& cv, SideBuf& s, size_t flag_block) {
   s.again = s.flag + 48;
   s.reorth = s.flag + 56;
   s.fin = s.flag + 60;
-  s.cpart = cv.take(4 * (size_t)((k + 255) / 256) * k);
+  s.pn = cv.take(4 * (size_t)k);
   s.pnorm2 = cv.take(4 * (size_t)k);
-  if (check) {
-    s.Tp = cv.take(planes_bytes(k, k));
-    s.D = cv.take(4 * kk);
-  }
+  if (check) s.dg = cv.take(8 * (size_t)k);
 }
 
 struct Ctx {
@@ -226,8 +223,7 @@ void make_groups(const Ctx& X, std::vector<GroupPlan>& groups) {
 // Records every launch of one group into `ops`, with all device data staged in
 // the arena; in sizing mode (ws == nullptr) only the sizes matter.
 struct Op {
-  enum Kind { GEMM, EW, SPLIT, ADAM, KEYS, ARGSORT, GATHER, COLSQ, COLSQFIN, VPERM, REDUCE, CHOL, COEFRED, RC, TAU,
-              FOAMN, CHECK } kind;
+  enum Kind { GEMM, EW, SPLIT, ADAM, KEYS, ARGSORT, GATHER, VPERM, REDUCE, CHOL, COEFRED, RC, TAU, FOAMN, CHECK } kind;
   size_t jobs = 0;
   int njobs = 0;
   int blocks = 0;
@@ -312,65 +308,38 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
   auto side = [&](int u) -> SideBuf& { return units[u].left ? G.mb[units[u].i].L : G.mb[units[u].i].R; };
   auto mat = [&](int u) -> const PcMat& { return X.mats[G.g0 + units[u].i]; };
   auto kof = [&](int u) { return units[u].left ? mat(u).m : mat(u).n; };
-  auto Fp = [&](int u) { return units[u].left ? mat(u).L : mat(u).R; };
   auto Qp = [&](int u) { return units[u].left ? mat(u).QL : mat(u).QR; };
   auto permo = [&](int u) { return units[u].left ? mat(u).perm_L : mat(u).perm_R; };
   auto flagp = [&](int u) -> const int* { return check ? B.wp<int>(side(u).flag) : nullptr; };
 
-  // three-plane splits of F and Q
+  // three-plane split of Q (F's planes come from the factor products)
   {
     size_t off;
-    EwJob* J = B.new_jobs<EwJob>(Op::SPLIT, 2 * nu, off);
+    EwJob* J = B.new_jobs<EwJob>(Op::SPLIT, nu, off);
     int blk = 0;
     for (int i = 0; i < nu; ++i) {
       const int k = kof(i);
-      for (int w = 0; w < 2; ++w) {
-        EwJob& j = J[2 * i + w];
-        j.a = w == 0 ? Fp(i) : Qp(i);
-        j.pa = B.wp<__nv_bfloat16>(w == 0 ? side(i).Fp : side(i).Qp);
-        j.pstride = B.pstride(k, k);
-        j.rows = k;
-        j.cols = k;
-        j.lda = k;
-        j.ldp = ldp_of(k);
-        j.blk_begin = blk;
-        blk += ew_blocks(k, k);
-      }
+      EwJob& j = J[i];
+      j.a = Qp(i);
+      j.pa = B.wp<__nv_bfloat16>(side(i).Qp);
+      j.pstride = B.pstride(k, k);
+      j.rows = k;
+      j.cols = k;
+      j.lda = k;
+      j.ldp = ldp_of(k);
+      j.blk_begin = blk;
+      blk += ew_blocks(k, k);
     }
     B.ops.back().blocks = blk;
-  }
-  if (check) {
-    // D = Q^T F Q: T = Q^T F (A = Q stored K x M), D = T Q (B = Q stored K x N)
-    TableLaunch& g1 = B.new_gemm(1, 1, MAO_K_PC_CHECK);
-    for (int i = 0; i < nu; ++i) {
-      const int k = kof(i);
-      const Split3 Tp = B.planes(side(i).Tp, k, k);
-      MAO_TRY(table_add(g1, B.maps, B.planes(side(i).Qp, k, k), B.planes(side(i).Fp, k, k), k, k, k, 0, 0, nullptr,
-                        &Tp, k, nullptr, 0, 1.f, 0.f, nullptr));
-    }
-    TableLaunch& g2 = B.new_gemm(0, 1, MAO_K_PC_CHECK);
-    for (int i = 0; i < nu; ++i) {
-      const int k = kof(i);
-      MAO_TRY(table_add(g2, B.maps, B.planes(side(i).Tp, k, k), B.planes(side(i).Qp, k, k), k, k, k, 0, 0,
-                        B.wp<float>(side(i).D), nullptr, k, nullptr, 0, 1.f, 0.f, nullptr));
-    }
-    size_t off;
-    CheckJob* J = B.new_jobs<CheckJob>(Op::CHECK, nu, off);
-    for (int i = 0; i < nu; ++i) {
-      J[i].D = B.wp<float>(side(i).D);
-      J[i].flag = B.wp<int>(side(i).flag);
-      J[i].rho = B.wp<float>(side(i).rho);
-      J[i].k = kof(i);
-    }
-    B.ops.back().blocks = nu;
   }
   // power step P = F Q (A = F K-major, B = Q stored K x N)
   {
     TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_POWER);
     for (int i = 0; i < nu; ++i) {
       const int k = kof(i);
+      // an adaptive check needs P itself, so the product is not gated
       MAO_TRY(table_add(g, B.maps, B.planes(side(i).Fp, k, k), B.planes(side(i).Qp, k, k), k, k, k, 0, 0,
-                        B.wp<float>(side(i).P), nullptr, k, nullptr, 0, 1.f, 0.f, flagp(i)));
+                        B.wp<float>(side(i).P), nullptr, k, nullptr, 0, 1.f, 0.f, nullptr));
     }
   }
   // keys and argsort
@@ -384,6 +353,10 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
       j.Q = Qp(i);
       j.P = B.wp<float>(side(i).P);
       j.key = B.wp<double>(side(i).keys);
+      j.pn = B.wp<float>(side(i).pn);
+      j.pn_sorted = B.wp<float>(side(i).pnorm2);
+      j.dg = check ? B.wp<double>(side(i).dg) : nullptr;
+      j.kflag = nullptr;
       j.perm = B.wp<int>(side(i).perm);
       j.perm_out = permo(i);
       j.flag = flagp(i);
@@ -395,6 +368,18 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
     }
     B.ops.back().blocks = kblk;
     Op o = B.ops.back();  // the argsort reuses the job array
+    if (check) {
+      size_t coff;
+      CheckJob* C = B.new_jobs<CheckJob>(Op::CHECK, nu, coff);
+      for (int i = 0; i < nu; ++i) {
+        C[i].dg = B.wp<double>(side(i).dg);
+        C[i].pn = B.wp<float>(side(i).pn);
+        C[i].flag = B.wp<int>(side(i).flag);
+        C[i].rho = B.wp<float>(side(i).rho);
+        C[i].k = kof(i);
+      }
+      B.ops.back().blocks = nu;
+    }
     o.kind = Op::ARGSORT;
     o.blocks = blk;
     B.ops.push_back(o);
@@ -422,33 +407,6 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
       blk += ew_blocks(k, k);
     }
     B.ops.back().blocks = blk;
-  }
-  // squared column norms of the gathered P (the reorthogonalisation criterion)
-  {
-    size_t off;
-    ColsqJob* J = B.new_jobs<ColsqJob>(Op::COLSQ, nu, off);
-    int blk = 0, fin = 0;
-    for (int i = 0; i < nu; ++i) {
-      const int k = kof(i);
-      ColsqJob& j = J[i];
-      j.src = B.wp<float>(side(i).Ps);
-      j.part = B.wp<float>(side(i).cpart);
-      j.out = B.wp<float>(side(i).pnorm2);
-      j.flag = flagp(i);
-      j.k = k;
-      j.rblocks = (k + 255) / 256;
-      j.cblocks = (k + 255) / 256;
-      j.blk_begin = blk;
-      blk += j.rblocks * j.cblocks;
-      j.fin_begin = fin;
-      fin += j.cblocks;
-    }
-    B.ops.back().blocks = blk;
-    Op o = B.ops.back();
-    o.kind = Op::COLSQFIN;
-    o.blocks = fin;
-    B.ops.push_back(o);
-    B.gemm_of_op.push_back(-1);
   }
   // QR by panels of kPanel columns: block Gram-Schmidt with two projection passes,
   // Cholesky-QR inside each panel (twice after the first pass, once after the second)
@@ -532,7 +490,7 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
       ch.blocks = (int)act.size();
       B.ops.push_back(ch);
       B.gemm_of_op.push_back(-1);
-      TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_QR);
+      TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_QR_APPLY);
       for (int i : act) {
         const int k = kof(i), w = wdt(i);
         __nv_bfloat16* r = B.wp<__nv_bfloat16>(side(i).rinv);
@@ -686,8 +644,9 @@ mao_status build_group(Builder& B, GroupPlan& G) {
     g.pa = g.pb = gpl;
     for (int i = 0; i < nm; ++i) {
       const PcMat& a = A(i);
-      MAO_TRY(table_add(g, B.maps, Gop(i), Gop(i), a.m, a.m, a.n, 0, 0, a.L, nullptr, a.m, a.L, a.m, 1.f - X.b2,
-                        X.b2, nullptr));
+      const Split3 Fp = B.planes(G.mb[i].L.Fp, a.m, a.m);  // planes of the new L for the refresh
+      MAO_TRY(table_add(g, B.maps, Gop(i), Gop(i), a.m, a.m, a.n, 0, 0, a.L, X.mode != 0 ? &Fp : nullptr, a.m, a.L,
+                        a.m, 1.f - X.b2, X.b2, nullptr));
     }
   }
   {
@@ -695,8 +654,9 @@ mao_status build_group(Builder& B, GroupPlan& G) {
     g.pa = g.pb = gpl;
     for (int i = 0; i < nm; ++i) {
       const PcMat& a = A(i);
-      MAO_TRY(table_add(g, B.maps, Gop(i), Gop(i), a.n, a.n, a.m, 0, 0, a.R, nullptr, a.n, a.R, a.n, 1.f - X.b2,
-                        X.b2, nullptr));
+      const Split3 Fp = B.planes(G.mb[i].R.Fp, a.n, a.n);
+      MAO_TRY(table_add(g, B.maps, Gop(i), Gop(i), a.n, a.n, a.m, 0, 0, a.R, X.mode != 0 ? &Fp : nullptr, a.n, a.R,
+                        a.n, 1.f - X.b2, X.b2, nullptr));
     }
   }
   // refresh, or plain planes of the bases
@@ -1029,10 +989,7 @@ mao_status run_ops(const Ctx& X, uint8_t* arena_dev, const BuiltGroup& bg, DevSt
       }
       case Op::KEYS: {
         LaunchScope ls(s, MAO_K_PC_SORT, 0.0, 0.0);
-        if (X.rf.sort)
-          pc_keys_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<SortJob>(op.jobs), n);
-        else
-          pc_identity_keys_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<SortJob>(op.jobs), n);
+        pc_keys_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<SortJob>(op.jobs), n, X.rf.sort ? 1 : 0);
         break;
       }
       case Op::ARGSORT: {
@@ -1056,18 +1013,8 @@ mao_status run_ops(const Ctx& X, uint8_t* arena_dev, const BuiltGroup& bg, DevSt
         break;
       }
       case Op::COEFRED: {
-        LaunchScope ls(s, MAO_K_PC_QR, 0.0, 0.0);
+        LaunchScope ls(s, MAO_K_PC_QR_REDUCE, 0.0, 0.0);
         pc_coef_reduce_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<CoefJob>(op.jobs), n);
-        break;
-      }
-      case Op::COLSQ: {
-        LaunchScope ls(s, MAO_K_PC_SORT, 0.0, 0.0);
-        pc_colsq_partial_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<ColsqJob>(op.jobs), n);
-        break;
-      }
-      case Op::COLSQFIN: {
-        LaunchScope ls(s, MAO_K_PC_SORT, 0.0, 0.0);
-        pc_colsq_final_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<ColsqJob>(op.jobs), n);
         break;
       }
       case Op::CHOL: {
