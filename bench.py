@@ -58,6 +58,12 @@ def parse():
     ap.add_argument("--optimizers", default="muon,soap,foam", help="comma list of muon, soap, foam")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    ap.add_argument("--launch-log", default=None,
+                    help="after the measurement, run one more step and write its launch list (kernel, work) here")
+    ap.add_argument("--traffic-csv", default=None,
+                    help="offline: ncu CSV (dram__bytes_read/write.sum, gpu__time_duration.sum) of a run made with "
+                         "--launch-log; folds the last step's launches into --traffic-out (no GPU needed)")
+    ap.add_argument("--traffic-out", default=os.path.join(ROOT, "profiles", "ncu_traffic.json"))
     return ap.parse_args()
 
 
@@ -145,8 +151,10 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_name, workload):
-    """DRAM bytes per launch from a committed ncu capture, if its sources match."""
+def ncu_traffic(kernel_name, flops_per_launch, bytes_per_launch):
+    """DRAM bytes per launch of a kernel from the committed ncu traffic summary, if the kernel
+    sources still match it.  The summary is measured on a workload small enough for ncu; its
+    DRAM bytes per algorithmic FLOP (or byte) scale to this launch's work."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
@@ -154,8 +162,101 @@ def ncu_traffic(kernel_name, workload):
         d = json.load(f)
     if d.get("source_hash") != kernel_source_hash():
         return None
-    e = d.get("kernels", {}).get(f"{workload}/{kernel_name}")
-    return None if e is None else e.get("dram_bytes_per_launch")
+    e = d.get("kernels", {}).get(kernel_name)
+    if e is None:
+        return None
+    if flops_per_launch > 0 and e.get("dram_bytes_per_flop") is not None:
+        return {"bytes": round(e["dram_bytes_per_flop"] * flops_per_launch),
+                "scaled_from": d.get("measured_on"), "by": "algorithmic flops"}
+    if bytes_per_launch > 0 and e.get("dram_bytes_per_alg_byte") is not None:
+        return {"bytes": round(e["dram_bytes_per_alg_byte"] * bytes_per_launch),
+                "scaled_from": d.get("measured_on"), "by": "algorithmic bytes"}
+    return None
+
+
+def write_launch_log(args, lib, L, LS, t, stream):
+    """One more step with the launch profiler recording kernel ids and work only."""
+    import torch
+    torch.cuda.synchronize()
+    lib.mao_profile_start(None, None, 0)
+    LS.step(t, stream)
+    n = lib.mao_profile_stop()
+    torch.cuda.synchronize()
+    info = (L.LaunchInfo * max(n, 1))()
+    L.check(lib.mao_profile_start(None, info, n))
+    LS.step(t, stream)  # the same t: the same launch plan
+    m = lib.mao_profile_stop()
+    torch.cuda.synchronize()
+    rows = [{"kernel": L.KERNEL_NAMES.get(info[i].kernel, str(info[i].kernel)), "flops": info[i].flops,
+             "bytes": info[i].bytes, "tc_flops": info[i].tc_flops} for i in range(min(n, m))]
+    with open(args.launch_log, "w") as f:
+        json.dump({"workload": args.workload, "optimizers": args.optimizers, "source_hash": kernel_source_hash(),
+                   "launches": rows}, f)
+
+
+def fold_traffic(args):
+    """Per kernel id: DRAM bytes per launch, per algorithmic FLOP and per algorithmic byte, from the
+    ncu CSV of a --launch-log run (its last len(launches) library launches are the logged step)."""
+    import csv
+    with open(args.launch_log) as f:
+        log = json.load(f)
+    rows = list(csv.reader(open(args.traffic_csv)))
+    head = None
+    per = {}
+    for r in rows:
+        if "Kernel Name" in r:
+            head = r
+            continue
+        if head is None or len(r) != len(head):
+            continue
+        d = dict(zip(head, r))
+        e = per.setdefault(int(d["ID"]), {})
+        e[d["Metric Name"]] = float(d["Metric Value"].replace(",", ""))
+    ids = sorted(per)
+    launches = log["launches"]
+    tail = ids[-len(launches):]
+    if len(tail) != len(launches):
+        raise SystemExit("fewer ncu launches than logged launches")
+    # each profiler id is launched by these kernels (first word of ncu's kernel name)
+    fam = {"muon_prep": ["muon_prep_kernel"], "muon_scale": ["muon_scale_kernel"], "muon_stats": ["muon_stats_kernel"],
+           "muon_update": ["muon_update_kernel"], "muon_colsq": ["muon_norm_tile_kernel"],
+           "muon_colscale": ["muon_norm_final_kernel"], "muon_rowscale": ["muon_norm_tile_kernel",
+                                                                          "muon_norm_final_kernel"],
+           "pc_elementwise": ["pc_momentum_kernel", "pc_split_kernel", "soap_adam_kernel", "foam_rc_partial_kernel",
+                              "foam_tau_kernel", "foam_n_kernel"],
+           "pc_sort": ["pc_keys_kernel", "pc_argsort_kernel", "pc_gather_cols_kernel", "soap_vperm_kernel"],
+           "pc_check": ["pc_check_kernel"], "pc_chol": ["qr_chol_kernel"], "pc_qr_reduce": ["pc_coef_reduce_kernel"],
+           "pc_stats": ["pc_stats_kernel"], "pc_panel": ["gemm_tc_table_kernel", "qr_gram_reduce_kernel"]}
+    names = {}
+    for r in rows:
+        if head is not None and len(r) == len(head) and "Kernel Name" not in r:
+            d = dict(zip(head, r))
+            names[int(d["ID"])] = d["Kernel Name"].split("(")[0].split("<")[0].split()[-1]
+    for rec, i in zip(launches, tail):
+        ok = fam.get(rec["kernel"], ["gemm_tc_table_kernel", "gemm_tc_kernel"])
+        if names[i] not in ok:
+            raise SystemExit(f"launch {i}: ncu saw {names[i]}, the log says {rec['kernel']}: not aligned")
+    agg = {}
+    for rec, i in zip(launches, tail):
+        m = per[i]
+        a = agg.setdefault(rec["kernel"], {"launches": 0, "dram": 0.0, "flops": 0.0, "bytes": 0.0, "ns": 0.0})
+        a["launches"] += 1
+        a["dram"] += m.get("dram__bytes_read.sum", 0.0) + m.get("dram__bytes_write.sum", 0.0)
+        a["flops"] += rec["flops"]
+        a["bytes"] += rec["bytes"]
+        a["ns"] += m.get("gpu__time_duration.sum", 0.0)
+    out = {"source_hash": log["source_hash"], "measured_on": log["workload"], "kernels": {}}
+    for k, a in sorted(agg.items()):
+        out["kernels"][k] = {
+            "launches": a["launches"],
+            "dram_bytes_per_launch": a["dram"] / a["launches"],
+            "dram_bytes_per_flop": (a["dram"] / a["flops"]) if a["flops"] > 0 else None,
+            "dram_bytes_per_alg_byte": (a["dram"] / a["bytes"]) if a["bytes"] > 0 else None,
+            "ncu_ms": a["ns"] / 1e6,
+        }
+    with open(args.traffic_out, "w") as f:
+        json.dump(out, f, indent=1)
+    print(json.dumps(out, indent=1))
 
 
 # ----------------------------------------------------------------------------- CPU (oracle) leg
@@ -392,6 +493,9 @@ def run_mine(args, rank, world, dist):
     barrier()
     e2e_ms = e0.elapsed_time(e1) / args.steps
 
+    if args.launch_log and rank == 0:
+        write_launch_log(args, lib, L, LS, t + 1, stream)
+
     tt = torch.tensor([ms, e2e_ms], device=dev)
     if dist is not None:
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -423,7 +527,10 @@ def run_mine(args, rank, world, dist):
             roof = {"bound": "hbm", "kernel": names.get(dom, str(dom)), "achieved": round(achieved, 1),
                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                     "peak_source": f"{peak_src} HBM copy"}
-        roof["traffic"] = ncu_traffic(names.get(dom, str(dom)), args.workload)
+        tr = ncu_traffic(names.get(dom, str(dom)), e["flops"] / e["n"], e["bytes"] / e["n"])
+        roof["traffic"] = tr["bytes"] if tr else None
+        if tr:
+            roof["traffic_source"] = f"ncu DRAM bytes per {tr['by']} on {tr['scaled_from']}, scaled to this launch"
         roof["launches"] = e["n"]
         roof["avg_launch_ms"] = round(avg_ms, 4)
     tot = max(sum(x["ms"] for x in per.values()), 1e-9)
@@ -505,6 +612,9 @@ def run_reference(args, rank, world):
 
 def main():
     args = parse()
+    if args.traffic_csv:
+        fold_traffic(args)
+        return 0
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if args.impl == "reference":

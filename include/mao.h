@@ -305,7 +305,8 @@ typedef enum {
   MAO_K_PC_PANEL = 21,       /* QR panel Gram products (tensor cores, K slices) and their reduction */
   MAO_K_PC_CHOL = 22,        /* QR panel Cholesky and R^{-1} (fp64, one block per panel) */
   MAO_K_PC_QR_APPLY = 23,    /* QR panel products W R^{-1} (tensor cores) */
-  MAO_K_PC_QR_REDUCE = 24    /* sum of the K-slice partials of the projection coefficients */
+  MAO_K_PC_QR_REDUCE = 24,   /* sum of the K-slice partials of the projection coefficients */
+  MAO_K_PC_STATS = 25        /* per-matrix diagnostics of a SOAP / FOAM step */
 } mao_kernel_id;
 
 /* What one recorded launch was: its kernel and its algorithmic work (useful
@@ -326,8 +327,8 @@ typedef struct {
  * every kernel launch of the library is bracketed by cudaEventRecord of
  * events[2i] and events[2i+1] on the launching stream (no synchronisation) and
  * info[i] describes it, for the first `capacity` launches.  `events` is a host
- * array of 2*capacity cudaEvent_t created by the caller; `info` a host array of
- * `capacity`.  mao_profile_stop() ends recording and returns how many launches
+ * array of 2*capacity cudaEvent_t created by the caller, or NULL to record only
+ * `info`; `info` a host array of `capacity`.  mao_profile_stop() ends recording and returns how many launches
  * happened since the start (which may exceed capacity).  Not thread-safe: one
  * profiling session per process at a time.
  */

@@ -191,7 +191,7 @@ Profiler& profiler() {
 }  // namespace mao
 
 extern "C" mao_status mao_profile_start(void** events, mao_launch_info* info, int32_t capacity) {
-  if (capacity < 0 || (capacity > 0 && (events == nullptr || info == nullptr))) return MAO_ERR_INVALID_ARG;
+  if (capacity < 0 || (capacity > 0 && info == nullptr)) return MAO_ERR_INVALID_ARG;
   Profiler& P = profiler();
   P.events = events;
   P.info = info;

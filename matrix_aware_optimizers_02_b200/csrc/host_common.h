@@ -112,11 +112,11 @@ struct LaunchScope {
       P.info[i].flops = flops;
       P.info[i].bytes = bytes;
       P.info[i].tc_flops = tc_flops >= 0.0 ? tc_flops : flops;
-      cudaEventRecord(static_cast<cudaEvent_t>(P.events[2 * i]), s);
+      if (P.events) cudaEventRecord(static_cast<cudaEvent_t>(P.events[2 * i]), s);
     }
   }
   ~LaunchScope() {
-    if (slot >= 0) cudaEventRecord(static_cast<cudaEvent_t>(profiler().events[2 * slot + 1]), s);
+    if (slot >= 0 && profiler().events) cudaEventRecord(static_cast<cudaEvent_t>(profiler().events[2 * slot + 1]), s);
   }
 };
 

@@ -1176,6 +1176,7 @@ mao_status run_step(const Ctx& X, const void* mats, size_t mats_bytes, void* wor
     MAO_TRY(run_ops(X, arena_dev, bg, status, s));
     if (stats) {
       const int nm = g.g1 - g.g0;
+      LaunchScope ls(s, MAO_K_PC_STATS, 0.0, 0.0);
       pc_stats_kernel<<<(nm + 127) / 128, 128, 0, s>>>(reinterpret_cast<const StatsJob*>(arena_dev + bg.stats_jobs),
                                                          nm, stats);
       MAO_CUDA_TRY(cudaGetLastError());
