@@ -23,6 +23,14 @@ typedef enum {
   MAO_GEMM_SPLIT2 = 5
 } mao_gemm_kind;
 
+/* Flags OR-ed into a table-mode kind (all but MAO_GEMM_BF16): run the problems
+ * on the one-CTA kernel (128 x 128 tiles) or on the CTA-pair kernel (256 x 128
+ * tiles, tcgen05 cta_group::2; kinds with a three-plane operand only, else
+ * MAO_ERR_UNSUPPORTED); without a flag the library chooses as it does inside the
+ * optimizer steps. */
+#define MAO_GEMM_FORCE_ONE_CTA 16
+#define MAO_GEMM_FORCE_CTA_PAIR 32
+
 /*
  * D[b] = A[b] * B[b]^T for b < batch, with fp32 accumulation and fp32 D.
  *   kind MAO_GEMM_BF16:   A, B bf16; one bf16 tensor-core product, accumulated

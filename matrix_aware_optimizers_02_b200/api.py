@@ -128,7 +128,8 @@ def muon_step(mats, **kw) -> None:
 
 
 def gemm(A: torch.Tensor, B: torch.Tensor, *, kind: str = "bf16", a_mn_major: bool = False,
-         b_mn_major: bool = False, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+         b_mn_major: bool = False, kernel: str = "auto",
+         stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """Verification entry: D[b] = A[b] @ B[b]^T through the tensor-core GEMM core.
 
     A is (batch, M, K) (or (batch, K, M) when a_mn_major); B is (batch, N, K)
@@ -139,10 +140,12 @@ def gemm(A: torch.Tensor, B: torch.Tensor, *, kind: str = "bf16", a_mn_major: bo
       "split3_bf16" fp32 A (three planes) times bf16 B;
       "bf16_split3" bf16 A times fp32 B (three planes);
       "split2"      fp32 operands held as two bf16 planes each, three products.
+    kernel ("auto", "one_cta", "cta_pair") picks the table-mode kernel for every kind but "bf16".
     Returns fp32 (batch, M, N).
     """
     lib = L.load()
     k = {"bf16": 0, "split3": 1, "bf16_fold": 2, "split3_bf16": 3, "bf16_split3": 4, "split2": 5}[kind]
+    k |= {"auto": 0, "one_cta": 16, "cta_pair": 32}[kernel]
     batch = A.shape[0]
     M = A.shape[2] if a_mn_major else A.shape[1]
     K = A.shape[1] if a_mn_major else A.shape[2]

@@ -74,9 +74,14 @@ void kind_planes(int32_t kind, int* pa, int* pb) {
   }
 }
 
-mao_status gemm_layout(int32_t kind, int32_t batch, int32_t M, int32_t N, int32_t K, TestLayout& T) {
+mao_status gemm_layout(int32_t kind_flags, int32_t batch, int32_t M, int32_t N, int32_t K, TestLayout& T) {
   if (batch < 1 || M < 1 || N < 1 || K < 1) return MAO_ERR_SHAPE;
+  const int32_t kind = kind_flags & 15;
+  if ((kind_flags & ~(15 | MAO_GEMM_FORCE_ONE_CTA | MAO_GEMM_FORCE_CTA_PAIR)) != 0) return MAO_ERR_INVALID_ARG;
   if (kind < MAO_GEMM_BF16 || kind > MAO_GEMM_SPLIT2) return MAO_ERR_INVALID_ARG;
+  if (kind == MAO_GEMM_BF16 && (kind_flags & ~15)) return MAO_ERR_INVALID_ARG;
+  if ((kind_flags & MAO_GEMM_FORCE_CTA_PAIR) && (kind == MAO_GEMM_BF16_FOLD || kind == MAO_GEMM_SPLIT2))
+    return MAO_ERR_UNSUPPORTED;
   Carver cv;
   cv.take(kStatusBytes);
   if (kind != MAO_GEMM_BF16) {
@@ -101,13 +106,14 @@ extern "C" mao_status mao_test_gemm_workspace_size(int32_t kind, int32_t batch, 
   return MAO_OK;
 }
 
-extern "C" mao_status mao_test_gemm(int32_t kind, int32_t a_mn_major, int32_t b_mn_major, const void* A,
+extern "C" mao_status mao_test_gemm(int32_t kind_flags, int32_t a_mn_major, int32_t b_mn_major, const void* A,
                                     const void* B, float* D, int32_t batch, int32_t M, int32_t N, int32_t K,
                                     void* workspace, size_t ws_bytes, mao_stream_t stream_) {
   if (A == nullptr || B == nullptr || D == nullptr || workspace == nullptr) return MAO_ERR_INVALID_ARG;
   if ((a_mn_major != 0 && a_mn_major != 1) || (b_mn_major != 0 && b_mn_major != 1)) return MAO_ERR_INVALID_ARG;
   TestLayout T;
-  MAO_TRY(gemm_layout(kind, batch, M, N, K, T));
+  MAO_TRY(gemm_layout(kind_flags, batch, M, N, K, T));
+  const int32_t kind = kind_flags & 15;
   if (ws_bytes < T.total) return MAO_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MAO_ERR_ALIGN;
   if (!aligned16(A) || !aligned16(B) || !aligned16(D)) return MAO_ERR_ALIGN;
@@ -163,6 +169,7 @@ extern "C" mao_status mao_test_gemm(int32_t kind, int32_t a_mn_major, int32_t b_
   L.b_mn = b_mn_major;
   L.pa = pa;
   L.pb = pb;
+  L.force_kernel = (kind_flags & MAO_GEMM_FORCE_CTA_PAIR) ? 2 : (kind_flags & MAO_GEMM_FORCE_ONE_CTA) ? 1 : 0;
   L.kernel_id = MAO_K_GEMM_TEST;
   for (int b = 0; b < batch; ++b) {
     const size_t ao = (size_t)b * M * K, bo = (size_t)b * N * K;

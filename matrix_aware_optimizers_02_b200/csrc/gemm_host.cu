@@ -210,7 +210,8 @@ mao_status table_add(TableLaunch& L, MapSet& maps, const Split3& A, const Split3
   for (int q = 0; q < L.pb; ++q)
     if (B.p[q] == nullptr) return MAO_ERR_INVALID_ARG;
   // operand views: inner extent = the stored matrix's columns, rows = its rows
-  const int abox = L.a_mn ? 64 : 128, bbox = L.b_mn ? 64 : 128;
+  // B boxes are 64 rows in both majors: a CTA pair loads half of a 128-column B tile each
+  const int abox = L.a_mn ? 64 : 128, bbox = 64;
   int idx[6];
   for (int q = 0; q < 3; ++q) {
     idx[q] = q < L.pa ? maps.get(A.p[q], A.cols, A.rows, A.ld, abox, L.a_mn) : -1;
@@ -268,7 +269,7 @@ StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off) {
   S.probs_off = A.take(sizeof(GemmProblem) * S.nprob, 64);
   GemmProblem* hp = A.hptr<GemmProblem>(S.probs_off);
   const CUtensorMap* mbase = A.dptr<const CUtensorMap>(maps_off);
-  int t = 0;
+  int t = 0, t2 = 0;
   for (int i = 0; i < S.nprob; ++i) {
     GemmProblem P = L.probs[i];
     for (int q = 0; q < 3; ++q) {
@@ -278,12 +279,21 @@ StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off) {
     }
     P.tile_begin = t;
     t += ((P.M + 127) / 128) * P.tiles_n;
+    P.tile_begin2 = t2;
+    t2 += ((P.M + 255) / 256) * P.tiles_n;
     // work recorded for the profiler: only problems that always run (a problem gated
     // by a device flag may be skipped, so it counts nothing: a lower bound)
     if (P.flag == nullptr) S.flops += 2.0 * P.M * (double)P.N * P.K;
     hp[i] = P;
   }
   S.total_tiles = t;
+  S.total_tiles2 = t2;
+  // the CTA-pair kernel when its 256-row tiles fill the GPU's pairs and waste at most
+  // a fifth of the rows (a 128-row remainder of M costs a half tile)
+  // the pair kernel serves operands with a three-plane side (verified bit-for-bit
+  // against the one-CTA kernel); bf16 x bf16 and two-plane products stay on one CTA
+  const bool pair_ok = L.pa == 3 || L.pb == 3;
+  S.pair = pair_ok && (L.force_kernel == 2 || (L.force_kernel == 0 && t2 >= 74 && 2.0 * t2 <= 1.2 * t));
   return S;
 }
 
@@ -292,13 +302,13 @@ mao_status table_launch(const Arena& A, const StagedLaunch& S, DevStatus* status
   GemmTableParams p;
   p.probs = A.dptr<const GemmProblem>(S.probs_off);
   p.nprob = S.nprob;
-  p.total_tiles = S.total_tiles;
+  p.total_tiles = S.pair ? S.total_tiles2 : S.total_tiles;
   p.status = status;
   const int key = S.pa * 10 + S.pb;
   switch (key) {
-    case 33: return launch_table_planes<3, 3>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops);
-    case 31: return launch_table_planes<3, 1>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops);
-    case 13: return launch_table_planes<1, 3>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops);
+    case 33: return launch_table_planes<3, 3>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops, S.pair);
+    case 31: return launch_table_planes<3, 1>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops, S.pair);
+    case 13: return launch_table_planes<1, 3>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops, S.pair);
     case 11: return launch_table_planes<1, 1>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops);
     case 22: return launch_table_planes<2, 2>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops);
     default: return MAO_ERR_INVALID_ARG;

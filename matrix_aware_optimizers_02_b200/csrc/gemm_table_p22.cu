@@ -2,5 +2,5 @@
 #include "gemm_table.cuh"
 
 namespace mao {
-template mao_status launch_table_planes<2, 2>(const GemmTableParams&, int, int, cudaStream_t, int, double);
+template mao_status launch_table_planes<2, 2>(const GemmTableParams&, int, int, cudaStream_t, int, double, bool);
 }  // namespace mao

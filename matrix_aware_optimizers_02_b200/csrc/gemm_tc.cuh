@@ -107,12 +107,13 @@ struct GemmProblem {
   float* out2;
   __nv_bfloat16* out2_p[3];
   int ld_out2, ld_out2p;
+  int tile_begin2;             // first tile in the CTA-pair numbering (256-row tiles)
 };
 
 struct GemmTableParams {
   const GemmProblem* probs;
   int nprob;
-  int total_tiles;
+  int total_tiles;   // 128-row tiles (one CTA each), or 256-row tiles for the CTA-pair kernel
   DevStatus* status;
 };
 
@@ -159,12 +160,15 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int k) {
   }
 }
 
-// Issue the TMA loads of one operand tile (one plane).
-template <int MN_MAJOR, int R, int ESIZE>
+// Issue the TMA loads of one operand tile (one plane).  K-major tiles of R rows
+// are loaded as R / BOXR boxes of BOXR rows (the descriptor's box height); the
+// boxes land back to back, which is the same layout as one R-row box.
+template <int MN_MAJOR, int R, int ESIZE, int BOXR = R>
 __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int k0,
                                              int mn0, int b) {
   if constexpr (!MN_MAJOR) {
-    tma_load_3d(dst, map, bar, k0, mn0, b);
+#pragma unroll
+    for (int i = 0; i < R / BOXR; ++i) tma_load_3d(dst + i * BOXR * 128, map, bar, k0, mn0 + i * BOXR, b);
   } else {
     constexpr int CHUNK = 128 / ESIZE;  // MN elements per 128-byte row
     constexpr int BK = 128 / ESIZE;
@@ -322,14 +326,15 @@ struct TableSource {
   __device__ DevStatus* status() const { return p.status; }
   __device__ void prefetch() const {}
   __device__ TileInfo decode(int tile, int BM, int BN) const {
+    const bool pair = BM == 256;
     int lo = 0, hi = p.nprob - 1;
 #pragma unroll 1
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (p.probs[mid].tile_begin <= tile) lo = mid; else hi = mid - 1;
+      if ((pair ? p.probs[mid].tile_begin2 : p.probs[mid].tile_begin) <= tile) lo = mid; else hi = mid - 1;
     }
     const GemmProblem& P = p.probs[lo];
-    const int r = tile - P.tile_begin;
+    const int r = tile - (pair ? P.tile_begin2 : P.tile_begin);
     TileInfo t;
 #pragma unroll
     for (int q = 0; q < 3; ++q) {
@@ -493,8 +498,8 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
             load_operand<A_MN, BM, Cfg::ESIZE>(st + q * Cfg::A_TILE, t.mapA[q], &full_bar[s], kc, am, t.b);
 #pragma unroll
           for (int q = 0; q < PB; ++q)
-            load_operand<B_MN, BN, Cfg::ESIZE>(st + PA * Cfg::A_TILE + q * Cfg::B_TILE, t.mapB[q], &full_bar[s], kc,
-                                               bn, t.b);
+            load_operand<B_MN, BN, Cfg::ESIZE, (EPI == EPI_TABLE ? 64 : BN)>(
+                st + PA * Cfg::A_TILE + q * Cfg::B_TILE, t.mapB[q], &full_bar[s], kc, bn, t.b);
         }
         if (!ok) break;
       }
@@ -662,6 +667,286 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }
+}
+
+// ------------------------------------------------------------------ CTA-pair kernel body
+// Table mode on a pair of CTAs (cluster of 2): the pair owns 256 x 128 output
+// tiles.  CTA r loads A rows [128 r, +128) and B columns [64 r, +64) of every
+// plane into its own shared memory, with the transfers counted on the first
+// CTA's mbarrier; the first CTA issues tcgen05.mma.cta_group::2 (M = 256,
+// N = 128), which reads both CTAs' tiles and writes each CTA's 128 accumulator
+// rows into that CTA's TMEM; its commits reach both CTAs' barriers.  Each CTA's
+// epilogue folds and stores its own rows and releases the accumulator on the
+// first CTA's barrier.  Per 128 x 128 of output a CTA loads 3/4 of the bytes of
+// the one-CTA kernel, which leaves room for a third pipeline stage.
+template <int A_MN, int B_MN, int PA, int PB>
+struct GemmPairCfg {
+  static constexpr int BM = 128;   // rows per CTA (the pair's tile has 256)
+  static constexpr int BN = 128;   // columns of the pair's tile
+  static constexpr int BNH = 64;   // columns of B loaded by each CTA
+  static constexpr int ESIZE = 2;
+  static constexpr int BK = 64;
+  static constexpr int UMMA_K = 16;
+  static constexpr int A_TILE = BM * 128;
+  static constexpr int B_TILE = BNH * 128;
+  static constexpr int STAGE_BYTES = PA * A_TILE + PB * B_TILE;
+  static constexpr int STAGES_FIT = (216 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+  static constexpr int PMAX = (PA > PB ? PA : PB) - 1;
+  static constexpr bool CORR = (PA > 1 || PB > 1);
+  static constexpr int ACC_COLS = CORR ? 2 * BN : BN;
+  static constexpr int KCH = 4;
+  // the pair allocates all of TMEM, so both CTAs' accumulators start at the same
+  // column (the pair MMA writes one address in both)
+  static constexpr int TMEM_COLS = 512;
+  static constexpr uint32_t IDESC = make_idesc(1u, A_MN, B_MN, 256, BN);
+  static constexpr int THREADS = 192;
+};
+
+template <int A_MN, int B_MN, int PA, int PB>
+__device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
+  using Cfg = GemmPairCfg<A_MN, B_MN, PA, PB>;
+  constexpr int BN = Cfg::BN, BK = Cfg::BK, STAGES = Cfg::STAGES;
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  __shared__ int prod_it_sh, mma_it_sh;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int npairs = gridDim.x >> 1;
+  const int pair_id = blockIdx.x >> 1;
+  DevStatus* status = src.status();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 256);  // both CTAs' epilogue threads (first CTA's barrier)
+    }
+    mbar_init(&drain_bar, 1);
+    abort_sh = 0;
+    prod_it_sh = 0;
+    mma_it_sh = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tmem_alloc_pair(&tmem_base_sh, Cfg::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_sh;
+  volatile int* abort_flag = &abort_sh;
+  const int total = src.total_tiles();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer (both CTAs)
+      int it = 0;
+      for (int tile = pair_id; tile < total; tile += npairs) {
+        const TileInfo t = src.decode(tile, 256, BN);
+        if (!t.valid) continue;
+#pragma unroll
+        for (int q = 0; q < PA; ++q) tensormap_acquire(t.mapA[q]);
+#pragma unroll
+        for (int q = 0; q < PB; ++q) tensormap_acquire(t.mapB[q]);
+        const int nk = (t.K + BK - 1) / BK;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&empty_bar[s], ph ^ 1, status, 11, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * Cfg::STAGE_BYTES;
+          if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * Cfg::STAGE_BYTES);
+          const uint32_t fb = mapa_shared(smem_u32(&full_bar[s]), 0);
+          const int am = t.am + t.m0 + 128 * (int)rank, bn = t.bn + t.n0 + Cfg::BNH * (int)rank;
+          const int kc = t.ko + kb * BK;
+#pragma unroll
+          for (int q = 0; q < PA; ++q) {
+            uint8_t* dst = st + q * Cfg::A_TILE;
+            if constexpr (!A_MN) {
+              tma_load_3d_pair(dst, t.mapA[q], fb, kc, am, 0);
+            } else {
+#pragma unroll
+              for (int c = 0; c < 128 / 64; ++c) tma_load_3d_pair(dst + c * BK * 128, t.mapA[q], fb, am + c * 64, kc, 0);
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < PB; ++q) {
+            uint8_t* dst = st + PA * Cfg::A_TILE + q * Cfg::B_TILE;
+            if constexpr (!B_MN) {
+              tma_load_3d_pair(dst, t.mapB[q], fb, kc, bn, 0);
+            } else {
+              tma_load_3d_pair(dst, t.mapB[q], fb, bn, kc, 0);
+            }
+          }
+        }
+        if (!ok) break;
+      }
+      prod_it_sh = it;
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------------ MMA issuer (first CTA)
+      int it = 0, used = 0;
+      bool ok = true;
+      for (int tile = pair_id; tile < total && ok; tile += npairs) {
+        const TileInfo t = src.decode(tile, 256, BN);
+        if (!t.valid) continue;
+        const int nk = (t.K + BK - 1) / BK;
+        const int nch = (nk + Cfg::KCH - 1) / Cfg::KCH;
+        for (int c = 0; c < nch && ok; ++c) {
+          const int acc = used & 1;
+          const uint32_t aph = (used >> 1) & 1;
+          ++used;
+          if (!mbar_wait(&tempty_bar[acc], aph ^ 1, status, 12, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + acc * Cfg::ACC_COLS;
+          const int kb0 = c * Cfg::KCH;
+          const int kb1 = min(nk, kb0 + Cfg::KCH);
+          for (int kb = kb0; kb < kb1; ++kb, ++it) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            if (!mbar_wait(&full_bar[s], ph, status, 13, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_base = smem_u32(smem + s * Cfg::STAGE_BYTES);
+            const uint32_t b_base = a_base + PA * Cfg::A_TILE;
+#pragma unroll
+            for (int k = 0; k < BK / Cfg::UMMA_K; ++k) {
+              const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
+              constexpr int pa[5] = {1, 0, 2, 0, 1};
+              constexpr int pb[5] = {1, 2, 0, 1, 0};
+              bool first = true;
+#pragma unroll
+              for (int q = 0; q < 5; ++q) {
+                if (pa[q] < PA && pb[q] < PB && pa[q] + pb[q] <= Cfg::PMAX) {
+                  umma_f16_pair(d_tmem + BN, operand_desc<A_MN, 128, 2>(a_base + pa[q] * Cfg::A_TILE, k),
+                                operand_desc<B_MN, Cfg::BNH, 2>(b_base + pb[q] * Cfg::B_TILE, k), Cfg::IDESC,
+                                first ? accum : 1u);
+                  first = false;
+                }
+              }
+              umma_f16_pair(d_tmem, operand_desc<A_MN, 128, 2>(a_base, k), operand_desc<B_MN, Cfg::BNH, 2>(b_base, k),
+                            Cfg::IDESC, accum);
+            }
+            umma_commit_pair(&empty_bar[s], 0x3);
+          }
+          if (!ok) break;
+          umma_commit_pair(&tfull_bar[acc], 0x3);
+        }
+      }
+      mma_it_sh = it;
+      umma_commit_pair(&drain_bar, 0x3);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    const uint32_t tempty_lead[2] = {mapa_shared(smem_u32(&tempty_bar[0]), 0), mapa_shared(smem_u32(&tempty_bar[1]), 0)};
+    int used = 0;
+    bool ok = true;
+    for (int tile = pair_id; tile < total && ok; tile += npairs) {
+      const TileInfo t = src.decode(tile, 256, BN);
+      if (!t.valid) continue;
+      const int row = t.m0 + 128 * (int)rank + row_in_tile;
+      const int ncols = src.cols(t);
+      const int nk = (t.K + BK - 1) / BK;
+      const int nch = (nk + Cfg::KCH - 1) / Cfg::KCH;
+      float run[BN];
+#pragma unroll
+      for (int j = 0; j < BN; ++j) run[j] = 0.0f;
+      for (int c = 0; c < nch; ++c) {
+        const int acc = used & 1;
+        const uint32_t aph = (used >> 1) & 1;
+        ++used;
+        const bool w = mbar_wait(&tfull_bar[acc], aph, status, 14, abort_flag);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS;
+#pragma unroll
+        for (int ch = 0; ch < BN / 32; ++ch) {
+          uint32_t rm[32];
+          tmem_ld_32x32b_x32(tacc + ch * 32, rm);
+          if constexpr (Cfg::CORR) {
+            uint32_t rc[32];
+            tmem_ld_32x32b_x32(tacc + BN + ch * 32, rc);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) run[ch * 32 + j] += __uint_as_float(rm[j]) + __uint_as_float(rc[j]);
+          } else {
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) run[ch * 32 + j] += __uint_as_float(rm[j]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive_cluster(tempty_lead[acc]);
+      }
+      if (!ok) break;
+#pragma unroll
+      for (int ch = 0; ch < BN / 32; ++ch)
+        if (t.n0 + ch * 32 < ncols) src.template epilogue<EPI_TABLE>(t, row, t.n0 + ch * 32, &run[ch * 32]);
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  // MMAs issued by the first CTA write both CTAs' TMEM: each CTA waits for the
+  // first CTA's final commit before releasing TMEM.  After an early exit the first
+  // CTA lets the loads still in flight land (its full barriers count both CTAs'
+  // bytes; neither producer runs more than STAGES loads ahead of the MMAs).
+  if (warp == 1 && lane == 0) mbar_wait(&drain_bar, 0, status, 15, abort_flag, false);
+  __syncthreads();
+  if (leader && warp == 0 && lane == 0) {
+    const int last = max(prod_it_sh, mma_it_sh + (*abort_flag ? STAGES : 0));
+    for (int j = mma_it_sh; j < last; ++j)
+      mbar_wait(&full_bar[j % STAGES], (j / STAGES) & 1, status, 16, abort_flag, false);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+template <int A_MN, int B_MN, int PA, int PB>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    gemm_tc_pair_kernel(const __grid_constant__ GemmTableParams p) {
+  TableSource src(p);
+  gemm_body_pair<A_MN, B_MN, PA, PB>(src);
 }
 
 template <int KIND, int A_MN, int B_MN, int EPI>

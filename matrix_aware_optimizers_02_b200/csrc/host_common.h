@@ -162,6 +162,7 @@ struct Split3 {
 struct TableLaunch {
   int a_mn = 0, b_mn = 0;
   int pa = 3, pb = 3;
+  int force_kernel = 0;  // 0: choose, 1: one-CTA kernel, 2: CTA-pair kernel (verification)
   int kernel_id = 0;
   std::vector<GemmProblem> probs;
   std::vector<int> map_idx;  // 6 per problem: A planes 0..2, B planes 0..2 (indices into the step's map list)
@@ -213,6 +214,8 @@ struct StagedLaunch {
   int total_tiles = 0;
   int a_mn = 0, b_mn = 0, kernel_id = 0;
   int pa = 3, pb = 3;
+  int total_tiles2 = 0;  // 256-row tiles (CTA-pair kernel)
+  bool pair = false;     // launch the CTA-pair kernel
   double flops = 0.0;
 };
 StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off);
@@ -221,6 +224,6 @@ mao_status table_launch(const Arena& A, const StagedLaunch& S, DevStatus* status
 // One table-mode launch for a plane pair (instantiated in gemm_table_p*.cu).
 template <int PA, int PB>
 mao_status launch_table_planes(const GemmTableParams& p, int a_mn, int b_mn, cudaStream_t stream, int kernel_id,
-                               double flops);
+                               double flops, bool pair = false);
 
 }  // namespace mao

@@ -100,3 +100,30 @@ def test_split2_has_sixteen_bit_products(api, shape):
     scale = torch.bmm(A.double().abs(), B.double().abs().transpose(1, 2))
     rel = ((D.double() - ref).abs() / scale).max().item()
     assert rel < 2.0 ** -15, rel
+
+
+PAIR_SHAPES = [(1, 256, 128, 64), (3, 200, 328, 136), (2, 384, 520, 1000), (1, 8, 8, 8), (5, 640, 256, 512)]
+
+
+@pytest.mark.parametrize("kernel", ["one_cta", "cta_pair"])
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("shape", PAIR_SHAPES)
+@pytest.mark.parametrize("kind,adt,bdt", [("split3", torch.float32, torch.float32)] + MIXED[1:])
+def test_table_kernels_agree(api, kind, adt, bdt, shape, a_mn, b_mn, kernel):
+    """Both table-mode kernels (128 x 128 tiles on one CTA; 256 x 128 tiles on a CTA
+    pair sharing tcgen05 cta_group::2) reach the fp32 accumulation level, and give
+    the same bits."""
+    batch, M, N, K = shape
+    gen = torch.Generator(device="cuda").manual_seed(11)
+    A = torch.randn((batch, M, K), generator=gen, device="cuda").to(adt)
+    B = torch.randn((batch, N, K), generator=gen, device="cuda").to(bdt)
+    Ain = A.transpose(1, 2).contiguous() if a_mn else A
+    Bin = B.transpose(1, 2).contiguous() if b_mn else B
+    D = api.gemm(Ain, Bin, kind=kind, a_mn_major=bool(a_mn), b_mn_major=bool(b_mn), kernel=kernel)
+    ref = torch.bmm(A.double(), B.double().transpose(1, 2))
+    scale = torch.bmm(A.double().abs(), B.double().abs().transpose(1, 2))
+    rel = ((D.double() - ref).abs() / scale).max().item()
+    assert rel < 4 * 2.0 ** -24 * K ** 0.5, rel
+    other = api.gemm(Ain, Bin, kind=kind, a_mn_major=bool(a_mn), b_mn_major=bool(b_mn),
+                     kernel="cta_pair" if kernel == "one_cta" else "one_cta")
+    assert torch.equal(D, other)
