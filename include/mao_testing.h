@@ -56,6 +56,15 @@ typedef enum {
  * aligned (holds the device status word and, for SPLIT3, the split operands and
  * the problem descriptors).
  */
+/*
+ * Kernel choice for every table-mode product of this process (verification of
+ * the optimizer steps on each kernel): 0 = the library's choice (default),
+ * 1 = the one-CTA kernel always, 2 = the CTA-pair kernel wherever it applies
+ * (a three-plane operand), whatever the launch's size.  Affects only calls made
+ * after it returns; not thread-safe with concurrent steps.
+ */
+MAO_API mao_status mao_test_set_table_kernel(int32_t policy);
+
 MAO_API mao_status mao_test_gemm_workspace_size(int32_t kind, int32_t batch, int32_t M, int32_t N, int32_t K,
                                         size_t* bytes);
 MAO_API mao_status mao_test_gemm(int32_t kind, int32_t a_mn_major, int32_t b_mn_major, const void* A, const void* B,

@@ -162,6 +162,14 @@ def gemm(A: torch.Tensor, B: torch.Tensor, *, kind: str = "bf16", a_mn_major: bo
     return D
 
 
+def set_table_kernel(kernel: str = "auto") -> None:
+    """Verification switch: run every fp32-faithful table-mode product of this process on
+    the library's choice ("auto"), the one-CTA kernel ("one_cta") or the CTA-pair kernel
+    wherever it applies ("cta_pair")."""
+    L.check(L.load().mao_test_set_table_kernel({"auto": 0, "one_cta": 1, "cta_pair": 2}[kernel]),
+            "mao_test_set_table_kernel")
+
+
 def _refresh(kind: str, k: int, pf: int, tol: float, sort: bool) -> "L.Refresh":
     kinds = {"every_k": L.REFRESH_EVERY_K, "adaptive": L.REFRESH_ADAPTIVE, "never": L.REFRESH_NEVER}
     if kind not in kinds:

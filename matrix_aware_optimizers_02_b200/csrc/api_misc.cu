@@ -97,6 +97,8 @@ mao_status gemm_layout(int32_t kind_flags, int32_t batch, int32_t M, int32_t N, 
 
 }  // namespace
 
+extern "C" mao_status mao_test_set_table_kernel(int32_t policy) { return set_table_kernel_policy(policy); }
+
 extern "C" mao_status mao_test_gemm_workspace_size(int32_t kind, int32_t batch, int32_t M, int32_t N, int32_t K,
                                                    size_t* bytes) {
   if (bytes == nullptr) return MAO_ERR_INVALID_ARG;

@@ -3,6 +3,8 @@
 // three bf16 planes split used by the fp32-faithful (SPLIT3) products.
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "host_common.h"
 
 namespace mao {
@@ -243,6 +245,16 @@ mao_status table_add(TableLaunch& L, MapSet& maps, const Split3& A, const Split3
   return MAO_OK;
 }
 
+namespace {
+std::atomic<int> g_table_policy{0};
+}
+int table_kernel_policy() { return g_table_policy.load(std::memory_order_relaxed); }
+mao_status set_table_kernel_policy(int policy) {
+  if (policy < 0 || policy > 2) return MAO_ERR_INVALID_ARG;
+  g_table_policy.store(policy, std::memory_order_relaxed);
+  return MAO_OK;
+}
+
 mao_status table_set_alt(TableLaunch& L, const int* sel, float* out2, const Split3* out2p, int ld_out2) {
   if (L.probs.empty() || sel == nullptr) return MAO_ERR_INVALID_ARG;
   GemmProblem& P = L.probs.back();
@@ -293,7 +305,8 @@ StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off) {
   // the pair kernel serves operands with a three-plane side (verified bit-for-bit
   // against the one-CTA kernel); bf16 x bf16 and two-plane products stay on one CTA
   const bool pair_ok = L.pa == 3 || L.pb == 3;
-  S.pair = pair_ok && (L.force_kernel == 2 || (L.force_kernel == 0 && t2 >= 74 && 2.0 * t2 <= 1.2 * t));
+  const int force = L.force_kernel ? L.force_kernel : table_kernel_policy();
+  S.pair = pair_ok && (force == 2 || (force == 0 && t2 >= 74 && 2.0 * t2 <= 1.2 * t));
   return S;
 }
 
