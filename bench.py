@@ -226,14 +226,15 @@ def fold_traffic(args):
                               "foam_tau_kernel", "foam_n_kernel"],
            "pc_sort": ["pc_keys_kernel", "pc_argsort_kernel", "pc_gather_cols_kernel", "soap_vperm_kernel"],
            "pc_check": ["pc_check_kernel"], "pc_chol": ["qr_chol_kernel"], "pc_qr_reduce": ["pc_coef_reduce_kernel"],
-           "pc_stats": ["pc_stats_kernel"], "pc_panel": ["gemm_tc_table_kernel", "qr_gram_reduce_kernel"]}
+           "pc_stats": ["pc_stats_kernel"],
+           "pc_panel": ["gemm_tc_table_kernel", "gemm_tc_pair_kernel", "qr_gram_reduce_kernel"]}
     names = {}
     for r in rows:
         if head is not None and len(r) == len(head) and "Kernel Name" not in r:
             d = dict(zip(head, r))
             names[int(d["ID"])] = d["Kernel Name"].split("(")[0].split("<")[0].split()[-1]
     for rec, i in zip(launches, tail):
-        ok = fam.get(rec["kernel"], ["gemm_tc_table_kernel", "gemm_tc_kernel"])
+        ok = fam.get(rec["kernel"], ["gemm_tc_table_kernel", "gemm_tc_pair_kernel", "gemm_tc_kernel"])
         if names[i] not in ok:
             raise SystemExit(f"launch {i}: ncu saw {names[i]}, the log says {rec['kernel']}: not aligned")
     agg = {}

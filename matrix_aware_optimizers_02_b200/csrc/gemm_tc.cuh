@@ -35,8 +35,8 @@
 //           five cross products whose size reaches the fp32 unit roundoff
 //           (x1y1, x0y2, x2y0, x0y1, x1y0) in a second one, so the large running
 //           sum is rounded once per k-step only.  The tensor core's accumulation
-//           truncates, so its error grows with every add: TMEM accumulates 64 of K
-//           at a time (256 for bf16 x bf16) and the epilogue warps fold those
+//           truncates, so its error grows with every add: TMEM accumulates 128 of
+//           K at a time (256 for bf16 x bf16) and the epilogue warps fold those
 //           partial sums (main + correction) into fp32 registers with
 //           round-to-nearest.  Same MMA count per K as a three-pass tf32 scheme,
 //           with fp32-level accuracy.
@@ -139,10 +139,11 @@ struct GemmCfg {
   static constexpr bool CORR = (PA > 1 || PB > 1);       // any cross product
   static constexpr int ACC_COLS = CORR ? 2 * BN : BN;    // main (+ correction) accumulator
   // SPLIT3: k-blocks per TMEM accumulation item.  The tensor core's accumulation
-  // truncates; products with a three-plane operand fold every k-block (4 truncating
-  // adds of 16 of K), bf16 x bf16 every 4 (its MMAs are too short to hide a fold
-  // per k-block).
-  static constexpr int KCH = CORR ? 1 : 4;
+  // truncates; products with a three-plane operand fold every 2 k-blocks (8
+  // truncating adds of 16 of K: within twice an fp32 evaluation's error, where
+  // 16 adds were not), bf16 x bf16 every 4.  A fold per k-block costs 8 % of the
+  // SOAP step: the epilogue's TMEM reads then no longer hide behind the MMAs.
+  static constexpr int KCH = CORR ? 2 : 4;
   static constexpr int TMEM_COLS = 2 * ACC_COLS;         // double-buffered
   static constexpr uint32_t IDESC = make_idesc(1u, A_MN, B_MN, BM, BN);
   static constexpr int THREADS = 192;
@@ -701,7 +702,7 @@ struct GemmPairCfg {
   static constexpr int PMAX = (PA > PB ? PA : PB) - 1;
   static constexpr bool CORR = (PA > 1 || PB > 1);
   static constexpr int ACC_COLS = CORR ? 2 * BN : BN;
-  static constexpr int KCH = CORR ? 1 : 4;  // as in the one-CTA kernel
+  static constexpr int KCH = CORR ? 2 : 4;  // as in the one-CTA kernel
   // the pair allocates all of TMEM, so both CTAs' accumulators start at the same
   // column (the pair MMA writes one address in both)
   static constexpr int TMEM_COLS = 512;
