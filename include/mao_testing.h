@@ -25,9 +25,9 @@ typedef enum {
 
 /* Flags OR-ed into a table-mode kind (all but MAO_GEMM_BF16): run the problems
  * on the one-CTA kernel (128 x 128 tiles) or on the CTA-pair kernel (256 x 128
- * tiles, tcgen05 cta_group::2; kinds with a three-plane operand only, else
- * MAO_ERR_UNSUPPORTED); without a flag the library chooses as it does inside the
- * optimizer steps. */
+ * tiles, tcgen05 cta_group::2); without a flag the library chooses as it does
+ * inside the optimizer steps (the pair kernel for products with a three-plane
+ * operand whose 256-row tiles fill the GPU). */
 #define MAO_GEMM_FORCE_ONE_CTA 16
 #define MAO_GEMM_FORCE_CTA_PAIR 32
 
@@ -59,8 +59,8 @@ typedef enum {
 /*
  * Kernel choice for every table-mode product of this process (verification of
  * the optimizer steps on each kernel): 0 = the library's choice (default),
- * 1 = the one-CTA kernel always, 2 = the CTA-pair kernel wherever it applies
- * (a three-plane operand), whatever the launch's size.  Affects only calls made
+ * 1 = the one-CTA kernel always, 2 = the CTA-pair kernel always, whatever the
+ * launch's size or plane counts.  Affects only calls made
  * after it returns; not thread-safe with concurrent steps.
  */
 MAO_API mao_status mao_test_set_table_kernel(int32_t policy);

@@ -80,8 +80,6 @@ mao_status gemm_layout(int32_t kind_flags, int32_t batch, int32_t M, int32_t N, 
   if ((kind_flags & ~(15 | MAO_GEMM_FORCE_ONE_CTA | MAO_GEMM_FORCE_CTA_PAIR)) != 0) return MAO_ERR_INVALID_ARG;
   if (kind < MAO_GEMM_BF16 || kind > MAO_GEMM_SPLIT2) return MAO_ERR_INVALID_ARG;
   if (kind == MAO_GEMM_BF16 && (kind_flags & ~15)) return MAO_ERR_INVALID_ARG;
-  if ((kind_flags & MAO_GEMM_FORCE_CTA_PAIR) && (kind == MAO_GEMM_BF16_FOLD || kind == MAO_GEMM_SPLIT2))
-    return MAO_ERR_UNSUPPORTED;
   Carver cv;
   cv.take(kStatusBytes);
   if (kind != MAO_GEMM_BF16) {

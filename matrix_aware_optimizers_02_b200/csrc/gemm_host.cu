@@ -301,12 +301,13 @@ StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off) {
   S.total_tiles = t;
   S.total_tiles2 = t2;
   // the CTA-pair kernel when its 256-row tiles fill the GPU's pairs and waste at most
-  // a fifth of the rows (a 128-row remainder of M costs a half tile)
-  // the pair kernel serves operands with a three-plane side (verified bit-for-bit
-  // against the one-CTA kernel); bf16 x bf16 and two-plane products stay on one CTA
-  const bool pair_ok = L.pa == 3 || L.pb == 3;
+  // a fifth of the rows (a 128-row remainder of M costs a half tile).  The library
+  // chooses it for products with a three-plane operand, where it relieves the
+  // shared-memory operand stream; bf16 x bf16 products are bound by their epilogue
+  // and stay on one CTA unless a caller forces the pair kernel.
+  const bool pair_auto = L.pa == 3 || L.pb == 3;
   const int force = L.force_kernel ? L.force_kernel : table_kernel_policy();
-  S.pair = pair_ok && (force == 2 || (force == 0 && t2 >= 74 && 2.0 * t2 <= 1.2 * t));
+  S.pair = force == 2 || (force == 0 && pair_auto && t2 >= 74 && 2.0 * t2 <= 1.2 * t);
   return S;
 }
 
@@ -322,8 +323,8 @@ mao_status table_launch(const Arena& A, const StagedLaunch& S, DevStatus* status
     case 33: return launch_table_planes<3, 3>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops, S.pair);
     case 31: return launch_table_planes<3, 1>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops, S.pair);
     case 13: return launch_table_planes<1, 3>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops, S.pair);
-    case 11: return launch_table_planes<1, 1>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops);
-    case 22: return launch_table_planes<2, 2>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops);
+    case 11: return launch_table_planes<1, 1>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops, S.pair);
+    case 22: return launch_table_planes<2, 2>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops, S.pair);
     default: return MAO_ERR_INVALID_ARG;
   }
 }

@@ -228,6 +228,6 @@ mao_status table_launch(const Arena& A, const StagedLaunch& S, DevStatus* status
 // One table-mode launch for a plane pair (instantiated in gemm_table_p*.cu).
 template <int PA, int PB>
 mao_status launch_table_planes(const GemmTableParams& p, int a_mn, int b_mn, cudaStream_t stream, int kernel_id,
-                               double flops, bool pair = false);
+                               double flops, bool pair);
 
 }  // namespace mao

@@ -156,6 +156,7 @@ def test_precond_workspace_size_is_independent_of_t(lib, kind, k, pf):
 def test_pair_kernel_flag_validation(lib):
     b = ctypes.c_size_t(0)
     assert lib.mao_test_gemm_workspace_size(1 | 32, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_OK
-    assert lib.mao_test_gemm_workspace_size(2 | 32, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_ERR_UNSUPPORTED
+    assert lib.mao_test_gemm_workspace_size(2 | 32, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_OK
+    assert lib.mao_test_gemm_workspace_size(5 | 32, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_OK
     assert lib.mao_test_gemm_workspace_size(0 | 16, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_ERR_INVALID_ARG
     assert lib.mao_test_gemm_workspace_size(1 | 64, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_ERR_INVALID_ARG
