@@ -57,6 +57,10 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--optimizers", default="muon,soap,foam", help="comma list of muon, soap, foam")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--soap-k", type=int, default=1, help="SOAP refreshes its bases every k steps")
+    ap.add_argument("--foam-kinds", type=int, default=0,
+                    help="instead of the bench line: FOAM alone for steps t = 1..N, each timed on its own, "
+                         "and the median ms of plain, check-only and check+refresh steps")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
     ap.add_argument("--launch-log", default=None,
                     help="after the measurement, run one more step and write its launch list (kernel, work) here")
@@ -329,7 +333,7 @@ class LayerSet:
     """W, G and the optimizer states of one synthetic layer set, plus one batch
     object per optimizer (sharing W, G and one workspace)."""
 
-    def __init__(self, specs, seed, dev, g_bf16, optimizers, norm):
+    def __init__(self, specs, seed, dev, g_bf16, optimizers, norm, soap_k=1):
         import torch
 
         from matrix_aware_optimizers_02_b200 import api, synth
@@ -352,7 +356,7 @@ class LayerSet:
                              "L": torch.eye(m, device=dev) * 1e-6, "R": torch.eye(n, device=dev) * 1e-6,
                              "QL": torch.eye(m, device=dev), "QR": torch.eye(n, device=dev)})
             self.batches["soap"] = api.SoapBatch(mats, beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3,
-                                                 refresh="every_k", k=1, with_stats=True, allocate=False)
+                                                 refresh="every_k", k=soap_k, with_stats=True, allocate=False)
         if "foam" in optimizers:
             mats = []
             for w, g in zip(self.W, self.G):
@@ -403,7 +407,7 @@ def run_mine(args, rank, world, dist):
     specs = specs_for(args.workload, args.seed)
     optimizers = [o.strip() for o in args.optimizers.split(",") if o.strip()]
     norm = MUON_NORM.get(args.workload, "none")
-    LS = LayerSet(specs, args.seed + 7919 * rank, dev, g_bf16, optimizers, norm)
+    LS = LayerSet(specs, args.seed + 7919 * rank, dev, g_bf16, optimizers, norm, soap_k=args.soap_k)
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -568,7 +572,9 @@ def run_mine(args, rank, world, dist):
         "config": {"workload": args.workload, "description": desc, "optimizers": LS.order,
                    "optimizer_ms": opt_ms,
                    "muon": {"mu": 0.95, "lr": 0.02, "ns_steps": 5, "norm": norm},
-                   "soap": {"beta1": 0.95, "beta2": 0.95, "eps": 1e-8, "refresh": "every step, sorted"},
+                   "soap": {"beta1": 0.95, "beta2": 0.95, "eps": 1e-8,
+                            "refresh": "every step, sorted" if args.soap_k == 1 else
+                            f"every {args.soap_k} steps, sorted"},
                    "foam": {"beta1": 0.95, "beta2": 0.95, "eps": 1e-8, "refresh": "adaptive pf=10 tol=0.1"},
                    "timed_steps_t": [args.warmup + 2, args.warmup + 1 + args.steps],
                    "matrices_per_rank": len(specs), "elements_per_rank": n_elems,
@@ -582,6 +588,45 @@ def run_mine(args, rank, world, dist):
         "clocks": clk,
     }
     return line
+
+
+def run_foam_kinds(args):
+    """FOAM alone on the workload for t = 1..N (adaptive, pf = 10, tol = 0.1, a fresh
+    gradient each step), each step bracketed by its own events and followed by a read
+    of the per-matrix refresh flags:
+    a step is plain ((t - 1) mod pf != 0), check-only (a check step where no matrix
+    refreshed) or check+refresh.  Returns one JSON object with the median of each kind."""
+    import torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    desc, g_bf16 = WORKLOADS[args.workload]
+    specs = specs_for(args.workload, args.seed)
+    LS = LayerSet(specs, args.seed, dev, g_bf16, ["foam"], "none")
+    b = LS.batches["foam"]
+    stream = torch.cuda.current_stream()
+    kinds = {"plain": [], "check": [], "check+refresh": []}
+    per_t = []
+    gen = torch.Generator(device=dev).manual_seed(args.seed + 1)
+    for t in range(1, args.foam_kinds + 1):
+        for g, sp in zip(LS.G, specs):  # a fresh gradient each step, outside the timed region
+            g.normal_(0.0, sp.g_std * sp.g_scale, generator=gen)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        b(t)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+        nref = sum(1 for r in b.stats_dict()["refreshed"] if r & 1)
+        kind = "plain" if (t - 1) % 10 else ("check+refresh" if nref else "check")
+        kinds[kind].append(ms)
+        per_t.append({"t": t, "kind": kind, "ms": round(ms, 3), "refreshed": nref})
+    if LS.status():
+        raise RuntimeError(f"device status {LS.status()}")
+    return {"metric": "FOAM step ms by step kind", "unit": "ms", "workload": args.workload, "description": desc,
+            "steps": args.foam_kinds, "median_ms": {k: (round(statistics.median(v), 3) if v else None)
+                                                    for k, v in kinds.items()},
+            "per_step": per_t, "note": "t = 1 includes first-touch costs; medians over the rest of each kind"}
 
 
 def run_reference(args, rank, world):
@@ -618,6 +663,9 @@ def main():
         return 0
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.foam_kinds > 0:
+        print(json.dumps(run_foam_kinds(args)), flush=True)
+        return 0
     if args.impl == "reference":
         line = run_reference(args, rank, world)
         if line is not None:
