@@ -328,6 +328,26 @@ def cpu_oracle_sample(workload, budget_s, seed, optimizers, t_foam=1):
     return total_ms, cores, sample
 
 
+# ----------------------------------------------------------------------------- ranks
+def rank_seed(seed, rank):
+    """Each rank owns its own synthetic layer set (weak scaling, no data-path collective)."""
+    return seed + 7919 * rank
+
+
+def reduce_times(values, dist, device):
+    """Max over ranks of each per-rank duration: the slowest rank bounds the job."""
+    import torch
+    tt = torch.tensor(list(values), device=device, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return tt.tolist()
+
+
+def per_layer_set(ms_max, world):
+    """ms per layer set for the whole job: `world` layer sets processed in ms_max."""
+    return ms_max / world
+
+
 # ----------------------------------------------------------------------------- the layer set on the GPU
 class LayerSet:
     """W, G and the optimizer states of one synthetic layer set, plus one batch
@@ -407,7 +427,7 @@ def run_mine(args, rank, world, dist):
     specs = specs_for(args.workload, args.seed)
     optimizers = [o.strip() for o in args.optimizers.split(",") if o.strip()]
     norm = MUON_NORM.get(args.workload, "none")
-    LS = LayerSet(specs, args.seed + 7919 * rank, dev, g_bf16, optimizers, norm, soap_k=args.soap_k)
+    LS = LayerSet(specs, rank_seed(args.seed, rank), dev, g_bf16, optimizers, norm, soap_k=args.soap_k)
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -501,10 +521,7 @@ def run_mine(args, rank, world, dist):
     if args.launch_log and rank == 0:
         write_launch_log(args, lib, L, LS, t + 1, stream)
 
-    tt = torch.tensor([ms, e2e_ms], device=dev)
-    if dist is not None:
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    ms_max, e2e_max = tt.tolist()
+    ms_max, e2e_max = reduce_times([ms, e2e_ms], dist, dev)
     if rank != 0:
         return None
 
@@ -557,7 +574,7 @@ def run_mine(args, rank, world, dist):
     n_elems = sum(s.m * s.n for s in specs)
     line = {
         "metric": "Muon/SOAP/FOAM step ms per layer set; % of tensor-core peak and HBM GB/s",
-        "value": round(ms_max / world, 4),
+        "value": round(per_layer_set(ms_max, world), 4),
         "unit": "ms",
         "n_gpus": world,
         "steps": args.steps,
@@ -582,7 +599,7 @@ def run_mine(args, rank, world, dist):
         "roofline": roof,
         "kernels": kernels,
         "cpu_baseline": cpu,
-        "e2e": {"value": round(e2e_max / world, 4), "unit": "ms", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": round(per_layer_set(e2e_max, world), 4), "unit": "ms", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": int(n_launch),
         "clocks": clk,
