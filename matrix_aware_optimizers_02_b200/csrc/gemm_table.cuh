@@ -31,7 +31,7 @@ mao_status launch_table_majors(const GemmTableParams& p, cudaStream_t stream, in
   // tensor-core products per multiply-add: pairs (i, j), i < PA, j < PB, i + j <= max(PA, PB) - 1
   constexpr int kProducts = (PA == 3 && PB == 3) ? 6 : (PA == 1 && PB == 1) ? 1 : 3;
   LaunchScope ls(stream, kernel_id, flops, 0.0, flops * kProducts);
-  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(p);
+  kern<<<grid, Cfg::TABLE_THREADS, Cfg::SMEM_BYTES, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? MAO_OK : MAO_ERR_CUDA;
 }
 

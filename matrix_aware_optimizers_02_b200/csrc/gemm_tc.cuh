@@ -147,6 +147,7 @@ struct GemmCfg {
   static constexpr int TMEM_COLS = 2 * ACC_COLS;         // double-buffered
   static constexpr uint32_t IDESC = make_idesc(1u, A_MN, B_MN, BM, BN);
   static constexpr int THREADS = 192;
+  static constexpr int TABLE_THREADS = 320;  // table mode: 8 epilogue warps
 };
 
 // Descriptor of one operand tile (rows = MN extent R, K extent = BK) at smem
@@ -427,6 +428,11 @@ template <int KIND, int A_MN, int B_MN, int EPI, class Src, int PA = (KIND == OP
 __device__ __forceinline__ void gemm_body(const Src& src) {
   using Cfg = GemmCfg<KIND, A_MN, B_MN, PA, PB>;
   constexpr int BM = Cfg::BM, BN = Cfg::BN, BK = Cfg::BK, STAGES = Cfg::STAGES;
+  // Table mode runs 8 epilogue warps, two per TMEM lane quarter, each taking half of
+  // the tile's columns: twice the memory operations in flight for its fp32 and
+  // plane stores, and half the fold registers per thread.
+  constexpr int EPI_WARPS = (EPI == EPI_TABLE) ? 8 : 4;
+  constexpr int COLS = BN * 4 / EPI_WARPS;  // columns per epilogue warp
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
@@ -452,7 +458,7 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 128);
+      mbar_init(&tempty_bar[a], 32 * EPI_WARPS);
     }
     mbar_init(&drain_bar, 1);
     abort_sh = 0;
@@ -583,7 +589,8 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    const int q = warp & 3;
+    const int q = warp & 3;                 // TMEM lane quarter this warp may read
+    const int cb = ((warp - 2) >> 2) * COLS;  // first column of this warp's share
     const int row_in_tile = q * 32 + lane;
     int used = 0;
     bool ok = true;
@@ -619,9 +626,9 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
         // fold the K-chunk accumulators (main + correction) into fp32 registers
         const int nk = (t.K + BK - 1) / BK;
         const int nch = (nk + Cfg::KCH - 1) / Cfg::KCH;
-        float run[BN];
+        float run[COLS];
 #pragma unroll
-        for (int j = 0; j < BN; ++j) run[j] = 0.0f;
+        for (int j = 0; j < COLS; ++j) run[j] = 0.0f;
         for (int c = 0; c < nch; ++c) {
           const int acc = used & 1;
           const uint32_t aph = (used >> 1) & 1;
@@ -632,9 +639,9 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
             break;
           }
           tc_fence_after();
-          const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS;
+          const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS + cb;
 #pragma unroll
-          for (int ch = 0; ch < BN / 32; ++ch) {
+          for (int ch = 0; ch < COLS / 32; ++ch) {
             uint32_t rm[32];
             tmem_ld_32x32b_x32(tacc + ch * 32, rm);
             if constexpr (Cfg::CORR) {
@@ -654,8 +661,8 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
         }
         if (!ok) break;
 #pragma unroll
-        for (int ch = 0; ch < BN / 32; ++ch)
-          if (t.n0 + ch * 32 < ncols) src.template epilogue<EPI>(t, row, t.n0 + ch * 32, &run[ch * 32]);
+        for (int ch = 0; ch < COLS / 32; ++ch)
+          if (t.n0 + cb + ch * 32 < ncols) src.template epilogue<EPI>(t, row, t.n0 + cb + ch * 32, &run[ch * 32]);
       }
     }
   }
@@ -707,7 +714,9 @@ struct GemmPairCfg {
   // column (the pair MMA writes one address in both)
   static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t IDESC = make_idesc(1u, A_MN, B_MN, 256, BN);
-  static constexpr int THREADS = 192;
+  static constexpr int EPI_WARPS = 8;  // two per TMEM lane quarter, half of the columns each
+  static constexpr int COLS = BN / 2;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
 };
 
 template <int A_MN, int B_MN, int PA, int PB>
@@ -743,7 +752,7 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 256);  // both CTAs' epilogue threads (first CTA's barrier)
+      mbar_init(&tempty_bar[a], 2 * 32 * Cfg::EPI_WARPS);  // both CTAs' epilogue threads (first CTA's barrier)
     }
     mbar_init(&drain_bar, 1);
     abort_sh = 0;
@@ -874,7 +883,9 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
     }
   } else {
     // -------------------------------------------------------------- epilogue (both CTAs)
+    constexpr int COLS = Cfg::COLS;
     const int q = warp & 3;
+    const int cb = ((warp - 2) >> 2) * COLS;
     const int row_in_tile = q * 32 + lane;
     const uint32_t tempty_lead[2] = {mapa_shared(smem_u32(&tempty_bar[0]), 0), mapa_shared(smem_u32(&tempty_bar[1]), 0)};
     int used = 0;
@@ -886,9 +897,9 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
       const int ncols = src.cols(t);
       const int nk = (t.K + BK - 1) / BK;
       const int nch = (nk + Cfg::KCH - 1) / Cfg::KCH;
-      float run[BN];
+      float run[COLS];
 #pragma unroll
-      for (int j = 0; j < BN; ++j) run[j] = 0.0f;
+      for (int j = 0; j < COLS; ++j) run[j] = 0.0f;
       for (int c = 0; c < nch; ++c) {
         const int acc = used & 1;
         const uint32_t aph = (used >> 1) & 1;
@@ -899,9 +910,9 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
           break;
         }
         tc_fence_after();
-        const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS;
+        const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS + cb;
 #pragma unroll
-        for (int ch = 0; ch < BN / 32; ++ch) {
+        for (int ch = 0; ch < COLS / 32; ++ch) {
           uint32_t rm[32];
           tmem_ld_32x32b_x32(tacc + ch * 32, rm);
           if constexpr (Cfg::CORR) {
@@ -921,8 +932,9 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
       }
       if (!ok) break;
 #pragma unroll
-      for (int ch = 0; ch < BN / 32; ++ch)
-        if (t.n0 + ch * 32 < ncols) src.template epilogue<EPI_TABLE>(t, row, t.n0 + ch * 32, &run[ch * 32]);
+      for (int ch = 0; ch < COLS / 32; ++ch)
+        if (t.n0 + cb + ch * 32 < ncols)
+          src.template epilogue<EPI_TABLE>(t, row, t.n0 + cb + ch * 32, &run[ch * 32]);
     }
   }
 
@@ -949,7 +961,7 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
 }
 
 template <int A_MN, int B_MN, int PA, int PB>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     gemm_tc_pair_kernel(const __grid_constant__ GemmTableParams p) {
   TableSource src(p);
   gemm_body_pair<A_MN, B_MN, PA, PB>(src);
@@ -962,7 +974,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
 }
 
 template <int A_MN, int B_MN, int PA, int PB>
-__global__ void __launch_bounds__(192, 1) gemm_tc_table_kernel(const __grid_constant__ GemmTableParams p) {
+__global__ void __launch_bounds__(320, 1) gemm_tc_table_kernel(const __grid_constant__ GemmTableParams p) {
   TableSource src(p);
   gemm_body<OP_SPLIT3, A_MN, B_MN, EPI_TABLE, TableSource, PA, PB>(src);
 }
