@@ -17,14 +17,15 @@
 //               fp32-faithful product.  A problem can be gated by a device flag
 //               (skipped when the flag is 0) for data-dependent work.
 //
-// Warp roles (192 threads):
+// Warp roles (192 threads; 320 in table mode, with warps 2..9 in the epilogue):
 //   warp 0      TMA producer (one elected lane): fills a STAGES-deep ring of
 //               A/B tiles in shared memory, 128-byte swizzled.
 //   warp 1      TMEM owner + MMA issuer (one elected lane): tcgen05.mma into one
 //               of two TMEM accumulators (BN fp32 columns each); commits free the
 //               smem slots and hand finished accumulators to the epilogue.
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//               lanes 32*(w%4)..+31 = tile rows), fused arithmetic, stores.
+//               lanes 32*(w%4)..+31 = tile rows), fused arithmetic, stores; in
+//               table mode two warps share each lane quarter, half the columns each.
 // The two accumulators let the epilogue of tile i overlap the MMAs of tile i+1.
 //
 // Operand kinds:
