@@ -145,6 +145,16 @@ def gemm(A: torch.Tensor, B: torch.Tensor, *, kind: str = "bf16", a_mn_major: bo
     """
     lib = L.load()
     k = {"bf16": 0, "split3": 1, "bf16_fold": 2, "split3_bf16": 3, "bf16_split3": 4, "split2": 5}[kind]
+    a_dt, b_dt = {"bf16": ("bf16", "bf16"), "split3": ("f32", "f32"), "bf16_fold": ("bf16", "bf16"),
+                  "split3_bf16": ("f32", "bf16"), "bf16_split3": ("bf16", "f32"), "split2": ("f32", "f32")}[kind]
+    dts = {"bf16": torch.bfloat16, "f32": torch.float32}
+    for name, X, dt in (("A", A, dts[a_dt]), ("B", B, dts[b_dt])):
+        if X.dim() != 3:
+            raise ValueError(f"{name} must be 3-D (batch, rows, cols), got {tuple(X.shape)}")
+        _check_mat(name, X, tuple(X.shape), dt)
+    if A.shape[0] != B.shape[0] or (A.shape[1] if a_mn_major else A.shape[2]) != (B.shape[1] if b_mn_major
+                                                                                   else B.shape[2]):
+        raise ValueError(f"A {tuple(A.shape)} and B {tuple(B.shape)} do not share batch and K")
     k |= {"auto": 0, "one_cta": 16, "cta_pair": 32}[kernel]
     batch = A.shape[0]
     M = A.shape[2] if a_mn_major else A.shape[1]
