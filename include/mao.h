@@ -108,7 +108,7 @@ typedef struct {
   float update_rms;    /* ||W_new - W_old||_F / sqrt(m n) (Muon); -1 where not computed (SOAP, FOAM) */
   float offdiag_ratio; /* FOAM/SOAP adaptive check ratio of this step, -1 if none ran */
   int32_t refreshed;   /* bit 0: right basis refreshed, bit 1: left basis refreshed */
-  int32_t nonfinite;   /* number of non-finite entries in W_new */
+  int32_t nonfinite;   /* number of non-finite entries in W_new (Muon); 0, not counted (SOAP, FOAM) */
 } mao_stats;
 
 /* ------------------------------------------------------------------ Muon */
