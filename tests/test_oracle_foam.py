@@ -123,3 +123,34 @@ def test_state_sizes_reproduce_printed_memory():
     assert round(foam, g["printed_digits"]) == g["foam_gib"]
     # a plausible slip (counting one factor instead of factor + basis) misses the figure
     assert round(sum(m * n * 2 + m * m + n * n for m, n in shapes) * L * bpe / 2 ** 30, 2) != g["soap_gib"]
+
+
+def test_weight_decay_is_decoupled():
+    rng = np.random.default_rng(42)
+    m, n = 6, 5
+    W = rng.standard_normal((m, n))
+    G = rng.standard_normal((m, n)) * 0.1
+    kw = dict(t=1, beta1=0.9, beta2=0.95, eps=1e-8, lr=0.01)
+    a = O.foam_step(W, G, O.FoamState.init(m, n), wd=0.0, **kw)
+    b = O.foam_step(W, G, O.FoamState.init(m, n), wd=0.3, **kw)
+    np.testing.assert_allclose(b.W - a.W, -0.01 * 0.3 * W, rtol=0, atol=1e-15)
+    np.testing.assert_array_equal(a.state.r, b.state.r)
+
+
+@pytest.mark.parametrize("t", [1, 2, 7])
+def test_raw_trace_differs_by_the_bias_correction(t):
+    """tau uses the bias-corrected trace tr(R / (1 - b2^t)); the literal tr(R) variant
+    gives exactly (1 - b2^t) times it, for any state."""
+    rng = np.random.default_rng(43 + t)
+    n, m = 4, 6
+    A = rng.standard_normal((n, n))
+    R = A @ A.T
+    r = np.abs(rng.standard_normal(m)) + 0.1
+    c = np.abs(rng.standard_normal(n)) + 0.1
+    b2 = 0.95
+    bc = O.foam_tau(R, r, c, t, b2)
+    raw = O.foam_tau(R, r, c, t, b2, raw_trace=True)
+    assert np.isclose(raw, bc * (1.0 - b2 ** t), rtol=1e-13)
+    # against the definition: tr(R^) / (||r^||_1 ||c^||_1) with every hat 1/(1 - b2^t)
+    h = 1.0 / (1.0 - b2 ** t)
+    assert np.isclose(bc, (np.trace(R) * h) / (np.sum(r) * h * np.sum(c) * h), rtol=1e-13)

@@ -214,3 +214,19 @@ def test_forced_permutation_replays_the_sort():
     c = O.soap_step(np.zeros((m, n)), G, st, t=1, beta1=0.9, beta2=0.9, eps=1e-8, lr=1.0,
                     force_perm_L=a.perm_L[::-1].copy(), force_perm_R=a.perm_R)
     assert not np.allclose(c.state.QL, a.state.QL)
+
+
+def test_weight_decay_is_decoupled():
+    """The recipe's weight decay acts on W alone: the steps with and without it differ
+    by exactly -lr wd W, whatever the gradient (a decay folded into the gradient or the
+    moments would change the Adam part too)."""
+    rng = np.random.default_rng(41)
+    m, n = 6, 5
+    W = rng.standard_normal((m, n))
+    G = rng.standard_normal((m, n)) * 0.1
+    kw = dict(t=1, beta1=0.9, beta2=0.95, eps=1e-8, lr=0.01)
+    a = O.soap_step(W, G, O.SoapState.init(m, n), wd=0.0, **kw)
+    b = O.soap_step(W, G, O.SoapState.init(m, n), wd=0.3, **kw)
+    np.testing.assert_allclose(b.W - a.W, -0.01 * 0.3 * W, rtol=0, atol=1e-15)
+    np.testing.assert_array_equal(a.state.M, b.state.M)
+    np.testing.assert_array_equal(a.state.V, b.state.V)
