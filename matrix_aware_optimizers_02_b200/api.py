@@ -103,9 +103,10 @@ class MuonBatch:
         self.workspace = workspace
 
     def __call__(self, stream: Optional[torch.cuda.Stream] = None) -> None:
-        st = self.lib.mao_muon_step(self.arr, self.count, ctypes.byref(self.params), self.workspace.data_ptr(),
-                                    self.ws_bytes, self.stats.data_ptr() if self.stats is not None else None,
-                                    _stream_handle(stream))
+        with torch.cuda.nvtx.range("mao.muon_step"):  # names the step's launches in a trace
+            st = self.lib.mao_muon_step(self.arr, self.count, ctypes.byref(self.params), self.workspace.data_ptr(),
+                                        self.ws_bytes, self.stats.data_ptr() if self.stats is not None else None,
+                                        _stream_handle(stream))
         L.check(st, "mao_muon_step")
 
     def device_status(self, stream: Optional[torch.cuda.Stream] = None) -> int:
@@ -255,9 +256,10 @@ class SoapBatch(_PrecondBatch):
 
     def __call__(self, t: int, stream: Optional[torch.cuda.Stream] = None) -> None:
         self.params.t = int(t)
-        st = self.lib.mao_soap_step(self.arr, self.count, ctypes.byref(self.params), self.workspace.data_ptr(),
-                                    self.ws_bytes, self.stats.data_ptr() if self.stats is not None else None,
-                                    _stream_handle(stream))
+        with torch.cuda.nvtx.range("mao.soap_step"):
+            st = self.lib.mao_soap_step(self.arr, self.count, ctypes.byref(self.params), self.workspace.data_ptr(),
+                                        self.ws_bytes, self.stats.data_ptr() if self.stats is not None else None,
+                                        _stream_handle(stream))
         L.check(st, "mao_soap_step")
 
 
@@ -297,7 +299,8 @@ class FoamBatch(_PrecondBatch):
 
     def __call__(self, t: int, stream: Optional[torch.cuda.Stream] = None) -> None:
         self.params.t = int(t)
-        st = self.lib.mao_foam_step(self.arr, self.count, ctypes.byref(self.params), self.workspace.data_ptr(),
-                                    self.ws_bytes, self.stats.data_ptr() if self.stats is not None else None,
-                                    _stream_handle(stream))
+        with torch.cuda.nvtx.range("mao.foam_step"):
+            st = self.lib.mao_foam_step(self.arr, self.count, ctypes.byref(self.params), self.workspace.data_ptr(),
+                                        self.ws_bytes, self.stats.data_ptr() if self.stats is not None else None,
+                                        _stream_handle(stream))
         L.check(st, "mao_foam_step")
