@@ -8,8 +8,9 @@ what the method computes.
 
 Everything here is NumPy in float64, one matrix at a time, in the order the
 source pages give.  Library primitives used as single steps: ``@`` (matmul),
-``numpy.linalg.qr`` (Householder QR), and, only in the self-check helpers at the
-bottom, ``numpy.linalg.svd`` / ``numpy.linalg.eigh``.
+``numpy.linalg.qr`` (Householder QR), ``numpy.linalg.svd`` (MOP's exact polar
+factor, which the pages define by the SVD), and, only in the self-check helpers
+at the bottom, ``numpy.linalg.eigh``.
 
 Sources (cited by page title and section):
   [SMB-review]  "SOAP, Muon and Beyond" (Korean review): §1-1 Problem definition
@@ -23,7 +24,7 @@ Sources (cited by page title and section):
   [MuonPlus]    "Muon+: Towards Better Muon via One Additional Normalization Step":
                 technical summary §2 Methodology.
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * Newton-Schulz form: the quintic X <- aX + (bA + cA^2)X with A = X X^T, run on
     the wide orientation (transposed when m > n); default (a,b,c) =
     (3.4445, -4.7750, 2.0315) each iteration.  The pages name Newton-Schulz only.
@@ -126,21 +127,53 @@ def muon_plus_norm(O, mode: int, eps: float = NORM_EPS):
     raise ValueError(f"unknown norm mode {mode}")
 
 
+def polar_exact(M):
+    """Exact polar factor U V^T of M = U S V^T from the thin SVD.
+
+    [SMB-summary] "Muon vs SOAP Comparison": MOP is Muon with the Newton-Schulz
+    approximation replaced by the exact polar decomposition computed by SVD.
+    """
+    U, _, Vt = np.linalg.svd(_f64(M), full_matrices=False)
+    return U @ Vt
+
+
 def muon_step(W, G, M, *, mu: float, lr: float, wd: float = 0.0, ns_coefs=None,
-              ns_steps: int = 5, norm: int = NORM_NONE):
-    """One Muon (or Muon+) step on one m x n matrix.
+              ns_steps: int = 5, norm: int = NORM_NONE, split=(1, 1), polar: str = "ns"):
+    """One Muon (or Muon+, or MOP) step on one m x n matrix.
 
     [MuonPlus] §2 Methodology: M <- mu M + (1-mu) G; O = Ortho(M) (Newton-Schulz);
     optionally O <- Norm^(d)(O); W <- W - lr sqrt(m/n) O.  Decoupled weight decay
     W(1 - lr wd) is the reading of the recipe's weight decay ([SMB-review] §3-2).
+
+    split = (sr, sc): the stored matrix holds sr x sc logical matrices of equal
+    size (a fused QKV projection is (1, 3) when q, k, v are column blocks).  The
+    recipe of [SMB-review] §3-2 (2) and §4-4 (2) orthogonalises each logical
+    matrix on its own; reading: every per-matrix quantity (the Frobenius
+    pre-normalisation, Newton-Schulz, Norm^(d) and the sqrt(m/n) scale) is that
+    of the logical block.
+    polar = "ns" (Newton-Schulz) or "exact" (MOP: the SVD polar factor).
     Returns (W_new, M_new, O) with O the final (normalised) direction.
     """
     W, G, M = _f64(W), _f64(G), _f64(M)
     m, n = W.shape
-    M_new = mu * M + (1.0 - mu) * G                       # M1
-    O = newton_schulz(M_new, ns_coefs, ns_steps)          # M2 + M3
-    O = muon_plus_norm(O, norm)                           # M4
-    W_new = W * (1.0 - lr * wd) - lr * np.sqrt(m / n) * O  # M5
+    sr, sc = split
+    if m % sr or n % sc:
+        raise ValueError(f"{m}x{n} does not split into {sr}x{sc} equal blocks")
+    mb, nb = m // sr, n // sc
+    M_new = mu * M + (1.0 - mu) * G                                   # M1
+    O = np.empty_like(M_new)
+    for i in range(sr):
+        for j in range(sc):
+            blk = M_new[i * mb:(i + 1) * mb, j * nb:(j + 1) * nb]
+            if polar == "exact":
+                ob = polar_exact(blk)                                 # MOP
+            elif polar == "ns":
+                ob = newton_schulz(blk, ns_coefs, ns_steps)           # M2 + M3
+            else:
+                raise ValueError(f"unknown polar method {polar}")
+            ob = muon_plus_norm(ob, norm)                             # M4
+            O[i * mb:(i + 1) * mb, j * nb:(j + 1) * nb] = ob
+    W_new = W * (1.0 - lr * wd) - lr * np.sqrt(mb / nb) * O          # M5 (every block has the same shape)
     return W_new, M_new, O
 
 
@@ -263,32 +296,61 @@ class SoapResult:
     rho_R: float = -1.0
 
 
+def soap_factors(L, R, G, beta2: float, dtype=np.float64):
+    """S1: L <- b2 L + (1-b2) G G^T ;  R <- b2 R + (1-b2) G^T G  ([SMB-review] §1-1)."""
+    G = _w(G, dtype)
+    return (beta2 * _w(L, dtype) + (1.0 - beta2) * (G @ G.T),
+            beta2 * _w(R, dtype) + (1.0 - beta2) * (G.T @ G))
+
+
+def soap_precondition(W, G, M, V, QL, QR, *, t: int, beta1: float, beta2: float, eps: float,
+                      lr: float, wd: float = 0.0, dtype=np.float64):
+    """S5-S8 in a given pair of bases ([SMB-summary] eq. (1), [SMB-review] §3-2 (3)):
+      S5  M <- b1 M + (1-b1) G
+      S6  Gh = QL^T G QR ;  Mh = QL^T M QR
+      S7  V <- b2 V + (1-b2) Gh^2 ;  N = (Mh/(1-b1^t)) / (sqrt(V/(1-b2^t)) + eps)
+      S8  U = QL N QR^T ;  W <- W(1 - lr wd) - lr U
+    Returns (W_new, M_new, V_new, U).  V is the second moment already expressed in
+    these bases (after any permutation of the refresh).
+    """
+    W, G, M, V, QL, QR = (_w(x, dtype) for x in (W, G, M, V, QL, QR))
+    M = beta1 * M + (1.0 - beta1) * G                      # S5
+    Gh = QL.T @ G @ QR                                     # S6
+    Mh = QL.T @ M @ QR
+    V = beta2 * V + (1.0 - beta2) * Gh * Gh                # S7
+    mhat = Mh / (1.0 - beta1 ** t)
+    vhat = V / (1.0 - beta2 ** t)
+    N = mhat / (np.sqrt(vhat) + eps)
+    U = QL @ N @ QR.T                                      # S8
+    W_new = W * (1.0 - lr * wd) - lr * U
+    return W_new, M, V, U
+
+
 def soap_step(W, G, state: SoapState, *, t: int, beta1: float, beta2: float,
               eps: float, lr: float, wd: float = 0.0, refresh_kind: int = REFRESH_EVERY_K,
-              k: int = 1, pf: int = 10, tol: float = 0.1, sort: bool = True,
+              k: int = 1, pf: int = 10, tol: float = 0.1, sort: bool = True, lag: bool = False,
               dtype=np.float64, force_perm_L=None, force_perm_R=None) -> SoapResult:
     """One two-sided SOAP step with the real-time eigenbasis refresh.
 
     Order ([SMB-review] §3-2 (4)): the current gradient enters the factors first,
     then the basis is refreshed from them (power step + QR), then the momentum is
     preconditioned in the refreshed basis:
-      S1  L <- b2 L + (1-b2) G G^T ;  R <- b2 R + (1-b2) G^T G   ([SMB-review] §1-1)
+      S1  factor EMAs (soap_factors)
       S2  refresh decision
       S3  sort keys diag(Q^T F Q), permutation, power step P = F Q
       S4  Q <- qr(P)
-      S5  M <- b1 M + (1-b1) G
-      S6  Gh = QL^T G QR ;  Mh = QL^T M QR                         (eq. (1))
-      S7  V <- b2 V + (1-b2) Gh^2 ;  N = (Mh/(1-b1^t)) / (sqrt(V/(1-b2^t)) + eps)
-      S8  U = QL N QR^T ;  W <- W(1 - lr wd) - lr U                   (eq. (1))
+      S5-S8  soap_precondition
+    lag=True takes the order of the standard implementation that [SMB-summary]
+    ("SOAP Instability Diagnosis") and [SMB-review] §2-1 (3) blame for the
+    slingshot instability: the refresh (S2-S4) runs on the factors as they were
+    before this step's gradient entered them, and S1 follows it.
     """
     W, G = _w(W, dtype), _w(G, dtype)
     s = state.copy(dtype)
     m, n = W.shape
-    # S1
-    s.L = beta2 * s.L + (1.0 - beta2) * (G @ G.T)
-    s.R = beta2 * s.R + (1.0 - beta2) * (G.T @ G)
-    # S2
-    refL, rhoL = refresh_decision(refresh_kind, t, k, pf, tol, s.L, s.QL, dtype)
+    if not lag:
+        s.L, s.R = soap_factors(s.L, s.R, G, beta2, dtype)                  # S1
+    refL, rhoL = refresh_decision(refresh_kind, t, k, pf, tol, s.L, s.QL, dtype)  # S2
     refR, rhoR = refresh_decision(refresh_kind, t, k, pf, tol, s.R, s.QR, dtype)
     permL = np.arange(m, dtype=np.int32)
     permR = np.arange(n, dtype=np.int32)
@@ -299,19 +361,10 @@ def soap_step(W, G, state: SoapState, *, t: int, beta1: float, beta2: float,
     if refR:
         s.QR, permR = refresh_basis(s.R, s.QR, sort, dtype, force_perm_R)
         s.V = s.V[:, permR]
-    # S5
-    s.M = beta1 * s.M + (1.0 - beta1) * G
-    # S6
-    Gh = s.QL.T @ G @ s.QR
-    Mh = s.QL.T @ s.M @ s.QR
-    # S7
-    s.V = beta2 * s.V + (1.0 - beta2) * Gh * Gh
-    mhat = Mh / (1.0 - beta1 ** t)
-    vhat = s.V / (1.0 - beta2 ** t)
-    N = mhat / (np.sqrt(vhat) + eps)
-    # S8
-    U = s.QL @ N @ s.QR.T
-    W_new = W * (1.0 - lr * wd) - lr * U
+    if lag:
+        s.L, s.R = soap_factors(s.L, s.R, G, beta2, dtype)                  # S1 after the refresh
+    W_new, s.M, s.V, U = soap_precondition(W, G, s.M, s.V, s.QL, s.QR, t=t, beta1=beta1, beta2=beta2,
+                                           eps=eps, lr=lr, wd=wd, dtype=dtype)
     return SoapResult(W_new, s, U, permL, permR, refL, refR, rhoL, rhoR)
 
 
@@ -363,9 +416,35 @@ def foam_tau(R, r, c, t: int, beta2: float, raw_trace: bool = False) -> float:
     return tr / (rn * cn)
 
 
+def foam_precondition(W, G, M, r, c, R, QR, *, t: int, beta1: float, beta2: float, eps: float,
+                      lr: float, wd: float = 0.0, raw_trace: bool = False, dtype=np.float64):
+    """F4-F6 in a given input-side basis QR ([FOAM-review] §1, §3):
+      F4  M <- b1 M + (1-b1) G ;  Gr = G QR ;  Mr = M QR
+      F5  r <- b2 r + (1-b2) rowmean(Gr^2) ; c <- b2 c + (1-b2) colmean(Gr^2) ;
+          v^_ij = tau r^_i c^_j ;  N = (Mr/(1-b1^t)) / (sqrt(v^) + eps)
+      F6  U = N QR^T ;  W <- W(1 - lr wd) - lr U
+    c is the column EMA already in QR's column order.  Returns
+    (W_new, M_new, r_new, c_new, U, tau).
+    """
+    W, G, M, r, c, QR = (_w(x, dtype) for x in (W, G, M, r, c, QR))
+    M = beta1 * M + (1.0 - beta1) * G                      # F4
+    Gr = G @ QR
+    Mr = M @ QR
+    G2 = Gr * Gr                                           # F5
+    r = beta2 * r + (1.0 - beta2) * np.mean(G2, axis=1)
+    c = beta2 * c + (1.0 - beta2) * np.mean(G2, axis=0)
+    tau = foam_tau(R, r, c, t, beta2, raw_trace)
+    bc2 = 1.0 - beta2 ** t
+    vhat = tau * np.outer(r / bc2, c / bc2)
+    N = (Mr / (1.0 - beta1 ** t)) / (np.sqrt(vhat) + eps)
+    U = N @ QR.T                                           # F6
+    W_new = W * (1.0 - lr * wd) - lr * U
+    return W_new, M, r, c, U, tau
+
+
 def foam_step(W, G, state: FoamState, *, t: int, beta1: float, beta2: float, eps: float,
               lr: float, wd: float = 0.0, refresh_kind: int = REFRESH_ADAPTIVE, k: int = 1,
-              pf: int = 10, tol: float = 0.1, sort: bool = True,
+              pf: int = 10, tol: float = 0.1, sort: bool = True, lag: bool = False,
               raw_trace: bool = False, dtype=np.float64, force_perm=None) -> FoamResult:
     """One FOAM step (input-only preconditioning, factored Adam moment).
 
@@ -373,38 +452,25 @@ def foam_step(W, G, state: FoamState, *, t: int, beta1: float, beta2: float, eps
       F1  R <- b2 R + (1-b2) G^T G             (input-side factor only; L dropped)
       F2  refresh decision (adaptive criterion, pf, tol)
       F3  refresh Q_R as in SOAP; the permutation also permutes c
-      F4  M <- b1 M + (1-b1) G ;  Gr = G Q_R ;  Mr = M Q_R     (G_rot = G Q_R)
-      F5  r <- b2 r + (1-b2) rowmean(Gr^2) ; c <- b2 c + (1-b2) colmean(Gr^2);
-          v^_ij = tau r^_i c^_j ;  N = (Mr/(1-b1^t)) / (sqrt(v^) + eps)
-      F6  U = N Q_R^T ;  W <- W(1 - lr wd) - lr U
+      F4-F6  foam_precondition
+    lag=True refreshes from R as it was before this step's gradient entered it
+    (F2-F3 before F1), as soap_step's lag does.
     """
     W, G = _w(W, dtype), _w(G, dtype)
     s = state.copy(dtype)
-    m, n = W.shape
-    # F1
-    s.R = beta2 * s.R + (1.0 - beta2) * (G.T @ G)
-    # F2
-    ref, rho = refresh_decision(refresh_kind, t, k, pf, tol, s.R, s.QR, dtype)
+    n = W.shape[1]
+    if not lag:
+        s.R = beta2 * s.R + (1.0 - beta2) * (G.T @ G)          # F1
+    ref, rho = refresh_decision(refresh_kind, t, k, pf, tol, s.R, s.QR, dtype)  # F2
     perm = np.arange(n, dtype=np.int32)
-    # F3
-    if ref:
+    if ref:                                                    # F3
         s.QR, perm = refresh_basis(s.R, s.QR, sort, dtype, force_perm)
         s.c = s.c[perm]
-    # F4
-    s.M = beta1 * s.M + (1.0 - beta1) * G
-    Gr = G @ s.QR
-    Mr = s.M @ s.QR
-    # F5
-    G2 = Gr * Gr
-    s.r = beta2 * s.r + (1.0 - beta2) * np.mean(G2, axis=1)
-    s.c = beta2 * s.c + (1.0 - beta2) * np.mean(G2, axis=0)
-    tau = foam_tau(s.R, s.r, s.c, t, beta2, raw_trace)
-    bc2 = 1.0 - beta2 ** t
-    vhat = tau * np.outer(s.r / bc2, s.c / bc2)
-    N = (Mr / (1.0 - beta1 ** t)) / (np.sqrt(vhat) + eps)
-    # F6
-    U = N @ s.QR.T
-    W_new = W * (1.0 - lr * wd) - lr * U
+    if lag:
+        s.R = beta2 * s.R + (1.0 - beta2) * (G.T @ G)          # F1 after the refresh
+    W_new, s.M, s.r, s.c, U, tau = foam_precondition(W, G, s.M, s.r, s.c, s.R, s.QR, t=t, beta1=beta1,
+                                                     beta2=beta2, eps=eps, lr=lr, wd=wd, raw_trace=raw_trace,
+                                                     dtype=dtype)
     return FoamResult(W_new, s, U, perm, ref, rho, tau)
 
 
@@ -427,23 +493,8 @@ def foam_state_elems(m: int, n: int) -> int:
 # --------------------------------------------------------------------------
 
 def polar_svd(M):
-    """Exact polar factor U V^T of M from the SVD ([SMB-review] §2-1 (2))."""
-    U, _, Vt = np.linalg.svd(_f64(M), full_matrices=False)
-    return U @ Vt
-
-
-def ns_closed_form(M, coefs, eps: float = NS_EPS):
-    """Newton-Schulz in closed form: U diag(phi_k o ... o phi_1(s_i/(||M||_F+eps))) V^T.
-
-    Each iteration maps every singular value of the normalised matrix through the
-    odd polynomial phi(x) = a x + b x^3 + c x^5 and leaves the singular vectors alone.
-    """
-    M = _f64(M)
-    U, S, Vt = np.linalg.svd(M, full_matrices=False)
-    x = S / (np.sqrt(np.sum(M * M)) + eps)
-    for (a, b, c) in coefs:
-        x = a * x + b * x ** 3 + c * x ** 5
-    return (U * x[None, :]) @ Vt
+    """Exact polar factor (self-check helper; the same as polar_exact)."""
+    return polar_exact(M)
 
 
 def _inv_quarter_root_psd(S, rtol: float = 1e-12):

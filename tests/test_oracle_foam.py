@@ -134,7 +134,9 @@ def test_weight_decay_is_decoupled():
     a = O.foam_step(W, G, O.FoamState.init(m, n), wd=0.0, **kw)
     b = O.foam_step(W, G, O.FoamState.init(m, n), wd=0.3, **kw)
     np.testing.assert_allclose(b.W - a.W, -0.01 * 0.3 * W, rtol=0, atol=1e-15)
-    np.testing.assert_array_equal(a.state.r, b.state.r)
+    # the decay touches W only: every moment, the factor and the basis are unchanged
+    for name in ("M", "r", "c", "R", "QR"):
+        np.testing.assert_array_equal(getattr(a.state, name), getattr(b.state, name))
 
 
 @pytest.mark.parametrize("t", [1, 2, 7])
@@ -154,3 +156,25 @@ def test_raw_trace_differs_by_the_bias_correction(t):
     # against the definition: tr(R^) / (||r^||_1 ||c^||_1) with every hat 1/(1 - b2^t)
     h = 1.0 / (1.0 - b2 ** t)
     assert np.isclose(bc, (np.trace(R) * h) / (np.sum(r) * h * np.sum(c) * h), rtol=1e-13)
+
+
+def test_foam_lagged_refresh_sorts_previous_gradient_columns():
+    """FOAM with lag=True (refresh before the current gradient enters R), beta2 = 0 and
+    diagonal gradients: the t = 2 basis is the permutation that sorts G_1's squared column
+    norms in descending order, and c follows that permutation."""
+    m, n = 5, 4
+    G1 = np.zeros((m, n))
+    G2 = np.zeros((m, n))
+    for i, (a, b) in enumerate(zip([1.0, 3.0, 2.0, 0.5], [2.0, 0.5, 1.0, 4.0])):
+        G1[i, i] = a
+        G2[i, i] = b
+    kw = dict(beta1=0.9, beta2=0.0, eps=1e-8, lr=1.0, refresh_kind=O.REFRESH_EVERY_K, k=1)
+    st = O.FoamState.init(m, n)
+    r1 = O.foam_step(np.zeros((m, n)), G1, st, t=1, lag=True, **kw)
+    assert np.array_equal(r1.state.QR, np.eye(n))
+    r2 = O.foam_step(np.zeros((m, n)), G2, r1.state, t=2, lag=True, **kw)
+    assert np.array_equal(r2.perm_R, [1, 2, 0, 3])
+    assert np.allclose(r2.state.QR, np.eye(n)[:, [1, 2, 0, 3]], atol=1e-15)
+    assert np.allclose(r2.state.R, G2.T @ G2, atol=1e-15)
+    fresh = O.foam_step(np.zeros((m, n)), G2, r1.state, t=2, lag=False, **kw)
+    assert np.array_equal(fresh.perm_R, [3, 0, 2, 1])

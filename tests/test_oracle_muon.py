@@ -159,3 +159,69 @@ def test_muon_plus_last_direction_is_unit():
     rc = O.muon_plus_norm(X, O.NORM_ROW_COL)
     assert np.allclose(np.linalg.norm(cr, axis=1), 1.0, atol=1e-6)
     assert np.allclose(np.linalg.norm(rc, axis=0), 1.0, atol=1e-6)
+
+
+# ------------------------------------------------------------------ MOP and the logical-matrix split
+
+@pytest.mark.parametrize("shape", [(6, 9), (9, 6), (7, 7)])
+def test_mop_exact_polar_from_constructed_svd(shape):
+    """MOP ([SMB-summary] "Muon vs SOAP Comparison"): the direction is U V^T of the momentum,
+    built from a constructed SVD (no SVD call in the expected value), and the update is
+    W - lr sqrt(m/n) U V^T."""
+    m, n = shape
+    rng = np.random.default_rng(31)
+    k = min(m, n)
+    U = synth.random_orthogonal(rng, m)[:, :k]
+    V = synth.random_orthogonal(rng, n)[:, :k]
+    S = rng.uniform(0.01, 5.0, size=k)
+    G = (U * S) @ V.T
+    W = rng.standard_normal((m, n))
+    lr, mu = 0.03, 0.9
+    Wn, Mn, Od = O.muon_step(W, G, np.zeros((m, n)), mu=mu, lr=lr, polar="exact")
+    assert np.allclose(Od, U @ V.T, atol=1e-12)
+    assert np.allclose(Wn, W - lr * np.sqrt(m / n) * (U @ V.T), atol=1e-12)
+    assert np.allclose(Mn, (1 - mu) * G, atol=1e-15)
+
+
+def _block_orthogonal(rng, b, count, scales):
+    return [s * synth.random_orthogonal(rng, b) for s in scales[:count]]
+
+
+def test_split_columns_orthogonalises_each_logical_matrix():
+    """A fused [q | k | v] matrix (split (1, 3)) with blocks s_i Q_i, Q_i orthogonal: each block
+    alone has every singular value s_i, so MOP gives [Q_1 Q_2 Q_3] and Newton-Schulz gives
+    phi^k(s_i / (s_i sqrt(b) + eps)) Q_i per block, each with sqrt(b/b) = 1 as the scale.  The
+    unsplit matrix (8 x 24) gives neither."""
+    rng = np.random.default_rng(32)
+    b = 8
+    Qs = [synth.random_orthogonal(rng, b) for _ in range(3)]
+    sc = [0.3, 1.7, 4.0]
+    M = np.concatenate([s * Q for s, Q in zip(sc, Qs)], axis=1)
+    W = np.zeros_like(M)
+    _, _, O_mop = O.muon_step(W, M, np.zeros_like(M), mu=0.0, lr=1.0, polar="exact", split=(1, 3))
+    assert np.allclose(O_mop, np.concatenate(Qs, axis=1), atol=1e-12)
+    coefs = [O.NS_DEFAULT_COEF] * 5
+    Wn, _, O_ns = O.muon_step(W, M, np.zeros_like(M), mu=0.0, lr=1.0, split=(1, 3))
+    want = np.concatenate([_phi_chain([s / (s * np.sqrt(b) + O.NS_EPS)], coefs)[0] * Q for s, Q in zip(sc, Qs)],
+                          axis=1)
+    assert np.allclose(O_ns, want, atol=1e-10)
+    assert np.allclose(Wn, -want, atol=1e-10)  # lr = 1, sqrt(8/8) = 1
+    _, _, O_whole = O.muon_step(W, M, np.zeros_like(M), mu=0.0, lr=1.0, polar="exact")
+    assert not np.allclose(O_whole, O_mop, atol=1e-3)
+
+
+def test_split_rows_uses_block_shape_for_scale_and_norm():
+    """Split (2, 1) of a 12 x 6 matrix into two 6 x 6 blocks: the scale is sqrt(6/6) = 1, not
+    sqrt(12/6); Muon+ row normalisation of an exact orthogonal block is the identity."""
+    rng = np.random.default_rng(33)
+    Q1, Q2 = synth.random_orthogonal(rng, 6), synth.random_orthogonal(rng, 6)
+    M = np.concatenate([2.0 * Q1, 0.5 * Q2], axis=0)
+    W = rng.standard_normal((12, 6))
+    lr = 0.1
+    Wn, _, Od = O.muon_step(W, M, np.zeros_like(M), mu=0.0, lr=lr, polar="exact", split=(2, 1),
+                            norm=O.NORM_ROW)
+    want = np.concatenate([Q1, Q2], axis=0)
+    assert np.allclose(Od, want, atol=1e-12)
+    assert np.allclose(Wn, W - lr * want, atol=1e-12)
+    with pytest.raises(ValueError):
+        O.muon_step(W, M, np.zeros_like(M), mu=0.0, lr=lr, split=(5, 1))

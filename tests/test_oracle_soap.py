@@ -230,3 +230,39 @@ def test_weight_decay_is_decoupled():
     np.testing.assert_allclose(b.W - a.W, -0.01 * 0.3 * W, rtol=0, atol=1e-15)
     np.testing.assert_array_equal(a.state.M, b.state.M)
     np.testing.assert_array_equal(a.state.V, b.state.V)
+
+
+# ------------------------------------------------------------------ lagged refresh (stale basis)
+
+def _diag_grad(d, m, n):
+    G = np.zeros((m, n))
+    for i, v in enumerate(d):
+        G[i, i] = v
+    return G
+
+
+def test_lagged_refresh_sees_the_previous_gradient_only():
+    """lag=True: the refresh runs on the factors before the current gradient enters them
+    ([SMB-summary] "SOAP Instability Diagnosis": the current gradient is left out of the
+    recalculation).  With beta2 = 0 and diagonal gradients the factors are diagonal, so the
+    refreshed basis is a permutation matrix in closed form:
+      t = 1: the old factors are 1e-6 I (all keys equal), so the basis stays I and the step is
+             elementwise Adam, U = G/(|G|+eps);
+      t = 2: the basis sorts the diagonal of G_1 G_1^T (not of G_2 G_2^T) in descending order.
+    Without lag, t = 2 sorts G_2's diagonal instead."""
+    m, n = 4, 5
+    G1 = _diag_grad([1.0, 3.0, 2.0, 0.5], m, n)
+    G2 = _diag_grad([2.0, 0.5, 1.0, 4.0], m, n)
+    kw = dict(beta1=0.9, beta2=0.0, eps=1e-8, lr=1.0)
+    st = O.SoapState.init(m, n)
+    r1 = O.soap_step(np.zeros((m, n)), G1, st, t=1, lag=True, **kw)
+    assert np.array_equal(r1.state.QL, np.eye(m)) and np.array_equal(r1.state.QR, np.eye(n))
+    assert np.allclose(r1.U, G1 / (np.abs(G1) + 1e-8), atol=1e-15)
+    r2 = O.soap_step(np.zeros((m, n)), G2, r1.state, t=2, lag=True, **kw)
+    order1 = [1, 2, 0, 3]  # G1's squared diagonal, descending
+    assert np.array_equal(r2.perm_L, order1)
+    assert np.allclose(r2.state.QL, np.eye(m)[:, order1], atol=1e-15)
+    # the factors still take in the current gradient, after the refresh
+    assert np.allclose(r2.state.L, G2 @ G2.T, atol=1e-15)
+    fresh = O.soap_step(np.zeros((m, n)), G2, r1.state, t=2, lag=False, **kw)
+    assert np.array_equal(fresh.perm_L, [3, 0, 2, 1])
