@@ -62,6 +62,12 @@ def parse():
                     help="instead of the bench line: FOAM alone for steps t = 1..N, each timed on its own, "
                          "and the median ms of plain, check-only and check+refresh steps")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other configurations' timings (Muon+ on the GPT-2-124M set, FOAM step kinds on "
+                         "the GPT-2-760M set) added to the bench line")
+    ap.add_argument("--cpu-baseline-full", action="store_true",
+                    help="instead of the bench line: time the float64 oracle once on every distinct shape of the "
+                         "workload for each optimizer (minutes) and print the table as JSON")
     ap.add_argument("--launch-log", default=None,
                     help="after the measurement, run one more step and write its launch list (kernel, work) here")
     ap.add_argument("--traffic-csv", default=None,
@@ -325,7 +331,60 @@ def cpu_oracle_sample(workload, budget_s, seed, optimizers, t_foam=1):
     cores = len(os.sched_getaffinity(0))
     sample = ("float64 NumPy oracle, each distinct shape's step time x its multiplicity (SOAP and FOAM steps "
               "with a basis refresh); " + "; ".join(parts))
-    return total_ms, cores, sample
+    return total_ms, cores, sample, blas_threads()
+
+
+def blas_threads():
+    """Threads of the BLAS library NumPy calls (threadpoolctl), or None."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads") for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else None
+    except Exception:
+        return None
+
+
+def cpu_full_table(workload, seed, optimizers):
+    """The float64 oracle timed once on every distinct shape of the workload, per optimizer
+    (SOAP and FOAM with a basis refresh), and the layer-set total = sum of time x count."""
+    from oracle import mao_oracle as O
+    specs = specs_for(workload, seed)
+    norm = {"col_row": O.NORM_COL_ROW}.get(MUON_NORM.get(workload, "none"), O.NORM_NONE)
+    shapes = {}
+    for sp in specs:
+        shapes[(sp.m, sp.n)] = shapes.get((sp.m, sp.n), 0) + 1
+    rng = np.random.default_rng(seed)
+    rows, total = [], 0.0
+    for opt in optimizers:
+        for (m, n), cnt in sorted(shapes.items()):
+            W = rng.standard_normal((m, n)) * 0.02
+            G = rng.standard_normal((m, n)) * 0.01
+            t0 = time.perf_counter()
+            if opt == "muon":
+                O.muon_step(W, G, np.zeros((m, n)), mu=0.95, lr=0.02, norm=norm)
+            elif opt == "soap":
+                O.soap_step(W, G, O.SoapState.init(m, n), t=1, beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3)
+            else:
+                O.foam_step(W, G, O.FoamState.init(m, n), t=1, beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3)
+            dt = time.perf_counter() - t0
+            rows.append({"optimizer": opt, "m": m, "n": n, "count": cnt, "s": round(dt, 3)})
+            total += dt * cnt
+            print(json.dumps(rows[-1]), file=sys.stderr, flush=True)
+    return {"workload": workload, "unit": "ms", "value": round(total * 1e3, 1), "cores": len(os.sched_getaffinity(0)),
+            "blas_threads": blas_threads(), "rows": rows}
+
+
+def committed_cpu_table(workload):
+    """The every-shape oracle timing committed under profiles/ for this workload (measured on
+    a GPU machine's host by --cpu-baseline-full), or None."""
+    p = os.path.join(ROOT, "profiles", f"cpu_oracle_{workload}.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    return {"value": d["value"], "unit": d["unit"], "cores": d["cores"], "blas_threads": d.get("blas_threads"),
+            "source": f"profiles/cpu_oracle_{workload}.json (bench.py --cpu-baseline-full, every distinct shape "
+                      "timed once, times its count)"}
 
 
 # ----------------------------------------------------------------------------- ranks
@@ -350,53 +409,65 @@ def per_layer_set(ms_max, world):
 
 # ----------------------------------------------------------------------------- the layer set on the GPU
 class LayerSet:
-    """W, G and the optimizer states of one synthetic layer set, plus one batch
-    object per optimizer (sharing W, G and one workspace)."""
+    """W, the optimizer states and `n_grad` gradient sets of one synthetic layer set,
+    plus, per optimizer, one batch object per gradient set (all sharing W, the states
+    and one workspace).  Step k uses gradient set k mod n_grad, so consecutive steps
+    see different gradients without any copy between them."""
 
-    def __init__(self, specs, seed, dev, g_bf16, optimizers, norm, soap_k=1):
+    def __init__(self, specs, seed, dev, g_bf16, optimizers, norm, soap_k=1, n_grad=3):
         import torch
 
         from matrix_aware_optimizers_02_b200 import api, synth
         self.torch = torch
         base = synth.torch_muon_inputs(specs, seed, dev, g_bf16=g_bf16)
         self.W = [w for (w, _, _) in base]
-        self.G = [g for (_, g, _) in base]
+        self.G_sets = [[g for (_, g, _) in base]]
         del base
+        gen = torch.Generator(device=dev)
+        for k in range(1, n_grad):
+            gen.manual_seed(seed * 1000003 + k)
+            self.G_sets.append([synth.torch_gaussian((sp.m, sp.n), sp.g_std * sp.g_scale, gen, dev,
+                                                     torch.bfloat16 if g_bf16 else torch.float32) for sp in specs])
+        self.G = self.G_sets[0]
+        self.n_grad = n_grad
         self.batches = {}
         z = torch.zeros
         if "muon" in optimizers:
-            mats = [(w, g, z(w.shape, device=dev)) for w, g in zip(self.W, self.G)]
-            self.batches["muon"] = api.MuonBatch(mats, mu=0.95, lr=0.02, norm=norm, with_stats=True,
-                                                 allocate=False)
+            M = [z(w.shape, device=dev) for w in self.W]
+            self.batches["muon"] = [api.MuonBatch(list(zip(self.W, Gs, M)), mu=0.95, lr=0.02, norm=norm,
+                                                  with_stats=True, allocate=False) for Gs in self.G_sets]
         if "soap" in optimizers:
-            mats = []
-            for w, g in zip(self.W, self.G):
+            st = []
+            for w in self.W:
                 m, n = w.shape
-                mats.append({"W": w, "G": g, "M": z((m, n), device=dev), "V": z((m, n), device=dev),
-                             "L": torch.eye(m, device=dev) * 1e-6, "R": torch.eye(n, device=dev) * 1e-6,
-                             "QL": torch.eye(m, device=dev), "QR": torch.eye(n, device=dev)})
-            self.batches["soap"] = api.SoapBatch(mats, beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3,
-                                                 refresh="every_k", k=soap_k, with_stats=True, allocate=False)
+                st.append({"M": z((m, n), device=dev), "V": z((m, n), device=dev),
+                           "L": torch.eye(m, device=dev) * 1e-6, "R": torch.eye(n, device=dev) * 1e-6,
+                           "QL": torch.eye(m, device=dev), "QR": torch.eye(n, device=dev)})
+            self.batches["soap"] = [api.SoapBatch([dict(d, W=w, G=g) for d, w, g in zip(st, self.W, Gs)], beta1=0.95,
+                                                  beta2=0.95, eps=1e-8, lr=3e-3, refresh="every_k", k=soap_k,
+                                                  with_stats=True, allocate=False) for Gs in self.G_sets]
         if "foam" in optimizers:
-            mats = []
-            for w, g in zip(self.W, self.G):
+            st = []
+            for w in self.W:
                 m, n = w.shape
-                mats.append({"W": w, "G": g, "M": z((m, n), device=dev), "r": z(m, device=dev),
-                             "c": z(n, device=dev), "R": torch.eye(n, device=dev) * 1e-6,
-                             "QR": torch.eye(n, device=dev)})
-            self.batches["foam"] = api.FoamBatch(mats, beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3,
-                                                 refresh="adaptive", pf=10, tol=0.1, with_stats=True,
-                                                 allocate=False)
+                st.append({"M": z((m, n), device=dev), "r": z(m, device=dev), "c": z(n, device=dev),
+                           "R": torch.eye(n, device=dev) * 1e-6, "QR": torch.eye(n, device=dev)})
+            self.batches["foam"] = [api.FoamBatch([dict(d, W=w, G=g) for d, w, g in zip(st, self.W, Gs)], beta1=0.95,
+                                                  beta2=0.95, eps=1e-8, lr=3e-3, refresh="adaptive", pf=10, tol=0.1,
+                                                  with_stats=True, allocate=False) for Gs in self.G_sets]
         self.order = [o for o in ("muon", "soap", "foam") if o in self.batches]
         # the steps run in order on one stream, so one workspace serves all of them
-        ws_bytes = max(b.ws_bytes for b in self.batches.values())
+        ws_bytes = max(b.ws_bytes for bs in self.batches.values() for b in bs)
         self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-        for b in self.batches.values():
-            b.attach_workspace(self.workspace)
+        for bs in self.batches.values():
+            for b in bs:
+                b.attach_workspace(self.workspace)
 
     def step(self, t, stream, events=None):
-        for i, name in enumerate(self.order):
-            b = self.batches[name]
+        """Step t (1-based) of every optimizer, on gradient set (t - 1) mod n_grad."""
+        gi = (t - 1) % self.n_grad
+        for name in self.order:
+            b = self.batches[name][gi]
             if events is not None:
                 events[name][0].record(stream)
             if name == "muon":
@@ -406,9 +477,13 @@ class LayerSet:
             if events is not None:
                 events[name][1].record(stream)
 
+    def stats_tensor(self, t):
+        """The stats array the first optimizer's step t writes."""
+        return self.batches[self.order[0]][(t - 1) % self.n_grad].stats
+
     def status(self):
-        for name, b in self.batches.items():
-            st = b.device_status()
+        for name, bs in self.batches.items():
+            st = bs[0].device_status()
             if st != 0:
                 return name, st
         return None
@@ -449,7 +524,8 @@ def run_mine(args, rank, world, dist):
     LS.step(t, stream)
     per_step_launches = lib.mao_profile_stop()
     torch.cuda.synchronize()
-    cap = min(per_step_launches * args.steps + 16, 60000)
+    # check and refresh steps launch more than the probe step: leave room for them
+    cap = min(int(per_step_launches * args.steps * 1.6) + 1024, 150000)
     Ev = ctypes.c_void_p * (2 * cap)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * cap)]
     for e in evs:  # torch creates the CUDA event object on its first record
@@ -496,11 +572,10 @@ def run_mine(args, rank, world, dist):
         e["bytes"] += info[i].bytes
         e["tc"] += info[i].tc_flops
 
-    # end-to-end: gradients from pinned host memory, the step, stats back to host
-    host_g = [g.cpu().pin_memory() for g in LS.G]
-    h2d = sum(g.numel() * g.element_size() for g in host_g)
-    res = LS.batches[LS.order[0]].stats
-    stats_host = torch.empty_like(res, device="cpu").pin_memory()
+    # end-to-end: this step's gradient set from pinned host memory, the step, stats back to host
+    host_sets = [[g.cpu().pin_memory() for g in Gs] for Gs in LS.G_sets]
+    h2d = sum(g.numel() * g.element_size() for g in host_sets[0])
+    stats_host = torch.empty_like(LS.stats_tensor(1), device="cpu").pin_memory()
     d2h = stats_host.numel() * stats_host.element_size()
     barrier()
     torch.cuda.synchronize()
@@ -509,17 +584,22 @@ def run_mine(args, rank, world, dist):
     e0.record(stream)
     for _ in range(args.steps):
         t += 1
-        for g, hg in zip(LS.G, host_g):
+        gi = (t - 1) % LS.n_grad
+        for g, hg in zip(LS.G_sets[gi], host_sets[gi]):
             g.copy_(hg, non_blocking=True)
         LS.step(t, stream)
-        stats_host.copy_(res, non_blocking=True)
+        stats_host.copy_(LS.stats_tensor(t), non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
+    del host_sets
     e2e_ms = e0.elapsed_time(e1) / args.steps
 
     if args.launch_log and rank == 0:
         write_launch_log(args, lib, L, LS, t + 1, stream)
+    order = list(LS.order)
+    del LS
+    torch.cuda.empty_cache()
 
     ms_max, e2e_max = reduce_times([ms, e2e_ms], dist, dev)
     if rank != 0:
@@ -568,8 +648,12 @@ def run_mine(args, rank, world, dist):
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        cpu_ms, cores, sample = cpu_oracle_sample(args.workload, args.cpu_budget_s, args.seed, LS.order)
-        cpu = {"value": round(cpu_ms, 1), "unit": "ms", "cores": cores, "kind": "oracle", "sample": sample}
+        cpu_ms, cores, sample, blas = cpu_oracle_sample(args.workload, args.cpu_budget_s, args.seed, order)
+        cpu = {"value": round(cpu_ms, 1), "unit": "ms", "cores": cores, "blas_threads": blas, "kind": "oracle",
+               "sample": sample}
+        full = committed_cpu_table(args.workload)
+        if full is not None:
+            cpu["every_shape_timed"] = full
 
     n_elems = sum(s.m * s.n for s in specs)
     line = {
@@ -586,7 +670,7 @@ def run_mine(args, rank, world, dist):
         "dtype": "bf16 operands / fp32 accumulate (Newton-Schulz); fp32-faithful split-bf16 products and fp32 "
                  "states (SOAP, FOAM)",
         "data": "synthetic (seeded Gaussian gradients, random weights)",
-        "config": {"workload": args.workload, "description": desc, "optimizers": LS.order,
+        "config": {"workload": args.workload, "description": desc, "optimizers": order,
                    "optimizer_ms": opt_ms,
                    "muon": {"mu": 0.95, "lr": 0.02, "ns_steps": 5, "norm": norm},
                    "soap": {"beta1": 0.95, "beta2": 0.95, "eps": 1e-8,
@@ -595,6 +679,8 @@ def run_mine(args, rank, world, dist):
                    "foam": {"beta1": 0.95, "beta2": 0.95, "eps": 1e-8, "refresh": "adaptive pf=10 tol=0.1"},
                    "timed_steps_t": [args.warmup + 2, args.warmup + 1 + args.steps],
                    "matrices_per_rank": len(specs), "elements_per_rank": n_elems,
+                   "gradient_sets": 3,
+                   "inputs": "three device-resident seeded gradient sets, step t uses set (t - 1) mod 3",
                    "l2_policy": "inputs larger than L2 (no flush)", "parallelism": f"independent layer sets x{world}"},
         "roofline": roof,
         "kernels": kernels,
@@ -604,27 +690,35 @@ def run_mine(args, rank, world, dist):
         "gpu_launches": int(n_launch),
         "clocks": clk,
     }
+    if world == 1 and not args.no_extra:
+        # the other configurations, timed on this GPU after the layer set above was freed
+        c4 = foam_kinds("gpt2_760m", 21, args.seed)
+        line["other_configs"] = {
+            "gpt2_124m_muon_plus_col_row": muon_set_ms("gpt2_124m", 20, 3, args.seed),
+            "gpt2_760m_foam_step_kinds": {"median_ms": c4["median_ms"], "steps": c4["steps"],
+                                          "note": "fresh fp32 gradient each step; medians over t >= 2"},
+        }
     return line
 
 
-def run_foam_kinds(args):
-    """FOAM alone on the workload for t = 1..N (adaptive, pf = 10, tol = 0.1, a fresh
-    gradient each step), each step bracketed by its own events and followed by a read
-    of the per-matrix refresh flags:
-    a step is plain ((t - 1) mod pf != 0), check-only (a check step where no matrix
-    refreshed) or check+refresh.  Returns one JSON object with the median of each kind."""
+def foam_kinds(workload, steps, seed):
+    """FOAM alone on the workload for t = 1..steps (adaptive, pf = 10, tol = 0.1, a fresh
+    gradient each step, drawn outside the timed region), each step bracketed by its own
+    events and followed by a read of the per-matrix refresh flags.  A step is plain
+    ((t - 1) mod pf != 0), check-only (a check step where no matrix refreshed) or
+    check+refresh.  Returns the median ms of each kind over t >= 2 (t = 1 also builds
+    the step's launch plan on the host while the GPU waits) and the per-step record."""
     import torch
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    desc, g_bf16 = WORKLOADS[args.workload]
-    specs = specs_for(args.workload, args.seed)
-    LS = LayerSet(specs, args.seed, dev, g_bf16, ["foam"], "none")
-    b = LS.batches["foam"]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    desc, g_bf16 = WORKLOADS[workload]
+    specs = specs_for(workload, seed)
+    LS = LayerSet(specs, seed, dev, g_bf16, ["foam"], "none", n_grad=1)
+    b = LS.batches["foam"][0]
     stream = torch.cuda.current_stream()
     kinds = {"plain": [], "check": [], "check+refresh": []}
     per_t = []
-    gen = torch.Generator(device=dev).manual_seed(args.seed + 1)
-    for t in range(1, args.foam_kinds + 1):
+    gen = torch.Generator(device=dev).manual_seed(seed + 1)
+    for t in range(1, steps + 1):
         for g, sp in zip(LS.G, specs):  # a fresh gradient each step, outside the timed region
             g.normal_(0.0, sp.g_std * sp.g_scale, generator=gen)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -636,14 +730,55 @@ def run_foam_kinds(args):
         ms = e0.elapsed_time(e1)
         nref = sum(1 for r in b.stats_dict()["refreshed"] if r & 1)
         kind = "plain" if (t - 1) % 10 else ("check+refresh" if nref else "check")
-        kinds[kind].append(ms)
+        if t > 1:
+            kinds[kind].append(ms)
         per_t.append({"t": t, "kind": kind, "ms": round(ms, 3), "refreshed": nref})
     if LS.status():
         raise RuntimeError(f"device status {LS.status()}")
-    return {"metric": "FOAM step ms by step kind", "unit": "ms", "workload": args.workload, "description": desc,
-            "steps": args.foam_kinds, "median_ms": {k: (round(statistics.median(v), 3) if v else None)
-                                                    for k, v in kinds.items()},
-            "per_step": per_t, "note": "t = 1 includes first-touch costs; medians over the rest of each kind"}
+    del LS, b
+    torch.cuda.empty_cache()
+    return {"workload": workload, "description": desc, "steps": steps,
+            "median_ms": {k: (round(statistics.median(v), 3) if v else None) for k, v in kinds.items()},
+            "per_step": per_t}
+
+
+def muon_set_ms(workload, steps, warmup, seed):
+    """Muon (+ the workload's Muon+ norm) alone on the workload: ms per step over `steps`
+    timed steps after `warmup`, three gradient sets in rotation."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _, g_bf16 = WORKLOADS[workload]
+    specs = specs_for(workload, seed)
+    norm = MUON_NORM.get(workload, "none")
+    LS = LayerSet(specs, seed, dev, g_bf16, ["muon"], norm)
+    stream = torch.cuda.current_stream()
+    t = 0
+    for _ in range(warmup):
+        t += 1
+        LS.step(t, stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        t += 1
+        LS.step(t, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if LS.status():
+        raise RuntimeError(f"device status {LS.status()}")
+    ms = e0.elapsed_time(e1) / steps
+    del LS
+    torch.cuda.empty_cache()
+    return {"workload": workload, "norm": norm, "matrices": len(specs), "ms_per_step": round(ms, 4),
+            "steps": steps, "warmup": warmup}
+
+
+def run_foam_kinds(args):
+    import torch
+    torch.cuda.set_device(0)
+    out = foam_kinds(args.workload, args.foam_kinds, args.seed)
+    out.update({"metric": "FOAM step ms by step kind", "unit": "ms"})
+    return out
 
 
 def run_reference(args, rank, world):
@@ -654,8 +789,8 @@ def run_reference(args, rank, world):
     per_step = []
     info = None
     for i in range(args.warmup + args.steps):
-        ms, cores, sample = cpu_oracle_sample(args.workload, args.cpu_budget_s / max(args.steps, 1), args.seed + i,
-                                              optimizers)
+        ms, cores, sample, _ = cpu_oracle_sample(args.workload, args.cpu_budget_s / max(args.steps, 1),
+                                                 args.seed + i, optimizers)
         if i >= args.warmup:
             per_step.append(ms)
             info = (cores, sample)
@@ -682,6 +817,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     if args.foam_kinds > 0:
         print(json.dumps(run_foam_kinds(args)), flush=True)
+        return 0
+    if args.cpu_baseline_full:
+        opts = [o.strip() for o in args.optimizers.split(",") if o.strip()]
+        print(json.dumps(cpu_full_table(args.workload, args.seed, opts)), flush=True)
         return 0
     if args.impl == "reference":
         line = run_reference(args, rank, world)

@@ -35,9 +35,11 @@
  *   - Errors: arguments, shapes, dtypes, alignment and workspace size are
  *     validated before anything is enqueued; on failure nothing is modified and
  *     the status says why.  A failed launch returns MAO_ERR_CUDA.  Conditions
- *     found on the device (a bounded wait that gave up) never trap: they are
- *     written to a status word at the start of the workspace, which
- *     mao_workspace_status() reads.
+ *     found on the device never trap: a bounded wait that gave up, and (when
+ *     stats are requested) a non-finite weight written by the step, are recorded
+ *     in a status word at the start of the workspace, which mao_workspace_status()
+ *     reads.  A non-finite gradient propagates: the step writes non-finite
+ *     weights and states, and the caller restores them from its own copy.
  *   - Initial state is the caller's job: L = R = 1e-6 I, Q = I,
  *     M = V = r = c = 0, t = 1 for the first step.
  */
@@ -51,7 +53,7 @@
 extern "C" {
 #endif
 
-#define MAO_VERSION 2
+#define MAO_VERSION 3
 
 #if defined(__GNUC__)
 #define MAO_API __attribute__((visibility("default")))
@@ -70,7 +72,7 @@ typedef enum {
   MAO_ERR_ALIGN = 4,       /* a device pointer not 16-byte aligned */
   MAO_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than the *_workspace_size() answer */
   MAO_ERR_CUDA = 6,        /* a CUDA runtime call or kernel launch failed */
-  MAO_ERR_NONFINITE = 7,   /* reserved for device-detected non-finite values */
+  MAO_ERR_NONFINITE = 7,   /* device status only: the step wrote a non-finite weight (stats requested) */
   MAO_ERR_TIMEOUT = 8,     /* a bounded device-side wait gave up (a defect, never expected) */
   MAO_ERR_UNSUPPORTED = 9, /* a valid request this build does not implement (e.g. no sm_100 device) */
   MAO_ERR_NOT_INITIALIZED = 10 /* a call that needs one-time set-up ran before it */
@@ -101,14 +103,20 @@ typedef struct {
   float tol;    /* ADAPTIVE threshold on the off-diagonal ratio */
   int32_t sort; /* 1: before the power step, order the basis by diag(Q^T F Q) descending
                    (stable) and permute the moment state with it; 0: keep the order */
+  int32_t lag;  /* 0: the current gradient enters the factors before the refresh (the
+                   real-time order of "SOAP, Muon and Beyond" review 3-2 (4));
+                   1: the refresh runs on the factors as they were before this step's
+                   gradient entered them, the order of the standard implementation
+                   that the summary's "SOAP Instability Diagnosis" names as a cause of
+                   the slingshot instability (kept to reproduce the stale basis) */
 } mao_refresh;
 
 /* Optional per-matrix diagnostics, written on the device (array of `count`). */
 typedef struct {
-  float update_rms;    /* ||W_new - W_old||_F / sqrt(m n) (Muon); -1 where not computed (SOAP, FOAM) */
+  float update_rms;    /* ||W_new - W_old||_F / sqrt(m n) */
   float offdiag_ratio; /* FOAM/SOAP adaptive check ratio of this step, -1 if none ran */
   int32_t refreshed;   /* bit 0: right basis refreshed, bit 1: left basis refreshed */
-  int32_t nonfinite;   /* number of non-finite entries in W_new (Muon); 0, not counted (SOAP, FOAM) */
+  int32_t nonfinite;   /* number of non-finite entries in W_new (also recorded in the status word) */
 } mao_stats;
 
 /* ------------------------------------------------------------------ Muon */
@@ -119,7 +127,21 @@ typedef struct {
   const void* G;   /* device m x n gradient, fp32 or bf16 (g_dtype) */
   int32_t g_dtype; /* mao_dtype */
   float* M;        /* device fp32 m x n momentum, updated in place */
+  int32_t split_rows, split_cols; /* 0 or 1: one matrix.  Otherwise the stored matrix
+                   holds split_rows x split_cols logical matrices of (m / split_rows) x
+                   (n / split_cols), each stepped as a matrix of its own (a fused QKV
+                   projection stored as [q | k | v] is split_cols = 3): its own
+                   pre-normalisation, orthogonalisation, Muon+ norms and
+                   sqrt(m_b / n_b) scale ("SOAP, Muon and Beyond" review 3-2 (2),
+                   4-4 (2)).  Each block width keeps the row rule above (n / split_cols
+                   a multiple of 4, of 8 for a bf16 G), else MAO_ERR_SHAPE */
 } mao_muon_mat;
+
+typedef enum {
+  MAO_POLAR_NS = 0,    /* Newton-Schulz with the given coefficients, bf16 operands */
+  MAO_POLAR_EXACT = 1  /* MOP: the polar factor U V^T to fp32 accuracy ("SOAP, Muon, and
+                          Beyond" summary, "Muon vs SOAP Comparison") */
+} mao_polar;
 
 typedef struct {
   float mu;             /* momentum EMA coefficient */
@@ -130,6 +152,7 @@ typedef struct {
   const float* ns_coef; /* host, ns_steps x 3 (a, b, c) per iteration, or NULL for
                            (3.4445, -4.7750, 2.0315) every iteration */
   int32_t norm;         /* mao_norm_mode */
+  int32_t polar;        /* mao_polar */
 } mao_muon_params;
 
 /*
@@ -176,6 +199,19 @@ MAO_API mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, const 
  */
 MAO_API mao_status mao_muon_step_noalloc(const mao_muon_mat* mats, int32_t count, const mao_muon_params* p,
                                          mao_stats* stats, mao_stream_t stream);
+
+/*
+ * mao_muon_noalloc_status — an addition of this library with no counterpart in the
+ * source pages.  mao_muon_step_noalloc keeps its device status word at the start of
+ * its static scratch, whose address the caller never sees, so mao_workspace_status
+ * cannot reach it; this call reads it instead.  It synchronises `stream` and returns
+ * MAO_OK if the last mao_muon_step_noalloc on the current device recorded no
+ * device-side condition, otherwise that condition (MAO_ERR_TIMEOUT: a bounded wait
+ * gave up and W may be partly updated; MAO_ERR_NONFINITE: with stats requested, a
+ * non-finite weight was written).  `where` (nullable) receives the site identifier.
+ * The first call on a device does the same address look-up as the step.
+ */
+MAO_API mao_status mao_muon_noalloc_status(mao_stream_t stream, int32_t* where);
 
 /* ------------------------------------------------------------------ SOAP */
 

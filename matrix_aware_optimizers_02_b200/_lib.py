@@ -28,10 +28,12 @@ MAO_ERR_NOT_INITIALIZED = 10
 MAO_F32, MAO_BF16 = 0, 1
 NORM_MODES = {"none": 0, "row": 1, "col": 2, "col_row": 3, "row_col": 4}
 REFRESH_EVERY_K, REFRESH_ADAPTIVE, REFRESH_NEVER = 0, 1, 2
+POLAR_NS, POLAR_EXACT = 0, 1
 
 
 class Refresh(ctypes.Structure):
-    _fields_ = [("kind", c_int32), ("k", c_int32), ("pf", c_int32), ("tol", c_float), ("sort", c_int32)]
+    _fields_ = [("kind", c_int32), ("k", c_int32), ("pf", c_int32), ("tol", c_float), ("sort", c_int32),
+                ("lag", c_int32)]
 
 
 class Stats(ctypes.Structure):
@@ -41,12 +43,12 @@ class Stats(ctypes.Structure):
 
 class MuonMat(ctypes.Structure):
     _fields_ = [("m", c_int32), ("n", c_int32), ("W", c_void_p), ("G", c_void_p), ("g_dtype", c_int32),
-                ("M", c_void_p)]
+                ("M", c_void_p), ("split_rows", c_int32), ("split_cols", c_int32)]
 
 
 class MuonParams(ctypes.Structure):
     _fields_ = [("mu", c_float), ("lr", c_float), ("wd", c_float), ("eps", c_float), ("ns_steps", c_int32),
-                ("ns_coef", POINTER(c_float)), ("norm", c_int32)]
+                ("ns_coef", POINTER(c_float)), ("norm", c_int32), ("polar", c_int32)]
 
 
 class SoapMat(ctypes.Structure):
@@ -88,6 +90,7 @@ SIGNATURES = {
     "mao_muon_step": (c_int32, [POINTER(MuonMat), c_int32, POINTER(MuonParams), c_void_p, c_size_t, c_void_p,
                                 c_void_p]),
     "mao_muon_step_noalloc": (c_int32, [POINTER(MuonMat), c_int32, POINTER(MuonParams), c_void_p, c_void_p]),
+    "mao_muon_noalloc_status": (c_int32, [c_void_p, POINTER(c_int32)]),
     "mao_soap_workspace_size": (c_int32, [POINTER(SoapMat), c_int32, POINTER(SoapParams), POINTER(c_size_t)]),
     "mao_soap_step": (c_int32, [POINTER(SoapMat), c_int32, POINTER(SoapParams), c_void_p, c_size_t, c_void_p,
                                 c_void_p]),

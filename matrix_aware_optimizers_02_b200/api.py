@@ -57,18 +57,22 @@ class MuonBatch:
     def __init__(self, mats: Sequence[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]], *, mu: float, lr: float,
                  wd: float = 0.0, eps: float = 1e-7, ns_steps: int = 5,
                  ns_coef: Optional[Sequence[Sequence[float]]] = None, norm: str = "none",
+                 split: Optional[Sequence[Tuple[int, int]]] = None, polar: str = "ns",
                  workspace: Optional[torch.Tensor] = None, with_stats: bool = False, allocate: bool = True):
         self.lib = L.load()
         self.mats = list(mats)
         n = len(self.mats)
         arr = (L.MuonMat * max(n, 1))()
         dev = None
+        if split is not None and len(split) != n:
+            raise ValueError("split must give one (split_rows, split_cols) pair per matrix")
         for i, (W, G, M) in enumerate(self.mats):
             m_, n_ = W.shape
             _check_mat("W", W, (m_, n_))
             _check_mat("G", G, (m_, n_), None)
             _check_mat("M", M, (m_, n_))
-            arr[i] = L.MuonMat(m_, n_, W.data_ptr(), G.data_ptr(), _g_dtype(G), M.data_ptr())
+            sr, sc = split[i] if split is not None else (1, 1)
+            arr[i] = L.MuonMat(m_, n_, W.data_ptr(), G.data_ptr(), _g_dtype(G), M.data_ptr(), int(sr), int(sc))
             dev = W.device
         self.arr = arr
         self.count = n
@@ -82,7 +86,10 @@ class MuonBatch:
             coef_ptr = ctypes.cast(self._coef, ctypes.POINTER(ctypes.c_float))
         if norm not in L.NORM_MODES:
             raise ValueError(f"norm must be one of {sorted(L.NORM_MODES)}")
-        self.params = L.MuonParams(mu, lr, wd, eps, ns_steps, coef_ptr, L.NORM_MODES[norm])
+        polars = {"ns": L.POLAR_NS, "exact": L.POLAR_EXACT}
+        if polar not in polars:
+            raise ValueError(f"polar must be one of {sorted(polars)}")
+        self.params = L.MuonParams(mu, lr, wd, eps, ns_steps, coef_ptr, L.NORM_MODES[norm], polars[polar])
         nbytes = ctypes.c_size_t(0)
         L.check(self.lib.mao_muon_workspace_size(arr, n, ctypes.byref(self.params), ctypes.byref(nbytes)),
                 "mao_muon_workspace_size")
@@ -181,11 +188,11 @@ def set_table_kernel(kernel: str = "auto") -> None:
             "mao_test_set_table_kernel")
 
 
-def _refresh(kind: str, k: int, pf: int, tol: float, sort: bool) -> "L.Refresh":
+def _refresh(kind: str, k: int, pf: int, tol: float, sort: bool, lag: bool = False) -> "L.Refresh":
     kinds = {"every_k": L.REFRESH_EVERY_K, "adaptive": L.REFRESH_ADAPTIVE, "never": L.REFRESH_NEVER}
     if kind not in kinds:
         raise ValueError(f"refresh must be one of {sorted(kinds)}")
-    return L.Refresh(kinds[kind], int(k), int(pf), float(tol), int(bool(sort)))
+    return L.Refresh(kinds[kind], int(k), int(pf), float(tol), int(bool(sort)), int(bool(lag)))
 
 
 class _PrecondBatch:
@@ -212,10 +219,13 @@ class _PrecondBatch:
         return self.lib.mao_workspace_status(self.workspace.data_ptr(), _stream_handle(stream), ctypes.byref(where))
 
     def stats_dict(self):
+        """Per-matrix diagnostics of the last step."""
         if self.stats is None:
             return None
         s = self.stats[: self.count].cpu()
-        return {"offdiag_ratio": s[:, 1].tolist(), "refreshed": s[:, 2].contiguous().view(torch.int32).tolist()}
+        return {"update_rms": s[:, 0].tolist(), "offdiag_ratio": s[:, 1].tolist(),
+                "refreshed": s[:, 2].contiguous().view(torch.int32).tolist(),
+                "nonfinite": s[:, 3].contiguous().view(torch.int32).tolist()}
 
 
 class SoapBatch(_PrecondBatch):
@@ -229,7 +239,7 @@ class SoapBatch(_PrecondBatch):
 
     def __init__(self, mats, *, beta1: float, beta2: float, eps: float, lr: float, wd: float = 0.0,
                  refresh: str = "every_k", k: int = 1, pf: int = 10, tol: float = 0.1, sort: bool = True,
-                 workspace: Optional[torch.Tensor] = None, with_stats: bool = False, t: int = 1,
+                 lag: bool = False, workspace: Optional[torch.Tensor] = None, with_stats: bool = False, t: int = 1,
                  allocate: bool = True):
         self.lib = L.load()
         self.mats = list(mats)
@@ -250,7 +260,7 @@ class SoapBatch(_PrecondBatch):
                                     pr.data_ptr() if pr is not None else None)
             dev = W.device
         self.count = n
-        self.params = L.SoapParams(beta1, beta2, eps, lr, wd, int(t), _refresh(refresh, k, pf, tol, sort))
+        self.params = L.SoapParams(beta1, beta2, eps, lr, wd, int(t), _refresh(refresh, k, pf, tol, sort, lag))
         self._finish(self.lib.mao_soap_workspace_size, n, dev if dev is not None else "cuda", workspace, with_stats,
                      allocate)
 
@@ -272,8 +282,8 @@ class FoamBatch(_PrecondBatch):
 
     def __init__(self, mats, *, beta1: float, beta2: float, eps: float, lr: float, wd: float = 0.0,
                  refresh: str = "adaptive", k: int = 1, pf: int = 10, tol: float = 0.1, sort: bool = True,
-                 tau_raw_trace: bool = False, workspace: Optional[torch.Tensor] = None, with_stats: bool = False,
-                 t: int = 1, allocate: bool = True):
+                 lag: bool = False, tau_raw_trace: bool = False, workspace: Optional[torch.Tensor] = None,
+                 with_stats: bool = False, t: int = 1, allocate: bool = True):
         self.lib = L.load()
         self.mats = list(mats)
         n = len(self.mats)
@@ -292,7 +302,7 @@ class FoamBatch(_PrecondBatch):
                                     pr.data_ptr() if pr is not None else None)
             dev = W.device
         self.count = n
-        self.params = L.FoamParams(beta1, beta2, eps, lr, wd, int(t), _refresh(refresh, k, pf, tol, sort),
+        self.params = L.FoamParams(beta1, beta2, eps, lr, wd, int(t), _refresh(refresh, k, pf, tol, sort, lag),
                                    int(bool(tau_raw_trace)))
         self._finish(self.lib.mao_foam_workspace_size, n, dev if dev is not None else "cuda", workspace, with_stats,
                      allocate)

@@ -255,6 +255,12 @@ mao_status set_table_kernel_policy(int policy) {
   return MAO_OK;
 }
 
+mao_status table_set_stats(TableLaunch& L, float2* upd) {
+  if (L.probs.empty() || upd == nullptr || L.probs.back().aux == nullptr) return MAO_ERR_INVALID_ARG;
+  L.probs.back().upd = upd;
+  return MAO_OK;
+}
+
 mao_status table_set_alt(TableLaunch& L, const int* sel, float* out2, const Split3* out2p, int ld_out2) {
   if (L.probs.empty() || sel == nullptr) return MAO_ERR_INVALID_ARG;
   GemmProblem& P = L.probs.back();

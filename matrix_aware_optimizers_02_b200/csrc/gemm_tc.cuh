@@ -110,6 +110,10 @@ struct GemmProblem {
   __nv_bfloat16* out2_p[3];
   int ld_out2, ld_out2p;
   int tile_begin2;             // first tile in the CTA-pair numbering (256-row tiles)
+  // Update statistics (nullptr = none): for every block of 32 output rows by 64
+  // columns, (sum of (out - aux)^2, number of non-finite out) is written to
+  // upd[(row / 32) * ceil(N / 64) + col / 64] by the one warp that stores that block.
+  float2* upd;
 };
 
 struct GemmTableParams {
@@ -362,13 +366,15 @@ struct TableSource {
   }
   __device__ int cols(const TileInfo& t) const { return p.probs[t.idx].N; }
 
-  template <int EPI>
-  __device__ __forceinline__ void epilogue(const TileInfo& t, int row, int col0, float* v) const {
+  // out = alpha * acc + beta * aux for 32 columns of one row; `st` accumulates the
+  // update statistics (sum of (out - aux)^2, non-finite count) when the problem asks.
+  __device__ __forceinline__ void epilogue_table(const TileInfo& t, int row, int col0, float* v, float2& st) const {
     const GemmProblem& P = p.probs[t.idx];
     if (row >= P.M) return;
     const bool full = (col0 + 32 <= P.N);
     if (P.aux != nullptr) {
       const float* a = P.aux + (long long)row * P.ld_aux + col0;
+      const bool want = P.upd != nullptr;
       if (full) {
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
@@ -377,9 +383,26 @@ struct TableSource {
           v[j + 1] = P.alpha * v[j + 1] + P.beta * q.y;
           v[j + 2] = P.alpha * v[j + 2] + P.beta * q.z;
           v[j + 3] = P.alpha * v[j + 3] + P.beta * q.w;
+          if (want) {
+            const float d0 = v[j] - q.x, d1 = v[j + 1] - q.y, d2 = v[j + 2] - q.z, d3 = v[j + 3] - q.w;
+            st.x += (d0 * d0 + d1 * d1) + (d2 * d2 + d3 * d3);
+            st.y += (float)(!isfinite(v[j]) + !isfinite(v[j + 1]) + !isfinite(v[j + 2]) + !isfinite(v[j + 3]));
+          }
         }
       } else {
-        for (int j = 0; j < 32; ++j) v[j] = (col0 + j < P.N) ? P.alpha * v[j] + P.beta * a[j] : 0.0f;
+        for (int j = 0; j < 32; ++j) {
+          if (col0 + j < P.N) {
+            const float old = a[j];
+            v[j] = P.alpha * v[j] + P.beta * old;
+            if (want) {
+              const float d = v[j] - old;
+              st.x += d * d;
+              st.y += isfinite(v[j]) ? 0.f : 1.f;
+            }
+          } else {
+            v[j] = 0.0f;
+          }
+        }
       }
     } else {
 #pragma unroll
@@ -421,6 +444,19 @@ struct TableSource {
         }
       }
     }
+  }
+
+  // Warp-level reduction of the update statistics of the 32 x 64 block whose first
+  // row / column are row0 / col0 (every lane of the warp calls this; fixed order).
+  __device__ __forceinline__ void flush_stats(const TileInfo& t, int row0, int col0, float2 st, int lane) const {
+    const GemmProblem& P = p.probs[t.idx];
+    if (P.upd == nullptr) return;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      st.x += __shfl_xor_sync(0xffffffffu, st.x, o);
+      st.y += __shfl_xor_sync(0xffffffffu, st.y, o);
+    }
+    if (lane == 0 && row0 < P.M && col0 < P.N) P.upd[(long long)(row0 >> 5) * ((P.N + 63) >> 6) + (col0 >> 6)] = st;
   }
 };
 
@@ -661,9 +697,18 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
           mbar_arrive(&tempty_bar[acc]);
         }
         if (!ok) break;
+        if constexpr (EPI == EPI_TABLE) {
+          static_assert(COLS == 64, "update statistics assume 64 columns per epilogue warp");
+          float2 st = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int ch = 0; ch < COLS / 32; ++ch)
-          if (t.n0 + cb + ch * 32 < ncols) src.template epilogue<EPI>(t, row, t.n0 + cb + ch * 32, &run[ch * 32]);
+          for (int ch = 0; ch < COLS / 32; ++ch)
+            if (t.n0 + cb + ch * 32 < ncols) src.epilogue_table(t, row, t.n0 + cb + ch * 32, &run[ch * 32], st);
+          src.flush_stats(t, t.m0 + q * 32, t.n0 + cb, st, lane);
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < COLS / 32; ++ch)
+            if (t.n0 + cb + ch * 32 < ncols) src.template epilogue<EPI>(t, row, t.n0 + cb + ch * 32, &run[ch * 32]);
+        }
       }
     }
   }
@@ -932,10 +977,12 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
         mbar_arrive_cluster(tempty_lead[acc]);
       }
       if (!ok) break;
+      static_assert(COLS == 64, "update statistics assume 64 columns per epilogue warp");
+      float2 st = make_float2(0.f, 0.f);
 #pragma unroll
       for (int ch = 0; ch < COLS / 32; ++ch)
-        if (t.n0 + cb + ch * 32 < ncols)
-          src.template epilogue<EPI_TABLE>(t, row, t.n0 + cb + ch * 32, &run[ch * 32]);
+        if (t.n0 + cb + ch * 32 < ncols) src.epilogue_table(t, row, t.n0 + cb + ch * 32, &run[ch * 32], st);
+      src.flush_stats(t, t.m0 + 128 * (int)rank + q * 32, t.n0 + cb, st, lane);
     }
   }
 

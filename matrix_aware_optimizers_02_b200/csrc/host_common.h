@@ -207,6 +207,10 @@ mao_status table_add(TableLaunch& L, MapSet& maps, const Split3& A, const Split3
 // on the device (sel is read by every tile's epilogue).
 mao_status table_set_alt(TableLaunch& L, const int* sel, float* out2, const Split3* out2p, int ld_out2);
 
+// Ask the last problem added to L for update statistics (see GemmProblem::upd):
+// `upd` holds ceil(M / 32) * ceil(N / 64) float2 slots.  Needs an aux operand.
+mao_status table_set_stats(TableLaunch& L, float2* upd);
+
 // Process-wide kernel choice for table-mode launches (0 auto, 1 one CTA, 2 CTA pair).
 int table_kernel_policy();
 mao_status set_table_kernel_policy(int policy);

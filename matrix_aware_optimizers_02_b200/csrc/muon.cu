@@ -39,7 +39,7 @@ struct MuonPlan {
   std::vector<MuonClass> cls;
   std::vector<int> mat_class, mat_slot;  // class of matrix p, its index in the class
   size_t off_table = 0, off_scale = 0, off_partial = 0, off_rowscale = 0, off_colscale = 0, off_rowpart = 0,
-         off_colpart = 0, off_updpart = 0, off_updbad = 0;
+         off_colpart = 0, off_updpart = 0, off_updbad = 0, off_ranges = 0;
   int tiles = 0;
   size_t total = 0;
   bool use_rows = false, use_cols = false;
@@ -59,13 +59,18 @@ mao_status validate(const mao_muon_mat* mats, int32_t count, const mao_muon_para
   if (p->ns_coef != nullptr)
     for (int i = 0; i < 3 * p->ns_steps; ++i)
       if (!std::isfinite(p->ns_coef[i])) return MAO_ERR_INVALID_ARG;
+  if (p->polar != MAO_POLAR_NS && p->polar != MAO_POLAR_EXACT) return MAO_ERR_INVALID_ARG;
   for (int i = 0; i < count; ++i) {
     const mao_muon_mat& a = mats[i];
     if (a.m < 1 || a.n < 1) return MAO_ERR_SHAPE;
     if ((long long)a.m * a.n > (1ll << 31) - 1) return MAO_ERR_SHAPE;
     if (a.g_dtype != MAO_F32 && a.g_dtype != MAO_BF16) return MAO_ERR_DTYPE;
-    if (a.n % 4 != 0) return MAO_ERR_SHAPE;
-    if (a.g_dtype == MAO_BF16 && a.n % 8 != 0) return MAO_ERR_SHAPE;
+    if (a.split_rows < 0 || a.split_cols < 0) return MAO_ERR_INVALID_ARG;
+    const int sr = std::max(a.split_rows, 1), sc = std::max(a.split_cols, 1);
+    if (a.m % sr != 0 || a.n % sc != 0) return MAO_ERR_SHAPE;
+    const int nb = a.n / sc;
+    if (nb % 4 != 0) return MAO_ERR_SHAPE;
+    if (a.g_dtype == MAO_BF16 && nb % 8 != 0) return MAO_ERR_SHAPE;
     if (check_ptrs) {
       if (a.W == nullptr || a.G == nullptr || a.M == nullptr) return MAO_ERR_INVALID_ARG;
       if (!aligned16(a.W) || !aligned16(a.G) || !aligned16(a.M)) return MAO_ERR_ALIGN;
@@ -74,7 +79,38 @@ mao_status validate(const mao_muon_mat* mats, int32_t count, const mao_muon_para
   return MAO_OK;
 }
 
-void plan(const mao_muon_mat* mats, int count, const mao_muon_params* p, MuonPlan& P) {
+// The logical matrices of a call: each caller matrix, or each block of a split one
+// (row-major block order, consecutive), with its leading dimension and owner.
+struct Logical {
+  std::vector<mao_muon_mat> mats;
+  std::vector<int> ld, owner;
+};
+
+void expand(const mao_muon_mat* mats, int count, Logical& L) {
+  L = Logical();
+  for (int i = 0; i < count; ++i) {
+    const mao_muon_mat& a = mats[i];
+    const int sr = std::max(a.split_rows, 1), sc = std::max(a.split_cols, 1);
+    const int mb = a.m / sr, nb = a.n / sc;
+    const size_t ge = a.g_dtype == MAO_BF16 ? 2 : 4;
+    for (int r = 0; r < sr; ++r)
+      for (int c = 0; c < sc; ++c) {
+        const size_t off = (size_t)r * mb * a.n + (size_t)c * nb;
+        mao_muon_mat b = a;
+        b.m = mb;
+        b.n = nb;
+        b.split_rows = b.split_cols = 1;
+        b.W = a.W ? a.W + off : nullptr;
+        b.M = a.M ? a.M + off : nullptr;
+        b.G = a.G ? static_cast<const void*>(static_cast<const uint8_t*>(a.G) + off * ge) : nullptr;
+        L.mats.push_back(b);
+        L.ld.push_back(a.n);
+        L.owner.push_back(i);
+      }
+  }
+}
+
+void plan(const mao_muon_mat* mats, int count, const int* ld, int callers, const mao_muon_params* p, MuonPlan& P) {
   P = MuonPlan();
   P.use_rows = norm_uses_rows(p->norm);
   P.use_cols = norm_uses_cols(p->norm);
@@ -114,6 +150,7 @@ void plan(const mao_muon_mat* mats, int count, const mao_muon_params* p, MuonPla
     MuonMatDev& D = P.table[i];
     D.m = mats[i].m;
     D.n = mats[i].n;
+    D.ld = ld[i];
     D.g_bf16 = mats[i].g_dtype == MAO_BF16;
     D.trans = D.m > D.n ? 1 : 0;
     D.ldx = round_up_int(std::max(D.m, D.n), 8);
@@ -139,6 +176,7 @@ void plan(const mao_muon_mat* mats, int count, const mao_muon_params* p, MuonPla
   }
   P.off_updpart = cv.take(sizeof(float) * (size_t)std::max(tiles, 1));
   P.off_updbad = cv.take(sizeof(int) * (size_t)std::max(tiles, 1));
+  P.off_ranges = cv.take(sizeof(MuonStatsRange) * (size_t)std::max(callers, 1));
   for (auto& c : P.cls) {
     const size_t cnt = c.mats.size();
     for (int k = 0; k < 2; ++k) c.off_X[k] = cv.take(2 * cnt * (size_t)c.s * c.ld_l);
@@ -158,18 +196,27 @@ extern "C" mao_status mao_muon_workspace_size(const mao_muon_mat* mats, int32_t 
                                               size_t* bytes) {
   if (bytes == nullptr) return MAO_ERR_INVALID_ARG;
   MAO_TRY(validate(mats, count, p, false));
+  Logical L;
+  expand(mats, count, L);
   MuonPlan P;
-  plan(mats, count, p, P);
+  plan(L.mats.data(), (int)L.mats.size(), L.ld.data(), count, p, P);
   *bytes = P.total;
   return MAO_OK;
 }
 
 extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, const mao_muon_params* p,
                                    void* workspace, size_t ws_bytes, mao_stats* stats, mao_stream_t stream_) {
+  const mao_muon_mat* const mats_in = mats;
   MAO_TRY(validate(mats, count, p, true));
   if (count == 0) return MAO_OK;
+  // from here on, work on the logical matrices (the blocks of split matrices)
+  Logical L;
+  expand(mats, count, L);
+  const int callers = count;
+  mats = L.mats.data();
+  count = (int)L.mats.size();
   MuonPlan P;
-  plan(mats, count, p, P);
+  plan(mats, count, L.ld.data(), callers, p, P);
   if (workspace == nullptr || ws_bytes < P.total) return MAO_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MAO_ERR_ALIGN;
   if (stats != nullptr && !aligned16(stats)) return MAO_ERR_ALIGN;
@@ -345,9 +392,19 @@ extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, con
   }
   MAO_CUDA_TRY(cudaGetLastError());
   if (stats) {
+    std::vector<MuonStatsRange> ranges(callers);
+    for (int c = 0; c < callers; ++c) ranges[c] = MuonStatsRange{0, 0, mats_in[c].m, mats_in[c].n};
+    for (int i = count - 1; i >= 0; --i) {  // blocks of one caller are consecutive
+      MuonStatsRange& r = ranges[L.owner[i]];
+      r.tile_begin = P.table[i].tile_begin;
+      r.tiles += P.table[i].tiles_r * P.table[i].tiles_c;
+    }
+    MAO_CUDA_TRY(cudaMemcpyAsync(ws + P.off_ranges, ranges.data(), sizeof(MuonStatsRange) * callers,
+                                 cudaMemcpyHostToDevice, stream));
     {
       LaunchScope ls(stream, MAO_K_MUON_STATS, 0.0, 8.0 * P.tiles);
-      muon_stats_kernel<<<(count + 7) / 8, 256, 0, stream>>>(T, count, updpart, updbad, stats);
+      muon_stats_kernel<<<(callers + 7) / 8, 256, 0, stream>>>(
+          reinterpret_cast<const MuonStatsRange*>(ws + P.off_ranges), callers, updpart, updbad, stats, status);
     }
     MAO_CUDA_TRY(cudaGetLastError());
   }

@@ -41,6 +41,7 @@ struct MuonMatDev {
   const float* oscale;     // multiplier of O (the pre-normalisation scale when no NS step ran), or nullptr
   int scale_slot;          // index of this matrix in the per-class-ordered scale array
   int m, n;
+  int ld;                  // leading dimension of W, G and M (n, or the stored width of a split matrix)
   int g_bf16;
   int trans;               // 1 if m > n: X = M^T
   int ldx;                 // leading dimension of X (elements, multiple of 8)
@@ -126,7 +127,7 @@ __global__ void __launch_bounds__(256) muon_prep_kernel(const MuonMatDev* __rest
     const int row = r0 + rl;
     float mv[4] = {0.f, 0.f, 0.f, 0.f};
     if (row < D.m && col < D.n) {  // n % 4 == 0: the 4 columns are all in or all out
-      const long long off = (long long)row * D.n + col;
+      const long long off = (long long)row * D.ld + col;
       float4 m4 = *reinterpret_cast<const float4*>(D.M + off);
       float g[4];
       if (D.g_bf16) {
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(256) muon_update_kernel(const MuonMatDev* __re
     const int row = r0 + ty + 16 * i;
     if (row >= D.m || col >= D.n) continue;
     const float rs = om * (use_rows ? D.rowscale[row] : 1.0f);
-    float* wp = D.W + (long long)row * D.n + col;
+    float* wp = D.W + (long long)row * D.ld + col;
     float4 w = *reinterpret_cast<float4*>(wp);
     float wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -338,17 +339,24 @@ __global__ void __launch_bounds__(256) muon_update_kernel(const MuonMatDev* __re
   }
 }
 
-// One warp per matrix.
-__global__ void muon_stats_kernel(const MuonMatDev* __restrict__ T, int count, const float* __restrict__ upd_partial,
-                                  const int* __restrict__ upd_nonfinite, mao_stats* __restrict__ stats) {
+// Tiles of one caller matrix (the blocks of a split matrix are consecutive).
+struct MuonStatsRange {
+  int tile_begin, tiles;
+  int m, n;
+};
+
+// One warp per caller matrix.  A non-finite weight is also recorded in the workspace
+// status word as MAO_ERR_NONFINITE (site 30), unless an error came first.
+__global__ void muon_stats_kernel(const MuonStatsRange* __restrict__ R, int count, const float* __restrict__ upd_partial,
+                                  const int* __restrict__ upd_nonfinite, mao_stats* __restrict__ stats,
+                                  DevStatus* status) {
   const int p = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (p >= count) return;
-  const MuonMatDev& D = T[p];
-  const int nt = D.tiles_r * D.tiles_c;
+  const MuonStatsRange& D = R[p];
   double s = 0.0;
   int b = 0;
-  for (int i = lane; i < nt; i += 32) {
+  for (int i = lane; i < D.tiles; i += 32) {
     s += (double)upd_partial[D.tile_begin + i];
     b += upd_nonfinite[D.tile_begin + i];
   }
@@ -360,6 +368,7 @@ __global__ void muon_stats_kernel(const MuonMatDev* __restrict__ T, int count, c
     stats[p].offdiag_ratio = -1.0f;
     stats[p].refreshed = 0;
     stats[p].nonfinite = b;
+    if (b > 0) report(status, MAO_ERR_NONFINITE, 30, p, b);
   }
 }
 

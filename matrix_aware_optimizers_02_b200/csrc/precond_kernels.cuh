@@ -873,28 +873,54 @@ __global__ void __launch_bounds__(256) pc_check_kernel(const CheckJob* __restric
   }
 }
 
-// Per-matrix diagnostics of a SOAP / FOAM step: refresh bits and the check ratio.
-// fixed_bits >= 0: the refresh was decided on the host (bits given); otherwise
-// read the device flags (bit 0 right side, bit 1 left side).
+// Per-matrix diagnostics of a SOAP / FOAM step: refresh bits, the check ratio and
+// the update statistics.  fixed_bits >= 0: the refresh was decided on the host
+// (bits given); otherwise read the device flags (bit 0 right side, bit 1 left side).
+// upd holds the update product's per-block partials (sum of squared weight
+// changes, non-finite count), nslots of them; they are summed in a fixed order.
 struct StatsJob {
   const int* flag_r;
   const int* flag_l;
   const float* rho;
+  const float2* upd;
+  int nslots;
   int fixed_bits;
   int index;  // position in the caller's stats array
+  int m, n;
 };
 
-__global__ void pc_stats_kernel(const StatsJob* __restrict__ J, int n, mao_stats* __restrict__ stats) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  const StatsJob& j = J[i];
+// One block of 256 threads per matrix.  A non-finite weight is also recorded in the
+// workspace status word as MAO_ERR_NONFINITE (site 31), unless an error came first.
+__global__ void __launch_bounds__(256) pc_stats_kernel(const StatsJob* __restrict__ J, mao_stats* __restrict__ stats,
+                                                       DevStatus* status) {
+  __shared__ double red[2][256];
+  const StatsJob& j = J[blockIdx.x];
+  double ss = 0.0, nf = 0.0;
+  for (int i = threadIdx.x; i < j.nslots; i += 256) {
+    const float2 v = j.upd[i];
+    ss += (double)v.x;
+    nf += (double)v.y;
+  }
+  red[0][threadIdx.x] = ss;
+  red[1][threadIdx.x] = nf;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (threadIdx.x < o) {
+      red[0][threadIdx.x] += red[0][threadIdx.x + o];
+      red[1][threadIdx.x] += red[1][threadIdx.x + o];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x != 0) return;
   int bits = j.fixed_bits;
   if (bits < 0) bits = ((j.flag_r && *j.flag_r) ? 1 : 0) | ((j.flag_l && *j.flag_l) ? 2 : 0);
+  const int bad = (int)red[1][0];
   mao_stats& st = stats[j.index];
-  st.update_rms = -1.0f;
+  st.update_rms = (float)sqrt(red[0][0] / ((double)j.m * (double)j.n));
   st.offdiag_ratio = j.rho ? *j.rho : -1.0f;
   st.refreshed = bits;
-  st.nonfinite = 0;
+  st.nonfinite = bad;
+  if (bad > 0) report(status, MAO_ERR_NONFINITE, 31, j.index, bad);
 }
 
 }  // namespace mao

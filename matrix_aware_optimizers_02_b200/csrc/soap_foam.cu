@@ -38,6 +38,7 @@ mao_status check_refresh(const mao_refresh& r) {
   if (r.kind == MAO_REFRESH_EVERY_K && r.k < 1) return MAO_ERR_INVALID_ARG;
   if (r.kind == MAO_REFRESH_ADAPTIVE && (r.pf < 1 || !std::isfinite(r.tol))) return MAO_ERR_INVALID_ARG;
   if (r.sort != 0 && r.sort != 1) return MAO_ERR_INVALID_ARG;
+  if (r.lag != 0 && r.lag != 1) return MAO_ERR_INVALID_ARG;
   return MAO_OK;
 }
 
@@ -106,8 +107,12 @@ struct MatBuf {
   size_t Gp, Mp, T1G, T1M, Vtmp, Gh, Mh;  // SOAP (N reuses T1G, T2 reuses Mp)
   size_t Gr, Mr;                          // FOAM (N reuses Gp)
   size_t rowpart, colpart, ctmp, tau;
+  size_t upd;                             // update-statistics slots of the weight-update product
   SideBuf L, R;
 };
+
+// Update-statistics slots of an m x n weight (32-row by 64-column blocks).
+inline int upd_slots(int m, int n) { return ((m + 31) / 32) * ((n + 63) / 64); }
 
 void side_layout(int k, bool check, Carver& cv, SideBuf& s, size_t flag_block) {
   const size_t kk = (size_t)k * k;
@@ -187,6 +192,7 @@ void plan_group_scratch(const Ctx& X, GroupPlan& G, size_t base) {
       b.tau = cv.take(16);
     }
     side_layout(a.n, check, cv, b.R, G.flags + (size_t)128 * (i - G.g0) + 64);
+    b.upd = cv.take(8 * (size_t)upd_slots(a.m, a.n));
   }
   G.scratch = cv.off - base;
 }
@@ -638,29 +644,63 @@ mao_status build_group(Builder& B, GroupPlan& G) {
     B.ops.back().blocks = blk;
     B.ops.back().bytes = bytes;
   }
-  // factor EMAs
-  if (!foam) {
-    TableLaunch& g = B.new_gemm(0, 0, MAO_K_PC_FACTOR);
-    g.pa = g.pb = gpl;
-    for (int i = 0; i < nm; ++i) {
-      const PcMat& a = A(i);
-      const Split3 Fp = B.planes(G.mb[i].L.Fp, a.m, a.m);  // planes of the new L for the refresh
-      MAO_TRY(table_add(g, B.maps, Gop(i), Gop(i), a.m, a.m, a.n, 0, 0, a.L, X.mode != 0 ? &Fp : nullptr, a.m, a.L,
-                        a.m, 1.f - X.b2, X.b2, nullptr));
+  // factor EMAs; with `planes` their epilogue also writes F's planes for the refresh
+  auto factor_products = [&](bool planes) -> mao_status {
+    if (!foam) {
+      TableLaunch& g = B.new_gemm(0, 0, MAO_K_PC_FACTOR);
+      g.pa = g.pb = gpl;
+      for (int i = 0; i < nm; ++i) {
+        const PcMat& a = A(i);
+        const Split3 Fp = B.planes(G.mb[i].L.Fp, a.m, a.m);
+        MAO_TRY(table_add(g, B.maps, Gop(i), Gop(i), a.m, a.m, a.n, 0, 0, a.L, planes ? &Fp : nullptr, a.m, a.L,
+                          a.m, 1.f - X.b2, X.b2, nullptr));
+      }
     }
-  }
-  {
     TableLaunch& g = B.new_gemm(1, 1, MAO_K_PC_FACTOR);
     g.pa = g.pb = gpl;
     for (int i = 0; i < nm; ++i) {
       const PcMat& a = A(i);
       const Split3 Fp = B.planes(G.mb[i].R.Fp, a.n, a.n);
-      MAO_TRY(table_add(g, B.maps, Gop(i), Gop(i), a.n, a.n, a.m, 0, 0, a.R, X.mode != 0 ? &Fp : nullptr, a.n, a.R,
+      MAO_TRY(table_add(g, B.maps, Gop(i), Gop(i), a.n, a.n, a.m, 0, 0, a.R, planes ? &Fp : nullptr, a.n, a.R,
                         a.n, 1.f - X.b2, X.b2, nullptr));
     }
+    return MAO_OK;
+  };
+  const bool lag = X.rf.lag != 0 && X.mode != 0;
+  if (lag) {
+    // The refresh sees the factors before this step's gradient: planes of the old
+    // F, the refresh, then the factor EMAs.
+    size_t off;
+    const int per = foam ? 1 : 2;
+    EwJob* J = B.new_jobs<EwJob>(Op::SPLIT, per * nm, off);
+    int blk = 0;
+    for (int i = 0; i < nm; ++i) {
+      const PcMat& a = A(i);
+      for (int s = 0; s < per; ++s) {
+        const bool right = foam || s == 1;
+        const int k = right ? a.n : a.m;
+        EwJob& j = J[per * i + s];
+        j.a = right ? a.R : a.L;
+        j.pa = B.wp<__nv_bfloat16>(right ? G.mb[i].R.Fp : G.mb[i].L.Fp);
+        j.pstride = B.pstride(k, k);
+        j.rows = k;
+        j.cols = k;
+        j.lda = k;
+        j.ldp = ldp_of(k);
+        j.blk_begin = blk;
+        blk += ew_blocks(k, k);
+      }
+    }
+    B.ops.back().blocks = blk;
+    MAO_TRY(build_refresh(B, G));
+    MAO_TRY(factor_products(false));
+  } else {
+    MAO_TRY(factor_products(X.mode != 0));
   }
   // refresh, or plain planes of the bases
-  if (X.mode != 0) {
+  if (lag) {
+    // done above
+  } else if (X.mode != 0) {
     MAO_TRY(build_refresh(B, G));
   } else {
     size_t off;
@@ -804,6 +844,7 @@ mao_status build_group(Builder& B, GroupPlan& G) {
         const PcMat& a = A(i);
         MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].Mp, a.m, a.n), B.planes(G.mb[i].R.Qp, a.n, a.n), a.m, a.n,
                           a.n, 0, 0, a.W, nullptr, a.n, a.W, a.n, -X.lr, 1.f - X.lr * X.wd, nullptr));
+        MAO_TRY(table_set_stats(g, B.wp<float2>(G.mb[i].upd)));
       }
     }
   } else {
@@ -894,6 +935,7 @@ mao_status build_group(Builder& B, GroupPlan& G) {
         const PcMat& a = A(i);
         MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].Gp, a.m, a.n), B.planes(G.mb[i].R.Qp, a.n, a.n), a.m, a.n,
                           a.n, 0, 0, a.W, nullptr, a.n, a.W, a.n, -X.lr, 1.f - X.lr * X.wd, nullptr));
+        MAO_TRY(table_set_stats(g, B.wp<float2>(G.mb[i].upd)));
       }
     }
   }
@@ -931,7 +973,12 @@ void add_stats_jobs(Builder& B, GroupPlan& G, BuiltGroup& bg) {
   std::memset(static_cast<void*>(S), 0, sizeof(StatsJob) * std::max(nm, 1));
   for (int i = 0; i < nm; ++i) {
     StatsJob& j = S[i];
+    const PcMat& a = B.X.mats[G.g0 + i];
     j.index = G.g0 + i;
+    j.upd = B.wp<float2>(G.mb[i].upd);
+    j.nslots = upd_slots(a.m, a.n);
+    j.m = a.m;
+    j.n = a.n;
     if (B.X.mode == 2) {
       j.flag_r = B.wp<int>(G.mb[i].R.flag);
       j.flag_l = B.X.foam ? nullptr : B.wp<int>(G.mb[i].L.flag);
@@ -1100,7 +1147,7 @@ mao_status make_plan(const Ctx& X, uint8_t* ws, StepPlan& P) {
 struct PlanCache {
   std::mutex mu;
   std::list<std::pair<std::string, std::shared_ptr<StepPlan>>> lru;
-  static constexpr size_t kMax = 8;
+  static constexpr size_t kMax = 16;
 };
 PlanCache& plan_cache() {
   static PlanCache c;
@@ -1177,8 +1224,8 @@ mao_status run_step(const Ctx& X, const void* mats, size_t mats_bytes, void* wor
     if (stats) {
       const int nm = g.g1 - g.g0;
       LaunchScope ls(s, MAO_K_PC_STATS, 0.0, 0.0);
-      pc_stats_kernel<<<(nm + 127) / 128, 128, 0, s>>>(reinterpret_cast<const StatsJob*>(arena_dev + bg.stats_jobs),
-                                                         nm, stats);
+      pc_stats_kernel<<<nm, 256, 0, s>>>(reinterpret_cast<const StatsJob*>(arena_dev + bg.stats_jobs), stats,
+                                         status);
       MAO_CUDA_TRY(cudaGetLastError());
     }
   }

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.mao_version() == 2
+    assert lib.mao_version() == 3
     for s in range(0, 11):
         assert len(lib.mao_status_string(s)) > 0
     assert lib.mao_status_string(999) == b"unknown status"
@@ -160,3 +160,41 @@ def test_pair_kernel_flag_validation(lib):
     assert lib.mao_test_gemm_workspace_size(5 | 32, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_OK
     assert lib.mao_test_gemm_workspace_size(0 | 16, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_ERR_INVALID_ARG
     assert lib.mao_test_gemm_workspace_size(1 | 64, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_ERR_INVALID_ARG
+
+
+def _muon_size(lib, mat, params=None):
+    p = params or L.MuonParams(0.95, 0.02, 0.0, 1e-7, 5, None, 0)
+    size = ctypes.c_size_t(0)
+    st = lib.mao_muon_workspace_size((L.MuonMat * 1)(mat), 1, ctypes.byref(p), ctypes.byref(size))
+    return st, size.value
+
+
+def test_muon_split_and_polar_validation(lib):
+    """A split matrix must divide into equal blocks whose widths keep 16-byte rows (a
+    multiple of 4 fp32, of 8 for a bf16 G); the polar method must be a known one."""
+    F32, BF16 = L.MAO_F32, L.MAO_BF16
+    st, split = _muon_size(lib, L.MuonMat(16, 96, A16, A16, F32, A16, 1, 3))
+    assert st == L.MAO_OK
+    st, whole = _muon_size(lib, L.MuonMat(16, 96, A16, A16, F32, A16))
+    assert st == L.MAO_OK and split != whole  # three 16 x 32 logical matrices, not one 16 x 96
+    assert _muon_size(lib, L.MuonMat(16, 24, A16, A16, F32, A16, 1, 6))[0] == L.MAO_OK     # width 4
+    assert _muon_size(lib, L.MuonMat(16, 48, A16, A16, BF16, A16, 1, 3))[0] == L.MAO_OK    # bf16 width 16
+    assert _muon_size(lib, L.MuonMat(16, 96, A16, A16, F32, A16, 1, 5))[0] == L.MAO_ERR_SHAPE   # 96 % 5
+    assert _muon_size(lib, L.MuonMat(16, 30, A16, A16, F32, A16, 1, 3))[0] == L.MAO_ERR_SHAPE   # width 10
+    assert _muon_size(lib, L.MuonMat(16, 48, A16, A16, BF16, A16, 1, 4))[0] == L.MAO_ERR_SHAPE  # bf16 width 12
+    assert _muon_size(lib, L.MuonMat(15, 32, A16, A16, F32, A16, 2, 1))[0] == L.MAO_ERR_SHAPE   # 15 % 2
+    assert _muon_size(lib, L.MuonMat(16, 32, A16, A16, F32, A16, -1, 1))[0] == L.MAO_ERR_INVALID_ARG
+    assert _muon_size(lib, L.MuonMat(16, 32, A16, A16, F32, A16),
+                      L.MuonParams(0.95, 0.02, 0.0, 1e-7, 5, None, 0, 2))[0] == L.MAO_ERR_INVALID_ARG
+    # the step validates the same way before anything is enqueued
+    assert _muon(lib, [L.MuonMat(16, 96, A16, A16, F32, A16, 1, 5)]) == L.MAO_ERR_SHAPE
+
+
+def test_refresh_lag_validation(lib):
+    m = n = 16
+    mats = (L.SoapMat * 1)(L.SoapMat(m, n, A16, A16, L.MAO_F32, A16, A16, A16, A16, A16, A16, None, None))
+    size = ctypes.c_size_t(0)
+    good = L.SoapParams(0.95, 0.95, 1e-8, 3e-3, 0.0, 1, L.Refresh(L.REFRESH_EVERY_K, 1, 10, 0.1, 1, 1))
+    assert lib.mao_soap_workspace_size(mats, 1, ctypes.byref(good), ctypes.byref(size)) == L.MAO_OK
+    bad = L.SoapParams(0.95, 0.95, 1e-8, 3e-3, 0.0, 1, L.Refresh(L.REFRESH_EVERY_K, 1, 10, 0.1, 1, 2))
+    assert lib.mao_soap_workspace_size(mats, 1, ctypes.byref(bad), ctypes.byref(size)) == L.MAO_ERR_INVALID_ARG
