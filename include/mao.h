@@ -139,8 +139,14 @@ typedef struct {
 
 typedef enum {
   MAO_POLAR_NS = 0,    /* Newton-Schulz with the given coefficients, bf16 operands */
-  MAO_POLAR_EXACT = 1  /* MOP: the polar factor U V^T to fp32 accuracy ("SOAP, Muon, and
-                          Beyond" summary, "Muon vs SOAP Comparison") */
+  MAO_POLAR_EXACT = 1  /* MOP ("SOAP, Muon, and Beyond" summary, "Muon vs SOAP Comparison"):
+                          the polar factor U V^T of each (logical) matrix to fp32 accuracy.
+                          ns_steps and ns_coef are ignored: the library runs 16 Newton-Schulz
+                          iterations in fp32-faithful arithmetic (three bf16 planes per fp32
+                          operand), 11 with (3.4445, -4.7750, 2.0315) that lift every singular
+                          value at least ~2e-7 ||M||_F into [0.23, 1.21], then 5 of
+                          (15/8, -10/8, 3/8), which converge cubically to 1.  Singular values
+                          below ~2e-7 ||M||_F are not resolved (they are fp32 noise there). */
 } mao_polar;
 
 typedef struct {
@@ -342,7 +348,8 @@ typedef enum {
   MAO_K_PC_CHOL = 22,        /* QR panel Cholesky and R^{-1} (fp64, one block per panel) */
   MAO_K_PC_QR_APPLY = 23,    /* QR panel products W R^{-1} (tensor cores) */
   MAO_K_PC_QR_REDUCE = 24,   /* sum of the K-slice partials of the projection coefficients */
-  MAO_K_PC_STATS = 25        /* per-matrix diagnostics of a SOAP / FOAM step */
+  MAO_K_PC_STATS = 25,       /* per-matrix diagnostics of a SOAP / FOAM step */
+  MAO_K_MOP_INIT = 26        /* exact polar factor: fp32 X0 = M / (||M||_F + eps) and its planes (HBM) */
 } mao_kernel_id;
 
 /* What one recorded launch was: its kernel and its algorithmic work (useful

@@ -82,7 +82,7 @@ KERNEL_NAMES = {1: "muon_prep", 2: "muon_scale", 3: "ns_gram", 4: "ns_poly", 5: 
                 7: "muon_colscale", 8: "muon_rowscale", 9: "muon_update", 10: "muon_stats", 11: "split3",
                 12: "gemm_test", 13: "pc_elementwise", 14: "pc_factor", 15: "pc_check", 16: "pc_power",
                 17: "pc_sort", 18: "pc_qr", 19: "pc_rotate", 20: "pc_update", 21: "pc_panel", 22: "pc_chol",
-                23: "pc_qr_apply", 24: "pc_qr_reduce", 25: "pc_stats"}
+                23: "pc_qr_apply", 24: "pc_qr_reduce", 25: "pc_stats", 26: "mop_init"}
 
 # name -> (restype, argtypes)
 SIGNATURES = {

@@ -273,4 +273,28 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   return v;
 }
 
+// Three-plane split of 4 consecutive values, stored as 8-byte groups per plane.
+__device__ __forceinline__ void store_split3x4(float4 x, __nv_bfloat16* base, long long off, long long pstride) {
+  float r[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int q = 0; q < 3; ++q) {
+    __nv_bfloat16 h[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      h[e] = __float2bfloat16_rn(r[e]);
+      r[e] -= __bfloat162float(h[e]);
+    }
+    *reinterpret_cast<uint2*>(base + q * pstride + off) = *reinterpret_cast<const uint2*>(h);
+  }
+}
+
+__device__ __forceinline__ void store_split3(float x, __nv_bfloat16* base, long long off, long long pstride) {
+#pragma unroll
+  for (int q = 0; q < 3; ++q) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    base[q * pstride + off] = h;
+    x -= __bfloat162float(h);
+  }
+}
+
 }  // namespace mao

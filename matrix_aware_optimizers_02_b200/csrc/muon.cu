@@ -27,6 +27,15 @@ namespace {
 constexpr float kDefaultCoef[3] = {3.4445f, -4.7750f, 2.0315f};
 constexpr int kMaxNsSteps = 16;
 
+// The exact polar factor (MOP): a fixed Newton-Schulz schedule run in fp32-faithful
+// arithmetic that converges to U V^T.  kMopGrow quintic steps with the default
+// coefficients lift every singular value of X0 = M / (||M||_F + eps) that is at least
+// ~2e-7 into [0.23, 1.21] (each multiplies a small singular value by 3.4445); kMopConv
+// steps of x -> (15 x - 10 x^3 + 3 x^5) / 8, whose fixed point 1 has zero first and
+// second derivatives (cubic convergence), then take all of them to 1 to fp32 rounding.
+constexpr int kMopGrow = 11, kMopConv = 5, kMopSteps = kMopGrow + kMopConv;
+constexpr float kMopConvCoef[3] = {15.0f / 8.0f, -10.0f / 8.0f, 3.0f / 8.0f};
+
 struct MuonClass {
   int s = 0, l = 0;           // X is s x l
   std::vector<int> mats;      // global matrix indices, in batch order
@@ -35,8 +44,17 @@ struct MuonClass {
   int scale_begin = 0;        // first slot in the scale array
 };
 
+// Per logical matrix buffers of the exact polar factor.
+struct ExactBuf {
+  size_t Xf[2], Xp[2];  // fp32 X (s x ld_l) and its three bf16 planes, ping-pong
+  size_t Af, Ap, Bp;    // fp32 A = X X^T (s x ld_s) and its planes; planes of B
+};
+
 struct MuonPlan {
   std::vector<MuonClass> cls;
+  bool exact = false;
+  std::vector<ExactBuf> ex;
+  size_t off_arena = 0, arena_cap = 0;  // staged problem tables and tensor maps (exact)
   std::vector<int> mat_class, mat_slot;  // class of matrix p, its index in the class
   size_t off_table = 0, off_scale = 0, off_partial = 0, off_rowscale = 0, off_colscale = 0, off_rowpart = 0,
          off_colpart = 0, off_updpart = 0, off_updbad = 0, off_ranges = 0;
@@ -183,7 +201,85 @@ void plan(const mao_muon_mat* mats, int count, const int* ld, int callers, const
     c.off_A = cv.take(2 * cnt * (size_t)c.s * c.ld_s);
     c.off_B = cv.take(2 * cnt * (size_t)c.s * c.ld_s);
   }
+  P.exact = p->polar == MAO_POLAR_EXACT;
+  if (P.exact) {
+    P.ex.assign(count, ExactBuf());
+    for (int i = 0; i < count; ++i) {
+      const MuonClass& C = P.cls[P.mat_class[i]];
+      ExactBuf& e = P.ex[i];
+      for (int k = 0; k < 2; ++k) {
+        e.Xf[k] = cv.take(4 * (size_t)C.s * C.ld_l);
+        e.Xp[k] = cv.take(2 * 3 * (size_t)C.s * C.ld_l);
+      }
+      e.Af = cv.take(4 * (size_t)C.s * C.ld_s);
+      e.Ap = cv.take(2 * 3 * (size_t)C.s * C.ld_s);
+      e.Bp = cv.take(2 * 3 * (size_t)C.s * C.ld_s);
+    }
+    // at most 27 tensor maps per matrix (3 planes of X[2] in three views, of A in two,
+    // of B in one) and one problem per matrix in each of 3 launches per iteration
+    P.arena_cap = (size_t)count * (27 * sizeof(CUtensorMap) + 3 * kMopSteps * sizeof(GemmProblem)) +
+                  (3 * kMopSteps + 1) * 64 + 4096;
+    P.off_arena = cv.take(P.arena_cap);
+  }
   P.total = cv.total();
+}
+
+// The fp32-faithful Newton-Schulz iteration of the exact polar factor, for every
+// logical matrix: per iteration A = X X^T, B = b A + c A A^T, X' = a X + B X as
+// table-mode products (the same arithmetic as the SOAP / FOAM contractions), with
+// the problem tables and tensor maps staged in the workspace's arena.
+mao_status run_exact_iterations(const MuonPlan& P, uint8_t* ws, DevStatus* status, cudaStream_t stream) {
+  const int count = (int)P.ex.size();
+  MapSet maps;
+  std::vector<TableLaunch> launches;
+  launches.reserve(3 * kMopSteps);
+  auto planes = [&](size_t off, int rows, int cols, int ld) {
+    const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(ws + off);
+    const size_t st = (size_t)rows * ld;
+    return Split3{{b, b + st, b + 2 * st}, rows, cols, ld};
+  };
+  for (int it = 0; it < kMopSteps; ++it) {
+    const float* cf = it < kMopGrow ? kDefaultCoef : kMopConvCoef;
+    const int cur = it % 2, nxt = 1 - cur;
+    launches.emplace_back();
+    TableLaunch& g = launches.back();
+    g.kernel_id = MAO_K_NS_GRAM;
+    launches.emplace_back();
+    TableLaunch& q = launches.back();
+    q.kernel_id = MAO_K_NS_POLY;
+    launches.emplace_back();
+    TableLaunch& x = launches.back();
+    x.kernel_id = MAO_K_NS_AXPY;
+    x.b_mn = 1;
+    for (int i = 0; i < count; ++i) {
+      const MuonClass& C = P.cls[P.mat_class[i]];
+      const ExactBuf& e = P.ex[i];
+      const Split3 Xc = planes(e.Xp[cur], C.s, C.l, C.ld_l), Xn = planes(e.Xp[nxt], C.s, C.l, C.ld_l);
+      const Split3 Ap = planes(e.Ap, C.s, C.s, C.ld_s), Bp = planes(e.Bp, C.s, C.s, C.ld_s);
+      float* Af = reinterpret_cast<float*>(ws + e.Af);
+      float* Xfc = reinterpret_cast<float*>(ws + e.Xf[cur]);
+      float* Xfn = reinterpret_cast<float*>(ws + e.Xf[nxt]);
+      // A = X X^T (s x s)
+      MAO_TRY(table_add(g, maps, Xc, Xc, C.s, C.s, C.l, 0, 0, Af, &Ap, C.ld_s, nullptr, 0, 1.f, 0.f, nullptr));
+      // B = c A A^T + b A (A is symmetric)
+      MAO_TRY(table_add(q, maps, Ap, Ap, C.s, C.s, C.s, 0, 0, nullptr, &Bp, C.ld_s, Af, C.ld_s, cf[2], cf[1],
+                        nullptr));
+      // X' = B X + a X (X read as K x N, MN-major)
+      MAO_TRY(table_add(x, maps, Bp, Xc, C.s, C.l, C.s, 0, 0, Xfn, &Xn, C.ld_l, Xfc, C.ld_l, 1.f, cf[0],
+                        nullptr));
+    }
+  }
+  MAO_TRY(maps.encode_all());
+  Arena arena;
+  arena.dev = ws + P.off_arena;
+  const size_t maps_off = arena.take(sizeof(CUtensorMap) * maps.maps.size(), 64);
+  std::memcpy(arena.host.data() + maps_off, maps.maps.data(), sizeof(CUtensorMap) * maps.maps.size());
+  std::vector<StagedLaunch> staged;
+  for (const TableLaunch& L : launches) staged.push_back(table_stage(arena, L, maps_off));
+  if (arena.host.size() > P.arena_cap) return MAO_ERR_WORKSPACE;  // the bound above is wrong: a defect
+  MAO_CUDA_TRY(cudaMemcpyAsync(arena.dev, arena.host.data(), arena.host.size(), cudaMemcpyHostToDevice, stream));
+  for (const StagedLaunch& S : staged) MAO_TRY(table_launch(arena, S, status, stream));
+  return MAO_OK;
 }
 
 }  // namespace
@@ -250,8 +346,15 @@ extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, con
     D.rowpart = rowpart ? rowpart + rp_off : nullptr;
     D.colscale = colscale ? colscale + cs_off : nullptr;
     D.colpart = colpart ? colpart + cp_off : nullptr;
-    D.oscale = (p->ns_steps == 0) ? scale + C.scale_begin + b : nullptr;
+    D.oscale = (p->ns_steps == 0 && !P.exact) ? scale + C.scale_begin + b : nullptr;
     D.scale_slot = C.scale_begin + b;
+    if (P.exact) {
+      const ExactBuf& e = P.ex[i];
+      D.Xe = reinterpret_cast<float*>(ws + e.Xf[0]);
+      D.Xep = reinterpret_cast<__nv_bfloat16*>(ws + e.Xp[0]);
+      D.xep_stride = (long long)C.s * C.ld_l;
+      D.Of = reinterpret_cast<const float*>(ws + e.Xf[kMopSteps % 2]);
+    }
     rs_off += D.m;
     cs_off += D.n;
     rp_off += (size_t)D.tiles_c * D.m;
@@ -284,8 +387,17 @@ extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, con
   }
   MAO_CUDA_TRY(cudaGetLastError());
 
+  // 3 (exact polar factor): fp32 X0 and its planes, then the fp32-faithful iteration
+  if (P.exact) {
+    {
+      LaunchScope ls(stream, MAO_K_MOP_INIT, 0.0, elems * (4.0 + 4.0 + 6.0));
+      mop_init_kernel<<<P.tiles, 256, 0, stream>>>(T, count, scale);
+    }
+    MAO_CUDA_TRY(cudaGetLastError());
+    MAO_TRY(run_exact_iterations(P, ws, status, stream));
+  }
   // 3: Newton-Schulz over every class, at most kMaxClasses per launch
-  if (p->ns_steps > 0) {
+  if (p->ns_steps > 0 && !P.exact) {
     const int ncls = (int)P.cls.size();
     struct ClassMaps {
       CUtensorMap XA[2], XB[2], XMN[2], AA, AB, BA;
@@ -357,9 +469,12 @@ extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, con
   auto norm_pass = [&](int rows_dir, int use_other) -> mao_status {
     {
       LaunchScope ls(stream, rows_dir ? MAO_K_MUON_ROWSCALE : MAO_K_MUON_COLSQ, 0.0, 2.0 * elems);
-      muon_norm_tile_kernel<<<P.tiles, 256, 0, stream>>>(T, count, rows_dir ? 0 : 1, rows_dir ? 1 : 0,
-                                                         (!rows_dir && use_other) ? 1 : 0,
-                                                         (rows_dir && use_other) ? 1 : 0);
+      const int wc = rows_dir ? 0 : 1, wr = rows_dir ? 1 : 0;
+      const int ur = (!rows_dir && use_other) ? 1 : 0, uc = (rows_dir && use_other) ? 1 : 0;
+      if (P.exact)
+        muon_norm_tile_kernel<float><<<P.tiles, 256, 0, stream>>>(T, count, wc, wr, ur, uc);
+      else
+        muon_norm_tile_kernel<__nv_bfloat16><<<P.tiles, 256, 0, stream>>>(T, count, wc, wr, ur, uc);
     }
     MAO_CUDA_TRY(cudaGetLastError());
     dim3 g((maxdim + 255) / 256, count);
@@ -387,8 +502,14 @@ extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, con
   const float decay = 1.0f - p->lr * p->wd;
   {
     LaunchScope ls(stream, MAO_K_MUON_UPDATE, 0.0, elems * (2.0 + 4.0 + 4.0));
-    muon_update_kernel<<<P.tiles, 256, 0, stream>>>(T, count, decay, P.use_rows ? 1 : 0, P.use_cols ? 1 : 0,
-                                                   stats ? updpart : nullptr, stats ? updbad : nullptr);
+    float* up = stats ? updpart : nullptr;
+    int* ub = stats ? updbad : nullptr;
+    if (P.exact)
+      muon_update_kernel<float><<<P.tiles, 256, 0, stream>>>(T, count, decay, P.use_rows ? 1 : 0,
+                                                            P.use_cols ? 1 : 0, up, ub);
+    else
+      muon_update_kernel<__nv_bfloat16><<<P.tiles, 256, 0, stream>>>(T, count, decay, P.use_rows ? 1 : 0,
+                                                                    P.use_cols ? 1 : 0, up, ub);
   }
   MAO_CUDA_TRY(cudaGetLastError());
   if (stats) {

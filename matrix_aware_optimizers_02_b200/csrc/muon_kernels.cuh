@@ -48,6 +48,12 @@ struct MuonMatDev {
   int tiles_r, tiles_c;    // 64 x 64 tiles of the m x n matrix
   int tile_begin;          // first tile (global block index) of this matrix
   float out_scale;         // lr * sqrt(m/n)
+  // exact polar factor (MOP): fp32 X0 = M / (||M||_F + eps) (s x l, ld = ldx) and its
+  // three bf16 planes (plane stride xep_stride), and the final fp32 O; nullptr otherwise
+  float* Xe;
+  __nv_bfloat16* Xep;
+  long long xep_stride;
+  const float* Of;
 };
 
 __device__ __forceinline__ int find_mat(const MuonMatDev* T, int count, int blk) {
@@ -68,15 +74,35 @@ __device__ __forceinline__ void bf16x4_to_float(uint2 raw, float* v) {
 // Tile of O in W's orientation: thread (ty, tx) receives rows r0 + ty + 16 i,
 // columns c0 + 4 tx + e; entries outside the matrix are 0.  `sm` is a 64 x 72
 // bf16 staging tile used for the transposed case (one __syncthreads inside).
-__device__ __forceinline__ void load_o_tile(const MuonMatDev& D, const __nv_bfloat16* X, int r0, int c0,
-                                            float (&v)[4][4], __nv_bfloat16 (*sm)[kTile + 8]) {
+// The staging tile of load_o_tile for O stored as OT (padding keeps rows 16-byte aligned).
+template <typename OT>
+struct OTile {
+  static constexpr int kPad = 16 / (int)sizeof(OT);
+  typedef OT Row[kTile + kPad];
+};
+
+__device__ __forceinline__ void o_to_float4(const float* p, float* v) {
+  const float4 q = *reinterpret_cast<const float4*>(p);
+  v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+}
+__device__ __forceinline__ void o_to_float4(const __nv_bfloat16* p, float* v) {
+  bf16x4_to_float(*reinterpret_cast<const uint2*>(p), v);
+}
+__device__ __forceinline__ float o_to_float(float x) { return x; }
+__device__ __forceinline__ float o_to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename OT>
+__device__ __forceinline__ OT o_zero() { return OT(0.0f); }
+
+template <typename OT>
+__device__ __forceinline__ void load_o_tile(const MuonMatDev& D, const OT* X, int r0, int c0, float (&v)[4][4],
+                                            typename OTile<OT>::Row* sm) {
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   if (!D.trans) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int row = r0 + ty + 16 * i, col = c0 + 4 * tx;
       if (row < D.m && col < D.n) {
-        bf16x4_to_float(*reinterpret_cast<const uint2*>(X + (long long)row * D.ldx + col), v[i]);
+        o_to_float4(X + (long long)row * D.ldx + col, v[i]);
       } else {
         v[i][0] = v[i][1] = v[i][2] = v[i][3] = 0.f;
       }
@@ -86,25 +112,36 @@ __device__ __forceinline__ void load_o_tile(const MuonMatDev& D, const __nv_bflo
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int xr = c0 + ty + 16 * i, xc = r0 + 4 * tx;
-      const __nv_bfloat16* src = X + (long long)xr * D.ldx + xc;
+      const OT* src = X + (long long)xr * D.ldx + xc;
       if (xr < D.n && xc + 4 <= D.m) {
-        uint2 raw = *reinterpret_cast<const uint2*>(src);
-        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&raw);
+        OT h[4];
+        if constexpr (sizeof(OT) == 2) {
+          *reinterpret_cast<uint2*>(h) = *reinterpret_cast<const uint2*>(src);
+        } else {
+          *reinterpret_cast<float4*>(h) = *reinterpret_cast<const float4*>(src);
+        }
 #pragma unroll
         for (int e = 0; e < 4; ++e) sm[ty + 16 * i][4 * tx + e] = h[e];
       } else {
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          sm[ty + 16 * i][4 * tx + e] = (xr < D.n && xc + e < D.m) ? src[e] : __float2bfloat16_rn(0.f);
+          sm[ty + 16 * i][4 * tx + e] = (xr < D.n && xc + e < D.m) ? src[e] : o_zero<OT>();
       }
     }
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) v[i][e] = __bfloat162float(sm[4 * tx + e][ty + 16 * i]);
+      for (int e = 0; e < 4; ++e) v[i][e] = o_to_float(sm[4 * tx + e][ty + 16 * i]);
   }
 }
+
+template <typename OT>
+__device__ __forceinline__ const OT* o_of(const MuonMatDev& D);
+template <>
+__device__ __forceinline__ const __nv_bfloat16* o_of<__nv_bfloat16>(const MuonMatDev& D) { return D.O; }
+template <>
+__device__ __forceinline__ const float* o_of<float>(const MuonMatDev& D) { return D.Of; }
 
 // ------------------------------------------------------------------ prep
 __global__ void __launch_bounds__(256) muon_prep_kernel(const MuonMatDev* __restrict__ T, int count, float mu,
@@ -190,6 +227,61 @@ __global__ void __launch_bounds__(256) muon_prep_kernel(const MuonMatDev* __rest
   }
 }
 
+// ------------------------------------------------------------------ exact polar factor
+// X0 = s M (s = 1 / (||M||_F + eps) from muon_scale_kernel) in fp32, transposed for a
+// tall matrix, and its three bf16 planes: the operand of the fp32-faithful iteration.
+// One 64 x 64 tile of the m x n matrix per block, as muon_prep_kernel.
+__global__ void __launch_bounds__(256) mop_init_kernel(const MuonMatDev* __restrict__ T, int count,
+                                                       const float* __restrict__ scale) {
+  __shared__ float tileT[kTile][kTile + 1];
+  const MuonMatDev& D = T[find_mat(T, count, blockIdx.x)];
+  const int local = blockIdx.x - D.tile_begin;
+  const int r0 = (local / D.tiles_c) * kTile, c0 = (local % D.tiles_c) * kTile;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int col = c0 + 4 * tx;
+  const float sc = scale[D.scale_slot];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rl = ty + 16 * i, row = r0 + rl;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row < D.m && col < D.n) {
+      x = *reinterpret_cast<const float4*>(D.M + (long long)row * D.ld + col);
+      x = make_float4(sc * x.x, sc * x.y, sc * x.z, sc * x.w);
+      if (!D.trans) {
+        const long long o = (long long)row * D.ldx + col;
+        *reinterpret_cast<float4*>(D.Xe + o) = x;
+        store_split3x4(x, D.Xep, o, D.xep_stride);
+      }
+    }
+    if (D.trans) {
+      tileT[4 * tx + 0][rl] = x.x;
+      tileT[4 * tx + 1][rl] = x.y;
+      tileT[4 * tx + 2][rl] = x.z;
+      tileT[4 * tx + 3][rl] = x.w;
+    }
+  }
+  if (!D.trans) return;
+  __syncthreads();
+  // X row = column of M: rows c0 + cl, columns r0 + 4 tx .. (m need not be a multiple of 4)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int cl = ty + 16 * i, xrow = c0 + cl, xcol = r0 + 4 * tx;
+    if (xrow >= D.n) continue;
+    const long long o = (long long)xrow * D.ldx + xcol;
+    if (xcol + 4 <= D.m) {
+      const float4 x = make_float4(tileT[cl][4 * tx], tileT[cl][4 * tx + 1], tileT[cl][4 * tx + 2],
+                                   tileT[cl][4 * tx + 3]);
+      *reinterpret_cast<float4*>(D.Xe + o) = x;
+      store_split3x4(x, D.Xep, o, D.xep_stride);
+    } else {
+      for (int e = 0; e < 4 && xcol + e < D.m; ++e) {
+        D.Xe[o + e] = tileT[cl][4 * tx + e];
+        store_split3(tileT[cl][4 * tx + e], D.Xep, o + e, D.xep_stride);
+      }
+    }
+  }
+}
+
 // One warp per matrix.
 __global__ void muon_scale_kernel(const MuonMatDev* __restrict__ T, int count, const float* __restrict__ partial,
                                   float eps, float* __restrict__ scale) {
@@ -208,10 +300,12 @@ __global__ void muon_scale_kernel(const MuonMatDev* __restrict__ T, int count, c
 // want_cols: write column partials (sum over the tile's rows of (O rs)^2)
 // want_rows: write row partials (sum over the tile's columns of (O cs)^2)
 // use_rows / use_cols: apply rowscale / colscale before squaring.
+// OT: element type of O (bf16 after Newton-Schulz, fp32 for the exact polar factor).
+template <typename OT>
 __global__ void __launch_bounds__(256) muon_norm_tile_kernel(const MuonMatDev* __restrict__ T, int count,
                                                              int want_cols, int want_rows, int use_rows,
                                                              int use_cols) {
-  __shared__ __nv_bfloat16 sm[kTile][kTile + 8];
+  __shared__ __align__(16) typename OTile<OT>::Row sm[kTile];
   __shared__ float csum[16][kTile];
   const MuonMatDev& D = T[find_mat(T, count, blockIdx.x)];
   const int local = blockIdx.x - D.tile_begin;
@@ -219,7 +313,7 @@ __global__ void __launch_bounds__(256) muon_norm_tile_kernel(const MuonMatDev* _
   const int r0 = tr * kTile, c0 = tc * kTile;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   float v[4][4];
-  load_o_tile(D, D.O, r0, c0, v, sm);
+  load_o_tile<OT>(D, o_of<OT>(D), r0, c0, v, sm);
   const float om = D.oscale ? *D.oscale : 1.0f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -278,11 +372,12 @@ __global__ void muon_norm_final_kernel(const MuonMatDev* __restrict__ T, int cou
 }
 
 // ------------------------------------------------------------------ update
+template <typename OT>
 __global__ void __launch_bounds__(256) muon_update_kernel(const MuonMatDev* __restrict__ T, int count,
                                                           float decay, int use_rows, int use_cols,
                                                           float* __restrict__ upd_partial,
                                                           int* __restrict__ upd_nonfinite) {
-  __shared__ __nv_bfloat16 sm[kTile][kTile + 8];
+  __shared__ __align__(16) typename OTile<OT>::Row sm[kTile];
   __shared__ float wsum[8];
   __shared__ int wbad[8];
   const MuonMatDev& D = T[find_mat(T, count, blockIdx.x)];
@@ -290,7 +385,7 @@ __global__ void __launch_bounds__(256) muon_update_kernel(const MuonMatDev* __re
   const int r0 = (local / D.tiles_c) * kTile, c0 = (local % D.tiles_c) * kTile;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   float v[4][4];
-  load_o_tile(D, D.O, r0, c0, v, sm);
+  load_o_tile<OT>(D, o_of<OT>(D), r0, c0, v, sm);
   const float om = D.oscale ? *D.oscale : 1.0f;
   const int col = c0 + 4 * tx;
   float cs[4] = {1.f, 1.f, 1.f, 1.f};

@@ -181,6 +181,34 @@ def kronecker_gradients(rng: np.random.Generator, m: int, n: int, Q: np.ndarray,
     return Gs, a, b, ks
 
 
+def drifting_spike_gradients(rng: np.random.Generator, m: int, n: int, steps: int, rank: int = 4,
+                             spike: float = 0.05, noise_std: float = 1e-3, omega: float = 0.05):
+    """A low-rank spike whose singular subspaces rotate slowly, plus noise, one G per step.
+
+    Fixed orthonormal U0 (m x 2 rank) and V0 (n x 2 rank); at step t (1-based) the
+    spike's k-th left vector is cos(omega t) U0[:, k] + sin(omega t) U0[:, rank + k]
+    (the same for the right vectors with V0), its singular value spike * (1 + k / rank),
+    and N(0, noise_std^2) noise is added.  Each direction turns by omega radians per
+    step, a quarter turn in pi / (2 omega) steps: a basis computed from older
+    gradients points away from the current ones.  Returns (list of float32 G_t,
+    function t -> (U_t, V_t) of the spike's directions).
+    """
+    U0 = random_orthogonal(rng, m)[:, :2 * rank]
+    V0 = random_orthogonal(rng, n)[:, :2 * rank]
+    sv = spike * (1.0 + np.arange(rank) / rank)
+
+    def dirs(t):
+        c, s = np.cos(omega * t), np.sin(omega * t)
+        return c * U0[:, :rank] + s * U0[:, rank:], c * V0[:, :rank] + s * V0[:, rank:]
+
+    Gs = []
+    for t in range(1, steps + 1):
+        U, V = dirs(t)
+        G = (U * sv[None, :]) @ V.T + rng.standard_normal((m, n)) * noise_std
+        Gs.append(G.astype(np.float32))
+    return Gs, dirs
+
+
 def random_orthogonal(rng: np.random.Generator, n: int) -> np.ndarray:
     """Haar-like orthogonal matrix from the QR of a Gaussian matrix (sign-fixed)."""
     Z = rng.standard_normal((n, n))

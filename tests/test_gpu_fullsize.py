@@ -1,0 +1,187 @@
+"""Parity at the full sizes of the benchmarked layer sets, through the C ABI, in the
+launch configuration the benchmark uses (bf16 gradients, refresh every step, sorted).
+
+* Muon on the 8B block's 4096 x 14336 and 14336 x 4096 matrices (Newton-Schulz at
+  s = 4096, K = 14336) and on a MoE expert triple at the extremes of its gradient
+  scale (s_e = 0.1 and 10): the float64 oracle in full.
+* SOAP on the MoE expert triple at s_e = 0.1 and 10, t = 1 and 2: the oracle in full
+  (gates of test_gpu_soap_foam).
+* SOAP on the 8B block's 4096 x 14336 and 14336 x 4096 matrices, t = 1 and 2.  A
+  float64 QR of the 14336 x 14336 factor takes minutes on the host, so the refreshed
+  basis is checked by the properties that define it, on 96 sampled columns:
+    - orthonormal columns: ||Q^T q_j - e_j|| <= 1e-4;
+    - Q is the positive-diagonal QR factor of P = F Q_prev[:, perm] with the oracle's
+      F: the part of P_j outside span(q_1..q_j) and the entries (Q^T P)_ij below the
+      diagonal stay below 1e-4 ||P_j||, and (Q^T P)_jj > 0 — for a full-rank P this
+      fixes Q uniquely (it equals any exact QR of P up to the fp32 backward error);
+    - the permutation equals the oracle's sort of diag(Q_prev^T F Q_prev) at every
+      position whose keys differ by more than 1e-5 relative.
+  The factors L, R and the moment M are compared with the oracle in full, and the
+  oracle's S5-S8 (soap_precondition) run in the device's validated bases give V and
+  the weight update, at the gates of test_gpu_soap_foam.
+* FOAM on the GPT-2-760M-shaped 6144 x 1536 and 1536 x 4608 matrices through an
+  adaptive check (t = 1 checks and refreshes, t = 2 is a plain step): the oracle in full.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from matrix_aware_optimizers_02_b200 import synth
+from oracle import mao_oracle as O
+from tests import gates
+from tests import test_gpu_soap_foam as P
+
+pytestmark = pytest.mark.gpu
+
+NS_TOL = 2e-2
+STATE_TOL = 1e-4
+SAMPLES = 96
+
+
+@pytest.fixture(scope="module")
+def api():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from matrix_aware_optimizers_02_b200 import api as A
+    return A
+
+
+def _np(x):
+    return x.double().cpu().numpy()
+
+
+# ------------------------------------------------------------------ Muon
+
+@pytest.mark.parametrize("shape", [(4096, 14336), (14336, 4096)])
+def test_muon_dense8b_full_size(api, shape):
+    m, n = shape
+    rng = np.random.default_rng(50)
+    W = (rng.standard_normal((m, n)) * 0.02).astype(np.float32)
+    G = synth.bf16_round((rng.standard_normal((m, n)) * 0.01).astype(np.float32)).astype(np.float32)
+    M = np.zeros((m, n), np.float32)
+    dev = [(torch.from_numpy(W).cuda(), torch.from_numpy(G).cuda().to(torch.bfloat16), torch.from_numpy(M).cuda())]
+    b = api.MuonBatch(dev, mu=0.95, lr=0.02, with_stats=True)
+    b()
+    assert b.device_status() == 0
+    Wg = _np(dev[0][0])
+    Wo, _, _ = O.muon_step(W.astype(np.float64), G.astype(np.float64), M.astype(np.float64), mu=0.95, lr=0.02)
+    dW, ref = Wg - W, Wo - W
+    lab = f"muon full {m}x{n}"
+    gates.check(lab, "muon dW (full size)", gates.rel(dW, ref), NS_TOL)
+    gates.check(lab, "muon dW max/rms (full size)", gates.max_over_rms(dW, ref), 10 * NS_TOL)
+    rms = float(np.linalg.norm(ref) / np.sqrt(m * n))
+    gates.check(lab, "muon update_rms (full size)", abs(b.stats_dict()["update_rms"][0] - rms) / rms, NS_TOL)
+
+
+@pytest.mark.parametrize("s_e", [0.1, 10.0])
+def test_muon_moe_expert_scales(api, s_e):
+    shapes = [(2048, 768), (2048, 768), (768, 2048)]
+    rng = np.random.default_rng(51)
+    inputs = []
+    for (m, n) in shapes:
+        W = (rng.standard_normal((m, n)) * 0.02).astype(np.float32)
+        G = synth.bf16_round((rng.standard_normal((m, n)) * 0.01 * s_e).astype(np.float32)).astype(np.float32)
+        inputs.append((W, G, np.zeros((m, n), np.float32)))
+    dev = [(torch.from_numpy(W).cuda(), torch.from_numpy(G).cuda().to(torch.bfloat16), torch.from_numpy(M).cuda())
+           for (W, G, M) in inputs]
+    b = api.MuonBatch(dev, mu=0.95, lr=0.02)
+    b()
+    assert b.device_status() == 0
+    for i, ((W, G, M), d) in enumerate(zip(inputs, dev)):
+        Wo, _, _ = O.muon_step(W.astype(np.float64), G.astype(np.float64), M.astype(np.float64), mu=0.95, lr=0.02)
+        dW, ref = _np(d[0]) - W, Wo - W
+        lab = f"muon expert s_e={s_e} #{i}"
+        gates.check(lab, "muon dW (expert scales)", gates.rel(dW, ref), NS_TOL)
+        gates.check(lab, "muon dW max/rms (expert scales)", gates.max_over_rms(dW, ref), 10 * NS_TOL)
+
+
+# ------------------------------------------------------------------ SOAP, MoE expert triple
+
+@pytest.mark.parametrize("s_e", [0.1, 10.0])
+def test_soap_moe_expert_scales(api, s_e):
+    P._soap_case(api, [(2048, 768), (2048, 768), (768, 2048)], steps=2, seed=52, g_scale=0.01 * s_e, g_bf16=True,
+                 label=f"soap expert s_e={s_e}")
+
+
+# ------------------------------------------------------------------ SOAP, 8B block matrices
+
+def _basis_properties(lab, Q, F, Qprev, perm, rng):
+    """Sampled checks that Q is the positive-diagonal QR factor of F Qprev[:, perm]."""
+    k = Q.shape[0]
+    cols = np.unique(np.concatenate([[0, 1, k // 2, k - 2, k - 1], rng.choice(k, SAMPLES, replace=False)]))
+    QtQ = Q.T @ Q[:, cols]
+    orth = np.linalg.norm(QtQ - np.eye(k)[:, cols], axis=0)
+    gates.check(lab, "soap basis orthonormality (sampled)", float(orth.max()), STATE_TOL)
+    Pc = F @ Qprev[:, perm[cols]]                      # sampled columns of P
+    R = Q.T @ Pc                                       # (Q^T P)[:, cols]
+    pn = np.linalg.norm(Pc, axis=0)
+    below = np.array([np.linalg.norm(R[j + 1:, c]) for c, j in enumerate(cols)]) / pn
+    gates.check(lab, "soap basis QR residual (sampled)", float(below.max()), STATE_TOL)
+    assert np.all(R[cols, np.arange(len(cols))] > 0), lab
+
+
+def _perm_vs_keys(lab, perm_gpu, F, Qprev):
+    """The device's sort equals the oracle's at every well-separated position."""
+    keys = O.rayleigh_keys(F, Qprev)
+    perm_or = O.sort_perm(keys)
+    ks = keys[perm_or]
+    P._perm_check(perm_gpu, perm_or, ks)
+
+
+@pytest.mark.parametrize("shape", [(4096, 14336), (14336, 4096)])
+def test_soap_dense8b_full_size(api, shape):
+    m, n = shape
+    rng = np.random.default_rng(53)
+    W = (rng.standard_normal((m, n)) * 0.02).astype(np.float32)
+    st = O.SoapState.init(m, n)
+    t32 = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()  # noqa: E731
+    d = {"W": t32(W), "G": torch.zeros((m, n), dtype=torch.bfloat16, device="cuda"), "M": t32(st.M),
+         "V": t32(st.V), "L": t32(st.L), "R": t32(st.R), "QL": t32(st.QL), "QR": t32(st.QR),
+         "perm_L": torch.zeros(m, dtype=torch.int32, device="cuda"),
+         "perm_R": torch.zeros(n, dtype=torch.int32, device="cuda")}
+    batch = api.SoapBatch([d], beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3, with_stats=True)
+    L, R, Mprev, V = st.L, st.R, st.M, st.V
+    QLp, QRp = np.eye(m), np.eye(n)
+    Wprev = W.astype(np.float64)
+    srng = np.random.default_rng(54)
+    for t in (1, 2):
+        G = synth.bf16_round((rng.standard_normal((m, n)) * 0.01).astype(np.float32)).astype(np.float64)
+        d["G"].copy_(torch.from_numpy(G.astype(np.float32)).to(torch.bfloat16))
+        batch(t)
+        assert batch.device_status() == 0
+        torch.cuda.synchronize()
+        lab = f"soap full {m}x{n} t={t}"
+        L, R = O.soap_factors(L, R, G, 0.95)
+        M_or = 0.95 * Mprev + 0.05 * G
+        P._compare(lab, "soap L (full size)", _np(d["L"]), L, STATE_TOL)
+        P._compare(lab, "soap R (full size)", _np(d["R"]), R, STATE_TOL)
+        P._compare(lab, "soap M (full size)", _np(d["M"]), M_or, STATE_TOL)
+        pl, pr = d["perm_L"].cpu().numpy(), d["perm_R"].cpu().numpy()
+        QL, QR = _np(d["QL"]), _np(d["QR"])
+        _perm_vs_keys(lab + " L", pl, L, QLp)
+        _perm_vs_keys(lab + " R", pr, R, QRp)
+        _basis_properties(lab + " L", QL, L, QLp, pl, srng)
+        _basis_properties(lab + " R", QR, R, QRp, pr, srng)
+        # S5-S8 in the device's validated bases; V follows the device's permutations
+        Vp = V[pl, :][:, pr]
+        kw = dict(t=t, beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3)
+        Wn, M, V, _ = O.soap_precondition(Wprev, G, Mprev, Vp, QL, QR, **kw)
+        Wn32, _, _, _ = O.soap_precondition(Wprev, G, Mprev, Vp, QL, QR, dtype=np.float32, **kw)
+        Mprev = M
+        Wg = _np(d["W"])
+        P._compare(lab, "soap V (full size)", _np(d["V"]), V, STATE_TOL)
+        ref, ref32 = Wn - Wprev, Wn32.astype(np.float64) - Wprev
+        gate = max(STATE_TOL, 2 * gates.rel(ref32, ref))
+        P._compare(lab, "soap dW (full size)", Wg - Wprev, ref, gate, ref32)
+        rms = float(np.linalg.norm(ref) / np.sqrt(m * n))
+        gates.check(lab, "soap update_rms (full size)", abs(batch.stats_dict()["update_rms"][0] - rms) / rms, gate)
+        # continue from the device's weight and bases (the oracle's own factors and moments)
+        QLp, QRp, Wprev = QL, QR, Wg
+
+
+# ------------------------------------------------------------------ FOAM, GPT-2-760M shapes
+
+def test_foam_gpt2_760m_shapes_adaptive(api):
+    P._foam_case(api, [(6144, 1536), (1536, 4608)], steps=2, seed=55, refresh="adaptive", pf=10, tol=0.1,
+                 label="foam 760m shapes")

@@ -123,17 +123,19 @@ def _gdev(G, g_bf16):
 
 def _soap_case(api, shapes, steps, seed, eps=1e-8, g_scale=1e-3, lr=3e-3, refresh="every_k", k=1, sort=True,
                g_bf16=False, kernel="auto", wd=0.0, replay=True, pf=10, tol=0.1, lag=False, grads=None,
-               label=None):
+               label=None, probe=None):
+    """`grads(t)` (optional) gives the step's gradients; `probe(t, dev)` (optional) sees the
+    device tensors after each step."""
     api.set_table_kernel(kernel)
     try:
         _soap_run(api, shapes, steps, seed, eps, g_scale, lr, refresh, k, sort, g_bf16, wd, replay, pf, tol, lag,
-                  grads, label or f"soap{shapes}s{seed}")
+                  grads, label or f"soap{shapes}s{seed}", probe)
     finally:
         api.set_table_kernel("auto")
 
 
 def _soap_run(api, shapes, steps, seed, eps, g_scale, lr, refresh, k, sort, g_bf16, wd, replay, pf, tol, lag,
-              grads, label):
+              grads, label, probe=None):
     rng = np.random.default_rng(seed)
     b1 = b2 = 0.95
     dev, ora, ora32, Ws, Ws32 = [], [], [], [], []
@@ -165,6 +167,8 @@ def _soap_run(api, shapes, steps, seed, eps, g_scale, lr, refresh, k, sort, g_bf
         batch(t)
         assert batch.device_status() == 0
         torch.cuda.synchronize()
+        if probe is not None:
+            probe(t, dev)
         stats = batch.stats_dict()
         for i, (m, n) in enumerate(shapes):
             d = dev[i]
@@ -296,17 +300,17 @@ def _soap_single(api, W0, grads, steps, replay):
 
 def _foam_case(api, shapes, steps, seed, refresh="adaptive", pf=10, tol=0.1, eps=1e-8, lr=3e-3, k=1,
                raw_trace=False, g_bf16=False, kernel="auto", wd=0.0, replay=True, lag=False, g_scale=0.01,
-               label=None):
+               label=None, grads=None):
     api.set_table_kernel(kernel)
     try:
         _foam_run(api, shapes, steps, seed, refresh, pf, tol, eps, lr, k, raw_trace, g_bf16, wd, replay, lag,
-                  g_scale, label or f"foam{shapes}s{seed}")
+                  g_scale, label or f"foam{shapes}s{seed}", grads)
     finally:
         api.set_table_kernel("auto")
 
 
 def _foam_run(api, shapes, steps, seed, refresh, pf, tol, eps, lr, k, raw_trace, g_bf16, wd, replay, lag, g_scale,
-              label):
+              label, grads=None):
     rng = np.random.default_rng(seed)
     b1 = b2 = 0.95
     dev, ora, Ws = [], [], []
@@ -323,7 +327,7 @@ def _foam_run(api, shapes, steps, seed, refresh, pf, tol, eps, lr, k, raw_trace,
     seen_at = [None] * len(shapes)  # gradients R had taken in at its last refresh
     gpu_prev = [w.copy() for w in Ws]
     for t in range(1, steps + 1):
-        Gs = [_grad(rng, s, g_scale, g_bf16) for s in shapes]
+        Gs = grads(t) if grads is not None else [_grad(rng, s, g_scale, g_bf16) for s in shapes]
         for d, G in zip(dev, Gs):
             d["G"].copy_(_gdev(G, g_bf16))
         batch(t)
