@@ -53,6 +53,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
+    ap.add_argument("--mode", choices=["sets", "layerwise"], default="sets",
+                    help="sets: every rank steps its own layer set (weak scaling, no collective); layerwise: one "
+                         "layer set split over the ranks by owner, updated weights exchanged by all-gather-V "
+                         "(strong scaling)")
     ap.add_argument("--workload", default="dense8b_moe", choices=sorted(WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--optimizers", default="muon,soap,foam", help="comma list of muon, soap, foam")
@@ -489,6 +493,103 @@ class LayerSet:
         return None
 
 
+class LayerwiseSet:
+    """One layer set split over the ranks by the layer-wise optimizer (whole matrices
+    owned by ranks, balanced by the cost model; the updated weights exchanged by the
+    all-gather-V).  Every rank holds W and the gradient sets in full (identical on all
+    ranks, as after a data-parallel gradient all-reduce) and optimizer state only for
+    the matrices it owns.  Same interface as LayerSet."""
+
+    def __init__(self, specs, seed, dev, g_bf16, optimizers, norm, dist, soap_k=1, n_grad=3):
+        import torch
+
+        from matrix_aware_optimizers_02_b200 import api, synth
+        from matrix_aware_optimizers_02_b200 import layerwise as LW
+        self.torch = torch
+        base = synth.torch_muon_inputs(specs, seed, dev, g_bf16=g_bf16)
+        self.W = [w for (w, _, _) in base]
+        self.G_sets = [[g for (_, g, _) in base]]
+        del base
+        gen = torch.Generator(device=dev)
+        for k in range(1, n_grad):
+            gen.manual_seed(seed * 1000003 + k)
+            self.G_sets.append([synth.torch_gaussian((sp.m, sp.n), sp.g_std * sp.g_scale, gen, dev,
+                                                     torch.bfloat16 if g_bf16 else torch.float32) for sp in specs])
+        self.G = self.G_sets[0]
+        self.n_grad = n_grad
+        world, rank = dist.get_world_size(), dist.get_rank()
+        kws = {"muon": dict(mu=0.95, lr=0.02, norm=norm),
+               "soap": dict(beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3, refresh="every_k", k=soap_k),
+               "foam": dict(beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3, refresh="adaptive", pf=10, tol=0.1)}
+        shapes = [(sp.m, sp.n) for sp in specs]
+        z = torch.zeros
+        self.order = [o for o in ("muon", "soap", "foam") if o in optimizers]
+        self.steps, self.owners, self.owned_count = {}, {}, {}
+        batches = []
+        for o in self.order:
+            owners = LW.assign_owners(shapes, world, o, LW.cost_for(o, kws[o]))
+            self.owners[o] = owners
+            mine = [i for i, r in enumerate(owners) if r == rank]
+            self.owned_count[o] = len(mine)
+            state = {}
+            for i in mine:
+                m, n = shapes[i]
+                if o == "muon":
+                    state[i] = {"M": z((m, n), device=dev)}
+                elif o == "soap":
+                    state[i] = {"M": z((m, n), device=dev), "V": z((m, n), device=dev),
+                                "L": torch.eye(m, device=dev) * 1e-6, "R": torch.eye(n, device=dev) * 1e-6,
+                                "QL": torch.eye(m, device=dev), "QR": torch.eye(n, device=dev)}
+                else:
+                    state[i] = {"M": z((m, n), device=dev), "r": z(m, device=dev), "c": z(n, device=dev),
+                                "R": torch.eye(n, device=dev) * 1e-6, "QR": torch.eye(n, device=dev)}
+            exchange = LW.AllGatherV(self.W, owners, dist)
+            per_set = []
+            for Gs in self.G_sets:
+                if o == "muon":
+                    mats = [(self.W[i], Gs[i], state[i]["M"] if i in state else None) for i in range(len(specs))]
+                else:
+                    mats = [dict(state.get(i, {}), W=self.W[i], G=Gs[i]) for i in range(len(specs))]
+
+                def make_batch(owned, o=o):
+                    b = {"muon": api.MuonBatch, "soap": api.SoapBatch, "foam": api.FoamBatch}[o](
+                        owned, with_stats=True, allocate=False, **kws[o])
+                    batches.append(b)
+                    return b
+                per_set.append(LW.LayerwiseStep(mats, o, dist, make_batch=make_batch, grads_reduced=True,
+                                                exchange=exchange, **kws[o]))
+            self.steps[o] = per_set
+        ws_bytes = max([b.ws_bytes for b in batches] + [256])
+        self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        for b in batches:
+            b.attach_workspace(self.workspace)
+        self._dummy_stats = torch.zeros((1, 4), dtype=torch.float32, device=dev)
+
+    def step(self, t, stream, events=None):
+        gi = (t - 1) % self.n_grad
+        for name in self.order:
+            lw = self.steps[name][gi]
+            if events is not None:
+                events[name][0].record(stream)
+            if name == "muon":
+                lw()
+            else:
+                lw(t)
+            if events is not None:
+                events[name][1].record(stream)
+
+    def stats_tensor(self, t):
+        b = self.steps[self.order[0]][(t - 1) % self.n_grad].batch
+        return b.stats if b is not None else self._dummy_stats
+
+    def status(self):
+        for name in self.order:
+            b = self.steps[name][0].batch
+            if b is not None and b.device_status() != 0:
+                return name, b.device_status()
+        return None
+
+
 # ----------------------------------------------------------------------------- main (mine)
 def run_mine(args, rank, world, dist):
     import torch
@@ -502,7 +603,13 @@ def run_mine(args, rank, world, dist):
     specs = specs_for(args.workload, args.seed)
     optimizers = [o.strip() for o in args.optimizers.split(",") if o.strip()]
     norm = MUON_NORM.get(args.workload, "none")
-    LS = LayerSet(specs, rank_seed(args.seed, rank), dev, g_bf16, optimizers, norm, soap_k=args.soap_k)
+    layerwise = args.mode == "layerwise"
+    if layerwise:
+        if dist is None:
+            raise SystemExit("--mode layerwise needs a process group (run under torchrun)")
+        LS = LayerwiseSet(specs, args.seed, dev, g_bf16, optimizers, norm, dist, soap_k=args.soap_k)
+    else:
+        LS = LayerSet(specs, rank_seed(args.seed, rank), dev, g_bf16, optimizers, norm, soap_k=args.soap_k)
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -658,14 +765,14 @@ def run_mine(args, rank, world, dist):
     n_elems = sum(s.m * s.n for s in specs)
     line = {
         "metric": "Muon/SOAP/FOAM step ms per layer set; % of tensor-core peak and HBM GB/s",
-        "value": round(per_layer_set(ms_max, world), 4),
+        "value": round(per_layer_set(ms_max, 1 if layerwise else world), 4),
         "unit": "ms",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms_max, 4),
         "higher_is_better": False,
-        "scaling": "weak",
+        "scaling": "strong" if layerwise else "weak",
         "vs_baseline": None,
         "dtype": "bf16 operands / fp32 accumulate (Newton-Schulz); fp32-faithful split-bf16 products and fp32 "
                  "states (SOAP, FOAM)",
@@ -681,11 +788,14 @@ def run_mine(args, rank, world, dist):
                    "matrices_per_rank": len(specs), "elements_per_rank": n_elems,
                    "gradient_sets": 3,
                    "inputs": "three device-resident seeded gradient sets, step t uses set (t - 1) mod 3",
-                   "l2_policy": "inputs larger than L2 (no flush)", "parallelism": f"independent layer sets x{world}"},
+                   "l2_policy": "inputs larger than L2 (no flush)",
+                   "parallelism": (f"layer-wise: one layer set, matrices owned by {world} ranks, all-gather-V of the "
+                                   "updated weights" if layerwise else f"independent layer sets x{world}")},
         "roofline": roof,
         "kernels": kernels,
         "cpu_baseline": cpu,
-        "e2e": {"value": round(per_layer_set(e2e_max, world), 4), "unit": "ms", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": round(per_layer_set(e2e_max, 1 if layerwise else world), 4), "unit": "ms",
+                "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": int(n_launch),
         "clocks": clk,
@@ -828,13 +938,21 @@ def main():
             print(json.dumps(line), flush=True)
         return 0
     dist = None
-    if world > 1:
+    if world > 1 or args.mode == "layerwise":
         import datetime
 
         import torch
         import torch.distributed as D
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-        D.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        if "MASTER_ADDR" in os.environ:
+            D.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        else:  # one process without torchrun: a one-rank group
+            import socket
+            with socket.socket() as sk:
+                sk.bind(("127.0.0.1", 0))
+                port = sk.getsockname()[1]
+            D.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                 timeout=datetime.timedelta(seconds=120))
         dist = D
     try:
         line = run_mine(args, rank, world, dist)

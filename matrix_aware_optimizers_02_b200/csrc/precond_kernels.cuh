@@ -314,6 +314,7 @@ __global__ void __launch_bounds__(256) soap_vperm_kernel(const VPermJob* __restr
 // dependent columns, and asks for a second pass, which restores orthogonality; the
 // triangular structure makes the final Q the positive-diagonal QR factor either way.
 constexpr int kPanel = 128;
+constexpr int kSuper = 2 * kPanel;  // columns projected together against the finished ones
 constexpr int kPanelSq = kPanel * kPanel;
 constexpr int kPackedUpper = kPanel * (kPanel + 1) / 2;  // packed upper triangle, row-major
 constexpr int kMaxParts = 16;                             // K slices of a panel Gram
@@ -643,11 +644,11 @@ __global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restr
 // kPanel fp32 each, in slice order), written as three bf16 planes (ld kPanel).
 // 1024 elements per block.
 struct CoefJob {
-  const float* part;      // nparts partials, part_stride elements apart
-  __nv_bfloat16* cp;      // planes (plane stride pstride)
+  const float* part;      // nparts partials, part_stride elements apart (rows x ld each)
+  __nv_bfloat16* cp;      // planes (plane stride pstride, ld ld)
   long long part_stride, pstride;
   const int* flag;
-  int rows, nparts;
+  int rows, ld, nparts;
   int blk_begin;
 };
 
@@ -660,7 +661,7 @@ __global__ void __launch_bounds__(256) pc_coef_reduce_kernel(const CoefJob* __re
   const CoefJob& j = J[lo];
   if (j.flag && *j.flag == 0) return;
   const long long e = ((long long)(blockIdx.x - j.blk_begin) * 256 + threadIdx.x) * 4;
-  if (e >= (long long)j.rows * kPanel) return;
+  if (e >= (long long)j.rows * j.ld) return;
   float4 v[8];
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int p0 = 0; p0 < j.nparts; p0 += 8) {

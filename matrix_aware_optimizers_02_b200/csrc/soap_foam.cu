@@ -96,7 +96,7 @@ inline size_t planes_bytes(int rows, int cols) { return 3 * 2 * (size_t)rows * l
 // Scratch of one side (k x k factor F with basis Q) of one matrix.
 struct SideBuf {
   size_t Fp, Qp, P, Ps, Psp;
-  size_t W, Wp, Cp;  // panel buffer (k x kPanel, fp32 and planes) and the coefficients
+  size_t W, Wp, Cp;  // super-panel buffer (k x kSuper, fp32 and planes) and the coefficients
   size_t Cpart;      // K-slice partials of the coefficients (large factors only)
   size_t pn, pnorm2, reorth, fin;  // squared column norms of P (original, sorted order); panel decisions
   size_t part, gs, rinv, keys, perm, flag, rho, bad, again;
@@ -122,10 +122,10 @@ void side_layout(int k, bool check, Carver& cv, SideBuf& s, size_t flag_block) {
   s.P = cv.take(4 * kk);
   s.Ps = cv.take(4 * kk);
   s.Psp = cv.take(planes_bytes(k, k));
-  s.W = cv.take(4 * (size_t)k * kPanel);
-  s.Wp = cv.take(planes_bytes(k, kPanel));
-  s.Cp = cv.take(planes_bytes(k, kPanel));
-  s.Cpart = k >= kCoefSplitMinK ? cv.take(4 * (size_t)kMaxCoefParts * k * kPanel) : 0;
+  s.W = cv.take(4 * (size_t)k * kSuper);
+  s.Wp = cv.take(planes_bytes(k, kSuper));
+  s.Cp = cv.take(planes_bytes(k, kSuper));
+  s.Cpart = k >= kCoefSplitMinK ? cv.take(4 * (size_t)kMaxCoefParts * k * kSuper) : 0;
   s.part = cv.take(4 * (size_t)parts * kPanelSq);
   s.gs = cv.take(8 * (size_t)kGsDoubles);
   s.rinv = cv.take(2 * 3 * (size_t)kPanelSq);
@@ -414,182 +414,229 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
     }
     B.ops.back().blocks = blk;
   }
-  // QR by panels of kPanel columns: block Gram-Schmidt with two projection passes,
-  // Cholesky-QR inside each panel (twice after the first pass, once after the second)
+  // QR by super-panels of kSuper = 2 kPanel columns (block Gram-Schmidt).  For each
+  // super-panel [c0, c0 + kSuper): one projection of all its columns against the
+  // finished columns [0, c0) (each pass over Q's planes serves 256 columns), then its
+  // two kPanel-column sub-panels in turn: the second is first projected against the
+  // first, and each is orthonormalised by Cholesky-QR (up to three passes, and a
+  // second projection against every finished column, all decided on the device).
   int maxk = 0;
   for (int i = 0; i < nu; ++i) maxk = std::max(maxk, kof(i));
-  const int npanels = (maxk + kPanel - 1) / kPanel;
+  const int nsuper = (maxk + kSuper - 1) / kSuper;
   enum { PS = 0, WA = 1, QF = 2 };
-  for (int pj = 0; pj < npanels; ++pj) {
-    const int c0 = pj * kPanel;
-    std::vector<int> act;
-    for (int i = 0; i < nu; ++i)
-      if (kof(i) > c0) act.push_back(i);
-    auto wdt = [&](int i) { return std::min(kPanel, kof(i) - c0); };
-    // a panel's fp32 storage and plane view (columns c0 .. c0 + w of Ps / Q, or a scratch buffer)
-    auto fp = [&](int i, int where, int* ld) -> float* {
-      const int k = kof(i);
-      switch (where) {
-        case PS: *ld = k; return B.wp<float>(side(i).Ps) + c0;
-        case WA: *ld = kPanel; return B.wp<float>(side(i).W);
-        default: *ld = k; return Qp(i) + c0;
-      }
-    };
-    auto pv = [&](int i, int where) -> Split3 {
-      const int k = kof(i), w = wdt(i);
-      Split3 v;
-      switch (where) {
-        case PS: v = B.planes(side(i).Psp, k, k); break;
-        case WA: v = B.planes(side(i).Wp, k, kPanel); break;
-        default: v = B.planes(side(i).Qp, k, k); break;
-      }
-      if (where == PS || where == QF)
-        for (int q = 0; q < 3; ++q) v.p[q] += c0;
-      v.cols = w;
-      return v;
-    };
-    // one Cholesky-QR of every active panel: dst = src R^{-1} (dst may be src).
-    // pass 0: the first pass; it decides on the device whether the second pass
-    //         (flag again), the second projection (reorth) and the final pass (fin)
-    //         run, and writes straight into Q's columns when none does;
-    // pass 1: the second pass (gated by again); pass 2: the final pass (gated by fin)
-    auto cholqr = [&](int src, int dst, int pass) -> mao_status {
-      auto gate = [&](int u) -> const int* {
-        return pass == 1 ? B.wp<int>(side(u).again) : pass == 2 ? B.wp<int>(side(u).fin) : flagp(u);
-      };
-      // Gram partials over K slices (fp32-faithful), one 128 x 128 tile each
-      TableLaunch& gg = B.new_gemm(1, 1, MAO_K_PC_PANEL);
-      const int nact = (int)act.size();
-      for (int i : act) {
-        const int k = kof(i), w = wdt(i);
-        const int sl = gram_slice(k, nact);
-        float* part = B.wp<float>(side(i).part);
-        const Split3 Wv = pv(i, src);
-        for (int s0 = 0, p = 0; s0 < k; s0 += sl, ++p)
-          MAO_TRY(table_add(gg, B.maps, Wv, Wv, w, w, std::min(sl, k - s0), 0, 0, part + (size_t)p * kPanelSq,
-                            nullptr, kPanel, nullptr, 0, 1.f, 0.f, gate(i), s0));
-      }
-      size_t off;
-      PanelJob* J = B.new_jobs<PanelJob>(Op::REDUCE, (int)act.size(), off);
-      for (size_t a = 0; a < act.size(); ++a) {
-        const int i = act[a];
+  for (int sp = 0; sp < nsuper; ++sp) {
+    const int c0 = sp * kSuper;
+    for (int half = 0; half < 2; ++half) {
+      const int cs = c0 + half * kPanel;  // first column of the sub-panel
+      std::vector<int> act;
+      for (int i = 0; i < nu; ++i)
+        if (kof(i) > cs) act.push_back(i);
+      if (act.empty()) break;
+      auto wdt = [&](int i) { return std::min(kPanel, kof(i) - cs); };
+      // a sub-panel's fp32 storage and plane view: columns cs .. cs + w of Ps / Q, or
+      // the sub-panel's half of the super-panel buffer W
+      auto fp = [&](int i, int where, int* ld) -> float* {
         const int k = kof(i);
-        PanelJob& j = J[a];
-        j.part = B.wp<float>(side(i).part);
-        j.gs = B.wp<double>(side(i).gs);
-        j.rinv = B.wp<__nv_bfloat16>(side(i).rinv);
-        j.bad = B.wp<int>(side(i).bad);
-        j.again = B.wp<int>(side(i).again);
-        j.flag = gate(i);
-        j.w = wdt(i);
-        j.nparts = (k + gram_slice(k, nact) - 1) / gram_slice(k, nact);
-        j.first = pass == 0 ? 1 : 0;
-        if (pass == 0) j.fin = B.wp<int>(side(i).fin);
-        if (pass == 0 && c0 > 0) {
-          j.pnorm2 = B.wp<float>(side(i).pnorm2) + c0;
-          j.reorth = B.wp<int>(side(i).reorth);
+        switch (where) {
+          case PS: *ld = k; return B.wp<float>(side(i).Ps) + cs;
+          case WA: *ld = kSuper; return B.wp<float>(side(i).W) + half * kPanel;
+          default: *ld = k; return Qp(i) + cs;
         }
-      }
-      B.ops.back().blocks = (int)act.size() * kRedBlocks;
-      Op ch = B.ops.back();  // the factorisation reuses the job array
-      ch.kind = Op::CHOL;
-      ch.blocks = (int)act.size();
-      B.ops.push_back(ch);
-      B.gemm_of_op.push_back(-1);
-      TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_QR_APPLY);
-      for (int i : act) {
+      };
+      auto pv = [&](int i, int where) -> Split3 {
         const int k = kof(i), w = wdt(i);
-        __nv_bfloat16* r = B.wp<__nv_bfloat16>(side(i).rinv);
-        const Split3 Ri{{r, r + kPanelSq, r + 2 * kPanelSq}, w, w, kPanel};
-        const Split3 out_p = pv(i, dst);
-        int ld = 0;
-        float* out = fp(i, dst, &ld);
-        MAO_TRY(table_add(g, B.maps, pv(i, src), Ri, k, w, w, 0, 0, out, &out_p, ld, nullptr, 0, 1.f, 0.f,
-                          gate(i)));
-        if (pass == 0) {  // final already: Q's columns
-          const Split3 q_p = pv(i, QF);
-          int ldq = 0;
-          float* q = fp(i, QF, &ldq);
-          MAO_TRY(table_set_alt(g, B.wp<int>(side(i).fin), q, &q_p, ldq));
+        Split3 v;
+        switch (where) {
+          case PS: v = B.planes(side(i).Psp, k, k); break;
+          case WA: v = B.planes(side(i).Wp, k, kSuper); break;
+          default: v = B.planes(side(i).Qp, k, k); break;
         }
-      }
-      return MAO_OK;
-    };
-    // remove the finished columns: C = Q[:, :c0]^T Y ; W = Y - Q[:, :c0] C (fp32 and planes)
-    // When the coefficient product has too few tiles to fill the GPU, the large
-    // factors split it over K into fp32 partials, summed (in slice order) into C's planes.
-    auto project = [&](int from) -> mao_status {
-      // the second projection runs only where the first one cancelled (flag set on the device)
-      auto pflag = [&](int u) -> const int* { return from == WA ? B.wp<int>(side(u).reorth) : flagp(u); };
-      int tiles = 0;
-      for (int i : act) tiles += (c0 + 127) / 128;
-      const int want = std::min(kMaxCoefParts, std::max(1, (2 * 148 + tiles - 1) / std::max(tiles, 1)));
-      TableLaunch& gc = B.new_gemm(1, 1, MAO_K_PC_QR);
-      std::vector<CoefJob> red;
-      int rblk = 0;
-      for (int i : act) {
-        const int k = kof(i), w = wdt(i);
-        Split3 C = B.planes(side(i).Cp, k, kPanel);
-        C.cols = w;
-        const int S = k >= kCoefSplitMinK ? want : 1;
-        if (S == 1) {
-          MAO_TRY(table_add(gc, B.maps, B.planes(side(i).Qp, k, k), pv(i, from), c0, w, k, 0, 0, nullptr, &C,
-                            kPanel, nullptr, 0, 1.f, 0.f, pflag(i)));
-          continue;
+        const int off = where == WA ? half * kPanel : cs;
+        for (int q = 0; q < 3; ++q) v.p[q] += off;
+        v.cols = w;
+        return v;
+      };
+      // one Cholesky-QR of every active sub-panel: dst = src R^{-1} (dst may be src).
+      // pass 0: the first pass; it decides on the device whether the second pass
+      //         (flag again), the second projection (reorth) and the final pass (fin)
+      //         run, and writes straight into Q's columns when none does;
+      // pass 1: the second pass (gated by again); pass 2: the final pass (gated by fin)
+      auto cholqr = [&](int src, int dst, int pass) -> mao_status {
+        auto gate = [&](int u) -> const int* {
+          return pass == 1 ? B.wp<int>(side(u).again) : pass == 2 ? B.wp<int>(side(u).fin) : flagp(u);
+        };
+        // Gram partials over K slices (fp32-faithful), one 128 x 128 tile each
+        TableLaunch& gg = B.new_gemm(1, 1, MAO_K_PC_PANEL);
+        const int nact = (int)act.size();
+        for (int i : act) {
+          const int k = kof(i), w = wdt(i);
+          const int sl = gram_slice(k, nact);
+          float* part = B.wp<float>(side(i).part);
+          const Split3 Wv = pv(i, src);
+          for (int s0 = 0, p = 0; s0 < k; s0 += sl, ++p)
+            MAO_TRY(table_add(gg, B.maps, Wv, Wv, w, w, std::min(sl, k - s0), 0, 0, part + (size_t)p * kPanelSq,
+                              nullptr, kPanel, nullptr, 0, 1.f, 0.f, gate(i), s0));
         }
-        const int sl = round_up_int((k + S - 1) / S, 64);
-        float* part = B.wp<float>(side(i).Cpart);
-        const long long pst = (long long)k * kPanel;
-        int p = 0;
-        for (int s0 = 0; s0 < k; s0 += sl, ++p)
-          MAO_TRY(table_add(gc, B.maps, B.planes(side(i).Qp, k, k), pv(i, from), c0, w, std::min(sl, k - s0), 0, 0,
-                            part + p * pst, nullptr, kPanel, nullptr, 0, 1.f, 0.f, pflag(i), s0));
-        CoefJob cj;
-        std::memset(&cj, 0, sizeof(cj));
-        cj.part = part;
-        cj.cp = B.wp<__nv_bfloat16>(side(i).Cp);
-        cj.part_stride = pst;
-        cj.pstride = B.pstride(k, kPanel);
-        cj.flag = pflag(i);
-        cj.rows = c0;
-        cj.nparts = p;
-        cj.blk_begin = rblk;
-        rblk += (c0 * kPanel + 1023) / 1024;
-        red.push_back(cj);
-      }
-      if (!red.empty()) {
         size_t off;
-        CoefJob* J = B.new_jobs<CoefJob>(Op::COEFRED, (int)red.size(), off);
-        for (size_t a = 0; a < red.size(); ++a) J[a] = red[a];
-        B.ops.back().blocks = rblk;
+        PanelJob* J = B.new_jobs<PanelJob>(Op::REDUCE, (int)act.size(), off);
+        for (size_t a = 0; a < act.size(); ++a) {
+          const int i = act[a];
+          const int k = kof(i);
+          PanelJob& j = J[a];
+          j.part = B.wp<float>(side(i).part);
+          j.gs = B.wp<double>(side(i).gs);
+          j.rinv = B.wp<__nv_bfloat16>(side(i).rinv);
+          j.bad = B.wp<int>(side(i).bad);
+          j.again = B.wp<int>(side(i).again);
+          j.flag = gate(i);
+          j.w = wdt(i);
+          j.nparts = (k + gram_slice(k, nact) - 1) / gram_slice(k, nact);
+          j.first = pass == 0 ? 1 : 0;
+          if (pass == 0) j.fin = B.wp<int>(side(i).fin);
+          if (pass == 0 && cs > 0) {
+            j.pnorm2 = B.wp<float>(side(i).pnorm2) + cs;
+            j.reorth = B.wp<int>(side(i).reorth);
+          }
+        }
+        B.ops.back().blocks = (int)act.size() * kRedBlocks;
+        Op ch = B.ops.back();  // the factorisation reuses the job array
+        ch.kind = Op::CHOL;
+        ch.blocks = (int)act.size();
+        B.ops.push_back(ch);
+        B.gemm_of_op.push_back(-1);
+        TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_QR_APPLY);
+        for (int i : act) {
+          const int k = kof(i), w = wdt(i);
+          __nv_bfloat16* r = B.wp<__nv_bfloat16>(side(i).rinv);
+          const Split3 Ri{{r, r + kPanelSq, r + 2 * kPanelSq}, w, w, kPanel};
+          const Split3 out_p = pv(i, dst);
+          int ld = 0;
+          float* out = fp(i, dst, &ld);
+          MAO_TRY(table_add(g, B.maps, pv(i, src), Ri, k, w, w, 0, 0, out, &out_p, ld, nullptr, 0, 1.f, 0.f,
+                            gate(i)));
+          if (pass == 0) {  // final already: Q's columns
+            const Split3 q_p = pv(i, QF);
+            int ldq = 0;
+            float* q = fp(i, QF, &ldq);
+            MAO_TRY(table_set_alt(g, B.wp<int>(side(i).fin), q, &q_p, ldq));
+          }
+        }
+        return MAO_OK;
+      };
+      // remove the columns [a0, a1) of Q from `width` columns of the source:
+      //   C = Q[:, a0:a1]^T Y (rows a0 .. a1 of the coefficient buffer);
+      //   W = Y - Q[:, a0:a1] C (fp32 and planes, into the super-panel buffer at column
+      //   `wcol`)
+      // `width` > kPanel projects the whole super-panel (its sources are Ps's columns).
+      // When the coefficient product has too few tiles to fill the GPU, the large
+      // factors split it over K into fp32 partials, summed (in slice order) into C's planes.
+      auto project = [&](const std::vector<int>& units, int from, int col, int a0, int a1, int wcol, int width,
+                         bool reorth) -> mao_status {
+        auto pflag = [&](int u) -> const int* { return reorth ? B.wp<int>(side(u).reorth) : flagp(u); };
+        auto wof = [&](int i) { return std::min(width, kof(i) - col); };
+        // a source view of `width` columns starting at column `col` (Ps) or `wcol` (W)
+        auto src_p = [&](int i) -> Split3 {
+          const int k = kof(i);
+          Split3 v = from == PS ? B.planes(side(i).Psp, k, k) : B.planes(side(i).Wp, k, kSuper);
+          const int off = from == PS ? col : wcol;
+          for (int q = 0; q < 3; ++q) v.p[q] += off;
+          v.cols = wof(i);
+          return v;
+        };
+        auto src_f = [&](int i, int* ld) -> const float* {
+          if (from == PS) {
+            *ld = kof(i);
+            return B.wp<float>(side(i).Ps) + col;
+          }
+          *ld = kSuper;
+          return B.wp<float>(side(i).W) + wcol;
+        };
+        const int rows = a1 - a0;
+        int tiles = 0;
+        for (size_t u = 0; u < units.size(); ++u) tiles += ((rows + 127) / 128) * ((width + 127) / 128);
+        const int want = std::min(kMaxCoefParts, std::max(1, (2 * 148 + tiles - 1) / std::max(tiles, 1)));
+        TableLaunch& gc = B.new_gemm(1, 1, MAO_K_PC_QR);
+        std::vector<CoefJob> red;
+        int rblk = 0;
+        for (int i : units) {
+          const int k = kof(i), w = wof(i);
+          Split3 C = B.planes(side(i).Cp, k, kSuper);
+          for (int q = 0; q < 3; ++q) C.p[q] += (size_t)a0 * kSuper;
+          C.rows = rows;
+          C.cols = w;
+          const int S = k >= kCoefSplitMinK ? want : 1;
+          if (S == 1) {
+            MAO_TRY(table_add(gc, B.maps, B.planes(side(i).Qp, k, k), src_p(i), rows, w, k, a0, 0, nullptr, &C,
+                              kSuper, nullptr, 0, 1.f, 0.f, pflag(i)));
+            continue;
+          }
+          const int sl = round_up_int((k + S - 1) / S, 64);
+          float* part = B.wp<float>(side(i).Cpart);
+          const long long pst = (long long)k * kSuper;
+          int p = 0;
+          for (int s0 = 0; s0 < k; s0 += sl, ++p)
+            MAO_TRY(table_add(gc, B.maps, B.planes(side(i).Qp, k, k), src_p(i), rows, w, std::min(sl, k - s0), a0,
+                              0, part + p * pst + (size_t)a0 * kSuper, nullptr, kSuper, nullptr, 0, 1.f, 0.f,
+                              pflag(i), s0));
+          CoefJob cj;
+          std::memset(&cj, 0, sizeof(cj));
+          cj.part = part + (size_t)a0 * kSuper;
+          cj.cp = B.wp<__nv_bfloat16>(side(i).Cp) + (size_t)a0 * kSuper;
+          cj.part_stride = pst;
+          cj.pstride = B.pstride(k, kSuper);
+          cj.flag = pflag(i);
+          cj.rows = rows;
+          cj.ld = kSuper;
+          cj.nparts = p;
+          cj.blk_begin = rblk;
+          rblk += (rows * kSuper + 1023) / 1024;
+          red.push_back(cj);
+        }
+        if (!red.empty()) {
+          size_t off;
+          CoefJob* J = B.new_jobs<CoefJob>(Op::COEFRED, (int)red.size(), off);
+          for (size_t a = 0; a < red.size(); ++a) J[a] = red[a];
+          B.ops.back().blocks = rblk;
+        }
+        TableLaunch& gw = B.new_gemm(0, 1, MAO_K_PC_QR);
+        for (int i : units) {
+          const int k = kof(i), w = wof(i);
+          Split3 C = B.planes(side(i).Cp, k, kSuper);
+          C.rows = a1;  // the product reads rows a0 .. a1 (K slice from a0)
+          C.cols = w;
+          Split3 Wp = B.planes(side(i).Wp, k, kSuper);
+          for (int q = 0; q < 3; ++q) Wp.p[q] += wcol;
+          Wp.cols = w;
+          int lda = 0;
+          const float* aux = src_f(i, &lda);
+          float* W = B.wp<float>(side(i).W) + wcol;
+          MAO_TRY(table_add(gw, B.maps, B.planes(side(i).Qp, k, k), C, k, w, rows, 0, 0, W, &Wp, kSuper, aux, lda,
+                            -1.f, 1.f, pflag(i), a0));
+        }
+        return MAO_OK;
+      };
+      // The products W R^{-1} run in place (each output row block reads only its own
+      // rows of W, all of K in one tile).
+      if (half == 0) {
+        if (c0 == 0) {
+          MAO_TRY(cholqr(PS, WA, 0));
+          MAO_TRY(cholqr(WA, WA, 1));
+          MAO_TRY(cholqr(WA, QF, 2));
+        } else {
+          MAO_TRY(project(act, PS, c0, 0, c0, 0, kSuper, false));  // the whole super-panel
+          MAO_TRY(cholqr(WA, WA, 0));
+          MAO_TRY(cholqr(WA, WA, 1));
+          MAO_TRY(project(act, WA, cs, 0, cs, 0, kPanel, true));
+          MAO_TRY(cholqr(WA, QF, 2));
+        }
+      } else {
+        // against the first sub-panel (from Ps when the super-panel is the first)
+        MAO_TRY(project(act, c0 == 0 ? PS : WA, cs, c0, cs, kPanel, kPanel, false));
+        MAO_TRY(cholqr(WA, WA, 0));
+        MAO_TRY(cholqr(WA, WA, 1));
+        MAO_TRY(project(act, WA, cs, 0, cs, kPanel, kPanel, true));
+        MAO_TRY(cholqr(WA, QF, 2));
       }
-      TableLaunch& gw = B.new_gemm(0, 1, MAO_K_PC_QR);
-      for (int i : act) {
-        const int k = kof(i), w = wdt(i);
-        Split3 C = B.planes(side(i).Cp, k, kPanel);
-        C.rows = c0;
-        C.cols = w;
-        const Split3 Wp = pv(i, WA);
-        int lda = 0, ldw = 0;
-        const float* aux = fp(i, from, &lda);
-        float* W = fp(i, WA, &ldw);
-        MAO_TRY(table_add(gw, B.maps, B.planes(side(i).Qp, k, k), C, k, w, c0, 0, 0, W, &Wp, ldw, aux, lda, -1.f,
-                          1.f, pflag(i)));
-      }
-      return MAO_OK;
-    };
-    // The products W R^{-1} run in place (each output row block reads only its own
-    // rows of W, all of K in one tile).
-    if (pj == 0) {
-      MAO_TRY(cholqr(PS, WA, 0));
-      MAO_TRY(cholqr(WA, WA, 1));
-      MAO_TRY(cholqr(WA, QF, 2));
-    } else {
-      MAO_TRY(project(PS));
-      MAO_TRY(cholqr(WA, WA, 0));
-      MAO_TRY(cholqr(WA, WA, 1));
-      MAO_TRY(project(WA));
-      MAO_TRY(cholqr(WA, QF, 2));
     }
   }
   return MAO_OK;

@@ -10,15 +10,16 @@ gate) pair is recorded in tests/gates.py):
     of its null space carry only the 1e-6 I ridge and are rounding noise in any
     fp32 arithmetic: the gate is then twice what an fp32 evaluation of the same
     steps by the oracle reaches, or 1e-4 if that is larger;
-  * the SOAP weight update: max(1e-4, 2x the oracle's own float32-mode error on the
-    same input), at every step.  Adam in the eigenbasis divides Mh by sqrt(V):
-    wherever the rotated gradient has been small on every step so far, both are
-    small and the ratio amplifies rounding; the float32 run of the oracle measures
-    that inherent floor (it exceeds 1e-4 on full-rank square cases at t = 2, e.g.
-    2.5e-4 on a 192 x 192 weight);
-  * the FOAM weight update: 1e-4 (its factored second moment is smooth);
+  * the weight update (SOAP and FOAM): max(1e-4, 2x the oracle's own float32-mode
+    error on the same input), at every step.  Adam in the eigenbasis divides Mh by
+    sqrt(V): wherever the rotated gradient has been small on every step so far, both
+    are small and the ratio amplifies rounding; the float32 run of the oracle
+    measures that inherent floor (SOAP: 2.5e-4 on a full-rank 192 x 192 weight at
+    t = 2; FOAM: 4.5e-3 on a 1536 x 4608 weight at t = 1, whose 4608-column factor
+    has rank 1536, so c is rounding noise in the null-space columns);
   * elementwise: max |err| / RMS(ref) below ten times the Frobenius gate, or below
-    twice the oracle's float32-mode value where the Frobenius gate is relaxed;
+    twice the oracle's float32-mode value where that is larger (the same
+    amplification acts on single coordinates, of the update and of V);
   * basis permutations: identical wherever the oracle's consecutive sorted keys
     differ by more than 1e-5 relative; refresh decisions identical when
     |rho - tol| > 1e-5, and rho^2 within 1e-5 absolute (the device derives it from
@@ -61,12 +62,13 @@ def _np(x):
 
 
 def _compare(label, name, got, ref, gate, ref32=None):
-    """Frobenius and elementwise checks of one quantity.  `ref32` (the oracle's float32
-    evaluation) relaxes the elementwise gate where the Frobenius gate is relaxed."""
+    """Frobenius and elementwise checks of one quantity.  With `ref32` (the oracle's
+    float32 evaluation of the same steps) the elementwise gate is at least twice what
+    that evaluation reaches."""
     gates.check(label, name, gates.rel(got, ref), gate)
     egate = ELEM_FACTOR * gate
-    if ref32 is not None and gate > STATE_TOL:
-        egate = max(ELEM_FACTOR * STATE_TOL, 2.0 * gates.max_over_rms(ref32, ref))
+    if ref32 is not None:
+        egate = max(egate, 2.0 * gates.max_over_rms(ref32, ref))
     gates.check(label, name + " max/rms", gates.max_over_rms(got, ref), egate)
 
 
@@ -187,7 +189,8 @@ def _soap_run(api, shapes, steps, seed, eps, g_scale, lr, refresh, k, sort, g_bf
                         assert bool(stats["refreshed"][i] & bit) == ref, (lab, side, rho)
                 assert abs(stats["offdiag_ratio"][i] ** 2 - res.rho_R ** 2) < 1e-5, (lab, res.rho_R)
             for name in ("M", "L", "R", "V"):
-                _compare(lab, "soap " + name, _np(d[name]), getattr(res.state, name), STATE_TOL)
+                _compare(lab, "soap " + name, _np(d[name]), getattr(res.state, name), STATE_TOL,
+                         getattr(r32.state, name).astype(np.float64))
             for name, rows, cols, refreshed in (("QL", m, n, res.refreshed_L), ("QR", n, m, res.refreshed_R)):
                 if refreshed:
                     seen_at[i][name] = t - 1 if lag else t
@@ -313,10 +316,12 @@ def _foam_run(api, shapes, steps, seed, refresh, pf, tol, eps, lr, k, raw_trace,
               label, grads=None):
     rng = np.random.default_rng(seed)
     b1 = b2 = 0.95
-    dev, ora, Ws = [], [], []
+    dev, ora, ora32, Ws, Ws32 = [], [], [], [], []
     for (m, n) in shapes:
         W = (rng.standard_normal((m, n)) * 0.02).astype(np.float32)
         st = O.FoamState.init(m, n)
+        ora32.append(st.copy(np.float32))
+        Ws32.append(W.copy())
         dev.append({"W": _t(W), "G": _gdev(np.zeros((m, n), np.float32), g_bf16), "M": _t(st.M), "r": _t(st.r),
                     "c": _t(st.c),
                     "R": _t(st.R), "QR": _t(st.QR), "perm_R": torch.zeros(n, dtype=torch.int32, device="cuda")})
@@ -352,31 +357,34 @@ def _foam_run(api, shapes, steps, seed, refresh, pf, tol, eps, lr, k, raw_trace,
                 # orthogonal Q: its absolute error is bounded by the fp32 basis's
                 # ||Q^T Q - I||, about 1e-6 at these sizes
                 assert abs(stats["offdiag_ratio"][i] ** 2 - res.rho ** 2) < 1e-5, (lab, res.rho)
+            # the float32 evaluation of the same step (same ordering as the float64 one)
+            src32 = (ora[i].copy(np.float32), Ws[i].astype(np.float32)) if replay else (ora32[i], Ws32[i])
+            r32 = O.foam_step(src32[1], Gs[i], src32[0], dtype=np.float32,
+                              force_perm=res.perm_R if res.refreshed else None, **kw)
             for name in ("M", "R", "r", "c"):
-                _compare(lab, "foam " + name, _np(d[name]), getattr(res.state, name), STATE_TOL)
+                _compare(lab, "foam " + name, _np(d[name]), getattr(res.state, name), STATE_TOL,
+                         getattr(r32.state, name).astype(np.float64))
             if res.refreshed:
                 seen_at[i] = t - 1 if lag else t
             full = seen_at[i] is None or seen_at[i] * m >= n
-            gate = STATE_TOL
-            q32 = None
-            if not full:
-                r32 = O.foam_step(Ws[i].astype(np.float32), Gs[i], ora[i].copy(np.float32), dtype=np.float32,
-                                  force_perm=res.perm_R, **kw)
-                q32 = r32.state.QR.astype(np.float64)
-                gate = max(STATE_TOL, 2 * gates.rel(q32, res.state.QR))
+            q32 = r32.state.QR.astype(np.float64)
+            gate = STATE_TOL if full else max(STATE_TOL, 2 * gates.rel(q32, res.state.QR))
             _compare(lab, "foam QR" + (" (full rank)" if full else " (rank-deficient)"), _np(d["QR"]),
                      res.state.QR, gate, q32)
             ref = res.W - Ws[i]
-            _compare(lab, "foam dW", _np(d["W"]) - gpu_prev[i], ref, STATE_TOL)
+            ref32 = r32.W.astype(np.float64) - src32[1].astype(np.float64)
+            gate = max(STATE_TOL, 2 * gates.rel(ref32, ref))
+            _compare(lab, "foam dW", _np(d["W"]) - gpu_prev[i], ref, gate, ref32)
             gpu_prev[i] = _np(d["W"])
             rms_ref = float(np.linalg.norm(ref) / np.sqrt(m * n))
-            gates.check(lab, "foam update_rms", abs(stats["update_rms"][i] - rms_ref) / rms_ref, STATE_TOL)
+            gates.check(lab, "foam update_rms", abs(stats["update_rms"][i] - rms_ref) / rms_ref, gate)
             assert stats["nonfinite"][i] == 0
             if replay:
                 ora[i] = O.FoamState(_np(d["M"]), _np(d["r"]), _np(d["c"]), _np(d["R"]), _np(d["QR"]))
                 Ws[i] = _np(d["W"])
             else:
                 ora[i], Ws[i] = res.state, res.W
+                ora32[i], Ws32[i] = r32.state, r32.W
 
 
 def test_foam_tall_adaptive_multistep(api):

@@ -1,5 +1,6 @@
-"""Layer-wise distributed step, host side on CPU: the owner assignment and the
-all-gather-V over two gloo ranks, with a stand-in for the per-rank GPU step."""
+"""Layer-wise distributed step, host side on CPU: the owner assignment, the cost
+model, and the reduce-to-owner + all-gather-V exchange over two gloo ranks, with a
+stand-in for the per-rank GPU step."""
 
 import os
 import socket
@@ -37,6 +38,22 @@ def test_cost_model_follows_shape_not_size():
     assert LW.state_bytes("foam", 4096, 1024) < LW.state_bytes("foam", 1024, 4096)
 
 
+def test_cost_model_follows_the_batch_settings():
+    # Newton-Schulz work is linear in the step count
+    assert LW.step_flops("muon", 768, 2304, ns_steps=16) == pytest.approx(16 / 5 * LW.step_flops("muon", 768, 2304))
+    # a refresh every k steps is paid once per k steps: the refresh part shrinks by k
+    full = LW.step_flops("soap", 2048, 768, refresh_period=1)
+    plain = LW.step_flops("soap", 2048, 768, refresh_period=1 << 40)
+    assert LW.step_flops("soap", 2048, 768, refresh_period=10) == pytest.approx(plain + (full - plain) / 10)
+    # the QR term is the built block Gram-Schmidt: 2 k^3 + 4 k^2 b with 128-column panels
+    assert LW.qr_flops(4096) == 2 * 4096 ** 3 + 4 * 4096 ** 2 * 128
+    c = LW.cost_for("soap", {"refresh": "every_k", "k": 10})
+    assert c("soap", 4096, 1024) == LW.step_cost("soap", 4096, 1024, 5, 10)
+    c = LW.cost_for("muon", {"ns_steps": 16})
+    assert c("muon", 4096, 1024) == LW.step_cost("muon", 4096, 1024, 16, 1)
+    assert LW.cost_for("foam", {})("foam", 1536, 4608) == LW.step_cost("foam", 1536, 4608, 5, 10)
+
+
 def test_lpt_matches_brute_force_optimum_bound():
     # four jobs on two ranks: longest-first reaches the optimum here
     cost = {(4, 1): 7.0, (3, 1): 5.0, (2, 1): 4.0, (1, 1): 4.0}
@@ -63,13 +80,15 @@ def _rank(rank, world, port, q):
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         shapes = [(8, 16), (16, 8), (24, 16), (8, 8), (32, 16)]
-        mats = [{"W": torch.full(s, float(i), dtype=torch.float32)} for i, s in enumerate(shapes)]
+        # every rank holds the same weights and its own local gradient: G_i = i + 10 rank
+        mats = [{"W": torch.full(s, float(i), dtype=torch.float32),
+                 "G": torch.full(s, float(i) + 10.0 * rank, dtype=torch.float32)} for i, s in enumerate(shapes)]
         stepped = []
 
         def make_batch(owned):
             def step(t):
-                for d in owned:  # stand-in for the GPU step: W <- W + t * (100 + rank)
-                    d["W"].add_(t * (100.0 + rank))
+                for d in owned:  # stand-in for the GPU step: W <- W - t * G (G reduced to its owner)
+                    d["W"].sub_(t * d["G"])
                 stepped.extend(id(d) for d in owned)
             return step
 
@@ -98,7 +117,9 @@ def test_two_ranks_step_owned_and_gather_all():
     for rank, owners, Ws, nstep in out:
         assert nstep == sum(1 for o in owners if o == rank)  # each rank stepped only what it owns
         for i, (W, o) in enumerate(zip(Ws, owners)):
-            expect = float(i) + 2 * (100.0 + o)  # the owner's update, on every rank
+            # the owner stepped with the mean gradient over the two ranks, i + 5, and every
+            # rank received its update
+            expect = float(i) - 2 * (float(i) + 5.0)
             t = torch.tensor(W)
             assert tuple(t.shape) == shapes[i]
             assert torch.all(t == expect), (rank, i, o)
