@@ -59,6 +59,9 @@ def parse():
                          "(strong scaling)")
     ap.add_argument("--workload", default="dense8b_moe", choices=sorted(WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--experts", type=int, default=256,
+                    help="experts of the MoE bank (moe_bank, dense8b_moe); fewer make a small case of the same "
+                         "shapes for profiling")
     ap.add_argument("--optimizers", default="muon,soap,foam", help="comma list of muon, soap, foam")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--soap-k", type=int, default=1, help="SOAP refreshes its bases every k steps")
@@ -81,10 +84,15 @@ def parse():
     return ap.parse_args()
 
 
+EXPERTS = [256]  # experts of the MoE bank (set from --experts)
+
+
 def specs_for(workload, seed):
     from matrix_aware_optimizers_02_b200 import synth
     if workload == "dense8b_moe":
-        return synth.specs_dense8b_moe(256, seed)
+        return synth.specs_dense8b_moe(EXPERTS[0], seed)
+    if workload == "moe_bank":
+        return synth.specs_moe_bank(EXPERTS[0], seed)
     return synth.WORKLOADS[workload]()
 
 
@@ -209,14 +217,18 @@ def write_launch_log(args, lib, L, LS, t, stream):
 
 
 def fold_traffic(args):
-    """Per kernel id: DRAM bytes per launch, per algorithmic FLOP and per algorithmic byte, from the
-    ncu CSV of a --launch-log run (its last len(launches) library launches are the logged step)."""
+    """Per kernel id: launches, ncu time and share, DRAM bytes per launch / per algorithmic
+    FLOP / per algorithmic byte, and the time-weighted tensor-pipe and DRAM utilisation,
+    from the ncu CSV of a --launch-log run (its last len(launches) library launches are the
+    logged step).  Metrics absent from the CSV are left out.  Writes --traffic-out (JSON)
+    and prints a markdown table."""
     import csv
     with open(args.launch_log) as f:
         log = json.load(f)
     rows = list(csv.reader(open(args.traffic_csv)))
     head = None
     per = {}
+    names = {}
     for r in rows:
         if "Kernel Name" in r:
             head = r
@@ -224,9 +236,18 @@ def fold_traffic(args):
         if head is None or len(r) != len(head):
             continue
         d = dict(zip(head, r))
-        e = per.setdefault(int(d["ID"]), {})
-        e[d["Metric Name"]] = float(d["Metric Value"].replace(",", ""))
-    ids = sorted(per)
+        try:
+            i = int(d["ID"])
+        except ValueError:
+            continue
+        e = per.setdefault(i, {})
+        try:
+            e[d["Metric Name"]] = float(d["Metric Value"].replace(",", ""))
+        except ValueError:
+            pass
+        names[i] = d["Kernel Name"].split("(")[0].split("<")[0].split()[-1].split("::")[-1]
+    ids = sorted(i for i in per if names.get(i, "").startswith(("gemm_tc", "muon_", "pc_", "soap_", "foam_", "qr_",
+                                                                   "mop_")))
     launches = log["launches"]
     tail = ids[-len(launches):]
     if len(tail) != len(launches):
@@ -236,17 +257,13 @@ def fold_traffic(args):
            "muon_update": ["muon_update_kernel"], "muon_colsq": ["muon_norm_tile_kernel"],
            "muon_colscale": ["muon_norm_final_kernel"], "muon_rowscale": ["muon_norm_tile_kernel",
                                                                           "muon_norm_final_kernel"],
+           "mop_init": ["mop_init_kernel"],
            "pc_elementwise": ["pc_momentum_kernel", "pc_split_kernel", "soap_adam_kernel", "foam_rc_partial_kernel",
                               "foam_tau_kernel", "foam_n_kernel"],
            "pc_sort": ["pc_keys_kernel", "pc_argsort_kernel", "pc_gather_cols_kernel", "soap_vperm_kernel"],
            "pc_check": ["pc_check_kernel"], "pc_chol": ["qr_chol_kernel"], "pc_qr_reduce": ["pc_coef_reduce_kernel"],
            "pc_stats": ["pc_stats_kernel"],
            "pc_panel": ["gemm_tc_table_kernel", "gemm_tc_pair_kernel", "qr_gram_reduce_kernel"]}
-    names = {}
-    for r in rows:
-        if head is not None and len(r) == len(head) and "Kernel Name" not in r:
-            d = dict(zip(head, r))
-            names[int(d["ID"])] = d["Kernel Name"].split("(")[0].split("<")[0].split()[-1]
     for rec, i in zip(launches, tail):
         ok = fam.get(rec["kernel"], ["gemm_tc_table_kernel", "gemm_tc_pair_kernel", "gemm_tc_kernel"])
         if names[i] not in ok:
@@ -254,24 +271,44 @@ def fold_traffic(args):
     agg = {}
     for rec, i in zip(launches, tail):
         m = per[i]
-        a = agg.setdefault(rec["kernel"], {"launches": 0, "dram": 0.0, "flops": 0.0, "bytes": 0.0, "ns": 0.0})
+        a = agg.setdefault(rec["kernel"], {"launches": 0, "dram": 0.0, "flops": 0.0, "bytes": 0.0, "ns": 0.0,
+                                           "tc_ns": 0.0, "dt_ns": 0.0, "has_dram": False, "has_tc": False})
+        ns = m.get("gpu__time_duration.sum", 0.0)
         a["launches"] += 1
-        a["dram"] += m.get("dram__bytes_read.sum", 0.0) + m.get("dram__bytes_write.sum", 0.0)
+        if "dram__bytes_read.sum" in m or "dram__bytes_write.sum" in m:
+            a["has_dram"] = True
+            a["dram"] += m.get("dram__bytes_read.sum", 0.0) + m.get("dram__bytes_write.sum", 0.0)
+        if "sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_elapsed" in m:
+            a["has_tc"] = True
+            a["tc_ns"] += ns * m["sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_elapsed"]
+        if "dram__throughput.avg.pct_of_peak_sustained_elapsed" in m:
+            a["dt_ns"] += ns * m["dram__throughput.avg.pct_of_peak_sustained_elapsed"]
         a["flops"] += rec["flops"]
         a["bytes"] += rec["bytes"]
-        a["ns"] += m.get("gpu__time_duration.sum", 0.0)
+        a["ns"] += ns
+    total_ns = sum(a["ns"] for a in agg.values()) or 1.0
     out = {"source_hash": log["source_hash"], "measured_on": log["workload"], "kernels": {}}
     for k, a in sorted(agg.items()):
-        out["kernels"][k] = {
-            "launches": a["launches"],
-            "dram_bytes_per_launch": a["dram"] / a["launches"],
-            "dram_bytes_per_flop": (a["dram"] / a["flops"]) if a["flops"] > 0 else None,
-            "dram_bytes_per_alg_byte": (a["dram"] / a["bytes"]) if a["bytes"] > 0 else None,
-            "ncu_ms": a["ns"] / 1e6,
-        }
+        rec = {"launches": a["launches"], "ncu_ms": a["ns"] / 1e6, "share": a["ns"] / total_ns}
+        if a["has_dram"]:
+            rec["dram_bytes_per_launch"] = a["dram"] / a["launches"]
+            rec["dram_bytes_per_flop"] = (a["dram"] / a["flops"]) if a["flops"] > 0 else None
+            rec["dram_bytes_per_alg_byte"] = (a["dram"] / a["bytes"]) if a["bytes"] > 0 else None
+        if a["has_tc"] and a["ns"] > 0:
+            rec["tensor_pipe_pct"] = a["tc_ns"] / a["ns"]
+        if a["dt_ns"] > 0 and a["ns"] > 0:
+            rec["dram_pct"] = a["dt_ns"] / a["ns"]
+        out["kernels"][k] = rec
     with open(args.traffic_out, "w") as f:
         json.dump(out, f, indent=1)
-    print(json.dumps(out, indent=1))
+    print(f"| kernel id | launches | ncu ms | share | tensor pipe % | DRAM % | DRAM B / alg B | DRAM B / FLOP |")
+    print("|---|---|---|---|---|---|---|---|")
+    for k, r in sorted(out["kernels"].items(), key=lambda kv: -kv[1]["share"]):
+        def f(x, fmt):
+            return fmt.format(x) if x is not None else ""
+        print(f"| {k} | {r['launches']} | {r['ncu_ms']:.3f} | {r['share']:.3f} | {f(r.get('tensor_pipe_pct'), '{:.1f}')} | "
+              f"{f(r.get('dram_pct'), '{:.1f}')} | {f(r.get('dram_bytes_per_alg_byte'), '{:.2f}')} | "
+              f"{f(r.get('dram_bytes_per_flop'), '{:.4f}')} |")
 
 
 # ----------------------------------------------------------------------------- CPU (oracle) leg
@@ -777,7 +814,7 @@ def run_mine(args, rank, world, dist):
         "dtype": "bf16 operands / fp32 accumulate (Newton-Schulz); fp32-faithful split-bf16 products and fp32 "
                  "states (SOAP, FOAM)",
         "data": "synthetic (seeded Gaussian gradients, random weights)",
-        "config": {"workload": args.workload, "description": desc, "optimizers": order,
+        "config": {"workload": args.workload, "description": desc, "experts": args.experts, "optimizers": order,
                    "optimizer_ms": opt_ms,
                    "muon": {"mu": 0.95, "lr": 0.02, "ns_steps": 5, "norm": norm},
                    "soap": {"beta1": 0.95, "beta2": 0.95, "eps": 1e-8,
@@ -920,6 +957,7 @@ def run_reference(args, rank, world):
 
 def main():
     args = parse()
+    EXPERTS[0] = args.experts
     if args.traffic_csv:
         fold_traffic(args)
         return 0

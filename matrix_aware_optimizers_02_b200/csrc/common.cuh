@@ -297,4 +297,16 @@ __device__ __forceinline__ void store_split3(float x, __nv_bfloat16* base, long 
   }
 }
 
+// Index of the work record that owns block `blk`: the last i with starts[i] <= blk,
+// over a compact array of first-block indices (a few cache lines, unlike the records
+// themselves, so the search costs little before the block's own memory traffic).
+__device__ __forceinline__ int find_start(const int* __restrict__ starts, int n, int blk) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(starts + mid) <= blk) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 }  // namespace mao

@@ -154,7 +154,8 @@ void plan(const mao_muon_mat* mats, int count, const int* ld, int callers, const
   }
   Carver cv;
   cv.take(kStatusBytes);
-  P.off_table = cv.take(sizeof(MuonMatDev) * (size_t)std::max(count, 1));
+  // the table, then the compact first-tile array that find_mat searches
+  P.off_table = cv.take((sizeof(MuonMatDev) + sizeof(int)) * (size_t)std::max(count, 1));
   P.off_scale = cv.take(sizeof(float) * (size_t)std::max(count, 1));
   int sb = 0;
   for (auto& c : P.cls) {
@@ -361,8 +362,11 @@ extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, con
     cp_off += (size_t)D.tiles_r * D.n;
   }
   MAO_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream));
-  MAO_CUDA_TRY(cudaMemcpyAsync(ws + P.off_table, P.table.data(), sizeof(MuonMatDev) * count,
-                               cudaMemcpyHostToDevice, stream));
+  std::vector<uint8_t> image((sizeof(MuonMatDev) + sizeof(int)) * count);
+  std::memcpy(image.data(), P.table.data(), sizeof(MuonMatDev) * count);
+  int* starts = reinterpret_cast<int*>(image.data() + sizeof(MuonMatDev) * count);
+  for (int i = 0; i < count; ++i) starts[i] = P.table[i].tile_begin;
+  MAO_CUDA_TRY(cudaMemcpyAsync(ws + P.off_table, image.data(), image.size(), cudaMemcpyHostToDevice, stream));
   const MuonMatDev* T = reinterpret_cast<const MuonMatDev*>(ws + P.off_table);
 
   // algorithmic bytes of the elementwise passes

@@ -56,13 +56,10 @@ struct MuonMatDev {
   const float* Of;
 };
 
+// The device table of `count` records is followed by the records' first tiles
+// (a compact int array): the block's matrix by a search that stays in L1.
 __device__ __forceinline__ int find_mat(const MuonMatDev* T, int count, int blk) {
-  int lo = 0, hi = count - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (T[mid].tile_begin <= blk) lo = mid; else hi = mid - 1;
-  }
-  return lo;
+  return find_start(reinterpret_cast<const int*>(T + count), count, blk);
 }
 
 __device__ __forceinline__ void bf16x4_to_float(uint2 raw, float* v) {

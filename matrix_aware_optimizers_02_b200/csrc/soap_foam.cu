@@ -273,9 +273,12 @@ struct Builder {
     return gemms.back();
   }
 
+  // A job array of n records, followed by room for two compact arrays of the
+  // records' first-block indices (filled by fill_starts once the records are final).
   template <class J>
   J* new_jobs(Op::Kind kind, int n, size_t& off) {
-    off = arena.take(sizeof(J) * std::max(n, 1), 64);
+    const size_t bytes = sizeof(J) * std::max(n, 1) + 2 * sizeof(int) * std::max(n, 1);
+    off = arena.take(bytes, 64);
     Op o;
     o.kind = kind;
     o.jobs = off;
@@ -283,10 +286,48 @@ struct Builder {
     ops.push_back(o);
     gemm_of_op.push_back(-1);
     J* p = arena.hptr<J>(off);
-    std::memset(static_cast<void*>(p), 0, sizeof(J) * std::max(n, 1));
+    std::memset(static_cast<void*>(p), 0, bytes);
     return p;
   }
 };
+
+// The compact first-block index arrays after every job array (job_starts() on the device).
+template <class J, class F>
+void fill_starts_of(Builder& B, const Op& op, F first_block, int which = 0) {
+  const int n = op.njobs;
+  const J* jobs = B.arena.hptr<J>(op.jobs);
+  int* st = reinterpret_cast<int*>(B.arena.host.data() + op.jobs + sizeof(J) * n) + which * n;
+  for (int i = 0; i < n; ++i) st[i] = first_block(jobs[i]);
+}
+
+void fill_starts(Builder& B) {
+  for (const Op& op : B.ops) {
+    if (op.kind == Op::GEMM || op.njobs <= 0) continue;
+    switch (op.kind) {
+      case Op::EW: case Op::SPLIT: case Op::ADAM: case Op::FOAMN:
+        fill_starts_of<EwJob>(B, op, [](const EwJob& j) { return j.blk_begin; });
+        break;
+      case Op::KEYS: case Op::ARGSORT:
+        fill_starts_of<SortJob>(B, op, [](const SortJob& j) { return j.key_blk_begin; }, 0);
+        fill_starts_of<SortJob>(B, op, [](const SortJob& j) { return j.col_blk_begin; }, 1);
+        break;
+      case Op::GATHER:
+        fill_starts_of<GatherJob>(B, op, [](const GatherJob& j) { return j.blk_begin; });
+        break;
+      case Op::VPERM:
+        fill_starts_of<VPermJob>(B, op, [](const VPermJob& j) { return j.blk_begin; });
+        break;
+      case Op::COEFRED:
+        fill_starts_of<CoefJob>(B, op, [](const CoefJob& j) { return j.blk_begin; });
+        break;
+      case Op::RC:
+        fill_starts_of<RcJob>(B, op, [](const RcJob& j) { return j.blk_begin; });
+        break;
+      default:
+        break;  // one block per record (REDUCE, CHOL, TAU, CHECK): no search
+    }
+  }
+}
 
 int ew_blocks(int rows, int cols) {
   const long long e = (long long)rows * cols;
@@ -337,6 +378,11 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
       blk += ew_blocks(k, k);
     }
     B.ops.back().blocks = blk;
+    {  // algorithmic bytes: the fp32 source read, three bf16 planes written
+      double bytes = 0;
+      for (int q = 0; q < B.ops.back().njobs; ++q) bytes += (double)J[q].rows * J[q].cols * (4 + 6);
+      B.ops.back().bytes = bytes;
+    }
   }
   // power step P = F Q (A = F K-major, B = Q stored K x N)
   {
@@ -739,6 +785,11 @@ mao_status build_group(Builder& B, GroupPlan& G) {
       }
     }
     B.ops.back().blocks = blk;
+    {  // algorithmic bytes: the fp32 source read, three bf16 planes written
+      double bytes = 0;
+      for (int q = 0; q < B.ops.back().njobs; ++q) bytes += (double)J[q].rows * J[q].cols * (4 + 6);
+      B.ops.back().bytes = bytes;
+    }
     MAO_TRY(build_refresh(B, G));
     MAO_TRY(factor_products(false));
   } else {
@@ -772,6 +823,11 @@ mao_status build_group(Builder& B, GroupPlan& G) {
       }
     }
     B.ops.back().blocks = blk;
+    {  // algorithmic bytes: the fp32 source read, three bf16 planes written
+      double bytes = 0;
+      for (int q = 0; q < B.ops.back().njobs; ++q) bytes += (double)J[q].rows * J[q].cols * (4 + 6);
+      B.ops.back().bytes = bytes;
+    }
     // identity permutations for the callers that asked for them
     bool any = false;
     for (int i = 0; i < nm; ++i) any = any || A(i).perm_R || (!foam && A(i).perm_L);
@@ -930,6 +986,9 @@ mao_status build_group(Builder& B, GroupPlan& G) {
         blk += j.tiles_c * j.tiles_r;
       }
       B.ops.back().blocks = blk;
+      double bytes = 0;
+      for (int q = 0; q < nm; ++q) bytes += (double)J[q].m * J[q].n * 4;  // Gr read once
+      B.ops.back().bytes = bytes;
     }
     {
       size_t off;
@@ -974,6 +1033,9 @@ mao_status build_group(Builder& B, GroupPlan& G) {
         blk += ew_blocks(a.m, a.n);
       }
       B.ops.back().blocks = blk;
+      double bytes = 0;
+      for (int q = 0; q < nm; ++q) bytes += (double)J[q].rows * J[q].cols * (4 + 6);  // Mr read, N planes
+      B.ops.back().bytes = bytes;
     }
     // U = N Q_R^T ; W update
     {
@@ -1001,6 +1063,7 @@ struct BuiltGroup {
 };
 
 mao_status finish_build(Builder& B, BuiltGroup& out) {
+  fill_starts(B);
   // maps after all problems are known
   out.maps_off = B.arena.take(sizeof(CUtensorMap) * std::max<size_t>(B.maps.keys.size(), 1), 64);
   if (B.ws) {
@@ -1072,7 +1135,7 @@ mao_status run_ops(const Ctx& X, uint8_t* arena_dev, const BuiltGroup& bg, DevSt
         break;
       }
       case Op::SPLIT: {
-        LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, 0.0);
+        LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, op.bytes);
         pc_split_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<EwJob>(op.jobs), n);
         break;
       }
@@ -1118,7 +1181,7 @@ mao_status run_ops(const Ctx& X, uint8_t* arena_dev, const BuiltGroup& bg, DevSt
         break;
       }
       case Op::RC: {
-        LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, 0.0);
+        LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, op.bytes);
         foam_rc_partial_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<RcJob>(op.jobs), n);
         break;
       }
@@ -1128,7 +1191,7 @@ mao_status run_ops(const Ctx& X, uint8_t* arena_dev, const BuiltGroup& bg, DevSt
         break;
       }
       case Op::FOAMN: {
-        LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, 0.0);
+        LaunchScope ls(s, MAO_K_PC_ELEMENTWISE, 0.0, op.bytes);
         foam_n_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<EwJob>(op.jobs), n, 1.f / bc1, 1.f / bc2, X.eps);
         break;
       }
