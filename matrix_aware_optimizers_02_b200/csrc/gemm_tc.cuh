@@ -17,15 +17,15 @@
 //               fp32-faithful product.  A problem can be gated by a device flag
 //               (skipped when the flag is 0) for data-dependent work.
 //
-// Warp roles (192 threads; 320 in table mode, with warps 2..9 in the epilogue):
+// Warp roles (320 threads):
 //   warp 0      TMA producer (one elected lane): fills a STAGES-deep ring of
 //               A/B tiles in shared memory, 128-byte swizzled.
 //   warp 1      TMEM owner + MMA issuer (one elected lane): tcgen05.mma into one
 //               of two TMEM accumulators (BN fp32 columns each); commits free the
 //               smem slots and hand finished accumulators to the epilogue.
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//               lanes 32*(w%4)..+31 = tile rows), fused arithmetic, stores; in
-//               table mode two warps share each lane quarter, half the columns each.
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
+//               lanes 32*(w%4)..+31 = tile rows), fused arithmetic, stores; two
+//               warps share each lane quarter, half the tile's columns each.
 // The two accumulators let the epilogue of tile i overlap the MMAs of tile i+1.
 //
 // Operand kinds:
@@ -151,8 +151,8 @@ struct GemmCfg {
   static constexpr int KCH = CORR ? 2 : 4;
   static constexpr int TMEM_COLS = 2 * ACC_COLS;         // double-buffered
   static constexpr uint32_t IDESC = make_idesc(1u, A_MN, B_MN, BM, BN);
-  static constexpr int THREADS = 192;
-  static constexpr int TABLE_THREADS = 320;  // table mode: 8 epilogue warps
+  static constexpr int THREADS = 320;        // producer, MMA issuer, 8 epilogue warps
+  static constexpr int TABLE_THREADS = 320;
 };
 
 // Descriptor of one operand tile (rows = MN extent R, K extent = BK) at smem
@@ -465,10 +465,10 @@ template <int KIND, int A_MN, int B_MN, int EPI, class Src, int PA = (KIND == OP
 __device__ __forceinline__ void gemm_body(const Src& src) {
   using Cfg = GemmCfg<KIND, A_MN, B_MN, PA, PB>;
   constexpr int BM = Cfg::BM, BN = Cfg::BN, BK = Cfg::BK, STAGES = Cfg::STAGES;
-  // Table mode runs 8 epilogue warps, two per TMEM lane quarter, each taking half of
-  // the tile's columns: twice the memory operations in flight for its fp32 and
-  // plane stores, and half the fold registers per thread.
-  constexpr int EPI_WARPS = (EPI == EPI_TABLE) ? 8 : 4;
+  // 8 epilogue warps, two per TMEM lane quarter, each taking half of the tile's
+  // columns: twice the memory operations in flight for the epilogue's aux reads and
+  // stores (and, in table mode, half the fold registers per thread).
+  constexpr int EPI_WARPS = 8;
   constexpr int COLS = BN * 4 / EPI_WARPS;  // columns per epilogue warp
 
   extern __shared__ uint8_t smem_raw[];
@@ -646,16 +646,16 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
           break;
         }
         tc_fence_after();
-        const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS;
+        const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS + cb;
 #pragma unroll 1
-        for (int ch = 0; ch < BN / 32; ++ch) {
+        for (int ch = 0; ch < COLS / 32; ++ch) {
           uint32_t rr[32];
           tmem_ld_32x32b_x32(tacc + ch * 32, rr);
           tmem_wait_ld();
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(rr[j]);
-          if (t.n0 + ch * 32 < ncols) src.template epilogue<EPI>(t, row, t.n0 + ch * 32, v);
+          if (t.n0 + cb + ch * 32 < ncols) src.template epilogue<EPI>(t, row, t.n0 + cb + ch * 32, v);
         }
         tc_fence_before();
         mbar_arrive(&tempty_bar[acc]);
@@ -1016,7 +1016,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
 }
 
 template <int KIND, int A_MN, int B_MN, int EPI>
-__global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(320, 1) gemm_tc_kernel(const __grid_constant__ GemmParams p) {
   ClassSource src(p);
   gemm_body<KIND, A_MN, B_MN, EPI>(src);
 }
