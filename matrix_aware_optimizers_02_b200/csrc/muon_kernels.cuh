@@ -155,33 +155,21 @@ __global__ void __launch_bounds__(256) muon_prep_kernel(const MuonMatDev* __rest
   const int col = c0 + tx * 4;
   const float om = 1.0f - mu;
   float acc = 0.0f;
-  // every load of the thread first, then the arithmetic and the stores (a store to M
-  // could alias a later row's load as far as the compiler knows)
-  float4 m4s[4];
-  float gs[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int row = r0 + ty + 16 * i;
-    if (row < D.m && col < D.n) {  // n % 4 == 0: the 4 columns are all in or all out
-      const long long off = (long long)row * D.ld + col;
-      m4s[i] = *reinterpret_cast<const float4*>(D.M + off);
-      if (D.g_bf16) {
-        bf16x4_to_float(*reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(D.G) + off), gs[i]);
-      } else {
-        const float4 g4 = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(D.G) + off);
-        gs[i][0] = g4.x; gs[i][1] = g4.y; gs[i][2] = g4.z; gs[i][3] = g4.w;
-      }
-    }
-  }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int rl = ty + 16 * i;
     const int row = r0 + rl;
     float mv[4] = {0.f, 0.f, 0.f, 0.f};
-    if (row < D.m && col < D.n) {
+    if (row < D.m && col < D.n) {  // n % 4 == 0: the 4 columns are all in or all out
       const long long off = (long long)row * D.ld + col;
-      const float4 m4 = m4s[i];
-      const float* g = gs[i];
+      float4 m4 = *reinterpret_cast<const float4*>(D.M + off);
+      float g[4];
+      if (D.g_bf16) {
+        bf16x4_to_float(*reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(D.G) + off), g);
+      } else {
+        float4 g4 = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(D.G) + off);
+        g[0] = g4.x; g[1] = g4.y; g[2] = g4.z; g[3] = g4.w;
+      }
       mv[0] = mu * m4.x + om * g[0];
       mv[1] = mu * m4.y + om * g[1];
       mv[2] = mu * m4.z + om * g[2];
@@ -404,19 +392,13 @@ __global__ void __launch_bounds__(256) muon_update_kernel(const MuonMatDev* __re
   }
   float acc = 0.f;
   int bad = 0;
-  float4 ws4[4];  // every W load first (stores could alias later loads as far as the compiler knows)
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int row = r0 + ty + 16 * i;
-    if (row < D.m && col < D.n) ws4[i] = *reinterpret_cast<const float4*>(D.W + (long long)row * D.ld + col);
-  }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int row = r0 + ty + 16 * i;
     if (row >= D.m || col >= D.n) continue;
     const float rs = om * (use_rows ? D.rowscale[row] : 1.0f);
     float* wp = D.W + (long long)row * D.ld + col;
-    const float4 w = ws4[i];
+    float4 w = *reinterpret_cast<float4*>(wp);
     float wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {

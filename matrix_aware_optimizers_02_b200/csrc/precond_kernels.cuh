@@ -55,70 +55,47 @@ __device__ __forceinline__ float4 load4(const void* base, long long off, int is_
   return *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + off);
 }
 
-// The 4-element groups of a job handled by this block, thread by thread: the
-// NG = kElemsPerBlock / 1024 groups of thread t are g0 + k * 256 + t.  Passes load every
-// group's inputs first and store afterwards, so that a thread has all its loads in
-// flight at once (stores to the outputs could alias the inputs of a later group as far
-// as the compiler knows).
-constexpr int kGroupsPerThread = kElemsPerBlock / 4 / 256;
-
-struct EwGroups {
-  int r[kGroupsPerThread], c[kGroupsPerThread];
-  bool ok[kGroupsPerThread];
-};
-
-__device__ __forceinline__ EwGroups ew_groups(int rows, int cols, int local) {
-  EwGroups g;
-  const long long groups = (long long)rows * (cols / 4);
-  const long long g0 = (long long)local * (kElemsPerBlock / 4);
-#pragma unroll
-  for (int k = 0; k < kGroupsPerThread; ++k) {
-    const long long q = g0 + k * 256 + threadIdx.x;
-    g.ok[k] = q < groups;
-    const long long qq = g.ok[k] ? q : 0;
-    g.r[k] = (int)(qq / (cols / 4));
-    g.c[k] = (int)(qq - (long long)g.r[k] * (cols / 4)) * 4;
+// Iterate the 4-element groups of the job handled by this block.  cols % 4 == 0.
+#define MAO_EW_LOOP(J, local, ...)                                                         \
+  {                                                                                        \
+    const long long _groups = (long long)(J).rows * ((J).cols / 4);                        \
+    const long long _g0 = (long long)(local) * (kElemsPerBlock / 4);                       \
+    for (int _k = 0; _k < kElemsPerBlock / 4 / 256; ++_k) {                                \
+      const long long _g = _g0 + _k * 256 + threadIdx.x;                                   \
+      if (_g >= _groups) break;                                                            \
+      const int r = (int)(_g / ((J).cols / 4));                                            \
+      const int c = (int)(_g - (long long)r * ((J).cols / 4)) * 4;                         \
+      __VA_ARGS__                                                                          \
+    }                                                                                      \
   }
-  return g;
-}
 
 // M <- b1 M + (1-b1) G.  a = G (lda), f0 = M (in place, ldf); planes of G -> pa
 // (unless nullptr), planes of the new M -> pb (ldp).
 __global__ void __launch_bounds__(256) pc_momentum_kernel(const EwJob* __restrict__ J, int n, float b1) {
   const EwJob& j = J[find_job(J, n, blockIdx.x)];
-  const EwGroups q = ew_groups(j.rows, j.cols, blockIdx.x - j.blk_begin);
-  float4 g[kGroupsPerThread], m[kGroupsPerThread];
-#pragma unroll
-  for (int k = 0; k < kGroupsPerThread; ++k) {
-    if (!q.ok[k]) continue;
-    g[k] = load4(j.a, (long long)q.r[k] * j.lda + q.c[k], j.a_bf16);
-    m[k] = *reinterpret_cast<const float4*>(j.f0 + (long long)q.r[k] * j.ldf + q.c[k]);
-  }
-#pragma unroll
-  for (int k = 0; k < kGroupsPerThread; ++k) {
-    if (!q.ok[k]) continue;
-    const float4 mn = make_float4(b1 * m[k].x + (1.f - b1) * g[k].x, b1 * m[k].y + (1.f - b1) * g[k].y,
-                                  b1 * m[k].z + (1.f - b1) * g[k].z, b1 * m[k].w + (1.f - b1) * g[k].w);
-    *reinterpret_cast<float4*>(j.f0 + (long long)q.r[k] * j.ldf + q.c[k]) = mn;
-    const long long o = (long long)q.r[k] * j.ldp + q.c[k];
-    if (j.pa) store_split3x4(g[k], j.pa, o, j.pstride);
+  const int local = blockIdx.x - j.blk_begin;
+  MAO_EW_LOOP(j, local, {
+    const float4 g = load4(j.a, (long long)r * j.lda + c, j.a_bf16);
+    float* mp = j.f0 + (long long)r * j.ldf + c;
+    const float4 m = *reinterpret_cast<const float4*>(mp);
+    const float4 mn = make_float4(b1 * m.x + (1.f - b1) * g.x, b1 * m.y + (1.f - b1) * g.y,
+                                  b1 * m.z + (1.f - b1) * g.z, b1 * m.w + (1.f - b1) * g.w);
+    *reinterpret_cast<float4*>(mp) = mn;
+    const long long o = (long long)r * j.ldp + c;
+    if (j.pa) store_split3x4(g, j.pa, o, j.pstride);
     store_split3x4(mn, j.pb, o, j.pstride);
-  }
+  })
 }
 
 // Three-plane split of an fp32 matrix: a (lda) -> pa planes (ldp).  Gated by flag.
 __global__ void __launch_bounds__(256) pc_split_kernel(const EwJob* __restrict__ J, int n) {
   const EwJob& j = J[find_job(J, n, blockIdx.x)];
   if (j.flag && *j.flag == 0) return;
-  const EwGroups q = ew_groups(j.rows, j.cols, blockIdx.x - j.blk_begin);
-  float4 x[kGroupsPerThread];
-#pragma unroll
-  for (int k = 0; k < kGroupsPerThread; ++k)
-    if (q.ok[k]) x[k] = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(j.a) +
-                                                         (long long)q.r[k] * j.lda + q.c[k]);
-#pragma unroll
-  for (int k = 0; k < kGroupsPerThread; ++k)
-    if (q.ok[k]) store_split3x4(x[k], j.pa, (long long)q.r[k] * j.ldp + q.c[k], j.pstride);
+  const int local = blockIdx.x - j.blk_begin;
+  MAO_EW_LOOP(j, local, {
+    const float4 x = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(j.a) + (long long)r * j.lda + c);
+    store_split3x4(x, j.pa, (long long)r * j.ldp + c, j.pstride);
+  })
 }
 
 // SOAP Adam in the eigenbasis.  a = Ghat (lda), b = Mhat (ldb), f0 = V (caller, ldf),
@@ -127,29 +104,21 @@ __global__ void __launch_bounds__(256) pc_split_kernel(const EwJob* __restrict__
 __global__ void __launch_bounds__(256) soap_adam_kernel(const EwJob* __restrict__ J, int n, float b2, float inv_bc1,
                                                         float inv_bc2, float eps) {
   const EwJob& j = J[find_job(J, n, blockIdx.x)];
-  const EwGroups q = ew_groups(j.rows, j.cols, blockIdx.x - j.blk_begin);
-  float4 g[kGroupsPerThread], m[kGroupsPerThread], vp[kGroupsPerThread];
-  const float* vsrc = j.f1 ? j.f1 : j.f0;
-#pragma unroll
-  for (int k = 0; k < kGroupsPerThread; ++k) {
-    if (!q.ok[k]) continue;
-    g[k] = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(j.a) + (long long)q.r[k] * j.lda + q.c[k]);
-    m[k] = *reinterpret_cast<const float4*>(j.b + (long long)q.r[k] * j.ldb + q.c[k]);
-    vp[k] = *reinterpret_cast<const float4*>(vsrc + (long long)q.r[k] * j.ldf + q.c[k]);
-  }
-#pragma unroll
-  for (int k = 0; k < kGroupsPerThread; ++k) {
-    if (!q.ok[k]) continue;
-    float gv[4] = {g[k].x, g[k].y, g[k].z, g[k].w}, mv[4] = {m[k].x, m[k].y, m[k].z, m[k].w};
-    float v[4] = {vp[k].x, vp[k].y, vp[k].z, vp[k].w}, nv[4];
+  const int local = blockIdx.x - j.blk_begin;
+  MAO_EW_LOOP(j, local, {
+    const float4 g = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(j.a) + (long long)r * j.lda + c);
+    const float4 m = *reinterpret_cast<const float4*>(j.b + (long long)r * j.ldb + c);
+    const long long of = (long long)r * j.ldf + c;
+    const float4 vp = *reinterpret_cast<const float4*>((j.f1 ? j.f1 : j.f0) + of);
+    float gv[4] = {g.x, g.y, g.z, g.w}, mv[4] = {m.x, m.y, m.z, m.w}, v[4] = {vp.x, vp.y, vp.z, vp.w}, nv[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       v[e] = b2 * v[e] + (1.f - b2) * gv[e] * gv[e];
       nv[e] = (mv[e] * inv_bc1) / (sqrtf(v[e] * inv_bc2) + eps);
     }
-    *reinterpret_cast<float4*>(j.f0 + (long long)q.r[k] * j.ldf + q.c[k]) = make_float4(v[0], v[1], v[2], v[3]);
-    store_split3x4(make_float4(nv[0], nv[1], nv[2], nv[3]), j.pa, (long long)q.r[k] * j.ldp + q.c[k], j.pstride);
-  }
+    *reinterpret_cast<float4*>(j.f0 + of) = make_float4(v[0], v[1], v[2], v[3]);
+    store_split3x4(make_float4(nv[0], nv[1], nv[2], nv[3]), j.pa, (long long)r * j.ldp + c, j.pstride);
+  })
 }
 
 // ------------------------------------------------------------------ sort keys / permutation
@@ -805,31 +774,20 @@ __global__ void __launch_bounds__(256) foam_tau_kernel(const TauJob* __restrict_
 __global__ void __launch_bounds__(256) foam_n_kernel(const EwJob* __restrict__ J, int n, float inv_bc1,
                                                      float inv_bc2, float eps) {
   const EwJob& j = J[find_job(J, n, blockIdx.x)];
-  const EwGroups q = ew_groups(j.rows, j.cols, blockIdx.x - j.blk_begin);
+  const int local = blockIdx.x - j.blk_begin;
   const float tau = *j.b;
-  float4 mr[kGroupsPerThread], cv[kGroupsPerThread];
-  float rv[kGroupsPerThread];
-#pragma unroll
-  for (int k = 0; k < kGroupsPerThread; ++k) {
-    if (!q.ok[k]) continue;
-    mr[k] = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(j.a) + (long long)q.r[k] * j.lda + q.c[k]);
-    cv[k] = *reinterpret_cast<const float4*>(j.vc + q.c[k]);
-    rv[k] = j.vr[q.r[k]];
-  }
-#pragma unroll
-  for (int k = 0; k < kGroupsPerThread; ++k) {
-    if (!q.ok[k]) continue;
-    const float ri = rv[k] * inv_bc2;
-    const float mv[4] = {mr[k].x, mr[k].y, mr[k].z, mr[k].w};
-    const float cc[4] = {cv[k].x, cv[k].y, cv[k].z, cv[k].w};
+  MAO_EW_LOOP(j, local, {
+    const float4 mr = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(j.a) + (long long)r * j.lda + c);
+    const float ri = j.vr[r] * inv_bc2;
+    const float mv[4] = {mr.x, mr.y, mr.z, mr.w};
     float nv[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float v = tau * ri * (cc[e] * inv_bc2);
+      const float v = tau * ri * (j.vc[c + e] * inv_bc2);
       nv[e] = (mv[e] * inv_bc1) / (sqrtf(v) + eps);
     }
-    store_split3x4(make_float4(nv[0], nv[1], nv[2], nv[3]), j.pa, (long long)q.r[k] * j.ldp + q.c[k], j.pstride);
-  }
+    store_split3x4(make_float4(nv[0], nv[1], nv[2], nv[3]), j.pa, (long long)r * j.ldp + c, j.pstride);
+  })
 }
 
 // Adaptive check: rho = ||offdiag D||_F / ||D||_F, flag = rho > tol (one block per matrix).
