@@ -86,7 +86,7 @@ mao_status gemm_layout(int32_t kind_flags, int32_t batch, int32_t M, int32_t N, 
     T.planes[0] = cv.take(3 * 2 * (size_t)batch * M * K);
     T.planes[1] = cv.take(3 * 2 * (size_t)batch * N * K);
     // per batch element: one problem and six descriptors
-    T.arena_bytes = align_up(sizeof(GemmProblem) * batch, 64) + sizeof(CUtensorMap) * 6 * batch + 256;
+    T.arena_bytes = align_up((sizeof(GemmProblem) + 2 * sizeof(int)) * batch, 64) + sizeof(CUtensorMap) * 6 * batch + 256;
     T.arena = cv.take(T.arena_bytes);
   }
   T.total = cv.total();

@@ -284,8 +284,10 @@ StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off) {
   S.pb = L.pb;
   S.kernel_id = L.kernel_id;
   if (S.nprob == 0) return S;
-  S.probs_off = A.take(sizeof(GemmProblem) * S.nprob, 64);
+  // the problem records, then their first tiles in both numberings (searched by the kernels)
+  S.probs_off = A.take(sizeof(GemmProblem) * S.nprob + 2 * sizeof(int) * S.nprob, 64);
   GemmProblem* hp = A.hptr<GemmProblem>(S.probs_off);
+  int* starts = reinterpret_cast<int*>(hp + S.nprob);
   const CUtensorMap* mbase = A.dptr<const CUtensorMap>(maps_off);
   int t = 0, t2 = 0;
   for (int i = 0; i < S.nprob; ++i) {
@@ -303,6 +305,8 @@ StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off) {
     // by a device flag may be skipped, so it counts nothing: a lower bound)
     if (P.flag == nullptr) S.flops += 2.0 * P.M * (double)P.N * P.K;
     hp[i] = P;
+    starts[i] = P.tile_begin;
+    starts[S.nprob + i] = P.tile_begin2;
   }
   S.total_tiles = t;
   S.total_tiles2 = t2;

@@ -339,12 +339,10 @@ struct TableSource {
   __device__ void prefetch() const {}
   __device__ TileInfo decode(int tile, int BM, int BN) const {
     const bool pair = BM == 256;
-    int lo = 0, hi = p.nprob - 1;
-#pragma unroll 1
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if ((pair ? p.probs[mid].tile_begin2 : p.probs[mid].tile_begin) <= tile) lo = mid; else hi = mid - 1;
-    }
+    // the staged table is followed by the problems' first tiles (one-CTA numbering, then
+    // the CTA-pair numbering): a compact search instead of probing the large records
+    const int* starts = reinterpret_cast<const int*>(p.probs + p.nprob) + (pair ? p.nprob : 0);
+    const int lo = find_start(starts, p.nprob, tile);
     const GemmProblem& P = p.probs[lo];
     const int r = tile - (pair ? P.tile_begin2 : P.tile_begin);
     TileInfo t;

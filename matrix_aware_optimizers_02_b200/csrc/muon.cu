@@ -218,8 +218,9 @@ void plan(const mao_muon_mat* mats, int count, const int* ld, int callers, const
     }
     // at most 27 tensor maps per matrix (3 planes of X[2] in three views, of A in two,
     // of B in one) and one problem per matrix in each of 3 launches per iteration
-    P.arena_cap = (size_t)count * (27 * sizeof(CUtensorMap) + 3 * kMopSteps * sizeof(GemmProblem)) +
-                  (3 * kMopSteps + 1) * 64 + 4096;
+    P.arena_cap =
+        (size_t)count * (27 * sizeof(CUtensorMap) + 3 * kMopSteps * (sizeof(GemmProblem) + 2 * sizeof(int))) +
+        (3 * kMopSteps + 1) * 64 + 4096;
     P.off_arena = cv.take(P.arena_cap);
   }
   P.total = cv.total();
