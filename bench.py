@@ -687,9 +687,10 @@ def run_mine(args, rank, world, dist):
     if clocks:
         clocks.start()
         time.sleep(0.3)
+    # the timed region: K steps as a caller runs them (the library only counts its launches)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    L.check(lib.mao_profile_start(ev_arr, info, cap))
+    lib.mao_profile_start(None, None, 0)
     t_start.record(stream)
     for k in range(args.steps):
         t += 1
@@ -706,9 +707,30 @@ def run_mine(args, rank, world, dist):
     if bad:
         raise RuntimeError(f"device status {bad} after timed steps")
 
+    # the kernel table and the roofline: K more steps with every library launch bracketed
+    # by events on its stream (the events themselves cost time, so this region is not the
+    # step time above)
+    barrier()
+    torch.cuda.synchronize()
+    k_start = torch.cuda.Event(enable_timing=True)
+    k_end = torch.cuda.Event(enable_timing=True)
+    L.check(lib.mao_profile_start(ev_arr, info, cap))
+    k_start.record(stream)
+    for k in range(args.steps):
+        t += 1
+        LS.step(t, stream)
+    k_end.record(stream)
+    n_prof = lib.mao_profile_stop()
+    torch.cuda.synchronize()
+    barrier()
+    ms_instrumented = k_start.elapsed_time(k_end) / args.steps
+    bad = LS.status()
+    if bad:
+        raise RuntimeError(f"device status {bad} after the instrumented steps")
+
     # per-kernel live durations
     per = {}
-    for i in range(min(n_launch, cap)):
+    for i in range(min(n_prof, cap)):
         kk = info[i].kernel
         d = evs[2 * i].elapsed_time(evs[2 * i + 1])
         e = per.setdefault(kk, {"ms": 0.0, "n": 0, "flops": 0.0, "bytes": 0.0, "tc": 0.0})
@@ -824,6 +846,9 @@ def run_mine(args, rank, world, dist):
                             f"every {args.soap_k} steps, sorted"},
                    "foam": {"beta1": 0.95, "beta2": 0.95, "eps": 1e-8, "refresh": "adaptive pf=10 tol=0.1"},
                    "timed_steps_t": [args.warmup + 2, args.warmup + 1 + args.steps],
+                   "kernel_table": (f"per-launch CUDA events over {args.steps} further steps (t = "
+                                    f"{args.warmup + 2 + args.steps}..{args.warmup + 1 + 2 * args.steps}); "
+                                    f"{round(ms_instrumented, 1)} ms per step with the events"),
                    "matrices_per_rank": len(specs), "elements_per_rank": n_elems,
                    "gradient_sets": 3,
                    "inputs": "three device-resident seeded gradient sets, step t uses set (t - 1) mod 3",

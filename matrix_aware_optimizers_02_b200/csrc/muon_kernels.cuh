@@ -62,6 +62,12 @@ __device__ __forceinline__ int find_mat(const MuonMatDev* T, int count, int blk)
   return find_start(reinterpret_cast<const int*>(T + count), count, blk);
 }
 
+// Start moving a line toward L2 without holding registers for it (the load that
+// follows finds it there, so the row loads of a thread overlap instead of queuing).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ void bf16x4_to_float(uint2 raw, float* v) {
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
   float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
@@ -155,6 +161,17 @@ __global__ void __launch_bounds__(256) muon_prep_kernel(const MuonMatDev* __rest
   const int col = c0 + tx * 4;
   const float om = 1.0f - mu;
   float acc = 0.0f;
+  if (col < D.n) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int row = r0 + ty + 16 * i;
+      if (row < D.m) {
+        const long long off = (long long)row * D.ld + col;
+        prefetch_l2(D.M + off);
+        prefetch_l2(static_cast<const char*>(D.G) + off * (D.g_bf16 ? 2 : 4));
+      }
+    }
+  }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int rl = ty + 16 * i;
@@ -381,10 +398,17 @@ __global__ void __launch_bounds__(256) muon_update_kernel(const MuonMatDev* __re
   const int local = blockIdx.x - D.tile_begin;
   const int r0 = (local / D.tiles_c) * kTile, c0 = (local % D.tiles_c) * kTile;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int col = c0 + 4 * tx;
+  if (col < D.n) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int row = r0 + ty + 16 * i;
+      if (row < D.m) prefetch_l2(D.W + (long long)row * D.ld + col);
+    }
+  }
   float v[4][4];
   load_o_tile<OT>(D, o_of<OT>(D), r0, c0, v, sm);
   const float om = D.oscale ? *D.oscale : 1.0f;
-  const int col = c0 + 4 * tx;
   float cs[4] = {1.f, 1.f, 1.f, 1.f};
   if (use_cols && col < D.n) {
 #pragma unroll
