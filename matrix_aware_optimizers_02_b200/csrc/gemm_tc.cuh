@@ -189,17 +189,51 @@ __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* ma
   }
 }
 
+// 256-bit global stores: a lane writes one whole 32-byte sector per instruction
+// (16-byte stores leave each sector half written twice, and the L1 sends both
+// halves to L2 as separate partial-sector writes).
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t* w) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
+__device__ __forceinline__ bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
+// 32 consecutive fp32 (16-byte aligned; whole sectors when 32-byte aligned)
+__device__ __forceinline__ void store_f32x32(float* dst, const float* v) {
+  if (aligned32(dst)) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+      uint32_t w[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[e] = __float_as_uint(v[j + e]);
+      st_global_v8(dst + j, w);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; j += 4)
+      *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+  }
+}
+
+// 32 consecutive bf16, rounded to nearest (16-byte aligned; whole sectors when
+// 32-byte aligned)
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v) {
-  uint4 pk[4];
-  uint32_t* w = reinterpret_cast<uint32_t*>(pk);
+  uint32_t w[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
     w[j] = *reinterpret_cast<uint32_t*>(&h);
   }
-  uint4* d = reinterpret_cast<uint4*>(dst);
+  if (aligned32(dst)) {
+    st_global_v8(dst, w);
+    st_global_v8(dst + 16, w + 8);
+  } else {
+    uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-  for (int j = 0; j < 4; ++j) d[j] = pk[j];
+    for (int j = 0; j < 4; ++j) d[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  }
 }
 
 __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float* v) {
@@ -283,7 +317,9 @@ struct ClassSource {
           *reinterpret_cast<float4*>(out + j) =
               make_float4(p.alpha * v[j], p.alpha * v[j + 1], p.alpha * v[j + 2], p.alpha * v[j + 3]);
       } else {
-        for (int j = 0; j < 32 && col0 + j < C.N; ++j) out[j] = p.alpha * v[j];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j < C.N) out[j] = p.alpha * v[j];
       }
     } else {
       const float s = C.scale ? C.scale[b] : 1.0f;
@@ -314,7 +350,9 @@ struct ClassSource {
       if (full) {
         store_bf16x32(out, v);
       } else {
-        for (int j = 0; j < 32 && col0 + j < C.N; ++j) out[j] = __float2bfloat16_rn(v[j]);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j < C.N) out[j] = __float2bfloat16_rn(v[j]);
       }
       if constexpr (EPI == EPI_AXPY_T) {
         if (C.out1 != nullptr) {
@@ -364,23 +402,52 @@ struct TableSource {
   }
   __device__ int cols(const TileInfo& t) const { return p.probs[t.idx].N; }
 
+  // One problem's epilogue parameters, read once per tile with the device-chosen
+  // destination resolved: held in registers, they are not re-read after every store
+  // (the stores could alias the problem records as far as the compiler knows).
+  struct Epi {
+    float* out;
+    __nv_bfloat16* outp[3];
+    const float* aux;
+    float2* upd;
+    int M, N, ld_out, ld_outp, ld_aux;
+    float alpha, beta;
+  };
+  __device__ __forceinline__ Epi epi(const TileInfo& t) const {
+    const GemmProblem& P = p.probs[t.idx];
+    Epi e;
+    const bool alt = (P.sel != nullptr) && (*P.sel == 0);
+    e.out = alt ? P.out2 : P.out;
+#pragma unroll
+    for (int q = 0; q < 3; ++q) e.outp[q] = alt ? P.out2_p[q] : P.out_p[q];
+    e.ld_out = alt ? P.ld_out2 : P.ld_out;
+    e.ld_outp = alt ? P.ld_out2p : P.ld_outp;
+    e.aux = P.aux;
+    e.upd = P.upd;
+    e.M = P.M;
+    e.N = P.N;
+    e.ld_aux = P.ld_aux;
+    e.alpha = P.alpha;
+    e.beta = P.beta;
+    return e;
+  }
+
   // out = alpha * acc + beta * aux for 32 columns of one row; `st` accumulates the
   // update statistics (sum of (out - aux)^2, non-finite count) when the problem asks.
-  __device__ __forceinline__ void epilogue_table(const TileInfo& t, int row, int col0, float* v, float2& st) const {
-    const GemmProblem& P = p.probs[t.idx];
-    if (row >= P.M) return;
-    const bool full = (col0 + 32 <= P.N);
-    if (P.aux != nullptr) {
-      const float* a = P.aux + (long long)row * P.ld_aux + col0;
-      const bool want = P.upd != nullptr;
+  __device__ __forceinline__ void epilogue_table(const Epi& e, int row, int col0, float* v, float2& st) const {
+    if (row >= e.M) return;
+    const bool full = (col0 + 32 <= e.N);
+    if (e.aux != nullptr) {
+      const float* a = e.aux + (long long)row * e.ld_aux + col0;
+      const bool want = e.upd != nullptr;
       if (full) {
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
           const float4 q = *reinterpret_cast<const float4*>(a + j);
-          v[j] = P.alpha * v[j] + P.beta * q.x;
-          v[j + 1] = P.alpha * v[j + 1] + P.beta * q.y;
-          v[j + 2] = P.alpha * v[j + 2] + P.beta * q.z;
-          v[j + 3] = P.alpha * v[j + 3] + P.beta * q.w;
+          v[j] = e.alpha * v[j] + e.beta * q.x;
+          v[j + 1] = e.alpha * v[j + 1] + e.beta * q.y;
+          v[j + 2] = e.alpha * v[j + 2] + e.beta * q.z;
+          v[j + 3] = e.alpha * v[j + 3] + e.beta * q.w;
           if (want) {
             const float d0 = v[j] - q.x, d1 = v[j + 1] - q.y, d2 = v[j + 2] - q.z, d3 = v[j + 3] - q.w;
             st.x += (d0 * d0 + d1 * d1) + (d2 * d2 + d3 * d3);
@@ -388,10 +455,11 @@ struct TableSource {
           }
         }
       } else {
+#pragma unroll
         for (int j = 0; j < 32; ++j) {
-          if (col0 + j < P.N) {
+          if (col0 + j < e.N) {
             const float old = a[j];
-            v[j] = P.alpha * v[j] + P.beta * old;
+            v[j] = e.alpha * v[j] + e.beta * old;
             if (want) {
               const float d = v[j] - old;
               st.x += d * d;
@@ -404,25 +472,20 @@ struct TableSource {
       }
     } else {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] *= P.alpha;
+      for (int j = 0; j < 32; ++j) v[j] *= e.alpha;
     }
-    const bool alt = (P.sel != nullptr) && (*P.sel == 0);
-    float* const out = alt ? P.out2 : P.out;
-    const int ld_out = alt ? P.ld_out2 : P.ld_out;
-    const long long off = (long long)row * ld_out + col0;
-    if (out != nullptr) {
-      float* o = out + off;
+    if (e.out != nullptr) {
+      float* o = e.out + (long long)row * e.ld_out + col0;
       if (full) {
-#pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(o + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        store_f32x32(o, v);
       } else {
-        for (int j = 0; j < 32 && col0 + j < P.N; ++j) o[j] = v[j];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j < e.N) o[j] = v[j];
       }
     }
-    __nv_bfloat16* const* out_p = alt ? P.out2_p : P.out_p;
-    if (out_p[0] != nullptr) {
-      const long long offp = (long long)row * (alt ? P.ld_out2p : P.ld_outp) + col0;
+    if (e.outp[0] != nullptr) {
+      const long long offp = (long long)row * e.ld_outp + col0;
       float r[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) r[j] = v[j];
@@ -434,11 +497,13 @@ struct TableSource {
           pq[j] = __bfloat162float(__float2bfloat16_rn(r[j]));
           r[j] -= pq[j];
         }
-        __nv_bfloat16* o = out_p[q] + offp;
+        __nv_bfloat16* o = e.outp[q] + offp;
         if (full) {
           store_bf16x32(o, pq);
         } else {
-          for (int j = 0; j < 32 && col0 + j < P.N; ++j) o[j] = __float2bfloat16_rn(pq[j]);
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (col0 + j < e.N) o[j] = __float2bfloat16_rn(pq[j]);
         }
       }
     }
@@ -446,15 +511,14 @@ struct TableSource {
 
   // Warp-level reduction of the update statistics of the 32 x 64 block whose first
   // row / column are row0 / col0 (every lane of the warp calls this; fixed order).
-  __device__ __forceinline__ void flush_stats(const TileInfo& t, int row0, int col0, float2 st, int lane) const {
-    const GemmProblem& P = p.probs[t.idx];
-    if (P.upd == nullptr) return;
+  __device__ __forceinline__ void flush_stats(const Epi& e, int row0, int col0, float2 st, int lane) const {
+    if (e.upd == nullptr) return;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       st.x += __shfl_xor_sync(0xffffffffu, st.x, o);
       st.y += __shfl_xor_sync(0xffffffffu, st.y, o);
     }
-    if (lane == 0 && row0 < P.M && col0 < P.N) P.upd[(long long)(row0 >> 5) * ((P.N + 63) >> 6) + (col0 >> 6)] = st;
+    if (lane == 0 && row0 < e.M && col0 < e.N) e.upd[(long long)(row0 >> 5) * ((e.N + 63) >> 6) + (col0 >> 6)] = st;
   }
 };
 
@@ -698,10 +762,11 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
         if constexpr (EPI == EPI_TABLE) {
           static_assert(COLS == 64, "update statistics assume 64 columns per epilogue warp");
           float2 st = make_float2(0.f, 0.f);
+          const auto e = src.epi(t);
 #pragma unroll
           for (int ch = 0; ch < COLS / 32; ++ch)
-            if (t.n0 + cb + ch * 32 < ncols) src.epilogue_table(t, row, t.n0 + cb + ch * 32, &run[ch * 32], st);
-          src.flush_stats(t, t.m0 + q * 32, t.n0 + cb, st, lane);
+            if (t.n0 + cb + ch * 32 < ncols) src.epilogue_table(e, row, t.n0 + cb + ch * 32, &run[ch * 32], st);
+          src.flush_stats(e, t.m0 + q * 32, t.n0 + cb, st, lane);
         } else {
 #pragma unroll
           for (int ch = 0; ch < COLS / 32; ++ch)
@@ -977,10 +1042,11 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
       if (!ok) break;
       static_assert(COLS == 64, "update statistics assume 64 columns per epilogue warp");
       float2 st = make_float2(0.f, 0.f);
+      const TableSource::Epi e = src.epi(t);
 #pragma unroll
       for (int ch = 0; ch < COLS / 32; ++ch)
-        if (t.n0 + cb + ch * 32 < ncols) src.epilogue_table(t, row, t.n0 + cb + ch * 32, &run[ch * 32], st);
-      src.flush_stats(t, t.m0 + 128 * (int)rank + q * 32, t.n0 + cb, st, lane);
+        if (t.n0 + cb + ch * 32 < ncols) src.epilogue_table(e, row, t.n0 + cb + ch * 32, &run[ch * 32], st);
+      src.flush_stats(e, t.m0 + 128 * (int)rank + q * 32, t.n0 + cb, st, lane);
     }
   }
 
