@@ -720,7 +720,7 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
           if (t.n0 + cb + ch * 32 < ncols) src.template epilogue<EPI>(t, row, t.n0 + cb + ch * 32, v);
         }
         tc_fence_before();
-        mbar_arrive(&tempty_bar[acc]);
+        mbar_arrive_relaxed(&tempty_bar[acc]);
       } else {
         // fold the K-chunk accumulators (main + correction) into fp32 registers
         const int nk = (t.K + BK - 1) / BK;
@@ -756,7 +756,7 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
             }
           }
           tc_fence_before();
-          mbar_arrive(&tempty_bar[acc]);
+          mbar_arrive_relaxed(&tempty_bar[acc]);
         }
         if (!ok) break;
         if constexpr (EPI == EPI_TABLE) {
@@ -1037,7 +1037,7 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
           }
         }
         tc_fence_before();
-        mbar_arrive_cluster(tempty_lead[acc]);
+        mbar_arrive_cluster_relaxed(tempty_lead[acc]);
       }
       if (!ok) break;
       static_assert(COLS == 64, "update statistics assume 64 columns per epilogue warp");
