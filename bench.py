@@ -211,8 +211,10 @@ def write_launch_log(args, lib, L, LS, t, stream):
         LS.step(t, stream)  # the same t: the same launch plan
     m = lib.mao_profile_stop()
     torch.cuda.synchronize()
-    rows = [{"kernel": L.KERNEL_NAMES.get(info[i].kernel, str(info[i].kernel)), "flops": info[i].flops,
-             "bytes": info[i].bytes, "tc_flops": info[i].tc_flops} for i in range(min(n, m))]
+    # executed work (device counters for the table-mode products), and the host's count
+    rows = [{"kernel": L.KERNEL_NAMES.get(info[i].kernel, str(info[i].kernel)), "flops": info[i].exec_flops,
+             "bytes": info[i].bytes, "tc_flops": info[i].exec_tc_flops, "planned_flops": info[i].flops}
+            for i in range(min(n, m))]
     with open(args.launch_log, "w") as f:
         json.dump({"workload": args.workload, "optimizers": args.optimizers, "source_hash": kernel_source_hash(),
                    "launches": rows}, f)
@@ -733,12 +735,15 @@ def run_mine(args, rank, world, dist):
     for i in range(min(n_prof, cap)):
         kk = info[i].kernel
         d = evs[2 * i].elapsed_time(evs[2 * i + 1])
-        e = per.setdefault(kk, {"ms": 0.0, "n": 0, "flops": 0.0, "bytes": 0.0, "tc": 0.0})
+        e = per.setdefault(kk, {"ms": 0.0, "n": 0, "flops": 0.0, "bytes": 0.0, "tc": 0.0, "planned": 0.0})
         e["ms"] += d
         e["n"] += 1
-        e["flops"] += info[i].flops
+        # the work the device executed (table-mode products count their computed tiles on
+        # the device, so the passes it decides to run are included)
+        e["flops"] += info[i].exec_flops
         e["bytes"] += info[i].bytes
-        e["tc"] += info[i].tc_flops
+        e["tc"] += info[i].exec_tc_flops
+        e["planned"] += info[i].flops
 
     # end-to-end: this step's gradient set from pinned host memory, the step, stats back to host
     host_sets = [[g.cpu().pin_memory() for g in Gs] for Gs in LS.G_sets]
@@ -790,7 +795,11 @@ def run_mine(args, rank, world, dist):
                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                     "useful_tflops": round(useful, 1),
                     "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step); achieved counts "
-                                   "the bf16 tensor-core products issued (6 per fp32-faithful multiply-add)"}
+                                   "the bf16 tensor-core products the kernel issued (6 per fp32-faithful "
+                                   "multiply-add), over the tiles it computed (device counters: the passes "
+                                   "decided on the device included)"}
+            if e["planned"] < e["flops"]:
+                roof["useful_tflops_host_counted"] = round((e["planned"] / e["n"]) / (avg_ms * 1e-3) / 1e12, 1)
         else:
             achieved = (e["bytes"] / e["n"]) / (avg_ms * 1e-3) / 1e9
             peak = peaks["hbm_gbs"]

@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define MAO_VERSION 3
+#define MAO_VERSION 4
 
 #if defined(__GNUC__)
 #define MAO_API __attribute__((visibility("default")))
@@ -363,6 +363,11 @@ typedef struct {
   double tc_flops;  /* tensor-core operations issued for `flops`: an fp32-faithful product of
                        three-plane operands issues six bf16 products per multiply-add, a
                        three-plane by one-plane product three, a bf16 product one */
+  double exec_flops;    /* operations the device executed, filled by mao_profile_stop(): for a
+                           table-mode product counted over the tiles it computed, problems that
+                           a device flag let run included; for every other launch equal to
+                           flops */
+  double exec_tc_flops; /* tensor-core operations the device issued for exec_flops */
 } mao_launch_info;
 
 /*
@@ -372,8 +377,10 @@ typedef struct {
  * info[i] describes it, for the first `capacity` launches.  `events` is a host
  * array of 2*capacity cudaEvent_t created by the caller, or NULL to record only
  * `info`; `info` a host array of `capacity`.  mao_profile_stop() ends recording and returns how many launches
- * happened since the start (which may exceed capacity).  Not thread-safe: one
- * profiling session per process at a time.
+ * happened since the start (which may exceed capacity); with an `info` array it
+ * synchronises the device and fills the exec_* fields (the table-mode kernels count
+ * their executed work in device counters that mao_profile_start allocates once and
+ * clears).  Not thread-safe: one profiling session per process at a time.
  */
 MAO_API mao_status mao_profile_start(void** events, mao_launch_info* info, int32_t capacity);
 MAO_API int32_t mao_profile_stop(void);

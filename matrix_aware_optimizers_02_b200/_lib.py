@@ -75,7 +75,7 @@ class FoamParams(ctypes.Structure):
 
 class LaunchInfo(ctypes.Structure):
     _fields_ = [("kernel", c_int32), ("pad", c_int32), ("flops", ctypes.c_double), ("bytes", ctypes.c_double),
-                ("tc_flops", ctypes.c_double)]
+                ("tc_flops", ctypes.c_double), ("exec_flops", ctypes.c_double), ("exec_tc_flops", ctypes.c_double)]
 
 
 KERNEL_NAMES = {1: "muon_prep", 2: "muon_scale", 3: "ns_gram", 4: "ns_poly", 5: "ns_axpy", 6: "muon_colsq",

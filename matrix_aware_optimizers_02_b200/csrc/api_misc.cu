@@ -200,6 +200,20 @@ Profiler& profiler() {
 extern "C" mao_status mao_profile_start(void** events, mao_launch_info* info, int32_t capacity) {
   if (capacity < 0 || (capacity > 0 && info == nullptr)) return MAO_ERR_INVALID_ARG;
   Profiler& P = profiler();
+  if (info != nullptr && capacity > 0) {
+    // executed-work counters: kept for the process, grown on demand, cleared here
+    if (P.work_cap < capacity) {
+      if (P.work) cudaFree(P.work);
+      P.work = nullptr;
+      P.work_cap = 0;
+      MAO_CUDA_TRY(cudaMalloc(reinterpret_cast<void**>(&P.work), 2 * sizeof(unsigned long long) * capacity));
+      P.work_cap = capacity;
+    }
+    MAO_CUDA_TRY(cudaMemset(P.work, 0, 2 * sizeof(unsigned long long) * capacity));
+    P.counted.assign(capacity, 0);
+  } else {
+    P.counted.assign(std::max(capacity, 0), 0);
+  }
   P.events = events;
   P.info = info;
   P.capacity = capacity;
@@ -211,5 +225,25 @@ extern "C" mao_status mao_profile_start(void** events, mao_launch_info* info, in
 extern "C" int32_t mao_profile_stop(void) {
   Profiler& P = profiler();
   P.active = false;
+  if (P.info == nullptr) return P.count;
+  const int n = std::min(P.count, P.capacity);
+  std::vector<unsigned long long> h;
+  bool have = false;
+  bool any = false;
+  for (int i = 0; i < n; ++i) any = any || P.counted[i];
+  if (any && P.work != nullptr) {
+    h.resize(2 * (size_t)n);
+    have = cudaDeviceSynchronize() == cudaSuccess &&
+           cudaMemcpy(h.data(), P.work, sizeof(unsigned long long) * h.size(), cudaMemcpyDeviceToHost) == cudaSuccess;
+  }
+  for (int i = 0; i < n; ++i) {
+    if (have && P.counted[i]) {
+      P.info[i].exec_flops = (double)h[2 * i];
+      P.info[i].exec_tc_flops = (double)h[2 * i + 1];
+    } else {
+      P.info[i].exec_flops = P.info[i].flops;
+      P.info[i].exec_tc_flops = P.info[i].tc_flops;
+    }
+  }
   return P.count;
 }

@@ -318,6 +318,7 @@ StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off) {
   const bool pair_auto = L.pa == 3 || L.pb == 3;
   const int force = L.force_kernel ? L.force_kernel : table_kernel_policy();
   S.pair = force == 2 || (force == 0 && pair_auto && t2 >= 74 && 2.0 * t2 <= 1.2 * t);
+  S.any = L.any;
   return S;
 }
 
@@ -328,6 +329,15 @@ mao_status table_launch(const Arena& A, const StagedLaunch& S, DevStatus* status
   p.nprob = S.nprob;
   p.total_tiles = S.pair ? S.total_tiles2 : S.total_tiles;
   p.status = status;
+  p.any = S.any;
+  p.work = nullptr;
+  Profiler& prof = profiler();
+  const int total = S.pair ? S.total_tiles2 : S.total_tiles;
+  if (prof.active && prof.work != nullptr && total > 0 && prof.count < prof.capacity) {
+    // the launch below takes the profiler's next slot
+    p.work = prof.work + 2 * (size_t)prof.count;
+    prof.counted[prof.count] = 1;
+  }
   const int key = S.pa * 10 + S.pb;
   switch (key) {
     case 33: return launch_table_planes<3, 3>(p, S.a_mn, S.b_mn, stream, S.kernel_id, S.flops, S.pair);

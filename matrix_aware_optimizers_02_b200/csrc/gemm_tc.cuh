@@ -121,6 +121,12 @@ struct GemmTableParams {
   int nprob;
   int total_tiles;   // 128-row tiles (one CTA each), or 256-row tiles for the CTA-pair kernel
   DevStatus* status;
+  // nullptr, or a flag that is 0 when every problem of the launch is gated off: the
+  // launch then returns before any setup
+  const int* any;
+  // nullptr, or two counters (profiling): the work (multiply-adds x 2) of the tiles
+  // the kernel computed, and the tensor-core operations it issued
+  unsigned long long* work;
 };
 
 // PA / PB: bf16 planes held per operand (SPLIT3 kinds only; 1 = a plain bf16
@@ -264,10 +270,17 @@ struct TileInfo {
   int ko;      // operand coordinate offset along K
 };
 
+// bf16 tensor-core products per multiply-add of a (PA, PB)-plane product
+template <int PA, int PB>
+constexpr int kTileProducts = (PA == 3 && PB == 3) ? 6 : (PA == 1 && PB == 1) ? 1 : 3;
+
 // ------------------------------------------------------------------ class mode
 struct ClassSource {
   const GemmParams& p;
   __device__ explicit ClassSource(const GemmParams& p_) : p(p_) {}
+  __device__ bool skip_all() const { return false; }
+  template <int PRODUCTS>
+  __device__ void count_work(const TileInfo&, int, int) const {}
   __device__ int total_tiles() const { return p.total_tiles; }
   __device__ DevStatus* status() const { return p.status; }
   __device__ void prefetch() const {
@@ -372,6 +385,18 @@ struct ClassSource {
 struct TableSource {
   const GemmTableParams& p;
   __device__ explicit TableSource(const GemmTableParams& p_) : p(p_) {}
+  __device__ bool skip_all() const { return p.any != nullptr && *p.any == 0; }
+  // Profiling: the work of one computed tile (called once per tile by the MMA issuer).
+  template <int PRODUCTS>
+  __device__ void count_work(const TileInfo& t, int BM, int BN) const {
+    if (p.work == nullptr) return;
+    const GemmProblem& P = p.probs[t.idx];
+    const unsigned long long rows = (unsigned long long)min(BM, P.M - t.m0);
+    const unsigned long long cols = (unsigned long long)min(BN, P.N - t.n0);
+    const unsigned long long f = 2ull * rows * cols * (unsigned long long)t.K;
+    atomicAdd(p.work, f);
+    atomicAdd(p.work + 1, f * PRODUCTS);
+  }
   __device__ int total_tiles() const { return p.total_tiles; }
   __device__ DevStatus* status() const { return p.status; }
   __device__ void prefetch() const {}
@@ -549,6 +574,7 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   DevStatus* status = src.status();
+  if (src.skip_all()) return;  // uniform over the grid
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -626,6 +652,7 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileInfo t = src.decode(tile, BM, BN);
         if (!t.valid) continue;
+        src.template count_work<kTileProducts<PA, PB>>(t, BM, BN);
         const int nk = (t.K + BK - 1) / BK;
         const int nch = (KIND == OP_SPLIT3) ? (nk + Cfg::KCH - 1) / Cfg::KCH : 1;
         for (int c = 0; c < nch && ok; ++c) {
@@ -853,6 +880,8 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
   const int npairs = gridDim.x >> 1;
   const int pair_id = blockIdx.x >> 1;
   DevStatus* status = src.status();
+  // uniform over the grid: both CTAs of a pair leave before any cluster operation
+  if (src.skip_all()) return;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -939,6 +968,7 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
       for (int tile = pair_id; tile < total && ok; tile += npairs) {
         const TileInfo t = src.decode(tile, 256, BN);
         if (!t.valid) continue;
+        src.template count_work<kTileProducts<PA, PB>>(t, 256, BN);
         const int nk = (t.K + BK - 1) / BK;
         const int nch = (nk + Cfg::KCH - 1) / Cfg::KCH;
         for (int c = 0; c < nch && ok; ++c) {

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -92,6 +93,11 @@ struct Profiler {
   mao_launch_info* info = nullptr;
   int capacity = 0;
   int count = 0;
+  // device counters of executed work, two per recorded launch (table-mode products
+  // only: `counted` marks the slots whose launch writes them)
+  unsigned long long* work = nullptr;
+  int work_cap = 0;
+  std::vector<char> counted;
 };
 Profiler& profiler();
 
@@ -164,6 +170,7 @@ struct TableLaunch {
   int pa = 3, pb = 3;
   int force_kernel = 0;  // 0: choose, 1: one-CTA kernel, 2: CTA-pair kernel (verification)
   int kernel_id = 0;
+  const int* any = nullptr;  // launch-level gate (GemmTableParams::any), or nullptr
   std::vector<GemmProblem> probs;
   std::vector<int> map_idx;  // 6 per problem: A planes 0..2, B planes 0..2 (indices into the step's map list)
 };
@@ -225,6 +232,7 @@ struct StagedLaunch {
   int total_tiles2 = 0;  // 256-row tiles (CTA-pair kernel)
   bool pair = false;     // launch the CTA-pair kernel
   double flops = 0.0;
+  const int* any = nullptr;
 };
 StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off);
 mao_status table_launch(const Arena& A, const StagedLaunch& S, DevStatus* status, cudaStream_t stream);

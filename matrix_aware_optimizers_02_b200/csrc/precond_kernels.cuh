@@ -156,27 +156,39 @@ __global__ void __launch_bounds__(256) pc_keys_kernel(const SortJob* __restrict_
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int i = (blockIdx.x - j.key_blk_begin) * 32 + lane;
   const bool dots = sort || j.dg;
-  double s0 = 0.0, s1 = 0.0;
-  float n0 = 0.f, n1 = 0.f;
+  // four rows per iteration (independent accumulators keep eight loads in flight)
+  double s[4] = {0.0, 0.0, 0.0, 0.0};
+  float nrm[4] = {0.f, 0.f, 0.f, 0.f};
   if (i < j.k) {
+    const float* P = j.P + i;
+    const float* Q = j.Q + i;
     int r = warp;
-    for (; r + 8 < j.k; r += 16) {
-      const float p0 = j.P[(long long)r * j.k + i], p1 = j.P[(long long)(r + 8) * j.k + i];
-      n0 += p0 * p0;
-      n1 += p1 * p1;
+    for (; r + 24 < j.k; r += 32) {
+      float p[4], q[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) p[u] = P[(long long)(r + 8 * u) * j.k];
       if (dots) {
-        s0 += (double)j.Q[(long long)r * j.k + i] * (double)p0;
-        s1 += (double)j.Q[(long long)(r + 8) * j.k + i] * (double)p1;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) q[u] = Q[(long long)(r + 8 * u) * j.k];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        nrm[u] += p[u] * p[u];
+        if (dots) s[u] += (double)q[u] * (double)p[u];
       }
     }
-    if (r < j.k) {
-      const float p0 = j.P[(long long)r * j.k + i];
-      n0 += p0 * p0;
-      if (dots) s0 += (double)j.Q[(long long)r * j.k + i] * (double)p0;
+#pragma unroll
+    for (int u = 0; u < 3; ++u) {  // at most three rows remain
+      const int rr = r + 8 * u;
+      if (rr < j.k) {
+        const float p0 = P[(long long)rr * j.k];
+        nrm[u] += p0 * p0;
+        if (dots) s[u] += (double)Q[(long long)rr * j.k] * (double)p0;
+      }
     }
   }
-  part[warp][lane] = s0 + s1;
-  partn[warp][lane] = n0 + n1;
+  part[warp][lane] = (s[0] + s[1]) + (s[2] + s[3]);
+  partn[warp][lane] = (nrm[0] + nrm[1]) + (nrm[2] + nrm[3]);
   __syncthreads();
   if (warp == 0 && i < j.k) {
     double s = 0.0;
@@ -342,9 +354,18 @@ struct PanelJob {
   int* fin;              // first pass: set to 1 when the panel needs a final Cholesky-QR pass
                          // (a second pass or a second projection ran), else 0
   const int* flag;
+  // first pass: launch-level gates set to 1 when this panel takes the second pass,
+  // the second projection or the final pass (nullptr: not tracked)
+  int* any_again;
+  int* any_reorth;
+  int* any_fin;
   int w, nparts;
   int first;
 };
+
+// Indices of a group's launch-level gates (ints): any second Cholesky-QR pass, any
+// second projection, any final pass.
+constexpr int kAnyAgain = 0, kAnyReorth = 1, kAnyFin = 2;
 
 // Selective reorthogonalisation (the classical criterion of Daniel, Gragg, Kaufman
 // and Stewart, per column): a second projection pass is needed when the first pass
@@ -355,9 +376,11 @@ constexpr double kReorthRatio = 0.5;
 __device__ __forceinline__ int pk(int r, int c) { return ((r * (2 * kPanel + 1 - r)) >> 1) + (c - r); }
 
 // kRedBlocks blocks per panel, block rb owns Gram rows [rb*kRedRows, +kRedRows).
-__global__ void __launch_bounds__(256) qr_gram_reduce_kernel(const PanelJob* __restrict__ J) {
+__global__ void __launch_bounds__(256) qr_gram_reduce_kernel(const PanelJob* __restrict__ J,
+                                                              const int* __restrict__ any) {
   __shared__ double dsh[kPanel];
   __shared__ double red[8];
+  if (any && *any == 0) return;  // no panel of the launch takes this pass
   const PanelJob& j = J[blockIdx.x / kRedBlocks];
   const int rb = blockIdx.x % kRedBlocks;
   if (j.flag && *j.flag == 0) return;
@@ -380,7 +403,10 @@ __global__ void __launch_bounds__(256) qr_gram_reduce_kernel(const PanelJob* __r
     if (rb == 0) j.gs[kPackedUpper + tid] = s;
   }
   cancel = __syncthreads_or(cancel);
-  if (j.pnorm2 && rb == 0 && tid == 0) *j.reorth = cancel ? 1 : 0;
+  if (j.pnorm2 && rb == 0 && tid == 0) {
+    *j.reorth = cancel ? 1 : 0;
+    if (cancel && j.any_reorth) *j.any_reorth = 1;
+  }
   // one 4-column group of one row per thread
   const int a = rb * kRedRows + (tid >> 5), b0 = (tid & 31) * 4;
   double g[4] = {0.0, 0.0, 0.0, 0.0};
@@ -431,7 +457,7 @@ __global__ void __launch_bounds__(256) qr_gram_reduce_kernel(const PanelJob* __r
 // broadcast, and inner products keep several independent accumulators.
 constexpr int kLdA = kPanel + 1;
 
-__global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restrict__ J) {
+__global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restrict__ J, const int* __restrict__ any) {
   extern __shared__ double chol_smem[];
   double* A = chol_smem;                  // [kPanel][kLdA]: Gs, then Rs, then Rs^{-1}
   double* T = A + kPanel * kLdA;          // [kPanel - 32][32] block-column workspace of the inverse
@@ -439,6 +465,7 @@ __global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restr
   double* rdi = ds + kPanel;              // 1 / Rs[k][k]
   __shared__ int nbad_sh;
   __shared__ double red_sh[8];
+  if (any && *any == 0) return;  // no panel of the launch takes this pass
   const PanelJob& j = J[blockIdx.x];
   if (j.flag && *j.flag == 0) return;
   const int w = j.w;
@@ -452,7 +479,9 @@ __global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restr
   if (tot <= kFastTol * kFastTol) {  // the first-order inverse is already in place
     if (j.first && tid == 0) {
       *j.again = 0;
-      *j.fin = j.reorth ? *j.reorth : 0;
+      const int fin = j.reorth ? *j.reorth : 0;
+      *j.fin = fin;
+      if (fin && j.any_fin) *j.any_fin = 1;
     }
     return;
   }
@@ -501,6 +530,7 @@ __global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restr
         if (lane == 0 && nbad) nbad_sh += nbad;
       }
       __syncthreads();
+      if (attempt == 0 && nbad_sh) break;  // broke down: start over, shifted
       const int nt = wp - o - 32;  // trailing columns
       if (nt == 0) break;
       // block row: Rs_bc = Rs_bb^{-T} G_bc, one column per thread (right-looking in registers)
@@ -637,8 +667,11 @@ __global__ void __launch_bounds__(256, 1) qr_chol_kernel(const PanelJob* __restr
 #pragma unroll
       for (int i = 0; i < 8; ++i) tot2 += red_sh[i];
       const int again = (shifted || tot2 > kAgainMeanInv * w) ? 1 : 0;
+      const int fin = again | (j.reorth ? *j.reorth : 0);
       *j.again = again;
-      *j.fin = again | (j.reorth ? *j.reorth : 0);
+      *j.fin = fin;
+      if (again && j.any_again) *j.any_again = 1;
+      if (fin && j.any_fin) *j.any_fin = 1;
     }
   }
 }
@@ -655,7 +688,9 @@ struct CoefJob {
   int blk_begin;
 };
 
-__global__ void __launch_bounds__(256) pc_coef_reduce_kernel(const CoefJob* __restrict__ J, int n) {
+__global__ void __launch_bounds__(256) pc_coef_reduce_kernel(const CoefJob* __restrict__ J, int n,
+                                                              const int* __restrict__ any) {
+  if (any && *any == 0) return;  // no factor of the launch takes this projection
   const int lo = find_start(job_starts(J, n), n, (int)blockIdx.x);
   const CoefJob& j = J[lo];
   if (j.flag && *j.flag == 0) return;

@@ -157,6 +157,10 @@ struct GroupPlan {
   int g0 = 0, g1 = 0;   // matrices [g0, g1)
   size_t scratch = 0;   // bytes of per-matrix scratch
   size_t flags = 0, flags_bytes = 0;  // all 64-byte flag blocks of the group, contiguous
+  // launch-level gates of the QR's device-decided passes (ints: any second pass, any
+  // second projection, any final pass among the group's factors), cleared before each
+  // sub-panel's first pass
+  size_t any = 0;
   std::vector<MatBuf> mb;
 };
 
@@ -167,6 +171,7 @@ void plan_group_scratch(const Ctx& X, GroupPlan& G, size_t base) {
   const bool check = X.mode == 2;
   G.flags_bytes = (size_t)64 * 2 * (G.g1 - G.g0);
   G.flags = cv.take(G.flags_bytes);
+  G.any = cv.take(16);
   bool g_one = true;  // every gradient of the group bf16: G is read directly (SOAP needs no plane copy)
   for (int i = G.g0; i < G.g1; ++i) g_one = g_one && X.mats[i].g_bf16;
   for (int i = G.g0; i < G.g1; ++i) {
@@ -229,11 +234,15 @@ void make_groups(const Ctx& X, std::vector<GroupPlan>& groups) {
 // Records every launch of one group into `ops`, with all device data staged in
 // the arena; in sizing mode (ws == nullptr) only the sizes matter.
 struct Op {
-  enum Kind { GEMM, EW, SPLIT, ADAM, KEYS, ARGSORT, GATHER, VPERM, REDUCE, CHOL, COEFRED, RC, TAU, FOAMN, CHECK } kind;
+  enum Kind { GEMM, EW, SPLIT, ADAM, KEYS, ARGSORT, GATHER, VPERM, REDUCE, CHOL, COEFRED, RC, TAU, FOAMN, CHECK, ZERO }
+      kind;
   size_t jobs = 0;
   int njobs = 0;
   int blocks = 0;
   double bytes = 0.0;
+  const int* any = nullptr;  // launch-level gate (REDUCE, CHOL, COEFRED), or nullptr
+  void* zero = nullptr;      // ZERO: device bytes cleared
+  size_t zero_bytes = 0;
 };
 
 struct Builder {
@@ -358,6 +367,7 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
   auto Qp = [&](int u) { return units[u].left ? mat(u).QL : mat(u).QR; };
   auto permo = [&](int u) { return units[u].left ? mat(u).perm_L : mat(u).perm_R; };
   auto flagp = [&](int u) -> const int* { return check ? B.wp<int>(side(u).flag) : nullptr; };
+  auto anyp = [&](int which) -> int* { return B.wp<int>(G.any) + which; };
 
   // three-plane split of Q (F's planes come from the factor products)
   {
@@ -511,8 +521,20 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
         auto gate = [&](int u) -> const int* {
           return pass == 1 ? B.wp<int>(side(u).again) : pass == 2 ? B.wp<int>(side(u).fin) : flagp(u);
         };
+        // the launch-level gate of a gated pass: set by the first pass when any factor
+        // takes it, so that a pass no factor takes costs no more than its launches
+        const int* lgate = pass == 1 ? anyp(kAnyAgain) : pass == 2 ? anyp(kAnyFin) : nullptr;
+        if (pass == 0) {
+          Op z;
+          z.kind = Op::ZERO;
+          z.zero = B.wp<int>(G.any);
+          z.zero_bytes = 16;
+          B.ops.push_back(z);
+          B.gemm_of_op.push_back(-1);
+        }
         // Gram partials over K slices (fp32-faithful), one 128 x 128 tile each
         TableLaunch& gg = B.new_gemm(1, 1, MAO_K_PC_PANEL);
+        gg.any = lgate;
         const int nact = (int)act.size();
         for (int i : act) {
           const int k = kof(i), w = wdt(i);
@@ -538,19 +560,26 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
           j.w = wdt(i);
           j.nparts = (k + gram_slice(k, nact) - 1) / gram_slice(k, nact);
           j.first = pass == 0 ? 1 : 0;
-          if (pass == 0) j.fin = B.wp<int>(side(i).fin);
+          if (pass == 0) {
+            j.fin = B.wp<int>(side(i).fin);
+            j.any_again = anyp(kAnyAgain);
+            j.any_fin = anyp(kAnyFin);
+          }
           if (pass == 0 && cs > 0) {
             j.pnorm2 = B.wp<float>(side(i).pnorm2) + cs;
             j.reorth = B.wp<int>(side(i).reorth);
+            j.any_reorth = anyp(kAnyReorth);
           }
         }
         B.ops.back().blocks = (int)act.size() * kRedBlocks;
+        B.ops.back().any = lgate;
         Op ch = B.ops.back();  // the factorisation reuses the job array
         ch.kind = Op::CHOL;
         ch.blocks = (int)act.size();
         B.ops.push_back(ch);
         B.gemm_of_op.push_back(-1);
         TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_QR_APPLY);
+        g.any = lgate;
         for (int i : act) {
           const int k = kof(i), w = wdt(i);
           __nv_bfloat16* r = B.wp<__nv_bfloat16>(side(i).rinv);
@@ -601,7 +630,9 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
         int tiles = 0;
         for (size_t u = 0; u < units.size(); ++u) tiles += ((rows + 127) / 128) * ((width + 127) / 128);
         const int want = std::min(kMaxCoefParts, std::max(1, (2 * 148 + tiles - 1) / std::max(tiles, 1)));
+        const int* lgate = reorth ? anyp(kAnyReorth) : nullptr;
         TableLaunch& gc = B.new_gemm(1, 1, MAO_K_PC_QR);
+        gc.any = lgate;
         std::vector<CoefJob> red;
         int rblk = 0;
         for (int i : units) {
@@ -643,8 +674,10 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
           CoefJob* J = B.new_jobs<CoefJob>(Op::COEFRED, (int)red.size(), off);
           for (size_t a = 0; a < red.size(); ++a) J[a] = red[a];
           B.ops.back().blocks = rblk;
+          B.ops.back().any = lgate;
         }
         TableLaunch& gw = B.new_gemm(0, 1, MAO_K_PC_QR);
+        gw.any = lgate;
         for (int i : units) {
           const int k = kof(i), w = wof(i);
           Split3 C = B.planes(side(i).Cp, k, kSuper);
@@ -1126,6 +1159,10 @@ mao_status run_ops(const Ctx& X, uint8_t* arena_dev, const BuiltGroup& bg, DevSt
       MAO_TRY(table_launch(A, bg.staged[bg.gemm_of_op[o]], status, s));
       continue;
     }
+    if (op.kind == Op::ZERO) {
+      MAO_CUDA_TRY(cudaMemsetAsync(op.zero, 0, op.zero_bytes, s));
+      continue;
+    }
     if (op.blocks <= 0) continue;
     const int n = op.njobs;
     switch (op.kind) {
@@ -1166,18 +1203,18 @@ mao_status run_ops(const Ctx& X, uint8_t* arena_dev, const BuiltGroup& bg, DevSt
       }
       case Op::REDUCE: {
         LaunchScope ls(s, MAO_K_PC_PANEL, 0.0, 0.0);
-        qr_gram_reduce_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<PanelJob>(op.jobs));
+        qr_gram_reduce_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<PanelJob>(op.jobs), op.any);
         break;
       }
       case Op::COEFRED: {
         LaunchScope ls(s, MAO_K_PC_QR_REDUCE, 0.0, 0.0);
-        pc_coef_reduce_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<CoefJob>(op.jobs), n);
+        pc_coef_reduce_kernel<<<op.blocks, 256, 0, s>>>(A.dptr<CoefJob>(op.jobs), n, op.any);
         break;
       }
       case Op::CHOL: {
         MAO_TRY(chol_attr());
         LaunchScope ls(s, MAO_K_PC_CHOL, 0.0, 0.0);
-        qr_chol_kernel<<<op.blocks, 256, kCholSmem, s>>>(A.dptr<PanelJob>(op.jobs));
+        qr_chol_kernel<<<op.blocks, 256, kCholSmem, s>>>(A.dptr<PanelJob>(op.jobs), op.any);
         break;
       }
       case Op::RC: {

@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.mao_version() == 3
+    assert lib.mao_version() == 4
     for s in range(0, 11):
         assert len(lib.mao_status_string(s)) > 0
     assert lib.mao_status_string(999) == b"unknown status"
