@@ -297,10 +297,14 @@ StagedLaunch table_stage(Arena& A, const TableLaunch& L, size_t maps_off) {
       P.mapA[q] = (mbase && ia >= 0) ? mbase + ia : nullptr;
       P.mapB[q] = (mbase && ib >= 0) ? mbase + ib : nullptr;
     }
+    // column tiles: the one-CTA kernel's are 256 wide for one-plane operands (GemmCfg)
+    const int bn1 = (L.pa == 1 && L.pb == 1) ? 256 : 128;
+    P.tiles_n = (P.N + bn1 - 1) / bn1;
+    P.tiles_n2 = (P.N + 127) / 128;
     P.tile_begin = t;
     t += ((P.M + 127) / 128) * P.tiles_n;
     P.tile_begin2 = t2;
-    t2 += ((P.M + 255) / 256) * P.tiles_n;
+    t2 += ((P.M + 255) / 256) * P.tiles_n2;
     // work recorded for the profiler: only problems that always run (a problem gated
     // by a device flag may be skipped, so it counts nothing: a lower bound)
     if (P.flag == nullptr) S.flops += 2.0 * P.M * (double)P.N * P.K;

@@ -101,7 +101,8 @@ struct GemmProblem {
   int m_off, n_off;            // operand coordinates of output row/column 0 (sub-block views)
   int k_off;                   // operand coordinate of K index 0 (a K slice; multiple of 8 for K-major operands)
   int ld_out, ld_aux, ld_outp;
-  int tiles_n, tile_begin;
+  int tiles_n, tile_begin;      // tiles_n: column tiles of the one-CTA kernel (128 or 256 wide)
+  int tiles_n2;                 // column tiles of the CTA-pair kernel (128 wide)
   float alpha, beta;
   // Alternate destination chosen on the device: when sel != nullptr and *sel == 0
   // the result goes to out2 / out2_p (leading dimensions ld_out2 / ld_out2p) instead.
@@ -136,7 +137,9 @@ struct GemmTableParams {
 template <int KIND, int A_MN, int B_MN, int PA = (KIND == OP_BF16 ? 1 : 3), int PB = PA>
 struct GemmCfg {
   static constexpr int BM = 128;
-  static constexpr int BN = (KIND == OP_BF16) ? 256 : 128;
+  // 128 x 256 tiles for one-plane operands (bf16 x bf16: one product per k-step, so the
+  // operand stream per multiply-add is the limit and wider tiles halve it per output)
+  static constexpr int BN = (KIND == OP_BF16 || (PA == 1 && PB == 1)) ? 256 : 128;
   static constexpr int ESIZE = 2;                      // bf16 planes
   static constexpr int BK = 64;                        // elements per 128-byte row
   static constexpr int UMMA_K = 16;                    // 32 bytes of K per MMA
@@ -220,6 +223,19 @@ __device__ __forceinline__ void store_f32x32(float* dst, const float* v) {
 #pragma unroll
     for (int j = 0; j < 32; j += 4)
       *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+  }
+}
+
+// 32 consecutive bf16 packed in pairs (16-byte aligned; whole sectors when 32-byte
+// aligned)
+__device__ __forceinline__ void store_bf16x32_packed(__nv_bfloat16* dst, const uint32_t* w) {
+  if (aligned32(dst)) {
+    st_global_v8(dst, w);
+    st_global_v8(dst + 16, w + 8);
+  } else {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) d[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
   }
 }
 
@@ -408,6 +424,7 @@ struct TableSource {
     const int lo = find_start(starts, p.nprob, tile);
     const GemmProblem& P = p.probs[lo];
     const int r = tile - (pair ? P.tile_begin2 : P.tile_begin);
+    const int tn = pair ? P.tiles_n2 : P.tiles_n;
     TileInfo t;
 #pragma unroll
     for (int q = 0; q < 3; ++q) {
@@ -416,8 +433,8 @@ struct TableSource {
     }
     t.idx = lo;
     t.b = 0;
-    t.m0 = (r / P.tiles_n) * BM;
-    t.n0 = (r % P.tiles_n) * BN;
+    t.m0 = (r / tn) * BM;
+    t.n0 = (r % tn) * BN;
     t.K = P.K;
     t.valid = (P.flag == nullptr) || (*P.flag != 0);
     t.am = P.m_off;
@@ -510,25 +527,28 @@ struct TableSource {
       }
     }
     if (e.outp[0] != nullptr) {
+      // the three planes are peeled off v in place (v's last use): plane q is the
+      // bf16 rounding of what the planes before it left
       const long long offp = (long long)row * e.ld_outp + col0;
-      float r[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) r[j] = v[j];
 #pragma unroll
       for (int q = 0; q < 3; ++q) {
-        float pq[32];
+        uint32_t w[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          pq[j] = __bfloat162float(__float2bfloat16_rn(r[j]));
-          r[j] -= pq[j];
+        for (int j = 0; j < 16; ++j) {
+          const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+          w[j] = *reinterpret_cast<const uint32_t*>(&h);
+          const float2 f = __bfloat1622float2(h);
+          v[2 * j] -= f.x;
+          v[2 * j + 1] -= f.y;
         }
         __nv_bfloat16* o = e.outp[q] + offp;
         if (full) {
-          store_bf16x32(o, pq);
+          store_bf16x32_packed(o, w);
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (col0 + j < e.N) o[j] = __float2bfloat16_rn(pq[j]);
+            if (col0 + j < e.N)
+              o[j] = __ushort_as_bfloat16((unsigned short)((j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xffffu)));
         }
       }
     }
@@ -787,13 +807,16 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
         }
         if (!ok) break;
         if constexpr (EPI == EPI_TABLE) {
-          static_assert(COLS == 64, "update statistics assume 64 columns per epilogue warp");
-          float2 st = make_float2(0.f, 0.f);
+          static_assert(COLS % 64 == 0, "update statistics are kept per 32 x 64 block");
           const auto e = src.epi(t);
 #pragma unroll
-          for (int ch = 0; ch < COLS / 32; ++ch)
-            if (t.n0 + cb + ch * 32 < ncols) src.epilogue_table(e, row, t.n0 + cb + ch * 32, &run[ch * 32], st);
-          src.flush_stats(e, t.m0 + q * 32, t.n0 + cb, st, lane);
+          for (int h = 0; h < COLS / 64; ++h) {
+            float2 st = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int ch = 2 * h; ch < 2 * h + 2; ++ch)
+              if (t.n0 + cb + ch * 32 < ncols) src.epilogue_table(e, row, t.n0 + cb + ch * 32, &run[ch * 32], st);
+            src.flush_stats(e, t.m0 + q * 32, t.n0 + cb + 64 * h, st, lane);
+          }
         } else {
 #pragma unroll
           for (int ch = 0; ch < COLS / 32; ++ch)
