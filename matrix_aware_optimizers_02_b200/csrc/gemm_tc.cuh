@@ -295,6 +295,7 @@ struct ClassSource {
   const GemmParams& p;
   __device__ explicit ClassSource(const GemmParams& p_) : p(p_) {}
   __device__ bool skip_all() const { return false; }
+  __device__ void prefetch_aux(const TileInfo&, int, int, int) const {}
   template <int PRODUCTS>
   __device__ void count_work(const TileInfo&, int, int) const {}
   __device__ int total_tiles() const { return p.total_tiles; }
@@ -402,6 +403,15 @@ struct TableSource {
   const GemmTableParams& p;
   __device__ explicit TableSource(const GemmTableParams& p_) : p(p_) {}
   __device__ bool skip_all() const { return p.any != nullptr && *p.any == 0; }
+  // L2 prefetch of the aux row segment [col0, col0 + cols) the epilogue thread of `row`
+  // will read, issued before the tile's K loop so that the reads after it hit L2.
+  __device__ __forceinline__ void prefetch_aux(const TileInfo& t, int row, int col0, int cols) const {
+    const GemmProblem& P = p.probs[t.idx];
+    if (P.aux == nullptr || row >= P.M) return;
+    const float* a = P.aux + (long long)row * P.ld_aux;
+    for (int c = col0; c < col0 + cols && c < P.N; c += 32)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(a + c));
+  }
   // Profiling: the work of one computed tile (called once per tile by the MMA issuer).
   template <int PRODUCTS>
   __device__ void count_work(const TileInfo& t, int BM, int BN) const {
@@ -769,6 +779,7 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
         tc_fence_before();
         mbar_arrive_relaxed(&tempty_bar[acc]);
       } else {
+        if constexpr (EPI == EPI_TABLE) src.prefetch_aux(t, row, t.n0 + cb, COLS);
         // fold the K-chunk accumulators (main + correction) into fp32 registers
         const int nk = (t.K + BK - 1) / BK;
         const int nch = (nk + Cfg::KCH - 1) / Cfg::KCH;
@@ -1057,6 +1068,7 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
       if (!t.valid) continue;
       const int row = t.m0 + 128 * (int)rank + row_in_tile;
       const int ncols = src.cols(t);
+      src.prefetch_aux(t, row, t.n0 + cb, COLS);
       const int nk = (t.K + BK - 1) / BK;
       const int nch = (nk + Cfg::KCH - 1) / Cfg::KCH;
       float run[COLS];

@@ -8,10 +8,12 @@
 //                 (fp32-faithful SPLIT3 tensor-core GEMMs with the EMA in the epilogue)
 //   refresh       per side, when the policy says so: [adaptive check D = Q^T F Q,
 //                 rho, flag] -> P = F Q -> keys diag(Q^T F Q) in fp64 -> stable
-//                 descending argsort -> gathered P -> QR (block Gram-Schmidt with
-//                 re-orthogonalisation; panels of 64 columns orthonormalised by
-//                 two fp64 Cholesky-QR passes) -> Q.  Every refresh kernel reads a
-//                 per-matrix device flag, so adaptive refreshes need no host sync.
+//                 descending argsort -> gathered P -> QR (block Gram-Schmidt by
+//                 256-column super-panels, 128-column panels orthonormalised by
+//                 Cholesky-QR with an fp64 factorisation; second passes and
+//                 re-orthogonalisation decided on the device) -> Q.  Every refresh
+//                 kernel reads a per-matrix device flag, so adaptive refreshes need
+//                 no host sync.
 //   SOAP          Gh, Mh = Q_L^T {G, M} Q_R ; Adam in the eigenbasis (V follows the
 //                 permutations) ; U = Q_L N Q_R^T fused with W <- W(1 - lr wd) - lr U
 //   FOAM          Gr, Mr = {G, M} Q_R ; r, c EMAs of row/column means of Gr^2 ; tau ;
