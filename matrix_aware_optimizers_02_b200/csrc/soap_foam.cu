@@ -907,32 +907,60 @@ mao_status build_group(Builder& B, GroupPlan& G) {
       }
       B.ops.back().blocks = blk;
     }
-    // T1 = Q_L^T {G, M}  (A = Q_L stored K x M, B = G / M stored K x N)
-    {
+    // Gh = Q_L^T G Q_R and Mh = Q_L^T M Q_R.  A bf16 G makes its first product a
+    // three-product one (one exact plane) and the second a six-product one (both
+    // operands three-plane), so G's pair is ordered to put the cheap product on the
+    // larger side: Q_L^T G first for m >= n, G Q_R first for m < n.  M's two products
+    // cost the same in either order: Q_L^T M first.
+    auto tall = [&](int i) { return gpl == 3 || A(i).m >= A(i).n; };
+    bool any_tall = false, any_wide = false;
+    for (int i = 0; i < nm; ++i) (tall(i) ? any_tall : any_wide) = true;
+    // T1G = Q_L^T G (tall G)   (A = Q_L stored K x M, B = G stored K x N)
+    if (any_tall) {
       TableLaunch& g = B.new_gemm(1, 1, MAO_K_PC_ROTATE);
       g.pb = gpl;
       for (int i = 0; i < nm; ++i) {
+        if (!tall(i)) continue;
         const PcMat& a = A(i);
         const Split3 T1G = B.planes(G.mb[i].T1G, a.m, a.n);
         MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].L.Qp, a.m, a.m), Gop(i), a.m, a.n, a.m, 0, 0, nullptr, &T1G,
                           a.n, nullptr, 0, 1.f, 0.f, nullptr));
       }
+    }
+    // T1G = G Q_R (wide G)   (A = G K-major, B = Q_R stored K x N)
+    if (any_wide) {
+      TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_ROTATE);
+      g.pa = gpl;
+      for (int i = 0; i < nm; ++i) {
+        if (tall(i)) continue;
+        const PcMat& a = A(i);
+        const Split3 T1G = B.planes(G.mb[i].T1G, a.m, a.n);
+        MAO_TRY(table_add(g, B.maps, Gop(i), B.planes(G.mb[i].R.Qp, a.n, a.n), a.m, a.n, a.n, 0, 0, nullptr, &T1G,
+                          a.n, nullptr, 0, 1.f, 0.f, nullptr));
+      }
+    }
+    // T1M = Q_L^T M, and Gh = Q_L^T T1G for the wide G
+    {
       TableLaunch& g2 = B.new_gemm(1, 1, MAO_K_PC_ROTATE);
       for (int i = 0; i < nm; ++i) {
         const PcMat& a = A(i);
         const Split3 T1M = B.planes(G.mb[i].T1M, a.m, a.n);
         MAO_TRY(table_add(g2, B.maps, B.planes(G.mb[i].L.Qp, a.m, a.m), B.planes(G.mb[i].Mp, a.m, a.n), a.m, a.n,
                           a.m, 0, 0, nullptr, &T1M, a.n, nullptr, 0, 1.f, 0.f, nullptr));
+        if (!tall(i))
+          MAO_TRY(table_add(g2, B.maps, B.planes(G.mb[i].L.Qp, a.m, a.m), B.planes(G.mb[i].T1G, a.m, a.n), a.m,
+                            a.n, a.m, 0, 0, B.wp<float>(G.mb[i].Gh), nullptr, a.n, nullptr, 0, 1.f, 0.f, nullptr));
       }
     }
-    // Gh, Mh = T1 Q_R (fp32)
+    // Gh = T1G Q_R (tall G), Mh = T1M Q_R (fp32)
     {
       TableLaunch& g = B.new_gemm(0, 1, MAO_K_PC_ROTATE);
       for (int i = 0; i < nm; ++i) {
         const PcMat& a = A(i);
         const Split3 Qr = B.planes(G.mb[i].R.Qp, a.n, a.n);
-        MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].T1G, a.m, a.n), Qr, a.m, a.n, a.n, 0, 0,
-                          B.wp<float>(G.mb[i].Gh), nullptr, a.n, nullptr, 0, 1.f, 0.f, nullptr));
+        if (tall(i))
+          MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].T1G, a.m, a.n), Qr, a.m, a.n, a.n, 0, 0,
+                            B.wp<float>(G.mb[i].Gh), nullptr, a.n, nullptr, 0, 1.f, 0.f, nullptr));
         MAO_TRY(table_add(g, B.maps, B.planes(G.mb[i].T1M, a.m, a.n), Qr, a.m, a.n, a.n, 0, 0,
                           B.wp<float>(G.mb[i].Mh), nullptr, a.n, nullptr, 0, 1.f, 0.f, nullptr));
       }
