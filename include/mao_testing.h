@@ -23,11 +23,12 @@ typedef enum {
   MAO_GEMM_SPLIT2 = 5
 } mao_gemm_kind;
 
-/* Flags OR-ed into a table-mode kind (all but MAO_GEMM_BF16): run the problems
- * on the one-CTA kernel (128 x 128 tiles) or on the CTA-pair kernel (256 x 128
- * tiles, tcgen05 cta_group::2); without a flag the library chooses as it does
- * inside the optimizer steps (the pair kernel for products with a three-plane
- * operand whose 256-row tiles fill the GPU). */
+/* Flags OR-ed into a kind: run the problems on the one-CTA kernel (128 x 128
+ * tiles; 128 x 256 for bf16 operands) or on the CTA-pair kernel (256 x 128 tiles
+ * for the fp32-faithful kinds, 256 x 256 for MAO_GEMM_BF16; tcgen05 cta_group::2);
+ * without a flag the library chooses as it does inside the optimizer steps (the
+ * pair kernel for products with a three-plane operand, and for the bf16
+ * Newton-Schulz products, whose 256-row tiles fill the GPU). */
 #define MAO_GEMM_FORCE_ONE_CTA 16
 #define MAO_GEMM_FORCE_CTA_PAIR 32
 
@@ -57,11 +58,11 @@ typedef enum {
  * the problem descriptors).
  */
 /*
- * Kernel choice for every table-mode product of this process (verification of
- * the optimizer steps on each kernel): 0 = the library's choice (default),
- * 1 = the one-CTA kernel always, 2 = the CTA-pair kernel always, whatever the
- * launch's size or plane counts.  Affects only calls made
- * after it returns; not thread-safe with concurrent steps.
+ * Kernel choice for every tensor-core product of this process (table-mode and
+ * the bf16 Newton-Schulz products; verification of the optimizer steps on each
+ * kernel): 0 = the library's choice (default), 1 = the one-CTA kernel always,
+ * 2 = the CTA-pair kernel always, whatever the launch's size or plane counts.
+ * Affects only calls made after it returns; not thread-safe with concurrent steps.
  */
 MAO_API mao_status mao_test_set_table_kernel(int32_t policy);
 

@@ -148,7 +148,7 @@ def gemm(A: torch.Tensor, B: torch.Tensor, *, kind: str = "bf16", a_mn_major: bo
       "split3_bf16" fp32 A (three planes) times bf16 B;
       "bf16_split3" bf16 A times fp32 B (three planes);
       "split2"      fp32 operands held as two bf16 planes each, three products.
-    kernel ("auto", "one_cta", "cta_pair") picks the table-mode kernel for every kind but "bf16".
+    kernel ("auto", "one_cta", "cta_pair") picks the one-CTA or the CTA-pair kernel.
     Returns fp32 (batch, M, N).
     """
     lib = L.load()

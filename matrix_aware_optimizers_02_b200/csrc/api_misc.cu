@@ -79,7 +79,6 @@ mao_status gemm_layout(int32_t kind_flags, int32_t batch, int32_t M, int32_t N, 
   const int32_t kind = kind_flags & 15;
   if ((kind_flags & ~(15 | MAO_GEMM_FORCE_ONE_CTA | MAO_GEMM_FORCE_CTA_PAIR)) != 0) return MAO_ERR_INVALID_ARG;
   if (kind < MAO_GEMM_BF16 || kind > MAO_GEMM_SPLIT2) return MAO_ERR_INVALID_ARG;
-  if (kind == MAO_GEMM_BF16 && (kind_flags & ~15)) return MAO_ERR_INVALID_ARG;
   Carver cv;
   cv.take(kStatusBytes);
   if (kind != MAO_GEMM_BF16) {
@@ -144,10 +143,11 @@ extern "C" mao_status mao_test_gemm(int32_t kind_flags, int32_t a_mn_major, int3
     p.alpha = 1.0f;
     p.status = status;
     MAO_TRY(encode_operand(&p.mapA[0], OP_BF16, a_mn_major, 128, view(A, a_rows, a_inner)));
-    MAO_TRY(encode_operand(&p.mapB[0], OP_BF16, b_mn_major, 256, view(B, b_rows, b_inner)));
+    MAO_TRY(encode_operand(&p.mapB[0], OP_BF16, b_mn_major, 128, view(B, b_rows, b_inner)));
     p.cls[0] = GemmClass{M, N, K, batch, 0, 0, 0, D, (long long)M * N, N, nullptr, 0, 0, nullptr, 0, 0, nullptr};
     finalize_classes(p);
-    return launch_gemm(OP_BF16, a_mn_major, b_mn_major, EPI_STORE_F32, p, stream, MAO_K_GEMM_TEST);
+    const int force = (kind_flags & MAO_GEMM_FORCE_CTA_PAIR) ? 2 : (kind_flags & MAO_GEMM_FORCE_ONE_CTA) ? 1 : 0;
+    return launch_gemm(OP_BF16, a_mn_major, b_mn_major, EPI_STORE_F32, p, stream, MAO_K_GEMM_TEST, force);
   }
 
   // table mode: the fp32 operands split into bf16 planes (a bf16 operand is its

@@ -73,16 +73,19 @@ mao_status encode_operand(CUtensorMap* map, int kind, int mn_major, int R, const
 }
 
 void finalize_classes(GemmParams& p) {
-  int t = 0;
+  int t = 0, t2 = 0;
   for (int c = 0; c < p.nclasses; ++c) {
     GemmClass& C = p.cls[c];
-    const int tm = (C.M + 127) / 128;
     C.tiles_n = (C.N + 255) / 256;
-    C.tiles_per_mat = tm * C.tiles_n;
+    C.tiles_per_mat = ((C.M + 127) / 128) * C.tiles_n;
+    C.tiles_per_mat2 = ((C.M + 255) / 256) * C.tiles_n;
     C.tile_begin = t;
+    C.tile_begin2 = t2;
     t += C.tiles_per_mat * C.count;
+    t2 += C.tiles_per_mat2 * C.count;
   }
-  p.total_tiles = t;
+  p.total_tiles = p.total_tiles1 = t;
+  p.total_tiles2 = t2;
 }
 
 namespace {
@@ -117,8 +120,52 @@ mao_status launch_one(const GemmParams& p, cudaStream_t stream, int kernel_id) {
   return cudaGetLastError() == cudaSuccess ? MAO_OK : MAO_ERR_CUDA;
 }
 
+// The same products on CTA pairs: 256 x 256 tiles (each CTA loads its 128 rows of A
+// and 128 of B's 256 columns), one cta_group::2 MMA per k-step.
+template <int A_MN, int B_MN, int EPI>
+mao_status launch_one_pair(const GemmParams& p, cudaStream_t stream, int kernel_id) {
+  using Cfg = GemmPairCfg<A_MN, B_MN, 1, 1, OP_BF16>;
+  DeviceInfo* d = nullptr;
+  MAO_TRY(device_info(&d));
+  auto kern = gemm_tc_pair_class_kernel<A_MN, B_MN, EPI>;
+  const int slot = (A_MN * 2 + B_MN) * 4 + EPI;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!d->gemm_pair_attr_set[slot]) {
+      MAO_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES));
+      d->gemm_pair_attr_set[slot] = true;
+    }
+  }
+  GemmParams q = p;
+  q.total_tiles = p.total_tiles2;
+  if (q.total_tiles <= 0) return MAO_OK;
+  const int max_pairs = d->sm_count / 2;
+  const int pairs = q.total_tiles < max_pairs ? q.total_tiles : max_pairs;
+  double flops = 0.0, bytes = 0.0;
+  const double ob = (EPI == EPI_STORE_F32) ? 4.0 : 2.0;
+  for (int c = 0; c < p.nclasses; ++c) {
+    const GemmClass& C = p.cls[c];
+    flops += 2.0 * C.count * (double)C.M * C.N * C.K;
+    bytes += C.count * (2.0 * ((double)C.M * C.K + (double)C.N * C.K) + ob * (double)C.M * C.N *
+                                                                              (EPI == EPI_AXPY_T ? 2 : 1) +
+                        ((EPI == EPI_POLY || EPI == EPI_AXPY_T) ? 2.0 * C.M * C.N : 0.0));
+  }
+  LaunchScope ls(stream, kernel_id, flops, bytes);
+  kern<<<2 * pairs, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(q);
+  return cudaGetLastError() == cudaSuccess ? MAO_OK : MAO_ERR_CUDA;
+}
+
 template <int KIND, int A_MN, int B_MN>
-mao_status launch_epi(int epi, const GemmParams& p, cudaStream_t s, int k) {
+mao_status launch_epi(int epi, const GemmParams& p, cudaStream_t s, int k, bool pair) {
+  if (pair) {
+    switch (epi) {
+      case EPI_STORE_F32: return launch_one_pair<A_MN, B_MN, EPI_STORE_F32>(p, s, k);
+      case EPI_GRAM: return launch_one_pair<A_MN, B_MN, EPI_GRAM>(p, s, k);
+      case EPI_POLY: return launch_one_pair<A_MN, B_MN, EPI_POLY>(p, s, k);
+      case EPI_AXPY_T: return launch_one_pair<A_MN, B_MN, EPI_AXPY_T>(p, s, k);
+      default: return MAO_ERR_INVALID_ARG;
+    }
+  }
   switch (epi) {
     case EPI_STORE_F32: return launch_one<KIND, A_MN, B_MN, EPI_STORE_F32>(p, s, k);
     case EPI_GRAM: return launch_one<KIND, A_MN, B_MN, EPI_GRAM>(p, s, k);
@@ -130,13 +177,19 @@ mao_status launch_epi(int epi, const GemmParams& p, cudaStream_t s, int k) {
 
 }  // namespace
 
-mao_status launch_gemm(int kind, int a_mn, int b_mn, int epi, const GemmParams& p, cudaStream_t stream, int k) {
+mao_status launch_gemm(int kind, int a_mn, int b_mn, int epi, const GemmParams& p, cudaStream_t stream, int k,
+                       int force) {
   if (kind != OP_BF16) return MAO_ERR_UNSUPPORTED;
-  if (!a_mn && !b_mn) return launch_epi<OP_BF16, 0, 0>(epi, p, stream, k);
-  if (!a_mn && b_mn) return launch_epi<OP_BF16, 0, 1>(epi, p, stream, k);
+  // CTA pairs when their 256-row tiles fill the GPU's pairs and waste at most a fifth
+  // of the rows (as for the table-mode products)
+  const int f = force ? force : table_kernel_policy();
+  const bool pair = f == 2 || (f == 0 && p.total_tiles2 >= 74 && 2.0 * p.total_tiles2 <= 1.2 * p.total_tiles1);
+  if (!a_mn && !b_mn) return launch_epi<OP_BF16, 0, 0>(epi, p, stream, k, pair);
+  if (!a_mn && b_mn) return launch_epi<OP_BF16, 0, 1>(epi, p, stream, k, pair);
   if (epi != EPI_STORE_F32) return MAO_ERR_UNSUPPORTED;
-  if (a_mn && !b_mn) return launch_one<OP_BF16, 1, 0, EPI_STORE_F32>(p, stream, k);
-  return launch_one<OP_BF16, 1, 1, EPI_STORE_F32>(p, stream, k);
+  if (a_mn && !b_mn)
+    return pair ? launch_one_pair<1, 0, EPI_STORE_F32>(p, stream, k) : launch_one<OP_BF16, 1, 0, EPI_STORE_F32>(p, stream, k);
+  return pair ? launch_one_pair<1, 1, EPI_STORE_F32>(p, stream, k) : launch_one<OP_BF16, 1, 1, EPI_STORE_F32>(p, stream, k);
 }
 
 // ------------------------------------------------------------------ three-plane split

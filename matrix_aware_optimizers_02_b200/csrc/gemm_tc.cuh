@@ -77,6 +77,7 @@ struct GemmClass {
   long long aux_bs;
   int aux_ld;
   const float* scale;  // per matrix of the class, or nullptr (= 1)
+  int tiles_per_mat2, tile_begin2;  // tiles_per_mat / tile_begin in the CTA-pair kernel's 256-row tiles
 };
 
 struct GemmParams {
@@ -84,7 +85,8 @@ struct GemmParams {
   CUtensorMap mapB[kMaxClasses];
   GemmClass cls[kMaxClasses];
   int nclasses;
-  int total_tiles;
+  int total_tiles;   // the tiles of the kernel launched (one-CTA or CTA-pair numbering)
+  int total_tiles1, total_tiles2;  // 128 x 256 one-CTA tiles, 256 x 256 pair tiles
   float alpha, beta, gamma;
   DevStatus* status;
 };
@@ -307,13 +309,15 @@ struct ClassSource {
     }
   }
   __device__ TileInfo decode(int tile, int BM, int BN) const {
+    const bool pair = BM == 256;
     int c = 0;
 #pragma unroll 1
-    while (c + 1 < p.nclasses && tile >= p.cls[c + 1].tile_begin) ++c;
+    while (c + 1 < p.nclasses && tile >= (pair ? p.cls[c + 1].tile_begin2 : p.cls[c + 1].tile_begin)) ++c;
     const GemmClass& C = p.cls[c];
-    const int local = tile - C.tile_begin;
-    const int b = local / C.tiles_per_mat;
-    const int r = local - b * C.tiles_per_mat;
+    const int local = tile - (pair ? C.tile_begin2 : C.tile_begin);
+    const int tpm = pair ? C.tiles_per_mat2 : C.tiles_per_mat;
+    const int b = local / tpm;
+    const int r = local - b * tpm;
     TileInfo t;
     t.mapA[0] = &p.mapA[c];
     t.mapB[0] = &p.mapB[c];
@@ -665,7 +669,7 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
             load_operand<A_MN, BM, Cfg::ESIZE>(st + q * Cfg::A_TILE, t.mapA[q], &full_bar[s], kc, am, t.b);
 #pragma unroll
           for (int q = 0; q < PB; ++q)
-            load_operand<B_MN, BN, Cfg::ESIZE, (EPI == EPI_TABLE ? 64 : BN)>(
+            load_operand<B_MN, BN, Cfg::ESIZE, (EPI == EPI_TABLE ? 64 : 128)>(
                 st + PA * Cfg::A_TILE + q * Cfg::B_TILE, t.mapB[q], &full_bar[s], kc, bn, t.b);
         }
         if (!ok) break;
@@ -862,11 +866,14 @@ __device__ __forceinline__ void gemm_body(const Src& src) {
 // epilogue folds and stores its own rows and releases the accumulator on the
 // first CTA's barrier.  Per 128 x 128 of output a CTA loads 3/4 of the bytes of
 // the one-CTA kernel, which leaves room for a third pipeline stage.
-template <int A_MN, int B_MN, int PA, int PB>
+template <int A_MN, int B_MN, int PA, int PB, int KIND = OP_SPLIT3>
 struct GemmPairCfg {
   static constexpr int BM = 128;   // rows per CTA (the pair's tile has 256)
-  static constexpr int BN = 128;   // columns of the pair's tile
-  static constexpr int BNH = 64;   // columns of B loaded by each CTA
+  // columns of the pair's tile: 128 for the fp32-faithful products (main and
+  // correction accumulators, double-buffered, fill the tensor memory), 256 for the
+  // bf16 Newton-Schulz products (one accumulator over the whole K)
+  static constexpr int BN = (KIND == OP_BF16) ? 256 : 128;
+  static constexpr int BNH = BN / 2;  // columns of B loaded by each CTA
   static constexpr int ESIZE = 2;
   static constexpr int BK = 64;
   static constexpr int UMMA_K = 16;
@@ -879,7 +886,8 @@ struct GemmPairCfg {
   static constexpr int PMAX = (PA > PB ? PA : PB) - 1;
   static constexpr bool CORR = (PA > 1 || PB > 1);
   static constexpr int ACC_COLS = CORR ? 2 * BN : BN;
-  static constexpr int KCH = CORR ? 2 : 4;  // as in the one-CTA kernel
+  // as in the one-CTA kernel; bf16 Newton-Schulz products accumulate the whole K
+  static constexpr int KCH = CORR ? 2 : (KIND == OP_BF16 ? (1 << 28) : 4);
   // the pair allocates all of TMEM, so both CTAs' accumulators start at the same
   // column (the pair MMA writes one address in both)
   static constexpr int TMEM_COLS = 512;
@@ -889,9 +897,12 @@ struct GemmPairCfg {
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
 };
 
-template <int A_MN, int B_MN, int PA, int PB>
-__device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
-  using Cfg = GemmPairCfg<A_MN, B_MN, PA, PB>;
+// KIND / EPI / Src: the fp32-faithful table products (OP_SPLIT3, EPI_TABLE,
+// TableSource) or the bf16 Newton-Schulz class products (OP_BF16, a class epilogue,
+// ClassSource; 256 x 256 pair tiles).
+template <int A_MN, int B_MN, int PA, int PB, int KIND = OP_SPLIT3, int EPI = EPI_TABLE, class Src = TableSource>
+__device__ __forceinline__ void gemm_body_pair(const Src& src) {
+  using Cfg = GemmPairCfg<A_MN, B_MN, PA, PB, KIND>;
   constexpr int BN = Cfg::BN, BK = Cfg::BK, STAGES = Cfg::STAGES;
 
   extern __shared__ uint8_t smem_raw[];
@@ -952,10 +963,12 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
       for (int tile = pair_id; tile < total; tile += npairs) {
         const TileInfo t = src.decode(tile, 256, BN);
         if (!t.valid) continue;
+        if constexpr (EPI == EPI_TABLE) {  // table descriptors live in global memory
 #pragma unroll
-        for (int q = 0; q < PA; ++q) tensormap_acquire(t.mapA[q]);
+          for (int q = 0; q < PA; ++q) tensormap_acquire(t.mapA[q]);
 #pragma unroll
-        for (int q = 0; q < PB; ++q) tensormap_acquire(t.mapB[q]);
+          for (int q = 0; q < PB; ++q) tensormap_acquire(t.mapB[q]);
+        }
         const int nk = (t.K + BK - 1) / BK;
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -974,19 +987,22 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
           for (int q = 0; q < PA; ++q) {
             uint8_t* dst = st + q * Cfg::A_TILE;
             if constexpr (!A_MN) {
-              tma_load_3d_pair(dst, t.mapA[q], fb, kc, am, 0);
+              tma_load_3d_pair(dst, t.mapA[q], fb, kc, am, t.b);
             } else {
 #pragma unroll
-              for (int c = 0; c < 128 / 64; ++c) tma_load_3d_pair(dst + c * BK * 128, t.mapA[q], fb, am + c * 64, kc, 0);
+              for (int c = 0; c < 128 / 64; ++c)
+                tma_load_3d_pair(dst + c * BK * 128, t.mapA[q], fb, am + c * 64, kc, t.b);
             }
           }
 #pragma unroll
           for (int q = 0; q < PB; ++q) {
             uint8_t* dst = st + PA * Cfg::A_TILE + q * Cfg::B_TILE;
             if constexpr (!B_MN) {
-              tma_load_3d_pair(dst, t.mapB[q], fb, kc, bn, 0);
+              tma_load_3d_pair(dst, t.mapB[q], fb, kc, bn, t.b);  // one box of BNH rows
             } else {
-              tma_load_3d_pair(dst, t.mapB[q], fb, bn, kc, 0);
+#pragma unroll
+              for (int c = 0; c < Cfg::BNH / 64; ++c)
+                tma_load_3d_pair(dst + c * BK * 128, t.mapB[q], fb, bn + c * 64, kc, t.b);
             }
           }
         }
@@ -1068,6 +1084,32 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
       if (!t.valid) continue;
       const int row = t.m0 + 128 * (int)rank + row_in_tile;
       const int ncols = src.cols(t);
+      if constexpr (EPI != EPI_TABLE) {
+        // bf16 class products: one accumulation item per tile, stored chunk by chunk
+        const int acc = used & 1;
+        const uint32_t aph = (used >> 1) & 1;
+        ++used;
+        const bool w = mbar_wait(&tfull_bar[acc], aph, status, 14, abort_flag);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS + cb;
+#pragma unroll 1
+        for (int ch = 0; ch < COLS / 32; ++ch) {
+          uint32_t rr[32];
+          tmem_ld_32x32b_x32(tacc + ch * 32, rr);
+          tmem_wait_ld();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(rr[j]);
+          if (t.n0 + cb + ch * 32 < ncols) src.template epilogue<EPI>(t, row, t.n0 + cb + ch * 32, v);
+        }
+        tc_fence_before();
+        mbar_arrive_cluster_relaxed(tempty_lead[acc]);
+        continue;
+      } else {
       src.prefetch_aux(t, row, t.n0 + cb, COLS);
       const int nk = (t.K + BK - 1) / BK;
       const int nch = (nk + Cfg::KCH - 1) / Cfg::KCH;
@@ -1105,13 +1147,17 @@ __device__ __forceinline__ void gemm_body_pair(const TableSource& src) {
         mbar_arrive_cluster_relaxed(tempty_lead[acc]);
       }
       if (!ok) break;
-      static_assert(COLS == 64, "update statistics assume 64 columns per epilogue warp");
-      float2 st = make_float2(0.f, 0.f);
-      const TableSource::Epi e = src.epi(t);
+      static_assert(COLS % 64 == 0, "update statistics are kept per 32 x 64 block");
+      const auto e = src.epi(t);
 #pragma unroll
-      for (int ch = 0; ch < COLS / 32; ++ch)
-        if (t.n0 + cb + ch * 32 < ncols) src.epilogue_table(e, row, t.n0 + cb + ch * 32, &run[ch * 32], st);
-      src.flush_stats(e, t.m0 + 128 * (int)rank + q * 32, t.n0 + cb, st, lane);
+      for (int h = 0; h < COLS / 64; ++h) {
+        float2 st = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int ch = 2 * h; ch < 2 * h + 2; ++ch)
+          if (t.n0 + cb + ch * 32 < ncols) src.epilogue_table(e, row, t.n0 + cb + ch * 32, &run[ch * 32], st);
+        src.flush_stats(e, t.m0 + 128 * (int)rank + q * 32, t.n0 + cb + 64 * h, st, lane);
+      }
+      }  // table products
     }
   }
 
@@ -1142,6 +1188,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     gemm_tc_pair_kernel(const __grid_constant__ GemmTableParams p) {
   TableSource src(p);
   gemm_body_pair<A_MN, B_MN, PA, PB>(src);
+}
+
+template <int A_MN, int B_MN, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
+    gemm_tc_pair_class_kernel(const __grid_constant__ GemmParams p) {
+  ClassSource src(p);
+  gemm_body_pair<A_MN, B_MN, 1, 1, OP_BF16, EPI, ClassSource>(src);
 }
 
 template <int KIND, int A_MN, int B_MN, int EPI>

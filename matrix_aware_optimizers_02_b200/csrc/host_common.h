@@ -51,6 +51,7 @@ struct DeviceInfo {
   int sm_count = 0;
   int major = 0, minor = 0;
   bool gemm_attr_set[64] = {};
+  bool gemm_pair_attr_set[64] = {};
 };
 
 mao_status device_info(DeviceInfo** out);
@@ -71,9 +72,11 @@ struct OperandView {
 mao_status encode_operand(CUtensorMap* map, int kind, int mn_major, int R, const OperandView& v);
 
 // Launch one class-mode (bf16) grouped GEMM of the given instantiation;
-// kernel_id tags the launch for the profiler.
+// kernel_id tags the launch for the profiler.  force: 0 = the library's choice
+// between the one-CTA kernel (128 x 256 tiles) and the CTA-pair kernel (256 x 256),
+// 1 = one CTA, 2 = CTA pairs.
 mao_status launch_gemm(int kind, int a_mn, int b_mn, int epi, const GemmParams& p, cudaStream_t stream,
-                       int kernel_id);
+                       int kernel_id, int force = 0);
 
 // Fill tile bookkeeping of the classes in p (M, N, K, count must be set).
 void finalize_classes(GemmParams& p);

@@ -415,12 +415,12 @@ extern "C" mao_status mao_muon_step(const mao_muon_mat* mats, int32_t count, con
         OperandView xv{ws + C.off_X[k], (uint64_t)C.l, (uint64_t)C.s, cnt, (uint64_t)C.ld_l,
                        (uint64_t)C.s * C.ld_l};
         MAO_TRY(encode_operand(&maps[c].XA[k], OP_BF16, 0, 128, xv));
-        MAO_TRY(encode_operand(&maps[c].XB[k], OP_BF16, 0, 256, xv));
+        MAO_TRY(encode_operand(&maps[c].XB[k], OP_BF16, 0, 128, xv));  // B boxes: 128 rows (a pair CTA's half)
         MAO_TRY(encode_operand(&maps[c].XMN[k], OP_BF16, 1, 256, xv));  // X as K x N (K = s rows)
       }
       OperandView av{ws + C.off_A, (uint64_t)C.s, (uint64_t)C.s, cnt, (uint64_t)C.ld_s, (uint64_t)C.s * C.ld_s};
       MAO_TRY(encode_operand(&maps[c].AA, OP_BF16, 0, 128, av));
-      MAO_TRY(encode_operand(&maps[c].AB, OP_BF16, 0, 256, av));
+      MAO_TRY(encode_operand(&maps[c].AB, OP_BF16, 0, 128, av));
       OperandView bv{ws + C.off_B, (uint64_t)C.s, (uint64_t)C.s, cnt, (uint64_t)C.ld_s, (uint64_t)C.s * C.ld_s};
       MAO_TRY(encode_operand(&maps[c].BA, OP_BF16, 0, 128, bv));
     }

@@ -158,8 +158,10 @@ def test_pair_kernel_flag_validation(lib):
     assert lib.mao_test_gemm_workspace_size(1 | 32, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_OK
     assert lib.mao_test_gemm_workspace_size(2 | 32, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_OK
     assert lib.mao_test_gemm_workspace_size(5 | 32, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_OK
-    assert lib.mao_test_gemm_workspace_size(0 | 16, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_ERR_INVALID_ARG
+    assert lib.mao_test_gemm_workspace_size(0 | 16, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_OK  # bf16 on one CTA
+    assert lib.mao_test_gemm_workspace_size(0 | 32, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_OK  # bf16 on CTA pairs
     assert lib.mao_test_gemm_workspace_size(1 | 64, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_ERR_INVALID_ARG
+    assert lib.mao_test_gemm_workspace_size(0 | 64, 1, 8, 8, 8, ctypes.byref(b)) == L.MAO_ERR_INVALID_ARG
 
 
 def _muon_size(lib, mat, params=None):

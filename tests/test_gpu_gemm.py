@@ -128,3 +128,25 @@ def test_table_kernels_agree(api, kind, adt, bdt, shape, a_mn, b_mn, kernel):
     other = api.gemm(Ain, Bin, kind=kind, a_mn_major=bool(a_mn), b_mn_major=bool(b_mn),
                      kernel="cta_pair" if kernel == "one_cta" else "one_cta")
     assert torch.equal(D, other)
+
+
+BF16_PAIR_SHAPES = [(1, 256, 256, 64), (3, 200, 328, 136), (2, 384, 520, 1000), (1, 8, 8, 8), (4, 640, 768, 512)]
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("shape", BF16_PAIR_SHAPES)
+def test_bf16_kernels_agree(api, shape, a_mn, b_mn):
+    """The bf16 Newton-Schulz products on one CTA (128 x 256 tiles) and on CTA pairs
+    (256 x 256 tiles, tcgen05 cta_group::2): both at the fp32 accumulation level of
+    exact bf16 products, and the same bits."""
+    batch, M, N, K = shape
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    A, B, Ain, Bin = _operands(batch, M, N, K, a_mn, b_mn, torch.bfloat16, gen)
+    ref = torch.bmm(A.double(), B.double().transpose(1, 2))
+    outs = []
+    for kernel in ("one_cta", "cta_pair"):
+        D = api.gemm(Ain, Bin, kind="bf16", a_mn_major=bool(a_mn), b_mn_major=bool(b_mn), kernel=kernel)
+        err = (D.double() - ref).abs().max().item()
+        assert err <= 1e-5 * K ** 0.5 * 4, (kernel, err)
+        outs.append(D)
+    assert torch.equal(outs[0], outs[1])
