@@ -315,56 +315,88 @@ __global__ void muon_scale_kernel(const MuonMatDev* __restrict__ T, int count, c
 // want_rows: write row partials (sum over the tile's columns of (O cs)^2)
 // use_rows / use_cols: apply rowscale / colscale before squaring.
 // OT: element type of O (bf16 after Newton-Schulz, fp32 for the exact polar factor).
+// The tile is read in storage order (X = O^T for a tall matrix), so no transpose is
+// needed: a storage row of a tall matrix is a column of O.  Thread (tx, ty) holds
+// storage rows ty + 16 i and storage columns 4 tx + e; "along" sums (over e and the
+// 16 threads of a half-warp) give per-storage-row partials, "across" sums (over i and
+// the 16 thread rows, in shared memory) per-storage-column partials.
 template <typename OT>
 __global__ void __launch_bounds__(256) muon_norm_tile_kernel(const MuonMatDev* __restrict__ T, int count,
                                                              int want_cols, int want_rows, int use_rows,
                                                              int use_cols) {
-  __shared__ __align__(16) typename OTile<OT>::Row sm[kTile];
   __shared__ float csum[16][kTile];
   const MuonMatDev& D = T[find_mat(T, count, blockIdx.x)];
   const int local = blockIdx.x - D.tile_begin;
   const int tr = local / D.tiles_c, tc = local % D.tiles_c;
   const int r0 = tr * kTile, c0 = tc * kTile;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float v[4][4];
-  load_o_tile<OT>(D, o_of<OT>(D), r0, c0, v, sm);
+  const bool t = D.trans != 0;
+  // storage extents and origin: rows s0.., columns q0.. of X (ld ldx)
+  const int srows = t ? D.n : D.m, scols = t ? D.m : D.n;
+  const int s0 = t ? c0 : r0, q0 = t ? r0 : c0;
+  const OT* X = o_of<OT>(D);
   const float om = D.oscale ? *D.oscale : 1.0f;
+  // the scale applied before squaring: rowscale (O rows) for column partials,
+  // colscale (O columns) for row partials; in storage order it is indexed by the
+  // storage column (O row) or storage row (O column)
+  const bool scale_on = want_cols ? (use_rows != 0) : (use_cols != 0);
+  const float* sc = want_cols ? D.rowscale : D.colscale;
+  const bool sc_by_col = want_cols ? t : !t;  // false: indexed by the storage row
+  float v[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int row = r0 + ty + 16 * i;
-    const float rs = (use_rows && row < D.m) ? D.rowscale[row] : 1.0f;
+    const int sr = s0 + ty + 16 * i, q = q0 + 4 * tx;
+    if (sr < srows && q + 4 <= scols) {
+      o_to_float4(X + (long long)sr * D.ldx + q, v[i]);
+    } else {  // the storage rows of a tall matrix are m long, which may not be a multiple of 4
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        v[i][e] = (sr < srows && q + e < scols) ? o_to_float(X[(long long)sr * D.ldx + q + e]) : 0.f;
+    }
+    float f[4] = {om, om, om, om};
+    if (scale_on) {
+      if (sc_by_col) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) f[e] *= (q + e < scols) ? sc[q + e] : 1.0f;
+      } else {
+        const float r = (sr < srows) ? sc[sr] : 1.0f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) f[e] *= r;
+      }
+    }
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int col = c0 + 4 * tx + e;
-      const float cs = (use_cols && col < D.n) ? D.colscale[col] : 1.0f;
-      v[i][e] *= om * (want_cols ? rs : cs);
+      const float x = v[i][e] * f[e];
+      v[i][e] = x * x;
     }
   }
-  if (want_rows) {
-    // row partial over this tile's 64 columns: the 16 threads of a row share a warp half
+  // per storage row: O rows of a wide matrix (row partials), O columns of a tall one
+  const bool along = t ? want_cols : want_rows;
+  if (along) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      float s = v[i][0] * v[i][0] + v[i][1] * v[i][1] + v[i][2] * v[i][2] + v[i][3] * v[i][3];
+      float s = (v[i][0] + v[i][1]) + (v[i][2] + v[i][3]);
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      const int row = r0 + ty + 16 * i;
-      if (tx == 0 && row < D.m) D.rowpart[(long long)tc * D.m + row] = s;
+      const int sr = s0 + ty + 16 * i;
+      if (tx == 0 && sr < srows) {
+        if (t) D.colpart[(long long)tr * D.n + sr] = s;  // O column sr, over O rows r0..
+        else D.rowpart[(long long)tc * D.m + sr] = s;    // O row sr, over O columns c0..
+      }
     }
-  }
-  if (want_cols) {
+  } else {
+    // per storage column: O columns of a wide matrix (column partials), O rows of a tall one
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float s = 0.f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) s += v[i][e] * v[i][e];
-      csum[ty][4 * tx + e] = s;
-    }
+    for (int e = 0; e < 4; ++e) csum[ty][4 * tx + e] = (v[0][e] + v[1][e]) + (v[2][e] + v[3][e]);
     __syncthreads();
     if (threadIdx.x < kTile) {
-      const int col = c0 + threadIdx.x;
+      const int q = q0 + threadIdx.x;
       float s = 0.f;
       for (int g = 0; g < 16; ++g) s += csum[g][threadIdx.x];
-      if (col < D.n) D.colpart[(long long)tr * D.n + col] = s;
+      if (q < scols) {
+        if (t) D.rowpart[(long long)tc * D.m + q] = s;  // O row q, over O columns c0..
+        else D.colpart[(long long)tr * D.n + q] = s;    // O column q, over O rows r0..
+      }
     }
   }
 }
