@@ -269,7 +269,8 @@ def fold_traffic(args):
            "pc_stats": ["pc_stats_kernel"],
            "pc_panel": ["gemm_tc_table_kernel", "gemm_tc_pair_kernel", "qr_gram_reduce_kernel"]}
     for rec, i in zip(launches, tail):
-        ok = fam.get(rec["kernel"], ["gemm_tc_table_kernel", "gemm_tc_pair_kernel", "gemm_tc_kernel"])
+        ok = fam.get(rec["kernel"], ["gemm_tc_table_kernel", "gemm_tc_pair_kernel", "gemm_tc_kernel",
+                                     "gemm_tc_pair_class_kernel"])
         if names[i] not in ok:
             raise SystemExit(f"launch {i}: ncu saw {names[i]}, the log says {rec['kernel']}: not aligned")
     agg = {}
