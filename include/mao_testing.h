@@ -66,6 +66,16 @@ typedef enum {
  */
 MAO_API mao_status mao_test_set_table_kernel(int32_t policy);
 
+/*
+ * Failure-path check of the bounded device waits: one thread waits, through the
+ * library's bounded mbarrier wait, on a barrier phase that nothing completes.  After
+ * the wait limit (1 s of %globaltimer) it records MAO_ERR_TIMEOUT with site 40 in the
+ * status word at workspace offset 0 and the kernel returns; the context stays usable.
+ * Read the result with mao_workspace_status.  workspace: >= 16 bytes, 256-byte
+ * aligned (its status word is cleared first).  No synchronisation.
+ */
+MAO_API mao_status mao_test_wait_timeout(void* workspace, size_t ws_bytes, mao_stream_t stream);
+
 MAO_API mao_status mao_test_gemm_workspace_size(int32_t kind, int32_t batch, int32_t M, int32_t N, int32_t K,
                                         size_t* bytes);
 MAO_API mao_status mao_test_gemm(int32_t kind, int32_t a_mn_major, int32_t b_mn_major, const void* A, const void* B,

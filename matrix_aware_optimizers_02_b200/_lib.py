@@ -107,6 +107,7 @@ SIGNATURES = {
     "mao_profile_stop": (c_int32, []),
     "mao_device_check": (c_int32, []),
     "mao_test_gemm_workspace_size": (c_int32, [c_int32, c_int32, c_int32, c_int32, c_int32, POINTER(c_size_t)]),
+    "mao_test_wait_timeout": (c_int32, [c_void_p, c_size_t, c_void_p]),
     "mao_test_set_table_kernel": (c_int32, [c_int32]),
     "mao_test_gemm": (c_int32, [c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_int32, c_int32, c_int32,
                                 c_int32, c_void_p, c_size_t, c_void_p]),

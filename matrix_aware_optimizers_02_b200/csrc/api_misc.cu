@@ -96,6 +96,36 @@ mao_status gemm_layout(int32_t kind_flags, int32_t batch, int32_t M, int32_t N, 
 
 extern "C" mao_status mao_test_set_table_kernel(int32_t policy) { return set_table_kernel_policy(policy); }
 
+namespace {
+
+// One thread waits on an mbarrier that nothing arrives at, through the same bounded
+// wait every kernel of the library uses: after kWaitLimitNs it records
+// MAO_ERR_TIMEOUT (site kTestWaitSite) and returns.  The other threads leave at once.
+constexpr int kTestWaitSite = 40;
+
+__global__ void test_wait_timeout_kernel(DevStatus* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_sh;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  abort_sh = 0;
+  volatile int* abort_flag = &abort_sh;
+  (void)mbar_wait(&bar, 0, status, kTestWaitSite, abort_flag);  // nothing completes the phase
+}
+
+}  // namespace
+
+extern "C" mao_status mao_test_wait_timeout(void* workspace, size_t ws_bytes, mao_stream_t stream_) {
+  if (workspace == nullptr || ws_bytes < sizeof(DevStatus)) return MAO_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MAO_ERR_ALIGN;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  DevStatus* status = reinterpret_cast<DevStatus*>(workspace);
+  MAO_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(DevStatus), stream));
+  test_wait_timeout_kernel<<<1, 32, 0, stream>>>(status);
+  return cudaGetLastError() == cudaSuccess ? MAO_OK : MAO_ERR_CUDA;
+}
+
 extern "C" mao_status mao_test_gemm_workspace_size(int32_t kind, int32_t batch, int32_t M, int32_t N, int32_t K,
                                                    size_t* bytes) {
   if (bytes == nullptr) return MAO_ERR_INVALID_ARG;

@@ -10,7 +10,13 @@
 * Determinism: two identical runs give bit-identical weights, states and stats.
 * Resume: a step taken after copying the whole state to the host and back into
   fresh buffers (a checkpoint) is bit-identical to the uninterrupted run.
+* Bounded waits: a wait on a barrier phase that nothing completes (a test entry of
+  the library, through the same bounded wait every kernel uses) gives up after its
+  limit, records MAO_ERR_TIMEOUT in the status word and returns; the context stays
+  usable.  No GPU fault, trap or endless loop is involved.
 """
+
+import ctypes
 
 import numpy as np
 import pytest
@@ -156,3 +162,27 @@ def test_resume_from_host_checkpoint(api, kind):
     for d, f in zip(mats, full):
         for name in ("W", "M", "R", "QR") + (("V", "L", "QL") if kind == "soap" else ("r", "c")):
             assert torch.equal(d[name], f[name]), name
+
+
+def test_bounded_wait_gives_up_and_reports(api):
+    lib = L.load()
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    addr = ws.data_ptr()
+    assert addr % 256 == 0
+    stream = torch.cuda.current_stream()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    L.check(lib.mao_test_wait_timeout(addr, ws.numel(), stream.cuda_stream), "wait timeout")
+    ev1.record(stream)
+    where = ctypes.c_int32(0)
+    st = lib.mao_workspace_status(addr, stream.cuda_stream, ctypes.byref(where))
+    assert st == L.MAO_ERR_TIMEOUT and where.value == 40, (st, where.value)
+    waited_ms = ev0.elapsed_time(ev1)
+    assert 900.0 <= waited_ms <= 5000.0, waited_ms  # the 1 s limit, then the kernel returned
+    # the context is still usable: a product after the timeout is right
+    A = torch.randn(2, 96, 64, device="cuda")
+    B = torch.randn(2, 80, 64, device="cuda")
+    D = api.gemm(A, B, kind="split3")
+    ref = torch.bmm(A.double(), B.double().transpose(1, 2))
+    assert (D.double() - ref).abs().max().item() < 1e-4
