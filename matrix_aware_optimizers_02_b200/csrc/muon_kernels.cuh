@@ -75,12 +75,15 @@ __device__ __forceinline__ void bf16x4_to_float(uint2 raw, float* v) {
 }
 
 // Tile of O in W's orientation: thread (ty, tx) receives rows r0 + ty + 16 i,
-// columns c0 + 4 tx + e; entries outside the matrix are 0.  `sm` is a 64 x 72
+// columns c0 + 4 tx + e; entries outside the matrix are 0.  `sm` is a 64 x 65
 // bf16 staging tile used for the transposed case (one __syncthreads inside).
-// The staging tile of load_o_tile for O stored as OT (padding keeps rows 16-byte aligned).
+// The staging tile of load_o_tile for O stored as OT.  Rows of 65 elements: the
+// transposed reads walk down a column with a stride of 4 rows across the lanes, which a
+// 65-element row spreads over distinct banks (a 72-element row put half the lanes on
+// one bank); every access to the tile is scalar, so no alignment is needed.
 template <typename OT>
 struct OTile {
-  static constexpr int kPad = 16 / (int)sizeof(OT);
+  static constexpr int kPad = 1;
   typedef OT Row[kTile + kPad];
 };
 
@@ -149,7 +152,7 @@ __device__ __forceinline__ const float* o_of<float>(const MuonMatDev& D) { retur
 // ------------------------------------------------------------------ prep
 __global__ void __launch_bounds__(256) muon_prep_kernel(const MuonMatDev* __restrict__ T, int count, float mu,
                                                         float* __restrict__ partial) {
-  __shared__ __nv_bfloat16 tileT[kTile][kTile + 8];
+  __shared__ __nv_bfloat16 tileT[kTile][kTile + 1];  // 65-element rows: conflict-free column writes
   __shared__ float wsum[8];
   const int blk = blockIdx.x;
   const MuonMatDev& D = T[find_mat(T, count, blk)];
