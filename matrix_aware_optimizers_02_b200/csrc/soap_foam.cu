@@ -472,32 +472,33 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
     }
     B.ops.back().blocks = blk;
   }
-  // QR by super-panels of kSuper = 2 kPanel columns (block Gram-Schmidt).  For each
-  // super-panel [c0, c0 + kSuper): one projection of all its columns against the
-  // finished columns [0, c0) (each pass over Q's planes serves 256 columns), then its
-  // two kPanel-column sub-panels in turn: the second is first projected against the
-  // first, and each is orthonormalised by Cholesky-QR (up to three passes, and a
-  // second projection against every finished column, all decided on the device).
+  // QR by super-panels of kSuper columns (block Gram-Schmidt).  For each super-panel
+  // [c0, c0 + kSuper): one projection of all its columns against the finished columns
+  // [0, c0) (each pass over Q's planes serves kSuper columns), then its kPanel-column
+  // sub-panels in turn: each after the first is projected against the super-panel's
+  // finished sub-panels, and each is orthonormalised by Cholesky-QR (up to three
+  // passes, and a second projection against every finished column, all decided on
+  // the device).
   int maxk = 0;
   for (int i = 0; i < nu; ++i) maxk = std::max(maxk, kof(i));
   const int nsuper = (maxk + kSuper - 1) / kSuper;
   enum { PS = 0, WA = 1, QF = 2 };
   for (int sp = 0; sp < nsuper; ++sp) {
     const int c0 = sp * kSuper;
-    for (int half = 0; half < 2; ++half) {
-      const int cs = c0 + half * kPanel;  // first column of the sub-panel
+    for (int sub = 0; sub < kSuper / kPanel; ++sub) {
+      const int cs = c0 + sub * kPanel;  // first column of the sub-panel
       std::vector<int> act;
       for (int i = 0; i < nu; ++i)
         if (kof(i) > cs) act.push_back(i);
       if (act.empty()) break;
       auto wdt = [&](int i) { return std::min(kPanel, kof(i) - cs); };
       // a sub-panel's fp32 storage and plane view: columns cs .. cs + w of Ps / Q, or
-      // the sub-panel's half of the super-panel buffer W
+      // the sub-panel's columns of the super-panel buffer W
       auto fp = [&](int i, int where, int* ld) -> float* {
         const int k = kof(i);
         switch (where) {
           case PS: *ld = k; return B.wp<float>(side(i).Ps) + cs;
-          case WA: *ld = kSuper; return B.wp<float>(side(i).W) + half * kPanel;
+          case WA: *ld = kSuper; return B.wp<float>(side(i).W) + sub * kPanel;
           default: *ld = k; return Qp(i) + cs;
         }
       };
@@ -509,7 +510,7 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
           case WA: v = B.planes(side(i).Wp, k, kSuper); break;
           default: v = B.planes(side(i).Qp, k, k); break;
         }
-        const int off = where == WA ? half * kPanel : cs;
+        const int off = where == WA ? sub * kPanel : cs;
         for (int q = 0; q < 3; ++q) v.p[q] += off;
         v.cols = w;
         return v;
@@ -698,7 +699,7 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
       };
       // The products W R^{-1} run in place (each output row block reads only its own
       // rows of W, all of K in one tile).
-      if (half == 0) {
+      if (sub == 0) {
         if (c0 == 0) {
           MAO_TRY(cholqr(PS, WA, 0));
           MAO_TRY(cholqr(WA, WA, 1));
@@ -711,11 +712,12 @@ mao_status build_refresh(Builder& B, GroupPlan& G) {
           MAO_TRY(cholqr(WA, QF, 2));
         }
       } else {
-        // against the first sub-panel (from Ps when the super-panel is the first)
-        MAO_TRY(project(act, c0 == 0 ? PS : WA, cs, c0, cs, kPanel, kPanel, false));
+        // against the super-panel's finished sub-panels (from Ps when the super-panel is
+        // the first)
+        MAO_TRY(project(act, c0 == 0 ? PS : WA, cs, c0, cs, sub * kPanel, kPanel, false));
         MAO_TRY(cholqr(WA, WA, 0));
         MAO_TRY(cholqr(WA, WA, 1));
-        MAO_TRY(project(act, WA, cs, 0, cs, kPanel, kPanel, true));
+        MAO_TRY(project(act, WA, cs, 0, cs, sub * kPanel, kPanel, true));
         MAO_TRY(cholqr(WA, QF, 2));
       }
     }
