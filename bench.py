@@ -845,10 +845,11 @@ def run_mine(args, rank, world, dist):
         "higher_is_better": False,
         "scaling": "strong" if layerwise else "weak",
         "vs_baseline": None,
-        "dtype": "bf16 operands / fp32 accumulate (Newton-Schulz); fp32-faithful split-bf16 products and fp32 "
-                 "states (SOAP, FOAM)",
+        "dtype": "bf16/fp32",
         "data": "synthetic (seeded Gaussian gradients, random weights)",
         "config": {"workload": args.workload, "description": desc, "experts": args.experts, "optimizers": order,
+                   "arithmetic": ("bf16 tensor-core operands with fp32 accumulation (Newton-Schulz); "
+                                  "fp32-faithful three-plane bf16 products and fp32 states and passes (SOAP, FOAM)"),
                    "optimizer_ms": opt_ms,
                    "muon": {"mu": 0.95, "lr": 0.02, "ns_steps": 5, "norm": norm},
                    "soap": {"beta1": 0.95, "beta2": 0.95, "eps": 1e-8,
