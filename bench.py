@@ -196,6 +196,41 @@ def ncu_traffic(kernel_name, flops_per_launch, bytes_per_launch):
     return None
 
 
+def roofline_of(name, e, peaks, peak_src, traffic):
+    """The roofline object of the bench line for one profiler id: `e` sums its launches
+    (n, ms, flops = executed useful FLOP, tc = tensor-core operations issued, planned =
+    the host's count of the ungated problems, bytes = algorithmic bytes); `traffic` is
+    ncu_traffic()'s scaled DRAM bytes per launch, or None."""
+    avg_ms = e["ms"] / e["n"]
+    if e["flops"] > 0:
+        # tensor-pipe work: the bf16 products issued (six per fp32-faithful multiply-add of
+        # three-plane operands), against the bf16 peak
+        achieved = (e["tc"] / e["n"]) / (avg_ms * 1e-3) / 1e12
+        useful = (e["flops"] / e["n"]) / (avg_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "kernel": name, "achieved": round(achieved, 1),
+                "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "useful_tflops": round(useful, 1),
+                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step); achieved counts "
+                               "the bf16 tensor-core products the kernel issued (6 per fp32-faithful "
+                               "multiply-add), over the tiles it computed (device counters: the passes "
+                               "decided on the device included)"}
+        if e["planned"] < e["flops"]:
+            roof["useful_tflops_host_counted"] = round((e["planned"] / e["n"]) / (avg_ms * 1e-3) / 1e12, 1)
+    else:
+        achieved = (e["bytes"] / e["n"]) / (avg_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "kernel": name, "achieved": round(achieved, 1),
+                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_src} HBM copy"}
+    roof["traffic"] = traffic["bytes"] if traffic else None
+    if traffic:
+        roof["traffic_source"] = f"ncu DRAM bytes per {traffic['by']} on {traffic['scaled_from']}, scaled to this launch"
+    roof["launches"] = e["n"]
+    roof["avg_launch_ms"] = round(avg_ms, 4)
+    return roof
+
+
 def write_launch_log(args, lib, L, LS, t, stream):
     """One more step with the launch profiler recording kernel ids and work only."""
     import torch
@@ -785,34 +820,9 @@ def run_mine(args, rank, world, dist):
     roof = None
     if dom is not None:
         e = per[dom]
-        avg_ms = e["ms"] / e["n"]
-        if e["flops"] > 0:
-            # tensor-pipe work: the bf16 products issued (six per fp32-faithful multiply-add of
-            # three-plane operands), against the measured bf16 peak
-            achieved = (e["tc"] / e["n"]) / (avg_ms * 1e-3) / 1e12
-            useful = (e["flops"] / e["n"]) / (avg_ms * 1e-3) / 1e12
-            peak = peaks["bf16_tflops_sustained"]
-            roof = {"bound": "tensor", "kernel": names.get(dom, str(dom)), "achieved": round(achieved, 1),
-                    "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                    "useful_tflops": round(useful, 1),
-                    "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step); achieved counts "
-                                   "the bf16 tensor-core products the kernel issued (6 per fp32-faithful "
-                                   "multiply-add), over the tiles it computed (device counters: the passes "
-                                   "decided on the device included)"}
-            if e["planned"] < e["flops"]:
-                roof["useful_tflops_host_counted"] = round((e["planned"] / e["n"]) / (avg_ms * 1e-3) / 1e12, 1)
-        else:
-            achieved = (e["bytes"] / e["n"]) / (avg_ms * 1e-3) / 1e9
-            peak = peaks["hbm_gbs"]
-            roof = {"bound": "hbm", "kernel": names.get(dom, str(dom)), "achieved": round(achieved, 1),
-                    "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                    "peak_source": f"{peak_src} HBM copy"}
-        tr = ncu_traffic(names.get(dom, str(dom)), e["flops"] / e["n"], e["bytes"] / e["n"])
-        roof["traffic"] = tr["bytes"] if tr else None
-        if tr:
-            roof["traffic_source"] = f"ncu DRAM bytes per {tr['by']} on {tr['scaled_from']}, scaled to this launch"
-        roof["launches"] = e["n"]
-        roof["avg_launch_ms"] = round(avg_ms, 4)
+        name = names.get(dom, str(dom))
+        tr = ncu_traffic(name, e["flops"] / e["n"], e["bytes"] / e["n"])
+        roof = roofline_of(name, e, peaks, peak_src, tr)
     tot = max(sum(x["ms"] for x in per.values()), 1e-9)
     kernels = {}
     for k, v in sorted(per.items()):

@@ -1,5 +1,6 @@
 """Measurement helpers of bench.py, on CPU: folding an ncu launch list onto the
-library's profiler ids, and scaling the committed DRAM traffic summary to a launch.
+library's profiler ids, scaling the committed DRAM traffic summary to a launch, and
+the roofline object of the bench line.
 
 The ncu CSV here is synthetic but has the layout ncu writes with --csv (one row per
 launch and metric, "ID", "Kernel Name", "Metric Name", "Metric Value")."""
@@ -109,3 +110,23 @@ def test_committed_traffic_summary_matches_the_sources():
     with open(bench.os.path.join(bench.ROOT, "profiles", "ncu_traffic.json")) as f:
         d = json.load(f)
     assert d["source_hash"] == bench.kernel_source_hash()
+
+
+def test_roofline_of_tensor_and_hbm_kernels():
+    peaks = {"bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+    # four launches of 2 ms: 1e12 useful FLOP each (0.8e12 counted by the host), 6e12 issued
+    e = {"n": 4, "ms": 8.0, "flops": 4.0e12, "tc": 24.0e12, "planned": 3.2e12, "bytes": 0.0}
+    r = bench.roofline_of("pc_qr", e, peaks, "fallback", {"bytes": 123, "by": "algorithmic flops",
+                                                           "scaled_from": "toy"})
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["kernel"] == "pc_qr"
+    assert r["achieved"] == pytest.approx(3000.0) and r["useful_tflops"] == pytest.approx(500.0)
+    assert r["frac"] == pytest.approx(3000.0 / 1400.0, abs=1e-4)
+    assert r["useful_tflops_host_counted"] == pytest.approx(400.0)
+    assert r["traffic"] == 123 and "toy" in r["traffic_source"]
+    assert r["launches"] == 4 and r["avg_launch_ms"] == pytest.approx(2.0)
+    # an HBM pass: 2 launches of 1 ms moving 5 GB each
+    e = {"n": 2, "ms": 2.0, "flops": 0.0, "tc": 0.0, "planned": 0.0, "bytes": 10.0e9}
+    r = bench.roofline_of("pc_elementwise", e, peaks, "measured", None)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(5000.0) and r["frac"] == pytest.approx(5000.0 / 6650.0, abs=1e-4)
+    assert r["traffic"] is None and "traffic_source" not in r
