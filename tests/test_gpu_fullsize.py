@@ -19,6 +19,8 @@ launch configuration the benchmark uses (bf16 gradients, refresh every step, sor
   The factors L, R and the moment M are compared with the oracle in full, and the
   oracle's S5-S8 (soap_precondition) run in the device's validated bases give V and
   the weight update, at the gates of test_gpu_soap_foam.
+* FOAM on the 8B block's 4096 x 14336 matrix (its 14336 x 14336 factor), t = 1 and 2,
+  checked like the SOAP case.
 * FOAM on the GPT-2-760M-shaped 6144 x 1536 and 1536 x 4608 matrices through an
   adaptive check (t = 1 checks and refreshes, t = 2 is a plain step): the oracle in full.
 """
@@ -106,18 +108,18 @@ def test_soap_moe_expert_scales(api, s_e):
 
 # ------------------------------------------------------------------ SOAP, 8B block matrices
 
-def _basis_properties(lab, Q, F, Qprev, perm, rng):
+def _basis_properties(lab, Q, F, Qprev, perm, rng, who="soap"):
     """Sampled checks that Q is the positive-diagonal QR factor of F Qprev[:, perm]."""
     k = Q.shape[0]
     cols = np.unique(np.concatenate([[0, 1, k // 2, k - 2, k - 1], rng.choice(k, SAMPLES, replace=False)]))
     QtQ = Q.T @ Q[:, cols]
     orth = np.linalg.norm(QtQ - np.eye(k)[:, cols], axis=0)
-    gates.check(lab, "soap basis orthonormality (sampled)", float(orth.max()), STATE_TOL)
+    gates.check(lab, f"{who} basis orthonormality (sampled)", float(orth.max()), STATE_TOL)
     Pc = F @ Qprev[:, perm[cols]]                      # sampled columns of P
     R = Q.T @ Pc                                       # (Q^T P)[:, cols]
     pn = np.linalg.norm(Pc, axis=0)
     below = np.array([np.linalg.norm(R[j + 1:, c]) for c, j in enumerate(cols)]) / pn
-    gates.check(lab, "soap basis QR residual (sampled)", float(below.max()), STATE_TOL)
+    gates.check(lab, f"{who} basis QR residual (sampled)", float(below.max()), STATE_TOL)
     assert np.all(R[cols, np.arange(len(cols))] > 0), lab
 
 
@@ -178,6 +180,58 @@ def test_soap_dense8b_full_size(api, shape):
         gates.check(lab, "soap update_rms (full size)", abs(batch.stats_dict()["update_rms"][0] - rms) / rms, gate)
         # continue from the device's weight and bases (the oracle's own factors and moments)
         QLp, QRp, Wprev = QL, QR, Wg
+
+
+# ------------------------------------------------------------------ FOAM, 8B block matrix
+
+def test_foam_dense8b_full_size(api):
+    """FOAM on the 8B block's 4096 x 14336 matrix (the 14336 x 14336 input-side factor),
+    refreshing every step, t = 1 and 2, checked like the SOAP case above: R and the
+    moments in full, the basis by its defining properties on sampled columns, the
+    permutation against the oracle's sort, and the oracle's F4-F6 in the device's
+    basis for the update."""
+    m, n = 4096, 14336
+    rng = np.random.default_rng(56)
+    W = (rng.standard_normal((m, n)) * 0.02).astype(np.float32)
+    st = O.FoamState.init(m, n)
+    t32 = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()  # noqa: E731
+    d = {"W": t32(W), "G": torch.zeros((m, n), dtype=torch.bfloat16, device="cuda"), "M": t32(st.M),
+         "r": t32(st.r), "c": t32(st.c), "R": t32(st.R), "QR": t32(st.QR),
+         "perm_R": torch.zeros(n, dtype=torch.int32, device="cuda")}
+    batch = api.FoamBatch([d], beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3, refresh="every_k", k=1,
+                          with_stats=True)
+    R, Mprev, r, c = st.R, st.M, st.r, st.c
+    QRp = np.eye(n)
+    Wprev = W.astype(np.float64)
+    srng = np.random.default_rng(57)
+    for t in (1, 2):
+        G = synth.bf16_round((rng.standard_normal((m, n)) * 0.01).astype(np.float32)).astype(np.float64)
+        d["G"].copy_(torch.from_numpy(G.astype(np.float32)).to(torch.bfloat16))
+        batch(t)
+        assert batch.device_status() == 0
+        torch.cuda.synchronize()
+        lab = f"foam full {m}x{n} t={t}"
+        R = 0.95 * R + 0.05 * (G.T @ G)
+        P._compare(lab, "foam R (full size)", _np(d["R"]), R, STATE_TOL)
+        pr = d["perm_R"].cpu().numpy()
+        QR = _np(d["QR"])
+        _perm_vs_keys(lab, pr, R, QRp)
+        _basis_properties(lab, QR, R, QRp, pr, srng, who="foam")
+        # F4-F6 in the device's validated basis; c follows the device's permutation
+        kw = dict(t=t, beta1=0.95, beta2=0.95, eps=1e-8, lr=3e-3)
+        rp, cp = r, c[pr]
+        Wn, M, r, c, _, _ = O.foam_precondition(Wprev, G, Mprev, rp, cp, R, QR, **kw)
+        Wn32, _, _, _, _, _ = O.foam_precondition(Wprev, G, Mprev, rp, cp, R, QR, dtype=np.float32, **kw)
+        Mprev = M
+        Wg = _np(d["W"])
+        P._compare(lab, "foam M (full size)", _np(d["M"]), M, STATE_TOL)
+        P._compare(lab, "foam r (full size)", _np(d["r"]), r, STATE_TOL)
+        P._compare(lab, "foam c (full size)", _np(d["c"]), c, STATE_TOL)
+        ref, ref32 = Wn - Wprev, Wn32.astype(np.float64) - Wprev
+        gate = max(STATE_TOL, 2 * gates.rel(ref32, ref))
+        P._compare(lab, "foam dW (full size)", Wg - Wprev, ref, gate, ref32)
+        # continue from the device's weight and basis (the oracle's own factor and moments)
+        QRp, Wprev = QR, Wg
 
 
 # ------------------------------------------------------------------ FOAM, GPT-2-760M shapes
